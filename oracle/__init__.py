@@ -1,0 +1,194 @@
+"""CPU oracle of the Beam MoE block forward pass (plain FP64 C via ctypes, numpy glue).
+
+TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the benchmark's CPU-baseline and
+reference arm use it.  The CUDA product path never imports it, and it imports nothing from the
+product package.  All arithmetic lives in beam_oracle.c; this module only marshals arrays.
+
+Functions, in the order of the Beam launch post's description of the block ("Welcome Beam" page,
+section "Mixture of Experts"):
+  router_scores  - sigmoid scores of all experts (FP64 logits)
+  select         - group-limited top-k: group score = sum of the top-2, keep 4 of 8 groups, top 8
+  route          - router_scores + select
+  permute        - stable (expert, token) grouping of the T*k routed pairs
+  expert_mlp     - one SwiGLU expert on a set of rows
+  combine        - routed_scale * sum_j w_j * expert_j(x)
+  forward        - the whole block on host tensors
+  forward_tokens - the whole block for a subset of tokens, fetching one expert's weights at a time
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Callable, Optional, Sequence
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+_dp = ctypes.POINTER(ctypes.c_double)
+_fp = ctypes.POINTER(ctypes.c_float)
+_i32p = ctypes.POINTER(ctypes.c_int32)
+_i64p = ctypes.POINTER(ctypes.c_int64)
+_u16p = ctypes.POINTER(ctypes.c_uint16)
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        L.oracle_num_threads.restype = ctypes.c_int
+        L.oracle_router_scores.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, _u16p, _fp, _dp, _dp]
+        L.oracle_router_scores.restype = None
+        L.oracle_select.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                    ctypes.c_int, _dp, _fp, _i32p, _i32p, _dp, _dp]
+        L.oracle_select.restype = ctypes.c_int
+        L.oracle_permute.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, _i32p, _i32p, _i64p, _i32p, _i32p]
+        L.oracle_permute.restype = ctypes.c_int
+        L.oracle_expert_mlp.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, _u16p, _u16p, _u16p, _u16p, _dp]
+        L.oracle_expert_mlp.restype = None
+        L.oracle_combine.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_double, _dp, _dp, _dp]
+        L.oracle_combine.restype = None
+        _lib = L
+    return _lib
+
+
+def num_threads() -> int:
+    return int(lib().oracle_num_threads())
+
+
+def _ptr(a: Optional[np.ndarray], typ):
+    if a is None:
+        return ctypes.cast(None, typ)
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(typ)
+
+
+def bf16_bits(t) -> np.ndarray:
+    """Raw 16-bit patterns of a bf16 torch tensor (or pass-through of a uint16 array)."""
+    if isinstance(t, np.ndarray):
+        assert t.dtype == np.uint16
+        return np.ascontiguousarray(t)
+    import torch
+    assert t.dtype == torch.bfloat16
+    return np.ascontiguousarray(t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+def bf16_bits_to_f64(bits: np.ndarray) -> np.ndarray:
+    return (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def router_scores(x_bits: np.ndarray, w_router: np.ndarray, return_logits: bool = False):
+    """Sigmoid scores [T,E] fp64 (and the FP64 logits) of x [T,H] (bf16 bits) under W_r [E,H] fp32."""
+    x_bits = np.ascontiguousarray(x_bits, dtype=np.uint16)
+    w_router = np.ascontiguousarray(w_router, dtype=np.float32)
+    T, H = x_bits.shape
+    E = w_router.shape[0]
+    assert w_router.shape[1] == H
+    score = np.empty((T, E), dtype=np.float64)
+    logit = np.empty((T, E), dtype=np.float64) if return_logits else None
+    lib().oracle_router_scores(T, H, E, _ptr(x_bits, _u16p), _ptr(w_router, _fp), _ptr(logit, _dp), _ptr(score, _dp))
+    return (score, logit) if return_logits else score
+
+
+def select(score: np.ndarray, layer: dict, bias: Optional[np.ndarray] = None):
+    """Group-limited top-k on scores [T,E].  Returns dict(ids, ids64, weight, margin)."""
+    score = np.ascontiguousarray(score, dtype=np.float64)
+    T, E = score.shape
+    k = layer["topk"]
+    ids = np.empty((T, k), dtype=np.int32)
+    ids64 = np.empty((T, k), dtype=np.int32)
+    weight = np.empty((T, k), dtype=np.float64)
+    margin = np.empty((T, 3), dtype=np.float64)
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    rc = lib().oracle_select(T, E, layer["n_groups"], layer["topk_groups"], k, layer["group_topn"],
+                             _ptr(score, _dp), _ptr(b, _fp), _ptr(ids, _i32p), _ptr(ids64, _i32p),
+                             _ptr(weight, _dp), _ptr(margin, _dp))
+    if rc != 0:
+        raise ValueError(f"oracle_select rejected the configuration (rc={rc})")
+    return dict(ids=ids, ids64=ids64, weight=weight, margin=margin)
+
+
+def route(x_bits: np.ndarray, w_router: np.ndarray, layer: dict, bias: Optional[np.ndarray] = None):
+    score = router_scores(x_bits, w_router)
+    out = select(score, layer, bias)
+    out["score"] = score
+    return out
+
+
+def permute(ids: np.ndarray, n_experts: int):
+    """Stable grouping by expert.  Returns dict(counts, offsets, row_src, dest_row)."""
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    T, k = ids.shape
+    counts = np.empty(n_experts, dtype=np.int32)
+    offsets = np.empty(n_experts + 1, dtype=np.int64)
+    row_src = np.empty(T * k, dtype=np.int32)
+    dest_row = np.empty(T * k, dtype=np.int32)
+    rc = lib().oracle_permute(T, k, n_experts, _ptr(ids, _i32p), _ptr(counts, _i32p), _ptr(offsets, _i64p),
+                              _ptr(row_src, _i32p), _ptr(dest_row, _i32p))
+    if rc != 0:
+        raise ValueError("oracle_permute: id out of range")
+    return dict(counts=counts, offsets=offsets, row_src=row_src, dest_row=dest_row)
+
+
+def expert_mlp(x_rows_bits: np.ndarray, wg_bits: np.ndarray, wu_bits: np.ndarray, wd_bits: np.ndarray) -> np.ndarray:
+    """SwiGLU expert on rows [n,H] (bf16 bits); weights bf16 bits; returns [n,H] fp64."""
+    x_rows_bits = np.ascontiguousarray(x_rows_bits, dtype=np.uint16)
+    n, H = x_rows_bits.shape
+    I = wg_bits.shape[0]
+    assert wg_bits.shape == (I, H) and wu_bits.shape == (I, H) and wd_bits.shape == (H, I)
+    out = np.empty((n, H), dtype=np.float64)
+    if n == 0:
+        return out
+    lib().oracle_expert_mlp(n, H, I, _ptr(x_rows_bits, _u16p), _ptr(np.ascontiguousarray(wg_bits), _u16p),
+                            _ptr(np.ascontiguousarray(wu_bits), _u16p), _ptr(np.ascontiguousarray(wd_bits), _u16p),
+                            _ptr(out, _dp))
+    return out
+
+
+def combine(expert_out: np.ndarray, weight: np.ndarray, routed_scale: float) -> np.ndarray:
+    """y [T,H] = routed_scale * sum_j weight[t,j] expert_out[t,j,:] (fp64)."""
+    expert_out = np.ascontiguousarray(expert_out, dtype=np.float64)
+    weight = np.ascontiguousarray(weight, dtype=np.float64)
+    T, k, H = expert_out.shape
+    y = np.empty((T, H), dtype=np.float64)
+    lib().oracle_combine(T, k, H, float(routed_scale), _ptr(expert_out, _dp), _ptr(weight, _dp), _ptr(y, _dp))
+    return y
+
+
+ExpertFetch = Callable[[int], Sequence[np.ndarray]]
+
+
+def experts_tokens(x_bits: np.ndarray, ids: np.ndarray, weight: np.ndarray, fetch: ExpertFetch,
+                   n_experts: int, routed_scale: float) -> np.ndarray:
+    """Expert half of the block for the given rows: x_bits [n,H], ids/weight [n,k].
+
+    `fetch(e)` returns (W_gate[e], W_up[e], W_down[e]) as bf16 bit arrays; it is called once per
+    expert that any of the rows uses, so the full weight set never has to sit in host memory.
+    """
+    n, H = x_bits.shape
+    k = ids.shape[1]
+    out = np.zeros((n, k, H), dtype=np.float64)
+    for e in range(n_experts):
+        rows, slots = np.nonzero(ids == e)
+        if rows.size == 0:
+            continue
+        wg, wu, wd = fetch(e)
+        out[rows, slots, :] = expert_mlp(x_bits[rows], wg, wu, wd)
+    return combine(out, weight, routed_scale)
+
+
+def forward(x_bits: np.ndarray, w_router: np.ndarray, bias: Optional[np.ndarray], fetch: ExpertFetch,
+            layer: dict, tokens: Optional[np.ndarray] = None):
+    """The whole block.  Routing for all T tokens; expert outputs for `tokens` (default: all).
+
+    Returns dict(route=..., tokens=..., y=[len(tokens),H] fp64).
+    """
+    r = route(x_bits, w_router, layer, bias)
+    T = x_bits.shape[0]
+    tok = np.arange(T) if tokens is None else np.asarray(tokens, dtype=np.int64)
+    y = experts_tokens(np.ascontiguousarray(x_bits[tok]), r["ids"][tok], r["weight"][tok], fetch,
+                       layer["n_experts"], layer["routed_scale"])
+    return dict(route=r, tokens=tok, y=y)

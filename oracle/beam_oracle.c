@@ -1,0 +1,292 @@
+/*
+ * Beam MoE block forward pass: plain, slow CPU oracle in FP64.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the benchmark's CPU-baseline /
+ * reference arm may load this library.  It shares no code, header or constant with the CUDA
+ * library; it is built separately (oracle/build.py) with gcc.
+ *
+ * What it computes, step by step, in the order of the Beam launch post ("Welcome Beam" page,
+ * section "Mixture of Experts"; the same text in the Hugging Face post flattened on the
+ * reducer.xgoose.org digest page; the Chinese digest on that page adds "sigmoid scoring, 8 experts,
+ * x2.5"):
+ *   1. score every expert with a sigmoid of the router projection, computed in FP32 by the model
+ *      ("Welcome Beam" page, section "Residual Stream": the router computes in FP32);
+ *   2. split the experts into n_groups contiguous groups; rank groups by the sum of each group's
+ *      top group_topn scores; keep the topk_groups best groups;
+ *   3. pick the topk experts with the largest scores inside the kept groups;
+ *   4. combine the experts' outputs with router weights normalised to sum 1, then scale by
+ *      routed_scale (2.5);
+ *   5. each expert is a SwiGLU MLP: Wd (SiLU(Wg x) * (Wu x)).
+ *
+ * Readings where the pages are silent (all listed in the design notes of this repository):
+ *   - an optional per-expert selection bias b is added to the scores for group and expert
+ *     selection only; the weights use the unbiased sigmoid scores (DeepSeek-V3's scheme, which the
+ *     pages name); b = 0 unless a workload sets it;
+ *   - groups are contiguous index ranges;
+ *   - ties go to the lower group / expert index; slots are in descending selected score;
+ *   - the selection decision is taken on scores rounded to FP32 (the router's precision on the
+ *     pages); the FP64 scores give the decision margins used to exclude near-ties from bit-exact
+ *     comparison.
+ *
+ * Arithmetic: logits, sigmoid, weights, expert MLP and the weighted sum in FP64 on the exact bf16
+ * inputs.  bf16 values arrive as their raw 16-bit patterns.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+static double bf16_bits_to_double(uint16_t b)
+{
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/*
+ * Step 1 (section "Mixture of Experts": "scores all 256 experts with a sigmoid"):
+ * logit[t,e] = sum_h x[t,h] * W_r[e,h] in FP64, score = 1 / (1 + exp(-logit)).
+ * x: [T,H] bf16 bits; w_router: [E,H] fp32; logit, score: [T,E] fp64.
+ */
+void oracle_router_scores(int64_t T, int H, int E, const uint16_t *x, const float *w_router,
+                          double *logit, double *score)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        double *xr = (double *)malloc(sizeof(double) * (size_t)H);
+        for (int h = 0; h < H; ++h) xr[h] = bf16_bits_to_double(x[t * H + h]);
+        for (int e = 0; e < E; ++e) {
+            const float *wr = w_router + (int64_t)e * H;
+            double acc = 0.0;
+            for (int h = 0; h < H; ++h) acc += xr[h] * (double)wr[h];
+            if (logit) logit[t * E + e] = acc;
+            score[t * E + e] = 1.0 / (1.0 + exp(-acc));
+        }
+        free(xr);
+    }
+}
+
+/* Index of the largest v[i] among alive[i] != 0; ties go to the lower index.  -1 if none. */
+static int argmax_alive(const double *v, const unsigned char *alive, int n)
+{
+    int best = -1;
+    for (int i = 0; i < n; ++i) {
+        if (!alive[i]) continue;
+        if (best < 0 || v[i] > v[best]) best = i;
+    }
+    return best;
+}
+
+/*
+ * Group-limited selection for one token (steps 2 and 3).  `sel` holds the selection values of the
+ * E experts (score + bias).  When `fp32` is set, every selection value and every group-score sum
+ * is rounded to FP32 (the decision precision of the model's router); otherwise FP64.
+ * Outputs the kept groups' mask and the topk expert ids in pick order (descending value).
+ * Returns the sorted group scores and selected values so the caller can take margins.
+ */
+static void select_one(int E, int G, int topk_groups, int topk, int group_topn, const double *sel_in,
+                       int fp32, unsigned char *group_kept, int32_t *ids, double *gs_sorted,
+                       double *sel_sorted_kept, int *n_kept_experts)
+{
+    const int per = E / G;
+    double sel[1024];
+    unsigned char alive[1024];
+    double gs[1024];
+    for (int e = 0; e < E; ++e) sel[e] = fp32 ? (double)(float)sel_in[e] : sel_in[e];
+
+    /* group score = sum of the group's top group_topn selection values, summed in pick order */
+    for (int g = 0; g < G; ++g) {
+        for (int i = 0; i < per; ++i) alive[i] = 1;
+        double s64 = 0.0;
+        float s32 = 0.0f;
+        for (int r = 0; r < group_topn; ++r) {
+            int i = argmax_alive(sel + g * per, alive, per);
+            alive[i] = 0;
+            if (fp32) s32 = s32 + (float)sel[g * per + i];
+            else s64 += sel[g * per + i];
+        }
+        gs[g] = fp32 ? (double)s32 : s64;
+    }
+    /* keep the topk_groups best groups (lower group index on ties) */
+    unsigned char galive[1024];
+    for (int g = 0; g < G; ++g) { galive[g] = 1; group_kept[g] = 0; }
+    for (int r = 0; r < G; ++r) {
+        int g = argmax_alive(gs, galive, G);
+        galive[g] = 0;
+        gs_sorted[r] = gs[g];
+        if (r < topk_groups) group_kept[g] = 1;
+    }
+    /* topk experts inside the kept groups (lower expert index on ties), in pick order */
+    for (int e = 0; e < E; ++e) alive[e] = group_kept[e / per];
+    int n = 0;
+    for (int e = 0; e < E; ++e) n += alive[e];
+    *n_kept_experts = n;
+    for (int r = 0; r < n; ++r) {
+        int e = argmax_alive(sel, alive, E);
+        alive[e] = 0;
+        sel_sorted_kept[r] = sel[e];
+        if (r < topk) ids[r] = e;
+    }
+}
+
+/*
+ * Steps 2-4 for T tokens.  score: [T,E] fp64 (from oracle_router_scores); bias: [E] fp32 or NULL.
+ * Outputs:
+ *   ids     [T,topk] int32  the decision taken on FP32-rounded values (the model's router precision)
+ *   ids64   [T,topk] int32  the same decision in FP64 (nullable)
+ *   weight  [T,topk] fp64   score[id] / sum of the selected scores (unbiased scores)
+ *   margin  [T,3]    fp64   FP64 decision margins (nullable):
+ *                           [0] group: 4th-best minus 5th-best group score (topk_groups-th vs next)
+ *                           [1] expert: topk-th minus next selection value inside the kept groups
+ *                           [2] order: smallest gap between consecutive selected values
+ *                           (+inf where no such comparison exists)
+ * Returns 0, or -1 for a configuration this plain implementation does not accept.
+ */
+int oracle_select(int64_t T, int E, int G, int topk_groups, int topk, int group_topn,
+                  const double *score, const float *bias, int32_t *ids, int32_t *ids64,
+                  double *weight, double *margin)
+{
+    if (E <= 0 || E > 1024 || G <= 0 || E % G || topk_groups < 1 || topk_groups > G ||
+        group_topn < 1 || group_topn > E / G || topk < 1 || topk > topk_groups * (E / G))
+        return -1;
+    int bad = 0;
+    #pragma omp parallel for schedule(static) reduction(+:bad)
+    for (int64_t t = 0; t < T; ++t) {
+        double sel[1024], gs_sorted[1024], sel_sorted[1024];
+        unsigned char kept[1024];
+        int32_t id32[1024], id64[1024];
+        int nk = 0;
+        const double *s = score + t * E;
+        /* the biased value in FP32 is the FP32 sum of the FP32 score and the FP32 bias */
+        for (int e = 0; e < E; ++e) {
+            float s32 = (float)s[e];
+            sel[e] = bias ? (double)(s32 + bias[e]) : (double)s32;
+        }
+        select_one(E, G, topk_groups, topk, group_topn, sel, 1, kept, id32, gs_sorted, sel_sorted, &nk);
+        for (int e = 0; e < E; ++e) sel[e] = s[e] + (bias ? (double)bias[e] : 0.0);
+        select_one(E, G, topk_groups, topk, group_topn, sel, 0, kept, id64, gs_sorted, sel_sorted, &nk);
+        for (int j = 0; j < topk; ++j) {
+            ids[t * topk + j] = id32[j];
+            if (ids64) ids64[t * topk + j] = id64[j];
+        }
+        double den = 0.0;
+        for (int j = 0; j < topk; ++j) den += s[id32[j]];
+        if (!(den > 0.0)) bad++;
+        for (int j = 0; j < topk; ++j) weight[t * topk + j] = s[id32[j]] / den;
+        if (margin) {
+            margin[t * 3 + 0] = topk_groups < G ? gs_sorted[topk_groups - 1] - gs_sorted[topk_groups] : INFINITY;
+            margin[t * 3 + 1] = topk < nk ? sel_sorted[topk - 1] - sel_sorted[topk] : INFINITY;
+            double mo = INFINITY;
+            for (int j = 0; j + 1 < topk; ++j) {
+                double d = sel_sorted[j] - sel_sorted[j + 1];
+                if (d < mo) mo = d;
+            }
+            margin[t * 3 + 2] = mo;
+        }
+    }
+    return bad ? -2 : 0;
+}
+
+/*
+ * Token -> expert dispatch (the pages only say each token runs on its 8 experts; this is the plain
+ * stable grouping of the T*topk (token, slot) pairs by expert).  Rows are ordered by
+ * (expert ascending, token ascending); q = t*topk + j.
+ *   counts[e]   number of pairs routed to e
+ *   offsets[e]  exclusive prefix sum of counts (offsets[E] = T*topk)
+ *   row_src[r]  the pair q placed in row r
+ *   dest_row[q] the row of pair q
+ * Returns 0, or -1 if an id is outside [0, E).
+ */
+int oracle_permute(int64_t T, int topk, int E, const int32_t *ids, int32_t *counts, int64_t *offsets,
+                   int32_t *row_src, int32_t *dest_row)
+{
+    const int64_t n = T * topk;
+    for (int e = 0; e < E; ++e) counts[e] = 0;
+    for (int64_t q = 0; q < n; ++q) {
+        if (ids[q] < 0 || ids[q] >= E) return -1;
+        counts[ids[q]]++;
+    }
+    offsets[0] = 0;
+    for (int e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
+    int64_t r = 0;
+    for (int e = 0; e < E; ++e)
+        for (int64_t q = 0; q < n; ++q)
+            if (ids[q] == e) {
+                row_src[r] = (int32_t)q;
+                dest_row[q] = (int32_t)r;
+                ++r;
+            }
+    return 0;
+}
+
+/*
+ * One SwiGLU expert ("each a SwiGLU MLP with an intermediate size of 2,560"; the SwiGLU product in
+ * FP32 on the model, here FP64) applied to n rows:
+ *   g = Wg x, u = Wu x, h = SiLU(g) * u with SiLU(z) = z / (1 + exp(-z)), out = Wd h.
+ * x_rows [n,H] bf16 bits; wg, wu [I,H] bf16 bits; wd [H,I] bf16 bits; out [n,H] fp64.
+ */
+void oracle_expert_mlp(int64_t n, int H, int I, const uint16_t *x_rows, const uint16_t *wg,
+                       const uint16_t *wu, const uint16_t *wd, double *out)
+{
+    double *xd = (double *)malloc(sizeof(double) * (size_t)(n * H));
+    double *hd = (double *)malloc(sizeof(double) * (size_t)(n * I));
+    for (int64_t q = 0; q < n * H; ++q) xd[q] = bf16_bits_to_double(x_rows[q]);
+
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t r = 0; r < n; ++r)
+        for (int i = 0; i < I; ++i) {
+            const double *xr = xd + r * H;
+            const uint16_t *gr = wg + (int64_t)i * H;
+            const uint16_t *ur = wu + (int64_t)i * H;
+            double g = 0.0, u = 0.0;
+            for (int h = 0; h < H; ++h) {
+                g += bf16_bits_to_double(gr[h]) * xr[h];
+                u += bf16_bits_to_double(ur[h]) * xr[h];
+            }
+            double silu = g / (1.0 + exp(-g));
+            hd[r * I + i] = silu * u;
+        }
+
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t r = 0; r < n; ++r)
+        for (int o = 0; o < H; ++o) {
+            const double *hr = hd + r * I;
+            const uint16_t *dr = wd + (int64_t)o * I;
+            double acc = 0.0;
+            for (int i = 0; i < I; ++i) acc += bf16_bits_to_double(dr[i]) * hr[i];
+            out[r * H + o] = acc;
+        }
+    free(xd);
+    free(hd);
+}
+
+/*
+ * Step 4 ("Expert outputs are combined with normalized router weights and scaled by 2.5"):
+ * y[t] = routed_scale * sum_j weight[t,j] * expert_out[t,j], summed over j = 0..topk-1.
+ * expert_out [T,topk,H] fp64; weight [T,topk] fp64; y [T,H] fp64.
+ */
+void oracle_combine(int64_t T, int topk, int H, double routed_scale, const double *expert_out,
+                    const double *weight, double *y)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t)
+        for (int h = 0; h < H; ++h) {
+            double acc = 0.0;
+            for (int j = 0; j < topk; ++j)
+                acc += weight[t * topk + j] * expert_out[(t * topk + j) * H + h];
+            y[t * H + h] = routed_scale * acc;
+        }
+}

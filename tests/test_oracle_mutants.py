@@ -1,0 +1,90 @@
+"""Plant plausible mistakes in copies of the oracle and check that the pins catch every one.
+
+Each mutant is the oracle's C source with one textual change, compiled to a temporary library
+and swapped in for the real one; at least one pin of test_oracle_pins.py must then fail.
+"""
+from __future__ import annotations
+
+import contextlib
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "beam_oracle.c")
+
+MUTANTS = {
+    "group_score_top1": ("for (int r = 0; r < group_topn; ++r) {", "for (int r = 0; r < 1; ++r) {"),
+    "no_group_limit": ("if (r < topk_groups) group_kept[g] = 1;", "group_kept[g] = 1;"),
+    "weights_use_bias": ("for (int j = 0; j < topk; ++j) den += s[id32[j]];",
+                         "for (int j = 0; j < topk; ++j) den += sel[id32[j]];"),
+    "ties_to_higher_index": ("if (best < 0 || v[i] > v[best]) best = i;", "if (best < 0 || v[i] >= v[best]) best = i;"),
+    "sigmoid_sign": ("score[t * E + e] = 1.0 / (1.0 + exp(-acc));", "score[t * E + e] = 1.0 / (1.0 + exp(acc));"),
+    "silu_sign": ("double silu = g / (1.0 + exp(-g));", "double silu = g / (1.0 + exp(g));"),
+    "silu_missing": ("hd[r * I + i] = silu * u;", "hd[r * I + i] = g * u;"),
+    "down_transposed": ("acc += bf16_bits_to_double(dr[i]) * hr[i];",
+                        "acc += bf16_bits_to_double(wd[(int64_t)i * H + o]) * hr[i];"),
+    "gate_up_swapped_role": ("double silu = g / (1.0 + exp(-g));", "double silu = u / (1.0 + exp(-u));"),
+    "no_routed_scale": ("y[t * H + h] = routed_scale * acc;", "y[t * H + h] = acc;"),
+    "permute_tokens_descending": ("for (int64_t q = 0; q < n; ++q)\n            if (ids[q] == e) {",
+                                  "for (int64_t q = n - 1; q >= 0; --q)\n            if (ids[q] == e) {"),
+    "offsets_inclusive": ("offsets[e + 1] = offsets[e] + counts[e];",
+                          "offsets[e + 1] = offsets[e] + counts[e] + (e == 0);"),
+}
+
+PINS = [
+    lambda: pins.test_bruteforce_tiny(False),
+    lambda: pins.test_bruteforce_tiny(True),
+    pins.test_hand_cases,
+    pins.test_invariants_beam_groups,
+    pins.test_all_groups_kept_is_plain_topk,
+    pins.test_single_expert_matches_torch_float64,
+    pins.test_k1_is_scaled_single_expert,
+    pins.test_forward_matches_torch_float64_composition,
+    pins.test_permute_matches_stable_argsort,
+]
+
+
+@contextlib.contextmanager
+def mutant_lib(tmp_path, name, old, new):
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutant {name}: snippet not found exactly once in the oracle"
+    path = tmp_path / f"{name}.c"
+    path.write_text(src.replace(old, new))
+    so = tmp_path / f"lib{name}.so"
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-o", str(so), str(path), "-lm"],
+                   check=True)
+    saved = oracle.lib()
+    oracle._lib = None
+    import oracle.build as ob
+    real_build = ob.build
+    ob.build = lambda *a, **k: str(so)
+    try:
+        oracle.lib()
+        yield
+    finally:
+        ob.build = real_build
+        oracle._lib = saved
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(tmp_path, name):
+    old, new = MUTANTS[name]
+    caught = []
+    with mutant_lib(tmp_path, name, old, new):
+        for pin in PINS:
+            try:
+                pin()
+            except (AssertionError, ValueError):
+                caught.append(pin)
+    assert caught, f"no pin caught the planted mistake '{name}'"
+
+
+def test_unmutated_copy_passes(tmp_path):
+    with mutant_lib(tmp_path, "identity", "int oracle_num_threads(void)", "int oracle_num_threads(void)"):
+        for pin in PINS:
+            pin()
