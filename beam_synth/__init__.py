@@ -14,7 +14,8 @@ SwiGLU intermediate 2,560; section "Attention": hidden size 5,120).  Distributio
   (fan-in scaling).
 
 Every tensor (and every expert of a weight tensor) has its own sub-seed derived from
-(workload seed, tensor id, expert).  Values depend on the generator device: the CPU generator
+(seed, tensor id, expert): x from the workload seed, W_r and the experts from the layer's weight
+seed (the Beam-shaped workloads are batches through one shared layer).  Values depend on the generator device: the CPU generator
 (Mersenne twister) and the CUDA generator (Philox) give different streams for one seed, so a
 workload states where each tensor is drawn (`expert_device`).  x and W_r are always drawn on the
 CPU; expert weights at Beam size are drawn on the GPU (20 GB would take minutes on the host) and
@@ -57,7 +58,12 @@ class Workload:
     outlier_scale: float = 30.0
     bias: str = "zero"            # "zero" or the name of a stored bias file under tests/golden/
     expert_device: str = "cpu"    # where expert weights are drawn ("cpu" or "cuda")
+    weight_seed: Optional[int] = None  # seed of the layer parameters (W_r, experts); default: seed
     description: str = ""
+
+    @property
+    def wseed(self) -> int:
+        return self.seed if self.weight_seed is None else self.weight_seed
 
     @property
     def layer(self) -> dict:
@@ -69,8 +75,10 @@ class Workload:
         return dataclasses.replace(self, T=T)
 
 
+# Beam-shaped workloads are batches through ONE layer: they share the layer parameters (seed 999)
+# and differ in T, x and the selection bias.
 _BEAM = dict(hidden=5120, inter=2560, n_experts=256, n_groups=8, topk_groups=4, topk=8,
-             group_topn=2, routed_scale=2.5, expert_device="cuda")
+             group_topn=2, routed_scale=2.5, expert_device="cuda", weight_seed=999)
 
 # The five Beam workloads (tiny brute-force case, decode, prefill, skewed routing, long prefill).
 WORKLOADS = {
@@ -144,7 +152,7 @@ def outlier_rows(wl: Workload, T: Optional[int] = None, seed_offset: int = 0) ->
 
 def make_router(wl: Workload) -> torch.Tensor:
     """W_r [E, H] fp32 on the CPU, N(0, 1/H)."""
-    g = _gen(sub_seed(wl.seed, "router"), "cpu")
+    g = _gen(sub_seed(wl.wseed, "router"), "cpu")
     return torch.randn(wl.n_experts, wl.hidden, generator=g, dtype=torch.float32) * (1.0 / wl.hidden) ** 0.5
 
 
@@ -173,7 +181,7 @@ def make_expert(wl: Workload, e: int, device: Optional[str] = None):
     H, I = wl.hidden, wl.inter
     out = []
     for name, shape, fan_in in (("gate", (I, H), H), ("up", (I, H), H), ("down", (H, I), I)):
-        g = _gen(sub_seed(wl.seed, name, e), device)
+        g = _gen(sub_seed(wl.wseed, name, e), device)
         w = torch.randn(*shape, generator=g, dtype=torch.float32, device=device) * (1.0 / fan_in) ** 0.5
         out.append(w.to(torch.bfloat16))
     return tuple(out)

@@ -1,0 +1,246 @@
+"""Beam MoE block forward pass on B200 (sm_100a): Python binding of libbeam_moe.so.
+
+Argument marshalling only: every step of the block runs in the library's CUDA kernels.  PyTorch
+provides device memory and the current stream.  There is no CPU fallback: if the library is not
+built, importing the binding's functions raises.
+
+The block (Beam launch post, "Welcome Beam" page, section "Mixture of Experts"): sigmoid router over
+256 experts, 8 contiguous groups of 32 ranked by the sum of their top-2 scores, 4 groups kept, top 8
+experts inside them, router weights normalised to sum 1, expert outputs combined and scaled by 2.5;
+each expert a SwiGLU MLP (hidden 5,120, intermediate 2,560).
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+import re
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "_lib", "libbeam_moe.so")
+HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "beam_moe.h")
+
+OK = 0
+ERR_INVALID_CONFIG = 1
+ERR_NULL = 2
+ERR_MISALIGNED = 3
+ERR_WORKSPACE_TOO_SMALL = 4
+ERR_UNSUPPORTED_DEVICE = 5
+ERR_CUDA = 6
+ERR_DEVICE_TIMEOUT = 7
+ERR_BAD_INDEX = 8
+ERR_INVALID_ARG = 9
+
+WS_ROUTE, WS_PERMUTE, WS_EXPERTS, WS_FORWARD = 0, 1, 2, 3
+
+
+class BeamMoeConfig(ctypes.Structure):
+    _fields_ = [("hidden", ctypes.c_int32), ("inter", ctypes.c_int32), ("n_experts", ctypes.c_int32),
+                ("n_groups", ctypes.c_int32), ("topk_groups", ctypes.c_int32), ("topk", ctypes.c_int32),
+                ("group_topn", ctypes.c_int32), ("routed_scale", ctypes.c_float)]
+
+
+@dataclasses.dataclass(frozen=True)
+class LayerConfig:
+    hidden: int = 5120
+    inter: int = 2560
+    n_experts: int = 256
+    n_groups: int = 8
+    topk_groups: int = 4
+    topk: int = 8
+    group_topn: int = 2
+    routed_scale: float = 2.5
+
+    def c(self) -> BeamMoeConfig:
+        return BeamMoeConfig(self.hidden, self.inter, self.n_experts, self.n_groups, self.topk_groups, self.topk,
+                             self.group_topn, self.routed_scale)
+
+
+BEAM_LAYER = LayerConfig()
+
+
+class BeamMoeError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {strerror(code)} (code {code})")
+
+
+_lib = None
+_vp = ctypes.c_void_p
+_cfgp = ctypes.POINTER(BeamMoeConfig)
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded CUDA library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m group_limited_routing_router_b200.build` (needs nvcc, sm_100a)")
+        L = ctypes.CDLL(LIB_PATH)
+        L.beam_moe_workspace_size.argtypes = [_cfgp, ctypes.c_int64, ctypes.c_int]
+        L.beam_moe_workspace_size.restype = ctypes.c_size_t
+        L.beam_moe_route.argtypes = [_cfgp, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp, _vp]
+        L.beam_moe_permute.argtypes = [_cfgp, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+        L.beam_moe_experts.argtypes = [_cfgp, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                       ctypes.c_size_t, _vp]
+        L.beam_moe_forward.argtypes = [_cfgp, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                       ctypes.c_size_t, _vp]
+        L.beam_moe_device_status.argtypes = [_vp]
+        L.beam_moe_selftest_timeout.argtypes = [ctypes.c_int64, _vp]
+        L.beam_moe_strerror.argtypes = [ctypes.c_int]
+        L.beam_moe_strerror.restype = ctypes.c_char_p
+        for name in ("beam_moe_route", "beam_moe_permute", "beam_moe_experts", "beam_moe_forward",
+                     "beam_moe_device_status", "beam_moe_selftest_timeout"):
+            getattr(L, name).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def declared_symbols() -> list:
+    """Entry points declared in include/beam_moe.h."""
+    with open(HEADER_PATH) as f:
+        return re.findall(r"BEAM_MOE_API\s+[\w\s\*]*?\b(beam_moe_\w+)\s*\(", f.read())
+
+
+def strerror(code: int) -> str:
+    return lib().beam_moe_strerror(int(code)).decode()
+
+
+def _check(code: int, where: str):
+    if code != OK:
+        raise BeamMoeError(code, where)
+
+
+def _cfg(cfg) -> BeamMoeConfig:
+    if isinstance(cfg, BeamMoeConfig):
+        return cfg
+    if isinstance(cfg, LayerConfig):
+        return cfg.c()
+    if isinstance(cfg, dict):
+        return LayerConfig(**cfg).c()
+    raise TypeError("cfg must be a LayerConfig, a dict of its fields or a BeamMoeConfig")
+
+
+def _dev(t: Optional[torch.Tensor], name: str, dtype, shape=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return t
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def workspace_size(cfg, T: int, which: int) -> int:
+    return int(lib().beam_moe_workspace_size(ctypes.byref(_cfg(cfg)), int(T), int(which)))
+
+
+def _workspace(cfg, T, which, ws, device):
+    need = workspace_size(cfg, T, which)
+    if ws is None:
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=device)
+    _dev(ws, "ws", torch.uint8)
+    return ws, ws.numel()
+
+
+def route(cfg, x: torch.Tensor, w_router: torch.Tensor, bias: Optional[torch.Tensor] = None,
+          ids: Optional[torch.Tensor] = None, w: Optional[torch.Tensor] = None, stream=None):
+    """Router: returns (topk_ids [T,k] int32, topk_w [T,k] fp32)."""
+    c = _cfg(cfg)
+    T = x.shape[0]
+    _dev(x, "x", torch.bfloat16, (T, c.hidden))
+    _dev(w_router, "w_router", torch.float32, (c.n_experts, c.hidden))
+    _dev(bias, "bias", torch.float32, (c.n_experts,))
+    ids = torch.empty(T, c.topk, dtype=torch.int32, device=x.device) if ids is None else ids
+    w = torch.empty(T, c.topk, dtype=torch.float32, device=x.device) if w is None else w
+    _dev(ids, "ids", torch.int32, (T, c.topk))
+    _dev(w, "w", torch.float32, (T, c.topk))
+    _check(lib().beam_moe_route(ctypes.byref(c), T, _ptr(x), _ptr(w_router), _ptr(bias), _ptr(ids), _ptr(w),
+                                _stream(stream)), "beam_moe_route")
+    return ids, w
+
+
+def permute(cfg, ids: torch.Tensor, ws: Optional[torch.Tensor] = None, stream=None) -> dict:
+    """Dispatch order: dict(counts [E] int32, offsets [E+1] int64, row_src [T*k], dest_row [T*k] int32)."""
+    c = _cfg(cfg)
+    T = ids.shape[0]
+    _dev(ids, "ids", torch.int32, (T, c.topk))
+    dev = ids.device
+    counts = torch.empty(c.n_experts, dtype=torch.int32, device=dev)
+    offsets = torch.empty(c.n_experts + 1, dtype=torch.int64, device=dev)
+    row_src = torch.empty(max(T * c.topk, 1), dtype=torch.int32, device=dev)
+    dest_row = torch.empty(max(T * c.topk, 1), dtype=torch.int32, device=dev)
+    ws, nbytes = _workspace(c, T, WS_PERMUTE, ws, dev)
+    _check(lib().beam_moe_permute(ctypes.byref(c), T, _ptr(ids), _ptr(counts), _ptr(offsets), _ptr(row_src),
+                                  _ptr(dest_row), _ptr(ws), nbytes, _stream(stream)), "beam_moe_permute")
+    return dict(counts=counts, offsets=offsets, row_src=row_src[:T * c.topk], dest_row=dest_row[:T * c.topk])
+
+
+def experts(cfg, x, ids, w, w_gate, w_up, w_down, y=None, ws=None, stream=None) -> torch.Tensor:
+    """Expert half for given routing: y [T,H] bf16 = scale * sum_j w[t,j] * E_{ids[t,j]}(x[t])."""
+    c = _cfg(cfg)
+    T = x.shape[0]
+    _dev(x, "x", torch.bfloat16, (T, c.hidden))
+    _dev(ids, "ids", torch.int32, (T, c.topk))
+    _dev(w, "w", torch.float32, (T, c.topk))
+    _dev(w_gate, "w_gate", torch.bfloat16, (c.n_experts, c.inter, c.hidden))
+    _dev(w_up, "w_up", torch.bfloat16, (c.n_experts, c.inter, c.hidden))
+    _dev(w_down, "w_down", torch.bfloat16, (c.n_experts, c.hidden, c.inter))
+    y = torch.empty(T, c.hidden, dtype=torch.bfloat16, device=x.device) if y is None else y
+    _dev(y, "y", torch.bfloat16, (T, c.hidden))
+    ws, nbytes = _workspace(c, T, WS_EXPERTS, ws, x.device)
+    _check(lib().beam_moe_experts(ctypes.byref(c), T, _ptr(x), _ptr(ids), _ptr(w), _ptr(w_gate), _ptr(w_up),
+                                  _ptr(w_down), _ptr(y), _ptr(ws), nbytes, _stream(stream)), "beam_moe_experts")
+    return y
+
+
+def forward(cfg, x, w_router, bias, w_gate, w_up, w_down, y=None, ids=None, w=None, ws=None, stream=None,
+            return_routing: bool = False):
+    """The whole block.  Returns y [T,H] bf16 (and (ids, w) when return_routing)."""
+    c = _cfg(cfg)
+    T = x.shape[0]
+    _dev(x, "x", torch.bfloat16, (T, c.hidden))
+    _dev(w_router, "w_router", torch.float32, (c.n_experts, c.hidden))
+    _dev(bias, "bias", torch.float32, (c.n_experts,))
+    _dev(w_gate, "w_gate", torch.bfloat16, (c.n_experts, c.inter, c.hidden))
+    _dev(w_up, "w_up", torch.bfloat16, (c.n_experts, c.inter, c.hidden))
+    _dev(w_down, "w_down", torch.bfloat16, (c.n_experts, c.hidden, c.inter))
+    y = torch.empty(T, c.hidden, dtype=torch.bfloat16, device=x.device) if y is None else y
+    _dev(y, "y", torch.bfloat16, (T, c.hidden))
+    if return_routing:
+        ids = torch.empty(T, c.topk, dtype=torch.int32, device=x.device) if ids is None else ids
+        w = torch.empty(T, c.topk, dtype=torch.float32, device=x.device) if w is None else w
+    _dev(ids, "ids", torch.int32, (T, c.topk))
+    _dev(w, "w", torch.float32, (T, c.topk))
+    ws, nbytes = _workspace(c, T, WS_FORWARD, ws, x.device)
+    _check(lib().beam_moe_forward(ctypes.byref(c), T, _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w_gate),
+                                  _ptr(w_up), _ptr(w_down), _ptr(y), _ptr(ids), _ptr(w), _ptr(ws), nbytes,
+                                  _stream(stream)), "beam_moe_forward")
+    return (y, ids, w) if return_routing else y
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream; return and clear the device status word."""
+    return int(lib().beam_moe_device_status(_stream(stream)))
+
+
+def selftest_timeout(timeout_us: int, stream=None):
+    _check(lib().beam_moe_selftest_timeout(int(timeout_us), _stream(stream)), "beam_moe_selftest_timeout")

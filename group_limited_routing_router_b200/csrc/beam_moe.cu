@@ -1,0 +1,395 @@
+// C ABI of the Beam MoE block forward pass on B200 (sm_100a): argument checks, workspace layout,
+// TMA descriptor encoding and the launch sequence
+//   router_topk -> permute_hist -> permute_scan -> permute_scatter -> gather_rows
+//   -> grouped GEMM (gate/up + SwiGLU) -> grouped GEMM (down) -> combine
+// all enqueued on the caller's stream with no host synchronisation.  The public contract is in
+// include/beam_moe.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/beam_moe.h"
+
+#include "common.cuh"
+#include "combine.cuh"
+#include "permute.cuh"
+#include "gemm.cuh"
+#include "router.cuh"
+
+namespace beam {
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int64_t kMaxTokens = int64_t(1) << 24;
+
+// ---- GEMM variants: (BN, smem stages, accumulator stages) -----------------------------------
+// "wide": experts see ~BN tokens (prefill); "narrow": a few tokens per expert (decode).
+using G1Wide = GemmCfg<true, 128, 4, 2>;
+using G2Wide = GemmCfg<false, 128, 6, 4>;
+using G1Narrow = GemmCfg<true, 32, 5, 2>;
+using G2Narrow = GemmCfg<false, 32, 8, 4>;
+#define G1_WIDE_KERNEL grouped_gemm_kernel<true, 128, 4, 2>
+#define G2_WIDE_KERNEL grouped_gemm_kernel<false, 128, 6, 4>
+#define G1_NARROW_KERNEL grouped_gemm_kernel<true, 32, 5, 2>
+#define G2_NARROW_KERNEL grouped_gemm_kernel<false, 32, 8, 4>
+
+struct DeviceInfo {
+    std::once_flag once;
+    int status = BEAM_MOE_OK;
+    int num_sms = 0;
+    int clock_khz = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+std::once_flag g_encode_once;
+EncodeTiledFn g_encode = nullptr;
+
+int init_device(int *dev_out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return BEAM_MOE_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return BEAM_MOE_ERR_UNSUPPORTED_DEVICE;
+    DeviceInfo &d = g_dev[dev];
+    std::call_once(d.once, [&]() {
+        int major = 0, minor = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.clock_khz, cudaDevAttrClockRate, dev) != cudaSuccess) {
+            d.status = BEAM_MOE_ERR_CUDA;
+            return;
+        }
+        if (major != 10 || minor != 0) {
+            d.status = BEAM_MOE_ERR_UNSUPPORTED_DEVICE;
+            return;
+        }
+        bool ok = cudaFuncSetAttribute(router_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kRtSmemFloats * 4) == cudaSuccess;
+        ok = ok && cudaFuncSetAttribute(G1_WIDE_KERNEL, cudaFuncAttributeMaxDynamicSharedMemorySize, G1Wide::kSmem) ==
+                       cudaSuccess;
+        ok = ok && cudaFuncSetAttribute(G2_WIDE_KERNEL, cudaFuncAttributeMaxDynamicSharedMemorySize, G2Wide::kSmem) ==
+                       cudaSuccess;
+        ok = ok && cudaFuncSetAttribute(G1_NARROW_KERNEL, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        G1Narrow::kSmem) == cudaSuccess;
+        ok = ok && cudaFuncSetAttribute(G2_NARROW_KERNEL, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        G2Narrow::kSmem) == cudaSuccess;
+        if (!ok) d.status = BEAM_MOE_ERR_CUDA;
+    });
+    *dev_out = dev;
+    return d.status;
+}
+
+EncodeTiledFn encode_fn() {
+    std::call_once(g_encode_once, []() {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    });
+    return g_encode;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int validate(const beam_moe_config *c) {
+    if (!c) return BEAM_MOE_ERR_NULL;
+    if (c->hidden < 64 || c->hidden > 65536 || c->hidden % 64 || c->inter < 64 || c->inter > 65536 ||
+        c->inter % 64)
+        return BEAM_MOE_ERR_INVALID_CONFIG;
+    if (c->n_experts < 1 || c->n_experts > 256 || c->n_groups < 1 || c->n_groups > 32 ||
+        c->n_experts % c->n_groups)
+        return BEAM_MOE_ERR_INVALID_CONFIG;
+    const int per = c->n_experts / c->n_groups;
+    if (c->topk_groups < 1 || c->topk_groups > c->n_groups) return BEAM_MOE_ERR_INVALID_CONFIG;
+    if (c->topk < 1 || c->topk > 16 || c->topk > c->topk_groups * per) return BEAM_MOE_ERR_INVALID_CONFIG;
+    if (c->group_topn < 1 || c->group_topn > 8 || c->group_topn > per) return BEAM_MOE_ERR_INVALID_CONFIG;
+    if (!(c->routed_scale == c->routed_scale)) return BEAM_MOE_ERR_INVALID_CONFIG;  // NaN
+    return BEAM_MOE_OK;
+}
+
+int check_T(const beam_moe_config *c, int64_t T) {
+    if (T < 0 || T > kMaxTokens || T * c->topk >= (int64_t(1) << 31)) return BEAM_MOE_ERR_INVALID_ARG;
+    return BEAM_MOE_OK;
+}
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+struct Layout {
+    size_t ids = 0, w = 0, hist = 0, counts = 0, offsets = 0, row_src = 0, dest_row = 0, xp = 0, h = 0, o = 0;
+    size_t total = 0;
+};
+
+int64_t n_chunks(int64_t T) { return (T + kPmTok - 1) / kPmTok; }
+
+Layout layout(const beam_moe_config *c, int64_t T, int which) {
+    Layout L;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off = align256(off + bytes);
+        return at;
+    };
+    const size_t R = static_cast<size_t>(T) * c->topk;
+    const size_t E = c->n_experts, H = c->hidden, I = c->inter;
+    if (which == BEAM_MOE_WS_ROUTE || T == 0) return L;
+    if (which == BEAM_MOE_WS_FORWARD) {
+        L.ids = take(R * 4);
+        L.w = take(R * 4);
+    }
+    L.hist = take(static_cast<size_t>(n_chunks(T)) * E * 4);
+    if (which == BEAM_MOE_WS_PERMUTE) {
+        L.total = off;
+        return L;
+    }
+    L.counts = take(E * 4);
+    L.offsets = take((E + 1) * 8);
+    L.row_src = take(R * 4);
+    L.dest_row = take(R * 4);
+    L.xp = take(R * H * 2);
+    L.h = take(R * I * 2);
+    L.o = take(R * H * 4);
+    L.total = off;
+    return L;
+}
+
+// 2D [rows][K] bf16 tensor, box {64, box_rows}, 128-byte swizzle.
+bool make_map_2d(CUtensorMap *m, const void *base, uint64_t K, uint64_t rows, uint32_t box_rows) {
+    const cuuint64_t dims[2] = {K, rows};
+    const cuuint64_t strides[1] = {K * 2};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3D [E][M][K] bf16 weights, box {64, 128, 1}, 128-byte swizzle.
+bool make_map_3d(CUtensorMap *m, const void *base, uint64_t K, uint64_t M, uint64_t E) {
+    const cuuint64_t dims[3] = {K, M, E};
+    const cuuint64_t strides[2] = {K * 2, K * M * 2};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kBK), static_cast<cuuint32_t>(kBM), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? BEAM_MOE_OK : BEAM_MOE_ERR_CUDA; }
+
+int enqueue_route(const beam_moe_config *c, int64_t T, const beam_bf16 *x, const float *w_router, const float *bias,
+                  int32_t *ids, float *w, cudaStream_t s) {
+    RouterParams p;
+    p.x = reinterpret_cast<const __nv_bfloat16 *>(x);
+    p.w = w_router;
+    p.bias = bias;
+    p.ids = ids;
+    p.wts = w;
+    p.T = T;
+    p.H = c->hidden;
+    p.E = c->n_experts;
+    p.G = c->n_groups;
+    p.topk_groups = c->topk_groups;
+    p.topk = c->topk;
+    p.group_topn = c->group_topn;
+    const int64_t tiles = (T + kRtTok - 1) / kRtTok;
+    router_topk_kernel<<<static_cast<unsigned>(tiles * kRtCluster), kRtThreads, kRtSmemFloats * 4, s>>>(p);
+    return launch_status();
+}
+
+int enqueue_permute(const beam_moe_config *c, int64_t T, const int32_t *ids, int32_t *counts, int64_t *offsets,
+                    int32_t *row_src, int32_t *dest_row, int32_t *hist, cudaStream_t s) {
+    const int nc = static_cast<int>(n_chunks(T));
+    permute_hist_kernel<<<nc, kPmThreads, 0, s>>>(ids, T, c->topk, c->n_experts, hist);
+    permute_scan_kernel<<<1, 1024, 0, s>>>(hist, nc, c->n_experts, counts, offsets);
+    permute_scatter_kernel<<<nc, kPmThreads, 0, s>>>(ids, T, c->topk, c->n_experts, hist, offsets, row_src,
+                                                    dest_row);
+    return launch_status();
+}
+
+int enqueue_experts(const beam_moe_config *c, int dev, int64_t T, const beam_bf16 *x, const int32_t *ids,
+                    const float *w, const beam_bf16 *wg, const beam_bf16 *wu, const beam_bf16 *wd, beam_bf16 *y,
+                    uint8_t *ws, const Layout &L, cudaStream_t s) {
+    int32_t *counts = reinterpret_cast<int32_t *>(ws + L.counts);
+    int64_t *offsets = reinterpret_cast<int64_t *>(ws + L.offsets);
+    int32_t *row_src = reinterpret_cast<int32_t *>(ws + L.row_src);
+    int32_t *dest_row = reinterpret_cast<int32_t *>(ws + L.dest_row);
+    int32_t *hist = reinterpret_cast<int32_t *>(ws + L.hist);
+    void *xp = ws + L.xp;
+    void *h = ws + L.h;
+    void *o = ws + L.o;
+    const int k = c->topk, E = c->n_experts, H = c->hidden, I = c->inter;
+    const uint64_t R = static_cast<uint64_t>(T) * k;
+
+    int rc = enqueue_permute(c, T, ids, counts, offsets, row_src, dest_row, hist, s);
+    if (rc) return rc;
+    gather_rows_kernel<<<static_cast<unsigned>(T), 128, 0, s>>>(reinterpret_cast<const uint4 *>(x), T, k, H / 8,
+                                                                dest_row, reinterpret_cast<uint4 *>(xp));
+    if ((rc = launch_status())) return rc;
+
+    const bool narrow = static_cast<double>(R) / E <= 24.0;
+    const int bn = narrow ? 32 : 128;
+    CUtensorMap m_wg, m_wu, m_xp, m_wd, m_h;
+    if (!encode_fn()) return BEAM_MOE_ERR_CUDA;
+    if (!make_map_3d(&m_wg, wg, H, I, E) || !make_map_3d(&m_wu, wu, H, I, E) || !make_map_2d(&m_xp, xp, H, R, bn) ||
+        !make_map_3d(&m_wd, wd, I, H, E) || !make_map_2d(&m_h, h, I, R, bn))
+        return BEAM_MOE_ERR_CUDA;
+    const int grid = g_dev[dev].num_sms;
+    GemmParams p1{counts, offsets, h, E, H, I, kDefaultTimeoutCycles};
+    GemmParams p2{counts, offsets, o, E, I, H, kDefaultTimeoutCycles};
+    if (narrow) {
+        G1_NARROW_KERNEL<<<grid, kGemmThreads, G1Narrow::kSmem, s>>>(m_wg, m_wu, m_xp, p1);
+        G2_NARROW_KERNEL<<<grid, kGemmThreads, G2Narrow::kSmem, s>>>(m_wd, m_wd, m_h, p2);
+    } else {
+        G1_WIDE_KERNEL<<<grid, kGemmThreads, G1Wide::kSmem, s>>>(m_wg, m_wu, m_xp, p1);
+        G2_WIDE_KERNEL<<<grid, kGemmThreads, G2Wide::kSmem, s>>>(m_wd, m_wd, m_h, p2);
+    }
+    if ((rc = launch_status())) return rc;
+    combine_kernel<<<static_cast<unsigned>(T), 256, 0, s>>>(reinterpret_cast<const float4 *>(o), dest_row, w, T, k,
+                                                            H / 4, c->routed_scale, reinterpret_cast<uint2 *>(y));
+    return launch_status();
+}
+
+__global__ void selftest_timeout_kernel(long long cycles) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        mbar_wait(&bar, 0, cycles);  // nobody arrives: the bounded wait expires and records the status
+    }
+}
+
+}  // namespace
+}  // namespace beam
+
+using namespace beam;
+
+extern "C" {
+
+size_t beam_moe_workspace_size(const beam_moe_config *cfg, int64_t T, int which) {
+    if (validate(cfg) || check_T(cfg, T)) return 0;
+    if (which < BEAM_MOE_WS_ROUTE || which > BEAM_MOE_WS_FORWARD) return 0;
+    return layout(cfg, T, which).total;
+}
+
+int beam_moe_route(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const float *w_router,
+                   const float *sel_bias, int32_t *topk_ids, float *topk_w, void *stream) {
+    int rc = validate(cfg);
+    if (rc) return rc;
+    if ((rc = check_T(cfg, T))) return rc;
+    if (!x || !w_router || !topk_ids || !topk_w) return BEAM_MOE_ERR_NULL;
+    if (!aligned16(x) || !aligned16(w_router)) return BEAM_MOE_ERR_MISALIGNED;
+    if (T == 0) return BEAM_MOE_OK;
+    int dev;
+    if ((rc = init_device(&dev))) return rc;
+    return enqueue_route(cfg, T, x, w_router, sel_bias, topk_ids, topk_w, static_cast<cudaStream_t>(stream));
+}
+
+int beam_moe_permute(const beam_moe_config *cfg, int64_t T, const int32_t *topk_ids, int32_t *counts,
+                     int64_t *offsets, int32_t *row_src, int32_t *dest_row, void *ws, size_t ws_bytes,
+                     void *stream) {
+    int rc = validate(cfg);
+    if (rc) return rc;
+    if ((rc = check_T(cfg, T))) return rc;
+    if (!counts || !offsets || (T > 0 && (!topk_ids || !row_src || !dest_row || !ws))) return BEAM_MOE_ERR_NULL;
+    if (ws && !aligned16(ws)) return BEAM_MOE_ERR_MISALIGNED;
+    const Layout L = layout(cfg, T, BEAM_MOE_WS_PERMUTE);
+    if (ws_bytes < L.total) return BEAM_MOE_ERR_WORKSPACE_TOO_SMALL;
+    int dev;
+    if ((rc = init_device(&dev))) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        // counts = 0, offsets = 0 keep the outputs well defined
+        if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * cfg->n_experts, s) != cudaSuccess ||
+            cudaMemsetAsync(offsets, 0, sizeof(int64_t) * (cfg->n_experts + 1), s) != cudaSuccess)
+            return BEAM_MOE_ERR_CUDA;
+        return BEAM_MOE_OK;
+    }
+    return enqueue_permute(cfg, T, topk_ids, counts, offsets, row_src, dest_row,
+                           reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + L.hist), s);
+}
+
+int beam_moe_experts(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const int32_t *topk_ids,
+                     const float *topk_w, const beam_bf16 *w_gate, const beam_bf16 *w_up, const beam_bf16 *w_down,
+                     beam_bf16 *y, void *ws, size_t ws_bytes, void *stream) {
+    int rc = validate(cfg);
+    if (rc) return rc;
+    if ((rc = check_T(cfg, T))) return rc;
+    if (!x || !topk_ids || !topk_w || !w_gate || !w_up || !w_down || !y || (T > 0 && !ws)) return BEAM_MOE_ERR_NULL;
+    if (!aligned16(x) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) || !aligned16(y) ||
+        (ws && !aligned16(ws)))
+        return BEAM_MOE_ERR_MISALIGNED;
+    const Layout L = layout(cfg, T, BEAM_MOE_WS_EXPERTS);
+    if (ws_bytes < L.total) return BEAM_MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (T == 0) return BEAM_MOE_OK;
+    int dev;
+    if ((rc = init_device(&dev))) return rc;
+    return enqueue_experts(cfg, dev, T, x, topk_ids, topk_w, w_gate, w_up, w_down, y, static_cast<uint8_t *>(ws), L,
+                           static_cast<cudaStream_t>(stream));
+}
+
+int beam_moe_forward(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const float *w_router,
+                     const float *sel_bias, const beam_bf16 *w_gate, const beam_bf16 *w_up, const beam_bf16 *w_down,
+                     beam_bf16 *y, int32_t *topk_ids_out, float *topk_w_out, void *ws, size_t ws_bytes, void *stream) {
+    int rc = validate(cfg);
+    if (rc) return rc;
+    if ((rc = check_T(cfg, T))) return rc;
+    if (!x || !w_router || !w_gate || !w_up || !w_down || !y || (T > 0 && !ws)) return BEAM_MOE_ERR_NULL;
+    if (!aligned16(x) || !aligned16(w_router) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) ||
+        !aligned16(y) || (ws && !aligned16(ws)))
+        return BEAM_MOE_ERR_MISALIGNED;
+    const Layout L = layout(cfg, T, BEAM_MOE_WS_FORWARD);
+    if (ws_bytes < L.total) return BEAM_MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (T == 0) return BEAM_MOE_OK;
+    int dev;
+    if ((rc = init_device(&dev))) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+    int32_t *ids = topk_ids_out ? topk_ids_out : reinterpret_cast<int32_t *>(wsb + L.ids);
+    float *w = topk_w_out ? topk_w_out : reinterpret_cast<float *>(wsb + L.w);
+    if ((rc = enqueue_route(cfg, T, x, w_router, sel_bias, ids, w, s))) return rc;
+    return enqueue_experts(cfg, dev, T, x, ids, w, w_gate, w_up, w_down, y, wsb, L, s);
+}
+
+int beam_moe_device_status(void *stream) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int v = BEAM_MOE_OK;
+    const int zero = BEAM_MOE_OK;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return BEAM_MOE_ERR_CUDA;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return BEAM_MOE_ERR_CUDA;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return BEAM_MOE_ERR_CUDA;
+    return v;
+}
+
+int beam_moe_selftest_timeout(int64_t timeout_us, void *stream) {
+    if (timeout_us < 1 || timeout_us > 1000000) return BEAM_MOE_ERR_INVALID_ARG;
+    int dev, rc;
+    if ((rc = init_device(&dev))) return rc;
+    const long long cycles = static_cast<long long>(timeout_us) * g_dev[dev].clock_khz / 1000;
+    selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(cycles);
+    return launch_status();
+}
+
+const char *beam_moe_strerror(int code) {
+    switch (code) {
+        case BEAM_MOE_OK: return "ok";
+        case BEAM_MOE_ERR_INVALID_CONFIG: return "invalid layer configuration";
+        case BEAM_MOE_ERR_NULL: return "a required pointer is NULL";
+        case BEAM_MOE_ERR_MISALIGNED: return "a pointer is not 16-byte aligned";
+        case BEAM_MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case BEAM_MOE_ERR_UNSUPPORTED_DEVICE: return "unsupported device (needs compute capability 10.0, sm_100a)";
+        case BEAM_MOE_ERR_CUDA: return "CUDA runtime or launch error";
+        case BEAM_MOE_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait timed out";
+        case BEAM_MOE_ERR_BAD_INDEX: return "an expert id outside [0, n_experts)";
+        case BEAM_MOE_ERR_INVALID_ARG: return "invalid argument (token count out of range)";
+        default: return "unknown error code";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,284 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM, TMA-fed).
+//
+//   G1 (gate/up + SwiGLU): for expert e and its rows r (tokens routed to e, in dispatch order)
+//        h[r, i] = SiLU(x[r] . W_gate[e, i]) * (x[r] . W_up[e, i])          (FP32, stored bf16)
+//   G2 (down):  o[r, j] = h[r] . W_down[e, j]                                 (FP32)
+// "each a SwiGLU MLP with an intermediate size of 2,560" ("Welcome Beam" page, section "Mixture of
+// Experts"); the SwiGLU product is computed in FP32 (section "Residual Stream").
+//
+// Orientation (swap-AB): the MMA's M side (128) walks the expert's weight rows, its N side the
+// expert's tokens (N = tokens rounded up to 16, at most BN).  At the Beam shapes an expert sees
+// ~8 tokens in a decode batch and ~128 in a 4096-token prefill, so putting tokens on N lets one
+// tile cover all of an expert's tokens and every weight byte crosses HBM once per call.
+//
+// Work item = (expert e, weight-row tile mt of 128, token tile nt of BN).  Items are numbered
+// expert-major, then mt, then nt, from the per-expert counts (read on the device; no host sync);
+// a persistent grid of one CTA per SM takes items round-robin.
+//
+// Warp roles (256 threads): warp 0 lane 0 = TMA producer; warp 1 = TMEM owner, lane 0 issues
+// tcgen05.mma; warps 4..7 = epilogue (warp 4+q reads TMEM lanes 32q..32q+31).  Shared memory is a
+// STAGES-deep ring of {A tile(s) 128x64 bf16, B tile BNx64 bf16}, 128-byte swizzled by TMA; TMEM
+// holds ACC double-buffered accumulators so the epilogue of one item overlaps the next item's MMAs.
+// Every wait is bounded (status word BEAM_MOE_ERR_DEVICE_TIMEOUT on expiry).
+#pragma once
+
+#include "common.cuh"
+
+namespace beam {
+
+constexpr int kBM = 128;  // weight rows per tile (UMMA M)
+constexpr int kBK = 64;   // K per stage: one 128-byte swizzle row of bf16
+constexpr int kGemmThreads = 256;
+
+constexpr int pow2_cols(int c) { return c <= 32 ? 32 : c <= 64 ? 64 : c <= 128 ? 128 : c <= 256 ? 256 : 512; }
+
+template <bool GATE_UP, int BN, int STAGES, int ACC>
+struct GemmCfg {
+    static constexpr int kA = kBM * kBK * 2;                 // one A tile, bytes
+    static constexpr int kB = BN * kBK * 2;                  // B tile, bytes
+    static constexpr int kNumA = GATE_UP ? 2 : 1;
+    static constexpr int kStage = kNumA * kA + kB;           // multiple of 1024
+    static constexpr int kAccCols = (GATE_UP ? 2 : 1) * BN;  // TMEM columns per accumulator stage
+    static constexpr int kTmemCols = pow2_cols(ACC * kAccCols);
+    static constexpr int kBarOff = STAGES * kStage;
+    static constexpr int kSmem = 1024 + kBarOff + 256 + 4 * (kPmMaxE + 1) + 64;
+    static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
+    static_assert(ACC * kAccCols <= 512, "TMEM has 512 columns");
+    static_assert(BN % 16 == 0 && BN <= 256, "UMMA N");
+};
+
+struct GemmParams {
+    const int32_t *counts;    // [E]
+    const int64_t *offsets;   // [E + 1]
+    void *out;                // G1: h [R, I] bf16; G2: o [R, H] fp32
+    int E;
+    int K;                    // reduction length (G1: H, G2: I)
+    int M;                    // weight rows (G1: I, G2: H)
+    long long timeout;
+};
+
+// Work-item decode from the per-CTA prefix table.
+struct Item {
+    int e, mt, nt, n_valid;
+    int64_t row0;
+};
+
+__device__ __forceinline__ Item decode_item(int item, const int *tile_start, int E, int n_mt, int BN,
+                                            const int32_t *counts, const int64_t *offsets) {
+    int lo = 0, hi = E - 1;  // largest e with tile_start[e] <= item
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (tile_start[mid] <= item) lo = mid;
+        else hi = mid - 1;
+    }
+    Item it;
+    it.e = lo;
+    const int cnt = counts[lo];
+    const int n_nt = (cnt + BN - 1) / BN;
+    const int local = item - tile_start[lo];
+    it.mt = local / n_nt;
+    it.nt = local - it.mt * n_nt;
+    it.n_valid = min(BN, cnt - it.nt * BN);
+    it.row0 = offsets[lo] + static_cast<int64_t>(it.nt) * BN;
+    return it;
+}
+
+template <bool GATE_UP, int BN, int STAGES, int ACC>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a0,  // W_gate (G1) / W_down (G2): [E][M][K]
+                        const __grid_constant__ CUtensorMap tm_a1,  // W_up (G1); unused for G2
+                        const __grid_constant__ CUtensorMap tm_b,   // x_perm (G1) / h (G2): [R][K]
+                        const GemmParams p) {
+    using C = GemmCfg<GATE_UP, BN, STAGES, ACC>;
+    extern __shared__ uint8_t gemm_smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(gemm_smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
+    uint64_t *empty = full + STAGES;
+    uint64_t *acc_full = empty + STAGES;
+    uint64_t *acc_empty = acc_full + ACC;
+    uint64_t *drain = acc_empty + ACC;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    int *tile_start = reinterpret_cast<int *>(smem + C::kBarOff + 256);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int E = p.E;
+    const int n_mt = (p.M + kBM - 1) / kBM;
+    const int n_kb = p.K / kBK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < ACC; ++a) {
+            mbar_init(&acc_full[a], 1);
+            mbar_init(&acc_empty[a], 4);
+        }
+        mbar_init(drain, 1);
+        fence_mbar_init();
+        prefetch_tensormap(&tm_a0);
+        if (GATE_UP) prefetch_tensormap(&tm_a1);
+        prefetch_tensormap(&tm_b);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    // per-expert item counts -> exclusive prefix (E <= 256 = blockDim.x)
+    {
+        __shared__ int warp_tot[kGemmThreads / 32];
+        const int e = threadIdx.x;
+        const int v = e < E ? n_mt * ((p.counts[e] + BN - 1) / BN) : 0;
+        int incl = v;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += o;
+        }
+        if (lane == 31) warp_tot[warp] = incl;
+        __syncthreads();
+        int base = 0;
+        for (int w = 0; w < warp; ++w) base += warp_tot[w];
+        if (e < E) tile_start[e] = base + incl - v;
+        if (e == E - 1) tile_start[E] = base + incl;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = tile_start[E];
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer ----------------
+            const uint64_t pol_w = policy_evict_first();  // weights: streamed once
+            const uint64_t pol_x = policy_evict_last();   // activations: re-read by other tiles
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued = 0, issued_phase = 0;  // per-stage: ever issued / phase of last issue
+            bool ok = true;
+            for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+                const Item it = decode_item(item, tile_start, E, n_mt, BN, p.counts, p.offsets);
+                for (int kb = 0; kb < n_kb; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, p.timeout)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *sa = smem + stage * C::kStage;
+                    mbar_arrive_expect_tx(&full[stage], C::kStage);
+                    tma_load_3d(sa, &tm_a0, &full[stage], kb * kBK, it.mt * kBM, it.e, pol_w);
+                    if (GATE_UP) tma_load_3d(sa + C::kA, &tm_a1, &full[stage], kb * kBK, it.mt * kBM, it.e, pol_w);
+                    tma_load_2d(sa + C::kNumA * C::kA, &tm_b, &full[stage], kb * kBK, static_cast<int>(it.row0), pol_x);
+                    issued |= 1u << stage;
+                    issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            // every load this thread issued has landed before the CTA may exit
+            for (int s = 0; s < STAGES; ++s)
+                if ((issued >> s) & 1u) mbar_wait(&full[s], (issued_phase >> s) & 1u, p.timeout);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer ----------------
+            int stage = 0, acc = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+                const Item it = decode_item(item, tile_start, E, n_mt, BN, p.counts, p.offsets);
+                const int n_mma = (it.n_valid + 15) & ~15;
+                const uint32_t idesc = umma_idesc_bf16(kBM, n_mma);
+                if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, p.timeout)) break;
+                tc_fence_after();
+                const uint32_t d0 = tmem_base + static_cast<uint32_t>(acc * C::kAccCols);
+                for (int kb = 0; kb < n_kb; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, p.timeout)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + stage * C::kStage);
+                    const uint64_t da0 = umma_desc_sw128(sa);
+                    const uint64_t da1 = umma_desc_sw128(sa + C::kA);
+                    const uint64_t db = umma_desc_sw128(sa + C::kNumA * C::kA);
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+                        // +32 bytes along K inside the swizzle row = +2 in the 16-byte address field
+                        umma_bf16(d0, da0 + 2 * kk, db + 2 * kk, idesc, accum);
+                        if (GATE_UP) umma_bf16(d0 + BN, da1 + 2 * kk, db + 2 * kk, idesc, accum);
+                    }
+                    umma_commit(&empty[stage]);  // frees the smem stage once these MMAs completed
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit(&acc_full[acc]);  // accumulator ready for the epilogue
+                if (++acc == ACC) {
+                    acc = 0;
+                    acc_phase ^= 1u;
+                }
+            }
+            // all issued MMAs complete before TMEM is released
+            umma_commit(drain);
+            mbar_wait(drain, 0, p.timeout);
+        }
+    } else if (warp >= 4) {
+        // ---------------- epilogue ----------------
+        const int q = warp - 4;  // TMEM lane quadrant
+        int acc = 0;
+        uint32_t acc_phase = 0;
+        for (int item = blockIdx.x; item < total; item += gridDim.x) {
+            const Item it = decode_item(item, tile_start, E, n_mt, BN, p.counts, p.offsets);
+            if (!mbar_wait(&acc_full[acc], acc_phase, p.timeout)) break;
+            tc_fence_after();
+            const int m = it.mt * kBM + q * 32 + lane;  // weight row of this thread
+            const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * C::kAccCols);
+            for (int c = 0; c < it.n_valid; c += 16) {
+                uint32_t r0[16];
+                tmem_ld16(tb + c, r0);
+                if (GATE_UP) {
+                    uint32_t r1[16];
+                    tmem_ld16(tb + BN + c, r1);
+                    tmem_ld_wait();
+                    if (m < p.M) {
+                        __nv_bfloat16 *h = reinterpret_cast<__nv_bfloat16 *>(p.out);
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            if (c + j < it.n_valid)
+                                h[(it.row0 + c + j) * p.M + m] =
+                                    __float2bfloat16_rn(silu_mul(__uint_as_float(r0[j]), __uint_as_float(r1[j])));
+                    }
+                } else {
+                    tmem_ld_wait();
+                    if (m < p.M) {
+                        float *o = reinterpret_cast<float *>(p.out);
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            if (c + j < it.n_valid) o[(it.row0 + c + j) * p.M + m] = __uint_as_float(r0[j]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+            if (++acc == ACC) {
+                acc = 0;
+                acc_phase ^= 1u;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+}
+
+}  // namespace beam

@@ -1,0 +1,254 @@
+// Router kernel R: FP32 router projection + sigmoid + group-limited top-k + weight normalisation.
+//
+// Beam launch post ("Welcome Beam" page, section "Mixture of Experts"): the router scores all
+// experts with a sigmoid, splits them into groups, keeps the best groups ranked by the sum of
+// each group's top-2 scores, then picks the top experts inside them; outputs are combined with
+// normalised router weights.  Section "Residual Stream": the router computes in FP32.
+//
+// Layout of the work (sm_100a):
+//   * one thread-block cluster of 8 CTAs per tile of 64 tokens; CTA r of the cluster computes the
+//     partial logits of all 64 tokens x 256 expert slots over the r-th eighth of the hidden
+//     dimension (split-K), with an 8x8 register tile per thread and double-buffered shared-memory
+//     staging (x widened from bf16 to fp32, which is exact);
+//   * the partial logits stay in each CTA's shared memory; after a cluster barrier, CTA r reduces
+//     tokens [8r, 8r+8) over the 8 CTAs through distributed shared memory, in rank order, so the
+//     FP32 sum order is fixed (deterministic);
+//   * one warp per token then does the selection with warp shuffles: lane l owns experts
+//     l, l+32, ..., each (value, index) comparison breaks ties toward the lower index, and every
+//     sum is taken in a fixed order (group score = top1 + top2 in pick order; weight denominator
+//     in slot order).
+#pragma once
+
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+
+namespace beam {
+
+namespace cg = cooperative_groups;
+
+constexpr int kRtTok = 64;       // tokens per cluster tile
+constexpr int kRtBK = 32;        // K per shared-memory stage
+constexpr int kRtThreads = 256;  // 8 warps
+constexpr int kRtCluster = 8;    // CTAs per cluster (split-K factor)
+constexpr int kRtSlots = 256;    // expert slots per tile (E <= 256)
+constexpr int kRtSmemFloats = 2 * kRtBK * kRtSlots + 2 * kRtBK * kRtTok;  // 20480 floats = 80 KB
+static_assert(kRtTok * kRtSlots <= 2 * kRtBK * kRtSlots, "partial logits must fit in the W staging area");
+
+struct RouterParams {
+    const __nv_bfloat16 *x;  // [T, H]
+    const float *w;          // [E, H]
+    const float *bias;       // [E] or nullptr
+    int32_t *ids;            // [T, k]
+    float *wts;              // [T, k]
+    int64_t T;
+    int H, E, G, topk_groups, topk, group_topn;
+};
+
+struct ArgMax {
+    float v;
+    int i;
+};
+
+// Warp-wide argmax of (value desc, index asc); every lane gets the winner.
+__device__ __forceinline__ ArgMax warp_argmax(float v, int i) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, v, off);
+        const int oi = __shfl_xor_sync(0xffffffffu, i, off);
+        if (ov > v || (ov == v && oi < i)) {
+            v = ov;
+            i = oi;
+        }
+    }
+    return {v, i};
+}
+
+__global__ void __cluster_dims__(kRtCluster, 1, 1) __launch_bounds__(kRtThreads, 1)
+    router_topk_kernel(const RouterParams p) {
+    extern __shared__ float4 rt_smem4[];
+    float *smem = reinterpret_cast<float *>(rt_smem4);
+    float *ws = smem;                            // [2][kRtBK][kRtSlots]
+    float *xs = smem + 2 * kRtBK * kRtSlots;     // [2][kRtBK][kRtTok]
+    float *part = smem;                          // [kRtTok][kRtSlots] after the K loop
+
+    cg::cluster_group cluster = cg::this_cluster();
+    const int rank = static_cast<int>(cluster.block_rank());
+    const int64_t t0 = static_cast<int64_t>(blockIdx.x / kRtCluster) * kRtTok;
+    const int tid = threadIdx.x;
+    const int tx = tid & 31, ty = tid >> 5;
+
+    // ---- split-K FP32 projection --------------------------------------------------------------
+    const int nsteps = p.H / kRtBK;
+    const int s_begin = rank * nsteps / kRtCluster;
+    const int s_end = (rank + 1) * nsteps / kRtCluster;
+
+    float acc[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
+
+    const int we = tid;  // expert row this thread stages
+    const bool w_ok = we < p.E;
+    const float *wrow = p.w + static_cast<int64_t>(w_ok ? we : 0) * p.H;
+    const int xt = tid & 63, xc = (tid >> 6) * 8;  // token, k-chunk of 8 this thread stages
+    const bool x_ok = (t0 + xt) < p.T;
+    const __nv_bfloat16 *xrow = p.x + (x_ok ? (t0 + xt) : 0) * static_cast<int64_t>(p.H);
+
+    float4 wreg[8];
+    uint4 xreg;
+    auto gload = [&](int s) {
+        const int k0 = s * kRtBK;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            wreg[i] = w_ok ? __ldg(reinterpret_cast<const float4 *>(wrow + k0) + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        xreg = x_ok ? __ldg(reinterpret_cast<const uint4 *>(xrow + k0 + xc)) : make_uint4(0u, 0u, 0u, 0u);
+    };
+    auto sstore = [&](int buf) {
+        float *wsb = ws + buf * kRtBK * kRtSlots;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            wsb[(4 * i + 0) * kRtSlots + we] = wreg[i].x;
+            wsb[(4 * i + 1) * kRtSlots + we] = wreg[i].y;
+            wsb[(4 * i + 2) * kRtSlots + we] = wreg[i].z;
+            wsb[(4 * i + 3) * kRtSlots + we] = wreg[i].w;
+        }
+        float *xsb = xs + buf * kRtBK * kRtTok;
+        const uint32_t xw[4] = {xreg.x, xreg.y, xreg.z, xreg.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            // bf16 -> fp32 is a 16-bit shift of the bit pattern (exact)
+            xsb[(xc + 2 * i) * kRtTok + xt] = __uint_as_float(xw[i] << 16);
+            xsb[(xc + 2 * i + 1) * kRtTok + xt] = __uint_as_float(xw[i] & 0xffff0000u);
+        }
+    };
+
+    if (s_begin < s_end) {
+        gload(s_begin);
+        sstore(0);
+        __syncthreads();
+        for (int s = s_begin; s < s_end; ++s) {
+            const int buf = (s - s_begin) & 1;
+            if (s + 1 < s_end) gload(s + 1);
+            const float *wsb = ws + buf * kRtBK * kRtSlots + tx * 8;
+            const float *xsb = xs + buf * kRtBK * kRtTok + ty * 8;
+#pragma unroll 8
+            for (int kk = 0; kk < kRtBK; ++kk) {
+                const float4 xa = *reinterpret_cast<const float4 *>(xsb + kk * kRtTok);
+                const float4 xb = *reinterpret_cast<const float4 *>(xsb + kk * kRtTok + 4);
+                const float4 wa = *reinterpret_cast<const float4 *>(wsb + kk * kRtSlots);
+                const float4 wb = *reinterpret_cast<const float4 *>(wsb + kk * kRtSlots + 4);
+                const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+                const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(xv[i], wv[j], acc[i][j]);
+            }
+            if (s + 1 < s_end) sstore(buf ^ 1);
+            __syncthreads();
+        }
+    }
+
+    // partial logits -> shared memory (the staging buffers are free after the last barrier)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        float *dst = part + (ty * 8 + i) * kRtSlots + tx * 8;
+        reinterpret_cast<float4 *>(dst)[0] = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+        reinterpret_cast<float4 *>(dst)[1] = make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
+    }
+    cluster.sync();
+
+    // ---- reduction over the cluster + selection: warp w owns token 8*rank + w of the tile ------
+    const int lane = tx, warp = ty;
+    const int tt = rank * 8 + warp;
+    const int64_t t = t0 + tt;
+    if (t < p.T) {
+        const int per = p.E / p.G;
+        float sc[8], sel[8];
+        int eid[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e = lane + 32 * j;
+            eid[j] = e;
+            float logit = 0.0f;
+            if (e < p.E) {
+#pragma unroll
+                for (int c = 0; c < kRtCluster; ++c) {
+                    const float *rp = cluster.map_shared_rank(part, c);
+                    logit += rp[tt * kRtSlots + e];
+                }
+            }
+            const float s = 1.0f / (1.0f + expf(-logit));
+            sc[j] = s;
+            sel[j] = (e < p.E) ? (p.bias ? s + p.bias[e] : s) : -INFINITY;
+        }
+
+        // group scores: sum of the group's top group_topn selection values, in pick order
+        uint32_t taken = 0;
+        float my_gs = -INFINITY;
+        for (int g = 0; g < p.G; ++g) {
+            float total = 0.0f;
+            for (int r = 0; r < p.group_topn; ++r) {
+                float bv = -INFINITY;
+                int bi = 0x7fffffff;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const bool cand = eid[j] < p.E && !((taken >> j) & 1u) && (eid[j] / per) == g;
+                    if (cand && (sel[j] > bv || (sel[j] == bv && eid[j] < bi))) {
+                        bv = sel[j];
+                        bi = eid[j];
+                    }
+                }
+                const ArgMax m = warp_argmax(bv, bi);
+                total = total + m.v;
+                if ((m.i & 31) == lane) taken |= 1u << (m.i >> 5);
+            }
+            if (lane == g) my_gs = total;
+        }
+        // keep the topk_groups best groups (lower group index on ties)
+        uint32_t kept = 0;
+        for (int r = 0; r < p.topk_groups; ++r) {
+            const bool cand = lane < p.G && !((kept >> lane) & 1u);
+            const ArgMax m = warp_argmax(cand ? my_gs : -INFINITY, cand ? lane : 0x7fffffff);
+            kept |= 1u << m.i;
+        }
+        // topk experts inside the kept groups, in pick order (descending selection value)
+        taken = 0;
+        float den = 0.0f, my_s = 0.0f;
+        int my_id = 0;
+        for (int r = 0; r < p.topk; ++r) {
+            float bv = -INFINITY;
+            int bi = 0x7fffffff;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const bool cand = eid[j] < p.E && !((taken >> j) & 1u) && ((kept >> (eid[j] / per)) & 1u);
+                if (cand && (sel[j] > bv || (sel[j] == bv && eid[j] < bi))) {
+                    bv = sel[j];
+                    bi = eid[j];
+                }
+            }
+            const ArgMax m = warp_argmax(bv, bi);
+            float s_owner = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (j == (m.i >> 5)) s_owner = sc[j];
+            if ((m.i & 31) == lane) taken |= 1u << (m.i >> 5);
+            const float s = __shfl_sync(0xffffffffu, s_owner, m.i & 31);
+            den = den + s;
+            if (lane == r) {
+                my_id = m.i;
+                my_s = s;
+            }
+        }
+        if (lane < p.topk) {
+            p.ids[t * p.topk + lane] = my_id;
+            p.wts[t * p.topk + lane] = my_s / den;
+        }
+    }
+    // no CTA may leave while another still reads its shared memory
+    cluster.sync();
+}
+
+}  // namespace beam

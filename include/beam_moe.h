@@ -1,0 +1,162 @@
+/*
+ * beam_moe.h - C ABI of the B200 (sm_100a) Beam Mixture-of-Experts block forward pass.
+ *
+ * The block (Beam launch post, "Welcome Beam" page, section "Mixture of Experts"; the same text in
+ * the flattened Hugging Face post on the reducer.xgoose.org digest page):
+ *   - the router scores all E experts with a sigmoid of x . W_r (computed in FP32: same page,
+ *     section "Residual Stream", which lists the router among the FP32 computations);
+ *   - experts form n_groups contiguous groups; groups are ranked by the sum of their group_topn
+ *     (2) best scores and the topk_groups (4) best groups are kept;
+ *   - the topk (8) best experts inside the kept groups run; there is no shared expert;
+ *   - expert outputs are combined with the router weights normalised to sum 1, then scaled by
+ *     routed_scale (2.5; the Chinese digest on the reducer.xgoose.org page: "scale by 2.5");
+ *   - every expert is a SwiGLU MLP, E_e(x) = W_down,e (SiLU(W_gate,e x) * (W_up,e x)), with
+ *     intermediate size 2,560 at hidden size 5,120 (sections "Mixture of Experts", "Attention").
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers on the current CUDA device, row-major, densely
+ *     packed.  bf16 tensors are passed as raw 16-bit patterns (beam_bf16).  The caller owns every
+ *     buffer, including the workspace; the library never allocates, frees or synchronises
+ *     (beam_moe_device_status is the one call that synchronises).
+ *   - Work is enqueued on `stream` (a cudaStream_t, NULL = legacy default stream) and returns
+ *     before it completes.  Return codes report argument / launch errors only; errors found by
+ *     the kernels (a bad expert id, a wait that timed out) are recorded in a per-device status
+ *     word that beam_moe_device_status returns.
+ *   - x, y, weights and the workspace must be 16-byte aligned; hidden and inter must be
+ *     multiples of 64.  T = 0 is valid and does nothing.
+ *   - Readings where the pages are silent: groups are contiguous index ranges; ties go to the
+ *     lower group / expert index; slot j of a token holds its j-th best expert (descending
+ *     selection value); an optional per-expert selection bias is added to the scores for group
+ *     and expert selection only, never to the weights.
+ *   - No C++ exception crosses this interface.  Every function is thread-safe.
+ */
+#ifndef BEAM_MOE_H
+#define BEAM_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define BEAM_MOE_API __attribute__((visibility("default")))
+#else
+#define BEAM_MOE_API
+#endif
+
+typedef uint16_t beam_bf16; /* raw bfloat16 bit pattern */
+
+/* Layer shape.  Beam: {5120, 2560, 256, 8, 4, 8, 2, 2.5f}. */
+typedef struct beam_moe_config {
+    int32_t hidden;       /* H: model width, multiple of 64, <= 65536 */
+    int32_t inter;        /* I: SwiGLU intermediate size, multiple of 64, <= 65536 */
+    int32_t n_experts;    /* E: 1..256 */
+    int32_t n_groups;     /* G: divides E, E/G <= 256 */
+    int32_t topk_groups;  /* groups kept per token, 1..G */
+    int32_t topk;         /* k: experts per token, 1..min(16, topk_groups*E/G) */
+    int32_t group_topn;   /* scores summed per group for the group ranking, 1..min(8, E/G) */
+    float routed_scale;   /* factor on the combined expert output (2.5) */
+} beam_moe_config;
+
+/* Return codes. */
+enum {
+    BEAM_MOE_OK = 0,
+    BEAM_MOE_ERR_INVALID_CONFIG = 1,     /* a config field outside the ranges above */
+    BEAM_MOE_ERR_NULL = 2,               /* a required pointer is NULL */
+    BEAM_MOE_ERR_MISALIGNED = 3,         /* a pointer is not 16-byte aligned */
+    BEAM_MOE_ERR_WORKSPACE_TOO_SMALL = 4,
+    BEAM_MOE_ERR_UNSUPPORTED_DEVICE = 5, /* the current device is not compute capability 10.0 */
+    BEAM_MOE_ERR_CUDA = 6,               /* a CUDA runtime / launch error */
+    BEAM_MOE_ERR_DEVICE_TIMEOUT = 7,     /* status word: a bounded device-side wait expired */
+    BEAM_MOE_ERR_BAD_INDEX = 8,          /* status word: an expert id outside [0, E) */
+    BEAM_MOE_ERR_INVALID_ARG = 9         /* T < 0 or T beyond the supported range */
+};
+
+/* Workspace kinds for beam_moe_workspace_size. */
+enum {
+    BEAM_MOE_WS_ROUTE = 0,
+    BEAM_MOE_WS_PERMUTE = 1,
+    BEAM_MOE_WS_EXPERTS = 2,
+    BEAM_MOE_WS_FORWARD = 3
+};
+
+/*
+ * Bytes of workspace the call `which` needs for T tokens (0 for ROUTE).  Pure host arithmetic:
+ * needs no device.  Returns 0 for an invalid config or T < 0.
+ */
+BEAM_MOE_API size_t beam_moe_workspace_size(const beam_moe_config *cfg, int64_t T, int which);
+
+/*
+ * Router: scores, group-limited selection and normalised weights for T tokens ("Mixture of
+ * Experts" section: score with a sigmoid, 8 groups, keep 4 by top-2 sum, top 8 inside).
+ *   x         [T, H]  bf16   token activations
+ *   w_router  [E, H]  fp32   router projection (logit_e = x . w_router[e], accumulated in FP32)
+ *   sel_bias  [E]     fp32   selection bias, or NULL for none
+ *   topk_ids  [T, k]  int32  out: chosen experts, slot j = j-th best selection value
+ *   topk_w    [T, k]  fp32   out: sigmoid score / sum of the chosen scores (sums to 1 per token)
+ */
+BEAM_MOE_API int beam_moe_route(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const float *w_router,
+                   const float *sel_bias, int32_t *topk_ids, float *topk_w, void *stream);
+
+/*
+ * Token -> expert dispatch: stable grouping of the T*k (token, slot) pairs by expert (the pages
+ * only say that each token runs on its 8 experts; the order is this library's convention).
+ *   topk_ids  [T, k]   int32  in: expert of each (token, slot)
+ *   counts    [E]      int32  out: pairs routed to each expert
+ *   offsets   [E + 1]  int64  out: exclusive prefix sum of counts; offsets[E] = T*k
+ *   row_src   [T * k]  int32  out: row r holds pair q = t*k + j; rows sorted by (expert, token)
+ *   dest_row  [T * k]  int32  out: inverse of row_src
+ *   ws        workspace of beam_moe_workspace_size(cfg, T, BEAM_MOE_WS_PERMUTE) bytes
+ * Ids outside [0, E) set BEAM_MOE_ERR_BAD_INDEX in the status word and leave the outputs
+ * undefined.
+ */
+BEAM_MOE_API int beam_moe_permute(const beam_moe_config *cfg, int64_t T, const int32_t *topk_ids, int32_t *counts,
+                     int64_t *offsets, int32_t *row_src, int32_t *dest_row, void *ws, size_t ws_bytes,
+                     void *stream);
+
+/*
+ * Expert half of the block for callers that route themselves:
+ *   y[t] = routed_scale * sum_{j<k} topk_w[t,j] * E_{topk_ids[t,j]}(x[t])   (sum in slot order, FP32)
+ *   x       [T, H]     bf16
+ *   topk_ids, topk_w   [T, k] int32 / fp32 (ids distinct per token)
+ *   w_gate  [E, I, H]  bf16   w_up [E, I, H] bf16   w_down [E, H, I] bf16
+ *   y       [T, H]     bf16   out (round to nearest even)
+ * The gate/up products are accumulated in FP32 on the tensor cores; SiLU(g)*u is computed in
+ * FP32 and stored as bf16 for the down projection, which accumulates in FP32.
+ */
+BEAM_MOE_API int beam_moe_experts(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const int32_t *topk_ids,
+                     const float *topk_w, const beam_bf16 *w_gate, const beam_bf16 *w_up,
+                     const beam_bf16 *w_down, beam_bf16 *y, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * The whole block: route, dispatch, gate/up + SwiGLU, down projection, weighted combine.
+ * topk_ids_out / topk_w_out ([T, k]) receive the routing when non-NULL.
+ */
+BEAM_MOE_API int beam_moe_forward(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const float *w_router,
+                     const float *sel_bias, const beam_bf16 *w_gate, const beam_bf16 *w_up,
+                     const beam_bf16 *w_down, beam_bf16 *y, int32_t *topk_ids_out, float *topk_w_out,
+                     void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Synchronises `stream`, then returns and clears the current device's status word
+ * (BEAM_MOE_OK, BEAM_MOE_ERR_DEVICE_TIMEOUT or BEAM_MOE_ERR_BAD_INDEX), or BEAM_MOE_ERR_CUDA.
+ */
+BEAM_MOE_API int beam_moe_device_status(void *stream);
+
+/*
+ * Test hook for the bounded waits: launches one block that waits on a device barrier nobody
+ * signals, giving up after about `timeout_us` microseconds (1..1000000), and records
+ * BEAM_MOE_ERR_DEVICE_TIMEOUT in the status word.  No fault, trap or hang is involved.
+ */
+BEAM_MOE_API int beam_moe_selftest_timeout(int64_t timeout_us, void *stream);
+
+/* Static description of a return code. */
+BEAM_MOE_API const char *beam_moe_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BEAM_MOE_H */

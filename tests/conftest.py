@@ -28,3 +28,11 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+@pytest.fixture(scope="session")
+def beam_weights():
+    """The shared Beam layer's expert weights (20 GB bf16), drawn once per session on cuda:0."""
+    import beam_synth as bs
+    wg, wu, wd = bs.make_experts(bs.WORKLOADS["prefill"], device="cuda")
+    return wg, wu, wd

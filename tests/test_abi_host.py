@@ -1,0 +1,100 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point the header declares,
+and rejects bad arguments on the host before any CUDA call."""
+import ctypes
+
+import pytest
+
+import group_limited_routing_router_b200 as bm
+from group_limited_routing_router_b200 import build as bm_build
+
+
+@pytest.fixture(scope="module")
+def L():
+    bm_build.build()
+    return bm.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = bm.declared_symbols()
+    assert set(names) >= {"beam_moe_route", "beam_moe_permute", "beam_moe_experts", "beam_moe_forward",
+                          "beam_moe_workspace_size", "beam_moe_device_status", "beam_moe_strerror",
+                          "beam_moe_selftest_timeout"}
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_strerror_covers_codes(L):
+    for code in range(0, 10):
+        s = bm.strerror(code)
+        assert s and s != "unknown error code"
+    assert bm.strerror(12345) == "unknown error code"
+
+
+def _cfg(**kw):
+    d = dict(hidden=5120, inter=2560, n_experts=256, n_groups=8, topk_groups=4, topk=8, group_topn=2,
+             routed_scale=2.5)
+    d.update(kw)
+    return bm.LayerConfig(**d).c()
+
+
+def test_workspace_sizes(L):
+    c = _cfg()
+    assert bm.workspace_size(c, 0, bm.WS_ROUTE) == 0
+    f = [bm.workspace_size(c, T, bm.WS_FORWARD) for T in (1, 256, 4096, 65536)]
+    assert all(b > a for a, b in zip(f, f[1:]))
+    # forward holds x_perm (bf16), h (bf16) and the fp32 expert outputs for all T*k rows
+    T = 4096
+    R = T * 8
+    assert f[2] >= R * 5120 * 2 + R * 2560 * 2 + R * 5120 * 4
+    assert bm.workspace_size(c, T, bm.WS_EXPERTS) < f[2]
+    assert bm.workspace_size(c, T, bm.WS_PERMUTE) >= 16 * 256 * 4
+    assert bm.workspace_size(c, -1, bm.WS_FORWARD) == 0
+    assert bm.workspace_size(c, 1 << 25, bm.WS_FORWARD) == 0
+    assert bm.workspace_size(c, 4, 99) == 0
+    assert bm.workspace_size(_cfg(hidden=100), 4, bm.WS_FORWARD) == 0
+
+
+@pytest.mark.parametrize("bad", [dict(hidden=96), dict(inter=0), dict(n_experts=257), dict(n_groups=3),
+                                 dict(topk_groups=9), dict(topk=17), dict(topk=0), dict(group_topn=0),
+                                 dict(group_topn=9), dict(n_groups=64, n_experts=256),
+                                 dict(routed_scale=float("nan"))])
+def test_invalid_config_rejected_on_host(L, bad):
+    c = _cfg(**bad)
+    p = ctypes.c_void_p(4096)  # never dereferenced: validation fails first
+    assert L.beam_moe_route(ctypes.byref(c), 4, p, p, None, p, p, None) == bm.ERR_INVALID_CONFIG
+    assert L.beam_moe_forward(ctypes.byref(c), 4, p, p, None, p, p, p, p, None, None, p, 1 << 40, None) == \
+        bm.ERR_INVALID_CONFIG
+    assert L.beam_moe_experts(ctypes.byref(c), 4, p, p, p, p, p, p, p, p, 1 << 40, None) == bm.ERR_INVALID_CONFIG
+
+
+def test_argument_errors_on_host(L):
+    c = _cfg()
+    p = ctypes.c_void_p(4096)
+    mis = ctypes.c_void_p(4104)
+    assert L.beam_moe_route(None, 4, p, p, None, p, p, None) == bm.ERR_NULL
+    assert L.beam_moe_route(ctypes.byref(c), 4, None, p, None, p, p, None) == bm.ERR_NULL
+    assert L.beam_moe_route(ctypes.byref(c), 4, mis, p, None, p, p, None) == bm.ERR_MISALIGNED
+    assert L.beam_moe_route(ctypes.byref(c), -1, p, p, None, p, p, None) == bm.ERR_INVALID_ARG
+    assert L.beam_moe_route(ctypes.byref(c), 0, p, p, None, p, p, None) == bm.OK  # T = 0: nothing to do
+    need = bm.workspace_size(c, 64, bm.WS_FORWARD)
+    assert L.beam_moe_forward(ctypes.byref(c), 64, p, p, None, p, p, p, p, None, None, p, need - 1, None) == \
+        bm.ERR_WORKSPACE_TOO_SMALL
+    assert L.beam_moe_forward(ctypes.byref(c), 64, p, p, None, p, p, mis, p, None, None, p, need, None) == \
+        bm.ERR_MISALIGNED
+    assert L.beam_moe_forward(ctypes.byref(c), 64, p, p, None, p, p, p, p, None, None, None, need, None) == \
+        bm.ERR_NULL
+    assert L.beam_moe_forward(ctypes.byref(c), 0, p, p, None, p, p, p, p, None, None, None, 0, None) == bm.OK
+    need_e = bm.workspace_size(c, 64, bm.WS_EXPERTS)
+    assert L.beam_moe_experts(ctypes.byref(c), 64, p, p, p, p, p, p, p, p, need_e - 256, None) == \
+        bm.ERR_WORKSPACE_TOO_SMALL
+    need_p = bm.workspace_size(c, 64, bm.WS_PERMUTE)
+    assert L.beam_moe_permute(ctypes.byref(c), 64, p, p, p, p, p, p, need_p - 1, None) == \
+        bm.ERR_WORKSPACE_TOO_SMALL
+    assert L.beam_moe_selftest_timeout(0, None) == bm.ERR_INVALID_ARG
+
+
+def test_binding_refuses_cpu_tensors(L):
+    import torch
+    x = torch.zeros(4, 5120, dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        bm.route(bm.BEAM_LAYER, x, torch.zeros(256, 5120))
