@@ -1,0 +1,373 @@
+#!/usr/bin/env python
+"""Benchmark of the Beam MoE block forward pass (group-limited routing + 8 SwiGLU experts) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload prefill] [--impl ours|reference]
+
+One step = one beam_moe_forward call over one batch (router, dispatch, gather, gate/up + SwiGLU
+GEMM, down GEMM, combine) with inputs and the 20.1 GB of expert weights already resident in HBM.
+The default workload is the T=4096 prefill chunk at Beam shapes.  Under torchrun each rank runs an
+independent replica (the path has no exchange step on one layer); value = tokens of all ranks /
+max-over-ranks device time.  Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (plain FP64 C, the test oracle) on a bounded token sample of the
+same workload on this host's cores; under torchrun only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import beam_synth as bs  # noqa: E402
+
+METRIC = "MoE-layer tokens/s (Beam shape, BF16, T=4096) and % of tensor/HBM roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture, keyed by
+# kernel; valid only while the kernel source hashes the same as at capture time.
+NCU_TRAFFIC = {}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="prefill", choices=["decode", "prefill", "skew", "long"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-sample", type=int, default=96, help="tokens in the CPU-oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "group_limited_routing_router_b200", "csrc")
+    for n in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+# ------------------------------------------------------------------------------------------------
+# algorithmic work (bytes the method must move, flops it must do), per step
+def algorithmic(wl: bs.Workload, n_act: int) -> dict:
+    T, H, I, E, k = wl.T, wl.hidden, wl.inter, wl.n_experts, wl.topk
+    R = T * k
+    w_expert = 3 * H * I * 2
+    return dict(
+        layer_flops=T * (2 * H * E + k * 6 * H * I),
+        layer_bytes=n_act * w_expert + E * H * 4 + 2 * T * H * 2 + T * k * 8,
+        stage_bytes={
+            "router": T * H * 2 + E * H * 4 + T * k * 8,
+            "dispatch": T * k * 4 + 2 * R * 4,
+            "gather": T * H * 2 + R * H * 2,
+            "gate_up_swiglu": n_act * 2 * I * H * 2 + R * H * 2 + R * I * 2,
+            "down": n_act * H * I * 2 + R * I * 2 + R * H * 4,
+            "combine": R * H * 4 + T * k * 8 + T * H * 2,
+        },
+        stage_flops={"router": 2 * T * H * E, "gate_up_swiglu": 4 * R * H * I, "down": 2 * R * H * I},
+    )
+
+
+# ------------------------------------------------------------------------------------------------
+class ClockSampler:
+    """nvidia-smi clock / throttle samples every 200 ms while the GPU works."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, local_rank: int):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        self.gpu = vis.split(",")[local_rank] if vis else str(local_rank)
+        self.file = tempfile.NamedTemporaryFile(mode="w+", suffix=".csv", delete=False)
+        self.proc = None
+        self.marks = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                                          "-i", self.gpu, "-lms", "200"], stdout=self.file,
+                                         stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.5)
+
+    def n_samples(self) -> int:
+        self.file.flush()
+        with open(self.file.name) as f:
+            return sum(1 for ln in f if ln.strip())
+
+    def mark(self):
+        self.marks.append(self.n_samples())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        self.proc.wait()
+        with open(self.file.name) as f:
+            rows = [ln.strip().split(", ") for ln in f if ln.strip()]
+        os.unlink(self.file.name)
+        lo, hi = (self.marks[0], self.marks[-1]) if len(self.marks) >= 2 else (0, len(rows))
+        sel = rows[lo:hi] if hi > lo else rows
+        sm = [float(r[1]) for r in sel if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in sel if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in sel for i in range(4) if len(r) > 5 + i and r[5 + i] == "Active"})
+        power = [float(r[3]) for r in sel if r[3].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(sel), "power_w_max": max(power) if power else None}
+
+
+# ------------------------------------------------------------------------------------------------
+def cpu_oracle_rate(wl, x_cpu, W, bias, wg, wu, wd, n_sample: int, route_all: bool = True) -> dict:
+    """Time the CPU oracle: routing (FP64 scores + selection) and the expert half on a token sample.
+    Expert weights are copied to the host expert by expert, outside the timed sections."""
+    import oracle
+    xb = oracle.bf16_bits(x_cpu)
+    b = None if bias is None else bias.cpu().numpy()
+    Wn = W.cpu().numpy()
+    T = wl.T
+    tok = bs.sample_tokens(wl, n_sample)
+    t0 = time.perf_counter()
+    if route_all:
+        r = oracle.route(xb, Wn, wl.layer, b)
+        ids, wts = r["ids"][tok], r["weight"][tok]
+        t_route_tok = (time.perf_counter() - t0) / T
+    else:
+        r = oracle.route(np.ascontiguousarray(xb[tok]), Wn, wl.layer, b)
+        ids, wts = r["ids"], r["weight"]
+        t_route_tok = (time.perf_counter() - t0) / len(tok)
+    xs = np.ascontiguousarray(xb[tok])
+    out = np.zeros((len(tok), wl.topk, wl.hidden))
+    t_exp = 0.0
+    for e in range(wl.n_experts):
+        rows, slots = np.nonzero(ids == e)
+        if rows.size == 0:
+            continue
+        w3 = (oracle.bf16_bits(wg[e]), oracle.bf16_bits(wu[e]), oracle.bf16_bits(wd[e]))
+        t1 = time.perf_counter()
+        out[rows, slots, :] = oracle.expert_mlp(xs[rows], *w3)
+        t_exp += time.perf_counter() - t1
+    t1 = time.perf_counter()
+    oracle.combine(out, wts, wl.routed_scale)
+    t_exp += time.perf_counter() - t1
+    secs = t_route_tok * len(tok) + t_exp
+    return {"value": len(tok) / secs, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "seconds": secs,
+            "sample": (f"router + group-limited selection on {'all ' + str(T) if route_all else len(tok)} tokens, "
+                       f"SwiGLU experts + combine on {len(tok)} seeded tokens of the {wl.name} batch; "
+                       "tokens/s = sample / (per-token routing time x sample + expert time)")}
+
+
+# ------------------------------------------------------------------------------------------------
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = bs.get(args.workload)
+    torch.cuda.set_device(0)
+    x = bs.make_x(wl)
+    W = bs.make_router(wl)
+    bias = bs.load_bias(wl)
+    wg, wu, wd = bs.make_experts(wl, device="cuda")
+    n = 16
+    rates, secs = [], []
+    for i in range(args.warmup + args.steps):
+        r = cpu_oracle_rate(wl, x, W, bias, wg, wu, wd, n, route_all=False)
+        if i >= args.warmup:
+            rates.append(r)
+            secs.append(r["seconds"])
+    tot = sum(secs)
+    value = n * args.steps / tot
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_dict(wl),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": rates[0]["cores"], "kind": "oracle",
+                             "sample": f"each step: the whole block (routing + experts + combine) for {n} seeded "
+                                       f"tokens of the {wl.name} batch, FP64 CPU oracle"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+def config_dict(wl):
+    return {"workload": f"{wl.name}: {wl.description}", "T": wl.T, "hidden": wl.hidden, "inter": wl.inter,
+            "n_experts": wl.n_experts, "n_groups": wl.n_groups, "topk_groups": wl.topk_groups, "topk": wl.topk,
+            "routed_scale": wl.routed_scale, "weights_bytes": 3 * wl.n_experts * wl.hidden * wl.inter * 2,
+            "l2": "no flush: every step streams the 20.1 GB of expert weights (> 126 MB L2)",
+            "parallelism": "replicas (one independent layer instance per GPU)"}
+
+
+def run_ours(args):
+    import group_limited_routing_router_b200 as bm
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(v: float) -> float:
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    wl = bs.get(args.workload)
+    layer = wl.layer
+    T, H = wl.T, wl.hidden
+    x_cpu = bs.make_x(wl)
+    W_cpu = bs.make_router(wl)
+    b_cpu = bs.load_bias(wl)
+    x = x_cpu.cuda()
+    W = W_cpu.cuda()
+    bias = None if b_cpu is None else b_cpu.cuda()
+    wg, wu, wd = bs.make_experts(wl, device="cuda")
+    ws = torch.empty(bm.workspace_size(layer, T, bm.WS_FORWARD), dtype=torch.uint8, device="cuda")
+    y = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    ids = torch.empty(T, wl.topk, dtype=torch.int32, device="cuda")
+    w = torch.empty(T, wl.topk, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        bm.forward(layer, x, W, bias, wg, wu, wd, y=y, ids=ids, w=w, ws=ws)
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    for _ in range(args.warmup):
+        step()
+    assert bm.device_status() == bm.OK
+    barrier()
+    clocks.mark()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    barrier()
+    clocks.mark()
+    # keep the GPU busy (untimed) until the sampler has seen at least 3 samples under load
+    t_extra = time.time()
+    while clocks.marks[-1] - clocks.marks[0] < 3 and time.time() - t_extra < 2.0:
+        for _ in range(10):
+            step()
+        torch.cuda.synchronize()
+        clocks.marks[-1] = clocks.n_samples()
+    clk = clocks.stop()
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1))
+    ms_step = ms_total / args.steps
+    value = world * T * args.steps / (ms_total / 1e3)
+    n_act = int((torch.bincount(ids.flatten().long(), minlength=wl.n_experts) > 0).sum().item())
+
+    # per-stage device time from events recorded between the launches (same stream)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        bm.forward_profiled(layer, x, W, bias, wg, wu, wd, evs[i], y, ids, w, ws)
+    torch.cuda.synchronize()
+    stage_ms = {name: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
+                for j, name in enumerate(bm.STAGES)}
+
+    # end to end through the public API with host buffers: H2D x, forward, D2H y every step
+    x_host = x_cpu.pin_memory()
+    y_host = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
+    for _ in range(2):
+        x.copy_(x_host, non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        x.copy_(x_host, non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+    e1.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_value = world * T * args.steps / (e2e_ms / 1e3)
+    assert bm.device_status() == bm.OK
+
+    alg = algorithmic(wl, n_act)
+    pk, pk_kind = peaks()
+    dom = max(stage_ms, key=stage_ms.get)
+    dom_bytes = alg["stage_bytes"][dom]
+    achieved = dom_bytes / (stage_ms[dom] / 1e3) / 1e9
+    src_hash = kernel_source_hash()
+    tr = NCU_TRAFFIC.get((dom, wl.name))
+    traffic = tr["bytes"] if tr and tr.get("source_hash") == src_hash else None
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / pk["hbm_gbs"], "traffic": traffic, "peak_kind": pk_kind,
+                "algorithmic_bytes_per_launch": dom_bytes, "launch_ms": stage_ms[dom]}
+    t_tensor = alg["layer_flops"] / (pk["bf16_tflops"] * 1e12)
+    t_hbm = alg["layer_bytes"] / (pk["hbm_gbs"] * 1e9)
+    t_roof = max(t_tensor, t_hbm)
+    layer_roof = {"bound": "hbm" if t_hbm >= t_tensor else "tensor", "roofline_ms": t_roof * 1e3,
+                  "roofline_tokens_s": T / t_roof, "frac": t_roof / (ms_step / 1e3),
+                  "tensor_ms": t_tensor * 1e3, "hbm_ms": t_hbm * 1e3, "active_experts": n_act,
+                  "achieved_tflops": alg["layer_flops"] / (ms_step / 1e3) / 1e12,
+                  "achieved_gbs": alg["layer_bytes"] / (ms_step / 1e3) / 1e9}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_rate(wl, x_cpu, W_cpu, b_cpu, wg, wu, wd, args.cpu_sample)
+        cpu.pop("seconds", None)
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(wl),
+            "roofline": roofline, "layer_roofline": layer_roof, "stage_ms": stage_ms, "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2,
+                    "d2h_bytes_per_step": T * H * 2},
+            "clocks": clk, "gpu_launches": 8 * args.steps, "kernel_source": src_hash}
+    if rank == 0:
+        print(json.dumps(line))
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

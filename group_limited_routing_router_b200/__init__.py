@@ -89,12 +89,14 @@ def lib() -> ctypes.CDLL:
                                        ctypes.c_size_t, _vp]
         L.beam_moe_forward.argtypes = [_cfgp, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                        ctypes.c_size_t, _vp]
+        L.beam_moe_forward_profiled.argtypes = [_cfgp, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                                _vp, ctypes.c_size_t, _vp, ctypes.POINTER(ctypes.c_void_p)]
         L.beam_moe_device_status.argtypes = [_vp]
         L.beam_moe_selftest_timeout.argtypes = [ctypes.c_int64, _vp]
         L.beam_moe_strerror.argtypes = [ctypes.c_int]
         L.beam_moe_strerror.restype = ctypes.c_char_p
         for name in ("beam_moe_route", "beam_moe_permute", "beam_moe_experts", "beam_moe_forward",
-                     "beam_moe_device_status", "beam_moe_selftest_timeout"):
+                     "beam_moe_forward_profiled", "beam_moe_device_status", "beam_moe_selftest_timeout"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -235,6 +237,27 @@ def forward(cfg, x, w_router, bias, w_gate, w_up, w_down, y=None, ids=None, w=No
                                   _ptr(w_up), _ptr(w_down), _ptr(y), _ptr(ids), _ptr(w), _ptr(ws), nbytes,
                                   _stream(stream)), "beam_moe_forward")
     return (y, ids, w) if return_routing else y
+
+
+STAGES = ("router", "dispatch", "gather", "gate_up_swiglu", "down", "combine")
+
+
+def forward_profiled(cfg, x, w_router, bias, w_gate, w_up, w_down, events, y, ids, w, ws, stream=None):
+    """forward() that records the 7 torch.cuda.Event objects in `events` around its stages (see
+    beam_moe_forward_profiled); all buffers are caller-provided so nothing is allocated per call."""
+    c = _cfg(cfg)
+    T = x.shape[0]
+    if len(events) != 7:
+        raise ValueError("need 7 events")
+    handles = (ctypes.c_void_p * 7)()
+    for i, e in enumerate(events):
+        if e.cuda_event == 0:  # torch creates the CUDA event at its first record
+            e.record()
+        handles[i] = e.cuda_event
+    _check(lib().beam_moe_forward_profiled(ctypes.byref(c), T, _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w_gate),
+                                           _ptr(w_up), _ptr(w_down), _ptr(y), _ptr(ids), _ptr(w), _ptr(ws),
+                                           ws.numel(), _stream(stream), handles), "beam_moe_forward_profiled")
+    return y
 
 
 def device_status(stream=None) -> int:

@@ -213,9 +213,14 @@ int enqueue_permute(const beam_moe_config *c, int64_t T, const int32_t *ids, int
     return launch_status();
 }
 
+// Records events[i] on s when profiling (events may be null).
+bool record(cudaEvent_t const *events, int i, cudaStream_t s) {
+    return !events || cudaEventRecord(events[i], s) == cudaSuccess;
+}
+
 int enqueue_experts(const beam_moe_config *c, int dev, int64_t T, const beam_bf16 *x, const int32_t *ids,
                     const float *w, const beam_bf16 *wg, const beam_bf16 *wu, const beam_bf16 *wd, beam_bf16 *y,
-                    uint8_t *ws, const Layout &L, cudaStream_t s) {
+                    uint8_t *ws, const Layout &L, cudaStream_t s, cudaEvent_t const *ev = nullptr) {
     int32_t *counts = reinterpret_cast<int32_t *>(ws + L.counts);
     int64_t *offsets = reinterpret_cast<int64_t *>(ws + L.offsets);
     int32_t *row_src = reinterpret_cast<int32_t *>(ws + L.row_src);
@@ -229,9 +234,11 @@ int enqueue_experts(const beam_moe_config *c, int dev, int64_t T, const beam_bf1
 
     int rc = enqueue_permute(c, T, ids, counts, offsets, row_src, dest_row, hist, s);
     if (rc) return rc;
+    if (!record(ev, 2, s)) return BEAM_MOE_ERR_CUDA;
     gather_rows_kernel<<<static_cast<unsigned>(T), 128, 0, s>>>(reinterpret_cast<const uint4 *>(x), T, k, H / 8,
                                                                 dest_row, reinterpret_cast<uint4 *>(xp));
     if ((rc = launch_status())) return rc;
+    if (!record(ev, 3, s)) return BEAM_MOE_ERR_CUDA;
 
     const bool narrow = static_cast<double>(R) / E <= 24.0;
     const int bn = narrow ? 32 : 128;
@@ -243,17 +250,19 @@ int enqueue_experts(const beam_moe_config *c, int dev, int64_t T, const beam_bf1
     const int grid = g_dev[dev].num_sms;
     GemmParams p1{counts, offsets, h, E, H, I, kDefaultTimeoutCycles};
     GemmParams p2{counts, offsets, o, E, I, H, kDefaultTimeoutCycles};
-    if (narrow) {
-        G1_NARROW_KERNEL<<<grid, kGemmThreads, G1Narrow::kSmem, s>>>(m_wg, m_wu, m_xp, p1);
-        G2_NARROW_KERNEL<<<grid, kGemmThreads, G2Narrow::kSmem, s>>>(m_wd, m_wd, m_h, p2);
-    } else {
-        G1_WIDE_KERNEL<<<grid, kGemmThreads, G1Wide::kSmem, s>>>(m_wg, m_wu, m_xp, p1);
-        G2_WIDE_KERNEL<<<grid, kGemmThreads, G2Wide::kSmem, s>>>(m_wd, m_wd, m_h, p2);
-    }
+    if (narrow) G1_NARROW_KERNEL<<<grid, kGemmThreads, G1Narrow::kSmem, s>>>(m_wg, m_wu, m_xp, p1);
+    else G1_WIDE_KERNEL<<<grid, kGemmThreads, G1Wide::kSmem, s>>>(m_wg, m_wu, m_xp, p1);
     if ((rc = launch_status())) return rc;
+    if (!record(ev, 4, s)) return BEAM_MOE_ERR_CUDA;
+    if (narrow) G2_NARROW_KERNEL<<<grid, kGemmThreads, G2Narrow::kSmem, s>>>(m_wd, m_wd, m_h, p2);
+    else G2_WIDE_KERNEL<<<grid, kGemmThreads, G2Wide::kSmem, s>>>(m_wd, m_wd, m_h, p2);
+    if ((rc = launch_status())) return rc;
+    if (!record(ev, 5, s)) return BEAM_MOE_ERR_CUDA;
     combine_kernel<<<static_cast<unsigned>(T), 256, 0, s>>>(reinterpret_cast<const float4 *>(o), dest_row, w, T, k,
                                                             H / 4, c->routed_scale, reinterpret_cast<uint2 *>(y));
-    return launch_status();
+    if ((rc = launch_status())) return rc;
+    if (!record(ev, 6, s)) return BEAM_MOE_ERR_CUDA;
+    return BEAM_MOE_OK;
 }
 
 __global__ void selftest_timeout_kernel(long long cycles) {
@@ -334,9 +343,14 @@ int beam_moe_experts(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, 
                            static_cast<cudaStream_t>(stream));
 }
 
-int beam_moe_forward(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const float *w_router,
-                     const float *sel_bias, const beam_bf16 *w_gate, const beam_bf16 *w_up, const beam_bf16 *w_down,
-                     beam_bf16 *y, int32_t *topk_ids_out, float *topk_w_out, void *ws, size_t ws_bytes, void *stream) {
+}  // extern "C"
+
+namespace beam {
+namespace {
+int forward_impl(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const float *w_router,
+                 const float *sel_bias, const beam_bf16 *w_gate, const beam_bf16 *w_up, const beam_bf16 *w_down,
+                 beam_bf16 *y, int32_t *topk_ids_out, float *topk_w_out, void *ws, size_t ws_bytes, void *stream,
+                 cudaEvent_t const *ev) {
     int rc = validate(cfg);
     if (rc) return rc;
     if ((rc = check_T(cfg, T))) return rc;
@@ -353,8 +367,32 @@ int beam_moe_forward(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, 
     uint8_t *wsb = static_cast<uint8_t *>(ws);
     int32_t *ids = topk_ids_out ? topk_ids_out : reinterpret_cast<int32_t *>(wsb + L.ids);
     float *w = topk_w_out ? topk_w_out : reinterpret_cast<float *>(wsb + L.w);
+    if (!record(ev, 0, s)) return BEAM_MOE_ERR_CUDA;
     if ((rc = enqueue_route(cfg, T, x, w_router, sel_bias, ids, w, s))) return rc;
-    return enqueue_experts(cfg, dev, T, x, ids, w, w_gate, w_up, w_down, y, wsb, L, s);
+    if (!record(ev, 1, s)) return BEAM_MOE_ERR_CUDA;
+    return enqueue_experts(cfg, dev, T, x, ids, w, w_gate, w_up, w_down, y, wsb, L, s, ev);
+}
+}  // namespace
+}  // namespace beam
+
+extern "C" {
+
+int beam_moe_forward(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const float *w_router,
+                     const float *sel_bias, const beam_bf16 *w_gate, const beam_bf16 *w_up, const beam_bf16 *w_down,
+                     beam_bf16 *y, int32_t *topk_ids_out, float *topk_w_out, void *ws, size_t ws_bytes, void *stream) {
+    return forward_impl(cfg, T, x, w_router, sel_bias, w_gate, w_up, w_down, y, topk_ids_out, topk_w_out, ws,
+                        ws_bytes, stream, nullptr);
+}
+
+int beam_moe_forward_profiled(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const float *w_router,
+                              const float *sel_bias, const beam_bf16 *w_gate, const beam_bf16 *w_up,
+                              const beam_bf16 *w_down, beam_bf16 *y, int32_t *topk_ids_out, float *topk_w_out,
+                              void *ws, size_t ws_bytes, void *stream, void *const *events) {
+    if (!events) return BEAM_MOE_ERR_NULL;
+    for (int i = 0; i < 7; ++i)
+        if (!events[i]) return BEAM_MOE_ERR_NULL;
+    return forward_impl(cfg, T, x, w_router, sel_bias, w_gate, w_up, w_down, y, topk_ids_out, topk_w_out, ws,
+                        ws_bytes, stream, reinterpret_cast<cudaEvent_t const *>(events));
 }
 
 int beam_moe_device_status(void *stream) {

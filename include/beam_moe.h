@@ -140,6 +140,21 @@ BEAM_MOE_API int beam_moe_forward(const beam_moe_config *cfg, int64_t T, const b
                      void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * beam_moe_forward that also records caller-created CUDA events (cudaEvent_t) on `stream` around
+ * its launches, for per-kernel timing:
+ *   events[0] before the router            events[4] after the gate/up + SwiGLU GEMM
+ *   events[1] after the router             events[5] after the down GEMM
+ *   events[2] after the dispatch kernels   events[6] after the combine
+ *   events[3] after the row gather
+ * Same results and launches as beam_moe_forward; `events` must hold 7 valid events.
+ */
+BEAM_MOE_API int beam_moe_forward_profiled(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x,
+                                           const float *w_router, const float *sel_bias, const beam_bf16 *w_gate,
+                                           const beam_bf16 *w_up, const beam_bf16 *w_down, beam_bf16 *y,
+                                           int32_t *topk_ids_out, float *topk_w_out, void *ws, size_t ws_bytes,
+                                           void *stream, void *const *events);
+
+/*
  * Synchronises `stream`, then returns and clears the current device's status word
  * (BEAM_MOE_OK, BEAM_MOE_ERR_DEVICE_TIMEOUT or BEAM_MOE_ERR_BAD_INDEX), or BEAM_MOE_ERR_CUDA.
  */
