@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <cmath>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -26,16 +27,21 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr int64_t kMaxTokens = int64_t(1) << 24;
 
-// ---- GEMM variants: (BN, smem stages, accumulator stages) -----------------------------------
-// "wide": experts see ~BN tokens (prefill); "narrow": a few tokens per expert (decode).
-using G1Wide = GemmCfg<true, 128, 4, 2>;
-using G2Wide = GemmCfg<false, 128, 6, 4>;
-using G1Narrow = GemmCfg<true, 32, 5, 2>;
-using G2Narrow = GemmCfg<false, 32, 8, 4>;
-#define G1_WIDE_KERNEL grouped_gemm_kernel<true, 128, 4, 2>
-#define G2_WIDE_KERNEL grouped_gemm_kernel<false, 128, 6, 4>
-#define G1_NARROW_KERNEL grouped_gemm_kernel<true, 32, 5, 2>
-#define G2_NARROW_KERNEL grouped_gemm_kernel<false, 32, 8, 4>
+// ---- GEMM variants: <gate/up?, BN, B box rows, smem stages, TMEM slots, slot columns> ----------
+// "wide": experts see up to ~190 tokens per tile (prefill); "narrow": a few tokens (decode).
+#define G1_WIDE_ARGS true, 192, 64, 4, 2, 256
+#define G2_WIDE_ARGS false, 192, 64, 5, 2, 256
+#define G1_NARROW_ARGS true, 32, 32, 6, 4, 64
+#define G2_NARROW_ARGS false, 32, 32, 10, 4, 32
+using G1Wide = GemmCfg<G1_WIDE_ARGS>;
+using G2Wide = GemmCfg<G2_WIDE_ARGS>;
+using G1Narrow = GemmCfg<G1_NARROW_ARGS>;
+using G2Narrow = GemmCfg<G2_NARROW_ARGS>;
+#define G1_WIDE_KERNEL grouped_gemm_kernel<G1_WIDE_ARGS>
+#define G2_WIDE_KERNEL grouped_gemm_kernel<G2_WIDE_ARGS>
+#define G1_NARROW_KERNEL grouped_gemm_kernel<G1_NARROW_ARGS>
+#define G2_NARROW_KERNEL grouped_gemm_kernel<G2_NARROW_ARGS>
+constexpr int kWideBN = 192, kWideBox = 64, kNarrowBN = 32, kNarrowBox = 32;
 
 struct DeviceInfo {
     std::once_flag once;
@@ -240,16 +246,22 @@ int enqueue_experts(const beam_moe_config *c, int dev, int64_t T, const beam_bf1
     if ((rc = launch_status())) return rc;
     if (!record(ev, 3, s)) return BEAM_MOE_ERR_CUDA;
 
-    const bool narrow = static_cast<double>(R) / E <= 24.0;
-    const int bn = narrow ? 32 : 128;
+    // Tile choice from the mean rows per expert: narrow tiles when experts see a handful of tokens.
+    const double mean_rows = static_cast<double>(R) / E;
+    const bool narrow = mean_rows <= 12.0;
+    const int bn = narrow ? kNarrowBN : kWideBN;
+    const int box = narrow ? kNarrowBox : kWideBox;
+    // Weights are read once per call when (almost) every expert fits one token tile: mark them
+    // evict-first so they do not push the reused activations out of L2.
+    const int weights_once = (mean_rows + 5.0 * std::sqrt(mean_rows) <= bn) ? 1 : 0;
     CUtensorMap m_wg, m_wu, m_xp, m_wd, m_h;
     if (!encode_fn()) return BEAM_MOE_ERR_CUDA;
-    if (!make_map_3d(&m_wg, wg, H, I, E) || !make_map_3d(&m_wu, wu, H, I, E) || !make_map_2d(&m_xp, xp, H, R, bn) ||
-        !make_map_3d(&m_wd, wd, I, H, E) || !make_map_2d(&m_h, h, I, R, bn))
+    if (!make_map_3d(&m_wg, wg, H, I, E) || !make_map_3d(&m_wu, wu, H, I, E) ||
+        !make_map_2d(&m_xp, xp, H, R, box) || !make_map_3d(&m_wd, wd, I, H, E) || !make_map_2d(&m_h, h, I, R, box))
         return BEAM_MOE_ERR_CUDA;
     const int grid = g_dev[dev].num_sms;
-    GemmParams p1{counts, offsets, h, E, H, I, kDefaultTimeoutCycles};
-    GemmParams p2{counts, offsets, o, E, I, H, kDefaultTimeoutCycles};
+    GemmParams p1{counts, offsets, h, E, H, I, weights_once, kDefaultTimeoutCycles};
+    GemmParams p2{counts, offsets, o, E, I, H, weights_once, kDefaultTimeoutCycles};
     if (narrow) G1_NARROW_KERNEL<<<grid, kGemmThreads, G1Narrow::kSmem, s>>>(m_wg, m_wu, m_xp, p1);
     else G1_WIDE_KERNEL<<<grid, kGemmThreads, G1Wide::kSmem, s>>>(m_wg, m_wu, m_xp, p1);
     if ((rc = launch_status())) return rc;
@@ -292,9 +304,9 @@ int beam_moe_route(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, co
     int rc = validate(cfg);
     if (rc) return rc;
     if ((rc = check_T(cfg, T))) return rc;
+    if (T == 0) return BEAM_MOE_OK;
     if (!x || !w_router || !topk_ids || !topk_w) return BEAM_MOE_ERR_NULL;
     if (!aligned16(x) || !aligned16(w_router)) return BEAM_MOE_ERR_MISALIGNED;
-    if (T == 0) return BEAM_MOE_OK;
     int dev;
     if ((rc = init_device(&dev))) return rc;
     return enqueue_route(cfg, T, x, w_router, sel_bias, topk_ids, topk_w, static_cast<cudaStream_t>(stream));
@@ -330,7 +342,8 @@ int beam_moe_experts(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, 
     int rc = validate(cfg);
     if (rc) return rc;
     if ((rc = check_T(cfg, T))) return rc;
-    if (!x || !topk_ids || !topk_w || !w_gate || !w_up || !w_down || !y || (T > 0 && !ws)) return BEAM_MOE_ERR_NULL;
+    if (T == 0) return BEAM_MOE_OK;
+    if (!x || !topk_ids || !topk_w || !w_gate || !w_up || !w_down || !y || !ws) return BEAM_MOE_ERR_NULL;
     if (!aligned16(x) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) || !aligned16(y) ||
         (ws && !aligned16(ws)))
         return BEAM_MOE_ERR_MISALIGNED;
@@ -354,7 +367,8 @@ int forward_impl(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, cons
     int rc = validate(cfg);
     if (rc) return rc;
     if ((rc = check_T(cfg, T))) return rc;
-    if (!x || !w_router || !w_gate || !w_up || !w_down || !y || (T > 0 && !ws)) return BEAM_MOE_ERR_NULL;
+    if (T == 0) return BEAM_MOE_OK;
+    if (!x || !w_router || !w_gate || !w_up || !w_down || !y || !ws) return BEAM_MOE_ERR_NULL;
     if (!aligned16(x) || !aligned16(w_router) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) ||
         !aligned16(y) || (ws && !aligned16(ws)))
         return BEAM_MOE_ERR_MISALIGNED;

@@ -8,8 +8,8 @@
 //
 // Orientation (swap-AB): the MMA's M side (128) walks the expert's weight rows, its N side the
 // expert's tokens (N = tokens rounded up to 16, at most BN).  At the Beam shapes an expert sees
-// ~8 tokens in a decode batch and ~128 in a 4096-token prefill, so putting tokens on N lets one
-// tile cover all of an expert's tokens and every weight byte crosses HBM once per call.
+// ~8 tokens in a decode batch and 128 +- 11 in a 4096-token prefill, so one token tile covers all of
+// an expert's tokens and every weight byte crosses HBM once per call.
 //
 // Work item = (expert e, weight-row tile mt of 128, token tile nt of BN).  Items are numbered
 // expert-major, then mt, then nt, from the per-expert counts (read on the device; no host sync);
@@ -17,8 +17,13 @@
 //
 // Warp roles (256 threads): warp 0 lane 0 = TMA producer; warp 1 = TMEM owner, lane 0 issues
 // tcgen05.mma; warps 4..7 = epilogue (warp 4+q reads TMEM lanes 32q..32q+31).  Shared memory is a
-// STAGES-deep ring of {A tile(s) 128x64 bf16, B tile BNx64 bf16}, 128-byte swizzled by TMA; TMEM
-// holds ACC double-buffered accumulators so the epilogue of one item overlaps the next item's MMAs.
+// STAGES-deep ring of {A tile(s) 128x64 bf16, B tile of up to BN x 64 bf16}, 128-byte swizzled by
+// TMA; the B tile is loaded in boxes of BOXN rows, only as many as the item's tokens need.
+//
+// TMEM holds NSLOT accumulator slots of SLOT_COLS fp32 columns, used round-robin.  G2 and small G1
+// items take one slot (G1: gate in its first half, up in its second half); a G1 item with more
+// than SLOT_COLS/2 tokens takes two consecutive slots (gate in one, up in the other), so large
+// experts stay in one token tile while small ones keep the epilogue overlapped with the next MMAs.
 // Every wait is bounded (status word BEAM_MOE_ERR_DEVICE_TIMEOUT on expiry).
 #pragma once
 
@@ -32,19 +37,22 @@ constexpr int kGemmThreads = 256;
 
 constexpr int pow2_cols(int c) { return c <= 32 ? 32 : c <= 64 ? 64 : c <= 128 ? 128 : c <= 256 ? 256 : 512; }
 
-template <bool GATE_UP, int BN, int STAGES, int ACC>
+template <bool GATE_UP, int BN, int BOXN, int STAGES, int NSLOT, int SLOT_COLS>
 struct GemmCfg {
     static constexpr int kA = kBM * kBK * 2;                 // one A tile, bytes
-    static constexpr int kB = BN * kBK * 2;                  // B tile, bytes
+    static constexpr int kB = BN * kBK * 2;                  // B tile, bytes (room for BN rows)
+    static constexpr int kBox = BOXN * kBK * 2;              // one B box, bytes
     static constexpr int kNumA = GATE_UP ? 2 : 1;
-    static constexpr int kStage = kNumA * kA + kB;           // multiple of 1024
-    static constexpr int kAccCols = (GATE_UP ? 2 : 1) * BN;  // TMEM columns per accumulator stage
-    static constexpr int kTmemCols = pow2_cols(ACC * kAccCols);
+    static constexpr int kStage = kNumA * kA + kB;
+    static constexpr int kTmemCols = pow2_cols(NSLOT * SLOT_COLS);
     static constexpr int kBarOff = STAGES * kStage;
     static constexpr int kSmem = 1024 + kBarOff + 256 + 4 * (kPmMaxE + 1) + 64;
-    static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
-    static_assert(ACC * kAccCols <= 512, "TMEM has 512 columns");
-    static_assert(BN % 16 == 0 && BN <= 256, "UMMA N");
+    static_assert(kStage % 1024 == 0 && kBox % 1024 == 0, "tiles must keep 1024-byte alignment");
+    static_assert(BN % BOXN == 0 && BN % 16 == 0 && BN <= 256, "token tile");
+    static_assert(NSLOT * SLOT_COLS <= 512, "TMEM has 512 columns");
+    static_assert(GATE_UP ? (BN <= SLOT_COLS && (NSLOT >= 2 || BN <= SLOT_COLS / 2)) : BN <= SLOT_COLS,
+                  "an item must fit in its TMEM slots");
+    static_assert(kSmem <= 232448, "shared memory per CTA");
 };
 
 struct GemmParams {
@@ -54,17 +62,18 @@ struct GemmParams {
     int E;
     int K;                    // reduction length (G1: H, G2: I)
     int M;                    // weight rows (G1: I, G2: H)
+    int weights_once;         // 1: each weight tile is read once per call -> L2 evict-first
     long long timeout;
 };
 
 // Work-item decode from the per-CTA prefix table.
 struct Item {
-    int e, mt, nt, n_valid;
+    int e, mt, nt, n_valid, n_mma;
     int64_t row0;
 };
 
-__device__ __forceinline__ Item decode_item(int item, const int *tile_start, int E, int n_mt, int BN,
-                                            const int32_t *counts, const int64_t *offsets) {
+__device__ __forceinline__ Item decode_item(int item, const int *tile_start, int E, int BN, const int32_t *counts,
+                                            const int64_t *offsets) {
     int lo = 0, hi = E - 1;  // largest e with tile_start[e] <= item
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -79,24 +88,31 @@ __device__ __forceinline__ Item decode_item(int item, const int *tile_start, int
     it.mt = local / n_nt;
     it.nt = local - it.mt * n_nt;
     it.n_valid = min(BN, cnt - it.nt * BN);
+    it.n_mma = (it.n_valid + 15) & ~15;
     it.row0 = offsets[lo] + static_cast<int64_t>(it.nt) * BN;
     return it;
 }
 
-template <bool GATE_UP, int BN, int STAGES, int ACC>
+// TMEM slots an item occupies.
+template <bool GATE_UP, int SLOT_COLS>
+__device__ __forceinline__ int slots_of(int n_mma) {
+    return (GATE_UP && n_mma > SLOT_COLS / 2) ? 2 : 1;
+}
+
+template <bool GATE_UP, int BN, int BOXN, int STAGES, int NSLOT, int SLOT_COLS>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a0,  // W_gate (G1) / W_down (G2): [E][M][K]
                         const __grid_constant__ CUtensorMap tm_a1,  // W_up (G1); unused for G2
-                        const __grid_constant__ CUtensorMap tm_b,   // x_perm (G1) / h (G2): [R][K]
+                        const __grid_constant__ CUtensorMap tm_b,   // x_perm (G1) / h (G2): [R][K], box BOXN rows
                         const GemmParams p) {
-    using C = GemmCfg<GATE_UP, BN, STAGES, ACC>;
+    using C = GemmCfg<GATE_UP, BN, BOXN, STAGES, NSLOT, SLOT_COLS>;
     extern __shared__ uint8_t gemm_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(gemm_smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
     uint64_t *empty = full + STAGES;
     uint64_t *acc_full = empty + STAGES;
-    uint64_t *acc_empty = acc_full + ACC;
-    uint64_t *drain = acc_empty + ACC;
+    uint64_t *acc_empty = acc_full + NSLOT;
+    uint64_t *drain = acc_empty + NSLOT;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     int *tile_start = reinterpret_cast<int *>(smem + C::kBarOff + 256);
 
@@ -110,7 +126,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
-        for (int a = 0; a < ACC; ++a) {
+        for (int a = 0; a < NSLOT; ++a) {
             mbar_init(&acc_full[a], 1);
             mbar_init(&acc_empty[a], 4);
         }
@@ -151,24 +167,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (warp == 0) {
         if (lane == 0) {
             // ---------------- TMA producer ----------------
-            const uint64_t pol_w = policy_evict_first();  // weights: streamed once
-            const uint64_t pol_x = policy_evict_last();   // activations: re-read by other tiles
+            const uint64_t pol_w = p.weights_once ? policy_evict_first() : policy_evict_normal();
+            const uint64_t pol_x = policy_evict_last();  // activations: re-read by the other weight-row tiles
             int stage = 0;
             uint32_t phase = 0;
-            uint32_t issued = 0, issued_phase = 0;  // per-stage: ever issued / phase of last issue
+            uint32_t issued = 0, issued_phase = 0;  // per stage: ever issued / phase of the last issue
             bool ok = true;
             for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
-                const Item it = decode_item(item, tile_start, E, n_mt, BN, p.counts, p.offsets);
+                const Item it = decode_item(item, tile_start, E, BN, p.counts, p.offsets);
+                const int nbox = (it.n_mma + BOXN - 1) / BOXN;
+                const uint32_t bytes = C::kNumA * C::kA + nbox * C::kBox;
                 for (int kb = 0; kb < n_kb; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, p.timeout)) {
                         ok = false;
                         break;
                     }
                     uint8_t *sa = smem + stage * C::kStage;
-                    mbar_arrive_expect_tx(&full[stage], C::kStage);
+                    mbar_arrive_expect_tx(&full[stage], bytes);
                     tma_load_3d(sa, &tm_a0, &full[stage], kb * kBK, it.mt * kBM, it.e, pol_w);
                     if (GATE_UP) tma_load_3d(sa + C::kA, &tm_a1, &full[stage], kb * kBK, it.mt * kBM, it.e, pol_w);
-                    tma_load_2d(sa + C::kNumA * C::kA, &tm_b, &full[stage], kb * kBK, static_cast<int>(it.row0), pol_x);
+                    uint8_t *sb = sa + C::kNumA * C::kA;
+                    for (int b = 0; b < nbox; ++b)
+                        tma_load_2d(sb + b * C::kBox, &tm_b, &full[stage], kb * kBK,
+                                    static_cast<int>(it.row0) + b * BOXN, pol_x);
                     issued |= 1u << stage;
                     issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == STAGES) {
@@ -184,16 +205,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else if (warp == 1) {
         if (lane == 0) {
             // ---------------- MMA issuer ----------------
-            int stage = 0, acc = 0;
-            uint32_t phase = 0, acc_phase = 0;
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t uses = 0;  // TMEM slot uses so far
             bool ok = true;
             for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
-                const Item it = decode_item(item, tile_start, E, n_mt, BN, p.counts, p.offsets);
-                const int n_mma = (it.n_valid + 15) & ~15;
-                const uint32_t idesc = umma_idesc_bf16(kBM, n_mma);
-                if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, p.timeout)) break;
+                const Item it = decode_item(item, tile_start, E, BN, p.counts, p.offsets);
+                const uint32_t idesc = umma_idesc_bf16(kBM, it.n_mma);
+                const int u = slots_of<GATE_UP, SLOT_COLS>(it.n_mma);
+                const int s0 = uses % NSLOT, s1 = (uses + 1) % NSLOT;
+                for (int i = 0; i < u && ok; ++i) {
+                    const uint32_t c = uses + i;
+                    ok = mbar_wait(&acc_empty[c % NSLOT], ((c / NSLOT) & 1u) ^ 1u, p.timeout);
+                }
+                if (!ok) break;
                 tc_fence_after();
-                const uint32_t d0 = tmem_base + static_cast<uint32_t>(acc * C::kAccCols);
+                const uint32_t d0 = tmem_base + static_cast<uint32_t>(s0 * SLOT_COLS);
+                const uint32_t d1 = tmem_base + static_cast<uint32_t>(u == 2 ? s1 * SLOT_COLS : s0 * SLOT_COLS + SLOT_COLS / 2);
                 for (int kb = 0; kb < n_kb; ++kb) {
                     if (!mbar_wait(&full[stage], phase, p.timeout)) {
                         ok = false;
@@ -209,7 +237,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
                         // +32 bytes along K inside the swizzle row = +2 in the 16-byte address field
                         umma_bf16(d0, da0 + 2 * kk, db + 2 * kk, idesc, accum);
-                        if (GATE_UP) umma_bf16(d0 + BN, da1 + 2 * kk, db + 2 * kk, idesc, accum);
+                        if (GATE_UP) umma_bf16(d1, da1 + 2 * kk, db + 2 * kk, idesc, accum);
                     }
                     umma_commit(&empty[stage]);  // frees the smem stage once these MMAs completed
                     if (++stage == STAGES) {
@@ -218,11 +246,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                 }
                 if (!ok) break;
-                umma_commit(&acc_full[acc]);  // accumulator ready for the epilogue
-                if (++acc == ACC) {
-                    acc = 0;
-                    acc_phase ^= 1u;
-                }
+                for (int i = 0; i < u; ++i) umma_commit(&acc_full[(uses + i) % NSLOT]);
+                uses += u;
             }
             // all issued MMAs complete before TMEM is released
             umma_commit(drain);
@@ -231,20 +256,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     } else if (warp >= 4) {
         // ---------------- epilogue ----------------
         const int q = warp - 4;  // TMEM lane quadrant
-        int acc = 0;
-        uint32_t acc_phase = 0;
+        uint32_t uses = 0;
         for (int item = blockIdx.x; item < total; item += gridDim.x) {
-            const Item it = decode_item(item, tile_start, E, n_mt, BN, p.counts, p.offsets);
-            if (!mbar_wait(&acc_full[acc], acc_phase, p.timeout)) break;
+            const Item it = decode_item(item, tile_start, E, BN, p.counts, p.offsets);
+            const int u = slots_of<GATE_UP, SLOT_COLS>(it.n_mma);
+            bool ok = true;
+            for (int i = 0; i < u && ok; ++i) {
+                const uint32_t c = uses + i;
+                ok = mbar_wait(&acc_full[c % NSLOT], (c / NSLOT) & 1u, p.timeout);
+            }
+            if (!ok) break;
             tc_fence_after();
+            const int s0 = uses % NSLOT, s1 = (uses + 1) % NSLOT;
             const int m = it.mt * kBM + q * 32 + lane;  // weight row of this thread
-            const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * C::kAccCols);
+            const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+            const uint32_t t0 = tmem_base + lane_off + static_cast<uint32_t>(s0 * SLOT_COLS);
+            const uint32_t t1 = tmem_base + lane_off +
+                                static_cast<uint32_t>(u == 2 ? s1 * SLOT_COLS : s0 * SLOT_COLS + SLOT_COLS / 2);
             for (int c = 0; c < it.n_valid; c += 16) {
                 uint32_t r0[16];
-                tmem_ld16(tb + c, r0);
+                tmem_ld16(t0 + c, r0);
                 if (GATE_UP) {
                     uint32_t r1[16];
-                    tmem_ld16(tb + BN + c, r1);
+                    tmem_ld16(t1 + c, r1);
                     tmem_ld_wait();
                     if (m < p.M) {
                         __nv_bfloat16 *h = reinterpret_cast<__nv_bfloat16 *>(p.out);
@@ -266,11 +300,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[acc]);
-            if (++acc == ACC) {
-                acc = 0;
-                acc_phase ^= 1u;
-            }
+            if (lane == 0)
+                for (int i = 0; i < u; ++i) mbar_arrive(&acc_empty[(uses + i) % NSLOT]);
+            uses += u;
         }
     }
     tc_fence_before();
