@@ -178,8 +178,10 @@ __device__ __forceinline__ int lane_id() { return threadIdx.x & 31; }
 __device__ __forceinline__ bool elect_lane0() { return (threadIdx.x & 31) == 0; }
 
 __device__ __forceinline__ float silu_mul(float g, float u) {
-    // SiLU(g) * u with SiLU(z) = z * sigmoid(z), in FP32.
-    return g / (1.0f + expf(-g)) * u;
+    // SiLU(g) * u with SiLU(z) = z * sigmoid(z), in FP32 with the fast exponential and division
+    // (a few ulp; the product is rounded to bf16 next).  For g -> -inf, exp overflows to +inf and
+    // the quotient is 0, the limit of SiLU.
+    return __fdividef(g, 1.0f + __expf(-g)) * u;
 }
 
 }  // namespace beam

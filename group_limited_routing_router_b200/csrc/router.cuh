@@ -29,11 +29,14 @@ namespace cg = cooperative_groups;
 
 constexpr int kRtTok = 64;       // tokens per cluster tile
 constexpr int kRtBK = 32;        // K per shared-memory stage
+constexpr int kRtWPad = kRtBK + 2;  // padded W row (floats): conflict-free 8-byte reads across experts
 constexpr int kRtThreads = 256;  // 8 warps
 constexpr int kRtCluster = 8;    // CTAs per cluster (split-K factor)
 constexpr int kRtSlots = 256;    // expert slots per tile (E <= 256)
-constexpr int kRtSmemFloats = 2 * kRtBK * kRtSlots + 2 * kRtBK * kRtTok;  // 20480 floats = 80 KB
-static_assert(kRtTok * kRtSlots <= 2 * kRtBK * kRtSlots, "partial logits must fit in the W staging area");
+constexpr int kRtWFloats = 2 * kRtSlots * kRtWPad;  // W stages [2][256][36]
+constexpr int kRtXFloats = 2 * kRtBK * kRtTok;      // x stages [2][32][64]
+constexpr int kRtSmemFloats = kRtWFloats + kRtXFloats;  // 22528 floats = 88 KB: two CTAs per SM
+static_assert(kRtTok * kRtSlots <= kRtWFloats, "partial logits must fit in the W staging area");
 
 struct RouterParams {
     const __nv_bfloat16 *x;  // [T, H]
@@ -64,19 +67,27 @@ __device__ __forceinline__ ArgMax warp_argmax(float v, int i) {
     return {v, i};
 }
 
-__global__ void __cluster_dims__(kRtCluster, 1, 1) __launch_bounds__(kRtThreads, 1)
+__device__ __forceinline__ void cp_async8(void *smem, const void *gmem, bool valid) {
+    // 8-byte global -> shared copy that bypasses registers; zero-fills when !valid
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_u32(smem)), "l"(gmem), "r"(valid ? 8 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+__global__ void __cluster_dims__(kRtCluster, 1, 1) __launch_bounds__(kRtThreads, 2)
     router_topk_kernel(const RouterParams p) {
     extern __shared__ float4 rt_smem4[];
     float *smem = reinterpret_cast<float *>(rt_smem4);
-    float *ws = smem;                            // [2][kRtBK][kRtSlots]
-    float *xs = smem + 2 * kRtBK * kRtSlots;     // [2][kRtBK][kRtTok]
-    float *part = smem;                          // [kRtTok][kRtSlots] after the K loop
+    float *ws = smem;                 // [2][kRtSlots][kRtWPad]  (expert-major, k contiguous)
+    float *xs = smem + kRtWFloats;    // [2][kRtBK][kRtTok]      (k-major, tokens contiguous)
+    float *part = smem;               // [kRtTok][kRtSlots] after the K loop
 
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = static_cast<int>(cluster.block_rank());
     const int64_t t0 = static_cast<int64_t>(blockIdx.x / kRtCluster) * kRtTok;
     const int tid = threadIdx.x;
-    const int tx = tid & 31, ty = tid >> 5;
+    const int tx = tid & 31, ty = tid >> 5;  // experts tx + 32j, tokens 8ty + i
 
     // ---- split-K FP32 projection --------------------------------------------------------------
     const int nsteps = p.H / kRtBK;
@@ -89,31 +100,26 @@ __global__ void __cluster_dims__(kRtCluster, 1, 1) __launch_bounds__(kRtThreads,
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[i][j] = 0.0f;
 
-    const int we = tid;  // expert row this thread stages
-    const bool w_ok = we < p.E;
-    const float *wrow = p.w + static_cast<int64_t>(w_ok ? we : 0) * p.H;
     const int xt = tid & 63, xc = (tid >> 6) * 8;  // token, k-chunk of 8 this thread stages
     const bool x_ok = (t0 + xt) < p.T;
     const __nv_bfloat16 *xrow = p.x + (x_ok ? (t0 + xt) : 0) * static_cast<int64_t>(p.H);
-
-    float4 wreg[8];
     uint4 xreg;
-    auto gload = [&](int s) {
-        const int k0 = s * kRtBK;
+
+    // W stage: thread e copies row e (32 floats) as 16 chunks of 8 B; rows are 34 floats apart in
+    // shared memory, so every destination is 8-byte aligned
+    const bool w_ok = tid < p.E;
+    const float *wrow = p.w + static_cast<int64_t>(w_ok ? tid : 0) * p.H;
+    auto w_async = [&](int s, int buf) {
+        float *dst = ws + buf * kRtSlots * kRtWPad + tid * kRtWPad;
+        const float *src = wrow + s * kRtBK;
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-            wreg[i] = w_ok ? __ldg(reinterpret_cast<const float4 *>(wrow + k0) + i) : make_float4(0.f, 0.f, 0.f, 0.f);
-        xreg = x_ok ? __ldg(reinterpret_cast<const uint4 *>(xrow + k0 + xc)) : make_uint4(0u, 0u, 0u, 0u);
+        for (int i = 0; i < 16; ++i) cp_async8(dst + 2 * i, src + 2 * i, w_ok);
+        cp_async_commit();
     };
-    auto sstore = [&](int buf) {
-        float *wsb = ws + buf * kRtBK * kRtSlots;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            wsb[(4 * i + 0) * kRtSlots + we] = wreg[i].x;
-            wsb[(4 * i + 1) * kRtSlots + we] = wreg[i].y;
-            wsb[(4 * i + 2) * kRtSlots + we] = wreg[i].z;
-            wsb[(4 * i + 3) * kRtSlots + we] = wreg[i].w;
-        }
+    auto x_load = [&](int s) {
+        xreg = x_ok ? __ldg(reinterpret_cast<const uint4 *>(xrow + s * kRtBK + xc)) : make_uint4(0u, 0u, 0u, 0u);
+    };
+    auto x_store = [&](int buf) {
         float *xsb = xs + buf * kRtBK * kRtTok;
         const uint32_t xw[4] = {xreg.x, xreg.y, xreg.z, xreg.w};
 #pragma unroll
@@ -125,39 +131,49 @@ __global__ void __cluster_dims__(kRtCluster, 1, 1) __launch_bounds__(kRtThreads,
     };
 
     if (s_begin < s_end) {
-        gload(s_begin);
-        sstore(0);
+        w_async(s_begin, 0);
+        x_load(s_begin);
+        x_store(0);
+        cp_async_wait_all();
         __syncthreads();
         for (int s = s_begin; s < s_end; ++s) {
             const int buf = (s - s_begin) & 1;
-            if (s + 1 < s_end) gload(s + 1);
-            const float *wsb = ws + buf * kRtBK * kRtSlots + tx * 8;
-            const float *xsb = xs + buf * kRtBK * kRtTok + ty * 8;
-#pragma unroll 8
-            for (int kk = 0; kk < kRtBK; ++kk) {
-                const float4 xa = *reinterpret_cast<const float4 *>(xsb + kk * kRtTok);
-                const float4 xb = *reinterpret_cast<const float4 *>(xsb + kk * kRtTok + 4);
-                const float4 wa = *reinterpret_cast<const float4 *>(wsb + kk * kRtSlots);
-                const float4 wb = *reinterpret_cast<const float4 *>(wsb + kk * kRtSlots + 4);
-                const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-                const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(xv[i], wv[j], acc[i][j]);
+            if (s + 1 < s_end) {
+                w_async(s + 1, buf ^ 1);
+                x_load(s + 1);
             }
-            if (s + 1 < s_end) sstore(buf ^ 1);
+            const float *wsb = ws + buf * kRtSlots * kRtWPad + tx * kRtWPad;
+            const float *xsb = xs + buf * kRtBK * kRtTok + ty * 8;
+#pragma unroll 4
+            for (int kp = 0; kp < kRtBK / 2; ++kp) {
+                float2 wv[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    wv[j] = *reinterpret_cast<const float2 *>(wsb + 32 * j * kRtWPad + 2 * kp);
+#pragma unroll
+                for (int kk = 0; kk < 2; ++kk) {
+                    const float4 xa = *reinterpret_cast<const float4 *>(xsb + (2 * kp + kk) * kRtTok);
+                    const float4 xb = *reinterpret_cast<const float4 *>(xsb + (2 * kp + kk) * kRtTok + 4);
+                    const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float wj = kk == 0 ? wv[j].x : wv[j].y;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) acc[i][j] = fmaf(xv[i], wj, acc[i][j]);
+                    }
+                }
+            }
+            if (s + 1 < s_end) x_store(buf ^ 1);
+            cp_async_wait_all();
             __syncthreads();
         }
     }
 
     // partial logits -> shared memory (the staging buffers are free after the last barrier)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        float *dst = part + (ty * 8 + i) * kRtSlots + tx * 8;
-        reinterpret_cast<float4 *>(dst)[0] = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
-        reinterpret_cast<float4 *>(dst)[1] = make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
-    }
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) part[(ty * 8 + i) * kRtSlots + tx + 32 * j] = acc[i][j];
     cluster.sync();
 
     // ---- reduction over the cluster + selection: warp w owns token 8*rank + w of the tile ------
@@ -167,11 +183,10 @@ __global__ void __cluster_dims__(kRtCluster, 1, 1) __launch_bounds__(kRtThreads,
     if (t < p.T) {
         const int per = p.E / p.G;
         float sc[8], sel[8];
-        int eid[8];
+#define EID(j) (lane + 32 * (j))
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const int e = lane + 32 * j;
-            eid[j] = e;
+            const int e = EID(j);
             float logit = 0.0f;
             if (e < p.E) {
 #pragma unroll
@@ -195,10 +210,10 @@ __global__ void __cluster_dims__(kRtCluster, 1, 1) __launch_bounds__(kRtThreads,
                 int bi = 0x7fffffff;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    const bool cand = eid[j] < p.E && !((taken >> j) & 1u) && (eid[j] / per) == g;
-                    if (cand && (sel[j] > bv || (sel[j] == bv && eid[j] < bi))) {
+                    const bool cand = EID(j) < p.E && !((taken >> j) & 1u) && (EID(j) / per) == g;
+                    if (cand && (sel[j] > bv || (sel[j] == bv && EID(j) < bi))) {
                         bv = sel[j];
-                        bi = eid[j];
+                        bi = EID(j);
                     }
                 }
                 const ArgMax m = warp_argmax(bv, bi);
@@ -223,10 +238,10 @@ __global__ void __cluster_dims__(kRtCluster, 1, 1) __launch_bounds__(kRtThreads,
             int bi = 0x7fffffff;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const bool cand = eid[j] < p.E && !((taken >> j) & 1u) && ((kept >> (eid[j] / per)) & 1u);
-                if (cand && (sel[j] > bv || (sel[j] == bv && eid[j] < bi))) {
+                const bool cand = EID(j) < p.E && !((taken >> j) & 1u) && ((kept >> (EID(j) / per)) & 1u);
+                if (cand && (sel[j] > bv || (sel[j] == bv && EID(j) < bi))) {
                     bv = sel[j];
-                    bi = eid[j];
+                    bi = EID(j);
                 }
             }
             const ArgMax m = warp_argmax(bv, bi);
@@ -246,6 +261,7 @@ __global__ void __cluster_dims__(kRtCluster, 1, 1) __launch_bounds__(kRtThreads,
             p.ids[t * p.topk + lane] = my_id;
             p.wts[t * p.topk + lane] = my_s / den;
         }
+#undef EID
     }
     // no CTA may leave while another still reads its shared memory
     cluster.sync();
