@@ -8,8 +8,8 @@
 // Layout of the work (sm_100a):
 //   * one thread-block cluster of 8 CTAs per tile of 64 tokens; CTA r of the cluster computes the
 //     partial logits of all 64 tokens x 256 expert slots over the r-th eighth of the hidden
-//     dimension (split-K), with an 8x8 register tile per thread and double-buffered shared-memory
-//     staging (x widened from bf16 to fp32, which is exact);
+//     dimension (split-K): 8x8 register tile per thread, 32x64 tile per warp, W staged by cp.async
+//     and x widened from bf16 to fp32 (exact) in double-buffered shared memory;
 //   * the partial logits stay in each CTA's shared memory; after a cluster barrier, CTA r reduces
 //     tokens [8r, 8r+8) over the 8 CTAs through distributed shared memory, in rank order, so the
 //     FP32 sum order is fixed (deterministic);
@@ -87,7 +87,12 @@ __global__ void __cluster_dims__(kRtCluster, 1, 1) __launch_bounds__(kRtThreads,
     const int rank = static_cast<int>(cluster.block_rank());
     const int64_t t0 = static_cast<int64_t>(blockIdx.x / kRtCluster) * kRtTok;
     const int tid = threadIdx.x;
-    const int tx = tid & 31, ty = tid >> 5;  // experts tx + 32j, tokens 8ty + i
+    const int tx = tid & 31, ty = tid >> 5;  // lane, warp
+    // 2-D warp tile: warp ty covers tokens 32*(ty&1) + [0,32) x experts 64*(ty>>1) + [0,64); lane
+    // (a = tx>>3, b = tx&7) owns tokens 32*(ty&1) + 8a + i and experts 64*(ty>>1) + b + 8j (i, j < 8),
+    // so every shared-memory read below is shared by 4 or 8 lanes and is conflict-free.
+    const int tok0 = 32 * (ty & 1) + 8 * (tx >> 3);
+    const int exp0 = 64 * (ty >> 1) + (tx & 7);
 
     // ---- split-K FP32 projection --------------------------------------------------------------
     const int nsteps = p.H / kRtBK;
@@ -142,14 +147,14 @@ __global__ void __cluster_dims__(kRtCluster, 1, 1) __launch_bounds__(kRtThreads,
                 w_async(s + 1, buf ^ 1);
                 x_load(s + 1);
             }
-            const float *wsb = ws + buf * kRtSlots * kRtWPad + tx * kRtWPad;
-            const float *xsb = xs + buf * kRtBK * kRtTok + ty * 8;
+            const float *wsb = ws + buf * kRtSlots * kRtWPad + exp0 * kRtWPad;
+            const float *xsb = xs + buf * kRtBK * kRtTok + tok0;
 #pragma unroll 4
             for (int kp = 0; kp < kRtBK / 2; ++kp) {
                 float2 wv[8];
 #pragma unroll
                 for (int j = 0; j < 8; ++j)
-                    wv[j] = *reinterpret_cast<const float2 *>(wsb + 32 * j * kRtWPad + 2 * kp);
+                    wv[j] = *reinterpret_cast<const float2 *>(wsb + 8 * j * kRtWPad + 2 * kp);
 #pragma unroll
                 for (int kk = 0; kk < 2; ++kk) {
                     const float4 xa = *reinterpret_cast<const float4 *>(xsb + (2 * kp + kk) * kRtTok);
@@ -173,7 +178,7 @@ __global__ void __cluster_dims__(kRtCluster, 1, 1) __launch_bounds__(kRtThreads,
 #pragma unroll
     for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) part[(ty * 8 + i) * kRtSlots + tx + 32 * j] = acc[i][j];
+        for (int j = 0; j < 8; ++j) part[(tok0 + i) * kRtSlots + exp0 + 8 * j] = acc[i][j];
     cluster.sync();
 
     // ---- reduction over the cluster + selection: warp w owns token 8*rank + w of the tile ------
