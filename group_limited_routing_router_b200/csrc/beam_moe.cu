@@ -445,3 +445,64 @@ const char *beam_moe_strerror(int code) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------------
+// beam_moe_permute_noalloc: the dispatch with its scratch in a fixed device array instead of a
+// caller-provided workspace, for callers that must not allocate device memory.
+namespace beam {
+namespace {
+
+// Per-chunk expert counts of the dispatch: ceil(T / 256) * n_experts ints at most.  One copy per
+// device that loads the library, held until the process exits.
+static __device__ __align__(256) int32_t g_noalloc_scratch[BEAM_MOE_NOALLOC_SCRATCH_INTS];
+
+struct NoallocSlot {
+    std::once_flag once;
+    int status = BEAM_MOE_ERR_CUDA;
+    int32_t *ptr = nullptr;  // device address of g_noalloc_scratch on this device
+};
+NoallocSlot g_noalloc[kMaxDevices];
+
+// On the first call for a device (that device current): resolve the array's device address.  The
+// name g_noalloc_scratch in host code only stands in for the symbol; kernels get this address.
+int noalloc_scratch(int dev, int32_t **out) {
+    NoallocSlot &s = g_noalloc[dev];
+    std::call_once(s.once, [&]() {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) == cudaSuccess && p) {
+            s.ptr = static_cast<int32_t *>(p);
+            s.status = BEAM_MOE_OK;
+        }
+    });
+    *out = s.ptr;
+    return s.status;
+}
+
+}  // namespace
+}  // namespace beam
+
+extern "C" {
+
+int beam_moe_permute_noalloc(const beam_moe_config *cfg, int64_t T, const int32_t *topk_ids, int32_t *counts,
+                             int64_t *offsets, int32_t *row_src, int32_t *dest_row, void *stream) {
+    int rc = validate(cfg);
+    if (rc) return rc;
+    if ((rc = check_T(cfg, T))) return rc;
+    if (n_chunks(T) * cfg->n_experts > BEAM_MOE_NOALLOC_SCRATCH_INTS) return BEAM_MOE_ERR_INVALID_ARG;
+    if (!counts || !offsets || (T > 0 && (!topk_ids || !row_src || !dest_row))) return BEAM_MOE_ERR_NULL;
+    int dev;
+    if ((rc = init_device(&dev))) return rc;
+    int32_t *scratch = nullptr;
+    if ((rc = noalloc_scratch(dev, &scratch))) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * cfg->n_experts, s) != cudaSuccess ||
+            cudaMemsetAsync(offsets, 0, sizeof(int64_t) * (cfg->n_experts + 1), s) != cudaSuccess)
+            return BEAM_MOE_ERR_CUDA;
+        return BEAM_MOE_OK;
+    }
+    // the histogram kernel writes every scratch entry the scan then reads: nothing to clear
+    return enqueue_permute(cfg, T, topk_ids, counts, offsets, row_src, dest_row, scratch, s);
+}
+
+}  // extern "C"

@@ -155,6 +155,29 @@ BEAM_MOE_API int beam_moe_forward_profiled(const beam_moe_config *cfg, int64_t T
                                            void *stream, void *const *events);
 
 /*
+ * beam_moe_permute without a workspace: the same dispatch (identical outputs), with its scratch in
+ * a fixed device array inside this library instead of caller memory.  The Beam pages have no
+ * counterpart; this exists for callers that cannot allocate device memory when they enqueue work,
+ * e.g. a plugin inside an inference server whose host framework owns all device memory, or a
+ * latency-critical loop where cudaMalloc is forbidden because it can synchronise the device.
+ *   - Limit: ceil(T / 256) * n_experts <= BEAM_MOE_NOALLOC_SCRATCH_INTS (65,536 ints = 256 KiB;
+ *     T <= 65,536 tokens at 256 experts); larger calls return BEAM_MOE_ERR_INVALID_ARG and
+ *     enqueue nothing.
+ *   - The array exists once per device that loads the library and stays allocated until the
+ *     process exits.  The first call on a device, with that device current, looks up the array's
+ *     device address (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Allocates nothing (no cudaMalloc, cudaFree or allocating library call).  Every call shares
+ *     the one array and it keeps the previous call's contents; each call overwrites every entry it
+ *     reads, so nothing needs clearing.  Calls whose executions overlap on the GPU (different
+ *     streams, or different host threads without ordering) race on the array: order them.
+ * Arguments and outputs as for beam_moe_permute.
+ */
+#define BEAM_MOE_NOALLOC_SCRATCH_INTS 65536
+BEAM_MOE_API int beam_moe_permute_noalloc(const beam_moe_config *cfg, int64_t T, const int32_t *topk_ids,
+                                          int32_t *counts, int64_t *offsets, int32_t *row_src, int32_t *dest_row,
+                                          void *stream);
+
+/*
  * Synchronises `stream`, then returns and clears the current device's status word
  * (BEAM_MOE_OK, BEAM_MOE_ERR_DEVICE_TIMEOUT or BEAM_MOE_ERR_BAD_INDEX), or BEAM_MOE_ERR_CUDA.
  */
