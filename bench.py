@@ -222,31 +222,62 @@ def config_dict(wl):
             "parallelism": "replicas (one independent layer instance per GPU)"}
 
 
+class Ranks:
+    """One process per GPU: barrier, max-over-ranks and the whole-job rate of independent replicas.
+
+    backend "nccl" on GPUs; "gloo" works the same way on CPU (used by the multi-rank tests)."""
+
+    def __init__(self, backend: str = "nccl", timeout_s: int = 120):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.backend = backend
+        self.dist = None
+        if self.world > 1:
+            import datetime
+
+            import torch.distributed as dist
+            kw = {"device_id": torch.device("cuda", self.local)} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+            self.dist = dist
+
+    def _sync_device(self):
+        if self.backend == "nccl" and torch.cuda.is_available():
+            torch.cuda.synchronize()
+
+    def barrier(self):
+        """Device synchronize, then a barrier over all ranks, then synchronize again."""
+        self._sync_device()
+        if self.dist is not None:
+            self.dist.barrier()
+        self._sync_device()
+
+    def max(self, v: float) -> float:
+        if self.dist is None:
+            return v
+        dev = "cuda" if self.backend == "nccl" else "cpu"
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def rate(self, units_per_rank: float, ms_this_rank: float) -> float:
+        """Whole-job units/s: all ranks' units over the slowest rank's time."""
+        return self.world * units_per_rank / (self.max(ms_this_rank) / 1e3)
+
+    def close(self):
+        if self.dist is not None:
+            self.dist.barrier()
+            self.dist.destroy_process_group()
+            self.dist = None
+
+
 def run_ours(args):
     import group_limited_routing_router_b200 as bm
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    ranks = Ranks("nccl")
+    world, rank, local = ranks.world, ranks.rank, ranks.local
     torch.cuda.set_device(local)
-    dist = None
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-        torch.cuda.synchronize()
-
-    def max_over_ranks(v: float) -> float:
-        if dist is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    barrier = ranks.barrier
 
     wl = bs.get(args.workload)
     layer = wl.layer
@@ -289,9 +320,9 @@ def run_ours(args):
         torch.cuda.synchronize()
         clocks.marks[-1] = clocks.n_samples()
     clk = clocks.stop()
-    ms_total = max_over_ranks(ev0.elapsed_time(ev1))
-    ms_step = ms_total / args.steps
-    value = world * T * args.steps / (ms_total / 1e3)
+    ms_this = ev0.elapsed_time(ev1)
+    value = ranks.rate(T * args.steps, ms_this)
+    ms_step = ranks.max(ms_this) / args.steps
     n_act = int((torch.bincount(ids.flatten().long(), minlength=wl.n_experts) > 0).sum().item())
 
     # per-stage device time from events recorded between the launches (same stream)
@@ -318,8 +349,7 @@ def run_ours(args):
         y_host.copy_(y, non_blocking=True)
     e1.record(stream)
     barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1))
-    e2e_value = world * T * args.steps / (e2e_ms / 1e3)
+    e2e_value = ranks.rate(T * args.steps, e0.elapsed_time(e1))
     assert bm.device_status() == bm.OK
 
     alg = algorithmic(wl, n_act)
@@ -356,9 +386,7 @@ def run_ours(args):
             "clocks": clk, "gpu_launches": 8 * args.steps, "kernel_source": src_hash}
     if rank == 0:
         print(json.dumps(line))
-    if dist is not None:
-        dist.barrier()
-        dist.destroy_process_group()
+    ranks.close()
 
 
 def main():
