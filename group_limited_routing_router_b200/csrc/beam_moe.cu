@@ -76,7 +76,7 @@ int init_device(int *dev_out) {
             return;
         }
         bool ok = cudaFuncSetAttribute(router_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kRtSmemFloats * 4) == cudaSuccess;
+                                       kRtSmemBytes) == cudaSuccess;
         ok = ok && cudaFuncSetAttribute(G1_WIDE_KERNEL, cudaFuncAttributeMaxDynamicSharedMemorySize, G1Wide::kSmem) ==
                        cudaSuccess;
         ok = ok && cudaFuncSetAttribute(G2_WIDE_KERNEL, cudaFuncAttributeMaxDynamicSharedMemorySize, G2Wide::kSmem) ==
@@ -189,6 +189,17 @@ bool make_map_3d(CUtensorMap *m, const void *base, uint64_t K, uint64_t M, uint6
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? BEAM_MOE_OK : BEAM_MOE_ERR_CUDA; }
 
+// Generic 2-D tensor map: [rows][inner] elements of `esize` bytes, box {box_inner, box_rows}.
+bool make_map_2d_any(CUtensorMap *m, CUtensorMapDataType dt, int esize, const void *base, uint64_t inner,
+                     uint64_t rows, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw) {
+    const cuuint64_t dims[2] = {inner, rows};
+    const cuuint64_t strides[1] = {inner * esize};
+    const cuuint32_t box[2] = {box_inner, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return encode_fn()(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int enqueue_route(const beam_moe_config *c, int64_t T, const beam_bf16 *x, const float *w_router, const float *bias,
                   int32_t *ids, float *w, cudaStream_t s) {
     RouterParams p;
@@ -204,8 +215,17 @@ int enqueue_route(const beam_moe_config *c, int64_t T, const beam_bf16 *x, const
     p.topk_groups = c->topk_groups;
     p.topk = c->topk;
     p.group_topn = c->group_topn;
+    // W_r tiles: 32 fp32 (one 128-byte swizzled row) x all 256 expert slots (rows >= E read as 0);
+    // x tiles: 32 bf16 (64-byte swizzled row) x 64 tokens (rows >= T read as 0)
+    CUtensorMap m_w, m_x;
+    if (!encode_fn()) return BEAM_MOE_ERR_CUDA;
+    if (!make_map_2d_any(&m_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, w_router, c->hidden, c->n_experts, kRtBK, kRtSlots,
+                         CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_2d_any(&m_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, c->hidden, T, kRtBK, kRtTok,
+                         CU_TENSOR_MAP_SWIZZLE_64B))
+        return BEAM_MOE_ERR_CUDA;
     const int64_t tiles = (T + kRtTok - 1) / kRtTok;
-    router_topk_kernel<<<static_cast<unsigned>(tiles * kRtCluster), kRtThreads, kRtSmemFloats * 4, s>>>(p);
+    router_topk_kernel<<<static_cast<unsigned>(tiles * kRtCluster), kRtThreads, kRtSmemBytes, s>>>(m_w, m_x, p);
     return launch_status();
 }
 

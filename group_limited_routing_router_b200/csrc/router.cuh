@@ -9,9 +9,9 @@
 //   * one thread-block cluster of 8 CTAs per tile of 64 tokens; CTA r of the cluster computes the
 //     partial logits of all 64 tokens x 256 expert slots over the r-th eighth of the hidden
 //     dimension (split-K).  128 threads, 8 tokens x 16 experts of FP32 accumulators per thread,
-//     32 tokens x 128 experts per warp; W staged by cp.async and x widened from bf16 to fp32
-//     (exact) in double-buffered shared memory.  Shared memory hands each lane about one float
-//     per wavefront, so the register tile is sized for 5.3 FMAs per float read;
+//     32 tokens x 128 experts per warp.  W (fp32) and x (bf16) tiles arrive by TMA into a 3-stage
+//     mbarrier pipeline (one thread issues two bulk copies per stage, so the compute warps issue
+//     no staging instructions); x is widened from bf16 to fp32 (exact) in registers;
 //   * the partial logits stay in each CTA's shared memory; after a cluster barrier, CTA r reduces
 //     tokens [8r, 8r+8) over the 8 CTAs through distributed shared memory, in rank order, so the
 //     FP32 sum order is fixed (deterministic);
@@ -28,16 +28,18 @@ namespace beam {
 
 namespace cg = cooperative_groups;
 
-constexpr int kRtTok = 64;          // tokens per cluster tile
-constexpr int kRtBK = 32;           // K per shared-memory stage
-constexpr int kRtWPad = kRtBK + 2;  // padded W row (floats): conflict-free 8-byte reads across experts
-constexpr int kRtThreads = 128;     // 4 warps
-constexpr int kRtCluster = 8;       // CTAs per cluster (split-K factor)
-constexpr int kRtSlots = 256;       // expert slots per tile (E <= 256)
-constexpr int kRtWFloats = 2 * kRtSlots * kRtWPad;      // W stages [2][256][34]
-constexpr int kRtXFloats = 2 * kRtBK * kRtTok;          // x stages [2][32][64]
-constexpr int kRtSmemFloats = kRtWFloats + kRtXFloats;  // 21504 floats = 84 KB: two CTAs per SM
-static_assert(kRtTok * kRtSlots <= kRtWFloats, "partial logits must fit in the W staging area");
+constexpr int kRtTok = 64;        // tokens per cluster tile
+constexpr int kRtBK = 32;         // K per pipeline stage (one 128-byte row of fp32 W)
+constexpr int kRtThreads = 128;   // 4 warps
+constexpr int kRtCluster = 8;     // CTAs per cluster (split-K factor)
+constexpr int kRtSlots = 256;     // expert slots per tile (E <= 256)
+constexpr int kRtStages = 3;      // TMA pipeline depth
+constexpr int kRtWBytes = kRtSlots * kRtBK * 4;  // W stage: [256 rows][32 fp32], 128-byte swizzle (32 KB)
+constexpr int kRtXBytes = kRtTok * kRtBK * 2;    // x stage: [64 rows][32 bf16], 64-byte swizzle (4 KB)
+constexpr int kRtStageBytes = kRtWBytes + kRtXBytes;
+constexpr int kRtSmemBytes = 1024 + kRtStages * kRtStageBytes + 128;  // + alignment + barriers: two CTAs per SM
+static_assert(kRtTok * kRtSlots * 4 <= kRtStages * kRtStageBytes, "partial logits must fit in the stages");
+static_assert(kRtStageBytes % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
 
 struct RouterParams {
     const __nv_bfloat16 *x;  // [T, H]
@@ -68,14 +70,6 @@ __device__ __forceinline__ ArgMax warp_argmax(float v, int i) {
     return {v, i};
 }
 
-__device__ __forceinline__ void cp_async8(void *smem, const void *gmem, bool valid) {
-    // 8-byte global -> shared copy that bypasses registers; zero-fills when !valid
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_u32(smem)), "l"(gmem), "r"(valid ? 8 : 0)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
 // Insert v into the descending pair (a1 >= a2).
 __device__ __forceinline__ void top2_insert(float &a1, float &a2, float v) {
     a2 = fmaxf(a2, fminf(a1, v));
@@ -83,28 +77,52 @@ __device__ __forceinline__ void top2_insert(float &a1, float &a2, float v) {
 }
 
 __global__ void __cluster_dims__(kRtCluster, 1, 1) __launch_bounds__(kRtThreads, 2)
-    router_topk_kernel(const RouterParams p) {
-    extern __shared__ float4 rt_smem4[];
-    float *smem = reinterpret_cast<float *>(rt_smem4);
-    float *ws = smem;                 // [2][kRtSlots][kRtWPad]  (expert-major, k contiguous)
-    float *xs = smem + kRtWFloats;    // [2][kRtBK][kRtTok]      (k-major, tokens contiguous)
-    float *part = smem;               // [kRtTok][kRtSlots] after the K loop
+    router_topk_kernel(const __grid_constant__ CUtensorMap tm_w,  // W_r [E][H] fp32, box {32, 256}
+                       const __grid_constant__ CUtensorMap tm_x,  // x [T][H] bf16, box {32, 64}
+                       const RouterParams p) {
+    extern __shared__ uint8_t rt_smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(rt_smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + kRtStages * kRtStageBytes);
+    uint64_t *empty = full + kRtStages;
+    float *part = reinterpret_cast<float *>(smem);  // [kRtTok][kRtSlots] after the K loop
 
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = static_cast<int>(cluster.block_rank());
     const int64_t t0 = static_cast<int64_t>(blockIdx.x / kRtCluster) * kRtTok;
     const int tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
-    // warp tile: tokens 32*(warp&1) + [0,32) x experts 128*(warp>>1) + [0,128); lane (a = lane>>3,
-    // b = lane&7) owns tokens tok0 + i (i < 8) and experts exp0 + 8j (j < 16).  W reads: 8 distinct
-    // rows per half-warp, 34 floats apart -> distinct banks; x reads: one address per quarter-warp.
-    const int tok0 = 32 * (warp & 1) + 8 * (lane >> 3);
-    const int exp0 = 128 * (warp >> 1) + (lane & 7);
+    // warp tile: tokens 32*(warp&1) + [0,32) x experts 128*(warp>>1) + [0,128).  Lane (a = lane>>3,
+    // b = lane&7) owns tokens tokA + 4i (i < 8) and experts expB + 8j (j < 16).
+    const int a = lane >> 3, b = lane & 7;
+    const int tokA = 32 * (warp & 1) + a;
+    const int expB = 128 * (warp >> 1) + b;
 
     // ---- split-K FP32 projection --------------------------------------------------------------
     const int nsteps = p.H / kRtBK;
     const int s_begin = rank * nsteps / kRtCluster;
     const int s_end = (rank + 1) * nsteps / kRtCluster;
+    const int n_my = s_end - s_begin;
+
+    if (tid == 0) {
+        for (int i = 0; i < kRtStages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kRtThreads / 32);
+        }
+        fence_mbar_init();
+        prefetch_tensormap(&tm_w);
+        prefetch_tensormap(&tm_x);
+    }
+    __syncthreads();
+    auto issue = [&](int i) {  // load step s_begin + i into stage i % kRtStages
+        uint8_t *st = smem + (i % kRtStages) * kRtStageBytes;
+        const int k0 = (s_begin + i) * kRtBK;
+        mbar_arrive_expect_tx(&full[i % kRtStages], kRtStageBytes);
+        tma_load_2d(st, &tm_w, &full[i % kRtStages], k0, 0, policy_evict_last());
+        tma_load_2d(st + kRtWBytes, &tm_x, &full[i % kRtStages], k0, static_cast<int>(t0), policy_evict_first());
+    };
+    int n_issued = 0;  // meaningful in thread 0
+    if (tid == 0)
+        for (; n_issued < kRtStages && n_issued < n_my; ++n_issued) issue(n_issued);
 
     float acc[8][16];
 #pragma unroll
@@ -112,95 +130,68 @@ __global__ void __cluster_dims__(kRtCluster, 1, 1) __launch_bounds__(kRtThreads,
 #pragma unroll
         for (int j = 0; j < 16; ++j) acc[i][j] = 0.0f;
 
-    // x stage: 64 tokens x 32 k bf16 = 256 chunks of 8 bf16; chunk c = tid + 128*h (h < 2) holds
-    // token c & 63, k-offset (c >> 6) * 8
-    uint4 xreg[2];
-    auto x_load = [&](int s) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int c = tid + kRtThreads * h;
-            const int xt = c & 63, xc = (c >> 6) * 8;
-            const bool ok = (t0 + xt) < p.T;
-            xreg[h] = ok ? __ldg(reinterpret_cast<const uint4 *>(p.x + (t0 + xt) * static_cast<int64_t>(p.H) +
-                                                                 s * kRtBK + xc))
-                         : make_uint4(0u, 0u, 0u, 0u);
-        }
-    };
-    auto x_store = [&](int buf) {
-        float *xsb = xs + buf * kRtBK * kRtTok;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int c = tid + kRtThreads * h;
-            const int xt = c & 63, xc = (c >> 6) * 8;
-            const uint32_t xw[4] = {xreg[h].x, xreg[h].y, xreg[h].z, xreg[h].w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                // bf16 -> fp32 is a 16-bit shift of the bit pattern (exact)
-                xsb[(xc + 2 * i) * kRtTok + xt] = __uint_as_float(xw[i] << 16);
-                xsb[(xc + 2 * i + 1) * kRtTok + xt] = __uint_as_float(xw[i] & 0xffff0000u);
-            }
-        }
-    };
-    // W stage: thread t copies rows t and t+128 (32 floats each) as 8-byte chunks; rows are 34 floats
-    // apart in shared memory, so every destination is 8-byte aligned
-    const bool w_ok0 = tid < p.E, w_ok1 = tid + kRtThreads < p.E;
-    const float *wrow0 = p.w + static_cast<int64_t>(w_ok0 ? tid : 0) * p.H;
-    const float *wrow1 = p.w + static_cast<int64_t>(w_ok1 ? tid + kRtThreads : 0) * p.H;
-    auto w_async = [&](int s, int buf) {
-        float *dst0 = ws + buf * kRtSlots * kRtWPad + tid * kRtWPad;
-        float *dst1 = dst0 + kRtThreads * kRtWPad;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            cp_async8(dst0 + 2 * i, wrow0 + s * kRtBK + 2 * i, w_ok0);
-            cp_async8(dst1 + 2 * i, wrow1 + s * kRtBK + 2 * i, w_ok1);
-        }
-        cp_async_commit();
-    };
-
-    if (s_begin < s_end) {
-        w_async(s_begin, 0);
-        x_load(s_begin);
-        x_store(0);
-        cp_async_wait_all();
-        __syncthreads();
-        for (int s = s_begin; s < s_end; ++s) {
-            const int buf = (s - s_begin) & 1;
-            if (s + 1 < s_end) {
-                w_async(s + 1, buf ^ 1);
-                x_load(s + 1);
-            }
-            const float *wsb = ws + buf * kRtSlots * kRtWPad + exp0 * kRtWPad;
-            const float *xsb = xs + buf * kRtBK * kRtTok + tok0;
+    // Every wait below is taken by all 32 lanes of a warp and its outcome made warp-uniform, so the
+    // warps stay converged; a timeout (status word set) stops the loop.
+    bool ok = true;
+    int i = 0;
+    for (; i < n_my && ok; ++i) {
+        const int st = i % kRtStages;
+        ok = __all_sync(0xffffffffu, mbar_wait(&full[st], (i / kRtStages) & 1u, kDefaultTimeoutCycles));
+        if (!ok) break;
+        const uint8_t *wsb = smem + st * kRtStageBytes;
+        const uint8_t *xsb = wsb + kRtWBytes;
 #pragma unroll 2
-            for (int kp = 0; kp < kRtBK / 2; ++kp) {
-                float2 wv[16];
+        for (int kp = 0; kp < kRtBK / 2; ++kp) {
+            // W row r (r & 7 == b), fp32 k = 2kp, 2kp+1: 16-byte chunk (kp>>1) ^ b of the 128-byte row
+            const int woff = ((((kp >> 1) ^ b) << 4) | ((kp & 1) << 3));
+            float2 wv[16];
 #pragma unroll
-                for (int j = 0; j < 16; ++j)
-                    wv[j] = *reinterpret_cast<const float2 *>(wsb + 8 * j * kRtWPad + 2 * kp);
+            for (int j = 0; j < 16; ++j)
+                wv[j] = *reinterpret_cast<const float2 *>(wsb + (expB + 8 * j) * 128 + woff);
+            // x row t, bf16 pair k = 2kp, 2kp+1: 16-byte chunk (kp>>2) ^ ((t>>1)&3) of the 64-byte row
+            uint32_t xp[8];
 #pragma unroll
-                for (int kk = 0; kk < 2; ++kk) {
-                    const float4 xa = *reinterpret_cast<const float4 *>(xsb + (2 * kp + kk) * kRtTok);
-                    const float4 xb = *reinterpret_cast<const float4 *>(xsb + (2 * kp + kk) * kRtTok + 4);
-                    const float xv[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+            for (int i2 = 0; i2 < 8; ++i2) {
+                const int t = tokA + 4 * i2;
+                xp[i2] = *reinterpret_cast<const uint32_t *>(
+                    xsb + t * 64 + ((((kp >> 2) ^ ((t >> 1) & 3)) << 4) | ((kp & 3) << 2)));
+            }
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const float wj = kk == 0 ? wv[j].x : wv[j].y;
+            for (int kk = 0; kk < 2; ++kk) {
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) acc[i][j] = fmaf(xv[i], wj, acc[i][j]);
+                for (int j = 0; j < 16; ++j) {
+                    const float wj = kk == 0 ? wv[j].x : wv[j].y;
+#pragma unroll
+                    for (int i2 = 0; i2 < 8; ++i2) {
+                        // bf16 -> fp32 is a 16-bit shift of the bit pattern (exact)
+                        const float xv = __uint_as_float(kk == 0 ? (xp[i2] << 16) : (xp[i2] & 0xffff0000u));
+                        acc[i2][j] = fmaf(xv, wj, acc[i2][j]);
                     }
                 }
             }
-            if (s + 1 < s_end) x_store(buf ^ 1);
-            cp_async_wait_all();
-            __syncthreads();
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
+        // warp 0 refills this stage with the step kRtStages ahead once every warp has released it
+        if (warp == 0 && i + kRtStages < n_my) {
+            ok = __all_sync(0xffffffffu, mbar_wait(&empty[st], (i / kRtStages) & 1u, kDefaultTimeoutCycles));
+            if (ok && lane == 0) {
+                issue(i + kRtStages);
+                ++n_issued;
+            }
+            __syncwarp();
         }
     }
+    // after a timeout, let this CTA's in-flight copies land before its shared memory is reused
+    if (tid == 0)
+        for (int q = i; q < n_issued; ++q) mbar_wait(&full[q % kRtStages], (q / kRtStages) & 1u, kDefaultTimeoutCycles);
+    __syncthreads();
 
-    // partial logits -> shared memory (the staging buffers are free after the last barrier)
+    // partial logits -> shared memory
 #pragma unroll
     for (int i = 0; i < 8; ++i)
 #pragma unroll
-        for (int j = 0; j < 16; ++j) part[(tok0 + i) * kRtSlots + exp0 + 8 * j] = acc[i][j];
+        for (int j = 0; j < 16; ++j) part[(tokA + 4 * i) * kRtSlots + expB + 8 * j] = acc[i][j];
     cluster.sync();
 
     // ---- reduction over the cluster + selection: warp w owns tokens 8*rank + w and 8*rank + w + 4
