@@ -1,6 +1,6 @@
 // C ABI of the Beam MoE block forward pass on B200 (sm_100a): argument checks, workspace layout,
 // TMA descriptor encoding and the launch sequence
-//   router_topk -> permute_hist -> permute_scan -> permute_scatter -> gather_rows
+//   router_topk -> permute_hist -> permute_scan -> permute_scatter -> [gather_rows, wide tiles]
 //   -> grouped GEMM (gate/up + SwiGLU) -> grouped GEMM (down) -> combine
 // all enqueued on the caller's stream with no host synchronisation.  The public contract is in
 // include/beam_moe.h.
@@ -27,12 +27,15 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr int64_t kMaxTokens = int64_t(1) << 24;
 
-// ---- GEMM variants: <gate/up?, BN, B box rows, smem stages, TMEM slots, slot columns> ----------
-// "wide": experts see up to ~190 tokens per tile (prefill); "narrow": a few tokens (decode).
-#define G1_WIDE_ARGS true, 192, 64, 4, 2, 256
-#define G2_WIDE_ARGS false, 192, 64, 5, 2, 256
-#define G1_NARROW_ARGS true, 32, 32, 6, 4, 64
-#define G2_NARROW_ARGS false, 32, 32, 10, 4, 32
+// ---- GEMM variants: <gate/up?, BN, B box rows, smem stages, TMEM slots, slot columns, gather?> -----
+// "wide": experts see up to ~190 tokens per tile (prefill): the dispatch also gathers x into
+// dispatch order (x_perm) and both GEMMs read their token rows with tiled 64-row TMA boxes.
+// "narrow": a few tokens per expert (decode): the gate/up GEMM gathers its rows straight from x
+// with TMA gather4 (four rows per instruction; cheap when an expert has a handful of tokens).
+#define G1_WIDE_ARGS true, 192, 64, 4, 2, 256, false
+#define G2_WIDE_ARGS false, 192, 64, 5, 2, 256, false
+#define G1_NARROW_ARGS true, 32, 1, 6, 4, 64, true
+#define G2_NARROW_ARGS false, 32, 32, 10, 4, 32, false
 using G1Wide = GemmCfg<G1_WIDE_ARGS>;
 using G2Wide = GemmCfg<G2_WIDE_ARGS>;
 using G1Narrow = GemmCfg<G1_NARROW_ARGS>;
@@ -42,6 +45,11 @@ using G2Narrow = GemmCfg<G2_NARROW_ARGS>;
 #define G1_NARROW_KERNEL grouped_gemm_kernel<G1_NARROW_ARGS>
 #define G2_NARROW_KERNEL grouped_gemm_kernel<G2_NARROW_ARGS>
 constexpr int kWideBN = 192, kWideBox = 64, kNarrowBN = 32, kNarrowBox = 32;
+
+// Tile family from the mean rows per expert (T*k/E): narrow when experts see a handful of tokens.
+bool narrow_tiles(const beam_moe_config *c, int64_t T) {
+    return static_cast<double>(T) * c->topk / c->n_experts <= 12.0;
+}
 
 struct DeviceInfo {
     std::once_flag once;
@@ -158,7 +166,7 @@ Layout layout(const beam_moe_config *c, int64_t T, int which) {
     L.offsets = take((E + 1) * 8);
     L.row_src = take(R * 4);
     L.dest_row = take(R * 4);
-    L.xp = take(R * H * 2);
+    if (!narrow_tiles(c, T)) L.xp = take(R * H * 2);  // x in dispatch order (wide tiles only)
     L.h = take(R * I * 2);
     L.o = take(R * H * 4);
     L.total = off;
@@ -252,38 +260,40 @@ int enqueue_experts(const beam_moe_config *c, int dev, int64_t T, const beam_bf1
     int32_t *row_src = reinterpret_cast<int32_t *>(ws + L.row_src);
     int32_t *dest_row = reinterpret_cast<int32_t *>(ws + L.dest_row);
     int32_t *hist = reinterpret_cast<int32_t *>(ws + L.hist);
-    void *xp = ws + L.xp;
     void *h = ws + L.h;
     void *o = ws + L.o;
     const int k = c->topk, E = c->n_experts, H = c->hidden, I = c->inter;
     const uint64_t R = static_cast<uint64_t>(T) * k;
+    const bool narrow = narrow_tiles(c, T);
 
     int rc = enqueue_permute(c, T, ids, counts, offsets, row_src, dest_row, hist, s);
     if (rc) return rc;
     if (!record(ev, 2, s)) return BEAM_MOE_ERR_CUDA;
-    gather_rows_kernel<<<static_cast<unsigned>(T), 128, 0, s>>>(reinterpret_cast<const uint4 *>(x), T, k, H / 8,
-                                                                dest_row, reinterpret_cast<uint4 *>(xp));
-    if ((rc = launch_status())) return rc;
+    if (!narrow) {
+        gather_rows_kernel<<<static_cast<unsigned>(T), 128, 0, s>>>(reinterpret_cast<const uint4 *>(x), T, k, H / 8,
+                                                                    dest_row, reinterpret_cast<uint4 *>(ws + L.xp));
+        if ((rc = launch_status())) return rc;
+    }
     if (!record(ev, 3, s)) return BEAM_MOE_ERR_CUDA;
 
-    // Tile choice from the mean rows per expert: narrow tiles when experts see a handful of tokens.
     const double mean_rows = static_cast<double>(R) / E;
-    const bool narrow = mean_rows <= 12.0;
     const int bn = narrow ? kNarrowBN : kWideBN;
     const int box = narrow ? kNarrowBox : kWideBox;
     // Weights are read once per call when (almost) every expert fits one token tile: mark them
     // evict-first so they do not push the reused activations out of L2.
-    const int weights_once = (mean_rows + 5.0 * std::sqrt(mean_rows) <= bn) ? 1 : 0;
-    CUtensorMap m_wg, m_wu, m_xp, m_wd, m_h;
+    const int once = (mean_rows + 4.0 * std::sqrt(mean_rows) <= bn) ? 1 : 0;
+    CUtensorMap m_wg, m_wu, m_b1, m_wd, m_h;
     if (!encode_fn()) return BEAM_MOE_ERR_CUDA;
-    if (!make_map_3d(&m_wg, wg, H, I, E) || !make_map_3d(&m_wu, wu, H, I, E) ||
-        !make_map_2d(&m_xp, xp, H, R, box) || !make_map_3d(&m_wd, wd, I, H, E) || !make_map_2d(&m_h, h, I, R, box))
+    const bool b1_ok = narrow ? make_map_2d(&m_b1, x, H, static_cast<uint64_t>(T), 1)   // gather4 rows of x
+                              : make_map_2d(&m_b1, ws + L.xp, H, R, box);              // tiled x_perm rows
+    if (!b1_ok || !make_map_3d(&m_wg, wg, H, I, E) || !make_map_3d(&m_wu, wu, H, I, E) ||
+        !make_map_3d(&m_wd, wd, I, H, E) || !make_map_2d(&m_h, h, I, R, box))
         return BEAM_MOE_ERR_CUDA;
     const int grid = g_dev[dev].num_sms;
-    GemmParams p1{counts, offsets, h, E, H, I, weights_once, kDefaultTimeoutCycles};
-    GemmParams p2{counts, offsets, o, E, I, H, weights_once, kDefaultTimeoutCycles};
-    if (narrow) G1_NARROW_KERNEL<<<grid, kGemmThreads, G1Narrow::kSmem, s>>>(m_wg, m_wu, m_xp, p1);
-    else G1_WIDE_KERNEL<<<grid, kGemmThreads, G1Wide::kSmem, s>>>(m_wg, m_wu, m_xp, p1);
+    GemmParams p1{counts, offsets, h, E, H, I, once, kDefaultTimeoutCycles, row_src, k};
+    GemmParams p2{counts, offsets, o, E, I, H, once, kDefaultTimeoutCycles, nullptr, k};
+    if (narrow) G1_NARROW_KERNEL<<<grid, kGemmThreads, G1Narrow::kSmem, s>>>(m_wg, m_wu, m_b1, p1);
+    else G1_WIDE_KERNEL<<<grid, kGemmThreads, G1Wide::kSmem, s>>>(m_wg, m_wu, m_b1, p1);
     if ((rc = launch_status())) return rc;
     if (!record(ev, 4, s)) return BEAM_MOE_ERR_CUDA;
     if (narrow) G2_NARROW_KERNEL<<<grid, kGemmThreads, G2Narrow::kSmem, s>>>(m_wd, m_wd, m_h, p2);

@@ -37,7 +37,7 @@ constexpr int kGemmThreads = 256;
 
 constexpr int pow2_cols(int c) { return c <= 32 ? 32 : c <= 64 ? 64 : c <= 128 ? 128 : c <= 256 ? 256 : 512; }
 
-template <bool GATE_UP, int BN, int BOXN, int STAGES, int NSLOT, int SLOT_COLS>
+template <bool GATE_UP, int BN, int BOXN, int STAGES, int NSLOT, int SLOT_COLS, bool GATHER = false>
 struct GemmCfg {
     static constexpr int kA = kBM * kBK * 2;                 // one A tile, bytes
     static constexpr int kB = BN * kBK * 2;                  // B tile, bytes (room for BN rows)
@@ -46,9 +46,11 @@ struct GemmCfg {
     static constexpr int kStage = kNumA * kA + kB;
     static constexpr int kTmemCols = pow2_cols(NSLOT * SLOT_COLS);
     static constexpr int kBarOff = STAGES * kStage;
-    static constexpr int kSmem = 1024 + kBarOff + 256 + 4 * (kPmMaxE + 1) + 64;
-    static_assert(kStage % 1024 == 0 && kBox % 1024 == 0, "tiles must keep 1024-byte alignment");
+    static constexpr int kTokOff = kBarOff + 256 + 4 * (kPmMaxE + 1);     // gathered token ids [BN]
+    static constexpr int kSmem = 1024 + kTokOff + (GATHER ? 4 * BN : 0) + 64;
+    static_assert(kStage % 1024 == 0 && (GATHER || kBox % 1024 == 0), "tiles must keep 1024-byte alignment");
     static_assert(BN % BOXN == 0 && BN % 16 == 0 && BN <= 256, "token tile");
+    static_assert(!GATHER || BOXN == 1, "gathered B rows come one row per box, four per instruction");
     static_assert(NSLOT * SLOT_COLS <= 512, "TMEM has 512 columns");
     static_assert(GATE_UP ? (BN <= SLOT_COLS && (NSLOT >= 2 || BN <= SLOT_COLS / 2)) : BN <= SLOT_COLS,
                   "an item must fit in its TMEM slots");
@@ -64,6 +66,8 @@ struct GemmParams {
     int M;                    // weight rows (G1: I, G2: H)
     int weights_once;         // 1: each weight tile is read once per call -> L2 evict-first
     long long timeout;
+    const int32_t *row_src;   // GATHER: dispatch row -> (token, slot) pair q; token = q / topk
+    int topk;
 };
 
 // Work-item decode from the per-CTA prefix table.
@@ -99,13 +103,14 @@ __device__ __forceinline__ int slots_of(int n_mma) {
     return (GATE_UP && n_mma > SLOT_COLS / 2) ? 2 : 1;
 }
 
-template <bool GATE_UP, int BN, int BOXN, int STAGES, int NSLOT, int SLOT_COLS>
+template <bool GATE_UP, int BN, int BOXN, int STAGES, int NSLOT, int SLOT_COLS, bool GATHER = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a0,  // W_gate (G1) / W_down (G2): [E][M][K]
                         const __grid_constant__ CUtensorMap tm_a1,  // W_up (G1); unused for G2
-                        const __grid_constant__ CUtensorMap tm_b,   // x_perm (G1) / h (G2): [R][K], box BOXN rows
+                        const __grid_constant__ CUtensorMap tm_b,   // B rows [rows][K]: box BOXN rows, or
+                                                                    // GATHER: x [T][K] with a one-row box
                         const GemmParams p) {
-    using C = GemmCfg<GATE_UP, BN, BOXN, STAGES, NSLOT, SLOT_COLS>;
+    using C = GemmCfg<GATE_UP, BN, BOXN, STAGES, NSLOT, SLOT_COLS, GATHER>;
     extern __shared__ uint8_t gemm_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(gemm_smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
@@ -115,6 +120,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     uint64_t *drain = acc_empty + NSLOT;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
     int *tile_start = reinterpret_cast<int *>(smem + C::kBarOff + 256);
+    int *tok = reinterpret_cast<int *>(smem + C::kTokOff);  // GATHER: token of each row of the item
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = p.E;
@@ -165,18 +171,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int total = tile_start[E];
 
     if (warp == 0) {
-        if (lane == 0) {
-            // ---------------- TMA producer ----------------
-            const uint64_t pol_w = p.weights_once ? policy_evict_first() : policy_evict_normal();
-            const uint64_t pol_x = policy_evict_last();  // activations: re-read by the other weight-row tiles
-            int stage = 0;
-            uint32_t phase = 0;
-            uint32_t issued = 0, issued_phase = 0;  // per stage: ever issued / phase of the last issue
-            bool ok = true;
-            for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
-                const Item it = decode_item(item, tile_start, E, BN, p.counts, p.offsets);
-                const int nbox = (it.n_mma + BOXN - 1) / BOXN;
-                const uint32_t bytes = C::kNumA * C::kA + nbox * C::kBox;
+        // ---------------- TMA producer (lane 0 issues; with GATHER the warp first loads the item's token ids)
+        const uint64_t pol_w = p.weights_once ? policy_evict_first() : policy_evict_normal();
+        const uint64_t pol_x = policy_evict_last();  // activations: re-read by the other weight-row tiles
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t issued = 0, issued_phase = 0;  // per stage: ever issued / phase of the last issue
+        bool ok = true;
+        for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+            const Item it = decode_item(item, tile_start, E, BN, p.counts, p.offsets);
+            if (GATHER) {
+                // rows past the expert's tokens (up to the MMA's N) repeat its first token: valid, ignored
+                for (int r = lane; r < it.n_mma; r += 32) {
+                    const int rr = r < it.n_valid ? r : 0;
+                    tok[r] = p.row_src[it.row0 + rr] / p.topk;
+                }
+                __syncwarp();
+            }
+            if (lane == 0) {
+                const int nbox = GATHER ? (it.n_mma + 3) / 4 : (it.n_mma + BOXN - 1) / BOXN;
+                const uint32_t bytes = C::kNumA * C::kA + nbox * (GATHER ? 4 * kBK * 2 : C::kBox);
                 for (int kb = 0; kb < n_kb; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, p.timeout)) {
                         ok = false;
@@ -187,9 +201,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     tma_load_3d(sa, &tm_a0, &full[stage], kb * kBK, it.mt * kBM, it.e, pol_w);
                     if (GATE_UP) tma_load_3d(sa + C::kA, &tm_a1, &full[stage], kb * kBK, it.mt * kBM, it.e, pol_w);
                     uint8_t *sb = sa + C::kNumA * C::kA;
-                    for (int b = 0; b < nbox; ++b)
-                        tma_load_2d(sb + b * C::kBox, &tm_b, &full[stage], kb * kBK,
-                                    static_cast<int>(it.row0) + b * BOXN, pol_x);
+                    if (GATHER) {
+                        for (int g = 0; g < nbox; ++g)  // rows 4g..4g+3 land 128 B apart, as a tiled box would
+                            tma_gather4(sb + g * 4 * kBK * 2, &tm_b, &full[stage], kb * kBK, tok[4 * g],
+                                        tok[4 * g + 1], tok[4 * g + 2], tok[4 * g + 3], pol_x);
+                    } else {
+                        for (int b = 0; b < nbox; ++b)
+                            tma_load_2d(sb + b * C::kBox, &tm_b, &full[stage], kb * kBK,
+                                        static_cast<int>(it.row0) + b * BOXN, pol_x);
+                    }
                     issued |= 1u << stage;
                     issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
                     if (++stage == STAGES) {
@@ -198,10 +218,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                 }
             }
-            // every load this thread issued has landed before the CTA may exit
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            stage = __shfl_sync(0xffffffffu, stage, 0);
+            phase = __shfl_sync(0xffffffffu, phase, 0);
+        }
+        // every load this thread issued has landed before the CTA may exit
+        if (lane == 0)
             for (int s = 0; s < STAGES; ++s)
                 if ((issued >> s) & 1u) mbar_wait(&full[s], (issued_phase >> s) & 1u, p.timeout);
-        }
     } else if (warp == 1) {
         if (lane == 0) {
             // ---------------- MMA issuer ----------------

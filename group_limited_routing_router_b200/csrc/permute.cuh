@@ -1,5 +1,5 @@
-// Dispatch kernels P: stable grouping of the T*k routed (token, slot) pairs by expert, plus the
-// row gather of x into that order.
+// Dispatch kernels P: stable grouping of the T*k routed (token, slot) pairs by expert, and the row
+// gather of x into that order for the wide-tile gate/up GEMM.
 //
 // The pages only say that each token runs on its 8 experts; this is the library's deterministic
 // convention: rows sorted by (expert ascending, token ascending).  Three launches:
@@ -129,7 +129,8 @@ __global__ void __launch_bounds__(kPmThreads) permute_scatter_kernel(const int32
     }
 }
 
-// x_perm[dest_row[t*k + j]] = x[t] for every slot j: each token row is read once and written k times.
+// x_perm[dest_row[t*k + j]] = x[t] for every slot j: each token row is read once and written k times
+// (the wide-tile gate/up GEMM reads its token rows from x_perm with tiled TMA boxes).
 __global__ void __launch_bounds__(128) gather_rows_kernel(const uint4 *__restrict__ x, int64_t T, int k, int nvec,
                                                             const int32_t *__restrict__ dest_row,
                                                             uint4 *__restrict__ xp) {

@@ -42,10 +42,10 @@ def test_workspace_sizes(L):
     assert bm.workspace_size(c, 0, bm.WS_ROUTE) == 0
     f = [bm.workspace_size(c, T, bm.WS_FORWARD) for T in (1, 256, 4096, 65536)]
     assert all(b > a for a, b in zip(f, f[1:]))
-    # forward holds x_perm (bf16), h (bf16) and the fp32 expert outputs for all T*k rows
+    # forward holds h (bf16) and the fp32 expert outputs for all T*k rows
     T = 4096
     R = T * 8
-    assert f[2] >= R * 5120 * 2 + R * 2560 * 2 + R * 5120 * 4
+    assert f[2] >= R * 2560 * 2 + R * 5120 * 4
     assert bm.workspace_size(c, T, bm.WS_EXPERTS) < f[2]
     assert bm.workspace_size(c, T, bm.WS_PERMUTE) >= 16 * 256 * 4
     assert bm.workspace_size(c, -1, bm.WS_FORWARD) == 0
