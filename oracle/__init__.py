@@ -14,6 +14,9 @@ section "Mixture of Experts"):
   combine        - routed_scale * sum_j w_j * expert_j(x)
   forward        - the whole block on host tensors
   forward_tokens - the whole block for a subset of tokens, fetching one expert's weights at a time
+  rmsnorm        - the sublayer norm (section "Residual Stream": normalised before and after)
+  scaled_residual- stream update sqrt((k-1)/k) * stream + z / sqrt(k) (same section)
+  block_forward  - pre-norm -> block -> post-norm -> scaled residual
 """
 from __future__ import annotations
 
@@ -51,6 +54,10 @@ def lib():
         L.oracle_expert_mlp.restype = None
         L.oracle_combine.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_double, _dp, _dp, _dp]
         L.oracle_combine.restype = None
+        L.oracle_rmsnorm.argtypes = [ctypes.c_int64, ctypes.c_int, _dp, _dp, ctypes.c_double, _dp]
+        L.oracle_rmsnorm.restype = None
+        L.oracle_scaled_residual.argtypes = [ctypes.c_int64, ctypes.c_int, _dp, _dp, ctypes.c_int, _dp]
+        L.oracle_scaled_residual.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -192,3 +199,53 @@ def forward(x_bits: np.ndarray, w_router: np.ndarray, bias: Optional[np.ndarray]
     y = experts_tokens(np.ascontiguousarray(x_bits[tok]), r["ids"][tok], r["weight"][tok], fetch,
                        layer["n_experts"], layer["routed_scale"])
     return dict(route=r, tokens=tok, y=y)
+
+
+def rmsnorm(x: np.ndarray, g: np.ndarray, eps: float) -> np.ndarray:
+    """RMSNorm over the last axis in FP64: x / sqrt(mean(x^2) + eps) * g."""
+    x = np.ascontiguousarray(x, dtype=np.float64)
+    T, H = x.shape
+    g = np.ascontiguousarray(g, dtype=np.float64)
+    assert g.shape == (H,)
+    out = np.empty_like(x)
+    lib().oracle_rmsnorm(T, H, _ptr(x, _dp), _ptr(g, _dp), float(eps), _ptr(out, _dp))
+    return out
+
+
+def scaled_residual(stream: np.ndarray, z: np.ndarray, step: int) -> np.ndarray:
+    """sqrt((k-1)/k) * stream + z / sqrt(k) for residual step k >= 2 (the embedding is step 1)."""
+    stream = np.ascontiguousarray(stream, dtype=np.float64)
+    z = np.ascontiguousarray(z, dtype=np.float64)
+    assert stream.shape == z.shape
+    T, H = stream.shape
+    out = np.empty_like(stream)
+    if lib().oracle_scaled_residual(T, H, _ptr(stream, _dp), _ptr(z, _dp), int(step), _ptr(out, _dp)) != 0:
+        raise ValueError("residual step must be >= 2")
+    return out
+
+
+def f64_to_bf16_bits(v: np.ndarray) -> np.ndarray:
+    """Round FP64 values to bf16 directly (8 significant bits, ties to even) and return the bit patterns."""
+    v = np.asarray(v, dtype=np.float64)
+    m, e = np.frexp(v)                              # v = m * 2^e, 0.5 <= |m| < 1
+    r = np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)    # np.rint rounds half to even
+    f = r.astype(np.float32)                        # exact: r has at most 8 significant bits
+    return np.ascontiguousarray((f.view(np.uint32) >> 16).astype(np.uint16))
+
+
+def block_forward(stream_bits: np.ndarray, g_pre: np.ndarray, g_post: np.ndarray, eps: float, step: int,
+                  w_router: np.ndarray, bias, fetch: ExpertFetch, layer: dict, tokens=None):
+    """The MoE sublayer with its norms and residual update.
+
+    u = bf16(RMSNorm(stream) * g_pre)      (the block's bf16 input activation)
+    y = MoE block of u                     (routing on all tokens, experts on `tokens`)
+    out = sqrt((k-1)/k) * stream + RMSNorm(y) * g_post / sqrt(k)
+    Returns dict(u_bits, route, tokens, y, out) with out in FP64 for the chosen tokens.
+    """
+    s64 = bf16_bits_to_f64(stream_bits)
+    u_bits = f64_to_bf16_bits(rmsnorm(s64, g_pre, eps))
+    f = forward(u_bits, w_router, bias, fetch, layer, tokens)
+    tok = f["tokens"]
+    z = rmsnorm(f["y"], g_post, eps)
+    out = scaled_residual(s64[tok], z, step)
+    return dict(u_bits=u_bits, route=f["route"], tokens=tok, y=f["y"], out=out)

@@ -290,3 +290,35 @@ void oracle_combine(int64_t T, int topk, int H, double routed_scale, const doubl
             y[t * H + h] = routed_scale * acc;
         }
 }
+
+/*
+ * Sublayer normalisation ("Welcome Beam" page, section "Residual Stream": every sublayer is
+ * normalised before and after; the norms compute in FP32 on the model, here FP64).  Reading: RMSNorm
+ * with a learned per-channel scale,
+ *   out[t,h] = x[t,h] / sqrt(mean_h x[t,h]^2 + eps) * g[h].
+ * x, out [T,H] fp64; g [H] fp64.
+ */
+void oracle_rmsnorm(int64_t T, int H, const double *x, const double *g, double eps, double *out)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        double ss = 0.0;
+        for (int h = 0; h < H; ++h) ss += x[t * H + h] * x[t * H + h];
+        const double inv = 1.0 / sqrt(ss / H + eps);
+        for (int h = 0; h < H; ++h) out[t * H + h] = x[t * H + h] * inv * g[h];
+    }
+}
+
+/*
+ * Scaled residual update (same section): the input embedding is step 1; at step k the sublayer
+ * output z is added with weight 1/sqrt(k) and the stream kept with weight sqrt((k-1)/k).
+ *   out = sqrt((k-1)/k) * stream + z / sqrt(k).
+ * Returns -1 for k < 2.
+ */
+int oracle_scaled_residual(int64_t T, int H, const double *stream, const double *z, int k, double *out)
+{
+    if (k < 2) return -1;
+    const double keep = sqrt((double)(k - 1) / (double)k), add = 1.0 / sqrt((double)k);
+    for (int64_t q = 0; q < T * (int64_t)H; ++q) out[q] = keep * stream[q] + add * z[q];
+    return 0;
+}

@@ -13,6 +13,7 @@ import subprocess
 import pytest
 
 import oracle
+from tests import test_oracle_norm_residual as nr
 from tests import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "beam_oracle.c")
@@ -34,6 +35,14 @@ MUTANTS = {
                                   "for (int64_t q = n - 1; q >= 0; --q)\n            if (ids[q] == e) {"),
     "offsets_inclusive": ("offsets[e + 1] = offsets[e] + counts[e];",
                           "offsets[e + 1] = offsets[e] + counts[e] + (e == 0);"),
+    "rmsnorm_sum_not_mean": ("const double inv = 1.0 / sqrt(ss / H + eps);",
+                             "const double inv = 1.0 / sqrt(ss + eps);"),
+    "rmsnorm_eps_outside_sqrt": ("const double inv = 1.0 / sqrt(ss / H + eps);",
+                                 "const double inv = 1.0 / (sqrt(ss / H) + eps);"),
+    "residual_weights_swapped": ("keep = sqrt((double)(k - 1) / (double)k), add = 1.0 / sqrt((double)k);",
+                                 "add = sqrt((double)(k - 1) / (double)k), keep = 1.0 / sqrt((double)k);"),
+    "residual_step_off_by_one": ("keep = sqrt((double)(k - 1) / (double)k), add = 1.0 / sqrt((double)k);",
+                                 "keep = sqrt((double)k / (double)(k + 1)), add = 1.0 / sqrt((double)(k + 1));"),
 }
 
 PINS = [
@@ -46,6 +55,10 @@ PINS = [
     pins.test_k1_is_scaled_single_expert,
     pins.test_forward_matches_torch_float64_composition,
     pins.test_permute_matches_stable_argsort,
+    nr.test_rmsnorm_matches_torch_float64,
+    nr.test_rmsnorm_closed_forms,
+    nr.test_residual_weights_are_unit_norm,
+    nr.test_every_addition_carries_equal_weight_after_104_steps,
 ]
 
 
