@@ -34,13 +34,18 @@ ERR_DEVICE_TIMEOUT = 7
 ERR_BAD_INDEX = 8
 ERR_INVALID_ARG = 9
 
-WS_ROUTE, WS_PERMUTE, WS_EXPERTS, WS_FORWARD = 0, 1, 2, 3
+WS_ROUTE, WS_PERMUTE, WS_EXPERTS, WS_FORWARD, WS_BLOCK = 0, 1, 2, 3, 4
 
 
 class BeamMoeConfig(ctypes.Structure):
     _fields_ = [("hidden", ctypes.c_int32), ("inter", ctypes.c_int32), ("n_experts", ctypes.c_int32),
                 ("n_groups", ctypes.c_int32), ("topk_groups", ctypes.c_int32), ("topk", ctypes.c_int32),
                 ("group_topn", ctypes.c_int32), ("routed_scale", ctypes.c_float)]
+
+
+class BeamMoeSublayer(ctypes.Structure):
+    _fields_ = [("pre_norm_weight", ctypes.c_void_p), ("post_norm_weight", ctypes.c_void_p),
+                ("eps", ctypes.c_float), ("step", ctypes.c_int32)]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -91,12 +96,15 @@ def lib() -> ctypes.CDLL:
                                        ctypes.c_size_t, _vp]
         L.beam_moe_forward_profiled.argtypes = [_cfgp, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                                 _vp, ctypes.c_size_t, _vp, ctypes.POINTER(ctypes.c_void_p)]
+        L.beam_moe_block_forward.argtypes = [_cfgp, ctypes.POINTER(BeamMoeSublayer), ctypes.c_int64, _vp, _vp, _vp,
+                                             _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
         L.beam_moe_device_status.argtypes = [_vp]
         L.beam_moe_selftest_timeout.argtypes = [ctypes.c_int64, _vp]
         L.beam_moe_strerror.argtypes = [ctypes.c_int]
         L.beam_moe_strerror.restype = ctypes.c_char_p
         for name in ("beam_moe_route", "beam_moe_permute", "beam_moe_experts", "beam_moe_forward",
-                     "beam_moe_forward_profiled", "beam_moe_device_status", "beam_moe_selftest_timeout"):
+                     "beam_moe_forward_profiled", "beam_moe_block_forward", "beam_moe_device_status",
+                     "beam_moe_selftest_timeout"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -237,6 +245,36 @@ def forward(cfg, x, w_router, bias, w_gate, w_up, w_down, y=None, ids=None, w=No
                                   _ptr(w_up), _ptr(w_down), _ptr(y), _ptr(ids), _ptr(w), _ptr(ws), nbytes,
                                   _stream(stream)), "beam_moe_forward")
     return (y, ids, w) if return_routing else y
+
+
+def block_forward(cfg, stream_in, pre_norm_weight, post_norm_weight, eps: float, step: int, w_router, bias,
+                  w_gate, w_up, w_down, stream_out=None, u=None, ids=None, w=None, ws=None, stream=None):
+    """One MoE sublayer on the residual stream (pre-norm, block, post-norm, scaled residual).
+
+    Returns stream_out [T,H] bf16 (pass stream_out=stream_in to update in place); `u`, `ids`, `w`,
+    when given, receive the pre-norm activation and the routing."""
+    c = _cfg(cfg)
+    T = stream_in.shape[0]
+    _dev(stream_in, "stream_in", torch.bfloat16, (T, c.hidden))
+    _dev(pre_norm_weight, "pre_norm_weight", torch.float32, (c.hidden,))
+    _dev(post_norm_weight, "post_norm_weight", torch.float32, (c.hidden,))
+    _dev(w_router, "w_router", torch.float32, (c.n_experts, c.hidden))
+    _dev(bias, "bias", torch.float32, (c.n_experts,))
+    _dev(w_gate, "w_gate", torch.bfloat16, (c.n_experts, c.inter, c.hidden))
+    _dev(w_up, "w_up", torch.bfloat16, (c.n_experts, c.inter, c.hidden))
+    _dev(w_down, "w_down", torch.bfloat16, (c.n_experts, c.hidden, c.inter))
+    stream_out = torch.empty_like(stream_in) if stream_out is None else stream_out
+    _dev(stream_out, "stream_out", torch.bfloat16, (T, c.hidden))
+    _dev(u, "u", torch.bfloat16, (T, c.hidden))
+    _dev(ids, "ids", torch.int32, (T, c.topk))
+    _dev(w, "w", torch.float32, (T, c.topk))
+    ws, nbytes = _workspace(c, T, WS_BLOCK, ws, stream_in.device)
+    sub = BeamMoeSublayer(pre_norm_weight.data_ptr(), post_norm_weight.data_ptr(), float(eps), int(step))
+    _check(lib().beam_moe_block_forward(ctypes.byref(c), ctypes.byref(sub), T, _ptr(stream_in), _ptr(w_router),
+                                        _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(stream_out),
+                                        _ptr(u), _ptr(ids), _ptr(w), _ptr(ws), nbytes, _stream(stream)),
+           "beam_moe_block_forward")
+    return stream_out
 
 
 STAGES = ("router", "dispatch", "gather", "gate_up_swiglu", "down", "combine")

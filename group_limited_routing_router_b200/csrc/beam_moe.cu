@@ -19,12 +19,14 @@
 #include "combine.cuh"
 #include "permute.cuh"
 #include "gemm.cuh"
+#include "norm.cuh"
 #include "router.cuh"
 
 namespace beam {
 namespace {
 
 constexpr int kMaxDevices = 64;
+constexpr int kMaxBlockHidden = 32768;  // the block's FP32 output row stays in shared memory
 constexpr int64_t kMaxTokens = int64_t(1) << 24;
 
 // ---- GEMM variants: <gate/up?, BN, B box rows, smem stages, TMEM slots, slot columns, gather?> -----
@@ -93,6 +95,8 @@ int init_device(int *dev_out) {
                                         G1Narrow::kSmem) == cudaSuccess;
         ok = ok && cudaFuncSetAttribute(G2_NARROW_KERNEL, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         G2Narrow::kSmem) == cudaSuccess;
+        ok = ok && cudaFuncSetAttribute(combine_norm_residual_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        kMaxBlockHidden * 4) == cudaSuccess;
         if (!ok) d.status = BEAM_MOE_ERR_CUDA;
     });
     *dev_out = dev;
@@ -136,7 +140,7 @@ int check_T(const beam_moe_config *c, int64_t T) {
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 struct Layout {
-    size_t ids = 0, w = 0, hist = 0, counts = 0, offsets = 0, row_src = 0, dest_row = 0, xp = 0, h = 0, o = 0;
+    size_t u = 0, ids = 0, w = 0, hist = 0, counts = 0, offsets = 0, row_src = 0, dest_row = 0, xp = 0, h = 0, o = 0;
     size_t total = 0;
 };
 
@@ -153,7 +157,8 @@ Layout layout(const beam_moe_config *c, int64_t T, int which) {
     const size_t R = static_cast<size_t>(T) * c->topk;
     const size_t E = c->n_experts, H = c->hidden, I = c->inter;
     if (which == BEAM_MOE_WS_ROUTE || T == 0) return L;
-    if (which == BEAM_MOE_WS_FORWARD) {
+    if (which == BEAM_MOE_WS_BLOCK) L.u = take(static_cast<size_t>(T) * H * 2);
+    if (which == BEAM_MOE_WS_FORWARD || which == BEAM_MOE_WS_BLOCK) {
         L.ids = take(R * 4);
         L.w = take(R * 4);
     }
@@ -252,9 +257,17 @@ bool record(cudaEvent_t const *events, int i, cudaStream_t s) {
     return !events || cudaEventRecord(events[i], s) == cudaSuccess;
 }
 
+// The block's last step when it runs on the residual stream: post-norm and scaled residual update.
+struct BlockTail {
+    const beam_bf16 *stream_in;
+    const float *g_post;
+    float eps, keep, add;
+};
+
 int enqueue_experts(const beam_moe_config *c, int dev, int64_t T, const beam_bf16 *x, const int32_t *ids,
                     const float *w, const beam_bf16 *wg, const beam_bf16 *wu, const beam_bf16 *wd, beam_bf16 *y,
-                    uint8_t *ws, const Layout &L, cudaStream_t s, cudaEvent_t const *ev = nullptr) {
+                    uint8_t *ws, const Layout &L, cudaStream_t s, cudaEvent_t const *ev = nullptr,
+                    const BlockTail *tail = nullptr) {
     int32_t *counts = reinterpret_cast<int32_t *>(ws + L.counts);
     int64_t *offsets = reinterpret_cast<int64_t *>(ws + L.offsets);
     int32_t *row_src = reinterpret_cast<int32_t *>(ws + L.row_src);
@@ -300,8 +313,14 @@ int enqueue_experts(const beam_moe_config *c, int dev, int64_t T, const beam_bf1
     else G2_WIDE_KERNEL<<<grid, kGemmThreads, G2Wide::kSmem, s>>>(m_wd, m_wd, m_h, p2);
     if ((rc = launch_status())) return rc;
     if (!record(ev, 5, s)) return BEAM_MOE_ERR_CUDA;
-    combine_kernel<<<static_cast<unsigned>(T), 256, 0, s>>>(reinterpret_cast<const float4 *>(o), dest_row, w, T, k,
-                                                            H / 4, c->routed_scale, reinterpret_cast<uint2 *>(y));
+    if (tail)
+        combine_norm_residual_kernel<<<static_cast<unsigned>(T), kNormThreads, H * 4, s>>>(
+            reinterpret_cast<const float4 *>(o), dest_row, w, k, H, c->routed_scale,
+            reinterpret_cast<const uint2 *>(tail->stream_in), tail->g_post, tail->eps, tail->keep, tail->add,
+            reinterpret_cast<uint2 *>(y));
+    else
+        combine_kernel<<<static_cast<unsigned>(T), 256, 0, s>>>(reinterpret_cast<const float4 *>(o), dest_row, w, T,
+                                                                k, H / 4, c->routed_scale, reinterpret_cast<uint2 *>(y));
     if ((rc = launch_status())) return rc;
     if (!record(ev, 6, s)) return BEAM_MOE_ERR_CUDA;
     return BEAM_MOE_OK;
@@ -325,7 +344,7 @@ extern "C" {
 
 size_t beam_moe_workspace_size(const beam_moe_config *cfg, int64_t T, int which) {
     if (validate(cfg) || check_T(cfg, T)) return 0;
-    if (which < BEAM_MOE_WS_ROUTE || which > BEAM_MOE_WS_FORWARD) return 0;
+    if (which < BEAM_MOE_WS_ROUTE || which > BEAM_MOE_WS_BLOCK) return 0;
     return layout(cfg, T, which).total;
 }
 
@@ -475,6 +494,47 @@ const char *beam_moe_strerror(int code) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------------
+// beam_moe_block_forward: pre-norm -> block -> post-norm -> scaled residual update.
+extern "C" int beam_moe_block_forward(const beam_moe_config *cfg, const beam_moe_sublayer *sub, int64_t T,
+                                      const beam_bf16 *stream_in, const float *w_router, const float *sel_bias,
+                                      const beam_bf16 *w_gate, const beam_bf16 *w_up, const beam_bf16 *w_down,
+                                      beam_bf16 *stream_out, beam_bf16 *u_out, int32_t *topk_ids_out,
+                                      float *topk_w_out, void *ws, size_t ws_bytes, void *stream) {
+    int rc = validate(cfg);
+    if (rc) return rc;
+    if (!sub) return BEAM_MOE_ERR_NULL;
+    if (cfg->hidden > kMaxBlockHidden || sub->step < 2 || !(sub->eps >= 0.0f) || !(sub->eps < INFINITY))
+        return BEAM_MOE_ERR_INVALID_CONFIG;
+    if ((rc = check_T(cfg, T))) return rc;
+    if (T == 0) return BEAM_MOE_OK;
+    if (!stream_in || !w_router || !w_gate || !w_up || !w_down || !stream_out || !ws || !sub->pre_norm_weight ||
+        !sub->post_norm_weight)
+        return BEAM_MOE_ERR_NULL;
+    if (!aligned16(stream_in) || !aligned16(w_router) || !aligned16(w_gate) || !aligned16(w_up) ||
+        !aligned16(w_down) || !aligned16(stream_out) || !aligned16(ws) || (u_out && !aligned16(u_out)) ||
+        !aligned16(sub->pre_norm_weight) || !aligned16(sub->post_norm_weight))
+        return BEAM_MOE_ERR_MISALIGNED;
+    const Layout L = layout(cfg, T, BEAM_MOE_WS_BLOCK);
+    if (ws_bytes < L.total) return BEAM_MOE_ERR_WORKSPACE_TOO_SMALL;
+    int dev;
+    if ((rc = init_device(&dev))) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+    beam_bf16 *u = u_out ? u_out : reinterpret_cast<beam_bf16 *>(wsb + L.u);
+    int32_t *ids = topk_ids_out ? topk_ids_out : reinterpret_cast<int32_t *>(wsb + L.ids);
+    float *w = topk_w_out ? topk_w_out : reinterpret_cast<float *>(wsb + L.w);
+    rmsnorm_bf16_kernel<<<static_cast<unsigned>(T), kNormThreads, 0, s>>>(
+        reinterpret_cast<const uint4 *>(stream_in), sub->pre_norm_weight, sub->eps, cfg->hidden,
+        reinterpret_cast<uint4 *>(u));
+    if ((rc = launch_status())) return rc;
+    if ((rc = enqueue_route(cfg, T, u, w_router, sel_bias, ids, w, s))) return rc;
+    const double k = sub->step;
+    const BlockTail tail{stream_in, sub->post_norm_weight, sub->eps, static_cast<float>(std::sqrt((k - 1.0) / k)),
+                         static_cast<float>(1.0 / std::sqrt(k))};
+    return enqueue_experts(cfg, dev, T, u, ids, w, w_gate, w_up, w_down, stream_out, wsb, L, s, nullptr, &tail);
+}
 
 // ------------------------------------------------------------------------------------------------
 // beam_moe_permute_noalloc: the dispatch with its scratch in a fixed device array instead of a

@@ -79,8 +79,23 @@ enum {
     BEAM_MOE_WS_ROUTE = 0,
     BEAM_MOE_WS_PERMUTE = 1,
     BEAM_MOE_WS_EXPERTS = 2,
-    BEAM_MOE_WS_FORWARD = 3
+    BEAM_MOE_WS_FORWARD = 3,
+    BEAM_MOE_WS_BLOCK = 4
 };
+
+/*
+ * The residual-stream wrapping of the block ("Welcome Beam" page, section "Residual Stream": every
+ * sublayer is normalised before and after; the embedding is step 1 and step k adds the sublayer
+ * output with weight 1/sqrt(k) while the stream keeps weight sqrt((k-1)/k); the norms compute in
+ * FP32).  Reading: RMSNorm, x / sqrt(mean(x^2) + eps) * weight.  Beam's MoE sublayer of layer l
+ * (0-based; layers 3..51 are MoE) is step k = 2l + 3.
+ */
+typedef struct beam_moe_sublayer {
+    const float *pre_norm_weight;   /* [H] fp32, device, 16-byte aligned: scale of the norm before the block */
+    const float *post_norm_weight;  /* [H] fp32, device, 16-byte aligned: scale of the norm after the block */
+    float eps;                      /* RMSNorm epsilon, >= 0 */
+    int32_t step;                   /* k >= 2 */
+} beam_moe_sublayer;
 
 /*
  * Bytes of workspace the call `which` needs for T tokens (0 for ROUTE).  Pure host arithmetic:
@@ -138,6 +153,21 @@ BEAM_MOE_API int beam_moe_forward(const beam_moe_config *cfg, int64_t T, const b
                      const float *sel_bias, const beam_bf16 *w_gate, const beam_bf16 *w_up,
                      const beam_bf16 *w_down, beam_bf16 *y, int32_t *topk_ids_out, float *topk_w_out,
                      void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * One MoE sublayer on the residual stream:
+ *   u          = bf16(RMSNorm(stream_in) * pre_norm_weight)        (FP32 arithmetic)
+ *   y          = the block of beam_moe_forward applied to u       (FP32, not rounded)
+ *   stream_out = bf16(sqrt((k-1)/k) * stream_in + RMSNorm(y) * post_norm_weight / sqrt(k))
+ *   stream_in, stream_out [T, H] bf16 (may be the same buffer); u_out [T, H] bf16 or NULL (then u
+ *   stays in the workspace); routing outputs as for beam_moe_forward.  Needs H <= 32768 and a
+ *   workspace of beam_moe_workspace_size(cfg, T, BEAM_MOE_WS_BLOCK) bytes.
+ */
+BEAM_MOE_API int beam_moe_block_forward(const beam_moe_config *cfg, const beam_moe_sublayer *sub, int64_t T,
+                                        const beam_bf16 *stream_in, const float *w_router, const float *sel_bias,
+                                        const beam_bf16 *w_gate, const beam_bf16 *w_up, const beam_bf16 *w_down,
+                                        beam_bf16 *stream_out, beam_bf16 *u_out, int32_t *topk_ids_out,
+                                        float *topk_w_out, void *ws, size_t ws_bytes, void *stream);
 
 /*
  * beam_moe_forward that also records caller-created CUDA events (cudaEvent_t) on `stream` around

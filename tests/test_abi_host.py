@@ -98,3 +98,16 @@ def test_binding_refuses_cpu_tensors(L):
     x = torch.zeros(4, 5120, dtype=torch.bfloat16)
     with pytest.raises(TypeError):
         bm.route(bm.BEAM_LAYER, x, torch.zeros(256, 5120))
+
+
+def test_block_rejects_bad_sublayer_on_host(L):
+    c = _cfg()
+    p = ctypes.c_void_p(4096)
+    for step, eps, hidden in ((1, 1e-6, 5120), (7, -1.0, 5120), (7, float("nan"), 5120), (7, 1e-6, 65536)):
+        cc = _cfg(hidden=hidden)
+        sub = bm.BeamMoeSublayer(4096, 4096, eps, step)
+        assert L.beam_moe_block_forward(ctypes.byref(cc), ctypes.byref(sub), 4, p, p, None, p, p, p, p, None, None,
+                                        None, p, 1 << 40, None) == bm.ERR_INVALID_CONFIG
+    assert L.beam_moe_block_forward(ctypes.byref(c), None, 4, p, p, None, p, p, p, p, None, None, None, p, 1 << 40,
+                                    None) == bm.ERR_NULL
+    assert bm.workspace_size(c, 4096, bm.WS_BLOCK) == bm.workspace_size(c, 4096, bm.WS_FORWARD) + 4096 * 5120 * 2
