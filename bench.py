@@ -64,6 +64,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-sample", type=int, default=96, help="tokens in the CPU-oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--block", action="store_true",
+                    help="time the MoE sublayer on the residual stream (pre-norm, block, post-norm, residual)")
     return ap.parse_args()
 
 
@@ -237,6 +239,13 @@ def config_dict(wl):
             "parallelism": "replicas (one independent layer instance per GPU)"}
 
 
+def launches_per_step(wl: bs.Workload, block: bool) -> int:
+    """Kernels one forward launches: router, 3 dispatch kernels, [row gather for wide tiles], gate/up,
+    down, combine; the sublayer adds the pre-norm (its combine is the fused post-norm kernel)."""
+    wide = wl.T * wl.topk / wl.n_experts > 12.0
+    return 7 + (1 if wide else 0) + (1 if block else 0)
+
+
 class Ranks:
     """One process per GPU: barrier, max-over-ranks and the whole-job rate of independent replicas.
 
@@ -310,8 +319,18 @@ def run_ours(args):
     w = torch.empty(T, wl.topk, dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
 
-    def step():
-        bm.forward(layer, x, W, bias, wg, wu, wd, y=y, ids=ids, w=w, ws=ws)
+    if args.block:
+        g_pre = torch.ones(H, dtype=torch.float32, device="cuda")
+        g_post = torch.ones(H, dtype=torch.float32, device="cuda")
+        ws_blk = torch.empty(bm.workspace_size(layer, T, bm.WS_BLOCK), dtype=torch.uint8, device="cuda")
+        block_step = 2 * 3 + 3  # the MoE sublayer of the first MoE layer (layer 3)
+
+        def step():
+            bm.block_forward(layer, x, g_pre, g_post, 1e-6, block_step, W, bias, wg, wu, wd, stream_out=y, ids=ids,
+                             w=w, ws=ws_blk)
+    else:
+        def step():
+            bm.forward(layer, x, W, bias, wg, wu, wd, y=y, ids=ids, w=w, ws=ws)
 
     clocks = ClockSampler(local)
     clocks.start()
@@ -398,7 +417,10 @@ def run_ours(args):
             "roofline": roofline, "layer_roofline": layer_roof, "stage_ms": stage_ms, "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2,
                     "d2h_bytes_per_step": T * H * 2},
-            "clocks": clk, "gpu_launches": 8 * args.steps, "kernel_source": src_hash}
+            "clocks": clk, "gpu_launches": launches_per_step(wl, args.block) * args.steps, "kernel_source": src_hash}
+    if args.block:
+        line["config"]["block"] = ("sublayer step: RMSNorm pre-norm + MoE block + fused post-norm and scaled residual "
+                                   "(step k=9); stage_ms/roofline are from the plain block's profiled launches")
     if rank == 0:
         print(json.dumps(line))
     ranks.close()
