@@ -115,9 +115,23 @@ PARITY_CASES = {
 }
 
 
+# Dense SwiGLU MLP of Beam's first three layers.  The intermediate size is not on the pages; this
+# build reads it as 20,480 (= 8 x 2,560, the MoE's active width), which also makes the page's
+# "8B" non-expert parameters add up (tests/test_closed_forms.py).
+DENSE = {
+    "dense_prefill": Workload("dense_prefill", T=4096, hidden=5120, inter=20480, n_experts=1, n_groups=1,
+                              topk_groups=1, topk=1, seed=3001, expert_device="cuda",
+                              description="dense SwiGLU, T=4096, hidden 5120, intermediate 20480"),
+    "dense_mid": Workload("dense_mid", T=300, hidden=512, inter=1024, n_experts=1, n_groups=1, topk_groups=1,
+                          topk=1, seed=3002, description="dense SwiGLU, ragged T, several tiles"),
+}
+
+
 def get(name: str) -> Workload:
     if name in WORKLOADS:
         return WORKLOADS[name]
+    if name in DENSE:
+        return DENSE[name]
     return PARITY_CASES[name]
 
 

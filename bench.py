@@ -40,10 +40,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # captured from hash the same; otherwise the JSON line reports null.
 _CSRC = os.path.join(ROOT, "group_limited_routing_router_b200", "csrc")
 NCU_TRAFFIC = {
-    ("gate_up_swiglu", "prefill"): {"bytes": 14.08e9 + 150.18e6, "files": ("gemm.cuh", "common.cuh"),
-                                    "hash": "2fcce525491947f0"},
-    ("down", "prefill"): {"bytes": 7.05e9 + 619.80e6, "files": ("gemm.cuh", "common.cuh"),
-                          "hash": "2fcce525491947f0"},
+    ("gate_up_swiglu", "prefill"): {"bytes": 14.14e9 + 151.86e6, "files": ("gemm.cuh", "common.cuh"),
+                                    "hash": "77aa225963823e2f"},
+    ("down", "prefill"): {"bytes": 7.06e9 + 620.98e6, "files": ("gemm.cuh", "common.cuh"),
+                          "hash": "77aa225963823e2f"},
 }
 
 
@@ -64,6 +64,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-sample", type=int, default=96, help="tokens in the CPU-oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--dense", action="store_true",
+                    help="time the dense SwiGLU MLP of Beam's first layers (T=4096, intermediate 20480)")
     ap.add_argument("--block", action="store_true",
                     help="time the MoE sublayer on the residual stream (pre-norm, block, post-norm, residual)")
     return ap.parse_args()
@@ -426,10 +428,56 @@ def run_ours(args):
     ranks.close()
 
 
+def run_dense(args):
+    """Dense SwiGLU MLP line: tokens/s and the tensor-core roofline of the whole call."""
+    import group_limited_routing_router_b200 as bm
+    ranks = Ranks("nccl")
+    torch.cuda.set_device(ranks.local)
+    wl = bs.DENSE["dense_prefill"]
+    T, H, I = wl.T, wl.hidden, wl.inter
+    x = bs.make_x(wl).cuda()
+    wg, wu, wd = (t[0].contiguous() for t in bs.make_experts(wl, device="cuda"))
+    y = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(bm.dense_workspace_size(H, I, T), dtype=torch.uint8, device="cuda")
+    clocks = ClockSampler(ranks.local)
+    clocks.start()
+    for _ in range(args.warmup):
+        bm.dense_swiglu(x, wg, wu, wd, y=y, ws=ws)
+    ranks.barrier()
+    clocks.mark()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        bm.dense_swiglu(x, wg, wu, wd, y=y, ws=ws)
+    e1.record()
+    ranks.barrier()
+    clocks.mark()
+    clk = clocks.stop()
+    assert bm.device_status() == bm.OK
+    ms = ranks.max(e0.elapsed_time(e1)) / args.steps
+    flops = 6.0 * T * H * I
+    pk, kind = peaks()
+    achieved = flops / (ms / 1e3) / 1e12
+    line = {"metric": "dense SwiGLU MLP tokens/s (Beam first layers, T=4096, intermediate 20480)",
+            "value": ranks.world * T / (ms / 1e3), "unit": "tokens/s", "n_gpus": ranks.world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"dense_prefill: {wl.description}", "T": T, "hidden": H, "inter": I},
+            "roofline": {"bound": "tensor", "kernel": "dense call (gate/up + down GEMMs + cast)",
+                         "achieved": achieved, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": achieved / pk["bf16_tflops"], "traffic": None, "peak_kind": kind},
+            "clocks": clk, "gpu_launches": 4 * args.steps}
+    if ranks.rank == 0:
+        print(json.dumps(line))
+    ranks.close()
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.dense:
+        run_dense(args)
     else:
         run_ours(args)
 

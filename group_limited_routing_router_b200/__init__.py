@@ -98,6 +98,11 @@ def lib() -> ctypes.CDLL:
                                                 _vp, ctypes.c_size_t, _vp, ctypes.POINTER(ctypes.c_void_p)]
         L.beam_moe_block_forward.argtypes = [_cfgp, ctypes.POINTER(BeamMoeSublayer), ctypes.c_int64, _vp, _vp, _vp,
                                              _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+        L.beam_moe_dense_workspace_size.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int64]
+        L.beam_moe_dense_workspace_size.restype = ctypes.c_size_t
+        L.beam_moe_dense_swiglu.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp,
+                                            _vp, ctypes.c_size_t, _vp]
+        L.beam_moe_dense_swiglu.restype = ctypes.c_int
         L.beam_moe_device_status.argtypes = [_vp]
         L.beam_moe_selftest_timeout.argtypes = [ctypes.c_int64, _vp]
         L.beam_moe_strerror.argtypes = [ctypes.c_int]
@@ -275,6 +280,28 @@ def block_forward(cfg, stream_in, pre_norm_weight, post_norm_weight, eps: float,
                                         _ptr(u), _ptr(ids), _ptr(w), _ptr(ws), nbytes, _stream(stream)),
            "beam_moe_block_forward")
     return stream_out
+
+
+def dense_workspace_size(hidden: int, inter: int, T: int) -> int:
+    return int(lib().beam_moe_dense_workspace_size(int(hidden), int(inter), int(T)))
+
+
+def dense_swiglu(x, w_gate, w_up, w_down, y=None, ws=None, stream=None):
+    """Dense SwiGLU MLP: y = W_down (SiLU(W_gate x) * (W_up x)), x [T,H] bf16, weights [I,H]/[H,I] bf16."""
+    T, H = x.shape
+    I = w_gate.shape[0]
+    _dev(x, "x", torch.bfloat16, (T, H))
+    _dev(w_gate, "w_gate", torch.bfloat16, (I, H))
+    _dev(w_up, "w_up", torch.bfloat16, (I, H))
+    _dev(w_down, "w_down", torch.bfloat16, (H, I))
+    y = torch.empty(T, H, dtype=torch.bfloat16, device=x.device) if y is None else y
+    _dev(y, "y", torch.bfloat16, (T, H))
+    need = dense_workspace_size(H, I, T)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device) if ws is None else ws
+    _dev(ws, "ws", torch.uint8)
+    _check(lib().beam_moe_dense_swiglu(H, I, T, _ptr(x), _ptr(w_gate), _ptr(w_up), _ptr(w_down), _ptr(y), _ptr(ws),
+                                       ws.numel(), _stream(stream)), "beam_moe_dense_swiglu")
+    return y
 
 
 STAGES = ("router", "dispatch", "gather", "gate_up_swiglu", "down", "combine")

@@ -537,6 +537,104 @@ extern "C" int beam_moe_block_forward(const beam_moe_config *cfg, const beam_moe
 }
 
 // ------------------------------------------------------------------------------------------------
+// beam_moe_dense_swiglu: the grouped engine with one expert that takes every token in order.
+namespace beam {
+namespace {
+
+__global__ void dense_schedule_kernel(int32_t *counts, int64_t *offsets, int64_t T) {
+    counts[0] = static_cast<int32_t>(T);
+    offsets[0] = 0;
+    offsets[1] = T;
+}
+
+__global__ void f32_to_bf16_kernel(const float4 *__restrict__ in, uint2 *__restrict__ out, int64_t n4) {
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const float4 v = __ldg(in + i);
+        uint2 r;
+        r.x = pack_bf16x2(v.x, v.y);
+        r.y = pack_bf16x2(v.z, v.w);
+        out[i] = r;
+    }
+}
+
+struct DenseLayout {
+    size_t counts = 0, offsets = 0, h = 0, o = 0, total = 0;
+};
+
+bool dense_shape_ok(int32_t H, int32_t I) {
+    return H >= 64 && H <= 65536 && H % 64 == 0 && I >= 64 && I <= 65536 && I % 64 == 0;
+}
+
+DenseLayout dense_layout(int32_t H, int32_t I, int64_t T) {
+    DenseLayout L;
+    if (T == 0) return L;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off = align256(off + bytes);
+        return at;
+    };
+    L.counts = take(4);
+    L.offsets = take(16);
+    L.h = take(static_cast<size_t>(T) * I * 2);
+    L.o = take(static_cast<size_t>(T) * H * 4);
+    L.total = off;
+    return L;
+}
+
+}  // namespace
+}  // namespace beam
+
+extern "C" size_t beam_moe_dense_workspace_size(int32_t hidden, int32_t inter, int64_t T) {
+    if (!dense_shape_ok(hidden, inter) || T < 0 || T > kMaxTokens) return 0;
+    return dense_layout(hidden, inter, T).total;
+}
+
+extern "C" int beam_moe_dense_swiglu(int32_t hidden, int32_t inter, int64_t T, const beam_bf16 *x,
+                                     const beam_bf16 *w_gate, const beam_bf16 *w_up, const beam_bf16 *w_down,
+                                     beam_bf16 *y, void *ws, size_t ws_bytes, void *stream) {
+    if (!dense_shape_ok(hidden, inter)) return BEAM_MOE_ERR_INVALID_CONFIG;
+    if (T < 0 || T > kMaxTokens) return BEAM_MOE_ERR_INVALID_ARG;
+    if (T == 0) return BEAM_MOE_OK;
+    if (!x || !w_gate || !w_up || !w_down || !y || !ws) return BEAM_MOE_ERR_NULL;
+    if (!aligned16(x) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) || !aligned16(y) ||
+        !aligned16(ws))
+        return BEAM_MOE_ERR_MISALIGNED;
+    const DenseLayout L = dense_layout(hidden, inter, T);
+    if (ws_bytes < L.total) return BEAM_MOE_ERR_WORKSPACE_TOO_SMALL;
+    int dev, rc;
+    if ((rc = init_device(&dev))) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+    int32_t *counts = reinterpret_cast<int32_t *>(wsb + L.counts);
+    int64_t *offsets = reinterpret_cast<int64_t *>(wsb + L.offsets);
+    void *h = wsb + L.h;
+    void *o = wsb + L.o;
+    dense_schedule_kernel<<<1, 1, 0, s>>>(counts, offsets, T);
+    if ((rc = launch_status())) return rc;
+    // x itself is the token-ordered B operand of the gate/up GEMM (wide tiles, 64-row boxes)
+    CUtensorMap m_wg, m_wu, m_x, m_wd, m_h;
+    if (!encode_fn()) return BEAM_MOE_ERR_CUDA;
+    if (!make_map_3d(&m_wg, w_gate, hidden, inter, 1) || !make_map_3d(&m_wu, w_up, hidden, inter, 1) ||
+        !make_map_2d(&m_x, x, hidden, static_cast<uint64_t>(T), kWideBox) ||
+        !make_map_3d(&m_wd, w_down, inter, hidden, 1) ||
+        !make_map_2d(&m_h, h, inter, static_cast<uint64_t>(T), kWideBox))
+        return BEAM_MOE_ERR_CUDA;
+    const int grid = g_dev[dev].num_sms;
+    GemmParams p1{counts, offsets, h, 1, hidden, inter, 0, kDefaultTimeoutCycles, nullptr, 1};
+    GemmParams p2{counts, offsets, o, 1, inter, hidden, 0, kDefaultTimeoutCycles, nullptr, 1};
+    G1_WIDE_KERNEL<<<grid, kGemmThreads, G1Wide::kSmem, s>>>(m_wg, m_wu, m_x, p1);
+    if ((rc = launch_status())) return rc;
+    G2_WIDE_KERNEL<<<grid, kGemmThreads, G2Wide::kSmem, s>>>(m_wd, m_wd, m_h, p2);
+    if ((rc = launch_status())) return rc;
+    const int64_t n4 = T * static_cast<int64_t>(hidden) / 4;
+    f32_to_bf16_kernel<<<static_cast<unsigned>(std::min<int64_t>((n4 + 255) / 256, 16384)), 256, 0, s>>>(
+        reinterpret_cast<const float4 *>(o), reinterpret_cast<uint2 *>(y), n4);
+    return launch_status();
+}
+
+// ------------------------------------------------------------------------------------------------
 // beam_moe_permute_noalloc: the dispatch with its scratch in a fixed device array instead of a
 // caller-provided workspace, for callers that must not allocate device memory.
 namespace beam {

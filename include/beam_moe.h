@@ -170,6 +170,19 @@ BEAM_MOE_API int beam_moe_block_forward(const beam_moe_config *cfg, const beam_m
                                         float *topk_w_out, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * Dense SwiGLU MLP (Beam's first three layers: "The first 3 layers use a dense SwiGLU MLP",
+ * "Welcome Beam" page, section "Mixture of Experts"):
+ *   y = W_down (SiLU(W_gate x) * (W_up x))  per token, no routing and no scale
+ *   x [T, hidden] bf16; w_gate, w_up [inter, hidden] bf16; w_down [hidden, inter] bf16; y [T, hidden] bf16
+ * The same tensor-core engine as the experts (one expert that takes every token).  hidden and inter
+ * are multiples of 64; the workspace is beam_moe_dense_workspace_size(hidden, inter, T) bytes.
+ */
+BEAM_MOE_API size_t beam_moe_dense_workspace_size(int32_t hidden, int32_t inter, int64_t T);
+BEAM_MOE_API int beam_moe_dense_swiglu(int32_t hidden, int32_t inter, int64_t T, const beam_bf16 *x,
+                                       const beam_bf16 *w_gate, const beam_bf16 *w_up, const beam_bf16 *w_down,
+                                       beam_bf16 *y, void *ws, size_t ws_bytes, void *stream);
+
+/*
  * beam_moe_forward that also records caller-created CUDA events (cudaEvent_t) on `stream` around
  * its launches, for per-kernel timing:
  *   events[0] before the router            events[4] after the gate/up + SwiGLU GEMM

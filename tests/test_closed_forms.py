@@ -38,3 +38,22 @@ def test_every_workload_is_consistent():
         assert wl.topk <= wl.topk_groups * wl.n_experts // wl.n_groups
         assert wl.group_topn <= wl.n_experts // wl.n_groups
         assert wl.hidden % 64 == 0 and wl.inter % 64 == 0
+
+
+def test_dense_intermediate_reading_matches_8b_non_expert():
+    """I_dense = 20,480 (a reading) with the pages' attention shapes gives the '8B' non-expert count.
+
+    Attention per layer: W_q 5120 x (48 x 128), W_k and W_v 5120 x (8 x 128), W_o (48 x 128) x 5120 and the
+    sigmoid output gate 5120 x (48 x 128) ('Welcome Beam', section 'Attention'); 52 layers; vocabulary
+    151,936 (tech-report page, 'Key Takeaways'), embeddings and LM head untied (reading); routers
+    49 x 256 x 5120; 3 dense SwiGLU layers of intermediate size I.
+    """
+    H, q, kv = 5120, 48 * 128, 8 * 128
+    attn = 52 * (H * q + 2 * H * kv + q * H + H * q)
+    emb = 2 * 151_936 * H
+    routers = 49 * 256 * H
+    I = bs.DENSE["dense_prefill"].inter
+    dense = 3 * 3 * H * I
+    total = attn + emb + routers + dense
+    assert I == 20480 and round(total / 1e9) == 8          # "8B parameters" replicated under EP
+    assert abs(total / 1e9 - 8.0) < 0.05
