@@ -224,3 +224,33 @@ def sample_tokens(wl: Workload, n: int, T: Optional[int] = None, include=None) -
     if include is not None and len(include):
         idx = np.union1d(idx, np.asarray(include, dtype=np.int64))
     return np.sort(idx.astype(np.int64))
+
+
+def quantize_mxfp8(w: torch.Tensor):
+    """Synthetic FP8 checkpoint: w [..., rows, K] (bf16) -> (q [..., rows, K] E4M3 codes (uint8),
+    scale [..., K/32, rows] UE8M0 codes (uint8)).
+
+    Input preparation only (the OCP MXFP8 layout): each block of 32 consecutive K elements of a row
+    gets the power-of-two scale 2^(c-127) with c = ceil(log2(amax / 448)) + 127, so the block's
+    largest magnitude maps to at most 448 (E4M3's largest finite value); elements are rounded to
+    E4M3 (nearest even).  All-zero blocks get c = 0."""
+    *lead, rows, K = w.shape
+    assert K % 32 == 0
+    wf = w.float().reshape(*lead, rows, K // 32, 32)
+    amax = wf.abs().amax(-1)
+    e = torch.ceil(torch.log2(torch.clamp(amax, min=1e-38) / 448.0))
+    code = torch.where(amax > 0, torch.clamp(e + 127, 1, 254), torch.zeros_like(e))
+    q = (wf / torch.exp2(code - 127).unsqueeze(-1)).to(torch.float8_e4m3fn).view(torch.uint8)
+    scale = code.to(torch.uint8).transpose(-1, -2).contiguous()  # [..., K/32, rows]
+    return q.reshape(*lead, rows, K).contiguous(), scale
+
+
+def make_experts_fp8(wl: Workload, device: Optional[str] = None):
+    """MXFP8 version of make_experts: dict with q_gate, s_gate, q_up, s_up, q_down, s_down."""
+    wg, wu, wd = make_experts(wl, device)
+    out = {}
+    for name, w in (("gate", wg), ("up", wu), ("down", wd)):
+        q, sc = quantize_mxfp8(w)
+        out["q_" + name], out["s_" + name] = q, sc
+        del w
+    return out

@@ -58,6 +58,9 @@ def lib():
         L.oracle_rmsnorm.restype = None
         L.oracle_scaled_residual.argtypes = [ctypes.c_int64, ctypes.c_int, _dp, _dp, ctypes.c_int, _dp]
         L.oracle_scaled_residual.restype = ctypes.c_int
+        L.oracle_dequant_mxfp8.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.POINTER(ctypes.c_uint8),
+                                           ctypes.POINTER(ctypes.c_uint8), _u16p]
+        L.oracle_dequant_mxfp8.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -249,3 +252,16 @@ def block_forward(stream_bits: np.ndarray, g_pre: np.ndarray, g_post: np.ndarray
     z = rmsnorm(f["y"], g_post, eps)
     out = scaled_residual(s64[tok], z, step)
     return dict(u_bits=u_bits, route=f["route"], tokens=tok, y=f["y"], out=out)
+
+
+def dequant_mxfp8(q: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    """Exact MXFP8 dequantisation to bf16 bits: q [rows,K] E4M3 codes, scale [K/32,rows] UE8M0 codes."""
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    scale = np.ascontiguousarray(scale, dtype=np.uint8)
+    rows, K = q.shape
+    assert scale.shape == (K // 32, rows)
+    out = np.empty((rows, K), dtype=np.uint16)
+    u8p = ctypes.POINTER(ctypes.c_uint8)
+    if lib().oracle_dequant_mxfp8(rows, K, q.ctypes.data_as(u8p), scale.ctypes.data_as(u8p), _ptr(out, _u16p)) != 0:
+        raise ValueError("MXFP8 weights with a NaN code or a value bf16 cannot hold exactly")
+    return out

@@ -322,3 +322,43 @@ int oracle_scaled_residual(int64_t T, int H, const double *stream, const double 
     for (int64_t q = 0; q < T * (int64_t)H; ++q) out[q] = keep * stream[q] + add * z[q];
     return 0;
 }
+
+/*
+ * FP8 expert weights ("Checkpoint formats: BF16, FP8, and NVFP4": "Welcome Beam" page, TL;DR; the
+ * pages give no recipe).  Reading: the OCP MXFP8 layout, E4M3 elements with one power-of-two
+ * (UE8M0) scale per 32 consecutive K elements of a weight row; this build stores the scales
+ * K-block-major, scale[kb][row].
+ *   E4M3: sign s, exponent e (4 bits, bias 7), mantissa m (3 bits); e = 15 with m = 7 is NaN;
+ *         e = 0 is subnormal, m * 2^-9; otherwise (1 + m/8) * 2^(e-7).
+ *   UE8M0: 2^(c - 127); c = 255 is NaN.
+ * w[row][k] = e4m3(q[row][k]) * 2^(scale[k/32][row] - 127), returned as bf16 bits.  Every such
+ * product has at most 4 significant bits, so it is exact in bf16 whenever it lies in bf16's range;
+ * returns -1 for a NaN code or a product that bf16 cannot hold exactly.
+ * q [rows,K] uint8; scale [K/32, rows] uint8; out [rows,K] bf16 bits.
+ */
+static double e4m3_value(uint8_t b)
+{
+    const int s = b >> 7, e = (b >> 3) & 15, m = b & 7;
+    if (e == 15 && m == 7) return NAN;
+    const double mag = e == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -mag : mag;
+}
+
+int oracle_dequant_mxfp8(int64_t rows, int K, const uint8_t *q, const uint8_t *scale, uint16_t *out)
+{
+    if (K % 32) return -1;
+    int bad = 0;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int k = 0; k < K; ++k) {
+            const uint8_t c = scale[(int64_t)(k / 32) * rows + r];
+            const double v = e4m3_value(q[r * K + k]);
+            if (c == 255 || isnan(v)) { bad = 1; out[r * K + k] = 0; continue; }
+            const double w = ldexp(v, (int)c - 127);
+            const float f = (float)w;
+            uint32_t u;
+            memcpy(&u, &f, sizeof u);
+            if ((double)f != w || (u & 0xffffu)) { bad = 1; out[r * K + k] = 0; continue; }
+            out[r * K + k] = (uint16_t)(u >> 16);
+        }
+    return bad ? -1 : 0;
+}

@@ -13,6 +13,7 @@ import subprocess
 import pytest
 
 import oracle
+from tests import test_oracle_fp8 as fp8
 from tests import test_oracle_norm_residual as nr
 from tests import test_oracle_pins as pins
 
@@ -43,6 +44,9 @@ MUTANTS = {
                                  "add = sqrt((double)(k - 1) / (double)k), keep = 1.0 / sqrt((double)k);"),
     "residual_step_off_by_one": ("keep = sqrt((double)(k - 1) / (double)k), add = 1.0 / sqrt((double)k);",
                                  "keep = sqrt((double)k / (double)(k + 1)), add = 1.0 / sqrt((double)(k + 1));"),
+    "e4m3_bias_8": ("ldexp(1.0 + m / 8.0, e - 7)", "ldexp(1.0 + m / 8.0, e - 8)"),
+    "e4m3_subnormal_exponent": ("ldexp((double)m, -9)", "ldexp((double)m, -10)"),
+    "mxfp8_scale_row_major": ("scale[(int64_t)(k / 32) * rows + r]", "scale[r * (K / 32) + k / 32]"),
 }
 
 PINS = [
@@ -59,6 +63,8 @@ PINS = [
     nr.test_rmsnorm_closed_forms,
     nr.test_residual_weights_are_unit_norm,
     nr.test_every_addition_carries_equal_weight_after_104_steps,
+    fp8.test_e4m3_decoder_matches_torch_for_all_codes,
+    fp8.test_scale_is_a_power_of_two_per_32_block,
 ]
 
 
