@@ -236,6 +236,9 @@ def quantize_mxfp8(w: torch.Tensor):
     E4M3 (nearest even).  All-zero blocks get c = 0."""
     *lead, rows, K = w.shape
     assert K % 32 == 0
+    if len(lead) == 1 and lead[0] > 8:  # bound the FP32 temporaries: a few experts at a time
+        parts = [quantize_mxfp8(w[i:i + 8]) for i in range(0, lead[0], 8)]
+        return torch.cat([p[0] for p in parts]), torch.cat([p[1] for p in parts])
     wf = w.float().reshape(*lead, rows, K // 32, 32)
     amax = wf.abs().amax(-1)
     e = torch.ceil(torch.log2(torch.clamp(amax, min=1e-38) / 448.0))
@@ -247,10 +250,12 @@ def quantize_mxfp8(w: torch.Tensor):
 
 def make_experts_fp8(wl: Workload, device: Optional[str] = None):
     """MXFP8 version of make_experts: dict with q_gate, s_gate, q_up, s_up, q_down, s_down."""
-    wg, wu, wd = make_experts(wl, device)
+    return quantize_experts(*make_experts(wl, device))
+
+
+def quantize_experts(wg: torch.Tensor, wu: torch.Tensor, wd: torch.Tensor):
+    """quantize_mxfp8 of the three expert weight tensors, as the dict make_experts_fp8 returns."""
     out = {}
     for name, w in (("gate", wg), ("up", wu), ("down", wd)):
-        q, sc = quantize_mxfp8(w)
-        out["q_" + name], out["s_" + name] = q, sc
-        del w
+        out["q_" + name], out["s_" + name] = quantize_mxfp8(w)
     return out

@@ -33,6 +33,7 @@ sys.path.insert(0, ROOT)
 import beam_synth as bs  # noqa: E402
 
 METRIC = "MoE-layer tokens/s (Beam shape, BF16, T=4096) and % of tensor/HBM roofline"
+METRIC_FP8 = "MoE-layer tokens/s (Beam shape, MXFP8 expert weights, T=4096) and % of tensor/HBM roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture of the
@@ -40,10 +41,15 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # captured from hash the same; otherwise the JSON line reports null.
 _CSRC = os.path.join(ROOT, "group_limited_routing_router_b200", "csrc")
 NCU_TRAFFIC = {
-    ("gate_up_swiglu", "prefill"): {"bytes": 14.14e9 + 151.86e6, "files": ("gemm.cuh", "common.cuh"),
-                                    "hash": "77aa225963823e2f"},
-    ("down", "prefill"): {"bytes": 7.06e9 + 620.98e6, "files": ("gemm.cuh", "common.cuh"),
-                          "hash": "77aa225963823e2f"},
+    ("gate_up_swiglu", "prefill"): {"bytes": 14137922816 + 151317504, "files": ("gemm.cuh", "common.cuh"),
+                                    "hash": "d598baf939e79caa"},
+    ("down", "prefill"): {"bytes": 7060850432 + 620517632, "files": ("gemm.cuh", "common.cuh"),
+                          "hash": "d598baf939e79caa"},
+    ("gate_up_swiglu_fp8", "prefill"): {"bytes": 8140484864 + 149472000,
+                                        "files": ("gemm_fp8.cuh", "gemm.cuh", "common.cuh"),
+                                        "hash": "203a6b9373e1eec4"},
+    ("down_fp8", "prefill"): {"bytes": 3993288960 + 618224640, "files": ("gemm_fp8.cuh", "gemm.cuh", "common.cuh"),
+                              "hash": "203a6b9373e1eec4"},
 }
 
 
@@ -68,6 +74,8 @@ def parse():
                     help="time the dense SwiGLU MLP of Beam's first layers (T=4096, intermediate 20480)")
     ap.add_argument("--block", action="store_true",
                     help="time the MoE sublayer on the residual stream (pre-norm, block, post-norm, residual)")
+    ap.add_argument("--fp8", action="store_true",
+                    help="MXFP8 expert weights (E4M3 + one power-of-two scale per 32 K elements)")
     return ap.parse_args()
 
 
@@ -91,10 +99,12 @@ def kernel_source_hash() -> str:
 
 # ------------------------------------------------------------------------------------------------
 # algorithmic work (bytes the method must move, flops it must do), per step
-def algorithmic(wl: bs.Workload, n_act: int) -> dict:
+def algorithmic(wl: bs.Workload, n_act: int, fp8: bool = False) -> dict:
+    """fp8: expert weights are 1-byte E4M3 codes plus one 1-byte scale code per 32 elements."""
     T, H, I, E, k = wl.T, wl.hidden, wl.inter, wl.n_experts, wl.topk
     R = T * k
-    w_expert = 3 * H * I * 2
+    wb = 1.0 + 1.0 / 32 if fp8 else 2.0  # bytes per expert weight element
+    w_expert = 3 * H * I * wb
     return dict(
         layer_flops=T * (2 * H * E + k * 6 * H * I),
         layer_bytes=n_act * w_expert + E * H * 4 + 2 * T * H * 2 + T * k * 8,
@@ -102,8 +112,8 @@ def algorithmic(wl: bs.Workload, n_act: int) -> dict:
             "router": T * H * 2 + E * H * 4 + T * k * 8,
             "dispatch": T * k * 4 + 2 * R * 4,
             "gather": T * H * 2 + R * H * 2,
-            "gate_up_swiglu": n_act * 2 * I * H * 2 + R * H * 2 + R * I * 2,
-            "down": n_act * H * I * 2 + R * I * 2 + R * H * 4,
+            "gate_up_swiglu": n_act * 2 * I * H * wb + R * H * 2 + R * I * 2,
+            "down": n_act * H * I * wb + R * I * 2 + R * H * 4,
             "combine": R * H * 4 + T * k * 8 + T * H * 2,
         },
         stage_flops={"router": 2 * T * H * E, "gate_up_swiglu": 4 * R * H * I, "down": 2 * R * H * I},
@@ -162,9 +172,21 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------------------------
-def cpu_oracle_rate(wl, x_cpu, W, bias, wg, wu, wd, n_sample: int, route_all: bool = True) -> dict:
+def bf16_fetch(wg, wu, wd):
+    import oracle
+    return lambda e: (oracle.bf16_bits(wg[e]), oracle.bf16_bits(wu[e]), oracle.bf16_bits(wd[e]))
+
+
+def fp8_fetch(w8):
+    """One expert's weights for the oracle: MXFP8 codes dequantised on the host by the oracle."""
+    import oracle
+    return lambda e: tuple(oracle.dequant_mxfp8(w8["q_" + n][e].cpu().numpy(), w8["s_" + n][e].cpu().numpy())
+                           for n in ("gate", "up", "down"))
+
+
+def cpu_oracle_rate(wl, x_cpu, W, bias, fetch, n_sample: int, route_all: bool = True) -> dict:
     """Time the CPU oracle: routing (FP64 scores + selection) and the expert half on a token sample.
-    Expert weights are copied to the host expert by expert, outside the timed sections."""
+    fetch(e) gives one expert's bf16 weight bits on the host; it runs outside the timed sections."""
     import oracle
     xb = oracle.bf16_bits(x_cpu)
     b = None if bias is None else bias.cpu().numpy()
@@ -187,7 +209,7 @@ def cpu_oracle_rate(wl, x_cpu, W, bias, wg, wu, wd, n_sample: int, route_all: bo
         rows, slots = np.nonzero(ids == e)
         if rows.size == 0:
             continue
-        w3 = (oracle.bf16_bits(wg[e]), oracle.bf16_bits(wu[e]), oracle.bf16_bits(wd[e]))
+        w3 = fetch(e)
         t1 = time.perf_counter()
         out[rows, slots, :] = oracle.expert_mlp(xs[rows], *w3)
         t_exp += time.perf_counter() - t1
@@ -216,7 +238,7 @@ def run_reference(args):
     n = 16
     rates, secs = [], []
     for i in range(args.warmup + args.steps):
-        r = cpu_oracle_rate(wl, x, W, bias, wg, wu, wd, n, route_all=False)
+        r = cpu_oracle_rate(wl, x, W, bias, bf16_fetch(wg, wu, wd), n, route_all=False)
         if i >= args.warmup:
             rates.append(r)
             secs.append(r["seconds"])
@@ -315,6 +337,14 @@ def run_ours(args):
     W = W_cpu.cuda()
     bias = None if b_cpu is None else b_cpu.cuda()
     wg, wu, wd = bs.make_experts(wl, device="cuda")
+    w8 = None
+    if args.fp8:
+        if args.block:
+            raise SystemExit("--fp8 and --block: the sublayer entry point takes bf16 expert weights")
+        w8 = bs.quantize_experts(wg, wu, wd)
+        del wg, wu, wd
+        wg = wu = wd = None
+        torch.cuda.empty_cache()
     ws = torch.empty(bm.workspace_size(layer, T, bm.WS_FORWARD), dtype=torch.uint8, device="cuda")
     y = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
     ids = torch.empty(T, wl.topk, dtype=torch.int32, device="cuda")
@@ -330,6 +360,9 @@ def run_ours(args):
         def step():
             bm.block_forward(layer, x, g_pre, g_post, 1e-6, block_step, W, bias, wg, wu, wd, stream_out=y, ids=ids,
                              w=w, ws=ws_blk)
+    elif args.fp8:
+        def step():
+            bm.forward_fp8(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws)
     else:
         def step():
             bm.forward(layer, x, W, bias, wg, wu, wd, y=y, ids=ids, w=w, ws=ws)
@@ -364,7 +397,10 @@ def run_ours(args):
     # per-stage device time from events recorded between the launches (same stream)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
     for i in range(args.steps):
-        bm.forward_profiled(layer, x, W, bias, wg, wu, wd, evs[i], y, ids, w, ws)
+        if args.fp8:
+            bm.forward_fp8(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws, events=evs[i])
+        else:
+            bm.forward_profiled(layer, x, W, bias, wg, wu, wd, evs[i], y, ids, w, ws)
     torch.cuda.synchronize()
     stage_ms = {name: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
                 for j, name in enumerate(bm.STAGES)}
@@ -388,13 +424,13 @@ def run_ours(args):
     e2e_value = ranks.rate(T * args.steps, e0.elapsed_time(e1))
     assert bm.device_status() == bm.OK
 
-    alg = algorithmic(wl, n_act)
+    alg = algorithmic(wl, n_act, args.fp8)
     pk, pk_kind = peaks()
     dom = max(stage_ms, key=stage_ms.get)
     dom_bytes = alg["stage_bytes"][dom]
     achieved = dom_bytes / (stage_ms[dom] / 1e3) / 1e9
     src_hash = kernel_source_hash()
-    tr = NCU_TRAFFIC.get((dom, wl.name))
+    tr = NCU_TRAFFIC.get((dom + ("_fp8" if args.fp8 else ""), wl.name))
     traffic = tr["bytes"] if tr and files_hash(tr["files"]) == tr["hash"] else None
     roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / pk["hbm_gbs"], "traffic": traffic, "peak_kind": pk_kind,
@@ -410,12 +446,20 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_oracle_rate(wl, x_cpu, W_cpu, b_cpu, wg, wu, wd, args.cpu_sample)
+        fetch = fp8_fetch(w8) if args.fp8 else bf16_fetch(wg, wu, wd)
+        cpu = cpu_oracle_rate(wl, x_cpu, W_cpu, b_cpu, fetch, args.cpu_sample)
         cpu.pop("seconds", None)
 
-    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": config_dict(wl),
+    cfg = config_dict(wl)
+    if args.fp8:
+        cfg["weights"] = ("MXFP8 experts: E4M3 codes + UE8M0 scale per 32 K elements (1.03 B/weight), rebuilt "
+                          "as bf16 in shared memory; router FP32")
+        cfg["weights_bytes"] = int(3 * wl.n_experts * wl.hidden * wl.inter * (1 + 1 / 32))
+        cfg["l2"] = "no flush: every step streams the 10.4 GB of FP8 expert weights and scales (> 126 MB L2)"
+    line = {"metric": METRIC_FP8 if args.fp8 else METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "fp8-e4m3 weights, bf16 MMA" if args.fp8 else "bf16",
+            "data": "synthetic", "config": cfg,
             "roofline": roofline, "layer_roofline": layer_roof, "stage_ms": stage_ms, "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2,
                     "d2h_bytes_per_step": T * H * 2},

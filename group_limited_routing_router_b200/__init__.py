@@ -48,6 +48,11 @@ class BeamMoeSublayer(ctypes.Structure):
                 ("eps", ctypes.c_float), ("step", ctypes.c_int32)]
 
 
+class BeamMoeFp8Experts(ctypes.Structure):
+    _fields_ = [("w_gate", ctypes.c_void_p), ("w_gate_scale", ctypes.c_void_p), ("w_up", ctypes.c_void_p),
+                ("w_up_scale", ctypes.c_void_p), ("w_down", ctypes.c_void_p), ("w_down_scale", ctypes.c_void_p)]
+
+
 @dataclasses.dataclass(frozen=True)
 class LayerConfig:
     hidden: int = 5120
@@ -96,6 +101,10 @@ def lib() -> ctypes.CDLL:
                                        ctypes.c_size_t, _vp]
         L.beam_moe_forward_profiled.argtypes = [_cfgp, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                                 _vp, ctypes.c_size_t, _vp, ctypes.POINTER(ctypes.c_void_p)]
+        _f8p = ctypes.POINTER(BeamMoeFp8Experts)
+        L.beam_moe_experts_fp8.argtypes = [_cfgp, ctypes.c_int64, _vp, _vp, _vp, _f8p, _vp, _vp, ctypes.c_size_t, _vp]
+        L.beam_moe_forward_fp8.argtypes = [_cfgp, ctypes.c_int64, _vp, _vp, _vp, _f8p, _vp, _vp, _vp, _vp,
+                                           ctypes.c_size_t, _vp, ctypes.POINTER(ctypes.c_void_p)]
         L.beam_moe_block_forward.argtypes = [_cfgp, ctypes.POINTER(BeamMoeSublayer), ctypes.c_int64, _vp, _vp, _vp,
                                              _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
         L.beam_moe_dense_workspace_size.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int64]
@@ -108,7 +117,8 @@ def lib() -> ctypes.CDLL:
         L.beam_moe_strerror.argtypes = [ctypes.c_int]
         L.beam_moe_strerror.restype = ctypes.c_char_p
         for name in ("beam_moe_route", "beam_moe_permute", "beam_moe_experts", "beam_moe_forward",
-                     "beam_moe_forward_profiled", "beam_moe_block_forward", "beam_moe_device_status",
+                     "beam_moe_forward_profiled", "beam_moe_block_forward", "beam_moe_experts_fp8",
+                     "beam_moe_forward_fp8", "beam_moe_device_status",
                      "beam_moe_selftest_timeout"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -252,6 +262,74 @@ def forward(cfg, x, w_router, bias, w_gate, w_up, w_down, y=None, ids=None, w=No
     return (y, ids, w) if return_routing else y
 
 
+FP8_KEYS = ("q_gate", "s_gate", "q_up", "s_up", "q_down", "s_down")
+
+
+def _fp8_experts(c: BeamMoeConfig, w8: dict) -> BeamMoeFp8Experts:
+    """MXFP8 expert weights: dict of uint8 CUDA tensors q_gate/q_up [E,I,H], q_down [E,H,I] (E4M3 codes)
+    and s_gate/s_up [E,H/32,I], s_down [E,I/32,H] (UE8M0 scale codes, K-block-major)."""
+    E, H, I = c.n_experts, c.hidden, c.inter
+    shapes = dict(q_gate=(E, I, H), q_up=(E, I, H), q_down=(E, H, I),
+                  s_gate=(E, H // 32, I), s_up=(E, H // 32, I), s_down=(E, I // 32, H))
+    for k in FP8_KEYS:
+        if k not in w8:
+            raise KeyError(f"FP8 experts need '{k}'")
+        _dev(w8[k], k, torch.uint8, shapes[k])
+    return BeamMoeFp8Experts(*(w8[k].data_ptr() for k in FP8_KEYS))
+
+
+def experts_fp8(cfg, x, ids, w, w8: dict, y=None, ws=None, stream=None) -> torch.Tensor:
+    """experts() with MXFP8 expert weights (see _fp8_experts for the layout)."""
+    c = _cfg(cfg)
+    T = x.shape[0]
+    _dev(x, "x", torch.bfloat16, (T, c.hidden))
+    _dev(ids, "ids", torch.int32, (T, c.topk))
+    _dev(w, "w", torch.float32, (T, c.topk))
+    f8 = _fp8_experts(c, w8)
+    y = torch.empty(T, c.hidden, dtype=torch.bfloat16, device=x.device) if y is None else y
+    _dev(y, "y", torch.bfloat16, (T, c.hidden))
+    ws, nbytes = _workspace(c, T, WS_EXPERTS, ws, x.device)
+    _check(lib().beam_moe_experts_fp8(ctypes.byref(c), T, _ptr(x), _ptr(ids), _ptr(w), ctypes.byref(f8), _ptr(y),
+                                      _ptr(ws), nbytes, _stream(stream)), "beam_moe_experts_fp8")
+    return y
+
+
+def _event_handles(events):
+    if events is None:
+        return None
+    if len(events) != 7:
+        raise ValueError("need 7 events")
+    handles = (ctypes.c_void_p * 7)()
+    for i, e in enumerate(events):
+        if e.cuda_event == 0:  # torch creates the CUDA event at its first record
+            e.record()
+        handles[i] = e.cuda_event
+    return handles
+
+
+def forward_fp8(cfg, x, w_router, bias, w8: dict, y=None, ids=None, w=None, ws=None, stream=None,
+                return_routing: bool = False, events=None):
+    """forward() with MXFP8 expert weights; `events` (7 torch.cuda.Event, optional) as in forward_profiled."""
+    c = _cfg(cfg)
+    T = x.shape[0]
+    _dev(x, "x", torch.bfloat16, (T, c.hidden))
+    _dev(w_router, "w_router", torch.float32, (c.n_experts, c.hidden))
+    _dev(bias, "bias", torch.float32, (c.n_experts,))
+    f8 = _fp8_experts(c, w8)
+    y = torch.empty(T, c.hidden, dtype=torch.bfloat16, device=x.device) if y is None else y
+    _dev(y, "y", torch.bfloat16, (T, c.hidden))
+    if return_routing:
+        ids = torch.empty(T, c.topk, dtype=torch.int32, device=x.device) if ids is None else ids
+        w = torch.empty(T, c.topk, dtype=torch.float32, device=x.device) if w is None else w
+    _dev(ids, "ids", torch.int32, (T, c.topk))
+    _dev(w, "w", torch.float32, (T, c.topk))
+    ws, nbytes = _workspace(c, T, WS_FORWARD, ws, x.device)
+    _check(lib().beam_moe_forward_fp8(ctypes.byref(c), T, _ptr(x), _ptr(w_router), _ptr(bias), ctypes.byref(f8),
+                                      _ptr(y), _ptr(ids), _ptr(w), _ptr(ws), nbytes, _stream(stream),
+                                      _event_handles(events)), "beam_moe_forward_fp8")
+    return (y, ids, w) if return_routing else y
+
+
 def block_forward(cfg, stream_in, pre_norm_weight, post_norm_weight, eps: float, step: int, w_router, bias,
                   w_gate, w_up, w_down, stream_out=None, u=None, ids=None, w=None, ws=None, stream=None):
     """One MoE sublayer on the residual stream (pre-norm, block, post-norm, scaled residual).
@@ -312,13 +390,7 @@ def forward_profiled(cfg, x, w_router, bias, w_gate, w_up, w_down, events, y, id
     beam_moe_forward_profiled); all buffers are caller-provided so nothing is allocated per call."""
     c = _cfg(cfg)
     T = x.shape[0]
-    if len(events) != 7:
-        raise ValueError("need 7 events")
-    handles = (ctypes.c_void_p * 7)()
-    for i, e in enumerate(events):
-        if e.cuda_event == 0:  # torch creates the CUDA event at its first record
-            e.record()
-        handles[i] = e.cuda_event
+    handles = _event_handles(events)
     _check(lib().beam_moe_forward_profiled(ctypes.byref(c), T, _ptr(x), _ptr(w_router), _ptr(bias), _ptr(w_gate),
                                            _ptr(w_up), _ptr(w_down), _ptr(y), _ptr(ids), _ptr(w), _ptr(ws),
                                            ws.numel(), _stream(stream), handles), "beam_moe_forward_profiled")

@@ -19,6 +19,7 @@
 #include "combine.cuh"
 #include "permute.cuh"
 #include "gemm.cuh"
+#include "gemm_fp8.cuh"
 #include "norm.cuh"
 #include "router.cuh"
 
@@ -38,15 +39,43 @@ constexpr int64_t kMaxTokens = int64_t(1) << 24;
 #define G2_WIDE_ARGS false, 192, 64, 5, 2, 256, false
 #define G1_NARROW_ARGS true, 32, 1, 6, 4, 64, true
 #define G2_NARROW_ARGS false, 32, 32, 10, 4, 32, false
-using G1Wide = GemmCfg<G1_WIDE_ARGS>;
-using G2Wide = GemmCfg<G2_WIDE_ARGS>;
-using G1Narrow = GemmCfg<G1_NARROW_ARGS>;
-using G2Narrow = GemmCfg<G2_NARROW_ARGS>;
-#define G1_WIDE_KERNEL grouped_gemm_kernel<G1_WIDE_ARGS>
-#define G2_WIDE_KERNEL grouped_gemm_kernel<G2_WIDE_ARGS>
-#define G1_NARROW_KERNEL grouped_gemm_kernel<G1_NARROW_ARGS>
-#define G2_NARROW_KERNEL grouped_gemm_kernel<G2_NARROW_ARGS>
+// FP8 variants: <gate/up?, BN, B box rows, weight stages (K = 128), B stages (K = 64), TMEM slots,
+// slot columns, gather?, bf16 A ring stages in TMEM>.  The A ring takes the TMEM columns the
+// accumulators leave; the prefill gate/up variant gives its accumulators 2 slots of 192 columns
+// (one item of more than 96 tokens at a time) so that two A ring stages fit.
+#define G1_WIDE_FP8_ARGS true, 192, 64, 3, 4, 2, 192, false, 2
+#define G2_WIDE_FP8_ARGS false, 192, 64, 4, 5, 2, 192, false, 4
+#define G1_NARROW_FP8_ARGS true, 32, 1, 5, 12, 2, 64, true, 6
+#define G2_NARROW_FP8_ARGS false, 32, 32, 9, 16, 4, 32, false, 12
 constexpr int kWideBN = 192, kWideBox = 64, kNarrowBN = 32, kNarrowBox = 32;
+
+template <bool G, int BN, int BOXN, int ST, int NS, int SC, bool GA>
+bool set_gemm_smem() {
+    return cudaFuncSetAttribute(grouped_gemm_kernel<G, BN, BOXN, ST, NS, SC, GA>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                GemmCfg<G, BN, BOXN, ST, NS, SC, GA>::kSmem) == cudaSuccess;
+}
+template <bool G, int BN, int BOXN, int W8, int BS, int NS, int SC, bool GA, int AS>
+bool set_gemm_fp8_smem() {
+    return cudaFuncSetAttribute(grouped_gemm_fp8_kernel<G, BN, BOXN, W8, BS, NS, SC, GA, AS>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Fp8GemmCfg<G, BN, BOXN, W8, BS, NS, SC, GA, AS>::kSmem) == cudaSuccess;
+}
+
+// a1 is ignored by the down projection.
+template <bool G, int BN, int BOXN, int ST, int NS, int SC, bool GA>
+void launch_gemm(int grid, cudaStream_t s, const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b,
+                 const GemmParams &p) {
+    grouped_gemm_kernel<G, BN, BOXN, ST, NS, SC, GA>
+        <<<grid, kGemmThreads, GemmCfg<G, BN, BOXN, ST, NS, SC, GA>::kSmem, s>>>(a0, a1, b, p);
+}
+// a1 and s1 are ignored by the down projection.
+template <bool G, int BN, int BOXN, int W8, int BS, int NS, int SC, bool GA, int AS>
+void launch_gemm_fp8(int grid, cudaStream_t s, const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &s0,
+                     const CUtensorMap &s1, const CUtensorMap &b, const GemmParams &p) {
+    using C = Fp8GemmCfg<G, BN, BOXN, W8, BS, NS, SC, GA, AS>;
+    grouped_gemm_fp8_kernel<G, BN, BOXN, W8, BS, NS, SC, GA, AS><<<grid, C::kThreads, C::kSmem, s>>>(a0, a1, s0, s1, b, p);
+}
 
 // Tile family from the mean rows per expert (T*k/E): narrow when experts see a handful of tokens.
 bool narrow_tiles(const beam_moe_config *c, int64_t T) {
@@ -87,14 +116,10 @@ int init_device(int *dev_out) {
         }
         bool ok = cudaFuncSetAttribute(router_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        kRtSmemBytes) == cudaSuccess;
-        ok = ok && cudaFuncSetAttribute(G1_WIDE_KERNEL, cudaFuncAttributeMaxDynamicSharedMemorySize, G1Wide::kSmem) ==
-                       cudaSuccess;
-        ok = ok && cudaFuncSetAttribute(G2_WIDE_KERNEL, cudaFuncAttributeMaxDynamicSharedMemorySize, G2Wide::kSmem) ==
-                       cudaSuccess;
-        ok = ok && cudaFuncSetAttribute(G1_NARROW_KERNEL, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        G1Narrow::kSmem) == cudaSuccess;
-        ok = ok && cudaFuncSetAttribute(G2_NARROW_KERNEL, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        G2Narrow::kSmem) == cudaSuccess;
+        ok = ok && set_gemm_smem<G1_WIDE_ARGS>() && set_gemm_smem<G2_WIDE_ARGS>() &&
+             set_gemm_smem<G1_NARROW_ARGS>() && set_gemm_smem<G2_NARROW_ARGS>();
+        ok = ok && set_gemm_fp8_smem<G1_WIDE_FP8_ARGS>() && set_gemm_fp8_smem<G2_WIDE_FP8_ARGS>() &&
+             set_gemm_fp8_smem<G1_NARROW_FP8_ARGS>() && set_gemm_fp8_smem<G2_NARROW_FP8_ARGS>();
         ok = ok && cudaFuncSetAttribute(combine_norm_residual_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         kMaxBlockHidden * 4) == cudaSuccess;
         if (!ok) d.status = BEAM_MOE_ERR_CUDA;
@@ -200,6 +225,28 @@ bool make_map_3d(CUtensorMap *m, const void *base, uint64_t K, uint64_t M, uint6
                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3D [E][M][K] E4M3 weights, box {128, 128, 1}: 128-byte rows (K = 128), 128-byte swizzle.
+bool make_map_3d_fp8(CUtensorMap *m, const void *base, uint64_t K, uint64_t M, uint64_t E) {
+    const cuuint64_t dims[3] = {K, M, E};
+    const cuuint64_t strides[2] = {K, K * M};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(2 * kBK), static_cast<cuuint32_t>(kBM), 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 3D [E][K/32][M] UE8M0 scale codes, box {128, 4, 1}: the four K blocks of one K = 128 stage.
+bool make_map_scale(CUtensorMap *m, const void *base, uint64_t M, uint64_t KB, uint64_t E) {
+    const cuuint64_t dims[3] = {M, KB, E};
+    const cuuint64_t strides[2] = {M, M * KB};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kBM), 4, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int launch_status() { return cudaGetLastError() == cudaSuccess ? BEAM_MOE_OK : BEAM_MOE_ERR_CUDA; }
 
 // Generic 2-D tensor map: [rows][inner] elements of `esize` bytes, box {box_inner, box_rows}.
@@ -264,10 +311,20 @@ struct BlockTail {
     float eps, keep, add;
 };
 
+// The experts' weights: bf16 [E][rows][K], or E4M3 codes with their scale codes.
+struct ExpertWeights {
+    const void *gate, *up, *down;
+    const uint8_t *s_gate, *s_up, *s_down;  // FP8 only: [E][K/32][rows]
+    bool fp8;
+};
+
+ExpertWeights bf16_weights(const beam_bf16 *wg, const beam_bf16 *wu, const beam_bf16 *wd) {
+    return ExpertWeights{wg, wu, wd, nullptr, nullptr, nullptr, false};
+}
+
 int enqueue_experts(const beam_moe_config *c, int dev, int64_t T, const beam_bf16 *x, const int32_t *ids,
-                    const float *w, const beam_bf16 *wg, const beam_bf16 *wu, const beam_bf16 *wd, beam_bf16 *y,
-                    uint8_t *ws, const Layout &L, cudaStream_t s, cudaEvent_t const *ev = nullptr,
-                    const BlockTail *tail = nullptr) {
+                    const float *w, const ExpertWeights &W, beam_bf16 *y, uint8_t *ws, const Layout &L,
+                    cudaStream_t s, cudaEvent_t const *ev = nullptr, const BlockTail *tail = nullptr) {
     int32_t *counts = reinterpret_cast<int32_t *>(ws + L.counts);
     int64_t *offsets = reinterpret_cast<int64_t *>(ws + L.offsets);
     int32_t *row_src = reinterpret_cast<int32_t *>(ws + L.row_src);
@@ -295,22 +352,39 @@ int enqueue_experts(const beam_moe_config *c, int dev, int64_t T, const beam_bf1
     // Weights are read once per call when (almost) every expert fits one token tile: mark them
     // evict-first so they do not push the reused activations out of L2.
     const int once = (mean_rows + 4.0 * std::sqrt(mean_rows) <= bn) ? 1 : 0;
-    CUtensorMap m_wg, m_wu, m_b1, m_wd, m_h;
+    CUtensorMap m_wg, m_wu, m_b1, m_wd, m_h, m_sg, m_su, m_sd;
     if (!encode_fn()) return BEAM_MOE_ERR_CUDA;
     const bool b1_ok = narrow ? make_map_2d(&m_b1, x, H, static_cast<uint64_t>(T), 1)   // gather4 rows of x
                               : make_map_2d(&m_b1, ws + L.xp, H, R, box);              // tiled x_perm rows
-    if (!b1_ok || !make_map_3d(&m_wg, wg, H, I, E) || !make_map_3d(&m_wu, wu, H, I, E) ||
-        !make_map_3d(&m_wd, wd, I, H, E) || !make_map_2d(&m_h, h, I, R, box))
-        return BEAM_MOE_ERR_CUDA;
+    bool w_ok;
+    if (W.fp8) {
+        w_ok = make_map_3d_fp8(&m_wg, W.gate, H, I, E) && make_map_3d_fp8(&m_wu, W.up, H, I, E) &&
+               make_map_3d_fp8(&m_wd, W.down, I, H, E) && make_map_scale(&m_sg, W.s_gate, I, H / 32, E) &&
+               make_map_scale(&m_su, W.s_up, I, H / 32, E) && make_map_scale(&m_sd, W.s_down, H, I / 32, E);
+    } else {
+        w_ok = make_map_3d(&m_wg, W.gate, H, I, E) && make_map_3d(&m_wu, W.up, H, I, E) &&
+               make_map_3d(&m_wd, W.down, I, H, E);
+    }
+    if (!b1_ok || !w_ok || !make_map_2d(&m_h, h, I, R, box)) return BEAM_MOE_ERR_CUDA;
     const int grid = g_dev[dev].num_sms;
     GemmParams p1{counts, offsets, h, E, H, I, once, kDefaultTimeoutCycles, row_src, k};
     GemmParams p2{counts, offsets, o, E, I, H, once, kDefaultTimeoutCycles, nullptr, k};
-    if (narrow) G1_NARROW_KERNEL<<<grid, kGemmThreads, G1Narrow::kSmem, s>>>(m_wg, m_wu, m_b1, p1);
-    else G1_WIDE_KERNEL<<<grid, kGemmThreads, G1Wide::kSmem, s>>>(m_wg, m_wu, m_b1, p1);
+    if (W.fp8) {
+        if (narrow) launch_gemm_fp8<G1_NARROW_FP8_ARGS>(grid, s, m_wg, m_wu, m_sg, m_su, m_b1, p1);
+        else launch_gemm_fp8<G1_WIDE_FP8_ARGS>(grid, s, m_wg, m_wu, m_sg, m_su, m_b1, p1);
+    } else {
+        if (narrow) launch_gemm<G1_NARROW_ARGS>(grid, s, m_wg, m_wu, m_b1, p1);
+        else launch_gemm<G1_WIDE_ARGS>(grid, s, m_wg, m_wu, m_b1, p1);
+    }
     if ((rc = launch_status())) return rc;
     if (!record(ev, 4, s)) return BEAM_MOE_ERR_CUDA;
-    if (narrow) G2_NARROW_KERNEL<<<grid, kGemmThreads, G2Narrow::kSmem, s>>>(m_wd, m_wd, m_h, p2);
-    else G2_WIDE_KERNEL<<<grid, kGemmThreads, G2Wide::kSmem, s>>>(m_wd, m_wd, m_h, p2);
+    if (W.fp8) {
+        if (narrow) launch_gemm_fp8<G2_NARROW_FP8_ARGS>(grid, s, m_wd, m_wd, m_sd, m_sd, m_h, p2);
+        else launch_gemm_fp8<G2_WIDE_FP8_ARGS>(grid, s, m_wd, m_wd, m_sd, m_sd, m_h, p2);
+    } else {
+        if (narrow) launch_gemm<G2_NARROW_ARGS>(grid, s, m_wd, m_wd, m_h, p2);
+        else launch_gemm<G2_WIDE_ARGS>(grid, s, m_wd, m_wd, m_h, p2);
+    }
     if ((rc = launch_status())) return rc;
     if (!record(ev, 5, s)) return BEAM_MOE_ERR_CUDA;
     if (tail)
@@ -385,45 +459,52 @@ int beam_moe_permute(const beam_moe_config *cfg, int64_t T, const int32_t *topk_
                            reinterpret_cast<int32_t *>(static_cast<uint8_t *>(ws) + L.hist), s);
 }
 
-int beam_moe_experts(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const int32_t *topk_ids,
-                     const float *topk_w, const beam_bf16 *w_gate, const beam_bf16 *w_up, const beam_bf16 *w_down,
-                     beam_bf16 *y, void *ws, size_t ws_bytes, void *stream) {
-    int rc = validate(cfg);
-    if (rc) return rc;
-    if ((rc = check_T(cfg, T))) return rc;
-    if (T == 0) return BEAM_MOE_OK;
-    if (!x || !topk_ids || !topk_w || !w_gate || !w_up || !w_down || !y || !ws) return BEAM_MOE_ERR_NULL;
-    if (!aligned16(x) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) || !aligned16(y) ||
-        (ws && !aligned16(ws)))
-        return BEAM_MOE_ERR_MISALIGNED;
-    const Layout L = layout(cfg, T, BEAM_MOE_WS_EXPERTS);
-    if (ws_bytes < L.total) return BEAM_MOE_ERR_WORKSPACE_TOO_SMALL;
-    if (T == 0) return BEAM_MOE_OK;
-    int dev;
-    if ((rc = init_device(&dev))) return rc;
-    return enqueue_experts(cfg, dev, T, x, topk_ids, topk_w, w_gate, w_up, w_down, y, static_cast<uint8_t *>(ws), L,
-                           static_cast<cudaStream_t>(stream));
-}
-
 }  // extern "C"
 
 namespace beam {
 namespace {
-int forward_impl(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const float *w_router,
-                 const float *sel_bias, const beam_bf16 *w_gate, const beam_bf16 *w_up, const beam_bf16 *w_down,
-                 beam_bf16 *y, int32_t *topk_ids_out, float *topk_w_out, void *ws, size_t ws_bytes, void *stream,
-                 cudaEvent_t const *ev) {
+// Argument checks of the experts' weights: every pointer set and 16-byte aligned.
+int weights_status(const ExpertWeights &W) {
+    if (!W.gate || !W.up || !W.down) return BEAM_MOE_ERR_NULL;
+    if (W.fp8 && (!W.s_gate || !W.s_up || !W.s_down)) return BEAM_MOE_ERR_NULL;
+    if (!aligned16(W.gate) || !aligned16(W.up) || !aligned16(W.down)) return BEAM_MOE_ERR_MISALIGNED;
+    if (W.fp8 && (!aligned16(W.s_gate) || !aligned16(W.s_up) || !aligned16(W.s_down))) return BEAM_MOE_ERR_MISALIGNED;
+    return BEAM_MOE_OK;
+}
+
+ExpertWeights fp8_weights(const beam_moe_fp8_experts *w8) {
+    return ExpertWeights{w8->w_gate, w8->w_up, w8->w_down, w8->w_gate_scale, w8->w_up_scale, w8->w_down_scale, true};
+}
+
+int experts_impl(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const int32_t *topk_ids,
+                 const float *topk_w, const ExpertWeights &W, beam_bf16 *y, void *ws, size_t ws_bytes, void *stream) {
     int rc = validate(cfg);
     if (rc) return rc;
     if ((rc = check_T(cfg, T))) return rc;
     if (T == 0) return BEAM_MOE_OK;
-    if (!x || !w_router || !w_gate || !w_up || !w_down || !y || !ws) return BEAM_MOE_ERR_NULL;
-    if (!aligned16(x) || !aligned16(w_router) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) ||
-        !aligned16(y) || (ws && !aligned16(ws)))
-        return BEAM_MOE_ERR_MISALIGNED;
+    if (!x || !topk_ids || !topk_w || !y || !ws) return BEAM_MOE_ERR_NULL;
+    if ((rc = weights_status(W))) return rc;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(ws)) return BEAM_MOE_ERR_MISALIGNED;
+    const Layout L = layout(cfg, T, BEAM_MOE_WS_EXPERTS);
+    if (ws_bytes < L.total) return BEAM_MOE_ERR_WORKSPACE_TOO_SMALL;
+    int dev;
+    if ((rc = init_device(&dev))) return rc;
+    return enqueue_experts(cfg, dev, T, x, topk_ids, topk_w, W, y, static_cast<uint8_t *>(ws), L,
+                           static_cast<cudaStream_t>(stream));
+}
+
+int forward_impl(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const float *w_router,
+                 const float *sel_bias, const ExpertWeights &W, beam_bf16 *y, int32_t *topk_ids_out,
+                 float *topk_w_out, void *ws, size_t ws_bytes, void *stream, cudaEvent_t const *ev) {
+    int rc = validate(cfg);
+    if (rc) return rc;
+    if ((rc = check_T(cfg, T))) return rc;
+    if (T == 0) return BEAM_MOE_OK;
+    if (!x || !w_router || !y || !ws) return BEAM_MOE_ERR_NULL;
+    if ((rc = weights_status(W))) return rc;
+    if (!aligned16(x) || !aligned16(w_router) || !aligned16(y) || !aligned16(ws)) return BEAM_MOE_ERR_MISALIGNED;
     const Layout L = layout(cfg, T, BEAM_MOE_WS_FORWARD);
     if (ws_bytes < L.total) return BEAM_MOE_ERR_WORKSPACE_TOO_SMALL;
-    if (T == 0) return BEAM_MOE_OK;
     int dev;
     if ((rc = init_device(&dev))) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -433,29 +514,55 @@ int forward_impl(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, cons
     if (!record(ev, 0, s)) return BEAM_MOE_ERR_CUDA;
     if ((rc = enqueue_route(cfg, T, x, w_router, sel_bias, ids, w, s))) return rc;
     if (!record(ev, 1, s)) return BEAM_MOE_ERR_CUDA;
-    return enqueue_experts(cfg, dev, T, x, ids, w, w_gate, w_up, w_down, y, wsb, L, s, ev);
+    return enqueue_experts(cfg, dev, T, x, ids, w, W, y, wsb, L, s, ev);
+}
+
+bool events_ok(void *const *events) {
+    if (!events) return false;
+    for (int i = 0; i < 7; ++i)
+        if (!events[i]) return false;
+    return true;
 }
 }  // namespace
 }  // namespace beam
 
 extern "C" {
 
+int beam_moe_experts(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const int32_t *topk_ids,
+                     const float *topk_w, const beam_bf16 *w_gate, const beam_bf16 *w_up, const beam_bf16 *w_down,
+                     beam_bf16 *y, void *ws, size_t ws_bytes, void *stream) {
+    return experts_impl(cfg, T, x, topk_ids, topk_w, bf16_weights(w_gate, w_up, w_down), y, ws, ws_bytes, stream);
+}
+
+int beam_moe_experts_fp8(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const int32_t *topk_ids,
+                         const float *topk_w, const beam_moe_fp8_experts *w8, beam_bf16 *y, void *ws, size_t ws_bytes,
+                         void *stream) {
+    if (!w8) return BEAM_MOE_ERR_NULL;
+    return experts_impl(cfg, T, x, topk_ids, topk_w, fp8_weights(w8), y, ws, ws_bytes, stream);
+}
+
 int beam_moe_forward(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const float *w_router,
                      const float *sel_bias, const beam_bf16 *w_gate, const beam_bf16 *w_up, const beam_bf16 *w_down,
                      beam_bf16 *y, int32_t *topk_ids_out, float *topk_w_out, void *ws, size_t ws_bytes, void *stream) {
-    return forward_impl(cfg, T, x, w_router, sel_bias, w_gate, w_up, w_down, y, topk_ids_out, topk_w_out, ws,
-                        ws_bytes, stream, nullptr);
+    return forward_impl(cfg, T, x, w_router, sel_bias, bf16_weights(w_gate, w_up, w_down), y, topk_ids_out,
+                        topk_w_out, ws, ws_bytes, stream, nullptr);
 }
 
 int beam_moe_forward_profiled(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const float *w_router,
                               const float *sel_bias, const beam_bf16 *w_gate, const beam_bf16 *w_up,
                               const beam_bf16 *w_down, beam_bf16 *y, int32_t *topk_ids_out, float *topk_w_out,
                               void *ws, size_t ws_bytes, void *stream, void *const *events) {
-    if (!events) return BEAM_MOE_ERR_NULL;
-    for (int i = 0; i < 7; ++i)
-        if (!events[i]) return BEAM_MOE_ERR_NULL;
-    return forward_impl(cfg, T, x, w_router, sel_bias, w_gate, w_up, w_down, y, topk_ids_out, topk_w_out, ws,
-                        ws_bytes, stream, reinterpret_cast<cudaEvent_t const *>(events));
+    if (!events_ok(events)) return BEAM_MOE_ERR_NULL;
+    return forward_impl(cfg, T, x, w_router, sel_bias, bf16_weights(w_gate, w_up, w_down), y, topk_ids_out,
+                        topk_w_out, ws, ws_bytes, stream, reinterpret_cast<cudaEvent_t const *>(events));
+}
+
+int beam_moe_forward_fp8(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const float *w_router,
+                         const float *sel_bias, const beam_moe_fp8_experts *w8, beam_bf16 *y, int32_t *topk_ids_out,
+                         float *topk_w_out, void *ws, size_t ws_bytes, void *stream, void *const *events) {
+    if (!w8 || (events && !events_ok(events))) return BEAM_MOE_ERR_NULL;
+    return forward_impl(cfg, T, x, w_router, sel_bias, fp8_weights(w8), y, topk_ids_out, topk_w_out, ws, ws_bytes,
+                        stream, reinterpret_cast<cudaEvent_t const *>(events));
 }
 
 int beam_moe_device_status(void *stream) {
@@ -533,7 +640,8 @@ extern "C" int beam_moe_block_forward(const beam_moe_config *cfg, const beam_moe
     const double k = sub->step;
     const BlockTail tail{stream_in, sub->post_norm_weight, sub->eps, static_cast<float>(std::sqrt((k - 1.0) / k)),
                          static_cast<float>(1.0 / std::sqrt(k))};
-    return enqueue_experts(cfg, dev, T, u, ids, w, w_gate, w_up, w_down, stream_out, wsb, L, s, nullptr, &tail);
+    return enqueue_experts(cfg, dev, T, u, ids, w, bf16_weights(w_gate, w_up, w_down), stream_out, wsb, L, s, nullptr,
+                           &tail);
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -624,9 +732,9 @@ extern "C" int beam_moe_dense_swiglu(int32_t hidden, int32_t inter, int64_t T, c
     const int grid = g_dev[dev].num_sms;
     GemmParams p1{counts, offsets, h, 1, hidden, inter, 0, kDefaultTimeoutCycles, nullptr, 1};
     GemmParams p2{counts, offsets, o, 1, inter, hidden, 0, kDefaultTimeoutCycles, nullptr, 1};
-    G1_WIDE_KERNEL<<<grid, kGemmThreads, G1Wide::kSmem, s>>>(m_wg, m_wu, m_x, p1);
+    launch_gemm<G1_WIDE_ARGS>(grid, s, m_wg, m_wu, m_x, p1);
     if ((rc = launch_status())) return rc;
-    G2_WIDE_KERNEL<<<grid, kGemmThreads, G2Wide::kSmem, s>>>(m_wd, m_wd, m_h, p2);
+    launch_gemm<G2_WIDE_ARGS>(grid, s, m_wd, m_wd, m_h, p2);
     if ((rc = launch_status())) return rc;
     const int64_t n4 = T * static_cast<int64_t>(hidden) / 4;
     f32_to_bf16_kernel<<<static_cast<unsigned>(std::min<int64_t>((n4 + 255) / 256, 16384)), 256, 0, s>>>(

@@ -97,10 +97,89 @@ __device__ __forceinline__ Item decode_item(int item, const int *tile_start, int
     return it;
 }
 
+// Per-expert item counts -> exclusive prefix in tile_start[0..E] (E <= 256 <= blockDim.x, which is a
+// multiple of 32 and at most 1024).  Contains __syncthreads: every thread of the block calls it.
+__device__ __forceinline__ void item_prefix(const int32_t *counts, int E, int n_mt, int BN, int *tile_start) {
+    __shared__ int warp_tot[32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e = threadIdx.x;
+    const int v = e < E ? n_mt * ((counts[e] + BN - 1) / BN) : 0;
+    int incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int base = 0;
+    for (int w = 0; w < warp; ++w) base += warp_tot[w];
+    if (e < E) tile_start[e] = base + incl - v;
+    if (e == E - 1) tile_start[E] = base + incl;
+}
+
 // TMEM slots an item occupies.
 template <bool GATE_UP, int SLOT_COLS>
 __device__ __forceinline__ int slots_of(int n_mma) {
     return (GATE_UP && n_mma > SLOT_COLS / 2) ? 2 : 1;
+}
+
+// Epilogue (warps 4..7; q = warp - 4 reads TMEM lanes 32q..32q+31): per item, wait for its
+// accumulator slot(s), then write G1: h = bf16(SiLU(gate) * up) or G2: o = fp32 accumulator for the
+// item's rows, and release the slot(s).
+template <bool GATE_UP, int BN, int NSLOT, int SLOT_COLS>
+__device__ __forceinline__ void gemm_epilogue(int q, const int *tile_start, int total, const GemmParams &p,
+                                              uint32_t tmem_base, uint64_t *acc_full, uint64_t *acc_empty) {
+    const int lane = threadIdx.x & 31;
+    const int E = p.E;
+    uint32_t uses = 0;
+    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+        const Item it = decode_item(item, tile_start, E, BN, p.counts, p.offsets);
+        const int u = slots_of<GATE_UP, SLOT_COLS>(it.n_mma);
+        bool ok = true;
+        for (int i = 0; i < u && ok; ++i) {
+            const uint32_t c = uses + i;
+            ok = mbar_wait(&acc_full[c % NSLOT], (c / NSLOT) & 1u, p.timeout);
+        }
+        if (!ok) break;
+        tc_fence_after();
+        const int s0 = uses % NSLOT, s1 = (uses + 1) % NSLOT;
+        const int m = it.mt * kBM + q * 32 + lane;  // weight row of this thread
+        const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+        const uint32_t t0 = tmem_base + lane_off + static_cast<uint32_t>(s0 * SLOT_COLS);
+        const uint32_t t1 = tmem_base + lane_off +
+                            static_cast<uint32_t>(u == 2 ? s1 * SLOT_COLS : s0 * SLOT_COLS + SLOT_COLS / 2);
+        for (int c = 0; c < it.n_valid; c += 16) {
+            uint32_t r0[16];
+            tmem_ld16(t0 + c, r0);
+            if (GATE_UP) {
+                uint32_t r1[16];
+                tmem_ld16(t1 + c, r1);
+                tmem_ld_wait();
+                if (m < p.M) {
+                    __nv_bfloat16 *h = reinterpret_cast<__nv_bfloat16 *>(p.out);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        if (c + j < it.n_valid)
+                            h[(it.row0 + c + j) * p.M + m] =
+                                __float2bfloat16_rn(silu_mul(__uint_as_float(r0[j]), __uint_as_float(r1[j])));
+                }
+            } else {
+                tmem_ld_wait();
+                if (m < p.M) {
+                    float *o = reinterpret_cast<float *>(p.out);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        if (c + j < it.n_valid) o[(it.row0 + c + j) * p.M + m] = __uint_as_float(r0[j]);
+                }
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0)
+            for (int i = 0; i < u; ++i) mbar_arrive(&acc_empty[(uses + i) % NSLOT]);
+        uses += u;
+    }
 }
 
 template <bool GATE_UP, int BN, int BOXN, int STAGES, int NSLOT, int SLOT_COLS, bool GATHER = false>
@@ -146,24 +225,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_alloc(tmem_slot, C::kTmemCols);
         tmem_relinquish();
     }
-    // per-expert item counts -> exclusive prefix (E <= 256 = blockDim.x)
-    {
-        __shared__ int warp_tot[kGemmThreads / 32];
-        const int e = threadIdx.x;
-        const int v = e < E ? n_mt * ((p.counts[e] + BN - 1) / BN) : 0;
-        int incl = v;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int o = __shfl_up_sync(0xffffffffu, incl, off);
-            if (lane >= off) incl += o;
-        }
-        if (lane == 31) warp_tot[warp] = incl;
-        __syncthreads();
-        int base = 0;
-        for (int w = 0; w < warp; ++w) base += warp_tot[w];
-        if (e < E) tile_start[e] = base + incl - v;
-        if (e == E - 1) tile_start[E] = base + incl;
-    }
+    item_prefix(p.counts, E, n_mt, BN, tile_start);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -278,56 +340,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_wait(drain, 0, p.timeout);
         }
     } else if (warp >= 4) {
-        // ---------------- epilogue ----------------
-        const int q = warp - 4;  // TMEM lane quadrant
-        uint32_t uses = 0;
-        for (int item = blockIdx.x; item < total; item += gridDim.x) {
-            const Item it = decode_item(item, tile_start, E, BN, p.counts, p.offsets);
-            const int u = slots_of<GATE_UP, SLOT_COLS>(it.n_mma);
-            bool ok = true;
-            for (int i = 0; i < u && ok; ++i) {
-                const uint32_t c = uses + i;
-                ok = mbar_wait(&acc_full[c % NSLOT], (c / NSLOT) & 1u, p.timeout);
-            }
-            if (!ok) break;
-            tc_fence_after();
-            const int s0 = uses % NSLOT, s1 = (uses + 1) % NSLOT;
-            const int m = it.mt * kBM + q * 32 + lane;  // weight row of this thread
-            const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
-            const uint32_t t0 = tmem_base + lane_off + static_cast<uint32_t>(s0 * SLOT_COLS);
-            const uint32_t t1 = tmem_base + lane_off +
-                                static_cast<uint32_t>(u == 2 ? s1 * SLOT_COLS : s0 * SLOT_COLS + SLOT_COLS / 2);
-            for (int c = 0; c < it.n_valid; c += 16) {
-                uint32_t r0[16];
-                tmem_ld16(t0 + c, r0);
-                if (GATE_UP) {
-                    uint32_t r1[16];
-                    tmem_ld16(t1 + c, r1);
-                    tmem_ld_wait();
-                    if (m < p.M) {
-                        __nv_bfloat16 *h = reinterpret_cast<__nv_bfloat16 *>(p.out);
-#pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            if (c + j < it.n_valid)
-                                h[(it.row0 + c + j) * p.M + m] =
-                                    __float2bfloat16_rn(silu_mul(__uint_as_float(r0[j]), __uint_as_float(r1[j])));
-                    }
-                } else {
-                    tmem_ld_wait();
-                    if (m < p.M) {
-                        float *o = reinterpret_cast<float *>(p.out);
-#pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            if (c + j < it.n_valid) o[(it.row0 + c + j) * p.M + m] = __uint_as_float(r0[j]);
-                    }
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                for (int i = 0; i < u; ++i) mbar_arrive(&acc_empty[(uses + i) % NSLOT]);
-            uses += u;
-        }
+        gemm_epilogue<GATE_UP, BN, NSLOT, SLOT_COLS>(warp - 4, tile_start, total, p, tmem_base, acc_full, acc_empty);
     }
     tc_fence_before();
     __syncthreads();

@@ -198,6 +198,50 @@ BEAM_MOE_API int beam_moe_forward_profiled(const beam_moe_config *cfg, int64_t T
                                            void *stream, void *const *events);
 
 /*
+ * FP8 expert weights.  The "Welcome Beam" page (TL;DR, "Checkpoint formats") lists BF16, FP8 and
+ * NVFP4 checkpoints but gives no quantisation recipe.  This library reads FP8 as the OCP MXFP8
+ * layout: E4M3 element codes (sign, 4-bit exponent with bias 7, 3-bit mantissa; exponent 0 is
+ * subnormal, m * 2^-9; 0x7f / 0xff are NaN) with one UE8M0 scale code c per 32 consecutive K
+ * elements of a weight row, the scale being 2^(c - 127) (c = 255 is NaN).  The dequantised weight
+ *   W[e][row][k] = e4m3(w[e][row][k]) * 2^(scale[e][k / 32][row] - 127)
+ * has at most 4 significant bits, so it is exactly a bf16 value whenever it lies in bf16's normal
+ * range; the kernels rebuild those bf16 values in shared memory and run the same tensor-core path
+ * as the bf16 weights, so results equal the bf16 entry points given the dequantised weights.
+ * Codes that are NaN give undefined results.  Scales are stored K-block-major (all rows of one
+ * 32-wide K block together), a layout of this library:
+ *   w_gate [E, I, H] u8    w_gate_scale [E, H/32, I] u8
+ *   w_up   [E, I, H] u8    w_up_scale   [E, H/32, I] u8
+ *   w_down [E, H, I] u8    w_down_scale [E, I/32, H] u8
+ * All six pointers are device memory, owned by the caller, 16-byte aligned.
+ */
+typedef struct beam_moe_fp8_experts {
+    const uint8_t *w_gate;
+    const uint8_t *w_gate_scale;
+    const uint8_t *w_up;
+    const uint8_t *w_up_scale;
+    const uint8_t *w_down;
+    const uint8_t *w_down_scale;
+} beam_moe_fp8_experts;
+
+/*
+ * beam_moe_experts with FP8 expert weights (beam_moe_fp8_experts).  Same workspace
+ * (BEAM_MOE_WS_EXPERTS), outputs and error codes; `w8` NULL -> BEAM_MOE_ERR_NULL.
+ */
+BEAM_MOE_API int beam_moe_experts_fp8(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x,
+                                      const int32_t *topk_ids, const float *topk_w, const beam_moe_fp8_experts *w8,
+                                      beam_bf16 *y, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * beam_moe_forward with FP8 expert weights: routing (unchanged: FP32 router weights), dispatch,
+ * FP8 experts, combine.  Same workspace (BEAM_MOE_WS_FORWARD), outputs and error codes.
+ * `events` is NULL, or 7 events recorded as by beam_moe_forward_profiled.
+ */
+BEAM_MOE_API int beam_moe_forward_fp8(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x,
+                                      const float *w_router, const float *sel_bias, const beam_moe_fp8_experts *w8,
+                                      beam_bf16 *y, int32_t *topk_ids_out, float *topk_w_out, void *ws,
+                                      size_t ws_bytes, void *stream, void *const *events);
+
+/*
  * beam_moe_permute without a workspace: the same dispatch (identical outputs), with its scratch in
  * a fixed device array inside this library instead of caller memory.  The Beam pages have no
  * counterpart; this exists for callers that cannot allocate device memory when they enqueue work,

@@ -36,3 +36,10 @@ def beam_weights():
     import beam_synth as bs
     wg, wu, wd = bs.make_experts(bs.WORKLOADS["prefill"], device="cuda")
     return wg, wu, wd
+
+
+@pytest.fixture(scope="session")
+def beam_weights_fp8(beam_weights):
+    """MXFP8 copy of the shared Beam layer's expert weights (10 GB codes + scales) on cuda:0."""
+    import beam_synth as bs
+    return bs.quantize_experts(*beam_weights)

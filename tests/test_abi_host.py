@@ -111,3 +111,37 @@ def test_block_rejects_bad_sublayer_on_host(L):
     assert L.beam_moe_block_forward(ctypes.byref(c), None, 4, p, p, None, p, p, p, p, None, None, None, p, 1 << 40,
                                     None) == bm.ERR_NULL
     assert bm.workspace_size(c, 4096, bm.WS_BLOCK) == bm.workspace_size(c, 4096, bm.WS_FORWARD) + 4096 * 5120 * 2
+
+
+def test_fp8_entry_points_check_arguments_on_host(L):
+    c = _cfg()
+    p, mis = 4096, 4104
+    need = bm.workspace_size(c, 64, bm.WS_FORWARD)
+    good = bm.BeamMoeFp8Experts(p, p, p, p, p, p)
+    q = ctypes.c_void_p(p)
+    assert L.beam_moe_forward_fp8(ctypes.byref(c), 64, q, q, None, None, q, None, None, q, need, None, None) == \
+        bm.ERR_NULL
+    assert L.beam_moe_experts_fp8(ctypes.byref(c), 64, q, q, q, None, q, q, need, None) == bm.ERR_NULL
+    for i in range(6):  # each of the six weight / scale pointers
+        vals = [p] * 6
+        vals[i] = 0
+        w8 = bm.BeamMoeFp8Experts(*vals)
+        assert L.beam_moe_forward_fp8(ctypes.byref(c), 64, q, q, None, ctypes.byref(w8), q, None, None, q, need,
+                                      None, None) == bm.ERR_NULL
+        vals[i] = mis
+        w8 = bm.BeamMoeFp8Experts(*vals)
+        assert L.beam_moe_forward_fp8(ctypes.byref(c), 64, q, q, None, ctypes.byref(w8), q, None, None, q, need,
+                                      None, None) == bm.ERR_MISALIGNED
+        assert L.beam_moe_experts_fp8(ctypes.byref(c), 64, q, q, q, ctypes.byref(w8), q, q, need, None) == \
+            bm.ERR_MISALIGNED
+    assert L.beam_moe_forward_fp8(ctypes.byref(c), 64, q, q, None, ctypes.byref(good), q, None, None, q, need - 1,
+                                  None, None) == bm.ERR_WORKSPACE_TOO_SMALL
+    bad = _cfg(hidden=96)
+    assert L.beam_moe_experts_fp8(ctypes.byref(bad), 64, q, q, q, ctypes.byref(good), q, q, need, None) == \
+        bm.ERR_INVALID_CONFIG
+    # events: NULL (no profiling) or 7 valid handles
+    ev = (ctypes.c_void_p * 7)()
+    assert L.beam_moe_forward_fp8(ctypes.byref(c), 64, q, q, None, ctypes.byref(good), q, None, None, q, need,
+                                  None, ev) == bm.ERR_NULL
+    assert L.beam_moe_forward_fp8(ctypes.byref(c), 0, q, q, None, ctypes.byref(good), q, None, None, None, 0,
+                                  None, None) == bm.OK
