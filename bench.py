@@ -41,15 +41,15 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # captured from hash the same; otherwise the JSON line reports null.
 _CSRC = os.path.join(ROOT, "group_limited_routing_router_b200", "csrc")
 NCU_TRAFFIC = {
-    ("gate_up_swiglu", "prefill"): {"bytes": 14137922816 + 151317504, "files": ("gemm.cuh", "common.cuh"),
-                                    "hash": "d598baf939e79caa"},
-    ("down", "prefill"): {"bytes": 7060850432 + 620517632, "files": ("gemm.cuh", "common.cuh"),
-                          "hash": "d598baf939e79caa"},
-    ("gate_up_swiglu_fp8", "prefill"): {"bytes": 8140484864 + 149472000,
+    ("gate_up_swiglu", "prefill"): {"bytes": 14067322368 + 151537152, "files": ("gemm.cuh", "common.cuh"),
+                                    "hash": "22b37ecce7f0f5cc"},
+    ("down", "prefill"): {"bytes": 7047173120 + 620304384, "files": ("gemm.cuh", "common.cuh"),
+                          "hash": "22b37ecce7f0f5cc"},
+    ("gate_up_swiglu_fp8", "prefill"): {"bytes": 8139558144 + 150100224,
                                         "files": ("gemm_fp8.cuh", "gemm.cuh", "common.cuh"),
-                                        "hash": "203a6b9373e1eec4"},
-    ("down_fp8", "prefill"): {"bytes": 3993288960 + 618224640, "files": ("gemm_fp8.cuh", "gemm.cuh", "common.cuh"),
-                              "hash": "203a6b9373e1eec4"},
+                                        "hash": "f225f76d4d9105b4"},
+    ("down_fp8", "prefill"): {"bytes": 3970746368 + 618352896, "files": ("gemm_fp8.cuh", "gemm.cuh", "common.cuh"),
+                              "hash": "f225f76d4d9105b4"},
 }
 
 
