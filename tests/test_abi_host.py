@@ -145,3 +145,14 @@ def test_fp8_entry_points_check_arguments_on_host(L):
                                   None, ev) == bm.ERR_NULL
     assert L.beam_moe_forward_fp8(ctypes.byref(c), 0, q, q, None, ctypes.byref(good), q, None, None, None, 0,
                                   None, None) == bm.OK
+
+
+def test_fp8_binding_refuses_bad_inputs_on_host(L):
+    import torch
+    x = torch.zeros(4, 5120, dtype=torch.bfloat16)
+    with pytest.raises(KeyError):
+        bm._fp8_experts(bm.BEAM_LAYER.c(), {"q_gate": None})
+    with pytest.raises(TypeError):
+        bm.forward_fp8(bm.BEAM_LAYER, x, torch.zeros(256, 5120), None, {})
+    with pytest.raises(TypeError):
+        bm.experts_fp8(bm.BEAM_LAYER, x, torch.zeros(4, 8, dtype=torch.int32), torch.zeros(4, 8), {})
