@@ -259,3 +259,51 @@ def quantize_experts(wg: torch.Tensor, wu: torch.Tensor, wd: torch.Tensor):
     for name, w in (("gate", wg), ("up", wu), ("down", wd)):
         out["q_" + name], out["s_" + name] = quantize_mxfp8(w)
     return out
+
+
+_E2M1_MID = torch.tensor([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+
+
+def _e2m1_codes(v: torch.Tensor) -> torch.Tensor:
+    """Round to the nearest E2M1 value (0, 0.5, 1, 1.5, 2, 3, 4, 6; ties to the even code) -> 4-bit codes."""
+    a = v.abs().clamp(max=6.0)
+    mid = _E2M1_MID.to(v.device)
+    lower = (a.unsqueeze(-1) > mid).sum(-1)                       # codes 0..7 by strict midpoints
+    tie = (lower < 7) & (a == mid[lower.clamp(max=6)])
+    code = lower + (tie & (lower % 2 == 1)).to(lower.dtype)
+    return (code | ((v < 0).to(code.dtype) << 3)).to(torch.uint8)
+
+
+def quantize_nvfp4(w: torch.Tensor):
+    """Synthetic NVFP4 checkpoint: w [n, rows, K] (bf16) -> (q [n, rows, K/2] uint8, two E2M1 codes per
+    byte, even k in the low nibble; scale [n, K/16, rows] E4M3 codes; global [n] fp32).
+
+    Input preparation only (NVIDIA's NVFP4 layout): per matrix a global scale amax / (6 * 448); per
+    block of 16 consecutive K elements an E4M3 scale amax_block / (6 * global), rounded to nearest
+    even; elements rounded to the nearest E2M1 value of w / (scale * global)."""
+    n, rows, K = w.shape
+    assert K % 16 == 0
+    if n > 8:  # bound the FP32 temporaries: a few matrices at a time
+        parts = [quantize_nvfp4(w[i:i + 8]) for i in range(0, n, 8)]
+        return tuple(torch.cat([p[j] for p in parts]) for j in range(3))
+    wf = w.float()
+    amax = wf.abs().amax(dim=(-1, -2))
+    glob = torch.where(amax > 0, amax / (6.0 * 448.0), torch.ones_like(amax))
+    blk = wf.reshape(n, rows, K // 16, 16)
+    s = (blk.abs().amax(-1) / (6.0 * glob[:, None, None])).clamp(max=448.0)
+    s_code = s.to(torch.float8_e4m3fn)
+    sv = s_code.float()
+    denom = (sv * glob[:, None, None]).unsqueeze(-1)
+    v = torch.where(denom > 0, blk / torch.where(denom > 0, denom, torch.ones_like(denom)), torch.zeros_like(blk))
+    codes = _e2m1_codes(v).reshape(n, rows, K)
+    q = (codes[..., 0::2] | (codes[..., 1::2] << 4)).contiguous()
+    scale = s_code.view(torch.uint8).transpose(-1, -2).contiguous()    # [n, K/16, rows]
+    return q, scale, glob.float()
+
+
+def quantize_experts_nvfp4(wg: torch.Tensor, wu: torch.Tensor, wd: torch.Tensor):
+    """quantize_nvfp4 of the three expert weight tensors: dict q_/s_/g_ for gate, up, down."""
+    out = {}
+    for name, w in (("gate", wg), ("up", wu), ("down", wd)):
+        out["q_" + name], out["s_" + name], out["g_" + name] = quantize_nvfp4(w)
+    return out

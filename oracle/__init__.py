@@ -61,6 +61,11 @@ def lib():
         L.oracle_dequant_mxfp8.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.POINTER(ctypes.c_uint8),
                                            ctypes.POINTER(ctypes.c_uint8), _u16p]
         L.oracle_dequant_mxfp8.restype = ctypes.c_int
+        L.oracle_dequant_nvfp4.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.POINTER(ctypes.c_uint8),
+                                           ctypes.POINTER(ctypes.c_uint8), ctypes.c_double, _dp]
+        L.oracle_dequant_nvfp4.restype = ctypes.c_int
+        L.oracle_expert_mlp_f64.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, _u16p, _dp, _dp, _dp, _dp]
+        L.oracle_expert_mlp_f64.restype = None
         _lib = L
     return _lib
 
@@ -265,3 +270,49 @@ def dequant_mxfp8(q: np.ndarray, scale: np.ndarray) -> np.ndarray:
     if lib().oracle_dequant_mxfp8(rows, K, q.ctypes.data_as(u8p), scale.ctypes.data_as(u8p), _ptr(out, _u16p)) != 0:
         raise ValueError("MXFP8 weights with a NaN code or a value bf16 cannot hold exactly")
     return out
+
+
+def dequant_nvfp4(q: np.ndarray, scale: np.ndarray, global_scale: float) -> np.ndarray:
+    """NVFP4 dequantisation to fp64: q [rows,K/2] packed E2M1 codes (even k in the low nibble),
+    scale [K/16,rows] E4M3 codes, one FP32 global scale."""
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    scale = np.ascontiguousarray(scale, dtype=np.uint8)
+    rows, K2 = q.shape
+    K = 2 * K2
+    assert scale.shape == (K // 16, rows)
+    out = np.empty((rows, K), dtype=np.float64)
+    u8p = ctypes.POINTER(ctypes.c_uint8)
+    if lib().oracle_dequant_nvfp4(rows, K, q.ctypes.data_as(u8p), scale.ctypes.data_as(u8p),
+                                  ctypes.c_double(float(global_scale)), _ptr(out, _dp)) != 0:
+        raise ValueError("NVFP4 scale code with the sign bit set, or NaN")
+    return out
+
+
+def expert_mlp_f64(x_rows_bits: np.ndarray, wg: np.ndarray, wu: np.ndarray, wd: np.ndarray) -> np.ndarray:
+    """SwiGLU expert on rows [n,H] (bf16 bits) with fp64 weights; returns [n,H] fp64."""
+    x_rows_bits = np.ascontiguousarray(x_rows_bits, dtype=np.uint16)
+    n, H = x_rows_bits.shape
+    I = wg.shape[0]
+    assert wg.shape == (I, H) and wu.shape == (I, H) and wd.shape == (H, I)
+    out = np.empty((n, H), dtype=np.float64)
+    if n == 0:
+        return out
+    lib().oracle_expert_mlp_f64(n, H, I, _ptr(x_rows_bits, _u16p),
+                                *(_ptr(np.ascontiguousarray(w, dtype=np.float64), _dp) for w in (wg, wu, wd)),
+                                _ptr(out, _dp))
+    return out
+
+
+def experts_tokens_f64(x_bits: np.ndarray, ids: np.ndarray, weight: np.ndarray, fetch,
+                       n_experts: int, routed_scale: float) -> np.ndarray:
+    """experts_tokens with fetch(e) returning fp64 weights (W_gate[e], W_up[e], W_down[e])."""
+    n, H = x_bits.shape
+    k = ids.shape[1]
+    out = np.zeros((n, k, H), dtype=np.float64)
+    for e in range(n_experts):
+        rows, slots = np.nonzero(ids == e)
+        if rows.size == 0:
+            continue
+        wg, wu, wd = fetch(e)
+        out[rows, slots, :] = expert_mlp_f64(x_bits[rows], wg, wu, wd)
+    return combine(out, weight, routed_scale)

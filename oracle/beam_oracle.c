@@ -362,3 +362,81 @@ int oracle_dequant_mxfp8(int64_t rows, int K, const uint8_t *q, const uint8_t *s
         }
     return bad ? -1 : 0;
 }
+
+/*
+ * NVFP4 expert weights ("Checkpoint formats: BF16, FP8, and NVFP4": "Welcome Beam" page, TL;DR;
+ * section "Hardware Requirements": the NVFP4 checkpoint keeps most parameters in 4 bits for
+ * Blackwell; the pages give no recipe).  Reading: NVIDIA's NVFP4 layout,
+ *   E2M1 elements: sign s, exponent e (2 bits, bias 1), mantissa m (1 bit); e = 0 is subnormal,
+ *                  m * 0.5; otherwise (1 + m/2) * 2^(e-1).  The 8 magnitudes: 0, 0.5, 1, 1.5, 2,
+ *                  3, 4, 6.
+ *   one E4M3 scale per 16 consecutive K elements of a weight row (a non-negative, finite code),
+ *   one FP32 scale per weight matrix.
+ * w[row][k] = e2m1(code(row, k)) * e4m3(scale[k/16][row]) * global, with two codes per byte:
+ * element k of a row is the low nibble of byte k/2 when k is even, the high nibble when k is odd.
+ * q [rows, K/2] uint8; scale [K/16, rows] uint8; out [rows, K] fp64.  Returns -1 (out undefined)
+ * for a scale code with the sign bit set or a NaN scale code.
+ */
+static double e2m1_value(uint8_t nibble)
+{
+    const int s = (nibble >> 3) & 1, e = (nibble >> 1) & 3, m = nibble & 1;
+    const double mag = e == 0 ? 0.5 * m : ldexp(1.0 + m / 2.0, e - 1);
+    return s ? -mag : mag;
+}
+
+int oracle_dequant_nvfp4(int64_t rows, int K, const uint8_t *q, const uint8_t *scale, double global,
+                         double *out)
+{
+    if (K % 16) return -1;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int k = 0; k < K; ++k) {
+            const uint8_t c = scale[(int64_t)(k / 16) * rows + r];
+            if (c & 0x80) return -1;
+            const double sv = e4m3_value(c);
+            if (isnan(sv)) return -1;
+            const uint8_t byte = q[r * (K / 2) + k / 2];
+            const uint8_t nib = (k & 1) ? (byte >> 4) : (byte & 15);
+            out[r * K + k] = e2m1_value(nib) * sv * global;
+        }
+    return 0;
+}
+
+/*
+ * The SwiGLU expert of oracle_expert_mlp with FP64 weights (for checkpoint formats whose
+ * dequantised weights are not bf16 values): out = Wd (SiLU(Wg x) * (Wu x)) per row, FP64.
+ * x_rows [n,H] bf16 bits; wg, wu [I,H] fp64; wd [H,I] fp64; out [n,H] fp64.
+ */
+void oracle_expert_mlp_f64(int64_t n, int H, int I, const uint16_t *x_rows, const double *wg,
+                           const double *wu, const double *wd, double *out)
+{
+    double *xd = (double *)malloc(sizeof(double) * (size_t)(n * H));
+    double *hd = (double *)malloc(sizeof(double) * (size_t)(n * I));
+    for (int64_t q = 0; q < n * H; ++q) xd[q] = bf16_bits_to_double(x_rows[q]);
+
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t r = 0; r < n; ++r)
+        for (int i = 0; i < I; ++i) {
+            const double *xr = xd + r * H;
+            const double *gr = wg + (int64_t)i * H;
+            const double *ur = wu + (int64_t)i * H;
+            double g = 0.0, u = 0.0;
+            for (int h = 0; h < H; ++h) {
+                g += gr[h] * xr[h];
+                u += ur[h] * xr[h];
+            }
+            const double act = g / (1.0 + exp(-g));  /* SiLU(g) */
+            hd[r * I + i] = act * u;
+        }
+
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t r = 0; r < n; ++r)
+        for (int o = 0; o < H; ++o) {
+            const double *hr = hd + r * I;
+            const double *dr = wd + (int64_t)o * I;
+            double acc = 0.0;
+            for (int i = 0; i < I; ++i) acc += dr[i] * hr[i];
+            out[r * H + o] = acc;
+        }
+    free(xd);
+    free(hd);
+}

@@ -14,6 +14,7 @@ import pytest
 
 import oracle
 from tests import test_oracle_fp8 as fp8
+from tests import test_oracle_nvfp4 as nv4
 from tests import test_oracle_norm_residual as nr
 from tests import test_oracle_pins as pins
 
@@ -47,6 +48,12 @@ MUTANTS = {
     "e4m3_bias_8": ("ldexp(1.0 + m / 8.0, e - 7)", "ldexp(1.0 + m / 8.0, e - 8)"),
     "e4m3_subnormal_exponent": ("ldexp((double)m, -9)", "ldexp((double)m, -10)"),
     "mxfp8_scale_row_major": ("scale[(int64_t)(k / 32) * rows + r]", "scale[r * (K / 32) + k / 32]"),
+    "e2m1_subnormal_quarter": ("e == 0 ? 0.5 * m :", "e == 0 ? 0.25 * m :"),
+    "e2m1_bias_0": ("ldexp(1.0 + m / 2.0, e - 1)", "ldexp(1.0 + m / 2.0, e)"),
+    "nvfp4_nibbles_swapped": ("(k & 1) ? (byte >> 4) : (byte & 15)", "(k & 1) ? (byte & 15) : (byte >> 4)"),
+    "nvfp4_scale_row_major": ("scale[(int64_t)(k / 16) * rows + r]", "scale[r * (K / 16) + k / 16]"),
+    "nvfp4_global_dropped": ("e2m1_value(nib) * sv * global", "e2m1_value(nib) * sv"),
+    "expert_f64_silu_missing": ("const double act = g / (1.0 + exp(-g));", "const double act = g;"),
 }
 
 PINS = [
@@ -65,6 +72,10 @@ PINS = [
     nr.test_every_addition_carries_equal_weight_after_104_steps,
     fp8.test_e4m3_decoder_matches_torch_for_all_codes,
     fp8.test_scale_is_a_power_of_two_per_32_block,
+    nv4.test_e2m1_decoder_all_codes_both_nibbles,
+    nv4.test_even_element_is_the_low_nibble,
+    nv4.test_block_scale_per_16_and_global_scale,
+    nv4.test_expert_mlp_f64_matches_torch_float64,
 ]
 
 
