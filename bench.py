@@ -34,6 +34,7 @@ import beam_synth as bs  # noqa: E402
 
 METRIC = "MoE-layer tokens/s (Beam shape, BF16, T=4096) and % of tensor/HBM roofline"
 METRIC_FP8 = "MoE-layer tokens/s (Beam shape, MXFP8 expert weights, T=4096) and % of tensor/HBM roofline"
+METRIC_NVFP4 = "MoE-layer tokens/s (Beam shape, NVFP4 expert weights, T=4096) and % of tensor/HBM roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture of the
@@ -74,6 +75,8 @@ def parse():
                     help="time the dense SwiGLU MLP of Beam's first layers (T=4096, intermediate 20480)")
     ap.add_argument("--block", action="store_true",
                     help="time the MoE sublayer on the residual stream (pre-norm, block, post-norm, residual)")
+    ap.add_argument("--nvfp4", action="store_true",
+                    help="NVFP4 expert weights (E2M1 + E4M3 scale per 16 K elements + FP32 per-matrix scale)")
     ap.add_argument("--fp8", action="store_true",
                     help="MXFP8 expert weights (E4M3 + one power-of-two scale per 32 K elements)")
     return ap.parse_args()
@@ -99,11 +102,13 @@ def kernel_source_hash() -> str:
 
 # ------------------------------------------------------------------------------------------------
 # algorithmic work (bytes the method must move, flops it must do), per step
-def algorithmic(wl: bs.Workload, n_act: int, fp8: bool = False) -> dict:
-    """fp8: expert weights are 1-byte E4M3 codes plus one 1-byte scale code per 32 elements."""
+def algorithmic(wl: bs.Workload, n_act: int, fmt: str = "bf16") -> dict:
+    """fmt "fp8": expert weights are 1-byte E4M3 codes plus one 1-byte scale code per 32 elements;
+    "nvfp4": half-byte E2M1 codes plus one 1-byte scale code per 16 elements (the per-matrix FP32
+    scales are negligible)."""
     T, H, I, E, k = wl.T, wl.hidden, wl.inter, wl.n_experts, wl.topk
     R = T * k
-    wb = 1.0 + 1.0 / 32 if fp8 else 2.0  # bytes per expert weight element
+    wb = {"bf16": 2.0, "fp8": 1.0 + 1.0 / 32, "nvfp4": 0.5 + 1.0 / 16}[fmt]  # bytes per expert weight element
     w_expert = 3 * H * I * wb
     return dict(
         layer_flops=T * (2 * H * E + k * 6 * H * I),
@@ -184,7 +189,14 @@ def fp8_fetch(w8):
                            for n in ("gate", "up", "down"))
 
 
-def cpu_oracle_rate(wl, x_cpu, W, bias, fetch, n_sample: int, route_all: bool = True) -> dict:
+def nvfp4_fetch(w4):
+    """One expert's weights for the oracle: NVFP4 codes dequantised to FP64 on the host by the oracle."""
+    import oracle
+    return lambda e: tuple(oracle.dequant_nvfp4(w4["q_" + n][e].cpu().numpy(), w4["s_" + n][e].cpu().numpy(),
+                                                float(w4["g_" + n][e].cpu())) for n in ("gate", "up", "down"))
+
+
+def cpu_oracle_rate(wl, x_cpu, W, bias, fetch, n_sample: int, route_all: bool = True, f64_weights: bool = False) -> dict:
     """Time the CPU oracle: routing (FP64 scores + selection) and the expert half on a token sample.
     fetch(e) gives one expert's bf16 weight bits on the host; it runs outside the timed sections."""
     import oracle
@@ -211,7 +223,7 @@ def cpu_oracle_rate(wl, x_cpu, W, bias, fetch, n_sample: int, route_all: bool = 
             continue
         w3 = fetch(e)
         t1 = time.perf_counter()
-        out[rows, slots, :] = oracle.expert_mlp(xs[rows], *w3)
+        out[rows, slots, :] = (oracle.expert_mlp_f64 if f64_weights else oracle.expert_mlp)(xs[rows], *w3)
         t_exp += time.perf_counter() - t1
     t1 = time.perf_counter()
     oracle.combine(out, wts, wl.routed_scale)
@@ -338,10 +350,11 @@ def run_ours(args):
     bias = None if b_cpu is None else b_cpu.cuda()
     wg, wu, wd = bs.make_experts(wl, device="cuda")
     w8 = None
-    if args.fp8:
+    fmt = "nvfp4" if args.nvfp4 else "fp8" if args.fp8 else "bf16"
+    if fmt != "bf16":
         if args.block:
-            raise SystemExit("--fp8 and --block: the sublayer entry point takes bf16 expert weights")
-        w8 = bs.quantize_experts(wg, wu, wd)
+            raise SystemExit("--fp8/--nvfp4 and --block: the sublayer entry point takes bf16 expert weights")
+        w8 = bs.quantize_experts(wg, wu, wd) if fmt == "fp8" else bs.quantize_experts_nvfp4(wg, wu, wd)
         del wg, wu, wd
         wg = wu = wd = None
         torch.cuda.empty_cache()
@@ -360,9 +373,12 @@ def run_ours(args):
         def step():
             bm.block_forward(layer, x, g_pre, g_post, 1e-6, block_step, W, bias, wg, wu, wd, stream_out=y, ids=ids,
                              w=w, ws=ws_blk)
-    elif args.fp8:
+    elif fmt == "fp8":
         def step():
             bm.forward_fp8(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws)
+    elif fmt == "nvfp4":
+        def step():
+            bm.forward_nvfp4(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws)
     else:
         def step():
             bm.forward(layer, x, W, bias, wg, wu, wd, y=y, ids=ids, w=w, ws=ws)
@@ -397,8 +413,10 @@ def run_ours(args):
     # per-stage device time from events recorded between the launches (same stream)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
     for i in range(args.steps):
-        if args.fp8:
+        if fmt == "fp8":
             bm.forward_fp8(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws, events=evs[i])
+        elif fmt == "nvfp4":
+            bm.forward_nvfp4(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws, events=evs[i])
         else:
             bm.forward_profiled(layer, x, W, bias, wg, wu, wd, evs[i], y, ids, w, ws)
     torch.cuda.synchronize()
@@ -424,13 +442,13 @@ def run_ours(args):
     e2e_value = ranks.rate(T * args.steps, e0.elapsed_time(e1))
     assert bm.device_status() == bm.OK
 
-    alg = algorithmic(wl, n_act, args.fp8)
+    alg = algorithmic(wl, n_act, fmt)
     pk, pk_kind = peaks()
     dom = max(stage_ms, key=stage_ms.get)
     dom_bytes = alg["stage_bytes"][dom]
     achieved = dom_bytes / (stage_ms[dom] / 1e3) / 1e9
     src_hash = kernel_source_hash()
-    tr = NCU_TRAFFIC.get((dom + ("_fp8" if args.fp8 else ""), wl.name))
+    tr = NCU_TRAFFIC.get((dom + ("" if fmt == "bf16" else "_" + fmt), wl.name))
     traffic = tr["bytes"] if tr and files_hash(tr["files"]) == tr["hash"] else None
     roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / pk["hbm_gbs"], "traffic": traffic, "peak_kind": pk_kind,
@@ -446,19 +464,27 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        fetch = fp8_fetch(w8) if args.fp8 else bf16_fetch(wg, wu, wd)
-        cpu = cpu_oracle_rate(wl, x_cpu, W_cpu, b_cpu, fetch, args.cpu_sample)
+        fetch = {"bf16": lambda: bf16_fetch(wg, wu, wd), "fp8": lambda: fp8_fetch(w8),
+                 "nvfp4": lambda: nvfp4_fetch(w8)}[fmt]()
+        cpu = cpu_oracle_rate(wl, x_cpu, W_cpu, b_cpu, fetch, args.cpu_sample, f64_weights=fmt == "nvfp4")
         cpu.pop("seconds", None)
 
     cfg = config_dict(wl)
-    if args.fp8:
+    if fmt == "fp8":
         cfg["weights"] = ("MXFP8 experts: E4M3 codes + UE8M0 scale per 32 K elements (1.03 B/weight), rebuilt "
-                          "as bf16 in shared memory; router FP32")
+                          "as bf16 in a TMEM ring; router FP32")
         cfg["weights_bytes"] = int(3 * wl.n_experts * wl.hidden * wl.inter * (1 + 1 / 32))
         cfg["l2"] = "no flush: every step streams the 10.4 GB of FP8 expert weights and scales (> 126 MB L2)"
-    line = {"metric": METRIC_FP8 if args.fp8 else METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+    elif fmt == "nvfp4":
+        cfg["weights"] = ("NVFP4 experts: E2M1 code pairs + E4M3 scale per 16 K elements + FP32 per-matrix scale "
+                          "(0.5625 B/weight), rebuilt as bf16 in a TMEM ring; router FP32")
+        cfg["weights_bytes"] = int(3 * wl.n_experts * wl.hidden * wl.inter * (0.5 + 1 / 16))
+        cfg["l2"] = "no flush: every step streams the 5.7 GB of NVFP4 expert weights and scales (> 126 MB L2)"
+    metric = {"bf16": METRIC, "fp8": METRIC_FP8, "nvfp4": METRIC_NVFP4}[fmt]
+    dtype = {"bf16": "bf16", "fp8": "fp8-e4m3 weights, bf16 MMA", "nvfp4": "nvfp4-e2m1 weights, bf16 MMA"}[fmt]
+    line = {"metric": metric, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "fp8-e4m3 weights, bf16 MMA" if args.fp8 else "bf16",
+            "scaling": "weak", "vs_baseline": None, "dtype": dtype,
             "data": "synthetic", "config": cfg,
             "roofline": roofline, "layer_roofline": layer_roof, "stage_ms": stage_ms, "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2,

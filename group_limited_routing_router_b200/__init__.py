@@ -53,6 +53,11 @@ class BeamMoeFp8Experts(ctypes.Structure):
                 ("w_up_scale", ctypes.c_void_p), ("w_down", ctypes.c_void_p), ("w_down_scale", ctypes.c_void_p)]
 
 
+class BeamMoeNvfp4Experts(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in ("w_gate", "w_gate_scale", "w_gate_global", "w_up", "w_up_scale",
+                                               "w_up_global", "w_down", "w_down_scale", "w_down_global")]
+
+
 @dataclasses.dataclass(frozen=True)
 class LayerConfig:
     hidden: int = 5120
@@ -105,6 +110,11 @@ def lib() -> ctypes.CDLL:
         L.beam_moe_experts_fp8.argtypes = [_cfgp, ctypes.c_int64, _vp, _vp, _vp, _f8p, _vp, _vp, ctypes.c_size_t, _vp]
         L.beam_moe_forward_fp8.argtypes = [_cfgp, ctypes.c_int64, _vp, _vp, _vp, _f8p, _vp, _vp, _vp, _vp,
                                            ctypes.c_size_t, _vp, ctypes.POINTER(ctypes.c_void_p)]
+        _f4p = ctypes.POINTER(BeamMoeNvfp4Experts)
+        L.beam_moe_experts_nvfp4.argtypes = [_cfgp, ctypes.c_int64, _vp, _vp, _vp, _f4p, _vp, _vp, ctypes.c_size_t,
+                                             _vp]
+        L.beam_moe_forward_nvfp4.argtypes = [_cfgp, ctypes.c_int64, _vp, _vp, _vp, _f4p, _vp, _vp, _vp, _vp,
+                                             ctypes.c_size_t, _vp, ctypes.POINTER(ctypes.c_void_p)]
         L.beam_moe_block_forward.argtypes = [_cfgp, ctypes.POINTER(BeamMoeSublayer), ctypes.c_int64, _vp, _vp, _vp,
                                              _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
         L.beam_moe_dense_workspace_size.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int64]
@@ -118,7 +128,8 @@ def lib() -> ctypes.CDLL:
         L.beam_moe_strerror.restype = ctypes.c_char_p
         for name in ("beam_moe_route", "beam_moe_permute", "beam_moe_experts", "beam_moe_forward",
                      "beam_moe_forward_profiled", "beam_moe_block_forward", "beam_moe_experts_fp8",
-                     "beam_moe_forward_fp8", "beam_moe_device_status",
+                     "beam_moe_forward_fp8", "beam_moe_experts_nvfp4", "beam_moe_forward_nvfp4",
+                     "beam_moe_device_status",
                      "beam_moe_selftest_timeout"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -327,6 +338,63 @@ def forward_fp8(cfg, x, w_router, bias, w8: dict, y=None, ids=None, w=None, ws=N
     _check(lib().beam_moe_forward_fp8(ctypes.byref(c), T, _ptr(x), _ptr(w_router), _ptr(bias), ctypes.byref(f8),
                                       _ptr(y), _ptr(ids), _ptr(w), _ptr(ws), nbytes, _stream(stream),
                                       _event_handles(events)), "beam_moe_forward_fp8")
+    return (y, ids, w) if return_routing else y
+
+
+NVFP4_KEYS = ("q_gate", "s_gate", "g_gate", "q_up", "s_up", "g_up", "q_down", "s_down", "g_down")
+
+
+def _nvfp4_experts(c: BeamMoeConfig, w4: dict) -> BeamMoeNvfp4Experts:
+    """NVFP4 expert weights: dict of CUDA tensors q_gate/q_up [E,I,H/2], q_down [E,H,I/2] (uint8, two E2M1
+    codes per byte, even k in the low nibble); s_gate/s_up [E,H/16,I], s_down [E,I/16,H] (uint8 E4M3
+    scale codes); g_gate/g_up/g_down [E] float32 (per-matrix scales)."""
+    E, H, I = c.n_experts, c.hidden, c.inter
+    shapes = dict(q_gate=(E, I, H // 2), q_up=(E, I, H // 2), q_down=(E, H, I // 2),
+                  s_gate=(E, H // 16, I), s_up=(E, H // 16, I), s_down=(E, I // 16, H),
+                  g_gate=(E,), g_up=(E,), g_down=(E,))
+    for k in NVFP4_KEYS:
+        if k not in w4:
+            raise KeyError(f"NVFP4 experts need '{k}'")
+        _dev(w4[k], k, torch.float32 if k.startswith("g_") else torch.uint8, shapes[k])
+    return BeamMoeNvfp4Experts(*(w4[k].data_ptr() for k in NVFP4_KEYS))
+
+
+def experts_nvfp4(cfg, x, ids, w, w4: dict, y=None, ws=None, stream=None) -> torch.Tensor:
+    """experts() with NVFP4 expert weights (see _nvfp4_experts for the layout)."""
+    c = _cfg(cfg)
+    T = x.shape[0]
+    _dev(x, "x", torch.bfloat16, (T, c.hidden))
+    _dev(ids, "ids", torch.int32, (T, c.topk))
+    _dev(w, "w", torch.float32, (T, c.topk))
+    f4 = _nvfp4_experts(c, w4)
+    y = torch.empty(T, c.hidden, dtype=torch.bfloat16, device=x.device) if y is None else y
+    _dev(y, "y", torch.bfloat16, (T, c.hidden))
+    ws, nbytes = _workspace(c, T, WS_EXPERTS, ws, x.device)
+    _check(lib().beam_moe_experts_nvfp4(ctypes.byref(c), T, _ptr(x), _ptr(ids), _ptr(w), ctypes.byref(f4), _ptr(y),
+                                        _ptr(ws), nbytes, _stream(stream)), "beam_moe_experts_nvfp4")
+    return y
+
+
+def forward_nvfp4(cfg, x, w_router, bias, w4: dict, y=None, ids=None, w=None, ws=None, stream=None,
+                  return_routing: bool = False, events=None):
+    """forward() with NVFP4 expert weights; `events` (7 torch.cuda.Event, optional) as in forward_profiled."""
+    c = _cfg(cfg)
+    T = x.shape[0]
+    _dev(x, "x", torch.bfloat16, (T, c.hidden))
+    _dev(w_router, "w_router", torch.float32, (c.n_experts, c.hidden))
+    _dev(bias, "bias", torch.float32, (c.n_experts,))
+    f4 = _nvfp4_experts(c, w4)
+    y = torch.empty(T, c.hidden, dtype=torch.bfloat16, device=x.device) if y is None else y
+    _dev(y, "y", torch.bfloat16, (T, c.hidden))
+    if return_routing:
+        ids = torch.empty(T, c.topk, dtype=torch.int32, device=x.device) if ids is None else ids
+        w = torch.empty(T, c.topk, dtype=torch.float32, device=x.device) if w is None else w
+    _dev(ids, "ids", torch.int32, (T, c.topk))
+    _dev(w, "w", torch.float32, (T, c.topk))
+    ws, nbytes = _workspace(c, T, WS_FORWARD, ws, x.device)
+    _check(lib().beam_moe_forward_nvfp4(ctypes.byref(c), T, _ptr(x), _ptr(w_router), _ptr(bias), ctypes.byref(f4),
+                                        _ptr(y), _ptr(ids), _ptr(w), _ptr(ws), nbytes, _stream(stream),
+                                        _event_handles(events)), "beam_moe_forward_nvfp4")
     return (y, ids, w) if return_routing else y
 
 

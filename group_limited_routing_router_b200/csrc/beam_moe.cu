@@ -43,10 +43,16 @@ constexpr int64_t kMaxTokens = int64_t(1) << 24;
 // slot columns, gather?, bf16 A ring stages in TMEM>.  The A ring takes the TMEM columns the
 // accumulators leave; the prefill gate/up variant gives its accumulators 2 slots of 192 columns
 // (one item of more than 96 tokens at a time) so that two A ring stages fit.
-#define G1_WIDE_FP8_ARGS true, 192, 64, 3, 4, 2, 192, false, 2
-#define G2_WIDE_FP8_ARGS false, 192, 64, 4, 5, 2, 192, false, 4
-#define G1_NARROW_FP8_ARGS true, 32, 1, 5, 12, 2, 64, true, 6
-#define G2_NARROW_FP8_ARGS false, 32, 32, 9, 16, 4, 32, false, 12
+#define G1_WIDE_FP8_ARGS true, 192, 64, 3, 4, 2, 192, false, 2, false
+#define G2_WIDE_FP8_ARGS false, 192, 64, 4, 5, 2, 192, false, 4, false
+#define G1_NARROW_FP8_ARGS true, 32, 1, 5, 12, 2, 64, true, 6, false
+#define G2_NARROW_FP8_ARGS false, 32, 32, 9, 16, 4, 32, false, 12, false
+// NVFP4 variants (last argument true): the same rings; a weight stage spans K = 256 (128 bytes of
+// E2M1 pairs per row) and its scale tiles are 8x larger, so they keep one stage fewer.
+#define G1_WIDE_NV4_ARGS true, 192, 64, 3, 4, 2, 192, false, 2, true
+#define G2_WIDE_NV4_ARGS false, 192, 64, 4, 5, 2, 192, false, 4, true
+#define G1_NARROW_NV4_ARGS true, 32, 1, 4, 12, 2, 64, true, 6, true
+#define G2_NARROW_NV4_ARGS false, 32, 32, 8, 16, 4, 32, false, 12, true
 constexpr int kWideBN = 192, kWideBox = 64, kNarrowBN = 32, kNarrowBox = 32;
 
 template <bool G, int BN, int BOXN, int ST, int NS, int SC, bool GA>
@@ -55,11 +61,11 @@ bool set_gemm_smem() {
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 GemmCfg<G, BN, BOXN, ST, NS, SC, GA>::kSmem) == cudaSuccess;
 }
-template <bool G, int BN, int BOXN, int W8, int BS, int NS, int SC, bool GA, int AS>
+template <bool G, int BN, int BOXN, int W8, int BS, int NS, int SC, bool GA, int AS, bool F4>
 bool set_gemm_fp8_smem() {
-    return cudaFuncSetAttribute(grouped_gemm_fp8_kernel<G, BN, BOXN, W8, BS, NS, SC, GA, AS>,
+    return cudaFuncSetAttribute(grouped_gemm_fp8_kernel<G, BN, BOXN, W8, BS, NS, SC, GA, AS, F4>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                Fp8GemmCfg<G, BN, BOXN, W8, BS, NS, SC, GA, AS>::kSmem) == cudaSuccess;
+                                Fp8GemmCfg<G, BN, BOXN, W8, BS, NS, SC, GA, AS, F4>::kSmem) == cudaSuccess;
 }
 
 // a1 is ignored by the down projection.
@@ -70,11 +76,12 @@ void launch_gemm(int grid, cudaStream_t s, const CUtensorMap &a0, const CUtensor
         <<<grid, kGemmThreads, GemmCfg<G, BN, BOXN, ST, NS, SC, GA>::kSmem, s>>>(a0, a1, b, p);
 }
 // a1 and s1 are ignored by the down projection.
-template <bool G, int BN, int BOXN, int W8, int BS, int NS, int SC, bool GA, int AS>
+template <bool G, int BN, int BOXN, int W8, int BS, int NS, int SC, bool GA, int AS, bool F4>
 void launch_gemm_fp8(int grid, cudaStream_t s, const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &s0,
-                     const CUtensorMap &s1, const CUtensorMap &b, const GemmParams &p) {
-    using C = Fp8GemmCfg<G, BN, BOXN, W8, BS, NS, SC, GA, AS>;
-    grouped_gemm_fp8_kernel<G, BN, BOXN, W8, BS, NS, SC, GA, AS><<<grid, C::kThreads, C::kSmem, s>>>(a0, a1, s0, s1, b, p);
+                     const CUtensorMap &s1, const CUtensorMap &b, const GemmParams &p, const AccScales &acc) {
+    using C = Fp8GemmCfg<G, BN, BOXN, W8, BS, NS, SC, GA, AS, F4>;
+    grouped_gemm_fp8_kernel<G, BN, BOXN, W8, BS, NS, SC, GA, AS, F4>
+        <<<grid, C::kThreads, C::kSmem, s>>>(a0, a1, s0, s1, b, p, acc);
 }
 
 // Tile family from the mean rows per expert (T*k/E): narrow when experts see a handful of tokens.
@@ -120,6 +127,8 @@ int init_device(int *dev_out) {
              set_gemm_smem<G1_NARROW_ARGS>() && set_gemm_smem<G2_NARROW_ARGS>();
         ok = ok && set_gemm_fp8_smem<G1_WIDE_FP8_ARGS>() && set_gemm_fp8_smem<G2_WIDE_FP8_ARGS>() &&
              set_gemm_fp8_smem<G1_NARROW_FP8_ARGS>() && set_gemm_fp8_smem<G2_NARROW_FP8_ARGS>();
+        ok = ok && set_gemm_fp8_smem<G1_WIDE_NV4_ARGS>() && set_gemm_fp8_smem<G2_WIDE_NV4_ARGS>() &&
+             set_gemm_fp8_smem<G1_NARROW_NV4_ARGS>() && set_gemm_fp8_smem<G2_NARROW_NV4_ARGS>();
         ok = ok && cudaFuncSetAttribute(combine_norm_residual_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         kMaxBlockHidden * 4) == cudaSuccess;
         if (!ok) d.status = BEAM_MOE_ERR_CUDA;
@@ -236,11 +245,18 @@ bool make_map_3d_fp8(CUtensorMap *m, const void *base, uint64_t K, uint64_t M, u
                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 3D [E][K/32][M] UE8M0 scale codes, box {128, 4, 1}: the four K blocks of one K = 128 stage.
-bool make_map_scale(CUtensorMap *m, const void *base, uint64_t M, uint64_t KB, uint64_t E) {
+// 3D [E][M][K/2] E2M1 code pairs, box {128 bytes, 128, 1}: K = 256 per box, 128-byte swizzle.
+bool make_map_3d_fp4(CUtensorMap *m, const void *base, uint64_t K, uint64_t M, uint64_t E) {
+    return make_map_3d_fp8(m, base, K / 2, M, E);
+}
+
+// 3D [E][K/blk][M] scale codes, box {128, kb_per_stage, 1}: the K blocks of one weight stage
+// (MXFP8: 4 blocks of 32 in K = 128; NVFP4: 16 blocks of 16 in K = 256).
+bool make_map_scale(CUtensorMap *m, const void *base, uint64_t M, uint64_t KB, uint64_t E,
+                    uint32_t kb_per_stage = 4) {
     const cuuint64_t dims[3] = {M, KB, E};
     const cuuint64_t strides[2] = {M, M * KB};
-    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kBM), 4, 1};
+    const cuuint32_t box[3] = {static_cast<cuuint32_t>(kBM), kb_per_stage, 1};
     const cuuint32_t estr[3] = {1, 1, 1};
     return encode_fn()(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void *>(base), dims, strides, box, estr,
                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -311,15 +327,17 @@ struct BlockTail {
     float eps, keep, add;
 };
 
-// The experts' weights: bf16 [E][rows][K], or E4M3 codes with their scale codes.
+// The experts' weights: bf16 [E][rows][K], E4M3 codes with their scale codes, or E2M1 code
+// pairs with their scale codes and per-matrix scales.
 struct ExpertWeights {
     const void *gate, *up, *down;
-    const uint8_t *s_gate, *s_up, *s_down;  // FP8 only: [E][K/32][rows]
-    bool fp8;
+    const uint8_t *s_gate, *s_up, *s_down;  // FP8: [E][K/32][rows]; FP4: [E][K/16][rows]
+    const float *g_gate, *g_up, *g_down;    // FP4 only: [E]
+    bool fp8, fp4;
 };
 
 ExpertWeights bf16_weights(const beam_bf16 *wg, const beam_bf16 *wu, const beam_bf16 *wd) {
-    return ExpertWeights{wg, wu, wd, nullptr, nullptr, nullptr, false};
+    return ExpertWeights{wg, wu, wd, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, false, false};
 }
 
 int enqueue_experts(const beam_moe_config *c, int dev, int64_t T, const beam_bf16 *x, const int32_t *ids,
@@ -357,7 +375,11 @@ int enqueue_experts(const beam_moe_config *c, int dev, int64_t T, const beam_bf1
     const bool b1_ok = narrow ? make_map_2d(&m_b1, x, H, static_cast<uint64_t>(T), 1)   // gather4 rows of x
                               : make_map_2d(&m_b1, ws + L.xp, H, R, box);              // tiled x_perm rows
     bool w_ok;
-    if (W.fp8) {
+    if (W.fp4) {
+        w_ok = make_map_3d_fp4(&m_wg, W.gate, H, I, E) && make_map_3d_fp4(&m_wu, W.up, H, I, E) &&
+               make_map_3d_fp4(&m_wd, W.down, I, H, E) && make_map_scale(&m_sg, W.s_gate, I, H / 16, E, 16) &&
+               make_map_scale(&m_su, W.s_up, I, H / 16, E, 16) && make_map_scale(&m_sd, W.s_down, H, I / 16, E, 16);
+    } else if (W.fp8) {
         w_ok = make_map_3d_fp8(&m_wg, W.gate, H, I, E) && make_map_3d_fp8(&m_wu, W.up, H, I, E) &&
                make_map_3d_fp8(&m_wd, W.down, I, H, E) && make_map_scale(&m_sg, W.s_gate, I, H / 32, E) &&
                make_map_scale(&m_su, W.s_up, I, H / 32, E) && make_map_scale(&m_sd, W.s_down, H, I / 32, E);
@@ -367,20 +389,29 @@ int enqueue_experts(const beam_moe_config *c, int dev, int64_t T, const beam_bf1
     }
     if (!b1_ok || !w_ok || !make_map_2d(&m_h, h, I, R, box)) return BEAM_MOE_ERR_CUDA;
     const int grid = g_dev[dev].num_sms;
+    // NVFP4: the rebuilt tiles hold e2m1 x scale x 2^-9; the per-matrix scales and 2^9 multiply the
+    // FP32 accumulators in the epilogue
     GemmParams p1{counts, offsets, h, E, H, I, once, kDefaultTimeoutCycles, row_src, k};
     GemmParams p2{counts, offsets, o, E, I, H, once, kDefaultTimeoutCycles, nullptr, k};
-    if (W.fp8) {
-        if (narrow) launch_gemm_fp8<G1_NARROW_FP8_ARGS>(grid, s, m_wg, m_wu, m_sg, m_su, m_b1, p1);
-        else launch_gemm_fp8<G1_WIDE_FP8_ARGS>(grid, s, m_wg, m_wu, m_sg, m_su, m_b1, p1);
+    const AccScales a1{W.g_gate, W.g_up, 512.0f}, a2{W.g_down, nullptr, 512.0f};
+    if (W.fp4) {
+        if (narrow) launch_gemm_fp8<G1_NARROW_NV4_ARGS>(grid, s, m_wg, m_wu, m_sg, m_su, m_b1, p1, a1);
+        else launch_gemm_fp8<G1_WIDE_NV4_ARGS>(grid, s, m_wg, m_wu, m_sg, m_su, m_b1, p1, a1);
+    } else if (W.fp8) {
+        if (narrow) launch_gemm_fp8<G1_NARROW_FP8_ARGS>(grid, s, m_wg, m_wu, m_sg, m_su, m_b1, p1, a1);
+        else launch_gemm_fp8<G1_WIDE_FP8_ARGS>(grid, s, m_wg, m_wu, m_sg, m_su, m_b1, p1, a1);
     } else {
         if (narrow) launch_gemm<G1_NARROW_ARGS>(grid, s, m_wg, m_wu, m_b1, p1);
         else launch_gemm<G1_WIDE_ARGS>(grid, s, m_wg, m_wu, m_b1, p1);
     }
     if ((rc = launch_status())) return rc;
     if (!record(ev, 4, s)) return BEAM_MOE_ERR_CUDA;
-    if (W.fp8) {
-        if (narrow) launch_gemm_fp8<G2_NARROW_FP8_ARGS>(grid, s, m_wd, m_wd, m_sd, m_sd, m_h, p2);
-        else launch_gemm_fp8<G2_WIDE_FP8_ARGS>(grid, s, m_wd, m_wd, m_sd, m_sd, m_h, p2);
+    if (W.fp4) {
+        if (narrow) launch_gemm_fp8<G2_NARROW_NV4_ARGS>(grid, s, m_wd, m_wd, m_sd, m_sd, m_h, p2, a2);
+        else launch_gemm_fp8<G2_WIDE_NV4_ARGS>(grid, s, m_wd, m_wd, m_sd, m_sd, m_h, p2, a2);
+    } else if (W.fp8) {
+        if (narrow) launch_gemm_fp8<G2_NARROW_FP8_ARGS>(grid, s, m_wd, m_wd, m_sd, m_sd, m_h, p2, a2);
+        else launch_gemm_fp8<G2_WIDE_FP8_ARGS>(grid, s, m_wd, m_wd, m_sd, m_sd, m_h, p2, a2);
     } else {
         if (narrow) launch_gemm<G2_NARROW_ARGS>(grid, s, m_wd, m_wd, m_h, p2);
         else launch_gemm<G2_WIDE_ARGS>(grid, s, m_wd, m_wd, m_h, p2);
@@ -465,15 +496,26 @@ namespace beam {
 namespace {
 // Argument checks of the experts' weights: every pointer set and 16-byte aligned.
 int weights_status(const ExpertWeights &W) {
+    const bool scaled = W.fp8 || W.fp4;
     if (!W.gate || !W.up || !W.down) return BEAM_MOE_ERR_NULL;
-    if (W.fp8 && (!W.s_gate || !W.s_up || !W.s_down)) return BEAM_MOE_ERR_NULL;
+    if (scaled && (!W.s_gate || !W.s_up || !W.s_down)) return BEAM_MOE_ERR_NULL;
+    if (W.fp4 && (!W.g_gate || !W.g_up || !W.g_down)) return BEAM_MOE_ERR_NULL;
     if (!aligned16(W.gate) || !aligned16(W.up) || !aligned16(W.down)) return BEAM_MOE_ERR_MISALIGNED;
-    if (W.fp8 && (!aligned16(W.s_gate) || !aligned16(W.s_up) || !aligned16(W.s_down))) return BEAM_MOE_ERR_MISALIGNED;
+    if (scaled && (!aligned16(W.s_gate) || !aligned16(W.s_up) || !aligned16(W.s_down))) return BEAM_MOE_ERR_MISALIGNED;
+    if (W.fp4 && ((reinterpret_cast<uintptr_t>(W.g_gate) | reinterpret_cast<uintptr_t>(W.g_up) |
+                   reinterpret_cast<uintptr_t>(W.g_down)) & 3u))
+        return BEAM_MOE_ERR_MISALIGNED;
     return BEAM_MOE_OK;
 }
 
 ExpertWeights fp8_weights(const beam_moe_fp8_experts *w8) {
-    return ExpertWeights{w8->w_gate, w8->w_up, w8->w_down, w8->w_gate_scale, w8->w_up_scale, w8->w_down_scale, true};
+    return ExpertWeights{w8->w_gate, w8->w_up, w8->w_down, w8->w_gate_scale, w8->w_up_scale, w8->w_down_scale,
+                         nullptr, nullptr, nullptr, true, false};
+}
+
+ExpertWeights nvfp4_weights(const beam_moe_nvfp4_experts *w4) {
+    return ExpertWeights{w4->w_gate, w4->w_up, w4->w_down, w4->w_gate_scale, w4->w_up_scale, w4->w_down_scale,
+                         w4->w_gate_global, w4->w_up_global, w4->w_down_global, false, true};
 }
 
 int experts_impl(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const int32_t *topk_ids,
@@ -539,6 +581,22 @@ int beam_moe_experts_fp8(const beam_moe_config *cfg, int64_t T, const beam_bf16 
                          void *stream) {
     if (!w8) return BEAM_MOE_ERR_NULL;
     return experts_impl(cfg, T, x, topk_ids, topk_w, fp8_weights(w8), y, ws, ws_bytes, stream);
+}
+
+int beam_moe_experts_nvfp4(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const int32_t *topk_ids,
+                           const float *topk_w, const beam_moe_nvfp4_experts *w4, beam_bf16 *y, void *ws,
+                           size_t ws_bytes, void *stream) {
+    if (!w4) return BEAM_MOE_ERR_NULL;
+    return experts_impl(cfg, T, x, topk_ids, topk_w, nvfp4_weights(w4), y, ws, ws_bytes, stream);
+}
+
+int beam_moe_forward_nvfp4(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const float *w_router,
+                           const float *sel_bias, const beam_moe_nvfp4_experts *w4, beam_bf16 *y,
+                           int32_t *topk_ids_out, float *topk_w_out, void *ws, size_t ws_bytes, void *stream,
+                           void *const *events) {
+    if (!w4 || (events && !events_ok(events))) return BEAM_MOE_ERR_NULL;
+    return forward_impl(cfg, T, x, w_router, sel_bias, nvfp4_weights(w4), y, topk_ids_out, topk_w_out, ws, ws_bytes,
+                        stream, reinterpret_cast<cudaEvent_t const *>(events));
 }
 
 int beam_moe_forward(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const float *w_router,

@@ -1,15 +1,20 @@
-// Grouped expert GEMMs with FP8 expert weights (MXFP8: E4M3 codes, one power-of-two UE8M0 scale
-// per 32 consecutive K elements of a weight row).  Same work items, orientation (swap-AB: weight
-// rows on the MMA's M side, the expert's tokens on N), accumulator slots and epilogue as the bf16
-// kernel in gemm.cuh; the tensor cores still multiply bf16 x bf16 into FP32.
-//
-// "Checkpoint formats: BF16, FP8, and NVFP4" ("Welcome Beam" page, TL;DR); the pages give no
-// quantisation recipe, so the layout is the OCP microscaling one, scales stored K-block-major.
+// Grouped expert GEMMs with block-scaled low-precision expert weights.  Same work items, orientation
+// (swap-AB: weight rows on the MMA's M side, the expert's tokens on N), accumulator slots and
+// epilogue as the bf16 kernel in gemm.cuh; the tensor cores still multiply bf16 x bf16 into FP32.
+//   FP8 (MXFP8): E4M3 codes, one power-of-two UE8M0 scale per 32 consecutive K elements.
+//   FP4 (NVFP4): E2M1 codes, two per byte (even k in the low nibble), one E4M3 scale per 16
+//     consecutive K elements, one FP32 scale per weight matrix.
+// "Checkpoint formats: BF16, FP8, and NVFP4" ("Welcome Beam" page, TL;DR; section "Hardware
+// Requirements": most parameters in 4 bits on Blackwell); the pages give no quantisation recipe,
+// so the layouts are the OCP microscaling and NVIDIA NVFP4 ones, scales stored K-block-major.
+// Both rebuild exact bf16 values: E4M3 x 2^k has at most 4 significant bits, E2M1 x E4M3 x 2^-9 at
+// most 6.  The NVFP4 per-matrix scale (times the 2^9) multiplies the FP32 accumulators in the
+// epilogue.
 //
 // Rings and roles (threads = 256 + 32 * converter warps):
-//   weight ring (W8STAGES): per stage the E4M3 A tile(s) of K = 128 (128 rows x 128 bytes, 128-byte
-//     swizzle: a weight row contributes 128 contiguous bytes, the piece size at which DRAM streams
-//     best) and their scale tiles [4 K-blocks][128 rows].  Warp 0 lane 0 loads it (TMA); the
+//   weight ring (W8STAGES): per stage the A tile(s) as 128 rows x 128 bytes (K = 128 of E4M3 or
+//     K = 256 of E2M1; 128-byte swizzle: a weight row contributes 128 contiguous bytes, the piece
+//     size at which DRAM streams best) and their scale tiles [K-blocks of the stage][128 rows].  Warp 0 lane 0 loads it (TMA); the
 //     converters release it as soon as they have read it, so the weight stream never waits on the
 //     tensor core.
 //   B ring (BSTAGES): one 64-wide k-step of the expert's token rows (tiled TMA boxes, or TMA
@@ -34,15 +39,17 @@ constexpr int round1024(int v) { return (v + 1023) / 1024 * 1024; }
 constexpr int fp8_gemm_threads(bool gate_up) { return 256 + 32 * kConvPerTile * (gate_up ? 2 : 1); }
 
 template <bool GATE_UP, int BN, int BOXN, int W8STAGES, int BSTAGES, int NSLOT, int SLOT_COLS, bool GATHER,
-          int ASTAGES>
+          int ASTAGES, bool FP4 = false>
 struct Fp8GemmCfg {
     static constexpr int kNumA = GATE_UP ? 2 : 1;
     static constexpr int kConvWarps = kConvPerTile * kNumA;
     static constexpr int kConvUnits = 8 / kConvPerTile;  // warp units per converter warp
     static constexpr int kThreads = fp8_gemm_threads(GATE_UP);
-    static constexpr int kK8 = 2 * kBK;                   // K per weight ring stage
-    static constexpr int kA8 = kBM * kK8;                 // one E4M3 A tile, bytes
-    static constexpr int kSc = (kK8 / 32) * kBM;          // one scale tile, bytes
+    static constexpr int kK8 = (FP4 ? 4 : 2) * kBK;       // K per weight ring stage
+    static constexpr int kSteps = kK8 / kBK;              // 64-wide k-steps per weight stage
+    static constexpr int kBlk = FP4 ? 16 : 32;            // K elements per scale code
+    static constexpr int kA8 = kBM * 128;                 // one A tile of the stage, bytes
+    static constexpr int kSc = (kK8 / kBlk) * kBM;        // one scale tile, bytes
     static constexpr int kScOff = kNumA * kA8;            // scale tiles after the A tiles
     static constexpr int kW8Stage = round1024(kNumA * (kA8 + kSc));
     static constexpr int kB = BN * kBK * 2;               // B tile of one 64-wide k-step
@@ -90,16 +97,106 @@ __device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t w, uint32_t f1, uint32
     hi = bf16x2_mul((b << 4) & 0x87F087F0u, f1);
 }
 
+// E2M1 -> bf16 by the same kind of integer rebuild.  For a code n = s ee m, the 16-bit pattern
+// s << 15 | (n & 7) << 6 read as bf16 has exponent field e and mantissa m000000: the value
+// e2m1(n) * 2^-126 (e = 0: m/2 * 2^-126, a bf16 subnormal).  For a byte holding codes n0 (low
+// nibble) and n1, lo * 0x1040 puts n0's magnitude at bits 6..8 and its sign at bit 15, and
+// hi * 0x01040000 puts n1's at bits 22..24 and 31; the two products use disjoint bits, and the
+// mask keeps those.  A bf16 multiply by the block scale s x 2^117 gives e2m1 x s x 2^-9, exact.
+__device__ __forceinline__ uint32_t e2m1x2_to_bf16x2(uint32_t byte, uint32_t f) {
+    const uint32_t pat = ((byte & 0x0Fu) * 0x1040u | (byte & 0xF0u) * 0x01040000u) & 0x81C081C0u;
+    return bf16x2_mul(pat, f);
+}
+// bf16x2 factor for an E4M3 block-scale code c (sign bit ignored): e4m3(c) x 2^117, exact (the
+// E4M3 value has at most 4 significant bits; 448 x 2^117 < 2^126).  (c & 0x7f) << 4 read as bf16 is
+// e4m3(c) x 2^-120, subnormal codes included; FP32 then multiplies by 2^118 and 2^119.
+__device__ __forceinline__ uint32_t e4m3_scale_factor(uint32_t c) {
+    float v = __uint_as_float(((c & 0x7Fu) << 4) << 16);
+    v *= 0x1p118f;
+    v *= 0x1p119f;
+    const uint32_t b = __float_as_uint(v) >> 16;
+    return b | (b << 16);
+}
+
+// Per-expert FP32 factors for the accumulators (NVFP4: the per-matrix scales times 2^9): A0 (gate or
+// down) and A1 (up), each multiplied by mul.
+struct AccScales {
+    const float *s0, *s1;
+    float mul;
+};
+
+// gemm_epilogue (gemm.cuh) with the accumulators first multiplied by the item's expert factors.
+template <bool GATE_UP, int BN, int NSLOT, int SLOT_COLS>
+__device__ __forceinline__ void gemm_epilogue_scaled(int q, const int *tile_start, int total, const GemmParams &p,
+                                                     const AccScales &acc, uint32_t tmem_base, uint64_t *acc_full,
+                                                     uint64_t *acc_empty) {
+    const int lane = threadIdx.x & 31;
+    const int E = p.E;
+    uint32_t uses = 0;
+    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+        const Item it = decode_item(item, tile_start, E, BN, p.counts, p.offsets);
+        const int u = slots_of<GATE_UP, SLOT_COLS>(it.n_mma);
+        bool ok = true;
+        for (int i = 0; i < u && ok; ++i) {
+            const uint32_t c = uses + i;
+            ok = mbar_wait(&acc_full[c % NSLOT], (c / NSLOT) & 1u, p.timeout);
+        }
+        if (!ok) break;
+        tc_fence_after();
+        const int s0 = uses % NSLOT, s1 = (uses + 1) % NSLOT;
+        const int m = it.mt * kBM + q * 32 + lane;  // weight row of this thread
+        const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+        const uint32_t t0 = tmem_base + lane_off + static_cast<uint32_t>(s0 * SLOT_COLS);
+        const uint32_t t1 = tmem_base + lane_off +
+                            static_cast<uint32_t>(u == 2 ? s1 * SLOT_COLS : s0 * SLOT_COLS + SLOT_COLS / 2);
+        const float f0 = acc.s0[it.e] * acc.mul;
+        const float f1 = GATE_UP ? acc.s1[it.e] * acc.mul : 1.0f;
+        for (int c = 0; c < it.n_valid; c += 16) {
+            uint32_t r0[16];
+            tmem_ld16(t0 + c, r0);
+            if (GATE_UP) {
+                uint32_t r1[16];
+                tmem_ld16(t1 + c, r1);
+                tmem_ld_wait();
+                if (m < p.M) {
+                    __nv_bfloat16 *h = reinterpret_cast<__nv_bfloat16 *>(p.out);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        if (c + j < it.n_valid)
+                            h[(it.row0 + c + j) * p.M + m] =
+                                __float2bfloat16_rn(silu_mul(f0 * __uint_as_float(r0[j]), f1 * __uint_as_float(r1[j])));
+                }
+            } else {
+                tmem_ld_wait();
+                if (m < p.M) {
+                    float *o = reinterpret_cast<float *>(p.out);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        if (c + j < it.n_valid)
+                            o[(it.row0 + c + j) * p.M + m] = f0 * __uint_as_float(r0[j]);
+                }
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0)
+            for (int i = 0; i < u; ++i) mbar_arrive(&acc_empty[(uses + i) % NSLOT]);
+        uses += u;
+    }
+}
+
 template <bool GATE_UP, int BN, int BOXN, int W8STAGES, int BSTAGES, int NSLOT, int SLOT_COLS, bool GATHER,
-          int ASTAGES>
+          int ASTAGES, bool FP4 = false>
 __global__ void __launch_bounds__(fp8_gemm_threads(GATE_UP), 1)
-    grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tm_a0,  // E4M3 W_gate (G1) / W_down (G2) [E][M][K]
-                            const __grid_constant__ CUtensorMap tm_a1,  // E4M3 W_up (G1); unused for G2
-                            const __grid_constant__ CUtensorMap tm_s0,  // scale codes of A0 [E][K/32][M]
+    grouped_gemm_fp8_kernel(const __grid_constant__ CUtensorMap tm_a0,  // codes of W_gate (G1) / W_down (G2):
+                                                                        // [E][M][K] E4M3, or [E][M][K/2] E2M1 pairs
+                            const __grid_constant__ CUtensorMap tm_a1,  // codes of W_up (G1); unused for G2
+                            const __grid_constant__ CUtensorMap tm_s0,  // scale codes of A0 [E][K/kBlk][M]
                             const __grid_constant__ CUtensorMap tm_s1,  // scale codes of A1
                             const __grid_constant__ CUtensorMap tm_b,   // B rows [rows][K] (GATHER: x [T][K])
-                            const GemmParams p) {
-    using C = Fp8GemmCfg<GATE_UP, BN, BOXN, W8STAGES, BSTAGES, NSLOT, SLOT_COLS, GATHER, ASTAGES>;
+                            const GemmParams p,
+                            const AccScales acc) {  // FP4: per-expert accumulator factors
+    using C = Fp8GemmCfg<GATE_UP, BN, BOXN, W8STAGES, BSTAGES, NSLOT, SLOT_COLS, GATHER, ASTAGES, FP4>;
     extern __shared__ uint8_t gemm_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(gemm_smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *w8_full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
@@ -119,7 +216,7 @@ __global__ void __launch_bounds__(fp8_gemm_threads(GATE_UP), 1)
     const int E = p.E;
     const int n_mt = (p.M + kBM - 1) / kBM;
     const int n_kb = p.K / kBK;          // 64-wide k-steps per item
-    const int n_w8 = (n_kb + 1) / 2;     // weight ring stages per item (the last may hold one k-step)
+    const int n_w8 = (n_kb + C::kSteps - 1) / C::kSteps;  // weight ring stages per item (the last may be partial)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < W8STAGES; ++s) {
@@ -160,7 +257,7 @@ __global__ void __launch_bounds__(fp8_gemm_threads(GATE_UP), 1)
     const int total = tile_start[E];
 
     if (warp == 0) {
-        // ---------------- weight producer: E4M3 tiles + scales, K = 128 per stage ----------------
+        // ---------------- weight producer: code tiles + scales, 128 bytes of each row per stage ----------------
         if (lane == 0) {
             const uint64_t pol_w = p.weights_once ? policy_evict_first() : policy_evict_normal();
             int stage = 0;
@@ -175,13 +272,14 @@ __global__ void __launch_bounds__(fp8_gemm_threads(GATE_UP), 1)
                     }
                     uint8_t *sa = smem + stage * C::kW8Stage;
                     mbar_arrive_expect_tx(&w8_full[stage], C::kNumA * (C::kA8 + C::kSc));
-                    tma_load_3d(sa, &tm_a0, &w8_full[stage], kb * C::kK8, it.mt * kBM, it.e, pol_w);
-                    tma_load_3d(sa + C::kScOff, &tm_s0, &w8_full[stage], it.mt * kBM, kb * (C::kK8 / 32), it.e,
-                                pol_w);
+                    // the code maps are byte-typed: 128 bytes of each row per stage
+                    tma_load_3d(sa, &tm_a0, &w8_full[stage], kb * 128, it.mt * kBM, it.e, pol_w);
+                    tma_load_3d(sa + C::kScOff, &tm_s0, &w8_full[stage], it.mt * kBM, kb * (C::kK8 / C::kBlk),
+                                it.e, pol_w);
                     if (GATE_UP) {
-                        tma_load_3d(sa + C::kA8, &tm_a1, &w8_full[stage], kb * C::kK8, it.mt * kBM, it.e, pol_w);
+                        tma_load_3d(sa + C::kA8, &tm_a1, &w8_full[stage], kb * 128, it.mt * kBM, it.e, pol_w);
                         tma_load_3d(sa + C::kScOff + C::kSc, &tm_s1, &w8_full[stage], it.mt * kBM,
-                                    kb * (C::kK8 / 32), it.e, pol_w);
+                                    kb * (C::kK8 / C::kBlk), it.e, pol_w);
                     }
                     issued |= 1u << stage;
                     issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
@@ -297,14 +395,20 @@ __global__ void __launch_bounds__(fp8_gemm_threads(GATE_UP), 1)
             mbar_wait(drain, 0, p.timeout);
         }
     } else if (warp >= 4 && warp < 8) {
-        gemm_epilogue<GATE_UP, BN, NSLOT, SLOT_COLS>(warp - 4, tile_start, total, p, tmem_base, acc_full, acc_empty);
+        if constexpr (FP4)
+            gemm_epilogue_scaled<GATE_UP, BN, NSLOT, SLOT_COLS>(warp - 4, tile_start, total, p, acc, tmem_base,
+                                                                acc_full, acc_empty);
+        else
+            gemm_epilogue<GATE_UP, BN, NSLOT, SLOT_COLS>(warp - 4, tile_start, total, p, tmem_base, acc_full,
+                                                         acc_empty);
     } else if (warp >= 8) {
-        // ---------------- converters: E4M3 (smem) -> bf16 A ring (TMEM) ----------------
+        // ---------------- converters: codes (smem) -> bf16 A ring (TMEM) ----------------
         // Converter warp wc = w - 8 owns TMEM lane quadrant wc % 4 (weight rows r = 32 (wc % 4) + lane)
         // and units u = wc / 4 + i * kConvWarps / 4 (i < kConvUnits) = (A tile u / 2, quarter u % 2) of
-        // each 64-wide k-step: per unit a thread reads 32 E4M3 codes (two 16-byte chunks of the
-        // 128-byte-swizzled row r) and their scale code, releases the weight stage after its last
-        // half, and writes the 32 bf16 values to 16 TMEM columns of lane r.
+        // each 64-wide k-step: per unit a thread reads 32 codes (E4M3: two 16-byte chunks of the
+        // 128-byte-swizzled row r, one scale code; E2M1: one chunk, two scale codes), releases the
+        // weight stage after its last k-step, and writes the 32 bf16 values to 16 TMEM columns of
+        // lane r.
         const int wc = warp - 8;
         const int r = 32 * (wc & 3) + lane;
         const uint32_t lane_base = static_cast<uint32_t>(32 * (wc & 3)) << 16;
@@ -314,40 +418,56 @@ __global__ void __launch_bounds__(fp8_gemm_threads(GATE_UP), 1)
         for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
             for (int kb = 0; kb < n_kb; ++kb, ++kstep) {
                 const uint32_t j = kstep % ASTAGES;
-                const int h = kb & 1;  // 64-wide half of the weight stage
-                const bool last = h == 1 || kb == n_kb - 1;
-                ok = __all_sync(0xffffffffu, (h == 1 || mbar_wait(&w8_full[stage], phase, p.timeout)) &&
+                const int h = kb % C::kSteps;  // 64-wide k-step within the weight stage
+                const bool last = h == C::kSteps - 1 || kb == n_kb - 1;
+                ok = __all_sync(0xffffffffu, (h != 0 || mbar_wait(&w8_full[stage], phase, p.timeout)) &&
                                                  mbar_wait(&a_free[j], ((kstep / ASTAGES) & 1u) ^ 1u, p.timeout));
                 if (!ok) break;
                 tc_fence_after();
                 const uint32_t st = smem_u32(smem + stage * C::kW8Stage);
                 uint4 q[C::kConvUnits][2];
-                uint32_t c[C::kConvUnits];
+                uint32_t c[C::kConvUnits][2];
                 bool big = false;
 #pragma unroll
                 for (int i = 0; i < C::kConvUnits; ++i) {
                     const int u = (wc >> 2) + i * (C::kConvWarps / 4);
                     const int a = u >> 1, hf = u & 1;
                     const uint32_t src = st + a * C::kA8 + r * 128;
-                    const int ch = 4 * h + 2 * hf;  // first 16-byte chunk of this thread's 32 codes
-                    q[i][0] = lds128(src + ((ch ^ (r & 7)) << 4));
-                    q[i][1] = lds128(src + (((ch + 1) ^ (r & 7)) << 4));
-                    c[i] = lds_u8(st + C::kScOff + a * C::kSc + (2 * h + hf) * kBM + r);
-                    big |= c[i] > 134u;
+                    const uint32_t sc = st + C::kScOff + a * C::kSc + r;
+                    if (FP4) {
+                        // 16 bytes = 32 codes at K 64h + 32hf of the stage: chunk 2h + hf; blocks of 16
+                        q[i][0] = lds128(src + (((2 * h + hf) ^ (r & 7)) << 4));
+                        c[i][0] = lds_u8(sc + (4 * h + 2 * hf) * kBM);
+                        c[i][1] = lds_u8(sc + (4 * h + 2 * hf + 1) * kBM);
+                    } else {
+                        const int ch = 4 * h + 2 * hf;  // first 16-byte chunk of this thread's 32 codes
+                        q[i][0] = lds128(src + ((ch ^ (r & 7)) << 4));
+                        q[i][1] = lds128(src + (((ch + 1) ^ (r & 7)) << 4));
+                        c[i][0] = lds_u8(sc + (2 * h + hf) * kBM);
+                        big |= c[i][0] > 134u;
+                    }
                 }
-                big = __any_sync(0xffffffffu, big);  // a scale code that needs the second factor
+                if (!FP4) big = __any_sync(0xffffffffu, big);  // a scale code that needs the second factor
                 uint32_t o[C::kConvUnits][16];
 #pragma unroll
                 for (int i = 0; i < C::kConvUnits; ++i) {
-                    const uint32_t qw[8] = {q[i][0].x, q[i][0].y, q[i][0].z, q[i][0].w,
-                                            q[i][1].x, q[i][1].y, q[i][1].z, q[i][1].w};
-                    const uint32_t f1 = fp8_factor1(c[i]);
+                    if (FP4) {
+                        const uint32_t qw[4] = {q[i][0].x, q[i][0].y, q[i][0].z, q[i][0].w};
+                        const uint32_t f[2] = {e4m3_scale_factor(c[i][0]), e4m3_scale_factor(c[i][1])};
 #pragma unroll
-                    for (int w = 0; w < 8; ++w) e4m3x4_to_bf16x4(qw[w], f1, o[i][2 * w], o[i][2 * w + 1]);
-                    if (big) {
-                        const uint32_t f2 = fp8_factor2(c[i]);
+                        for (int b = 0; b < 16; ++b)  // byte b holds K 2b, 2b+1: TMEM column b of the unit
+                            o[i][b] = e2m1x2_to_bf16x2((qw[b >> 2] >> (8 * (b & 3))) & 0xFFu, f[b >> 3]);
+                    } else {
+                        const uint32_t qw[8] = {q[i][0].x, q[i][0].y, q[i][0].z, q[i][0].w,
+                                                q[i][1].x, q[i][1].y, q[i][1].z, q[i][1].w};
+                        const uint32_t f1 = fp8_factor1(c[i][0]);
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) o[i][e] = bf16x2_mul(o[i][e], f2);
+                        for (int w = 0; w < 8; ++w) e4m3x4_to_bf16x4(qw[w], f1, o[i][2 * w], o[i][2 * w + 1]);
+                        if (big) {
+                            const uint32_t f2 = fp8_factor2(c[i][0]);
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) o[i][e] = bf16x2_mul(o[i][e], f2);
+                        }
                     }
                 }
                 if (last) {

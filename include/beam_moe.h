@@ -242,6 +242,49 @@ BEAM_MOE_API int beam_moe_forward_fp8(const beam_moe_config *cfg, int64_t T, con
                                       size_t ws_bytes, void *stream, void *const *events);
 
 /*
+ * NVFP4 expert weights.  The "Welcome Beam" page (TL;DR, "Checkpoint formats"; section "Hardware
+ * Requirements": the NVFP4 checkpoint keeps most parameters in 4 bits for Blackwell) gives no
+ * quantisation recipe.  This library reads NVFP4 as NVIDIA's layout: E2M1 element codes (sign,
+ * 2-bit exponent with bias 1, 1-bit mantissa; exponent 0 is subnormal, m * 0.5; magnitudes 0, 0.5,
+ * 1, 1.5, 2, 3, 4, 6), two per byte with element k of a row in the low nibble of byte k/2 when k is
+ * even and in the high nibble when k is odd; one E4M3 scale code per 16 consecutive K elements of
+ * a weight row (non-negative, finite); one FP32 scale per weight matrix:
+ *   W[e][row][k] = e2m1(code(e, row, k)) * e4m3(scale[e][k / 16][row]) * global[e]
+ * The kernels rebuild e2m1 * e4m3 * 2^-9, which bf16 holds exactly, run the bf16 tensor-core path,
+ * and multiply the FP32 accumulators by global[e] * 2^9.  Scale codes with the sign bit set or NaN
+ * give undefined results.
+ *   w_gate [E, I, H/2] u8    w_gate_scale [E, H/16, I] u8    w_gate_global [E] f32
+ *   w_up   [E, I, H/2] u8    w_up_scale   [E, H/16, I] u8    w_up_global   [E] f32
+ *   w_down [E, H, I/2] u8    w_down_scale [E, I/16, H] u8    w_down_global [E] f32
+ * All nine pointers are device memory, owned by the caller; the code and scale arrays 16-byte
+ * aligned, the scales 4-byte aligned.
+ */
+typedef struct beam_moe_nvfp4_experts {
+    const uint8_t *w_gate;
+    const uint8_t *w_gate_scale;
+    const float *w_gate_global;
+    const uint8_t *w_up;
+    const uint8_t *w_up_scale;
+    const float *w_up_global;
+    const uint8_t *w_down;
+    const uint8_t *w_down_scale;
+    const float *w_down_global;
+} beam_moe_nvfp4_experts;
+
+/* beam_moe_experts with NVFP4 expert weights; same workspace, outputs and error codes. */
+BEAM_MOE_API int beam_moe_experts_nvfp4(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x,
+                                        const int32_t *topk_ids, const float *topk_w,
+                                        const beam_moe_nvfp4_experts *w4, beam_bf16 *y, void *ws, size_t ws_bytes,
+                                        void *stream);
+
+/* beam_moe_forward with NVFP4 expert weights; `events` is NULL or 7 events (as for the FP8 call). */
+BEAM_MOE_API int beam_moe_forward_nvfp4(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x,
+                                        const float *w_router, const float *sel_bias,
+                                        const beam_moe_nvfp4_experts *w4, beam_bf16 *y, int32_t *topk_ids_out,
+                                        float *topk_w_out, void *ws, size_t ws_bytes, void *stream,
+                                        void *const *events);
+
+/*
  * beam_moe_permute without a workspace: the same dispatch (identical outputs), with its scratch in
  * a fixed device array inside this library instead of caller memory.  The Beam pages have no
  * counterpart; this exists for callers that cannot allocate device memory when they enqueue work,

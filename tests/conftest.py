@@ -43,3 +43,10 @@ def beam_weights_fp8(beam_weights):
     """MXFP8 copy of the shared Beam layer's expert weights (10 GB codes + scales) on cuda:0."""
     import beam_synth as bs
     return bs.quantize_experts(*beam_weights)
+
+
+@pytest.fixture(scope="session")
+def beam_weights_nvfp4(beam_weights):
+    """NVFP4 copy of the shared Beam layer's expert weights (5.3 GB codes + scales) on cuda:0."""
+    import beam_synth as bs
+    return bs.quantize_experts_nvfp4(*beam_weights)

@@ -156,3 +156,30 @@ def test_fp8_binding_refuses_bad_inputs_on_host(L):
         bm.forward_fp8(bm.BEAM_LAYER, x, torch.zeros(256, 5120), None, {})
     with pytest.raises(TypeError):
         bm.experts_fp8(bm.BEAM_LAYER, x, torch.zeros(4, 8, dtype=torch.int32), torch.zeros(4, 8), {})
+
+
+def test_nvfp4_entry_points_check_arguments_on_host(L):
+    c = _cfg()
+    p, mis = 4096, 4104
+    need = bm.workspace_size(c, 64, bm.WS_FORWARD)
+    q = ctypes.c_void_p(p)
+    good = bm.BeamMoeNvfp4Experts(*([p] * 9))
+    assert L.beam_moe_forward_nvfp4(ctypes.byref(c), 64, q, q, None, None, q, None, None, q, need, None, None) == \
+        bm.ERR_NULL
+    assert L.beam_moe_experts_nvfp4(ctypes.byref(c), 64, q, q, q, None, q, q, need, None) == bm.ERR_NULL
+    for i in range(9):  # each code, scale and per-matrix-scale pointer
+        vals = [p] * 9
+        vals[i] = 0
+        w4 = bm.BeamMoeNvfp4Experts(*vals)
+        assert L.beam_moe_forward_nvfp4(ctypes.byref(c), 64, q, q, None, ctypes.byref(w4), q, None, None, q, need,
+                                        None, None) == bm.ERR_NULL
+        vals[i] = mis + (2 if i % 3 == 2 else 0)  # codes / scale codes: 16-byte rule; per-matrix scales: 4-byte
+        w4 = bm.BeamMoeNvfp4Experts(*vals)
+        assert L.beam_moe_experts_nvfp4(ctypes.byref(c), 64, q, q, q, ctypes.byref(w4), q, q, need, None) == \
+            bm.ERR_MISALIGNED
+    assert L.beam_moe_forward_nvfp4(ctypes.byref(c), 64, q, q, None, ctypes.byref(good), q, None, None, q, need - 1,
+                                    None, None) == bm.ERR_WORKSPACE_TOO_SMALL
+    assert L.beam_moe_forward_nvfp4(ctypes.byref(c), 0, q, q, None, ctypes.byref(good), q, None, None, None, 0,
+                                    None, None) == bm.OK
+    with pytest.raises(KeyError):
+        bm._nvfp4_experts(bm.BEAM_LAYER.c(), {"q_gate": None})
