@@ -14,14 +14,14 @@
 // Rings and roles (threads = 256 + 32 * converter warps):
 //   weight ring (W8STAGES): per stage the A tile(s) as 128 rows x 128 bytes (K = 128 of E4M3 or
 //     K = 256 of E2M1; 128-byte swizzle: a weight row contributes 128 contiguous bytes, the piece
-//     size at which DRAM streams best) and their scale tiles [K-blocks of the stage][128 rows].  Warp 0 lane 0 loads it (TMA); the
-//     converters release it as soon as they have read it, so the weight stream never waits on the
-//     tensor core.
+//     size at which DRAM streams best) and their scale tiles [K-blocks of the stage][128 rows].
+//     Warp 0 lane 0 loads it (TMA); the converters release it as soon as they have read it, so the
+//     weight stream never waits on the tensor core.
 //   B ring (BSTAGES): one 64-wide k-step of the expert's token rows (tiled TMA boxes, or TMA
 //     gather4 straight from x).  Warp 2 loads it; the MMA releases it.
 //   A ring (ASTAGES, in TMEM after the accumulator slots): the bf16 A tile(s) of one 64-wide
-//     k-step.  Converter warps (from warp 8 on) rebuild them from E4M3 with tcgen05.st; the MMA
-//     reads its A operand from TMEM and frees the stage with tcgen05.commit.
+//     k-step.  Converter warps (from warp 8 on) rebuild them from the codes with tcgen05.st; the
+//     MMA reads its A operand from TMEM and frees the stage with tcgen05.commit.
 //   Warp 1 lane 0 issues tcgen05.mma; warps 4..7 run the epilogue.
 // Every wait is bounded (status word BEAM_MOE_ERR_DEVICE_TIMEOUT on expiry).
 #pragma once
