@@ -50,14 +50,14 @@ typedef uint16_t beam_bf16; /* raw bfloat16 bit pattern */
 
 /* Layer shape.  Beam: {5120, 2560, 256, 8, 4, 8, 2, 2.5f}. */
 typedef struct beam_moe_config {
-    int32_t hidden;       /* H: model width, multiple of 64, <= 65536 */
-    int32_t inter;        /* I: SwiGLU intermediate size, multiple of 64, <= 65536 */
+    int32_t hidden;       /* H: model width, multiple of 64, 64..65536 */
+    int32_t inter;        /* I: SwiGLU intermediate size, multiple of 64, 64..65536 */
     int32_t n_experts;    /* E: 1..256 */
-    int32_t n_groups;     /* G: divides E, E/G <= 256 */
+    int32_t n_groups;     /* G: 1..32, divides E */
     int32_t topk_groups;  /* groups kept per token, 1..G */
     int32_t topk;         /* k: experts per token, 1..min(16, topk_groups*E/G) */
     int32_t group_topn;   /* scores summed per group for the group ranking, 1..min(8, E/G) */
-    float routed_scale;   /* factor on the combined expert output (2.5) */
+    float routed_scale;   /* factor on the combined expert output (2.5); not NaN */
 } beam_moe_config;
 
 /* Return codes. */
@@ -71,7 +71,7 @@ enum {
     BEAM_MOE_ERR_CUDA = 6,               /* a CUDA runtime / launch error */
     BEAM_MOE_ERR_DEVICE_TIMEOUT = 7,     /* status word: a bounded device-side wait expired */
     BEAM_MOE_ERR_BAD_INDEX = 8,          /* status word: an expert id outside [0, E) */
-    BEAM_MOE_ERR_INVALID_ARG = 9         /* T < 0 or T beyond the supported range */
+    BEAM_MOE_ERR_INVALID_ARG = 9         /* T < 0, T > 2^24 or T * k >= 2^31 */
 };
 
 /* Workspace kinds for beam_moe_workspace_size. */
