@@ -57,6 +57,35 @@ int oracle_num_threads(void)
 }
 
 /*
+ * Evaluation order of the dot products below.  Every output is one sum over the reduction index
+ * taken in increasing order, acc = ((0 + a_0 b_0) + a_1 b_1) + ..., exactly as a plain loop per
+ * output computes it.  Rows of activations are taken RB at a time, stored transposed (xb[h*RB + r]),
+ * so the RB independent sums of one weight row advance together; no sum is split or reordered, so
+ * every value is the one the plain per-output loop gives.
+ */
+#define RB 8
+
+/* acc[r] = sum_{h=0}^{K-1} xb[h*RB + r] * w[h] for r < RB, each sum in increasing h. */
+static void dot_rows(int K, const double *xb, const double *w, double *acc)
+{
+    double a[RB] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+    for (int h = 0; h < K; ++h)
+        for (int r = 0; r < RB; ++r) a[r] += xb[(int64_t)h * RB + r] * w[h];
+    for (int r = 0; r < RB; ++r) acc[r] = a[r];
+}
+
+/* Rows [r0, r0 + nr) of a [*,K] bf16-bit matrix, widened to FP64 (exact) and transposed into
+ * xb[k*RB + r]; rows nr..RB-1 are zero. */
+static void bf16_rows_to_block(const uint16_t *rows, int64_t r0, int nr, int K, double *xb)
+{
+    for (int k = 0; k < K; ++k)
+        for (int r = 0; r < RB; ++r)
+            xb[(int64_t)k * RB + r] = r < nr ? bf16_bits_to_double(rows[(r0 + r) * K + k]) : 0.0;
+}
+
+static int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+/*
  * Step 1 (section "Mixture of Experts": "scores all 256 experts with a sigmoid"):
  * logit[t,e] = sum_h x[t,h] * W_r[e,h] in FP64, score = 1 / (1 + exp(-logit)).
  * x: [T,H] bf16 bits; w_router: [E,H] fp32; logit, score: [T,E] fp64.
@@ -64,19 +93,29 @@ int oracle_num_threads(void)
 void oracle_router_scores(int64_t T, int H, int E, const uint16_t *x, const float *w_router,
                           double *logit, double *score)
 {
-    #pragma omp parallel for schedule(static)
-    for (int64_t t = 0; t < T; ++t) {
-        double *xr = (double *)malloc(sizeof(double) * (size_t)H);
-        for (int h = 0; h < H; ++h) xr[h] = bf16_bits_to_double(x[t * H + h]);
-        for (int e = 0; e < E; ++e) {
-            const float *wr = w_router + (int64_t)e * H;
-            double acc = 0.0;
-            for (int h = 0; h < H; ++h) acc += xr[h] * (double)wr[h];
-            if (logit) logit[t * E + e] = acc;
-            score[t * E + e] = 1.0 / (1.0 + exp(-acc));
+    double *wr = (double *)malloc(sizeof(double) * (size_t)E * (size_t)H);
+    for (int64_t q = 0; q < (int64_t)E * H; ++q) wr[q] = (double)w_router[q];
+    const int64_t nb = (T + RB - 1) / RB;
+    #pragma omp parallel
+    {
+        double *xb = (double *)malloc(sizeof(double) * (size_t)H * RB);
+        #pragma omp for schedule(static)
+        for (int64_t b = 0; b < nb; ++b) {
+            const int nr = (int)min64(RB, T - b * RB);
+            bf16_rows_to_block(x, b * RB, nr, H, xb);
+            for (int e = 0; e < E; ++e) {
+                double acc[RB];
+                dot_rows(H, xb, wr + (int64_t)e * H, acc);
+                for (int r = 0; r < nr; ++r) {
+                    const int64_t t = b * RB + r;
+                    if (logit) logit[t * E + e] = acc[r];
+                    score[t * E + e] = 1.0 / (1.0 + exp(-acc[r]));
+                }
+            }
         }
-        free(xr);
+        free(xb);
     }
+    free(wr);
 }
 
 /* Index of the largest v[i] among alive[i] != 0; ties go to the lower index.  -1 if none. */
@@ -241,36 +280,51 @@ int oracle_permute(int64_t T, int topk, int E, const int32_t *ids, int32_t *coun
 void oracle_expert_mlp(int64_t n, int H, int I, const uint16_t *x_rows, const uint16_t *wg,
                        const uint16_t *wu, const uint16_t *wd, double *out)
 {
-    double *xd = (double *)malloc(sizeof(double) * (size_t)(n * H));
-    double *hd = (double *)malloc(sizeof(double) * (size_t)(n * I));
-    for (int64_t q = 0; q < n * H; ++q) xd[q] = bf16_bits_to_double(x_rows[q]);
+    const int64_t nb = (n + RB - 1) / RB;
+    double *xb = (double *)malloc(sizeof(double) * (size_t)(nb * H * RB));  /* x, RB rows per block */
+    double *hb = (double *)malloc(sizeof(double) * (size_t)(nb * I * RB));  /* h, same blocking */
+    for (int64_t b = 0; b < nb; ++b) bf16_rows_to_block(x_rows, b * RB, (int)min64(RB, n - b * RB), H, xb + b * H * RB);
 
-    #pragma omp parallel for collapse(2) schedule(static)
-    for (int64_t r = 0; r < n; ++r)
-        for (int i = 0; i < I; ++i) {
-            const double *xr = xd + r * H;
-            const uint16_t *gr = wg + (int64_t)i * H;
-            const uint16_t *ur = wu + (int64_t)i * H;
-            double g = 0.0, u = 0.0;
-            for (int h = 0; h < H; ++h) {
-                g += bf16_bits_to_double(gr[h]) * xr[h];
-                u += bf16_bits_to_double(ur[h]) * xr[h];
+    /* g = Wg x, u = Wu x, h = SiLU(g) * u */
+    #pragma omp parallel
+    {
+        double *wgr = (double *)malloc(sizeof(double) * (size_t)H);
+        double *wur = (double *)malloc(sizeof(double) * (size_t)H);
+        #pragma omp for collapse(2) schedule(static)
+        for (int64_t b = 0; b < nb; ++b)
+            for (int i = 0; i < I; ++i) {
+                for (int h = 0; h < H; ++h) {
+                    wgr[h] = bf16_bits_to_double(wg[(int64_t)i * H + h]);
+                    wur[h] = bf16_bits_to_double(wu[(int64_t)i * H + h]);
+                }
+                double g[RB], u[RB];
+                dot_rows(H, xb + b * H * RB, wgr, g);
+                dot_rows(H, xb + b * H * RB, wur, u);
+                for (int r = 0; r < RB; ++r) {
+                    double silu = g[r] / (1.0 + exp(-g[r]));
+                    hb[(b * I + i) * RB + r] = silu * u[r];
+                }
             }
-            double silu = g / (1.0 + exp(-g));
-            hd[r * I + i] = silu * u;
-        }
+        free(wgr);
+        free(wur);
+    }
 
-    #pragma omp parallel for collapse(2) schedule(static)
-    for (int64_t r = 0; r < n; ++r)
-        for (int o = 0; o < H; ++o) {
-            const double *hr = hd + r * I;
-            const uint16_t *dr = wd + (int64_t)o * I;
-            double acc = 0.0;
-            for (int i = 0; i < I; ++i) acc += bf16_bits_to_double(dr[i]) * hr[i];
-            out[r * H + o] = acc;
-        }
-    free(xd);
-    free(hd);
+    /* out = Wd h */
+    #pragma omp parallel
+    {
+        double *wdr = (double *)malloc(sizeof(double) * (size_t)I);
+        #pragma omp for collapse(2) schedule(static)
+        for (int64_t b = 0; b < nb; ++b)
+            for (int o = 0; o < H; ++o) {
+                for (int i = 0; i < I; ++i) wdr[i] = bf16_bits_to_double(wd[(int64_t)o * I + i]);
+                double acc[RB];
+                dot_rows(I, hb + b * I * RB, wdr, acc);
+                for (int r = 0; r < RB && b * RB + r < n; ++r) out[(b * RB + r) * H + o] = acc[r];
+            }
+        free(wdr);
+    }
+    free(xb);
+    free(hb);
 }
 
 /*
@@ -409,34 +463,30 @@ int oracle_dequant_nvfp4(int64_t rows, int K, const uint8_t *q, const uint8_t *s
 void oracle_expert_mlp_f64(int64_t n, int H, int I, const uint16_t *x_rows, const double *wg,
                            const double *wu, const double *wd, double *out)
 {
-    double *xd = (double *)malloc(sizeof(double) * (size_t)(n * H));
-    double *hd = (double *)malloc(sizeof(double) * (size_t)(n * I));
-    for (int64_t q = 0; q < n * H; ++q) xd[q] = bf16_bits_to_double(x_rows[q]);
+    const int64_t nb = (n + RB - 1) / RB;
+    double *xb = (double *)malloc(sizeof(double) * (size_t)(nb * H * RB));
+    double *hb = (double *)malloc(sizeof(double) * (size_t)(nb * I * RB));
+    for (int64_t b = 0; b < nb; ++b) bf16_rows_to_block(x_rows, b * RB, (int)min64(RB, n - b * RB), H, xb + b * H * RB);
 
     #pragma omp parallel for collapse(2) schedule(static)
-    for (int64_t r = 0; r < n; ++r)
+    for (int64_t b = 0; b < nb; ++b)
         for (int i = 0; i < I; ++i) {
-            const double *xr = xd + r * H;
-            const double *gr = wg + (int64_t)i * H;
-            const double *ur = wu + (int64_t)i * H;
-            double g = 0.0, u = 0.0;
-            for (int h = 0; h < H; ++h) {
-                g += gr[h] * xr[h];
-                u += ur[h] * xr[h];
+            double g[RB], u[RB];
+            dot_rows(H, xb + b * H * RB, wg + (int64_t)i * H, g);
+            dot_rows(H, xb + b * H * RB, wu + (int64_t)i * H, u);
+            for (int r = 0; r < RB; ++r) {
+                const double act = g[r] / (1.0 + exp(-g[r]));  /* SiLU(g) */
+                hb[(b * I + i) * RB + r] = act * u[r];
             }
-            const double act = g / (1.0 + exp(-g));  /* SiLU(g) */
-            hd[r * I + i] = act * u;
         }
 
     #pragma omp parallel for collapse(2) schedule(static)
-    for (int64_t r = 0; r < n; ++r)
+    for (int64_t b = 0; b < nb; ++b)
         for (int o = 0; o < H; ++o) {
-            const double *hr = hd + r * I;
-            const double *dr = wd + (int64_t)o * I;
-            double acc = 0.0;
-            for (int i = 0; i < I; ++i) acc += dr[i] * hr[i];
-            out[r * H + o] = acc;
+            double acc[RB];
+            dot_rows(I, hb + b * I * RB, wd + (int64_t)o * I, acc);
+            for (int r = 0; r < RB && b * RB + r < n; ++r) out[(b * RB + r) * H + o] = acc[r];
         }
-    free(xd);
-    free(hd);
+    free(xb);
+    free(hb);
 }

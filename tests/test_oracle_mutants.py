@@ -26,12 +26,13 @@ MUTANTS = {
     "weights_use_bias": ("for (int j = 0; j < topk; ++j) den += s[id32[j]];",
                          "for (int j = 0; j < topk; ++j) den += sel[id32[j]];"),
     "ties_to_higher_index": ("if (best < 0 || v[i] > v[best]) best = i;", "if (best < 0 || v[i] >= v[best]) best = i;"),
-    "sigmoid_sign": ("score[t * E + e] = 1.0 / (1.0 + exp(-acc));", "score[t * E + e] = 1.0 / (1.0 + exp(acc));"),
-    "silu_sign": ("double silu = g / (1.0 + exp(-g));", "double silu = g / (1.0 + exp(g));"),
-    "silu_missing": ("hd[r * I + i] = silu * u;", "hd[r * I + i] = g * u;"),
-    "down_transposed": ("acc += bf16_bits_to_double(dr[i]) * hr[i];",
-                        "acc += bf16_bits_to_double(wd[(int64_t)i * H + o]) * hr[i];"),
-    "gate_up_swapped_role": ("double silu = g / (1.0 + exp(-g));", "double silu = u / (1.0 + exp(-u));"),
+    "sigmoid_sign": ("score[t * E + e] = 1.0 / (1.0 + exp(-acc[r]));",
+                     "score[t * E + e] = 1.0 / (1.0 + exp(acc[r]));"),
+    "silu_sign": ("double silu = g[r] / (1.0 + exp(-g[r]));", "double silu = g[r] / (1.0 + exp(g[r]));"),
+    "silu_missing": ("hb[(b * I + i) * RB + r] = silu * u[r];", "hb[(b * I + i) * RB + r] = g[r] * u[r];"),
+    "down_transposed": ("wdr[i] = bf16_bits_to_double(wd[(int64_t)o * I + i]);",
+                        "wdr[i] = bf16_bits_to_double(wd[(int64_t)i * H + o]);"),
+    "gate_up_swapped_role": ("double silu = g[r] / (1.0 + exp(-g[r]));", "double silu = u[r] / (1.0 + exp(-u[r]));"),
     "no_routed_scale": ("y[t * H + h] = routed_scale * acc;", "y[t * H + h] = acc;"),
     "permute_tokens_descending": ("for (int64_t q = 0; q < n; ++q)\n            if (ids[q] == e) {",
                                   "for (int64_t q = n - 1; q >= 0; --q)\n            if (ids[q] == e) {"),
@@ -53,7 +54,7 @@ MUTANTS = {
     "nvfp4_nibbles_swapped": ("(k & 1) ? (byte >> 4) : (byte & 15)", "(k & 1) ? (byte & 15) : (byte >> 4)"),
     "nvfp4_scale_row_major": ("scale[(int64_t)(k / 16) * rows + r]", "scale[r * (K / 16) + k / 16]"),
     "nvfp4_global_dropped": ("e2m1_value(nib) * sv * global", "e2m1_value(nib) * sv"),
-    "expert_f64_silu_missing": ("const double act = g / (1.0 + exp(-g));", "const double act = g;"),
+    "expert_f64_silu_missing": ("const double act = g[r] / (1.0 + exp(-g[r]));", "const double act = g[r];"),
 }
 
 PINS = [
