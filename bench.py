@@ -69,7 +69,10 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="prefill", choices=["decode", "prefill", "skew", "long"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--cpu-sample", type=int, default=96, help="tokens in the CPU-oracle baseline sample")
+    ap.add_argument("--also", default=None,
+                    help="comma-separated workloads timed after the headline one in the same process "
+                         "(default: decode,skew,long for bf16, decode for --fp8/--nvfp4, none for --block)")
+    ap.add_argument("--cpu-sample", type=int, default=1024, help="tokens in the CPU-oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--dense", action="store_true",
                     help="time the dense SwiGLU MLP of Beam's first layers (T=4096, intermediate 20480)")
@@ -103,7 +106,14 @@ def kernel_source_hash() -> str:
 # ------------------------------------------------------------------------------------------------
 # algorithmic work (bytes the method must move, flops it must do), per step
 def algorithmic(wl: bs.Workload, n_act: int, fmt: str = "bf16") -> dict:
-    """fmt "fp8": expert weights are 1-byte E4M3 codes plus one 1-byte scale code per 32 elements;
+    """The layer's algorithmic work and each stage's share of it.
+
+    Layer bytes = each active expert's weights once + W_r + x in + y out + ids and weights; the
+    dispatch copies (x_perm), h and the FP32 expert outputs are implementation choices and count in
+    no stage's algorithmic bytes (they appear in the ncu traffic).  Stage shares: router = x, W_r
+    and its ids/weights out; gate/up = its weights + x; down = its weights; combine = y out + the
+    ids/weights it reads; dispatch and gather = the ids they read.
+    fmt "fp8": expert weights are 1-byte E4M3 codes plus one 1-byte scale code per 32 elements;
     "nvfp4": half-byte E2M1 codes plus one 1-byte scale code per 16 elements (the per-matrix FP32
     scales are negligible)."""
     T, H, I, E, k = wl.T, wl.hidden, wl.inter, wl.n_experts, wl.topk
@@ -115,11 +125,11 @@ def algorithmic(wl: bs.Workload, n_act: int, fmt: str = "bf16") -> dict:
         layer_bytes=n_act * w_expert + E * H * 4 + 2 * T * H * 2 + T * k * 8,
         stage_bytes={
             "router": T * H * 2 + E * H * 4 + T * k * 8,
-            "dispatch": T * k * 4 + 2 * R * 4,
-            "gather": T * H * 2 + R * H * 2,
-            "gate_up_swiglu": n_act * 2 * I * H * wb + R * H * 2 + R * I * 2,
-            "down": n_act * H * I * wb + R * I * 2 + R * H * 4,
-            "combine": R * H * 4 + T * k * 8 + T * H * 2,
+            "dispatch": T * k * 4,
+            "gather": T * k * 4,
+            "gate_up_swiglu": n_act * 2 * I * H * wb + T * H * 2,
+            "down": n_act * H * I * wb,
+            "combine": T * H * 2 + T * k * 8,
         },
         stage_flops={"router": 2 * T * H * E, "gate_up_swiglu": 4 * R * H * I, "down": 2 * R * H * I},
     )
@@ -158,28 +168,45 @@ class ClockSampler:
         self.marks.append(self.n_samples())
 
     def stop(self) -> dict:
+        """Stops sampling; returns the summary of every sample taken."""
+        self.rows = []
+        if self.proc is not None:
+            self.proc.terminate()
+            self.proc.wait()
+            with open(self.file.name) as f:
+                self.rows = [ln.strip().split(", ") for ln in f if ln.strip()]
+        return self.summary(0, len(self.rows))
+
+    def summary(self, lo: int, hi: int) -> dict:
+        """Median SM clock, max clock, throttle reasons and peak power over samples [lo, hi)."""
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
-        self.proc.terminate()
-        self.proc.wait()
-        with open(self.file.name) as f:
-            rows = [ln.strip().split(", ") for ln in f if ln.strip()]
-        os.unlink(self.file.name)
-        lo, hi = (self.marks[0], self.marks[-1]) if len(self.marks) >= 2 else (0, len(rows))
-        sel = rows[lo:hi] if hi > lo else rows
-        sm = [float(r[1]) for r in sel if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in sel if r[2].replace(".", "").isdigit()]
+        sel = self.rows[lo:hi] if hi > lo else self.rows
+        sm = [float(r[1]) for r in sel if len(r) > 1 and r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in sel if len(r) > 2 and r[2].replace(".", "").isdigit()]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in sel for i in range(4) if len(r) > 5 + i and r[5 + i] == "Active"})
-        power = [float(r[3]) for r in sel if r[3].replace(".", "").isdigit()]
+        power = [float(r[3]) for r in sel if len(r) > 3 and r[3].replace(".", "").isdigit()]
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
                 "reasons": reasons, "samples": len(sel), "power_w_max": max(power) if power else None}
+
+    def cleanup(self):
+        try:
+            os.unlink(self.file.name)
+        except OSError:
+            pass
 
 
 # ------------------------------------------------------------------------------------------------
 def bf16_fetch(wg, wu, wd):
-    import oracle
-    return lambda e: (oracle.bf16_bits(wg[e]), oracle.bf16_bits(wu[e]), oracle.bf16_bits(wd[e]))
+    """One expert's weights for the oracle: bf16 bits from one host copy of the layer (made on first use)."""
+    host = []
+
+    def fetch(e):
+        if not host:
+            host.extend(t.cpu().view(torch.int16).numpy().view(np.uint16) for t in (wg, wu, wd))
+        return host[0][e], host[1][e], host[2][e]
+    return fetch
 
 
 def fp8_fetch(w8):
@@ -247,10 +274,14 @@ def run_reference(args):
     W = bs.make_router(wl)
     bias = bs.load_bias(wl)
     wg, wu, wd = bs.make_experts(wl, device="cuda")
-    n = 16
+    # one host copy of the layer (the oracle reads each expert it needs from it, untimed)
+    host = tuple(t.cpu().view(torch.int16).numpy().view(np.uint16) for t in (wg, wu, wd))
+    del wg, wu, wd
+    fetch = lambda e: (host[0][e], host[1][e], host[2][e])  # noqa: E731
+    n = 32
     rates, secs = [], []
     for i in range(args.warmup + args.steps):
-        r = cpu_oracle_rate(wl, x, W, bias, bf16_fetch(wg, wu, wd), n, route_all=False)
+        r = cpu_oracle_rate(wl, x, W, bias, fetch, n, route_all=False)
         if i >= args.warmup:
             rates.append(r)
             secs.append(r["seconds"])
@@ -331,6 +362,44 @@ class Ranks:
             self.dist = None
 
 
+def layer_inputs(wl):
+    """x, W_r and bias of a workload: host copies and device tensors."""
+    x_cpu = bs.make_x(wl)
+    W_cpu = bs.make_router(wl)
+    b_cpu = bs.load_bias(wl)
+    return dict(x_cpu=x_cpu, W_cpu=W_cpu, b_cpu=b_cpu, x=x_cpu.cuda(), W=W_cpu.cuda(),
+                bias=None if b_cpu is None else b_cpu.cuda())
+
+
+def roofline_of(wl, fmt, stage_ms, n_act, ms_step, pk, pk_kind):
+    """Layer roofline and the dominant kernel's roofline (HBM GB/s or tensor TFLOP/s, whichever
+    bounds it at this workload) from the measured stage times."""
+    alg = algorithmic(wl, n_act, fmt)
+    t_tensor = alg["layer_flops"] / (pk["bf16_tflops"] * 1e12)
+    t_hbm = alg["layer_bytes"] / (pk["hbm_gbs"] * 1e9)
+    t_roof = max(t_tensor, t_hbm)
+    layer = {"bound": "hbm" if t_hbm >= t_tensor else "tensor", "roofline_ms": t_roof * 1e3,
+             "roofline_tokens_s": wl.T / t_roof, "frac": t_roof / (ms_step / 1e3),
+             "tensor_ms": t_tensor * 1e3, "hbm_ms": t_hbm * 1e3, "active_experts": n_act,
+             "achieved_tflops": alg["layer_flops"] / (ms_step / 1e3) / 1e12,
+             "achieved_gbs": alg["layer_bytes"] / (ms_step / 1e3) / 1e9}
+    dom = max(stage_ms, key=stage_ms.get)
+    sec = stage_ms[dom] / 1e3
+    by = alg["stage_bytes"][dom]
+    fl = alg["stage_flops"].get(dom, 0.0)
+    t_b = by / (pk["hbm_gbs"] * 1e9)
+    t_f = fl / (pk["bf16_tflops"] * 1e12)
+    if dom in ("gate_up_swiglu", "down") and t_f > t_b and fmt == "bf16":
+        roof = {"bound": "tensor", "kernel": dom, "achieved": fl / sec / 1e12, "peak": pk["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": fl / sec / 1e12 / pk["bf16_tflops"], "peak_kind": pk_kind,
+                "algorithmic_flops_per_launch": fl, "launch_ms": stage_ms[dom]}
+    else:
+        roof = {"bound": "hbm", "kernel": dom, "achieved": by / sec / 1e9, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                "frac": by / sec / 1e9 / pk["hbm_gbs"], "peak_kind": pk_kind, "algorithmic_bytes_per_launch": by,
+                "launch_ms": stage_ms[dom]}
+    return layer, roof
+
+
 def run_ours(args):
     import group_limited_routing_router_b200 as bm
 
@@ -342,15 +411,14 @@ def run_ours(args):
     wl = bs.get(args.workload)
     layer = wl.layer
     T, H = wl.T, wl.hidden
-    x_cpu = bs.make_x(wl)
-    W_cpu = bs.make_router(wl)
-    b_cpu = bs.load_bias(wl)
-    x = x_cpu.cuda()
-    W = W_cpu.cuda()
-    bias = None if b_cpu is None else b_cpu.cuda()
+    fmt = "nvfp4" if args.nvfp4 else "fp8" if args.fp8 else "bf16"
+    if args.also is None:
+        also = [] if args.block else (["decode", "skew", "long"] if fmt == "bf16" else ["decode"])
+    else:
+        also = [n for n in args.also.split(",") if n]
+    also = [n for n in also if n != wl.name]
     wg, wu, wd = bs.make_experts(wl, device="cuda")
     w8 = None
-    fmt = "nvfp4" if args.nvfp4 else "fp8" if args.fp8 else "bf16"
     if fmt != "bf16":
         if args.block:
             raise SystemExit("--fp8/--nvfp4 and --block: the sublayer entry point takes bf16 expert weights")
@@ -358,73 +426,96 @@ def run_ours(args):
         del wg, wu, wd
         wg = wu = wd = None
         torch.cuda.empty_cache()
-    ws = torch.empty(bm.workspace_size(layer, T, bm.WS_FORWARD), dtype=torch.uint8, device="cuda")
-    y = torch.empty(T, H, dtype=torch.bfloat16, device="cuda")
-    ids = torch.empty(T, wl.topk, dtype=torch.int32, device="cuda")
-    w = torch.empty(T, wl.topk, dtype=torch.float32, device="cuda")
+    T_max = max([T] + [bs.get(n).T for n in also])
+    ws = torch.empty(bm.workspace_size(layer, T_max, bm.WS_FORWARD), dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream()
 
-    if args.block:
-        g_pre = torch.ones(H, dtype=torch.float32, device="cuda")
-        g_post = torch.ones(H, dtype=torch.float32, device="cuda")
-        ws_blk = torch.empty(bm.workspace_size(layer, T, bm.WS_BLOCK), dtype=torch.uint8, device="cuda")
-        block_step = 2 * 3 + 3  # the MoE sublayer of the first MoE layer (layer 3)
+    def make_step(inp, y, ids, w):
+        x, W, bias = inp["x"], inp["W"], inp["bias"]
+        if args.block:
+            g_pre = torch.ones(H, dtype=torch.float32, device="cuda")
+            g_post = torch.ones(H, dtype=torch.float32, device="cuda")
+            ws_blk = torch.empty(bm.workspace_size(layer, x.shape[0], bm.WS_BLOCK), dtype=torch.uint8, device="cuda")
+            block_step = 2 * 3 + 3  # the MoE sublayer of the first MoE layer (layer 3)
+            return lambda: bm.block_forward(layer, x, g_pre, g_post, 1e-6, block_step, W, bias, wg, wu, wd,
+                                            stream_out=y, ids=ids, w=w, ws=ws_blk)
+        if fmt == "fp8":
+            return lambda: bm.forward_fp8(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws)
+        if fmt == "nvfp4":
+            return lambda: bm.forward_nvfp4(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws)
+        return lambda: bm.forward(layer, x, W, bias, wg, wu, wd, y=y, ids=ids, w=w, ws=ws)
 
-        def step():
-            bm.block_forward(layer, x, g_pre, g_post, 1e-6, block_step, W, bias, wg, wu, wd, stream_out=y, ids=ids,
-                             w=w, ws=ws_blk)
-    elif fmt == "fp8":
-        def step():
-            bm.forward_fp8(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws)
-    elif fmt == "nvfp4":
-        def step():
-            bm.forward_nvfp4(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws)
-    else:
-        def step():
-            bm.forward(layer, x, W, bias, wg, wu, wd, y=y, ids=ids, w=w, ws=ws)
+    def profiled(inp, y, ids, w, ev):
+        x, W, bias = inp["x"], inp["W"], inp["bias"]
+        if fmt == "fp8":
+            bm.forward_fp8(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws, events=ev)
+        elif fmt == "nvfp4":
+            bm.forward_nvfp4(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws, events=ev)
+        else:
+            bm.forward_profiled(layer, x, W, bias, wg, wu, wd, ev, y, ids, w, ws)
 
     clocks = ClockSampler(local)
     clocks.start()
-    for _ in range(args.warmup):
-        step()
-    assert bm.device_status() == bm.OK
-    barrier()
-    clocks.mark()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ev0.record(stream)
-    for _ in range(args.steps):
-        step()
-    ev1.record(stream)
-    barrier()
-    clocks.mark()
-    # keep the GPU busy (untimed) until the sampler has seen at least 3 samples under load
-    t_extra = time.time()
-    while clocks.marks[-1] - clocks.marks[0] < 3 and time.time() - t_extra < 2.0:
-        for _ in range(10):
-            step()
-        torch.cuda.synchronize()
-        clocks.marks[-1] = clocks.n_samples()
-    clk = clocks.stop()
-    ms_this = ev0.elapsed_time(ev1)
-    value = ranks.rate(T * args.steps, ms_this)
-    ms_step = ranks.max(ms_this) / args.steps
-    n_act = int((torch.bincount(ids.flatten().long(), minlength=wl.n_experts) > 0).sum().item())
+    pk, pk_kind = peaks()
 
-    # per-stage device time from events recorded between the launches (same stream)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
-    for i in range(args.steps):
-        if fmt == "fp8":
-            bm.forward_fp8(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws, events=evs[i])
-        elif fmt == "nvfp4":
-            bm.forward_nvfp4(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws, events=evs[i])
-        else:
-            bm.forward_profiled(layer, x, W, bias, wg, wu, wd, evs[i], y, ids, w, ws)
-    torch.cuda.synchronize()
-    stage_ms = {name: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
-                for j, name in enumerate(bm.STAGES)}
+    def measure(wlx, steps, warmup, headline):
+        """Device time of `steps` calls (max over ranks), stage times from profiled calls, routing stats."""
+        inp = layer_inputs(wlx)
+        y = torch.empty(wlx.T, H, dtype=torch.bfloat16, device="cuda")
+        ids = torch.empty(wlx.T, wlx.topk, dtype=torch.int32, device="cuda")
+        w = torch.empty(wlx.T, wlx.topk, dtype=torch.float32, device="cuda")
+        step = make_step(inp, y, ids, w)
+        for _ in range(warmup):
+            step()
+        assert bm.device_status() == bm.OK
+        barrier()
+        mark0 = clocks.n_samples()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        for _ in range(steps):
+            step()
+        ev1.record(stream)
+        barrier()
+        # keep the GPU busy (untimed) until the sampler has seen at least 3 samples under load
+        t_extra = time.time()
+        while clocks.n_samples() - mark0 < 3 and time.time() - t_extra < 2.0:
+            for _ in range(10):
+                step()
+            torch.cuda.synchronize()
+        span = (mark0, clocks.n_samples())
+        ms_this = ev0.elapsed_time(ev1)
+        ms_step = ranks.max(ms_this) / steps
+        value = ranks.rate(wlx.T * steps, ms_this)
+        counts = torch.bincount(ids.flatten().long(), minlength=wlx.n_experts)
+        n_act = int((counts > 0).sum().item())
+        # per-stage device time from events recorded between the launches (same stream)
+        n_prof = min(steps, 20)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(n_prof)]
+        for i in range(n_prof):
+            profiled(inp, y, ids, w, evs[i])
+        torch.cuda.synchronize()
+        stage_ms = {name: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
+                    for j, name in enumerate(bm.STAGES)}
+        layer_roof, roof = roofline_of(wlx, fmt, stage_ms, n_act, ms_step, pk, pk_kind)
+        out = dict(value=value, ms_per_step=ms_step, steps=steps, warmup=warmup, layer_roofline=layer_roof,
+                   roofline=roof, stage_ms=stage_ms, clock_span=span,
+                   load={"max_over_mean": float(counts.max().item() / counts.float().mean().item()),
+                         "experts_with_no_token": int((counts == 0).sum().item())})
+        if headline:
+            out["inp"], out["step"], out["y"] = inp, step, y
+        return out
+
+    head = measure(wl, args.steps, args.warmup, True)
+    others = {}
+    for n in also:
+        wlx = bs.get(n)
+        k_steps = max(3, min(args.steps, int(2000.0 / max(head["ms_per_step"] * wlx.T / T, 1e-3))))
+        others[n] = measure(wlx, k_steps, max(3, min(args.warmup, 5)), False)
 
     # end to end through the public API with host buffers: H2D x, forward, D2H y every step
-    x_host = x_cpu.pin_memory()
+    inp, step, y = head.pop("inp"), head.pop("step"), head.pop("y")
+    x = inp["x"]
+    x_host = inp["x_cpu"].pin_memory()
     y_host = torch.empty(T, H, dtype=torch.bfloat16).pin_memory()
     for _ in range(2):
         x.copy_(x_host, non_blocking=True)
@@ -441,32 +532,23 @@ def run_ours(args):
     barrier()
     e2e_value = ranks.rate(T * args.steps, e0.elapsed_time(e1))
     assert bm.device_status() == bm.OK
+    clk_all = clocks.stop()
+    clk = clocks.summary(*head.pop("clock_span"))
+    for n in others:
+        others[n]["clocks"] = clocks.summary(*others[n].pop("clock_span"))
+    clocks.cleanup()
 
-    alg = algorithmic(wl, n_act, fmt)
-    pk, pk_kind = peaks()
-    dom = max(stage_ms, key=stage_ms.get)
-    dom_bytes = alg["stage_bytes"][dom]
-    achieved = dom_bytes / (stage_ms[dom] / 1e3) / 1e9
+    roofline = head["roofline"]
+    tr = NCU_TRAFFIC.get((roofline["kernel"] + ("" if fmt == "bf16" else "_" + fmt), wl.name))
+    roofline["traffic"] = tr["bytes"] if tr and files_hash(tr["files"]) == tr["hash"] else None
     src_hash = kernel_source_hash()
-    tr = NCU_TRAFFIC.get((dom + ("" if fmt == "bf16" else "_" + fmt), wl.name))
-    traffic = tr["bytes"] if tr and files_hash(tr["files"]) == tr["hash"] else None
-    roofline = {"bound": "hbm", "kernel": dom, "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / pk["hbm_gbs"], "traffic": traffic, "peak_kind": pk_kind,
-                "algorithmic_bytes_per_launch": dom_bytes, "launch_ms": stage_ms[dom]}
-    t_tensor = alg["layer_flops"] / (pk["bf16_tflops"] * 1e12)
-    t_hbm = alg["layer_bytes"] / (pk["hbm_gbs"] * 1e9)
-    t_roof = max(t_tensor, t_hbm)
-    layer_roof = {"bound": "hbm" if t_hbm >= t_tensor else "tensor", "roofline_ms": t_roof * 1e3,
-                  "roofline_tokens_s": T / t_roof, "frac": t_roof / (ms_step / 1e3),
-                  "tensor_ms": t_tensor * 1e3, "hbm_ms": t_hbm * 1e3, "active_experts": n_act,
-                  "achieved_tflops": alg["layer_flops"] / (ms_step / 1e3) / 1e12,
-                  "achieved_gbs": alg["layer_bytes"] / (ms_step / 1e3) / 1e9}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         fetch = {"bf16": lambda: bf16_fetch(wg, wu, wd), "fp8": lambda: fp8_fetch(w8),
                  "nvfp4": lambda: nvfp4_fetch(w8)}[fmt]()
-        cpu = cpu_oracle_rate(wl, x_cpu, W_cpu, b_cpu, fetch, args.cpu_sample, f64_weights=fmt == "nvfp4")
+        cpu = cpu_oracle_rate(wl, inp["x_cpu"], inp["W_cpu"], inp["b_cpu"], fetch, args.cpu_sample,
+                              f64_weights=fmt == "nvfp4")
         cpu.pop("seconds", None)
 
     cfg = config_dict(wl)
@@ -482,14 +564,23 @@ def run_ours(args):
         cfg["l2"] = "no flush: every step streams the 5.7 GB of NVFP4 expert weights and scales (> 126 MB L2)"
     metric = {"bf16": METRIC, "fp8": METRIC_FP8, "nvfp4": METRIC_NVFP4}[fmt]
     dtype = {"bf16": "bf16", "fp8": "fp8-e4m3 weights, bf16 MMA", "nvfp4": "nvfp4-e2m1 weights, bf16 MMA"}[fmt]
-    line = {"metric": metric, "value": value, "unit": "tokens/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+    n_launch = launches_per_step(wl, args.block)
+    line = {"metric": metric, "value": head["value"], "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": dtype,
             "data": "synthetic", "config": cfg,
-            "roofline": roofline, "layer_roofline": layer_roof, "stage_ms": stage_ms, "cpu_baseline": cpu,
+            "roofline": roofline, "layer_roofline": head["layer_roofline"], "stage_ms": head["stage_ms"],
+            "load": head["load"], "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": T * H * 2,
                     "d2h_bytes_per_step": T * H * 2},
-            "clocks": clk, "gpu_launches": launches_per_step(wl, args.block) * args.steps, "kernel_source": src_hash}
+            "clocks": clk, "clocks_whole_run": clk_all,
+            "gpu_launches": n_launch * args.steps, "kernel_source": src_hash}
+    if others:
+        line["workloads"] = {n: {"T": bs.get(n).T, "tokens_s": o["value"], "ms_per_step": o["ms_per_step"],
+                                 "steps": o["steps"], "warmup": o["warmup"], "layer_roofline": o["layer_roofline"],
+                                 "roofline": o["roofline"], "stage_ms": o["stage_ms"], "load": o["load"],
+                                 "clocks": o["clocks"], "workload": config_dict(bs.get(n))["workload"]}
+                             for n, o in others.items()}
     if args.block:
         line["config"]["block"] = ("sublayer step: RMSNorm pre-norm + MoE block + fused post-norm and scaled residual "
                                    "(step k=9); stage_ms/roofline are from the plain block's profiled launches")
@@ -522,7 +613,9 @@ def run_dense(args):
     e1.record()
     ranks.barrier()
     clocks.mark()
-    clk = clocks.stop()
+    clocks.stop()
+    clk = clocks.summary(clocks.marks[0], clocks.marks[-1])
+    clocks.cleanup()
     assert bm.device_status() == bm.OK
     ms = ranks.max(e0.elapsed_time(e1)) / args.steps
     flops = 6.0 * T * H * I

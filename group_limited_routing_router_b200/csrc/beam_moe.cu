@@ -811,25 +811,33 @@ namespace {
 static __device__ __align__(256) int32_t g_noalloc_scratch[BEAM_MOE_NOALLOC_SCRATCH_INTS];
 
 struct NoallocSlot {
-    std::once_flag once;
-    int status = BEAM_MOE_ERR_CUDA;
-    int32_t *ptr = nullptr;  // device address of g_noalloc_scratch on this device
+    std::mutex mu;
+    std::atomic<int32_t *> ptr{nullptr};  // device address of g_noalloc_scratch on this device
 };
 NoallocSlot g_noalloc[kMaxDevices];
 
-// On the first call for a device (that device current): resolve the array's device address.  The
-// name g_noalloc_scratch in host code only stands in for the symbol; kernels get this address.
+// Resolves the array's device address for the current device `dev` (the name g_noalloc_scratch in
+// host code only stands in for the symbol; kernels get this address).  Only a successful lookup is
+// kept: after a failure (for example a first call made during stream capture) the next call tries
+// again.
 int noalloc_scratch(int dev, int32_t **out) {
     NoallocSlot &s = g_noalloc[dev];
-    std::call_once(s.once, [&]() {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) == cudaSuccess && p) {
-            s.ptr = static_cast<int32_t *>(p);
-            s.status = BEAM_MOE_OK;
+    int32_t *p = s.ptr.load(std::memory_order_acquire);
+    if (!p) {
+        std::lock_guard<std::mutex> lock(s.mu);
+        p = s.ptr.load(std::memory_order_relaxed);
+        if (!p) {
+            void *addr = nullptr;
+            if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || !addr) {
+                cudaGetLastError();  // clear this error so that a later launch check does not report it
+                return BEAM_MOE_ERR_CUDA;
+            }
+            p = static_cast<int32_t *>(addr);
+            s.ptr.store(p, std::memory_order_release);
         }
-    });
-    *out = s.ptr;
-    return s.status;
+    }
+    *out = p;
+    return BEAM_MOE_OK;
 }
 
 }  // namespace

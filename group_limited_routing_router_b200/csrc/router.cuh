@@ -215,7 +215,9 @@ __global__ void __cluster_dims__(kRtCluster, 1, 1) __launch_bounds__(kRtThreads,
             }
             const float s = 1.0f / (1.0f + expf(-logit));
             sc[j] = s;
-            sel[j] = (e < p.E) ? (p.bias ? s + p.bias[e] : s) : -INFINITY;
+            const float v = p.bias ? s + p.bias[e] : s;
+            // a NaN (from NaN in x, W_r or the bias) ranks below every number, so the ids stay in [0, E)
+            sel[j] = (e < p.E && v == v) ? v : -INFINITY;
         }
 
         // group scores: sum of the group's top group_topn selection values, in pick order

@@ -111,6 +111,8 @@ BEAM_MOE_API size_t beam_moe_workspace_size(const beam_moe_config *cfg, int64_t 
  *   sel_bias  [E]     fp32   selection bias, or NULL for none
  *   topk_ids  [T, k]  int32  out: chosen experts, slot j = j-th best selection value
  *   topk_w    [T, k]  fp32   out: sigmoid score / sum of the chosen scores (sums to 1 per token)
+ * A NaN selection value (NaN in x, w_router or sel_bias) ranks below every number: the ids stay
+ * valid, distinct and inside the kept groups, and the weights of such a token may be NaN.
  */
 BEAM_MOE_API int beam_moe_route(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const float *w_router,
                    const float *sel_bias, int32_t *topk_ids, float *topk_w, void *stream);
@@ -295,7 +297,9 @@ BEAM_MOE_API int beam_moe_forward_nvfp4(const beam_moe_config *cfg, int64_t T, c
  *     enqueue nothing.
  *   - The array exists once per device that loads the library and stays allocated until the
  *     process exits.  The first call on a device, with that device current, looks up the array's
- *     device address (cudaGetSymbolAddress); make that first call before any stream capture.
+ *     device address (cudaGetSymbolAddress); make that first call before any stream capture.  If
+ *     the lookup fails the call returns BEAM_MOE_ERR_CUDA and enqueues nothing; only a successful
+ *     lookup is kept, so the next call on that device tries again.
  *   - Allocates nothing (no cudaMalloc, cudaFree or allocating library call).  Every call shares
  *     the one array and it keeps the previous call's contents; each call overwrites every entry it
  *     reads, so nothing needs clearing.  Calls whose executions overlap on the GPU (different

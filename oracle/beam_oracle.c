@@ -402,6 +402,7 @@ int oracle_dequant_mxfp8(int64_t rows, int K, const uint8_t *q, const uint8_t *s
 {
     if (K % 32) return -1;
     int bad = 0;
+    #pragma omp parallel for schedule(static) reduction(|:bad)
     for (int64_t r = 0; r < rows; ++r)
         for (int k = 0; k < K; ++k) {
             const uint8_t c = scale[(int64_t)(k / 32) * rows + r];
@@ -429,7 +430,7 @@ int oracle_dequant_mxfp8(int64_t rows, int K, const uint8_t *q, const uint8_t *s
  * w[row][k] = e2m1(code(row, k)) * e4m3(scale[k/16][row]) * global, with two codes per byte:
  * element k of a row is the low nibble of byte k/2 when k is even, the high nibble when k is odd.
  * q [rows, K/2] uint8; scale [K/16, rows] uint8; out [rows, K] fp64.  Returns -1 (out undefined)
- * for a scale code with the sign bit set or a NaN scale code.
+ * when any scale code has the sign bit set or is NaN.
  */
 static double e2m1_value(uint8_t nibble)
 {
@@ -442,17 +443,18 @@ int oracle_dequant_nvfp4(int64_t rows, int K, const uint8_t *q, const uint8_t *s
                          double *out)
 {
     if (K % 16) return -1;
+    int bad = 0;
+    #pragma omp parallel for schedule(static) reduction(|:bad)
     for (int64_t r = 0; r < rows; ++r)
         for (int k = 0; k < K; ++k) {
             const uint8_t c = scale[(int64_t)(k / 16) * rows + r];
-            if (c & 0x80) return -1;
             const double sv = e4m3_value(c);
-            if (isnan(sv)) return -1;
+            if ((c & 0x80) || isnan(sv)) { bad = 1; out[r * K + k] = 0.0; continue; }
             const uint8_t byte = q[r * (K / 2) + k / 2];
             const uint8_t nib = (k & 1) ? (byte >> 4) : (byte & 15);
             out[r * K + k] = e2m1_value(nib) * sv * global;
         }
-    return 0;
+    return bad ? -1 : 0;
 }
 
 /*

@@ -9,11 +9,24 @@ Routing protocol (the pages fix no tie rule; the oracle's reading is lower index
     1e-6 (compared per expert id);
   * tokens below a margin are excluded from the bit-exact comparison, counted, and must still be a
     valid choice: at most topk_groups groups, whose total group score is within 1e-6 of the best
-    possible, and experts whose total selection value is within 1e-6 of the best inside them.
-Output protocol: |y_gpu - y_oracle| <= 2e-2 * RMS(y_oracle) + half_ulp_bf16(y_oracle) elementwise over
-the compared tokens.  The second term is the rounding of the exact result to the BF16 output format
-itself (up to 2^-8 |y|, about 0.02 RMS at the 5-sigma elements of a 21M-element output), which no
-BF16 output can avoid; the raw max |err| / RMS is reported beside it.
+    possible, and experts whose total selection value is within 1e-6 of the best inside them.  The
+    output of every excluded token whose set differs is still checked: the oracle recomputes it from
+    the GPU's expert ids (oracle_y_checked).
+
+Output protocol (compare_y), for y_gpu (BF16) against the oracle's FP64 y, RMS = RMS(y_oracle):
+  * literal bound where BF16 can meet it: on every element whose BF16 spacing is fine enough that
+    rounding alone uses at most a quarter of the budget (half a BF16 ulp of y_oracle <= 5e-3 RMS,
+    which holds for |y_oracle| below 1.28 to 2.56 RMS, by where the binades fall), the literal
+    max |y_gpu - y_oracle| <= 2e-2 RMS;
+  * every element: y_gpu must be the round-to-nearest BF16 value of some v with
+    |v - y_oracle| <= 2e-2 RMS, i.e. the distance from y_oracle to y_gpu's BF16 rounding interval is
+    at most 2e-2 RMS.  Where |y_oracle| is above ~5 RMS, half a BF16 ulp is itself more than 1e-2 RMS
+    (and above 8 RMS more than 2e-2 RMS), so the raw difference of a correctly rounded output can
+    exceed 2e-2 RMS with no error in the computation at all;
+  * reported, not enforced: the raw max |y_gpu - y_oracle| / RMS (the literal quantity), the same
+    against bf16(y_oracle), and how many elements differ from bf16(y_oracle) by more than 2e-2 RMS and
+    by exactly one BF16 step (an FP32 result and the exact one on opposite sides of a rounding
+    midpoint: one step is 0.031 RMS at |y| in [4, 8) RMS).
 """
 from __future__ import annotations
 
@@ -32,9 +45,12 @@ def to_dev(t: torch.Tensor) -> torch.Tensor:
 
 
 class Case:
-    """Inputs of one workload on the GPU plus what the oracle needs on the host."""
+    """Inputs of one workload on the GPU plus what the oracle needs on the host.
 
-    def __init__(self, wl: bs.Workload, T=None, weights=None):
+    weights: the experts as GPU tensors (drawn here when None); host: the same weights as host bf16
+    bit arrays (the oracle then reads them instead of copying each expert back from the GPU)."""
+
+    def __init__(self, wl: bs.Workload, T=None, weights=None, host=None):
         self.wl = wl
         self.T = wl.T if T is None else T
         self.layer = wl.layer
@@ -51,9 +67,12 @@ class Case:
             wg, wu, wd = bs.make_experts(wl)
             weights = (to_dev(wg), to_dev(wu), to_dev(wd))
         self.wg, self.wu, self.wd = weights
+        self.host = host
         self._route = None
 
     def fetch(self, e: int):
+        if self.host is not None:
+            return tuple(h[e] for h in self.host)
         return (oracle.bf16_bits(self.wg[e]), oracle.bf16_bits(self.wu[e]), oracle.bf16_bits(self.wd[e]))
 
     def oracle_route(self):
@@ -113,6 +132,48 @@ def compare_routing(r: dict, layer: dict, ids_gpu: np.ndarray, w_gpu: np.ndarray
                 n_near_miss=int((np.min(margin[:, :2], axis=1) < 1e-5).sum() - (~sel_clear).sum()))
 
 
+def oracle_weights_for(score: np.ndarray, ids: np.ndarray) -> np.ndarray:
+    """The oracle's normalised weights for a given choice of experts: its FP64 sigmoid scores of those
+    experts divided by their sum (the normalisation step, applied to another expert set)."""
+    s = np.take_along_axis(score, ids.astype(np.int64), 1)
+    return s / s.sum(1, keepdims=True)
+
+
+def oracle_y_checked(route: dict, st: dict, ids_gpu: np.ndarray, tokens: np.ndarray, y_oracle_route: np.ndarray,
+                     y_of) -> np.ndarray:
+    """Oracle outputs for `tokens` to compare with a GPU forward pass: the oracle's own outputs
+    (y_oracle_route, rows aligned with tokens) where the GPU chose the oracle's expert set, and, for
+    excluded tokens where it chose another valid set, the oracle recomputed on the GPU's ids with
+    the oracle's weights for them.  y_of(ids, w, tokens) runs the oracle's expert half."""
+    y = np.array(y_oracle_route, copy=True)
+    diff = np.nonzero(~st["set_equal"][tokens])[0]
+    if diff.size:
+        tk = tokens[diff]
+        ids = np.zeros_like(route["ids"])
+        w = np.zeros_like(route["weight"])
+        ids[tk] = ids_gpu[tk]
+        w[tk] = oracle_weights_for(route["score"][tk], ids_gpu[tk])
+        y[diff] = y_of(ids, w, tk)
+    return y
+
+
+def bf16_interval(y_gpu: np.ndarray):
+    """Lower and upper ends of the set of real values that round (to nearest) to each BF16 value:
+    the value +- half the spacing to its lower / upper BF16 neighbour."""
+    b = oracle.f64_to_bf16_bits(y_gpu).astype(np.int32)  # exact: y_gpu already holds BF16 values
+    mag = b & 0x7FFF
+    sign = np.where(b & 0x8000, -1.0, 1.0)
+    up = oracle.bf16_bits_to_f64(np.minimum(mag + 1, 0x7F7F).astype(np.uint16))
+    dn = oracle.bf16_bits_to_f64(np.maximum(mag - 1, 0).astype(np.uint16))
+    a = oracle.bf16_bits_to_f64(mag.astype(np.uint16))
+    half_up = (up - a) / 2
+    half_dn = np.where(mag == 0, half_up, (a - dn) / 2)
+    lo_mag, hi_mag = a - half_dn, a + half_up
+    lo = np.where(sign > 0, lo_mag, -hi_mag)
+    hi = np.where(sign > 0, hi_mag, -lo_mag)
+    return lo, hi
+
+
 def half_ulp_bf16(y: np.ndarray) -> np.ndarray:
     """Half a BF16 unit in the last place at |y| (8 significant bits): 2^(floor(log2|y|) - 8)."""
     a = np.abs(y)
@@ -122,15 +183,34 @@ def half_ulp_bf16(y: np.ndarray) -> np.ndarray:
 
 def compare_y(y_gpu: np.ndarray, y_or: np.ndarray, what: str = "y") -> dict:
     y_gpu = y_gpu.astype(np.float64)
+    if y_or.size == 0:
+        return dict(max_err=0.0, rms=0.0, rel=0.0, rel_dist=0.0, rel_vs_bf16=0.0, n_over_vs_bf16=0,
+                    n_one_step=0, rows_within_own_rms=1.0)
     err = np.abs(y_gpu - y_or)
-    rms = float(np.sqrt(np.mean(y_or ** 2))) if y_or.size else 0.0
-    max_err = float(err.max()) if err.size else 0.0
-    excess = err - half_ulp_bf16(y_or)
-    max_excess = float(excess.max()) if err.size else 0.0
-    assert max_excess <= Y_TOL * rms, \
-        f"{what}: max(|err| - half ulp) {max_excess:.4g} > {Y_TOL} * RMS {rms:.4g} (raw max|err| {max_err:.4g})"
-    row_rms = np.sqrt(np.mean(y_or ** 2, axis=1)) if y_or.size else np.zeros(0)
-    row_ok = np.all(excess <= Y_TOL * row_rms[:, None] + 1e-30, axis=1) if y_or.size else np.zeros(0, bool)
+    rms = float(np.sqrt(np.mean(y_or ** 2)))
+    tol = Y_TOL * rms
+    max_err = float(err.max())
+    # literal bound wherever BF16 rounding alone takes at most a quarter of it
+    fine = half_ulp_bf16(y_or) <= 0.25 * tol
+    lit = float(err[fine].max()) if fine.any() else 0.0
+    assert lit <= tol, f"{what}: max |err| {lit:.4g} > {Y_TOL} * RMS {rms:.4g} on the elements with fine BF16 spacing"
+    # everywhere: distance from y_oracle to the BF16 rounding interval of y_gpu
+    lo, hi = bf16_interval(y_gpu)
+    dist = np.maximum(0.0, np.maximum(lo - y_or, y_or - hi))
+    max_dist = float(dist.max())
+    assert max_dist <= tol, \
+        f"{what}: y_oracle lies {max_dist:.4g} from the BF16 rounding interval of y_gpu > {Y_TOL} * RMS {rms:.4g}"
+    # reported: against the oracle rounded to BF16
+    yb = oracle.bf16_bits_to_f64(oracle.f64_to_bf16_bits(y_or))
+    eb = np.abs(y_gpu - yb)
+    over = eb > tol
+    bg = oracle.f64_to_bf16_bits(y_gpu).astype(np.int32)
+    bo = oracle.f64_to_bf16_bits(y_or).astype(np.int32)
+    one_step = over & (np.abs(bg - bo) == 1)
+    row_rms = np.sqrt(np.mean(y_or ** 2, axis=1))
+    row_ok = np.all(dist <= Y_TOL * row_rms[:, None] + 1e-30, axis=1)
     return dict(max_err=max_err, rms=rms, rel=max_err / rms if rms else 0.0,
-                rel_excess=max_excess / rms if rms else 0.0,
-                rows_within_own_rms=float(row_ok.mean()) if row_ok.size else 1.0)
+                rel_fine=lit / rms if rms else 0.0, rel_dist=max_dist / rms if rms else 0.0,
+                rel_vs_bf16=float(eb.max()) / rms if rms else 0.0, n_over_vs_bf16=int(over.sum()),
+                n_one_step=int(one_step.sum()), n_elements=int(y_or.size),
+                rows_within_own_rms=float(row_ok.mean()))

@@ -88,9 +88,9 @@ def test_block_beam_small_T(beam_weights):
     _check(parity.Case(bs.get("beam_small_T"), weights=beam_weights), 9)
 
 
-def test_block_prefill_sampled(beam_weights):
+def test_block_prefill_sampled(bank):
     wl = bs.get("prefill")
-    _check(parity.Case(wl, weights=beam_weights), 11, tokens=bs.sample_tokens(wl, 24))
+    _check(bank.case("prefill"), 11, tokens=bs.sample_tokens(wl, 64))
 
 
 def test_block_in_place_equals_out_of_place():

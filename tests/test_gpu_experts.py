@@ -1,12 +1,12 @@
 """Expert half (dispatch, gate/up + SwiGLU GEMM, down GEMM, combine) vs the CPU oracle, on the
-oracle's own routing: max |y - y_oracle| <= 2e-2 * RMS(y_oracle)."""
+oracle's own routing, under the output protocol of tests/parity.py (compare_y)."""
 import numpy as np
 import pytest
 import torch
 
 import beam_synth as bs
 import group_limited_routing_router_b200 as bm
-from tests import parity
+from tests import fullsize, parity
 
 pytestmark = pytest.mark.gpu
 
@@ -33,17 +33,16 @@ def test_experts_small(name, beam_weights):
     print(f"{name}: {st}")
 
 
-@pytest.mark.parametrize("name,n_sample", [("decode", 48), ("prefill", 32), ("skew", 32), ("long", 16)])
-def test_experts_full_size_sampled(name, n_sample, beam_weights):
-    wl = bs.get(name)
-    case = parity.Case(wl, weights=beam_weights)
+@pytest.mark.parametrize("name", fullsize.FULL)
+def test_experts_full_size(name, bank):
+    """The expert half on the oracle's routing at full size; outputs on the workload's token sample."""
+    case = bank.case(name)
     r = case.oracle_route()
     y = _experts(case, r["ids"], r["weight"])
-    out = bs.outlier_rows(wl)
-    tok = bs.sample_tokens(wl, n_sample, include=out[:16])
-    st = parity.compare_y(y[tok], case.oracle_y(r["ids"], r["weight"], tok), name)
-    print(f"{name}: sampled {len(tok)} tokens: {st}")
     assert np.isfinite(y).all()
+    tok = fullsize.sample(name)
+    st = parity.compare_y(y[tok], bank.oracle_y("bf16", name), name)
+    print(f"{name}: {len(tok)} tokens: {st}")
 
 
 def test_experts_k1_and_ragged_tokens():
@@ -54,8 +53,8 @@ def test_experts_k1_and_ragged_tokens():
     parity.compare_y(y, case.oracle_y(r["ids"], r["weight"], np.arange(wl.T)), "k1")
 
 
-def test_experts_deterministic(beam_weights):
-    case = parity.Case(bs.get("prefill"), weights=beam_weights)
+def test_experts_deterministic(bank):
+    case = bank.case("prefill")
     r = case.oracle_route()
     a = _experts(case, r["ids"], r["weight"])
     b = _experts(case, r["ids"], r["weight"])

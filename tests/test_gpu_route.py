@@ -30,9 +30,9 @@ def test_route_small(name, beam_weights):
 
 
 @pytest.mark.parametrize("name", ["decode", "prefill", "skew", "long"])
-def test_route_full_size(name, beam_weights):
+def test_route_full_size(name, bank):
     wl = bs.get(name)
-    case = parity.Case(wl, weights=beam_weights)
+    case = bank.case(name)
     ids, w = _route_gpu(case)
     st = parity.compare_routing(case.oracle_route(), case.layer, ids, w, case.bias_np)
     print(f"{name}: T={wl.T} excluded={st['n_excluded']} (same set {st['n_excluded_same_set']}) "
@@ -49,8 +49,8 @@ def test_route_full_size(name, beam_weights):
         assert counts.max() > 10 * mean and (counts == 0).sum() >= 8
 
 
-def test_route_deterministic(beam_weights):
-    case = parity.Case(bs.get("prefill"), weights=beam_weights)
+def test_route_deterministic(bank):
+    case = bank.case("prefill")
     a = bm.route(case.layer, case.x, case.w_router)
     b = bm.route(case.layer, case.x, case.w_router)
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])

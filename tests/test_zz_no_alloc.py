@@ -5,8 +5,9 @@ whose host framework owns all device memory, or a latency-critical loop where an
 synchronise the device.  For them the library offers a dispatch entry point whose scratch is a fixed
 array inside the library (256 KiB per device, enough for 65,536 tokens at 256 experts).  These tests
 call it through the C ABI and require outputs identical to the workspace entry point's, on
-consecutive calls that reuse the shared array with different sizes.  The file is named so that pytest
-collects it after every other test.
+consecutive calls that reuse the shared array with different sizes.  Its tests carry the `last`
+marker, which the collection hook in conftest.py moves behind every other test (the file name sorts
+last as well), so a run that stops at the first failure has run everything else first.
 """
 import ctypes
 
@@ -52,6 +53,7 @@ def _noalloc(layer, ids_dev):
 
 
 @pytest.mark.gpu
+@pytest.mark.last
 def test_noalloc_permute_matches_workspace_permute_on_consecutive_calls():
     cases = [(_layer(256, 8), _ids(4096, 256, 8, 1)),     # Beam prefill shape
              (_layer(64, 6), _ids(777, 64, 6, 2)),        # smaller call: the array keeps stale entries
@@ -67,6 +69,7 @@ def test_noalloc_permute_matches_workspace_permute_on_consecutive_calls():
             assert torch.equal(got[key], ref[key]), key
 
 
+@pytest.mark.last
 def test_noalloc_permute_rejects_sizes_beyond_its_array():
     layer = _layer(256, 8)
     p = ctypes.c_void_p(4096)  # never dereferenced: the size check fails first
