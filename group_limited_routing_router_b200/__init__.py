@@ -122,6 +122,13 @@ def lib() -> ctypes.CDLL:
         L.beam_moe_dense_swiglu.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp,
                                             _vp, ctypes.c_size_t, _vp]
         L.beam_moe_dense_swiglu.restype = ctypes.c_int
+        L.beam_moe_gather_rows.argtypes = [_cfgp, ctypes.c_int64, _vp, _vp, _vp, _vp]
+        L.beam_moe_expert_rows_workspace_size.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                                          ctypes.c_int64]
+        L.beam_moe_expert_rows_workspace_size.restype = ctypes.c_size_t
+        L.beam_moe_expert_rows.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int64, _vp, _vp,
+                                           _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+        L.beam_moe_combine.argtypes = [_cfgp, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp]
         L.beam_moe_device_status.argtypes = [_vp]
         L.beam_moe_selftest_timeout.argtypes = [ctypes.c_int64, _vp]
         L.beam_moe_strerror.argtypes = [ctypes.c_int]
@@ -129,7 +136,7 @@ def lib() -> ctypes.CDLL:
         for name in ("beam_moe_route", "beam_moe_permute", "beam_moe_experts", "beam_moe_forward",
                      "beam_moe_forward_profiled", "beam_moe_block_forward", "beam_moe_experts_fp8",
                      "beam_moe_forward_fp8", "beam_moe_experts_nvfp4", "beam_moe_forward_nvfp4",
-                     "beam_moe_device_status",
+                     "beam_moe_device_status", "beam_moe_gather_rows", "beam_moe_expert_rows", "beam_moe_combine",
                      "beam_moe_selftest_timeout"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -271,6 +278,57 @@ def forward(cfg, x, w_router, bias, w_gate, w_up, w_down, y=None, ids=None, w=No
                                   _ptr(w_up), _ptr(w_down), _ptr(y), _ptr(ids), _ptr(w), _ptr(ws), nbytes,
                                   _stream(stream)), "beam_moe_forward")
     return (y, ids, w) if return_routing else y
+
+
+def gather_rows(cfg, x: torch.Tensor, dest_row: torch.Tensor, out: Optional[torch.Tensor] = None,
+                stream=None) -> torch.Tensor:
+    """Token rows in dispatch order: out[dest_row[t*k + j]] = x[t] -> [T*k, H] bf16."""
+    c = _cfg(cfg)
+    T = x.shape[0]
+    _dev(x, "x", torch.bfloat16, (T, c.hidden))
+    _dev(dest_row, "dest_row", torch.int32, (T * c.topk,))
+    out = torch.empty(T * c.topk, c.hidden, dtype=torch.bfloat16, device=x.device) if out is None else out
+    _dev(out, "out", torch.bfloat16, (T * c.topk, c.hidden))
+    _check(lib().beam_moe_gather_rows(ctypes.byref(c), T, _ptr(x), _ptr(dest_row), _ptr(out), _stream(stream)),
+           "beam_moe_gather_rows")
+    return out
+
+
+def expert_rows(x_rows: torch.Tensor, row_expert: torch.Tensor, w_gate, w_up, w_down,
+                out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The experts on rows that each name one (local) expert: [R, H] fp32, unweighted, in row order."""
+    R, H = x_rows.shape
+    E, I, _ = w_gate.shape
+    _dev(x_rows, "x_rows", torch.bfloat16, (R, H))
+    _dev(row_expert, "row_expert", torch.int32, (R,))
+    _dev(w_gate, "w_gate", torch.bfloat16, (E, I, H))
+    _dev(w_up, "w_up", torch.bfloat16, (E, I, H))
+    _dev(w_down, "w_down", torch.bfloat16, (E, H, I))
+    out = torch.empty(R, H, dtype=torch.float32, device=x_rows.device) if out is None else out
+    _dev(out, "out", torch.float32, (R, H))
+    need = int(lib().beam_moe_expert_rows_workspace_size(H, I, E, R))
+    if ws is None:
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=x_rows.device)
+    _dev(ws, "ws", torch.uint8)
+    _check(lib().beam_moe_expert_rows(H, I, E, R, _ptr(x_rows), _ptr(row_expert), _ptr(w_gate), _ptr(w_up),
+                                      _ptr(w_down), _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
+           "beam_moe_expert_rows")
+    return out
+
+
+def combine(cfg, o_rows: torch.Tensor, dest_row: torch.Tensor, w: torch.Tensor, y: Optional[torch.Tensor] = None,
+            stream=None) -> torch.Tensor:
+    """y [T,H] bf16 = routed_scale * sum_j w[t,j] * o_rows[dest_row[t*k+j]] (FP32, slot order)."""
+    c = _cfg(cfg)
+    T = w.shape[0]
+    _dev(o_rows, "o_rows", torch.float32, (T * c.topk, c.hidden))
+    _dev(dest_row, "dest_row", torch.int32, (T * c.topk,))
+    _dev(w, "w", torch.float32, (T, c.topk))
+    y = torch.empty(T, c.hidden, dtype=torch.bfloat16, device=o_rows.device) if y is None else y
+    _dev(y, "y", torch.bfloat16, (T, c.hidden))
+    _check(lib().beam_moe_combine(ctypes.byref(c), T, _ptr(o_rows), _ptr(dest_row), _ptr(w), _ptr(y),
+                                  _stream(stream)), "beam_moe_combine")
+    return y
 
 
 FP8_KEYS = ("q_gate", "s_gate", "q_up", "s_up", "q_down", "s_down")

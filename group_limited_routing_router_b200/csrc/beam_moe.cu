@@ -868,3 +868,143 @@ int beam_moe_permute_noalloc(const beam_moe_config *cfg, int64_t T, const int32_
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------------
+// Expert-parallel building blocks: the gather of token rows into dispatch order, the experts on
+// rows that arrive already dispatched (each row with one local expert id, FP32 outputs in the rows'
+// own order), and the weighted combine of dispatch-ordered FP32 expert outputs.  Together with
+// route and permute they are the steps of one rank of an expert-parallel layer whose exchanges
+// (all-to-all of token rows and of expert outputs) the caller makes.
+namespace beam {
+namespace {
+
+struct RowsLayout {
+    size_t hist = 0, counts = 0, offsets = 0, row_src = 0, dest_row = 0, xp = 0, h = 0, total = 0;
+};
+
+bool rows_shape_ok(int32_t H, int32_t I, int32_t E) {
+    return H >= 64 && H <= 65536 && H % 64 == 0 && I >= 64 && I <= 65536 && I % 64 == 0 && E >= 1 && E <= 256;
+}
+
+// Rows per expert decide the tile family as in the forward pass (k = 1: one row per "token").
+bool rows_narrow(int32_t E, int64_t R) { return static_cast<double>(R) / E <= 12.0; }
+
+RowsLayout rows_layout(int32_t H, int32_t I, int32_t E, int64_t R) {
+    RowsLayout L;
+    if (R == 0) return L;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off = align256(off + bytes);
+        return at;
+    };
+    L.hist = take(static_cast<size_t>(n_chunks(R)) * E * 4);
+    L.counts = take(static_cast<size_t>(E) * 4);
+    L.offsets = take((static_cast<size_t>(E) + 1) * 8);
+    L.row_src = take(static_cast<size_t>(R) * 4);
+    L.dest_row = take(static_cast<size_t>(R) * 4);
+    if (!rows_narrow(E, R)) L.xp = take(static_cast<size_t>(R) * H * 2);
+    L.h = take(static_cast<size_t>(R) * I * 2);
+    L.total = off;
+    return L;
+}
+
+}  // namespace
+}  // namespace beam
+
+extern "C" {
+
+int beam_moe_gather_rows(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const int32_t *dest_row,
+                         beam_bf16 *x_rows, void *stream) {
+    int rc = validate(cfg);
+    if (rc) return rc;
+    if ((rc = check_T(cfg, T))) return rc;
+    if (T == 0) return BEAM_MOE_OK;
+    if (!x || !dest_row || !x_rows) return BEAM_MOE_ERR_NULL;
+    if (!aligned16(x) || !aligned16(x_rows)) return BEAM_MOE_ERR_MISALIGNED;
+    int dev;
+    if ((rc = init_device(&dev))) return rc;
+    gather_rows_kernel<<<static_cast<unsigned>(T), 128, 0, static_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const uint4 *>(x), T, cfg->topk, cfg->hidden / 8, dest_row, reinterpret_cast<uint4 *>(x_rows));
+    return launch_status();
+}
+
+size_t beam_moe_expert_rows_workspace_size(int32_t hidden, int32_t inter, int32_t n_experts, int64_t R) {
+    if (!rows_shape_ok(hidden, inter, n_experts) || R < 0 || R > kMaxTokens) return 0;
+    return rows_layout(hidden, inter, n_experts, R).total;
+}
+
+int beam_moe_expert_rows(int32_t hidden, int32_t inter, int32_t n_experts, int64_t R, const beam_bf16 *x_rows,
+                         const int32_t *row_expert, const beam_bf16 *w_gate, const beam_bf16 *w_up,
+                         const beam_bf16 *w_down, float *o_rows, void *ws, size_t ws_bytes, void *stream) {
+    if (!rows_shape_ok(hidden, inter, n_experts)) return BEAM_MOE_ERR_INVALID_CONFIG;
+    if (R < 0 || R > kMaxTokens) return BEAM_MOE_ERR_INVALID_ARG;
+    if (R == 0) return BEAM_MOE_OK;
+    if (!x_rows || !row_expert || !w_gate || !w_up || !w_down || !o_rows || !ws) return BEAM_MOE_ERR_NULL;
+    if (!aligned16(x_rows) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_down) || !aligned16(o_rows) ||
+        !aligned16(ws))
+        return BEAM_MOE_ERR_MISALIGNED;
+    const RowsLayout L = rows_layout(hidden, inter, n_experts, R);
+    if (ws_bytes < L.total) return BEAM_MOE_ERR_WORKSPACE_TOO_SMALL;
+    int dev, rc;
+    if ((rc = init_device(&dev))) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+    int32_t *counts = reinterpret_cast<int32_t *>(wsb + L.counts);
+    int64_t *offsets = reinterpret_cast<int64_t *>(wsb + L.offsets);
+    int32_t *row_src = reinterpret_cast<int32_t *>(wsb + L.row_src);
+    int32_t *dest_row = reinterpret_cast<int32_t *>(wsb + L.dest_row);
+    // each row is a "token" with one expert: the dispatch groups rows by expert, rows in order
+    beam_moe_config c1{hidden, inter, n_experts, 1, 1, 1, 1, 1.0f};
+    if ((rc = enqueue_permute(&c1, R, row_expert, counts, offsets, row_src, dest_row,
+                              reinterpret_cast<int32_t *>(wsb + L.hist), s)))
+        return rc;
+    const bool narrow = rows_narrow(n_experts, R);
+    if (!narrow) {
+        gather_rows_kernel<<<static_cast<unsigned>(R), 128, 0, s>>>(reinterpret_cast<const uint4 *>(x_rows), R, 1,
+                                                                    hidden / 8, dest_row,
+                                                                    reinterpret_cast<uint4 *>(wsb + L.xp));
+        if ((rc = launch_status())) return rc;
+    }
+    const int box = narrow ? kNarrowBox : kWideBox;
+    const int bn = narrow ? kNarrowBN : kWideBN;
+    const double mean_rows = static_cast<double>(R) / n_experts;
+    const int once = (mean_rows + 4.0 * std::sqrt(mean_rows) <= bn) ? 1 : 0;
+    CUtensorMap m_wg, m_wu, m_b1, m_wd, m_h;
+    if (!encode_fn()) return BEAM_MOE_ERR_CUDA;
+    const bool b1_ok = narrow ? make_map_2d(&m_b1, x_rows, hidden, static_cast<uint64_t>(R), 1)
+                              : make_map_2d(&m_b1, wsb + L.xp, hidden, static_cast<uint64_t>(R), box);
+    if (!b1_ok || !make_map_3d(&m_wg, w_gate, hidden, inter, n_experts) ||
+        !make_map_3d(&m_wu, w_up, hidden, inter, n_experts) || !make_map_3d(&m_wd, w_down, inter, hidden, n_experts) ||
+        !make_map_2d(&m_h, wsb + L.h, inter, static_cast<uint64_t>(R), box))
+        return BEAM_MOE_ERR_CUDA;
+    const int grid = g_dev[dev].num_sms;
+    GemmParams p1{counts, offsets, wsb + L.h, n_experts, hidden, inter, once, kDefaultTimeoutCycles, row_src, 1,
+                  nullptr};
+    // the down projection stores dispatch row r at the caller's row row_src[r] (k = 1)
+    GemmParams p2{counts, offsets, o_rows, n_experts, inter, hidden, once, kDefaultTimeoutCycles, nullptr, 1, row_src};
+    if (narrow) launch_gemm<G1_NARROW_ARGS>(grid, s, m_wg, m_wu, m_b1, p1);
+    else launch_gemm<G1_WIDE_ARGS>(grid, s, m_wg, m_wu, m_b1, p1);
+    if ((rc = launch_status())) return rc;
+    if (narrow) launch_gemm<G2_NARROW_ARGS>(grid, s, m_wd, m_wd, m_h, p2);
+    else launch_gemm<G2_WIDE_ARGS>(grid, s, m_wd, m_wd, m_h, p2);
+    return launch_status();
+}
+
+int beam_moe_combine(const beam_moe_config *cfg, int64_t T, const float *o_rows, const int32_t *dest_row,
+                     const float *topk_w, beam_bf16 *y, void *stream) {
+    int rc = validate(cfg);
+    if (rc) return rc;
+    if ((rc = check_T(cfg, T))) return rc;
+    if (T == 0) return BEAM_MOE_OK;
+    if (!o_rows || !dest_row || !topk_w || !y) return BEAM_MOE_ERR_NULL;
+    if (!aligned16(o_rows) || !aligned16(y)) return BEAM_MOE_ERR_MISALIGNED;
+    int dev;
+    if ((rc = init_device(&dev))) return rc;
+    combine_kernel<<<static_cast<unsigned>(T), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const float4 *>(o_rows), dest_row, topk_w, T, cfg->topk, cfg->hidden / 4, cfg->routed_scale,
+        reinterpret_cast<uint2 *>(y));
+    return launch_status();
+}
+
+}  // extern "C"

@@ -68,6 +68,7 @@ struct GemmParams {
     long long timeout;
     const int32_t *row_src;   // GATHER: dispatch row -> (token, slot) pair q; token = q / topk
     int topk;
+    const int32_t *out_row;   // G2 only, nullable: dispatch row r is stored at output row out_row[r]
 };
 
 // Work-item decode from the per-CTA prefix table.
@@ -170,7 +171,11 @@ __device__ __forceinline__ void gemm_epilogue(int q, const int *tile_start, int 
                     float *o = reinterpret_cast<float *>(p.out);
 #pragma unroll
                     for (int j = 0; j < 16; ++j)
-                        if (c + j < it.n_valid) o[(it.row0 + c + j) * p.M + m] = __uint_as_float(r0[j]);
+                        if (c + j < it.n_valid) {
+                            const int64_t r = it.row0 + c + j;
+                            const int64_t dst = p.out_row ? static_cast<int64_t>(__ldg(p.out_row + r)) : r;
+                            o[dst * p.M + m] = __uint_as_float(r0[j]);
+                        }
                 }
             }
         }

@@ -287,6 +287,56 @@ BEAM_MOE_API int beam_moe_forward_nvfp4(const beam_moe_config *cfg, int64_t T, c
                                         void *const *events);
 
 /*
+ * Expert parallelism ("Welcome Beam" page, section "Multi-GPU and multi-node": each expert lives on
+ * one device while the non-expert parameters are replicated; the device count divides 256).  One
+ * rank of an expert-parallel layer over N devices, rank r owning experts [r E/N, (r+1) E/N), runs:
+ *   beam_moe_route, beam_moe_permute        on its own tokens, over all E experts;
+ *   beam_moe_gather_rows                    its token rows in dispatch order (expert-major), so the
+ *                                           rows for rank d are one contiguous block, rows
+ *                                           [offsets[d E/N], offsets[(d+1) E/N]);
+ *   (caller) all-to-all of those blocks     each rank receives the rows for its experts;
+ *   beam_moe_expert_rows                    its local experts on the received rows (FP32 outputs in
+ *                                           the received order);
+ *   (caller) all-to-all back                the outputs return to the token's rank in dispatch order;
+ *   beam_moe_combine                        the weighted sum in slot order, x routed_scale, bf16.
+ * With the same inputs the result is bit-identical to beam_moe_forward on one device: each output
+ * row sees the same GEMM tiles and K order, and the combine the same FP32 order.
+ */
+
+/*
+ * x_rows[dest_row[t k + j]] = x[t] for every token t and slot j (dest_row from beam_moe_permute; a
+ * negative entry, from an invalid id, writes nothing).  x [T, H], x_rows [T k, H] bf16.
+ */
+BEAM_MOE_API int beam_moe_gather_rows(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x,
+                                      const int32_t *dest_row, beam_bf16 *x_rows, void *stream);
+
+/* Workspace bytes of beam_moe_expert_rows for R rows (0 for an invalid shape or R < 0). */
+BEAM_MOE_API size_t beam_moe_expert_rows_workspace_size(int32_t hidden, int32_t inter, int32_t n_experts,
+                                                        int64_t R);
+
+/*
+ * The SwiGLU experts on rows that each name one expert: o_rows[q] = W_down,e (SiLU(W_gate,e x_q) *
+ * (W_up,e x_q)) with e = row_expert[q] in [0, n_experts), in FP32 (SwiGLU product in FP32, h
+ * rounded to bf16 as in the forward pass), unweighted and unscaled, in the rows' own order.
+ *   x_rows [R, H] bf16; row_expert [R] int32; w_gate, w_up [n_experts, I, H], w_down [n_experts, H, I]
+ *   bf16 (the caller's local experts); o_rows [R, H] fp32 out; workspace of
+ *   beam_moe_expert_rows_workspace_size bytes.  An id outside [0, n_experts) sets
+ *   BEAM_MOE_ERR_BAD_INDEX in the status word and leaves that row of o_rows unwritten.
+ */
+BEAM_MOE_API int beam_moe_expert_rows(int32_t hidden, int32_t inter, int32_t n_experts, int64_t R,
+                                      const beam_bf16 *x_rows, const int32_t *row_expert, const beam_bf16 *w_gate,
+                                      const beam_bf16 *w_up, const beam_bf16 *w_down, float *o_rows, void *ws,
+                                      size_t ws_bytes, void *stream);
+
+/*
+ * y[t] = bf16(routed_scale * sum_{j<k} topk_w[t, j] * o_rows[dest_row[t k + j]]), FP32 fused
+ * multiply-adds in slot order from zero, one multiply by routed_scale, round to nearest even.
+ *   o_rows [T k, H] fp32 in dispatch order; dest_row [T k]; topk_w [T, k] fp32; y [T, H] bf16.
+ */
+BEAM_MOE_API int beam_moe_combine(const beam_moe_config *cfg, int64_t T, const float *o_rows,
+                                  const int32_t *dest_row, const float *topk_w, beam_bf16 *y, void *stream);
+
+/*
  * beam_moe_permute without a workspace: the same dispatch (identical outputs), with its scratch in
  * a fixed device array inside this library instead of caller memory.  The Beam pages have no
  * counterpart; this exists for callers that cannot allocate device memory when they enqueue work,
