@@ -17,6 +17,8 @@ section "Mixture of Experts"):
   rmsnorm        - the sublayer norm (section "Residual Stream": normalised before and after)
   scaled_residual- stream update sqrt((k-1)/k) * stream + z / sqrt(k) (same section)
   block_forward  - pre-norm -> block -> post-norm -> scaled residual
+  quant_mxfp8_rows, expert_mlp_mx8, experts_tokens_mx8
+                 - the block-scaled FP8 path: MXFP8 activations (x and h) around the FP8 experts
 """
 from __future__ import annotations
 
@@ -66,6 +68,12 @@ def lib():
         L.oracle_dequant_nvfp4.restype = ctypes.c_int
         L.oracle_expert_mlp_f64.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, _u16p, _dp, _dp, _dp, _dp]
         L.oracle_expert_mlp_f64.restype = None
+        L.oracle_quant_mxfp8_rows.argtypes = [ctypes.c_int64, ctypes.c_int, _dp, ctypes.POINTER(ctypes.c_uint8),
+                                              ctypes.POINTER(ctypes.c_uint8), _dp]
+        L.oracle_quant_mxfp8_rows.restype = ctypes.c_int
+        L.oracle_expert_mlp_mx8.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, _u16p, _u16p, _u16p, _u16p,
+                                            _dp]
+        L.oracle_expert_mlp_mx8.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -315,4 +323,50 @@ def experts_tokens_f64(x_bits: np.ndarray, ids: np.ndarray, weight: np.ndarray, 
             continue
         wg, wu, wd = fetch(e)
         out[rows, slots, :] = expert_mlp_f64(x_bits[rows], wg, wu, wd)
+    return combine(out, weight, routed_scale)
+
+
+def quant_mxfp8_rows(v: np.ndarray):
+    """MXFP8 activation rows (blocks of 32 along the last axis): returns (codes [rows,K] uint8,
+    scale codes [rows,K/32] uint8, dequantised values [rows,K] fp64)."""
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    rows, K = v.shape
+    q = np.empty((rows, K), dtype=np.uint8)
+    sc = np.empty((rows, K // 32), dtype=np.uint8)
+    deq = np.empty((rows, K), dtype=np.float64)
+    u8p = ctypes.POINTER(ctypes.c_uint8)
+    if lib().oracle_quant_mxfp8_rows(rows, K, _ptr(v, _dp), q.ctypes.data_as(u8p), sc.ctypes.data_as(u8p),
+                                     _ptr(deq, _dp)) != 0:
+        raise ValueError("MXFP8 activations: K not a multiple of 32, or a scale outside UE8M0")
+    return q, sc, deq
+
+
+def expert_mlp_mx8(x_rows_bits: np.ndarray, wg_bits: np.ndarray, wu_bits: np.ndarray, wd_bits: np.ndarray):
+    """The block-scaled FP8 path's SwiGLU expert: MXFP8 x, then h quantised to MXFP8 before the down
+    projection (FP64 on the dequantised values); weights as bf16 bits.  Returns [n,H] fp64."""
+    x_rows_bits = np.ascontiguousarray(x_rows_bits, dtype=np.uint16)
+    n, H = x_rows_bits.shape
+    I = wg_bits.shape[0]
+    assert wg_bits.shape == (I, H) and wu_bits.shape == (I, H) and wd_bits.shape == (H, I)
+    out = np.empty((n, H), dtype=np.float64)
+    if n == 0:
+        return out
+    if lib().oracle_expert_mlp_mx8(n, H, I, _ptr(x_rows_bits, _u16p), _ptr(np.ascontiguousarray(wg_bits), _u16p),
+                                   _ptr(np.ascontiguousarray(wu_bits), _u16p),
+                                   _ptr(np.ascontiguousarray(wd_bits), _u16p), _ptr(out, _dp)) != 0:
+        raise ValueError("MXFP8 activations: a scale outside UE8M0")
+    return out
+
+
+def experts_tokens_mx8(x_bits: np.ndarray, ids: np.ndarray, weight: np.ndarray, fetch: ExpertFetch,
+                       n_experts: int, routed_scale: float) -> np.ndarray:
+    """experts_tokens of the block-scaled FP8 path (expert_mlp_mx8 per expert)."""
+    n, H = x_bits.shape
+    k = ids.shape[1]
+    out = np.zeros((n, k, H), dtype=np.float64)
+    for e in range(n_experts):
+        rows, slots = np.nonzero(ids == e)
+        if rows.size == 0:
+            continue
+        out[rows, slots, :] = expert_mlp_mx8(x_bits[rows], *fetch(e))
     return combine(out, weight, routed_scale)

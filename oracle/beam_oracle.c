@@ -492,3 +492,140 @@ void oracle_expert_mlp_f64(int64_t n, int H, int I, const uint16_t *x_rows, cons
     free(xb);
     free(hb);
 }
+
+/*
+ * MXFP8 activations for the block-scaled FP8 path (reading; the pages name FP8 checkpoints but
+ * give no recipe, and a tensor-core product of FP8 weights needs FP8 activations too).  OCP MXFP8
+ * applied to activation rows: every block of 32 consecutive K elements of a row shares one UE8M0
+ * scale 2^(c - 127), c = 127 + the smallest integer e with amax <= 448 * 2^e (amax = the block's
+ * largest magnitude; c = 0 for an all-zero block), and each element becomes the E4M3 value nearest
+ * to v * 2^(127 - c), ties to even.  The layer then computes on the dequantised values.
+ */
+static uint8_t e4m3_round_code(double a)  /* |a| <= 448: nearest E4M3 value, ties to even */
+{
+    const int s = signbit(a) ? 1 : 0;
+    const double m = fabs(a);
+    const int e = m >= ldexp(1.0, -6) ? ilogb(m) : -6;   /* subnormals share the quantum 2^-9 */
+    const double quantum = ldexp(1.0, e - 3);
+    const double r = nearbyint(m / quantum) * quantum;    /* default rounding mode: half to even */
+    if (r == 0.0) return (uint8_t)(s << 7);
+    const int re = ilogb(r);
+    if (re < -6) return (uint8_t)((s << 7) | (int)ldexp(r, 9));            /* subnormal: r = m 2^-9 */
+    const int mant = (int)(ldexp(r, -re) * 8.0) - 8;
+    return (uint8_t)((s << 7) | ((re + 7) << 3) | mant);
+}
+
+/* The UE8M0 scale code of a block with largest magnitude amax (finite). */
+static int mx_scale_code(double amax)
+{
+    if (amax == 0.0) return 0;
+    int e = ilogb(amax) - 8;
+    if (amax > ldexp(448.0, e)) e += 1;
+    return e + 127;
+}
+
+/*
+ * rows x K activations v (fp64) -> E4M3 codes q [rows,K], scale codes scale [rows,K/32] and the
+ * dequantised values deq [rows,K] (fp64; any of q, scale may be NULL).  Returns -1 if K % 32 or a
+ * scale code falls outside 1..254 (an exponent UE8M0 cannot hold).
+ */
+int oracle_quant_mxfp8_rows(int64_t rows, int K, const double *v, uint8_t *q, uint8_t *scale, double *deq)
+{
+    if (K % 32) return -1;
+    int bad = 0;
+    #pragma omp parallel for schedule(static) reduction(|:bad)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int kb = 0; kb < K / 32; ++kb) {
+            const double *blk = v + r * K + kb * 32;
+            double amax = 0.0;
+            for (int i = 0; i < 32; ++i) amax = fmax(amax, fabs(blk[i]));
+            const int c = mx_scale_code(amax);
+            if (amax != 0.0 && (c < 1 || c > 254)) { bad = 1; continue; }
+            if (scale) scale[r * (K / 32) + kb] = (uint8_t)c;
+            for (int i = 0; i < 32; ++i) {
+                const uint8_t code = amax == 0.0 ? 0 : e4m3_round_code(ldexp(blk[i], 127 - c));
+                if (q) q[r * K + kb * 32 + i] = code;
+                deq[r * K + kb * 32 + i] = amax == 0.0 ? 0.0 : ldexp(e4m3_value(code), c - 127);
+            }
+        }
+    return bad ? -1 : 0;
+}
+
+/*
+ * The SwiGLU expert of the block-scaled FP8 path on n rows: x~ = MXFP8(x) per row, g = Wg x~,
+ * u = Wu x~, h = SiLU(g) * u, h~ = MXFP8(h) per row (blocks of 32 along the intermediate axis),
+ * out = Wd h~, all in FP64 on the dequantised values.  Weights are bf16 bits (an MXFP8 checkpoint's
+ * dequantised weights are bf16 values).  x_rows [n,H] bf16 bits; wg, wu [I,H]; wd [H,I]; out [n,H].
+ * Returns -1 for an activation block whose scale UE8M0 cannot hold.
+ */
+int oracle_expert_mlp_mx8(int64_t n, int H, int I, const uint16_t *x_rows, const uint16_t *wg,
+                          const uint16_t *wu, const uint16_t *wd, double *out)
+{
+    if (H % 32 || I % 32) return -1;
+    const int64_t nb = (n + RB - 1) / RB;
+    double *xd = (double *)malloc(sizeof(double) * (size_t)(n * H));
+    double *xq = (double *)malloc(sizeof(double) * (size_t)(n * H));
+    double *hd = (double *)malloc(sizeof(double) * (size_t)(n * I));
+    double *hq = (double *)malloc(sizeof(double) * (size_t)(n * I));
+    double *xb = (double *)malloc(sizeof(double) * (size_t)(nb * H * RB));
+    double *hb = (double *)malloc(sizeof(double) * (size_t)(nb * I * RB));
+    int rc = 0;
+    for (int64_t q = 0; q < n * H; ++q) xd[q] = bf16_bits_to_double(x_rows[q]);
+    if (oracle_quant_mxfp8_rows(n, H, xd, NULL, NULL, xq)) { rc = -1; goto done; }
+    /* x~ in the blocked layout of dot_rows */
+    for (int64_t b = 0; b < nb; ++b)
+        for (int h = 0; h < H; ++h)
+            for (int r = 0; r < RB; ++r)
+                xb[(b * H + h) * RB + r] = b * RB + r < n ? xq[(b * RB + r) * H + h] : 0.0;
+
+    #pragma omp parallel
+    {
+        double *wgr = (double *)malloc(sizeof(double) * (size_t)H);
+        double *wur = (double *)malloc(sizeof(double) * (size_t)H);
+        #pragma omp for collapse(2) schedule(static)
+        for (int64_t b = 0; b < nb; ++b)
+            for (int i = 0; i < I; ++i) {
+                for (int h = 0; h < H; ++h) {
+                    wgr[h] = bf16_bits_to_double(wg[(int64_t)i * H + h]);
+                    wur[h] = bf16_bits_to_double(wu[(int64_t)i * H + h]);
+                }
+                double g[RB], u[RB];
+                dot_rows(H, xb + b * H * RB, wgr, g);
+                dot_rows(H, xb + b * H * RB, wur, u);
+                for (int r = 0; r < RB && b * RB + r < n; ++r) {
+                    const double silu_g = g[r] / (1.0 + exp(-g[r]));
+                    hd[(b * RB + r) * I + i] = silu_g * u[r];
+                }
+            }
+        free(wgr);
+        free(wur);
+    }
+    if (oracle_quant_mxfp8_rows(n, I, hd, NULL, NULL, hq)) { rc = -1; goto done; }
+    for (int64_t b = 0; b < nb; ++b)
+        for (int i = 0; i < I; ++i)
+            for (int r = 0; r < RB; ++r)
+                hb[(b * I + i) * RB + r] = b * RB + r < n ? hq[(b * RB + r) * I + i] : 0.0;
+
+    #pragma omp parallel
+    {
+        double *wdr = (double *)malloc(sizeof(double) * (size_t)I);
+        #pragma omp for collapse(2) schedule(static)
+        for (int64_t b = 0; b < nb; ++b)
+            for (int o = 0; o < H; ++o) {
+                const uint16_t *wd_row = wd + (int64_t)o * I;  /* W_down row o */
+                for (int i = 0; i < I; ++i) wdr[i] = bf16_bits_to_double(wd_row[i]);
+                double acc[RB];
+                dot_rows(I, hb + b * I * RB, wdr, acc);
+                for (int r = 0; r < RB && b * RB + r < n; ++r) out[(b * RB + r) * H + o] = acc[r];
+            }
+        free(wdr);
+    }
+done:
+    free(xd);
+    free(xq);
+    free(hd);
+    free(hq);
+    free(xb);
+    free(hb);
+    return rc;
+}

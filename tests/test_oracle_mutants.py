@@ -14,6 +14,7 @@ import pytest
 
 import oracle
 from tests import test_oracle_fp8 as fp8
+from tests import test_oracle_mx8act as mx8
 from tests import test_oracle_nvfp4 as nv4
 from tests import test_oracle_norm_residual as nr
 from tests import test_oracle_pins as pins
@@ -54,6 +55,14 @@ MUTANTS = {
     "nvfp4_nibbles_swapped": ("(k & 1) ? (byte >> 4) : (byte & 15)", "(k & 1) ? (byte & 15) : (byte >> 4)"),
     "nvfp4_scale_row_major": ("scale[(int64_t)(k / 16) * rows + r]", "scale[r * (K / 16) + k / 16]"),
     "nvfp4_global_dropped": ("e2m1_value(nib) * sv * global", "e2m1_value(nib) * sv"),
+    "e4m3_round_truncate": ("const double r = nearbyint(m / quantum) * quantum;",
+                            "const double r = floor(m / quantum) * quantum;"),
+    "mx_scale_too_small": ("if (amax > ldexp(448.0, e)) e += 1;", "if (amax > ldexp(480.0, e)) e += 1;"),
+    "mx8_h_not_quantised": ("hb[(b * I + i) * RB + r] = b * RB + r < n ? hq[(b * RB + r) * I + i] : 0.0;",
+                            "hb[(b * I + i) * RB + r] = b * RB + r < n ? hd[(b * RB + r) * I + i] : 0.0;"),
+    "mx8_silu_missing": ("hd[(b * RB + r) * I + i] = silu_g * u[r];", "hd[(b * RB + r) * I + i] = g[r] * u[r];"),
+    "mx8_x_not_quantised": ("xb[(b * H + h) * RB + r] = b * RB + r < n ? xq[(b * RB + r) * H + h] : 0.0;",
+                            "xb[(b * H + h) * RB + r] = b * RB + r < n ? xd[(b * RB + r) * H + h] : 0.0;"),
     "expert_f64_silu_missing": ("const double act = g[r] / (1.0 + exp(-g[r]));", "const double act = g[r];"),
 }
 
@@ -77,6 +86,9 @@ PINS = [
     nv4.test_even_element_is_the_low_nibble,
     nv4.test_block_scale_per_16_and_global_scale,
     nv4.test_expert_mlp_f64_matches_torch_float64,
+    mx8.test_quantised_rows_match_torch_e4m3_cast_and_scale_rule,
+    mx8.test_ties_round_to_even_code,
+    mx8.test_expert_mx8_matches_torch_float64_composition,
 ]
 
 
