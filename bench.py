@@ -34,6 +34,8 @@ import beam_synth as bs  # noqa: E402
 
 METRIC = "MoE-layer tokens/s (Beam shape, BF16, T=4096) and % of tensor/HBM roofline"
 METRIC_FP8 = "MoE-layer tokens/s (Beam shape, MXFP8 expert weights, T=4096) and % of tensor/HBM roofline"
+METRIC_MXFP8 = ("MoE-layer tokens/s (Beam shape, MXFP8 expert weights and activations on block-scaled tensor cores, "
+                "T=4096) and % of tensor/HBM roofline")
 METRIC_NVFP4 = "MoE-layer tokens/s (Beam shape, NVFP4 expert weights, T=4096) and % of tensor/HBM roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -71,9 +73,12 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--also", default=None,
                     help="comma-separated workloads timed after the headline one in the same process "
-                         "(default: decode,skew,long for bf16, decode for --fp8/--nvfp4, none for --block)")
+                         "(default: decode,skew,long for bf16, decode for --fp8/--mxfp8/--nvfp4, none for --block)")
     ap.add_argument("--cpu-sample", type=int, default=1024, help="tokens in the CPU-oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ep", action="store_true",
+                    help="expert parallelism over the N ranks (E/N experts each, all-to-all dispatch and combine); "
+                         "each rank brings its own batch of the workload (weak scaling)")
     ap.add_argument("--dense", action="store_true",
                     help="time the dense SwiGLU MLP of Beam's first layers (T=4096, intermediate 20480)")
     ap.add_argument("--block", action="store_true",
@@ -82,6 +87,8 @@ def parse():
                     help="NVFP4 expert weights (E2M1 + E4M3 scale per 16 K elements + FP32 per-matrix scale)")
     ap.add_argument("--fp8", action="store_true",
                     help="MXFP8 expert weights (E4M3 + one power-of-two scale per 32 K elements)")
+    ap.add_argument("--mxfp8", action="store_true",
+                    help="the native FP8 path: MXFP8 weights and activations, block-scaled tcgen05 MMA")
     return ap.parse_args()
 
 
@@ -118,7 +125,7 @@ def algorithmic(wl: bs.Workload, n_act: int, fmt: str = "bf16") -> dict:
     scales are negligible)."""
     T, H, I, E, k = wl.T, wl.hidden, wl.inter, wl.n_experts, wl.topk
     R = T * k
-    wb = {"bf16": 2.0, "fp8": 1.0 + 1.0 / 32, "nvfp4": 0.5 + 1.0 / 16}[fmt]  # bytes per expert weight element
+    wb = {"bf16": 2.0, "fp8": 1.0 + 1.0 / 32, "mxfp8": 1.0 + 1.0 / 32, "nvfp4": 0.5 + 1.0 / 16}[fmt]  # bytes per expert weight element
     w_expert = 3 * H * I * wb
     return dict(
         layer_flops=T * (2 * H * E + k * 6 * H * I),
@@ -223,7 +230,7 @@ def nvfp4_fetch(w4):
                                                 float(w4["g_" + n][e].cpu())) for n in ("gate", "up", "down"))
 
 
-def cpu_oracle_rate(wl, x_cpu, W, bias, fetch, n_sample: int, route_all: bool = True, f64_weights: bool = False) -> dict:
+def cpu_oracle_rate(wl, x_cpu, W, bias, fetch, n_sample: int, route_all: bool = True, fmt: str = "bf16") -> dict:
     """Time the CPU oracle: routing (FP64 scores + selection) and the expert half on a token sample.
     fetch(e) gives one expert's bf16 weight bits on the host; it runs outside the timed sections."""
     import oracle
@@ -250,7 +257,8 @@ def cpu_oracle_rate(wl, x_cpu, W, bias, fetch, n_sample: int, route_all: bool = 
             continue
         w3 = fetch(e)
         t1 = time.perf_counter()
-        out[rows, slots, :] = (oracle.expert_mlp_f64 if f64_weights else oracle.expert_mlp)(xs[rows], *w3)
+        expert = {"nvfp4": oracle.expert_mlp_f64, "mxfp8": oracle.expert_mlp_mx8}.get(fmt, oracle.expert_mlp)
+        out[rows, slots, :] = expert(xs[rows], *w3)
         t_exp += time.perf_counter() - t1
     t1 = time.perf_counter()
     oracle.combine(out, wts, wl.routed_scale)
@@ -411,7 +419,7 @@ def run_ours(args):
     wl = bs.get(args.workload)
     layer = wl.layer
     T, H = wl.T, wl.hidden
-    fmt = "nvfp4" if args.nvfp4 else "fp8" if args.fp8 else "bf16"
+    fmt = "nvfp4" if args.nvfp4 else "fp8" if args.fp8 else "mxfp8" if args.mxfp8 else "bf16"
     if args.also is None:
         also = [] if args.block else (["decode", "skew", "long"] if fmt == "bf16" else ["decode"])
     else:
@@ -422,7 +430,7 @@ def run_ours(args):
     if fmt != "bf16":
         if args.block:
             raise SystemExit("--fp8/--nvfp4 and --block: the sublayer entry point takes bf16 expert weights")
-        w8 = bs.quantize_experts(wg, wu, wd) if fmt == "fp8" else bs.quantize_experts_nvfp4(wg, wu, wd)
+        w8 = bs.quantize_experts_nvfp4(wg, wu, wd) if fmt == "nvfp4" else bs.quantize_experts(wg, wu, wd)
         del wg, wu, wd
         wg = wu = wd = None
         torch.cuda.empty_cache()
@@ -441,6 +449,8 @@ def run_ours(args):
                                             stream_out=y, ids=ids, w=w, ws=ws_blk)
         if fmt == "fp8":
             return lambda: bm.forward_fp8(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws)
+        if fmt == "mxfp8":
+            return lambda: bm.forward_mxfp8(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws)
         if fmt == "nvfp4":
             return lambda: bm.forward_nvfp4(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws)
         return lambda: bm.forward(layer, x, W, bias, wg, wu, wd, y=y, ids=ids, w=w, ws=ws)
@@ -449,6 +459,8 @@ def run_ours(args):
         x, W, bias = inp["x"], inp["W"], inp["bias"]
         if fmt == "fp8":
             bm.forward_fp8(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws, events=ev)
+        elif fmt == "mxfp8":
+            bm.forward_mxfp8(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws, events=ev)
         elif fmt == "nvfp4":
             bm.forward_nvfp4(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws, events=ev)
         else:
@@ -545,13 +557,18 @@ def run_ours(args):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        fetch = {"bf16": lambda: bf16_fetch(wg, wu, wd), "fp8": lambda: fp8_fetch(w8),
+        fetch = {"bf16": lambda: bf16_fetch(wg, wu, wd), "fp8": lambda: fp8_fetch(w8), "mxfp8": lambda: fp8_fetch(w8),
                  "nvfp4": lambda: nvfp4_fetch(w8)}[fmt]()
         cpu = cpu_oracle_rate(wl, inp["x_cpu"], inp["W_cpu"], inp["b_cpu"], fetch, args.cpu_sample,
-                              f64_weights=fmt == "nvfp4")
+                              fmt=fmt)
         cpu.pop("seconds", None)
 
     cfg = config_dict(wl)
+    if fmt == "mxfp8":
+        cfg["weights"] = ("MXFP8 experts: E4M3 codes + UE8M0 scale per 32 K elements (1.03 B/weight) and MXFP8 "
+                          "activations (x, h per row, blocks of 32) on tcgen05 kind::mxf8f6f4; router FP32")
+        cfg["weights_bytes"] = int(3 * wl.n_experts * wl.hidden * wl.inter * (1 + 1 / 32))
+        cfg["l2"] = "no flush: every step streams the 10.4 GB of FP8 expert weights and scales (> 126 MB L2)"
     if fmt == "fp8":
         cfg["weights"] = ("MXFP8 experts: E4M3 codes + UE8M0 scale per 32 K elements (1.03 B/weight), rebuilt "
                           "as bf16 in a TMEM ring; router FP32")
@@ -562,8 +579,9 @@ def run_ours(args):
                           "(0.5625 B/weight), rebuilt as bf16 in a TMEM ring; router FP32")
         cfg["weights_bytes"] = int(3 * wl.n_experts * wl.hidden * wl.inter * (0.5 + 1 / 16))
         cfg["l2"] = "no flush: every step streams the 5.7 GB of NVFP4 expert weights and scales (> 126 MB L2)"
-    metric = {"bf16": METRIC, "fp8": METRIC_FP8, "nvfp4": METRIC_NVFP4}[fmt]
-    dtype = {"bf16": "bf16", "fp8": "fp8-e4m3 weights, bf16 MMA", "nvfp4": "nvfp4-e2m1 weights, bf16 MMA"}[fmt]
+    metric = {"bf16": METRIC, "fp8": METRIC_FP8, "mxfp8": METRIC_MXFP8, "nvfp4": METRIC_NVFP4}[fmt]
+    dtype = {"bf16": "bf16", "fp8": "fp8-e4m3 weights, bf16 MMA", "mxfp8": "fp8-e4m3 weights and activations",
+             "nvfp4": "nvfp4-e2m1 weights, bf16 MMA"}[fmt]
     n_launch = launches_per_step(wl, args.block)
     line = {"metric": metric, "value": head["value"], "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
@@ -635,10 +653,59 @@ def run_dense(args):
     ranks.close()
 
 
+def run_ep(args):
+    """Expert-parallel line: N ranks, each with E/N experts and its own batch; tokens/s of all ranks
+    over the slowest rank's device time.  One rank runs the same code with a trivial exchange."""
+    import group_limited_routing_router_b200 as bm
+    from group_limited_routing_router_b200 import ep
+
+    ranks = Ranks("nccl")
+    torch.cuda.set_device(ranks.local)
+    wl = bs.get(args.workload)
+    part = ep.Partition(wl.n_experts, ranks.world)
+    own = part.experts_of(ranks.rank)
+    full = bs.make_experts(wl, device="cuda")  # drawn per expert from its own sub-seed: keep this rank's slice
+    wg, wu, wd = (t[own.start:own.stop].contiguous() for t in full)
+    del full
+    torch.cuda.empty_cache()
+    import dataclasses
+    inp = layer_inputs(dataclasses.replace(wl, seed=wl.seed + 7919 * ranks.rank))
+    rank = ep.Rank(part, ranks.rank, ep.GpuOps(wl.layer, inp["W"], inp["bias"], wg, wu, wd))
+    group = ranks.dist.group.WORLD if ranks.dist is not None else None
+
+    def step():
+        if ranks.dist is None:
+            return ep.forward_emulated([rank], [inp["x"]])[0]
+        return ep.forward(rank, inp["x"], group)
+
+    for _ in range(args.warmup):
+        step()
+    assert bm.device_status() == bm.OK
+    ranks.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        step()
+    e1.record()
+    ranks.barrier()
+    ms = e0.elapsed_time(e1)
+    value = ranks.rate(wl.T * args.steps, ms)
+    line = {"metric": METRIC + " [expert parallel]", "value": value, "unit": "tokens/s", "n_gpus": ranks.world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ranks.max(ms) / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {**config_dict(wl), "parallelism": f"expert parallel: {part.per_rank} experts per rank",
+                       "note": "host-synchronising exchange (split sizes read back); every rank its own batch"}}
+    if ranks.rank == 0:
+        print(json.dumps(line))
+    ranks.close()
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args)
+    elif args.ep:
+        run_ep(args)
     elif args.dense:
         run_dense(args)
     else:

@@ -20,6 +20,7 @@
 #include "permute.cuh"
 #include "gemm.cuh"
 #include "gemm_fp8.cuh"
+#include "gemm_mx8.cuh"
 #include "norm.cuh"
 #include "router.cuh"
 
@@ -53,6 +54,12 @@ constexpr int64_t kMaxTokens = int64_t(1) << 24;
 #define G2_WIDE_NV4_ARGS false, 192, 64, 4, 5, 2, 192, false, 4, true
 #define G1_NARROW_NV4_ARGS true, 32, 1, 4, 12, 2, 64, true, 6, true
 #define G2_NARROW_NV4_ARGS false, 32, 32, 8, 16, 4, 32, false, 12, true
+// Block-scaled FP8 variants (tcgen05 kind::mxf8f6f4): <gate/up?, BN, B box rows, stages (K = 128),
+// TMEM slots, slot columns, gather?>; each stage also holds its scale atoms and TMEM scale columns.
+#define G1_WIDE_MX8_ARGS true, 192, 64, 3, 2, 192, false
+#define G2_WIDE_MX8_ARGS false, 192, 64, 5, 2, 192, false
+#define G1_NARROW_MX8_ARGS true, 32, 1, 5, 4, 64, true
+#define G2_NARROW_MX8_ARGS false, 32, 32, 10, 4, 32, false
 constexpr int kWideBN = 192, kWideBox = 64, kNarrowBN = 32, kNarrowBox = 32;
 
 template <bool G, int BN, int BOXN, int ST, int NS, int SC, bool GA>
@@ -66,6 +73,19 @@ bool set_gemm_fp8_smem() {
     return cudaFuncSetAttribute(grouped_gemm_fp8_kernel<G, BN, BOXN, W8, BS, NS, SC, GA, AS, F4>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 Fp8GemmCfg<G, BN, BOXN, W8, BS, NS, SC, GA, AS, F4>::kSmem) == cudaSuccess;
+}
+
+template <bool G, int BN, int BOXN, int ST, int NS, int SC, bool GA>
+bool set_gemm_mx8_smem() {
+    return cudaFuncSetAttribute(grouped_gemm_mx8_kernel<G, BN, BOXN, ST, NS, SC, GA>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Mx8GemmCfg<G, BN, BOXN, ST, NS, SC, GA>::kSmem) == cudaSuccess;
+}
+template <bool G, int BN, int BOXN, int ST, int NS, int SC, bool GA>
+void launch_gemm_mx8(int grid, cudaStream_t s, const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &s0,
+                     const CUtensorMap &s1, const CUtensorMap &b, const Mx8Params &p) {
+    grouped_gemm_mx8_kernel<G, BN, BOXN, ST, NS, SC, GA>
+        <<<grid, kGemmThreads, Mx8GemmCfg<G, BN, BOXN, ST, NS, SC, GA>::kSmem, s>>>(a0, a1, s0, s1, b, p);
 }
 
 // a1 is ignored by the down projection.
@@ -129,6 +149,8 @@ int init_device(int *dev_out) {
              set_gemm_fp8_smem<G1_NARROW_FP8_ARGS>() && set_gemm_fp8_smem<G2_NARROW_FP8_ARGS>();
         ok = ok && set_gemm_fp8_smem<G1_WIDE_NV4_ARGS>() && set_gemm_fp8_smem<G2_WIDE_NV4_ARGS>() &&
              set_gemm_fp8_smem<G1_NARROW_NV4_ARGS>() && set_gemm_fp8_smem<G2_NARROW_NV4_ARGS>();
+        ok = ok && set_gemm_mx8_smem<G1_WIDE_MX8_ARGS>() && set_gemm_mx8_smem<G2_WIDE_MX8_ARGS>() &&
+             set_gemm_mx8_smem<G1_NARROW_MX8_ARGS>() && set_gemm_mx8_smem<G2_NARROW_MX8_ARGS>();
         ok = ok && cudaFuncSetAttribute(combine_norm_residual_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         kMaxBlockHidden * 4) == cudaSuccess;
         if (!ok) d.status = BEAM_MOE_ERR_CUDA;
@@ -431,6 +453,104 @@ int enqueue_experts(const beam_moe_config *c, int dev, int64_t T, const beam_bf1
     return BEAM_MOE_OK;
 }
 
+// ---- block-scaled FP8 path (MXFP8 weights and activations, tcgen05 kind::mxf8f6f4) ----------------
+bool mx8_shape_ok(const beam_moe_config *c) { return c->hidden % 128 == 0 && c->inter % 128 == 0; }
+
+struct Mx8Layout {
+    size_t ids = 0, w = 0, hist = 0, counts = 0, offsets = 0, row_src = 0, dest_row = 0, xq = 0, xs = 0, xqp = 0,
+           hq = 0, hs = 0, o = 0, total = 0;
+};
+
+Mx8Layout mx8_layout(const beam_moe_config *c, int64_t T) {
+    Mx8Layout L;
+    if (T == 0) return L;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off = align256(off + bytes);
+        return at;
+    };
+    const size_t R = static_cast<size_t>(T) * c->topk;
+    const size_t E = c->n_experts, H = c->hidden, I = c->inter;
+    L.ids = take(R * 4);
+    L.w = take(R * 4);
+    L.hist = take(static_cast<size_t>(n_chunks(T)) * E * 4);
+    L.counts = take(E * 4);
+    L.offsets = take((E + 1) * 8);
+    L.row_src = take(R * 4);
+    L.dest_row = take(R * 4);
+    L.xq = take(static_cast<size_t>(T) * H);
+    L.xs = take(static_cast<size_t>(T) * (H / 32));
+    if (!narrow_tiles(c, T)) L.xqp = take(R * H);  // x codes in dispatch order (wide tiles only)
+    L.hq = take(R * I);
+    L.hs = take(R * (I / 32));
+    L.o = take(R * H * 4);
+    L.total = off;
+    return L;
+}
+
+int enqueue_experts_mx8(const beam_moe_config *c, int dev, int64_t T, const beam_bf16 *x, const int32_t *ids,
+                        const float *w, const beam_moe_fp8_experts *W, beam_bf16 *y, uint8_t *ws, const Mx8Layout &L,
+                        cudaStream_t s, cudaEvent_t const *ev) {
+    int32_t *counts = reinterpret_cast<int32_t *>(ws + L.counts);
+    int64_t *offsets = reinterpret_cast<int64_t *>(ws + L.offsets);
+    int32_t *row_src = reinterpret_cast<int32_t *>(ws + L.row_src);
+    int32_t *dest_row = reinterpret_cast<int32_t *>(ws + L.dest_row);
+    const int k = c->topk, E = c->n_experts, H = c->hidden, I = c->inter;
+    const uint64_t R = static_cast<uint64_t>(T) * k;
+    const bool narrow = narrow_tiles(c, T);
+
+    int rc = enqueue_permute(c, T, ids, counts, offsets, row_src, dest_row, reinterpret_cast<int32_t *>(ws + L.hist), s);
+    if (rc) return rc;
+    if (!record(ev, 2, s)) return BEAM_MOE_ERR_CUDA;
+    // x -> MXFP8 codes and scales (every token once), then the codes into dispatch order (wide tiles)
+    const int64_t n_blocks = T * static_cast<int64_t>(H / 32);
+    quant_mx8_rows_kernel<<<static_cast<unsigned>((n_blocks * 4 + 255) / 256), 256, 0, s>>>(
+        reinterpret_cast<const uint4 *>(x), n_blocks, reinterpret_cast<uint2 *>(ws + L.xq), ws + L.xs);
+    if ((rc = launch_status())) return rc;
+    if (!narrow) {
+        gather_rows_kernel<<<static_cast<unsigned>(T), 128, 0, s>>>(reinterpret_cast<const uint4 *>(ws + L.xq), T, k,
+                                                                    H / 16, dest_row, reinterpret_cast<uint4 *>(ws + L.xqp));
+        if ((rc = launch_status())) return rc;
+    }
+    if (!record(ev, 3, s)) return BEAM_MOE_ERR_CUDA;
+
+    const double mean_rows = static_cast<double>(R) / E;
+    const int bn = narrow ? kNarrowBN : kWideBN;
+    const int box = narrow ? kNarrowBox : kWideBox;
+    const int once = (mean_rows + 4.0 * std::sqrt(mean_rows) <= bn) ? 1 : 0;
+    CUtensorMap m_wg, m_wu, m_wd, m_sg, m_su, m_sd, m_b1, m_b2;
+    if (!encode_fn()) return BEAM_MOE_ERR_CUDA;
+    const bool b1_ok = narrow ? make_map_2d_any(&m_b1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws + L.xq, H,
+                                                static_cast<uint64_t>(T), kMxBK, 1, CU_TENSOR_MAP_SWIZZLE_128B)
+                              : make_map_2d_any(&m_b1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws + L.xqp, H, R, kMxBK, box,
+                                                CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!b1_ok ||
+        !make_map_2d_any(&m_b2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws + L.hq, I, R, kMxBK, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_3d_fp8(&m_wg, W->w_gate, H, I, E) || !make_map_3d_fp8(&m_wu, W->w_up, H, I, E) ||
+        !make_map_3d_fp8(&m_wd, W->w_down, I, H, E) || !make_map_scale(&m_sg, W->w_gate_scale, I, H / 32, E) ||
+        !make_map_scale(&m_su, W->w_up_scale, I, H / 32, E) || !make_map_scale(&m_sd, W->w_down_scale, H, I / 32, E))
+        return BEAM_MOE_ERR_CUDA;
+    const int grid = g_dev[dev].num_sms;
+    Mx8Params p1{counts, offsets, E, H, I, once, kDefaultTimeoutCycles, row_src, k, ws + L.xs, 1, ws + L.hq, ws + L.hs,
+                 nullptr};
+    Mx8Params p2{counts, offsets, E, I, H, once, kDefaultTimeoutCycles, row_src, k, ws + L.hs, 0, nullptr, nullptr,
+                 reinterpret_cast<float *>(ws + L.o)};
+    if (narrow) launch_gemm_mx8<G1_NARROW_MX8_ARGS>(grid, s, m_wg, m_wu, m_sg, m_su, m_b1, p1);
+    else launch_gemm_mx8<G1_WIDE_MX8_ARGS>(grid, s, m_wg, m_wu, m_sg, m_su, m_b1, p1);
+    if ((rc = launch_status())) return rc;
+    if (!record(ev, 4, s)) return BEAM_MOE_ERR_CUDA;
+    if (narrow) launch_gemm_mx8<G2_NARROW_MX8_ARGS>(grid, s, m_wd, m_wd, m_sd, m_sd, m_b2, p2);
+    else launch_gemm_mx8<G2_WIDE_MX8_ARGS>(grid, s, m_wd, m_wd, m_sd, m_sd, m_b2, p2);
+    if ((rc = launch_status())) return rc;
+    if (!record(ev, 5, s)) return BEAM_MOE_ERR_CUDA;
+    combine_kernel<<<static_cast<unsigned>(T), 256, 0, s>>>(reinterpret_cast<const float4 *>(ws + L.o), dest_row, w, T,
+                                                            k, H / 4, c->routed_scale, reinterpret_cast<uint2 *>(y));
+    if ((rc = launch_status())) return rc;
+    if (!record(ev, 6, s)) return BEAM_MOE_ERR_CUDA;
+    return BEAM_MOE_OK;
+}
+
 __global__ void selftest_timeout_kernel(long long cycles) {
     __shared__ uint64_t bar;
     if (threadIdx.x == 0) {
@@ -449,7 +569,8 @@ extern "C" {
 
 size_t beam_moe_workspace_size(const beam_moe_config *cfg, int64_t T, int which) {
     if (validate(cfg) || check_T(cfg, T)) return 0;
-    if (which < BEAM_MOE_WS_ROUTE || which > BEAM_MOE_WS_BLOCK) return 0;
+    if (which < BEAM_MOE_WS_ROUTE || which > BEAM_MOE_WS_MXFP8) return 0;
+    if (which == BEAM_MOE_WS_MXFP8) return mx8_shape_ok(cfg) ? mx8_layout(cfg, T).total : 0;
     return layout(cfg, T, which).total;
 }
 
@@ -621,6 +742,56 @@ int beam_moe_forward_fp8(const beam_moe_config *cfg, int64_t T, const beam_bf16 
     if (!w8 || (events && !events_ok(events))) return BEAM_MOE_ERR_NULL;
     return forward_impl(cfg, T, x, w_router, sel_bias, fp8_weights(w8), y, topk_ids_out, topk_w_out, ws, ws_bytes,
                         stream, reinterpret_cast<cudaEvent_t const *>(events));
+}
+
+namespace {
+int mx8_common_checks(const beam_moe_config *cfg, int64_t T, const beam_moe_fp8_experts *w8, const void *x,
+                      const void *y, void *ws, size_t ws_bytes, void *const *events) {
+    int rc = validate(cfg);
+    if (rc) return rc;
+    if (!mx8_shape_ok(cfg)) return BEAM_MOE_ERR_INVALID_CONFIG;
+    if ((rc = check_T(cfg, T))) return rc;
+    if (!w8 || (events && !events_ok(events))) return BEAM_MOE_ERR_NULL;
+    if (T == 0) return BEAM_MOE_OK;
+    if (!x || !y || !ws) return BEAM_MOE_ERR_NULL;
+    if ((rc = weights_status(fp8_weights(w8)))) return rc;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(ws)) return BEAM_MOE_ERR_MISALIGNED;
+    if (ws_bytes < mx8_layout(cfg, T).total) return BEAM_MOE_ERR_WORKSPACE_TOO_SMALL;
+    return BEAM_MOE_OK;
+}
+}  // namespace
+
+int beam_moe_experts_mxfp8(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const int32_t *topk_ids,
+                           const float *topk_w, const beam_moe_fp8_experts *w8, beam_bf16 *y, void *ws,
+                           size_t ws_bytes, void *stream) {
+    int rc = mx8_common_checks(cfg, T, w8, x, y, ws, ws_bytes, nullptr);
+    if (rc || T == 0) return rc;
+    if (!topk_ids || !topk_w) return BEAM_MOE_ERR_NULL;
+    int dev;
+    if ((rc = init_device(&dev))) return rc;
+    return enqueue_experts_mx8(cfg, dev, T, x, topk_ids, topk_w, w8, y, static_cast<uint8_t *>(ws),
+                               mx8_layout(cfg, T), static_cast<cudaStream_t>(stream), nullptr);
+}
+
+int beam_moe_forward_mxfp8(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const float *w_router,
+                           const float *sel_bias, const beam_moe_fp8_experts *w8, beam_bf16 *y, int32_t *topk_ids_out,
+                           float *topk_w_out, void *ws, size_t ws_bytes, void *stream, void *const *events) {
+    int rc = mx8_common_checks(cfg, T, w8, x, y, ws, ws_bytes, events);
+    if (rc || T == 0) return rc;
+    if (!w_router) return BEAM_MOE_ERR_NULL;
+    if (!aligned16(w_router)) return BEAM_MOE_ERR_MISALIGNED;
+    int dev;
+    if ((rc = init_device(&dev))) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+    const Mx8Layout L = mx8_layout(cfg, T);
+    int32_t *ids = topk_ids_out ? topk_ids_out : reinterpret_cast<int32_t *>(wsb + L.ids);
+    float *w = topk_w_out ? topk_w_out : reinterpret_cast<float *>(wsb + L.w);
+    cudaEvent_t const *ev = reinterpret_cast<cudaEvent_t const *>(events);
+    if (!record(ev, 0, s)) return BEAM_MOE_ERR_CUDA;
+    if ((rc = enqueue_route(cfg, T, x, w_router, sel_bias, ids, w, s))) return rc;
+    if (!record(ev, 1, s)) return BEAM_MOE_ERR_CUDA;
+    return enqueue_experts_mx8(cfg, dev, T, x, ids, w, w8, y, wsb, L, s, ev);
 }
 
 int beam_moe_device_status(void *stream) {

@@ -1,0 +1,512 @@
+// Grouped expert GEMMs on the block-scaled FP8 tensor-core path: tcgen05.mma kind::mxf8f6f4 with
+// E4M3 weights and E4M3 activations, one UE8M0 scale per 32 K elements on each side, FP32
+// accumulation in TMEM.  The weights are an MXFP8 checkpoint ("Checkpoint formats: BF16, FP8, and
+// NVFP4": "Welcome Beam" page, TL;DR); the activations (x for the gate/up projection, h for the
+// down projection) are quantised to MXFP8 per row in blocks of 32 along K, the reading this path
+// takes (the pages give no FP8 recipe).
+//
+//   G1 (gate/up + SwiGLU): h[r, i] = SiLU(x~[r] . W_gate[e, i]) * (x~[r] . W_up[e, i]) in FP32,
+//        then h~ = MXFP8(h) per row: blocks of 32 consecutive i are the 32 lanes of one epilogue
+//        warp, so the block maximum is a warp reduction; codes h_q [R][I], scales h_s [R][I/32].
+//   G2 (down): o[r, j] = h~[r] . W_down[e, j]  (FP32)
+//
+// Same work items, swap-AB orientation (weight rows on the MMA's M side, the expert's tokens on N),
+// accumulator slots and persistent grid as gemm.cuh.  Per stage K = 128 (one 128-byte row of E4M3
+// per operand row, 128-byte swizzle), i.e. four MMAs of K = 32, one per scale block.
+//
+// Scale factors.  The MMA reads them from TMEM: for an operand of up to 128 rows and one stage,
+// a 512-byte atom byte[16 (r % 32) + 4 (r / 32) + kb] (row r, K-block kb of the stage) copied by
+// tcgen05.cp .32x128b.warpx4 into four TMEM columns (row r at lane r % 32 of every lane quarter,
+// column r / 32, byte kb); a B operand of up to 256 rows takes two atoms (eight columns).  The MMA
+// of K-block kb selects byte kb (scale-factor id in the instruction descriptor and in the top two
+// bits of the TMEM address).  Each smem stage has its own TMEM scale columns.
+//
+// Warp roles (256 threads):
+//   warp 0 lane 0  TMA: A tile(s) [128 rows x 128 B], their raw scale tiles [4 K-blocks][128 rows]
+//                  (the checkpoint's K-block-major layout), B rows (tiled boxes of dispatch-ordered
+//                  rows, or gather4 of token rows);
+//   warp 1         TMEM owner; lane 0 issues tcgen05.cp (scales) and tcgen05.mma;
+//   warp 2         scale-factor builder: per stage, B's scales straight from global memory (one
+//                  32-bit word = the stage's 4 K-blocks of one row) and A's from the raw tiles
+//                  (a 4x4 byte transpose per lane), written as atoms; then fence.proxy.async and
+//                  the stage's sf_ready barrier;
+//   warps 4..7     epilogue.
+// Every wait is bounded (status word BEAM_MOE_ERR_DEVICE_TIMEOUT on expiry).
+#pragma once
+
+#include "gemm.cuh"
+
+namespace beam {
+
+constexpr int kMxBK = 128;        // K per stage (bytes of an E4M3 row)
+constexpr int kMxAtom = 512;      // scale atom: 128 rows x 4 K-blocks
+
+template <bool GATE_UP, int BN, int BOXN, int STAGES, int NSLOT, int SLOT_COLS, bool GATHER>
+struct Mx8GemmCfg {
+    static constexpr int kNumA = GATE_UP ? 2 : 1;
+    static constexpr int kA = kBM * kMxBK;                 // 16 KB
+    static constexpr int kB = BN * kMxBK;
+    static constexpr int kBox = BOXN * kMxBK;
+    static constexpr int kSfbAtoms = (BN + 127) / 128;
+    static constexpr int kRawA = 4 * kBM;                  // raw scale tile [4][128]
+    // stage: [A tiles][B][raw SFA x kNumA][SFA atoms x kNumA][SFB atoms]
+    static constexpr int kBOff = kNumA * kA;
+    static constexpr int kRawOff = kBOff + kB;
+    static constexpr int kAtomOff = kRawOff + kNumA * kRawA;
+    static constexpr int kStage = (kAtomOff + (kNumA + kSfbAtoms) * kMxAtom + 1023) / 1024 * 1024;
+    static constexpr int kSfColsPerStage = 4 * (kNumA + kSfbAtoms);
+    static constexpr int kSfCol = NSLOT * SLOT_COLS;       // first TMEM scale column
+    static constexpr int kTmemCols = 512;
+    static constexpr int kBarOff = STAGES * kStage;
+    static constexpr int kTokOff = kBarOff + 512 + 4 * (kPmMaxE + 1);
+    static constexpr int kSmem = 1024 + kTokOff + 4 * BN + 64;
+    static_assert(kA % 1024 == 0 && kB % 1024 == 0 && (GATHER || kBox % 1024 == 0), "swizzled tiles");
+    static_assert(BN % BOXN == 0 && BN % 16 == 0 && BN <= 256, "token tile");
+    static_assert(!GATHER || BOXN == 1, "gathered B rows: one-row boxes, four per instruction");
+    static_assert(kSfCol + STAGES * kSfColsPerStage <= 512, "TMEM has 512 columns");
+    static_assert(GATE_UP ? (BN <= SLOT_COLS && (NSLOT >= 2 || BN <= SLOT_COLS / 2)) : BN <= SLOT_COLS,
+                  "an item must fit in its TMEM slots");
+    static_assert((3 * STAGES + 2 * NSLOT + 1) * 8 + 4 <= 512, "barriers");
+    static_assert(kSmem <= 232448, "shared memory per CTA");
+};
+
+struct Mx8Params {
+    const int32_t *counts;     // [E]
+    const int64_t *offsets;    // [E + 1]
+    int E;
+    int K;                     // reduction length (G1: H, G2: I), multiple of 128
+    int M;                     // weight rows (G1: I, G2: H)
+    int weights_once;
+    long long timeout;
+    const int32_t *row_src;    // dispatch row -> (token, slot) pair q
+    int topk;
+    // activation scales: B row n of an item is dispatch row r = row0 + n; its scale row is
+    // s_rows[sf_token ? row_src[r] / topk : r] with K/32 bytes per row
+    const uint8_t *b_scale;
+    int sf_token;
+    // G1 outputs: h codes [R][M] and scales [R][M/32]; G2 output: o [R][M] fp32
+    uint8_t *h_q;
+    uint8_t *h_s;
+    float *o;
+};
+
+// Instruction descriptor, kind::mxf8f6f4 with block scaling: A and B E4M3 (format 0), K-major,
+// N >> 3 at [17,23), UE8M0 scales (bit 23), M >> 4 at [24,29); scale-factor ids at [4,6) (B) and
+// [29,31) (A) select the K-block's byte.
+__device__ __forceinline__ uint32_t umma_idesc_mx8(int M, int N, uint32_t sf_id) {
+    return (sf_id << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) | (static_cast<uint32_t>(M >> 4) << 24) |
+           (sf_id << 29);
+}
+
+__device__ __forceinline__ void umma_mx8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+        : "memory");
+}
+
+// Shared-memory descriptor of a 512-byte scale atom for tcgen05.cp .32x128b: 32 rows of 16 bytes,
+// no swizzle, 8-row core matrices 128 bytes apart (stride byte offset), version 1.
+__device__ __forceinline__ uint64_t sf_atom_desc(uint32_t smem_addr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>(128u >> 4) << 16;
+    d |= static_cast<uint64_t>(128u >> 4) << 32;
+    d |= static_cast<uint64_t>(1u) << 46;
+    return d;
+}
+
+__device__ __forceinline__ void tmem_cp_sf_atom(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Atom byte offset of (row r, word of the stage's 4 K-blocks) for rows < 256 (two atoms).
+__device__ __forceinline__ int sf_atom_off(int r) { return (r >> 7) * kMxAtom + 16 * (r & 31) + 4 * ((r >> 5) & 3); }
+
+// UE8M0 code of a block whose largest magnitude is amax (finite): 127 + the smallest e with
+// amax <= 448 * 2^e; 0 for amax = 0.  448 = 1.75 * 2^8, so e = E - 8, plus one when the mantissa
+// of amax exceeds 1.75.  Returns the code and the FP32 factor 2^-e that scales the block into E4M3.
+__device__ __forceinline__ uint32_t mx_scale_code(float amax, float &inv) {
+    const uint32_t u = __float_as_uint(amax);
+    if (amax == 0.0f) {
+        inv = 0.0f;
+        return 0u;
+    }
+    const int E = static_cast<int>((u >> 23) & 0xFFu) - 127;
+    const int e = E - 8 + ((u & 0x7FFFFFu) > 0x600000u ? 1 : 0);
+    inv = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+    return static_cast<uint32_t>(e + 127);
+}
+
+// Two FP32 values (already scaled into E4M3 range) -> two E4M3 codes (nearest, ties to even).
+__device__ __forceinline__ uint32_t e4m3x2_from_f32(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// G1 epilogue with MXFP8 h: the 32 lanes of warp q hold weight rows (i) 32q..32q+31 of the tile,
+// one block of 32 along i per token column.
+template <int BN, int NSLOT, int SLOT_COLS>
+__device__ __forceinline__ void mx8_epilogue_g1(int q, const int *tile_start, int total, const Mx8Params &p,
+                                                uint32_t tmem_base, uint64_t *acc_full, uint64_t *acc_empty) {
+    const int lane = threadIdx.x & 31;
+    uint32_t uses = 0;
+    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+        const Item it = decode_item(item, tile_start, p.E, BN, p.counts, p.offsets);
+        const int u = slots_of<true, SLOT_COLS>(it.n_mma);
+        bool ok = true;
+        for (int i = 0; i < u && ok; ++i) {
+            const uint32_t c = uses + i;
+            ok = mbar_wait(&acc_full[c % NSLOT], (c / NSLOT) & 1u, p.timeout);
+        }
+        if (!ok) break;
+        tc_fence_after();
+        const int s0 = uses % NSLOT, s1 = (uses + 1) % NSLOT;
+        const int m = it.mt * kBM + q * 32 + lane;
+        const bool row_ok = m < p.M;
+        const int blk = (it.mt * kBM + q * 32) >> 5;  // this warp's block of 32 along i
+        const bool blk_ok = blk * 32 < p.M;
+        const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+        const uint32_t t0 = tmem_base + lane_off + static_cast<uint32_t>(s0 * SLOT_COLS);
+        const uint32_t t1 = tmem_base + lane_off +
+                            static_cast<uint32_t>(u == 2 ? s1 * SLOT_COLS : s0 * SLOT_COLS + SLOT_COLS / 2);
+        for (int c = 0; c < it.n_valid; c += 16) {
+            uint32_t rg[16], ru[16];
+            tmem_ld16(t0 + c, rg);
+            tmem_ld16(t1 + c, ru);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const float hv = row_ok ? silu_mul(__uint_as_float(rg[j]), __uint_as_float(ru[j])) : 0.0f;
+                float amax = fabsf(hv);
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+                float inv;
+                const uint32_t code = mx_scale_code(amax, inv);
+                if (c + j < it.n_valid && blk_ok) {
+                    const int64_t r = it.row0 + c + j;
+                    if (row_ok) p.h_q[r * p.M + m] = static_cast<uint8_t>(e4m3x2_from_f32(hv * inv, 0.0f) & 0xFFu);
+                    if (lane == 0) p.h_s[r * (p.M >> 5) + blk] = static_cast<uint8_t>(code);
+                }
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0)
+            for (int i = 0; i < u; ++i) mbar_arrive(&acc_empty[(uses + i) % NSLOT]);
+        uses += u;
+    }
+}
+
+// G2 epilogue: FP32 o rows in dispatch order.
+template <int BN, int NSLOT, int SLOT_COLS>
+__device__ __forceinline__ void mx8_epilogue_g2(int q, const int *tile_start, int total, const Mx8Params &p,
+                                                uint32_t tmem_base, uint64_t *acc_full, uint64_t *acc_empty) {
+    const int lane = threadIdx.x & 31;
+    uint32_t uses = 0;
+    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+        const Item it = decode_item(item, tile_start, p.E, BN, p.counts, p.offsets);
+        if (!mbar_wait(&acc_full[uses % NSLOT], (uses / NSLOT) & 1u, p.timeout)) break;
+        tc_fence_after();
+        const int m = it.mt * kBM + q * 32 + lane;
+        const uint32_t t0 =
+            tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>((uses % NSLOT) * SLOT_COLS);
+        for (int c = 0; c < it.n_valid; c += 16) {
+            uint32_t r0[16];
+            tmem_ld16(t0 + c, r0);
+            tmem_ld_wait();
+            if (m < p.M) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    if (c + j < it.n_valid) p.o[(it.row0 + c + j) * p.M + m] = __uint_as_float(r0[j]);
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[uses % NSLOT]);
+        uses += 1;
+    }
+}
+
+template <bool GATE_UP, int BN, int BOXN, int STAGES, int NSLOT, int SLOT_COLS, bool GATHER>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    grouped_gemm_mx8_kernel(const __grid_constant__ CUtensorMap tm_a0,  // W_gate (G1) / W_down (G2): E4M3 [E][M][K]
+                            const __grid_constant__ CUtensorMap tm_a1,  // W_up (G1); unused for G2
+                            const __grid_constant__ CUtensorMap tm_s0,  // scale codes [E][K/32][M] of a0
+                            const __grid_constant__ CUtensorMap tm_s1,  // of a1
+                            const __grid_constant__ CUtensorMap tm_b,   // B rows E4M3 [rows][K]
+                            const Mx8Params p) {
+    using C = Mx8GemmCfg<GATE_UP, BN, BOXN, STAGES, NSLOT, SLOT_COLS, GATHER>;
+    extern __shared__ uint8_t mx8_smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(mx8_smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
+    uint64_t *sf_ready = full + STAGES;
+    uint64_t *empty = sf_ready + STAGES;
+    uint64_t *acc_full = empty + STAGES;
+    uint64_t *acc_empty = acc_full + NSLOT;
+    uint64_t *drain = acc_empty + NSLOT;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    int *tile_start = reinterpret_cast<int *>(smem + C::kBarOff + 512);
+    int *tok = reinterpret_cast<int *>(smem + C::kTokOff);  // GATHER: token of each row of the item
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int E = p.E;
+    const int n_mt = (p.M + kBM - 1) / kBM;
+    const int n_kb = p.K / kMxBK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&sf_ready[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < NSLOT; ++a) {
+            mbar_init(&acc_full[a], 1);
+            mbar_init(&acc_empty[a], 4);
+        }
+        mbar_init(drain, 1);
+        fence_mbar_init();
+        prefetch_tensormap(&tm_a0);
+        prefetch_tensormap(&tm_s0);
+        if (GATE_UP) {
+            prefetch_tensormap(&tm_a1);
+            prefetch_tensormap(&tm_s1);
+        }
+        prefetch_tensormap(&tm_b);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    item_prefix(p.counts, E, n_mt, BN, tile_start);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = tile_start[E];
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        const uint64_t pol_w = p.weights_once ? policy_evict_first() : policy_evict_normal();
+        const uint64_t pol_x = policy_evict_last();
+        int stage = 0;
+        uint32_t phase = 0;
+        uint32_t issued = 0, issued_phase = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+            const Item it = decode_item(item, tile_start, E, BN, p.counts, p.offsets);
+            if (GATHER) {
+                for (int r = lane; r < it.n_mma; r += 32) {
+                    const int rr = r < it.n_valid ? r : 0;
+                    tok[r] = p.row_src[it.row0 + rr] / p.topk;
+                }
+                __syncwarp();
+            }
+            if (lane == 0) {
+                const int nbox = GATHER ? (it.n_mma + 3) / 4 : (it.n_mma + BOXN - 1) / BOXN;
+                const uint32_t bytes = C::kNumA * (C::kA + C::kRawA) + nbox * (GATHER ? 4 * kMxBK : C::kBox);
+                for (int kb = 0; kb < n_kb; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, p.timeout)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *st = smem + stage * C::kStage;
+                    mbar_arrive_expect_tx(&full[stage], bytes);
+                    tma_load_3d(st, &tm_a0, &full[stage], kb * kMxBK, it.mt * kBM, it.e, pol_w);
+                    tma_load_3d(st + C::kRawOff, &tm_s0, &full[stage], it.mt * kBM, 4 * kb, it.e, pol_w);
+                    if (GATE_UP) {
+                        tma_load_3d(st + C::kA, &tm_a1, &full[stage], kb * kMxBK, it.mt * kBM, it.e, pol_w);
+                        tma_load_3d(st + C::kRawOff + C::kRawA, &tm_s1, &full[stage], it.mt * kBM, 4 * kb, it.e,
+                                    pol_w);
+                    }
+                    uint8_t *sb = st + C::kBOff;
+                    if (GATHER) {
+                        for (int g = 0; g < nbox; ++g)
+                            tma_gather4(sb + g * 4 * kMxBK, &tm_b, &full[stage], kb * kMxBK, tok[4 * g], tok[4 * g + 1],
+                                        tok[4 * g + 2], tok[4 * g + 3], pol_x);
+                    } else {
+                        for (int bx = 0; bx < nbox; ++bx)
+                            tma_load_2d(sb + bx * C::kBox, &tm_b, &full[stage], kb * kMxBK,
+                                        static_cast<int>(it.row0) + bx * BOXN, pol_x);
+                    }
+                    issued |= 1u << stage;
+                    issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            stage = __shfl_sync(0xffffffffu, stage, 0);
+            phase = __shfl_sync(0xffffffffu, phase, 0);
+        }
+        if (lane == 0)
+            for (int s = 0; s < STAGES; ++s)
+                if ((issued >> s) & 1u) mbar_wait(&full[s], (issued_phase >> s) & 1u, p.timeout);
+    } else if (warp == 2) {
+        // ---------------- scale-factor builder ----------------
+        const int kbs = p.K >> 5;  // scale bytes per activation row
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+            const Item it = decode_item(item, tile_start, E, BN, p.counts, p.offsets);
+            for (int kb = 0; kb < n_kb && ok; ++kb) {
+                // B: one word (the stage's 4 K-blocks) per row, loaded before the stage's data lands
+                uint32_t wb[(BN + 31) / 32];
+#pragma unroll
+                for (int i = 0; i < (BN + 31) / 32; ++i) {
+                    const int n = lane + 32 * i;
+                    wb[i] = 0u;
+                    if (n < it.n_valid) {
+                        const int64_t r = it.row0 + n;
+                        const int64_t srow = p.sf_token ? static_cast<int64_t>(p.row_src[r] / p.topk) : r;
+                        wb[i] = __ldg(reinterpret_cast<const uint32_t *>(p.b_scale + srow * kbs + 4 * kb));
+                    }
+                }
+                ok = __all_sync(0xffffffffu, mbar_wait(&full[stage], phase, p.timeout));
+                if (!ok) break;
+                uint8_t *st = smem + stage * C::kStage;
+                uint8_t *atoms = st + C::kAtomOff;
+#pragma unroll
+                for (int i = 0; i < (BN + 31) / 32; ++i) {
+                    const int n = lane + 32 * i;
+                    if (n < BN) *reinterpret_cast<uint32_t *>(atoms + C::kNumA * kMxAtom + sf_atom_off(n)) = wb[i];
+                }
+                // A: raw [4 K-blocks][128 rows] -> atom; lane l takes rows 4l..4l+3
+#pragma unroll
+                for (int a = 0; a < C::kNumA; ++a) {
+                    const uint8_t *raw = st + C::kRawOff + a * C::kRawA;
+                    uint32_t w[4];
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) w[k4] = *reinterpret_cast<const uint32_t *>(raw + k4 * kBM + 4 * lane);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t sel = static_cast<uint32_t>(i | ((4 + i) << 4));
+                        const uint32_t lo = __byte_perm(w[0], w[1], sel);
+                        const uint32_t hi = __byte_perm(w[2], w[3], sel);
+                        *reinterpret_cast<uint32_t *>(atoms + a * kMxAtom + sf_atom_off(4 * lane + i)) =
+                            __byte_perm(lo, hi, 0x5410);
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sf_ready[stage]);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer ----------------
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t uses = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+                const Item it = decode_item(item, tile_start, E, BN, p.counts, p.offsets);
+                const int u = slots_of<GATE_UP, SLOT_COLS>(it.n_mma);
+                const int s0 = uses % NSLOT, s1 = (uses + 1) % NSLOT;
+                for (int i = 0; i < u && ok; ++i) {
+                    const uint32_t c = uses + i;
+                    ok = mbar_wait(&acc_empty[c % NSLOT], ((c / NSLOT) & 1u) ^ 1u, p.timeout);
+                }
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t d0 = tmem_base + static_cast<uint32_t>(s0 * SLOT_COLS);
+                const uint32_t d1 =
+                    tmem_base + static_cast<uint32_t>(u == 2 ? s1 * SLOT_COLS : s0 * SLOT_COLS + SLOT_COLS / 2);
+                for (int kb = 0; kb < n_kb; ++kb) {
+                    if (!mbar_wait(&sf_ready[stage], phase, p.timeout)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + stage * C::kStage);
+                    const uint32_t atoms = sa + C::kAtomOff;
+                    const uint32_t sf_col = tmem_base + static_cast<uint32_t>(C::kSfCol + stage * C::kSfColsPerStage);
+#pragma unroll
+                    for (int a = 0; a < C::kNumA + C::kSfbAtoms; ++a)
+                        tmem_cp_sf_atom(sf_col + 4 * a, sf_atom_desc(atoms + a * kMxAtom));
+                    const uint32_t sfb = sf_col + 4 * C::kNumA;
+                    const uint64_t da0 = umma_desc_sw128(sa);
+                    const uint64_t da1 = umma_desc_sw128(sa + C::kA);
+                    const uint64_t db = umma_desc_sw128(sa + C::kBOff);
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const uint32_t accum = (kb > 0 || k4 > 0) ? 1u : 0u;
+                        const uint32_t idesc = umma_idesc_mx8(kBM, it.n_mma, static_cast<uint32_t>(k4));
+                        const uint32_t byte = static_cast<uint32_t>(k4) << 30;
+                        // +32 bytes along K inside the swizzle row = +2 in the 16-byte address field
+                        umma_mx8(d0, da0 + 2 * k4, db + 2 * k4, idesc, sf_col | byte, sfb | byte, accum);
+                        if (GATE_UP) umma_mx8(d1, da1 + 2 * k4, db + 2 * k4, idesc, (sf_col + 4) | byte, sfb | byte, accum);
+                    }
+                    umma_commit(&empty[stage]);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                for (int i = 0; i < u; ++i) umma_commit(&acc_full[(uses + i) % NSLOT]);
+                uses += u;
+            }
+            umma_commit(drain);
+            mbar_wait(drain, 0, p.timeout);
+        }
+    } else if (warp >= 4) {
+        if (GATE_UP) mx8_epilogue_g1<BN, NSLOT, SLOT_COLS>(warp - 4, tile_start, total, p, tmem_base, acc_full, acc_empty);
+        else mx8_epilogue_g2<BN, NSLOT, SLOT_COLS>(warp - 4, tile_start, total, p, tmem_base, acc_full, acc_empty);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+}
+
+// x [T][H] bf16 -> MXFP8 codes x_q [T][H] and scale codes x_s [T][H/32]: 4 threads per block of 32,
+// 8 elements each (one 16-byte load, one 8-byte store).
+__global__ void __launch_bounds__(256) quant_mx8_rows_kernel(const uint4 *__restrict__ x, int64_t n_blocks,
+                                                             uint2 *__restrict__ q, uint8_t *__restrict__ s) {
+    const int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;  // 8-element group
+    const int64_t blk = t >> 2;
+    const bool live = blk < n_blocks;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (live) v = __ldg(x + t);
+    float f[8];
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    float inv;
+    const uint32_t code = mx_scale_code(amax, inv);
+    uint2 out;
+    out.x = e4m3x2_from_f32(f[0] * inv, f[1] * inv) | (e4m3x2_from_f32(f[2] * inv, f[3] * inv) << 16);
+    out.y = e4m3x2_from_f32(f[4] * inv, f[5] * inv) | (e4m3x2_from_f32(f[6] * inv, f[7] * inv) << 16);
+    if (live) {
+        q[t] = out;
+        if ((t & 3) == 0) s[blk] = static_cast<uint8_t>(code);
+    }
+}
+
+}  // namespace beam

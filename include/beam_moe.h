@@ -80,7 +80,8 @@ enum {
     BEAM_MOE_WS_PERMUTE = 1,
     BEAM_MOE_WS_EXPERTS = 2,
     BEAM_MOE_WS_FORWARD = 3,
-    BEAM_MOE_WS_BLOCK = 4
+    BEAM_MOE_WS_BLOCK = 4,
+    BEAM_MOE_WS_MXFP8 = 5  /* beam_moe_experts_mxfp8 and beam_moe_forward_mxfp8 */
 };
 
 /*
@@ -285,6 +286,26 @@ BEAM_MOE_API int beam_moe_forward_nvfp4(const beam_moe_config *cfg, int64_t T, c
                                         const beam_moe_nvfp4_experts *w4, beam_bf16 *y, int32_t *topk_ids_out,
                                         float *topk_w_out, void *ws, size_t ws_bytes, void *stream,
                                         void *const *events);
+
+/*
+ * Native FP8 path: the same MXFP8 expert weights (beam_moe_fp8_experts) multiplied on the tensor
+ * cores with block scaling (tcgen05.mma kind::mxf8f6f4: E4M3 x E4M3, one UE8M0 scale per 32 K
+ * elements on each side, FP32 accumulation).  The activations are quantised to MXFP8 as well: x per
+ * token and h per dispatch row, in blocks of 32 along the reduction axis, each block scaled by the
+ * smallest power of two that brings its largest magnitude to <= 448, elements rounded to the
+ * nearest E4M3 value (ties to even).  This is a reading (the pages give no FP8 recipe): results
+ * differ from beam_moe_forward_fp8 (bf16 activations) by the activation rounding.  Requires hidden
+ * and inter to be multiples of 128.  Workspace: beam_moe_workspace_size(cfg, T, BEAM_MOE_WS_MXFP8).
+ * Other arguments, outputs and error codes as beam_moe_experts_fp8 / beam_moe_forward_fp8
+ * (`events`: NULL or 7 events recorded between the stages).
+ */
+BEAM_MOE_API int beam_moe_experts_mxfp8(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x,
+                                        const int32_t *topk_ids, const float *topk_w, const beam_moe_fp8_experts *w8,
+                                        beam_bf16 *y, void *ws, size_t ws_bytes, void *stream);
+BEAM_MOE_API int beam_moe_forward_mxfp8(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x,
+                                        const float *w_router, const float *sel_bias, const beam_moe_fp8_experts *w8,
+                                        beam_bf16 *y, int32_t *topk_ids_out, float *topk_w_out, void *ws,
+                                        size_t ws_bytes, void *stream, void *const *events);
 
 /*
  * Expert parallelism ("Welcome Beam" page, section "Multi-GPU and multi-node": each expert lives on

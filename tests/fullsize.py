@@ -11,7 +11,8 @@ Token samples (oracle outputs are compared on these; routing and dispatch on eve
   prefill  512 seeded tokens
   skew     4096 seeded tokens
   long     4096 seeded tokens plus every outlier row (655)
-The FP8 and NVFP4 checkpoints are compared on decode (all tokens) and prefill (256 seeded tokens).
+The FP8 and NVFP4 checkpoints are compared on decode (all tokens) and prefill (256 seeded tokens), on
+the converter paths and on the native FP8 path ("mxfp8": MXFP8 activations too).
 """
 from __future__ import annotations
 
@@ -70,7 +71,10 @@ class Bank:
         return self._nv4
 
     def fetch(self, fmt: str):
-        """fetch(e) of the oracle: one expert's weights (bf16 bits, or FP64 for NVFP4) on the host."""
+        """fetch(e) of the oracle: one expert's weights (bf16 bits, or FP64 for NVFP4) on the host.
+        "mxfp8" (the native FP8 path) reads the FP8 checkpoint like "fp8"."""
+        if fmt == "mxfp8":
+            fmt = "fp8"
         if fmt == "bf16":
             h = self.host()
             return lambda e: (h[0][e], h[1][e], h[2][e])
@@ -96,8 +100,7 @@ class Bank:
     def y_of(self, fmt: str, name: str):
         """y_of(ids, w, tokens): the oracle's expert half on `tokens` of workload `name`."""
         c = self.case(name)
-        f64 = fmt == "nvfp4"
-        run = oracle.experts_tokens_f64 if f64 else oracle.experts_tokens
+        run = _RUN[fmt]
         fetch = self.fetch(fmt)
 
         def y_of(ids, w, tokens):
@@ -123,13 +126,17 @@ class Bank:
                 spans.append((n, at, at + len(tok)))
                 at += len(tok)
             x = np.ascontiguousarray(np.concatenate(xs))
-            run = oracle.experts_tokens_f64 if fmt == "nvfp4" else oracle.experts_tokens
+            run = _RUN[fmt]
             L = self.wl.layer
             y = run(x, np.concatenate(ids), np.concatenate(ws), self.fetch(fmt), L["n_experts"], L["routed_scale"])
             for n, a, b in spans:
                 self._y[(fmt, n)] = y[a:b]
         return self._y[key]
 
+
+# the oracle's expert half per weight format
+_RUN = {"bf16": oracle.experts_tokens, "fp8": oracle.experts_tokens, "nvfp4": oracle.experts_tokens_f64,
+        "mxfp8": oracle.experts_tokens_mx8}
 
 _BANK: Optional[Bank] = None
 

@@ -13,20 +13,27 @@ Routing protocol (the pages fix no tie rule; the oracle's reading is lower index
     output of every excluded token whose set differs is still checked: the oracle recomputes it from
     the GPU's expert ids (oracle_y_checked).
 
-Output protocol (compare_y), for y_gpu (BF16) against the oracle's FP64 y, RMS = RMS(y_oracle):
+Output protocol (compare_y), for y_gpu (BF16) against the oracle's FP64 y, per token t (one output
+row) with tol_t = 2e-2 * RMS(y_oracle[t]):
   * literal bound where BF16 can meet it: on every element whose BF16 spacing is fine enough that
-    rounding alone uses at most a quarter of the budget (half a BF16 ulp of y_oracle <= 5e-3 RMS,
-    which holds for |y_oracle| below 1.28 to 2.56 RMS, by where the binades fall), the literal
-    max |y_gpu - y_oracle| <= 2e-2 RMS;
+    rounding alone uses at most a quarter of the budget (half a BF16 ulp of y_oracle <= tol_t / 4,
+    which holds for |y_oracle| below 1.28 to 2.56 row RMS, by where the binades fall), the literal
+    |y_gpu - y_oracle| <= tol_t;
   * every element: y_gpu must be the round-to-nearest BF16 value of some v with
-    |v - y_oracle| <= 2e-2 RMS, i.e. the distance from y_oracle to y_gpu's BF16 rounding interval is
-    at most 2e-2 RMS.  Where |y_oracle| is above ~5 RMS, half a BF16 ulp is itself more than 1e-2 RMS
-    (and above 8 RMS more than 2e-2 RMS), so the raw difference of a correctly rounded output can
-    exceed 2e-2 RMS with no error in the computation at all;
-  * reported, not enforced: the raw max |y_gpu - y_oracle| / RMS (the literal quantity), the same
-    against bf16(y_oracle), and how many elements differ from bf16(y_oracle) by more than 2e-2 RMS and
-    by exactly one BF16 step (an FP32 result and the exact one on opposite sides of a rounding
-    midpoint: one step is 0.031 RMS at |y| in [4, 8) RMS).
+    |v - y_oracle| <= tol_t, i.e. the distance from y_oracle to y_gpu's BF16 rounding interval is at
+    most tol_t.  Where |y_oracle| is above ~5 row RMS, half a BF16 ulp is itself more than 1e-2 RMS
+    (above 8 RMS more than 2e-2 RMS), so the raw difference of a correctly rounded output can exceed
+    the bound with no error in the computation at all;
+  * "the output RMS" is read per token: each token's output row is checked at its own scale.  On
+    batches whose rows share one scale this is the whole-output rule; on the long batch, whose 1%
+    of x30 outlier rows carry ~900x larger outputs, the whole-output RMS (~90x a normal row's)
+    would leave the normal rows essentially unchecked, while the per-token rule checks every row
+    at its own scale;
+  * reported, not enforced: the raw max |y_gpu - y_oracle| / RMS of the whole output (the literal
+    quantity), the distance rule against the whole-output RMS, the difference from bf16(y_oracle),
+    and how many elements differ from bf16(y_oracle) by more than 2e-2 RMS and by exactly one BF16
+    step (an FP32 result and the exact one on opposite sides of a rounding midpoint: one step is
+    0.031 RMS at |y| in [4, 8) RMS).
 """
 from __future__ import annotations
 
@@ -184,33 +191,34 @@ def half_ulp_bf16(y: np.ndarray) -> np.ndarray:
 def compare_y(y_gpu: np.ndarray, y_or: np.ndarray, what: str = "y") -> dict:
     y_gpu = y_gpu.astype(np.float64)
     if y_or.size == 0:
-        return dict(max_err=0.0, rms=0.0, rel=0.0, rel_dist=0.0, rel_vs_bf16=0.0, n_over_vs_bf16=0,
-                    n_one_step=0, rows_within_own_rms=1.0)
+        return dict(max_err=0.0, rms=0.0, rel=0.0, rel_row=0.0, rel_dist_row=0.0, rel_dist=0.0, rel_vs_bf16=0.0,
+                    n_over_vs_bf16=0, n_one_step=0, n_elements=0)
     err = np.abs(y_gpu - y_or)
     rms = float(np.sqrt(np.mean(y_or ** 2)))
-    tol = Y_TOL * rms
-    max_err = float(err.max())
-    # literal bound wherever BF16 rounding alone takes at most a quarter of it
+    row_rms = np.sqrt(np.mean(y_or ** 2, axis=1, keepdims=True))
+    tol = Y_TOL * row_rms
+    assert np.all(row_rms > 0), f"{what}: a token's output is exactly zero"
+    # literal bound per token, wherever BF16 rounding alone takes at most a quarter of it
     fine = half_ulp_bf16(y_or) <= 0.25 * tol
-    lit = float(err[fine].max()) if fine.any() else 0.0
-    assert lit <= tol, f"{what}: max |err| {lit:.4g} > {Y_TOL} * RMS {rms:.4g} on the elements with fine BF16 spacing"
-    # everywhere: distance from y_oracle to the BF16 rounding interval of y_gpu
+    ratio_fine = np.where(fine, err / tol, 0.0)
+    worst = float(ratio_fine.max())
+    t_w = int(np.unravel_index(np.argmax(ratio_fine), err.shape)[0])
+    assert worst <= 1.0, (f"{what}: token {t_w}: max |err| {worst * Y_TOL:.4g} x its RMS > {Y_TOL} on the elements "
+                          f"with fine BF16 spacing")
+    # everywhere: distance from y_oracle to the BF16 rounding interval of y_gpu, per token
     lo, hi = bf16_interval(y_gpu)
     dist = np.maximum(0.0, np.maximum(lo - y_or, y_or - hi))
-    max_dist = float(dist.max())
-    assert max_dist <= tol, \
-        f"{what}: y_oracle lies {max_dist:.4g} from the BF16 rounding interval of y_gpu > {Y_TOL} * RMS {rms:.4g}"
-    # reported: against the oracle rounded to BF16
+    dist_ratio = float((dist / tol).max())
+    assert dist_ratio <= 1.0, (f"{what}: y_oracle lies {dist_ratio * Y_TOL:.4g} x the token's RMS from the BF16 "
+                               f"rounding interval of y_gpu (> {Y_TOL})")
+    # reported: the whole-output quantities and the comparison against the oracle rounded to BF16
     yb = oracle.bf16_bits_to_f64(oracle.f64_to_bf16_bits(y_or))
     eb = np.abs(y_gpu - yb)
-    over = eb > tol
+    over = eb > Y_TOL * rms
     bg = oracle.f64_to_bf16_bits(y_gpu).astype(np.int32)
     bo = oracle.f64_to_bf16_bits(y_or).astype(np.int32)
     one_step = over & (np.abs(bg - bo) == 1)
-    row_rms = np.sqrt(np.mean(y_or ** 2, axis=1))
-    row_ok = np.all(dist <= Y_TOL * row_rms[:, None] + 1e-30, axis=1)
-    return dict(max_err=max_err, rms=rms, rel=max_err / rms if rms else 0.0,
-                rel_fine=lit / rms if rms else 0.0, rel_dist=max_dist / rms if rms else 0.0,
-                rel_vs_bf16=float(eb.max()) / rms if rms else 0.0, n_over_vs_bf16=int(over.sum()),
-                n_one_step=int(one_step.sum()), n_elements=int(y_or.size),
-                rows_within_own_rms=float(row_ok.mean()))
+    return dict(max_err=float(err.max()), rms=rms, rel=float(err.max()) / rms, rel_row=float((err / tol).max()) * Y_TOL,
+                rel_fine_row=worst * Y_TOL, rel_dist_row=dist_ratio * Y_TOL, rel_dist=float(dist.max()) / rms,
+                rel_vs_bf16=float(eb.max()) / rms, n_over_vs_bf16=int(over.sum()), n_one_step=int(one_step.sum()),
+                n_elements=int(y_or.size))

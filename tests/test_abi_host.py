@@ -183,3 +183,24 @@ def test_nvfp4_entry_points_check_arguments_on_host(L):
                                     None, None) == bm.OK
     with pytest.raises(KeyError):
         bm._nvfp4_experts(bm.BEAM_LAYER.c(), {"q_gate": None})
+
+
+def test_mxfp8_entry_points_check_arguments_on_host(L):
+    """The native FP8 path needs hidden and inter in multiples of 128 and checks its own workspace size."""
+    p = ctypes.c_void_p(4096)
+    good = bm.BeamMoeFp8Experts(4096, 4096, 4096, 4096, 4096, 4096)
+    for bad in (dict(hidden=320), dict(inter=192)):
+        c = _cfg(**bad)
+        assert bm.workspace_size(c, 64, bm.WS_MXFP8) == 0
+        assert L.beam_moe_forward_mxfp8(ctypes.byref(c), 64, p, p, None, ctypes.byref(good), p, None, None, p,
+                                        1 << 40, None, None) == bm.ERR_INVALID_CONFIG
+        assert L.beam_moe_experts_mxfp8(ctypes.byref(c), 64, p, p, p, ctypes.byref(good), p, p, 1 << 40, None) == \
+            bm.ERR_INVALID_CONFIG
+    c = _cfg()
+    need = bm.workspace_size(c, 64, bm.WS_MXFP8)
+    assert need > 0 and bm.workspace_size(c, 4096, bm.WS_MXFP8) < bm.workspace_size(c, 4096, bm.WS_FORWARD)
+    assert L.beam_moe_forward_mxfp8(ctypes.byref(c), 64, p, p, None, ctypes.byref(good), p, None, None, p, need - 1,
+                                    None, None) == bm.ERR_WORKSPACE_TOO_SMALL
+    assert L.beam_moe_forward_mxfp8(ctypes.byref(c), 64, p, p, None, None, p, None, None, p, need, None, None) == \
+        bm.ERR_NULL
+    assert L.beam_moe_experts_mxfp8(ctypes.byref(c), 0, p, p, p, ctypes.byref(good), p, p, 0, None) == bm.OK
