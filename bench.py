@@ -76,6 +76,9 @@ def parse():
                          "(default: decode,skew,long for bf16, decode for --fp8/--mxfp8/--nvfp4, none for --block)")
     ap.add_argument("--cpu-sample", type=int, default=1024, help="tokens in the CPU-oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="profiling only: a reduced Beam-shaped layer with this many experts (8 groups, keep 4, top 8)")
+    ap.add_argument("--tokens", type=int, default=None, help="profiling only: override the workload's T")
     ap.add_argument("--ep", action="store_true",
                     help="expert parallelism over the N ranks (E/N experts each, all-to-all dispatch and combine); "
                          "each rank brings its own batch of the workload (weak scaling)")
@@ -370,6 +373,23 @@ class Ranks:
             self.dist = None
 
 
+def reduced(wl, args):
+    """The workload with --experts / --tokens applied (profiling cases: a few GB instead of 20)."""
+    import dataclasses
+    kw = {}
+    if args.experts:
+        kw["n_experts"] = args.experts
+    if args.tokens:
+        kw["T"] = args.tokens
+    if kw:
+        kw["name"] = f"{wl.name}_E{args.experts or wl.n_experts}_T{args.tokens or wl.T}"
+        kw["description"] = (f"profiling case: Beam shapes with {args.experts or wl.n_experts} experts, "
+                             f"T={args.tokens or wl.T}")
+        kw["bias"] = "zero"
+        return dataclasses.replace(wl, **kw)
+    return wl
+
+
 def layer_inputs(wl):
     """x, W_r and bias of a workload: host copies and device tensors."""
     x_cpu = bs.make_x(wl)
@@ -416,7 +436,7 @@ def run_ours(args):
     torch.cuda.set_device(local)
     barrier = ranks.barrier
 
-    wl = bs.get(args.workload)
+    wl = reduced(bs.get(args.workload), args)
     layer = wl.layer
     T, H = wl.T, wl.hidden
     fmt = "nvfp4" if args.nvfp4 else "fp8" if args.fp8 else "mxfp8" if args.mxfp8 else "bf16"
@@ -424,6 +444,8 @@ def run_ours(args):
         also = [] if args.block else (["decode", "skew", "long"] if fmt == "bf16" else ["decode"])
     else:
         also = [n for n in args.also.split(",") if n]
+    if (args.experts or args.tokens) and args.also is None:
+        also = []
     also = [n for n in also if n != wl.name]
     wg, wu, wd = bs.make_experts(wl, device="cuda")
     w8 = None

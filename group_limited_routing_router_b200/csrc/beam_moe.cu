@@ -85,7 +85,7 @@ template <bool G, int BN, int BOXN, int ST, int NS, int SC, bool GA>
 void launch_gemm_mx8(int grid, cudaStream_t s, const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &s0,
                      const CUtensorMap &s1, const CUtensorMap &b, const Mx8Params &p) {
     grouped_gemm_mx8_kernel<G, BN, BOXN, ST, NS, SC, GA>
-        <<<grid, kGemmThreads, Mx8GemmCfg<G, BN, BOXN, ST, NS, SC, GA>::kSmem, s>>>(a0, a1, s0, s1, b, p);
+        <<<grid, kMxThreads, Mx8GemmCfg<G, BN, BOXN, ST, NS, SC, GA>::kSmem, s>>>(a0, a1, s0, s1, b, p);
 }
 
 // a1 is ignored by the down projection.

@@ -21,7 +21,7 @@
 // of K-block kb selects byte kb (scale-factor id in the instruction descriptor and in the top two
 // bits of the TMEM address).  Each smem stage has its own TMEM scale columns.
 //
-// Warp roles (256 threads):
+// Warp roles (384 threads):
 //   warp 0 lane 0  TMA: A tile(s) [128 rows x 128 B], their raw scale tiles [4 K-blocks][128 rows]
 //                  (the checkpoint's K-block-major layout), B rows (tiled boxes of dispatch-ordered
 //                  rows, or gather4 of token rows);
@@ -30,7 +30,8 @@
 //                  32-bit word = the stage's 4 K-blocks of one row) and A's from the raw tiles
 //                  (a 4x4 byte transpose per lane), written as atoms; then fence.proxy.async and
 //                  the stage's sf_ready barrier;
-//   warps 4..7     epilogue.
+//   warps 4..11    epilogue: two warps per TMEM lane quarter (warp w reads lanes 32 (w % 4)..+31),
+//                  taking alternate 16-column chunks of the item's tokens.
 // Every wait is bounded (status word BEAM_MOE_ERR_DEVICE_TIMEOUT on expiry).
 #pragma once
 
@@ -39,6 +40,8 @@
 namespace beam {
 
 constexpr int kMxBK = 128;        // K per stage (bytes of an E4M3 row)
+constexpr int kMxThreads = 384;   // warps 0..3 producer / MMA / scale factors / idle, 4..11 epilogue
+constexpr int kMxEpiWarps = 8;
 constexpr int kMxAtom = 512;      // scale atom: 128 rows x 4 K-blocks
 
 template <bool GATE_UP, int BN, int BOXN, int STAGES, int NSLOT, int SLOT_COLS, bool GATHER>
@@ -155,7 +158,7 @@ __device__ __forceinline__ uint32_t e4m3x2_from_f32(float lo, float hi) {
 // G1 epilogue with MXFP8 h: the 32 lanes of warp q hold weight rows (i) 32q..32q+31 of the tile,
 // one block of 32 along i per token column.
 template <int BN, int NSLOT, int SLOT_COLS>
-__device__ __forceinline__ void mx8_epilogue_g1(int q, const int *tile_start, int total, const Mx8Params &p,
+__device__ __forceinline__ void mx8_epilogue_g1(int q, int half, const int *tile_start, int total, const Mx8Params &p,
                                                 uint32_t tmem_base, uint64_t *acc_full, uint64_t *acc_empty) {
     const int lane = threadIdx.x & 31;
     uint32_t uses = 0;
@@ -178,7 +181,7 @@ __device__ __forceinline__ void mx8_epilogue_g1(int q, const int *tile_start, in
         const uint32_t t0 = tmem_base + lane_off + static_cast<uint32_t>(s0 * SLOT_COLS);
         const uint32_t t1 = tmem_base + lane_off +
                             static_cast<uint32_t>(u == 2 ? s1 * SLOT_COLS : s0 * SLOT_COLS + SLOT_COLS / 2);
-        for (int c = 0; c < it.n_valid; c += 16) {
+        for (int c = 16 * half; c < it.n_valid; c += 32) {
             uint32_t rg[16], ru[16];
             tmem_ld16(t0 + c, rg);
             tmem_ld16(t1 + c, ru);
@@ -186,9 +189,8 @@ __device__ __forceinline__ void mx8_epilogue_g1(int q, const int *tile_start, in
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
                 const float hv = row_ok ? silu_mul(__uint_as_float(rg[j]), __uint_as_float(ru[j])) : 0.0f;
-                float amax = fabsf(hv);
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+                // the block maximum: |h| >= 0, so its bit pattern orders like the value
+                const float amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(hv))));
                 float inv;
                 const uint32_t code = mx_scale_code(amax, inv);
                 if (c + j < it.n_valid && blk_ok) {
@@ -208,7 +210,7 @@ __device__ __forceinline__ void mx8_epilogue_g1(int q, const int *tile_start, in
 
 // G2 epilogue: FP32 o rows in dispatch order.
 template <int BN, int NSLOT, int SLOT_COLS>
-__device__ __forceinline__ void mx8_epilogue_g2(int q, const int *tile_start, int total, const Mx8Params &p,
+__device__ __forceinline__ void mx8_epilogue_g2(int q, int half, const int *tile_start, int total, const Mx8Params &p,
                                                 uint32_t tmem_base, uint64_t *acc_full, uint64_t *acc_empty) {
     const int lane = threadIdx.x & 31;
     uint32_t uses = 0;
@@ -219,7 +221,7 @@ __device__ __forceinline__ void mx8_epilogue_g2(int q, const int *tile_start, in
         const int m = it.mt * kBM + q * 32 + lane;
         const uint32_t t0 =
             tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>((uses % NSLOT) * SLOT_COLS);
-        for (int c = 0; c < it.n_valid; c += 16) {
+        for (int c = 16 * half; c < it.n_valid; c += 32) {
             uint32_t r0[16];
             tmem_ld16(t0 + c, r0);
             tmem_ld_wait();
@@ -237,7 +239,7 @@ __device__ __forceinline__ void mx8_epilogue_g2(int q, const int *tile_start, in
 }
 
 template <bool GATE_UP, int BN, int BOXN, int STAGES, int NSLOT, int SLOT_COLS, bool GATHER>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kMxThreads, 1)
     grouped_gemm_mx8_kernel(const __grid_constant__ CUtensorMap tm_a0,  // W_gate (G1) / W_down (G2): E4M3 [E][M][K]
                             const __grid_constant__ CUtensorMap tm_a1,  // W_up (G1); unused for G2
                             const __grid_constant__ CUtensorMap tm_s0,  // scale codes [E][K/32][M] of a0
@@ -270,7 +272,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         for (int a = 0; a < NSLOT; ++a) {
             mbar_init(&acc_full[a], 1);
-            mbar_init(&acc_empty[a], 4);
+            mbar_init(&acc_empty[a], kMxEpiWarps);
         }
         mbar_init(drain, 1);
         fence_mbar_init();
@@ -466,8 +468,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             mbar_wait(drain, 0, p.timeout);
         }
     } else if (warp >= 4) {
-        if (GATE_UP) mx8_epilogue_g1<BN, NSLOT, SLOT_COLS>(warp - 4, tile_start, total, p, tmem_base, acc_full, acc_empty);
-        else mx8_epilogue_g2<BN, NSLOT, SLOT_COLS>(warp - 4, tile_start, total, p, tmem_base, acc_full, acc_empty);
+        const int q = warp & 3, half = (warp - 4) >> 2;
+        if (GATE_UP) mx8_epilogue_g1<BN, NSLOT, SLOT_COLS>(q, half, tile_start, total, p, tmem_base, acc_full, acc_empty);
+        else mx8_epilogue_g2<BN, NSLOT, SLOT_COLS>(q, half, tile_start, total, p, tmem_base, acc_full, acc_empty);
     }
     tc_fence_before();
     __syncthreads();
