@@ -19,6 +19,8 @@ section "Mixture of Experts"):
   block_forward  - pre-norm -> block -> post-norm -> scaled residual
   quant_mxfp8_rows, expert_mlp_mx8, experts_tokens_mx8
                  - the block-scaled FP8 path: MXFP8 activations (x and h) around the FP8 experts
+  quant_nvfp4_rows, expert_mlp_w4a4, experts_tokens_w4a4
+                 - the 4-bit path: NVFP4 activations (x and h) around NVFP4 experts
 """
 from __future__ import annotations
 
@@ -74,6 +76,11 @@ def lib():
         L.oracle_expert_mlp_mx8.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, _u16p, _u16p, _u16p, _u16p,
                                             _dp]
         L.oracle_expert_mlp_mx8.restype = ctypes.c_int
+        L.oracle_quant_nvfp4_rows.argtypes = [ctypes.c_int64, ctypes.c_int, _dp, ctypes.c_int,
+                                              ctypes.POINTER(ctypes.c_uint8), ctypes.POINTER(ctypes.c_uint8), _dp, _dp]
+        L.oracle_quant_nvfp4_rows.restype = ctypes.c_int
+        L.oracle_expert_mlp_w4a4.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, _u16p, _dp, _dp, _dp, _dp]
+        L.oracle_expert_mlp_w4a4.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -369,4 +376,51 @@ def experts_tokens_mx8(x_bits: np.ndarray, ids: np.ndarray, weight: np.ndarray, 
         if rows.size == 0:
             continue
         out[rows, slots, :] = expert_mlp_mx8(x_bits[rows], *fetch(e))
+    return combine(out, weight, routed_scale)
+
+
+def quant_nvfp4_rows(v: np.ndarray, per_row_scale: bool = True):
+    """NVFP4 activation rows (blocks of 16 along the last axis): returns (E2M1 codes [rows,K] uint8 (one
+    per element), E4M3 scale codes [rows,K/16] uint8, row scales [rows] fp64, dequantised [rows,K])."""
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    rows, K = v.shape
+    q = np.empty((rows, K), dtype=np.uint8)
+    sc = np.empty((rows, K // 16), dtype=np.uint8)
+    g = np.empty(rows, dtype=np.float64)
+    deq = np.empty((rows, K), dtype=np.float64)
+    u8p = ctypes.POINTER(ctypes.c_uint8)
+    if lib().oracle_quant_nvfp4_rows(rows, K, _ptr(v, _dp), int(per_row_scale), q.ctypes.data_as(u8p),
+                                     sc.ctypes.data_as(u8p), _ptr(g, _dp), _ptr(deq, _dp)) != 0:
+        raise ValueError("NVFP4 activations: K not a multiple of 16")
+    return q, sc, g, deq
+
+
+def expert_mlp_w4a4(x_rows_bits: np.ndarray, wg: np.ndarray, wu: np.ndarray, wd: np.ndarray) -> np.ndarray:
+    """The 4-bit path's SwiGLU expert: NVFP4 x (per-row power-of-two scale), h quantised to NVFP4 (row
+    scale 1) before the down projection; FP64 weights (dequantised NVFP4).  Returns [n,H] fp64."""
+    x_rows_bits = np.ascontiguousarray(x_rows_bits, dtype=np.uint16)
+    n, H = x_rows_bits.shape
+    I = wg.shape[0]
+    assert wg.shape == (I, H) and wu.shape == (I, H) and wd.shape == (H, I)
+    out = np.empty((n, H), dtype=np.float64)
+    if n == 0:
+        return out
+    if lib().oracle_expert_mlp_w4a4(n, H, I, _ptr(x_rows_bits, _u16p),
+                                    *(_ptr(np.ascontiguousarray(w, dtype=np.float64), _dp) for w in (wg, wu, wd)),
+                                    _ptr(out, _dp)) != 0:
+        raise ValueError("4-bit expert: hidden and inter must be multiples of 16")
+    return out
+
+
+def experts_tokens_w4a4(x_bits: np.ndarray, ids: np.ndarray, weight: np.ndarray, fetch,
+                        n_experts: int, routed_scale: float) -> np.ndarray:
+    """experts_tokens of the 4-bit path (expert_mlp_w4a4 per expert; fetch gives FP64 weights)."""
+    n, H = x_bits.shape
+    k = ids.shape[1]
+    out = np.zeros((n, k, H), dtype=np.float64)
+    for e in range(n_experts):
+        rows, slots = np.nonzero(ids == e)
+        if rows.size == 0:
+            continue
+        out[rows, slots, :] = expert_mlp_w4a4(x_bits[rows], *fetch(e))
     return combine(out, weight, routed_scale)

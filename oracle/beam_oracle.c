@@ -629,3 +629,138 @@ done:
     free(hb);
     return rc;
 }
+
+/*
+ * NVFP4 activations for the 4-bit tensor-core path (reading; the pages name NVFP4 checkpoints
+ * "for Blackwell" but give no recipe; a native FP4 product needs FP4 activations).  NVFP4 applied to
+ * activation rows: a row scale g (a power of two), one E4M3 scale code per 16 consecutive K elements
+ * and E2M1 elements:
+ *   g = 2^e with e the smallest integer such that amax_row <= 2688 g (2688 = 6 x 448), when the row
+ *       scale is per row; g = 1 otherwise (the caller's choice);
+ *   s = the E4M3 value nearest to amax_block / (6 g) (ties to even, at most 448);
+ *   q = the E2M1 value nearest to v / (s g) (ties to even, magnitudes above 6 become 6; 0 if s = 0);
+ *   dequantised value q s g.
+ * v [rows,K] fp64; codes [rows,K] (one E2M1 code per element, 0..15) and scale codes
+ * [rows,K/16] (any may be NULL); g [rows] (out); deq [rows,K].  Returns -1 if K % 16.
+ */
+static double e2m1_round(double m)  /* m >= 0: nearest E2M1 magnitude, ties to even, at most 6 */
+{
+    if (m >= 6.0) return 6.0;
+    const double quantum = m < 2.0 ? 0.5 : (m < 4.0 ? 1.0 : 2.0);
+    const double rounded = nearbyint(m / quantum) * quantum;  /* half to even */
+    return rounded > 6.0 ? 6.0 : rounded;
+}
+
+static uint8_t e2m1_code_of(double v)  /* v already on the E2M1 grid */
+{
+    const double m = fabs(v);
+    const int s = signbit(v) ? 8 : 0;
+    if (m < 1.0) return (uint8_t)(s | (m == 0.5 ? 1 : 0));
+    const int e = ilogb(m);                        /* 0, 1 or 2 */
+    const int mant = ldexp(m, -e) > 1.0 ? 1 : 0;
+    return (uint8_t)(s | ((e + 1) << 1) | mant);
+}
+
+int oracle_quant_nvfp4_rows(int64_t rows, int K, const double *v, int per_row_scale, uint8_t *codes,
+                            uint8_t *scale, double *g_out, double *deq)
+{
+    if (K % 16) return -1;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const double *row = v + r * K;
+        double g = 1.0;
+        if (per_row_scale) {
+            double amax = 0.0;
+            for (int k = 0; k < K; ++k) amax = fmax(amax, fabs(row[k]));
+            if (amax > 0.0) {
+                int e = ilogb(amax / 2688.0);
+                if (amax > ldexp(2688.0, e)) e += 1;
+                while (e > -1074 && amax <= ldexp(2688.0, e - 1)) e -= 1;
+                g = ldexp(1.0, e);
+            }
+        }
+        g_out[r] = g;
+        for (int kb = 0; kb < K / 16; ++kb) {
+            double amax = 0.0;
+            for (int i = 0; i < 16; ++i) amax = fmax(amax, fabs(row[kb * 16 + i]));
+            double a = amax / (6.0 * g);
+            if (a > 448.0) a = 448.0;
+            const uint8_t sc = e4m3_round_code(a);
+            const double s = e4m3_value(sc);
+            if (scale) scale[r * (K / 16) + kb] = sc;
+            for (int i = 0; i < 16; ++i) {
+                const double x = row[kb * 16 + i];
+                double q = 0.0;
+                if (s > 0.0) {
+                    q = e2m1_round(fabs(x) / (s * g));
+                    if (signbit(x)) q = -q;
+                }
+                if (codes) codes[r * K + kb * 16 + i] = e2m1_code_of(q);
+                deq[r * K + kb * 16 + i] = q * s * g;
+            }
+        }
+    }
+    return 0;
+}
+
+/*
+ * The SwiGLU expert of the 4-bit path on n rows: x~ = NVFP4(x) with a per-row power-of-two scale,
+ * g = Wg x~, u = Wu x~, h = SiLU(g) * u, h~ = NVFP4(h) with row scale 1 (the h tiles are produced
+ * a slice of the intermediate axis at a time, so no row-wide scale is known when they are
+ * quantised), out = Wd h~, FP64 on the dequantised values; weights FP64 (NVFP4 dequantised).
+ * x_rows [n,H] bf16 bits; wg, wu [I,H]; wd [H,I]; out [n,H].
+ */
+int oracle_expert_mlp_w4a4(int64_t n, int H, int I, const uint16_t *x_rows, const double *wg, const double *wu,
+                           const double *wd, double *out)
+{
+    if (H % 16 || I % 16) return -1;
+    const int64_t nb = (n + RB - 1) / RB;
+    double *xd = (double *)malloc(sizeof(double) * (size_t)(n * H));
+    double *x4 = (double *)malloc(sizeof(double) * (size_t)(n * H));
+    double *gx = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+    double *hd = (double *)malloc(sizeof(double) * (size_t)(n * I));
+    double *h4 = (double *)malloc(sizeof(double) * (size_t)(n * I));
+    double *gh = (double *)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+    double *xb = (double *)malloc(sizeof(double) * (size_t)(nb * H * RB));
+    double *hb = (double *)malloc(sizeof(double) * (size_t)(nb * I * RB));
+    for (int64_t q = 0; q < n * H; ++q) xd[q] = bf16_bits_to_double(x_rows[q]);
+    oracle_quant_nvfp4_rows(n, H, xd, 1, NULL, NULL, gx, x4);
+    for (int64_t b = 0; b < nb; ++b)
+        for (int h = 0; h < H; ++h)
+            for (int r = 0; r < RB; ++r)
+                xb[(b * H + h) * RB + r] = b * RB + r < n ? x4[(b * RB + r) * H + h] : 0.0;
+
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < nb; ++b)
+        for (int i = 0; i < I; ++i) {
+            double g[RB], u[RB];
+            dot_rows(H, xb + b * H * RB, wg + (int64_t)i * H, g);
+            dot_rows(H, xb + b * H * RB, wu + (int64_t)i * H, u);
+            for (int r = 0; r < RB && b * RB + r < n; ++r) {
+                const double silu4 = g[r] / (1.0 + exp(-g[r]));
+                hd[(b * RB + r) * I + i] = silu4 * u[r];
+            }
+        }
+    oracle_quant_nvfp4_rows(n, I, hd, 0, NULL, NULL, gh, h4);
+    for (int64_t b = 0; b < nb; ++b)
+        for (int i = 0; i < I; ++i)
+            for (int r = 0; r < RB; ++r)
+                hb[(b * I + i) * RB + r] = b * RB + r < n ? h4[(b * RB + r) * I + i] : 0.0;
+
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < nb; ++b)
+        for (int o = 0; o < H; ++o) {
+            double acc[RB];
+            dot_rows(I, hb + b * I * RB, wd + (int64_t)o * I, acc);
+            for (int r = 0; r < RB && b * RB + r < n; ++r) out[(b * RB + r) * H + o] = acc[r];
+        }
+    free(xd);
+    free(x4);
+    free(gx);
+    free(hd);
+    free(h4);
+    free(gh);
+    free(xb);
+    free(hb);
+    return 0;
+}

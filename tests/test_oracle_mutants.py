@@ -15,6 +15,7 @@ import pytest
 import oracle
 from tests import test_oracle_fp8 as fp8
 from tests import test_oracle_mx8act as mx8
+from tests import test_oracle_w4a4 as w4a4
 from tests import test_oracle_nvfp4 as nv4
 from tests import test_oracle_norm_residual as nr
 from tests import test_oracle_pins as pins
@@ -63,6 +64,11 @@ MUTANTS = {
     "mx8_silu_missing": ("hd[(b * RB + r) * I + i] = silu_g * u[r];", "hd[(b * RB + r) * I + i] = g[r] * u[r];"),
     "mx8_x_not_quantised": ("xb[(b * H + h) * RB + r] = b * RB + r < n ? xq[(b * RB + r) * H + h] : 0.0;",
                             "xb[(b * H + h) * RB + r] = b * RB + r < n ? xd[(b * RB + r) * H + h] : 0.0;"),
+    "e2m1_round_truncate": ("const double rounded = nearbyint(m / quantum) * quantum;",
+                            "const double rounded = floor(m / quantum) * quantum;"),
+    "nvfp4_act_scale_without_6": ("double a = amax / (6.0 * g);", "double a = amax / g;"),
+    "w4a4_h_row_scale": ("oracle_quant_nvfp4_rows(n, I, hd, 0,", "oracle_quant_nvfp4_rows(n, I, hd, 1,"),
+    "w4a4_silu_missing": ("hd[(b * RB + r) * I + i] = silu4 * u[r];", "hd[(b * RB + r) * I + i] = g[r] * u[r];"),
     "expert_f64_silu_missing": ("const double act = g[r] / (1.0 + exp(-g[r]));", "const double act = g[r];"),
 }
 
@@ -89,6 +95,9 @@ PINS = [
     mx8.test_quantised_rows_match_torch_e4m3_cast_and_scale_rule,
     mx8.test_ties_round_to_even_code,
     mx8.test_expert_mx8_matches_torch_float64_composition,
+    w4a4.test_nvfp4_rows_match_exhaustive_search_and_torch_e4m3,
+    w4a4.test_codes_decode_to_the_dequantised_values,
+    w4a4.test_expert_w4a4_matches_torch_float64_composition,
 ]
 
 

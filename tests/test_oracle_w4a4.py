@@ -1,0 +1,92 @@
+"""Pins of the oracle's NVFP4 activations (4-bit path), checked against an exhaustive nearest search on
+the E2M1 grid, torch's float8 E4M3 cast and a torch float64 composition, none of it the oracle's code.
+
+Reading (the pages give no recipe): activations are quantised per row with a power-of-two row scale g
+(the smallest bringing the row's largest magnitude to at most 6 x 448; 1 for h), one E4M3 scale per
+16 elements (the nearest E4M3 value to amax / (6 g)) and E2M1 elements (nearest, ties to even,
+saturating at 6).
+"""
+import numpy as np
+import torch
+
+import oracle
+
+E2M1 = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def _nearest_e2m1(m: np.ndarray) -> np.ndarray:
+    """Nearest grid value by exhaustive search; ties to the even code (index)."""
+    d = np.abs(m[..., None] - E2M1)
+    best = d.min(-1, keepdims=True)
+    cand = np.where(d == best, np.arange(8), 99)
+    idx = np.where((cand % 2 == 0) & (cand < 99), cand, 99).min(-1)        # an even tie winner if any
+    idx = np.where(idx == 99, cand.min(-1), idx)
+    return E2M1[idx]
+
+
+def _ref_quant(v: np.ndarray, per_row: bool):
+    rows, K = v.shape
+    amax_row = np.abs(v).max(1)
+    g = np.ones(rows)
+    if per_row:
+        e = np.floor(np.log2(np.maximum(amax_row, 1e-300) / 2688.0)) - 2
+        for _ in range(6):
+            e = np.where(amax_row > 2688.0 * np.exp2(e), e + 1, e)
+        g = np.where(amax_row > 0, np.exp2(e), 1.0)
+    blk = v.reshape(rows, K // 16, 16)
+    a = np.minimum(np.abs(blk).max(-1) / (6 * g[:, None]), 448.0)
+    s = torch.from_numpy(a).to(torch.float8_e4m3fn).double().numpy()
+    with np.errstate(divide="ignore", invalid="ignore"):
+        m = np.where(s[..., None] > 0, np.abs(blk) / (s[..., None] * g[:, None, None]), 0.0)
+    q = np.sign(blk) * _nearest_e2m1(np.minimum(m, 6.0))
+    return (q * s[..., None] * g[:, None, None]).reshape(rows, K), g
+
+
+def _rows(seed, rows=12, K=256):
+    rng = np.random.default_rng(seed)
+    v = rng.standard_normal((rows, K)) * np.exp(rng.standard_normal((rows, 1)) * 3)
+    v[0, :16] = 0.0
+    v[1, 16:32] *= 1e-5
+    v[2, :] = np.round(v[2, :] * 4) / 4   # values on quarter steps: E2M1 ties after scaling
+    return v
+
+
+def test_nvfp4_rows_match_exhaustive_search_and_torch_e4m3():
+    for seed in range(4):
+        v = _rows(seed)
+        for per_row in (True, False):
+            q, sc, g, deq = oracle.quant_nvfp4_rows(v, per_row)
+            ref, gref = _ref_quant(v, per_row)
+            np.testing.assert_array_equal(g, gref)
+            np.testing.assert_array_equal(deq, ref)
+            if per_row:
+                top = np.abs(v).max(1) / g
+                assert np.all(top <= 2688.0) and np.all(top[np.abs(v).max(1) > 0] > 1344.0)
+
+
+def test_codes_decode_to_the_dequantised_values():
+    v = _rows(9)
+    q, sc, g, deq = oracle.quant_nvfp4_rows(v, True)
+    mag = E2M1[q & 7] * np.where(q & 8, -1.0, 1.0)
+    s = torch.from_numpy(sc.view(np.int8)).view(torch.float8_e4m3fn).double().numpy()
+    np.testing.assert_array_equal(mag * s.repeat(16, axis=1) * g[:, None], deq)
+
+
+def test_expert_w4a4_matches_torch_float64_composition():
+    """Two weight scales: O(1) intermediate values, and ~1e-4 ones whose 16-blocks fall below E4M3's
+    normal range under the row scale 1 that h uses (where a per-row power of two would differ)."""
+    rng = np.random.default_rng(11)
+    n, H, I = 7, 256, 128
+    x = torch.from_numpy(rng.standard_normal((n, H))).to(torch.bfloat16)
+    bits = x.view(torch.int16).numpy().view(np.uint16)
+    for scale in (1.0, 1e-2):
+        wg, wu = (rng.standard_normal((I, H)) / 16 * scale for _ in range(2))
+        wd = rng.standard_normal((H, I)) / 11
+        got = oracle.expert_mlp_w4a4(bits, wg, wu, wd)
+        xq, _ = _ref_quant(x.double().numpy(), True)
+        g = xq @ wg.T
+        u = xq @ wu.T
+        h = torch.nn.functional.silu(torch.from_numpy(g)).numpy() * u
+        hq, _ = _ref_quant(h, False)
+        ref = hq @ wd.T
+        np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
