@@ -34,6 +34,8 @@ import beam_synth as bs  # noqa: E402
 
 METRIC = "MoE-layer tokens/s (Beam shape, BF16, T=4096) and % of tensor/HBM roofline"
 METRIC_FP8 = "MoE-layer tokens/s (Beam shape, MXFP8 expert weights, T=4096) and % of tensor/HBM roofline"
+METRIC_W4A4 = ("MoE-layer tokens/s (Beam shape, NVFP4 expert weights and activations on block-scaled tensor cores, "
+               "T=4096) and % of tensor/HBM roofline")
 METRIC_MXFP8 = ("MoE-layer tokens/s (Beam shape, MXFP8 expert weights and activations on block-scaled tensor cores, "
                 "T=4096) and % of tensor/HBM roofline")
 METRIC_NVFP4 = "MoE-layer tokens/s (Beam shape, NVFP4 expert weights, T=4096) and % of tensor/HBM roofline"
@@ -90,6 +92,8 @@ def parse():
                     help="NVFP4 expert weights (E2M1 + E4M3 scale per 16 K elements + FP32 per-matrix scale)")
     ap.add_argument("--fp8", action="store_true",
                     help="MXFP8 expert weights (E4M3 + one power-of-two scale per 32 K elements)")
+    ap.add_argument("--w4a4", action="store_true",
+                    help="the 4-bit path: NVFP4 weights and activations, block-scaled tcgen05 MMA")
     ap.add_argument("--mxfp8", action="store_true",
                     help="the native FP8 path: MXFP8 weights and activations, block-scaled tcgen05 MMA")
     return ap.parse_args()
@@ -128,7 +132,8 @@ def algorithmic(wl: bs.Workload, n_act: int, fmt: str = "bf16") -> dict:
     scales are negligible)."""
     T, H, I, E, k = wl.T, wl.hidden, wl.inter, wl.n_experts, wl.topk
     R = T * k
-    wb = {"bf16": 2.0, "fp8": 1.0 + 1.0 / 32, "mxfp8": 1.0 + 1.0 / 32, "nvfp4": 0.5 + 1.0 / 16}[fmt]  # bytes per expert weight element
+    wb = {"bf16": 2.0, "fp8": 1.0 + 1.0 / 32, "mxfp8": 1.0 + 1.0 / 32, "nvfp4": 0.5 + 1.0 / 16,
+          "w4a4": 0.5 + 1.0 / 16}[fmt]  # bytes per expert weight element
     w_expert = 3 * H * I * wb
     return dict(
         layer_flops=T * (2 * H * E + k * 6 * H * I),
@@ -260,7 +265,8 @@ def cpu_oracle_rate(wl, x_cpu, W, bias, fetch, n_sample: int, route_all: bool = 
             continue
         w3 = fetch(e)
         t1 = time.perf_counter()
-        expert = {"nvfp4": oracle.expert_mlp_f64, "mxfp8": oracle.expert_mlp_mx8}.get(fmt, oracle.expert_mlp)
+        expert = {"nvfp4": oracle.expert_mlp_f64, "mxfp8": oracle.expert_mlp_mx8,
+                  "w4a4": oracle.expert_mlp_w4a4}.get(fmt, oracle.expert_mlp)
         out[rows, slots, :] = expert(xs[rows], *w3)
         t_exp += time.perf_counter() - t1
     t1 = time.perf_counter()
@@ -439,7 +445,8 @@ def run_ours(args):
     wl = reduced(bs.get(args.workload), args)
     layer = wl.layer
     T, H = wl.T, wl.hidden
-    fmt = "nvfp4" if args.nvfp4 else "fp8" if args.fp8 else "mxfp8" if args.mxfp8 else "bf16"
+    fmt = ("nvfp4" if args.nvfp4 else "fp8" if args.fp8 else "mxfp8" if args.mxfp8 else "w4a4" if args.w4a4
+           else "bf16")
     if args.also is None:
         also = [] if args.block else (["decode", "skew", "long"] if fmt == "bf16" else ["decode"])
     else:
@@ -452,7 +459,7 @@ def run_ours(args):
     if fmt != "bf16":
         if args.block:
             raise SystemExit("--fp8/--nvfp4 and --block: the sublayer entry point takes bf16 expert weights")
-        w8 = bs.quantize_experts_nvfp4(wg, wu, wd) if fmt == "nvfp4" else bs.quantize_experts(wg, wu, wd)
+        w8 = bs.quantize_experts_nvfp4(wg, wu, wd) if fmt in ("nvfp4", "w4a4") else bs.quantize_experts(wg, wu, wd)
         del wg, wu, wd
         wg = wu = wd = None
         torch.cuda.empty_cache()
@@ -473,6 +480,8 @@ def run_ours(args):
             return lambda: bm.forward_fp8(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws)
         if fmt == "mxfp8":
             return lambda: bm.forward_mxfp8(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws)
+        if fmt == "w4a4":
+            return lambda: bm.forward_w4a4(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws)
         if fmt == "nvfp4":
             return lambda: bm.forward_nvfp4(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws)
         return lambda: bm.forward(layer, x, W, bias, wg, wu, wd, y=y, ids=ids, w=w, ws=ws)
@@ -483,6 +492,8 @@ def run_ours(args):
             bm.forward_fp8(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws, events=ev)
         elif fmt == "mxfp8":
             bm.forward_mxfp8(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws, events=ev)
+        elif fmt == "w4a4":
+            bm.forward_w4a4(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws, events=ev)
         elif fmt == "nvfp4":
             bm.forward_nvfp4(layer, x, W, bias, w8, y=y, ids=ids, w=w, ws=ws, events=ev)
         else:
@@ -580,12 +591,19 @@ def run_ours(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         fetch = {"bf16": lambda: bf16_fetch(wg, wu, wd), "fp8": lambda: fp8_fetch(w8), "mxfp8": lambda: fp8_fetch(w8),
+                 "w4a4": lambda: nvfp4_fetch(w8),
                  "nvfp4": lambda: nvfp4_fetch(w8)}[fmt]()
         cpu = cpu_oracle_rate(wl, inp["x_cpu"], inp["W_cpu"], inp["b_cpu"], fetch, args.cpu_sample,
                               fmt=fmt)
         cpu.pop("seconds", None)
 
     cfg = config_dict(wl)
+    if fmt == "w4a4":
+        cfg["weights"] = ("NVFP4 experts (E2M1 + E4M3 per 16 K + FP32 per matrix, 0.5625 B/weight) and NVFP4 "
+                          "activations (x per token with a power-of-two scale, h per row) on tcgen05 "
+                          "kind::mxf4nvf4; router FP32")
+        cfg["weights_bytes"] = int(3 * wl.n_experts * wl.hidden * wl.inter * (0.5 + 1 / 16))
+        cfg["l2"] = "no flush: every step streams the 5.7 GB of NVFP4 expert weights and scales (> 126 MB L2)"
     if fmt == "mxfp8":
         cfg["weights"] = ("MXFP8 experts: E4M3 codes + UE8M0 scale per 32 K elements (1.03 B/weight) and MXFP8 "
                           "activations (x, h per row, blocks of 32) on tcgen05 kind::mxf8f6f4; router FP32")
@@ -601,9 +619,9 @@ def run_ours(args):
                           "(0.5625 B/weight), rebuilt as bf16 in a TMEM ring; router FP32")
         cfg["weights_bytes"] = int(3 * wl.n_experts * wl.hidden * wl.inter * (0.5 + 1 / 16))
         cfg["l2"] = "no flush: every step streams the 5.7 GB of NVFP4 expert weights and scales (> 126 MB L2)"
-    metric = {"bf16": METRIC, "fp8": METRIC_FP8, "mxfp8": METRIC_MXFP8, "nvfp4": METRIC_NVFP4}[fmt]
+    metric = {"bf16": METRIC, "fp8": METRIC_FP8, "mxfp8": METRIC_MXFP8, "nvfp4": METRIC_NVFP4, "w4a4": METRIC_W4A4}[fmt]
     dtype = {"bf16": "bf16", "fp8": "fp8-e4m3 weights, bf16 MMA", "mxfp8": "fp8-e4m3 weights and activations",
-             "nvfp4": "nvfp4-e2m1 weights, bf16 MMA"}[fmt]
+             "nvfp4": "nvfp4-e2m1 weights, bf16 MMA", "w4a4": "nvfp4-e2m1 weights and activations"}[fmt]
     n_launch = launches_per_step(wl, args.block)
     line = {"metric": metric, "value": head["value"], "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,

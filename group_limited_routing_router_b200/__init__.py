@@ -34,7 +34,7 @@ ERR_DEVICE_TIMEOUT = 7
 ERR_BAD_INDEX = 8
 ERR_INVALID_ARG = 9
 
-WS_ROUTE, WS_PERMUTE, WS_EXPERTS, WS_FORWARD, WS_BLOCK, WS_MXFP8 = 0, 1, 2, 3, 4, 5
+WS_ROUTE, WS_PERMUTE, WS_EXPERTS, WS_FORWARD, WS_BLOCK, WS_MXFP8, WS_W4A4 = 0, 1, 2, 3, 4, 5, 6
 
 
 class BeamMoeConfig(ctypes.Structure):
@@ -126,6 +126,10 @@ def lib() -> ctypes.CDLL:
                                              _vp]
         L.beam_moe_forward_mxfp8.argtypes = [_cfgp, ctypes.c_int64, _vp, _vp, _vp, _f8p, _vp, _vp, _vp, _vp,
                                              ctypes.c_size_t, _vp, ctypes.POINTER(ctypes.c_void_p)]
+        L.beam_moe_experts_w4a4.argtypes = [_cfgp, ctypes.c_int64, _vp, _vp, _vp, _f4p, _vp, _vp, ctypes.c_size_t,
+                                            _vp]
+        L.beam_moe_forward_w4a4.argtypes = [_cfgp, ctypes.c_int64, _vp, _vp, _vp, _f4p, _vp, _vp, _vp, _vp,
+                                            ctypes.c_size_t, _vp, ctypes.POINTER(ctypes.c_void_p)]
         L.beam_moe_gather_rows.argtypes = [_cfgp, ctypes.c_int64, _vp, _vp, _vp, _vp]
         L.beam_moe_expert_rows_workspace_size.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                                           ctypes.c_int64]
@@ -140,7 +144,8 @@ def lib() -> ctypes.CDLL:
         for name in ("beam_moe_route", "beam_moe_permute", "beam_moe_experts", "beam_moe_forward",
                      "beam_moe_forward_profiled", "beam_moe_block_forward", "beam_moe_experts_fp8",
                      "beam_moe_forward_fp8", "beam_moe_experts_nvfp4", "beam_moe_forward_nvfp4",
-                     "beam_moe_device_status", "beam_moe_gather_rows", "beam_moe_experts_mxfp8", "beam_moe_forward_mxfp8", "beam_moe_expert_rows", "beam_moe_combine",
+                     "beam_moe_device_status", "beam_moe_gather_rows", "beam_moe_experts_mxfp8", "beam_moe_forward_mxfp8",
+                     "beam_moe_experts_w4a4", "beam_moe_forward_w4a4", "beam_moe_expert_rows", "beam_moe_combine",
                      "beam_moe_selftest_timeout"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
@@ -497,6 +502,46 @@ def forward_nvfp4(cfg, x, w_router, bias, w4: dict, y=None, ids=None, w=None, ws
     _check(lib().beam_moe_forward_nvfp4(ctypes.byref(c), T, _ptr(x), _ptr(w_router), _ptr(bias), ctypes.byref(f4),
                                         _ptr(y), _ptr(ids), _ptr(w), _ptr(ws), nbytes, _stream(stream),
                                         _event_handles(events)), "beam_moe_forward_nvfp4")
+    return (y, ids, w) if return_routing else y
+
+
+def experts_w4a4(cfg, x, ids, w, w4: dict, y=None, ws=None, stream=None) -> torch.Tensor:
+    """The expert half on the 4-bit path: NVFP4 weights (as experts_nvfp4) times NVFP4 activations on
+    block-scaled tensor cores (x per token with a power-of-two scale, h per row)."""
+    c = _cfg(cfg)
+    T = x.shape[0]
+    _dev(x, "x", torch.bfloat16, (T, c.hidden))
+    _dev(ids, "ids", torch.int32, (T, c.topk))
+    _dev(w, "w", torch.float32, (T, c.topk))
+    f4 = _nvfp4_experts(c, w4)
+    y = torch.empty(T, c.hidden, dtype=torch.bfloat16, device=x.device) if y is None else y
+    _dev(y, "y", torch.bfloat16, (T, c.hidden))
+    ws, nbytes = _workspace(c, T, WS_W4A4, ws, x.device)
+    _check(lib().beam_moe_experts_w4a4(ctypes.byref(c), T, _ptr(x), _ptr(ids), _ptr(w), ctypes.byref(f4), _ptr(y),
+                                       _ptr(ws), nbytes, _stream(stream)), "beam_moe_experts_w4a4")
+    return y
+
+
+def forward_w4a4(cfg, x, w_router, bias, w4: dict, y=None, ids=None, w=None, ws=None, stream=None,
+                 return_routing: bool = False, events=None):
+    """forward() on the 4-bit path (see experts_w4a4); `events` as in forward_fp8."""
+    c = _cfg(cfg)
+    T = x.shape[0]
+    _dev(x, "x", torch.bfloat16, (T, c.hidden))
+    _dev(w_router, "w_router", torch.float32, (c.n_experts, c.hidden))
+    _dev(bias, "bias", torch.float32, (c.n_experts,))
+    f4 = _nvfp4_experts(c, w4)
+    y = torch.empty(T, c.hidden, dtype=torch.bfloat16, device=x.device) if y is None else y
+    _dev(y, "y", torch.bfloat16, (T, c.hidden))
+    if return_routing:
+        ids = torch.empty(T, c.topk, dtype=torch.int32, device=x.device) if ids is None else ids
+        w = torch.empty(T, c.topk, dtype=torch.float32, device=x.device) if w is None else w
+    _dev(ids, "ids", torch.int32, (T, c.topk))
+    _dev(w, "w", torch.float32, (T, c.topk))
+    ws, nbytes = _workspace(c, T, WS_W4A4, ws, x.device)
+    _check(lib().beam_moe_forward_w4a4(ctypes.byref(c), T, _ptr(x), _ptr(w_router), _ptr(bias), ctypes.byref(f4),
+                                       _ptr(y), _ptr(ids), _ptr(w), _ptr(ws), nbytes, _stream(stream),
+                                       _event_handles(events)), "beam_moe_forward_w4a4")
     return (y, ids, w) if return_routing else y
 
 

@@ -56,10 +56,16 @@ constexpr int64_t kMaxTokens = int64_t(1) << 24;
 #define G2_NARROW_NV4_ARGS false, 32, 32, 8, 16, 4, 32, false, 12, true
 // Block-scaled FP8 variants (tcgen05 kind::mxf8f6f4): <gate/up?, BN, B box rows, stages (K = 128),
 // TMEM slots, slot columns, gather?>; each stage also holds its scale atoms and TMEM scale columns.
-#define G1_WIDE_MX8_ARGS true, 192, 64, 3, 2, 192, false
-#define G2_WIDE_MX8_ARGS false, 192, 64, 5, 2, 192, false
-#define G1_NARROW_MX8_ARGS true, 32, 1, 5, 4, 64, true
-#define G2_NARROW_MX8_ARGS false, 32, 32, 10, 4, 32, false
+#define G1_WIDE_MX8_ARGS true, 192, 64, 3, 2, 192, false, false
+#define G2_WIDE_MX8_ARGS false, 192, 64, 5, 2, 192, false, false
+#define G1_NARROW_MX8_ARGS true, 32, 1, 5, 4, 64, true, false
+#define G2_NARROW_MX8_ARGS false, 32, 32, 10, 4, 32, false, false
+// The 4-bit path (kind::mxf4nvf4): four scale-atom sets per stage, so fewer stages and a token tile
+// of at most 128 in the wide family (one B atom per set).
+#define G1_WIDE_NV4X_ARGS true, 128, 64, 3, 2, 128, false, true
+#define G2_WIDE_NV4X_ARGS false, 128, 64, 5, 2, 128, false, true
+#define G1_NARROW_NV4X_ARGS true, 32, 1, 4, 4, 64, true, true
+#define G2_NARROW_NV4X_ARGS false, 32, 32, 8, 4, 32, false, true
 constexpr int kWideBN = 192, kWideBox = 64, kNarrowBN = 32, kNarrowBox = 32;
 
 template <bool G, int BN, int BOXN, int ST, int NS, int SC, bool GA>
@@ -75,17 +81,17 @@ bool set_gemm_fp8_smem() {
                                 Fp8GemmCfg<G, BN, BOXN, W8, BS, NS, SC, GA, AS, F4>::kSmem) == cudaSuccess;
 }
 
-template <bool G, int BN, int BOXN, int ST, int NS, int SC, bool GA>
+template <bool G, int BN, int BOXN, int ST, int NS, int SC, bool GA, bool F4>
 bool set_gemm_mx8_smem() {
-    return cudaFuncSetAttribute(grouped_gemm_mx8_kernel<G, BN, BOXN, ST, NS, SC, GA>,
+    return cudaFuncSetAttribute(grouped_gemm_mx8_kernel<G, BN, BOXN, ST, NS, SC, GA, F4>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                Mx8GemmCfg<G, BN, BOXN, ST, NS, SC, GA>::kSmem) == cudaSuccess;
+                                Mx8GemmCfg<G, BN, BOXN, ST, NS, SC, GA, F4>::kSmem) == cudaSuccess;
 }
-template <bool G, int BN, int BOXN, int ST, int NS, int SC, bool GA>
+template <bool G, int BN, int BOXN, int ST, int NS, int SC, bool GA, bool F4>
 void launch_gemm_mx8(int grid, cudaStream_t s, const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &s0,
                      const CUtensorMap &s1, const CUtensorMap &b, const Mx8Params &p) {
-    grouped_gemm_mx8_kernel<G, BN, BOXN, ST, NS, SC, GA>
-        <<<grid, kMxThreads, Mx8GemmCfg<G, BN, BOXN, ST, NS, SC, GA>::kSmem, s>>>(a0, a1, s0, s1, b, p);
+    grouped_gemm_mx8_kernel<G, BN, BOXN, ST, NS, SC, GA, F4>
+        <<<grid, kMxThreads, Mx8GemmCfg<G, BN, BOXN, ST, NS, SC, GA, F4>::kSmem, s>>>(a0, a1, s0, s1, b, p);
 }
 
 // a1 is ignored by the down projection.
@@ -141,8 +147,10 @@ int init_device(int *dev_out) {
             d.status = BEAM_MOE_ERR_UNSUPPORTED_DEVICE;
             return;
         }
-        bool ok = cudaFuncSetAttribute(router_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kRtSmemBytes) == cudaSuccess;
+        bool ok = cudaFuncSetAttribute(router_topk_kernel<kRtTok>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       rt_smem_bytes(kRtTok)) == cudaSuccess &&
+                  cudaFuncSetAttribute(router_topk_kernel<kRtTokSmall>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       rt_smem_bytes(kRtTokSmall)) == cudaSuccess;
         ok = ok && set_gemm_smem<G1_WIDE_ARGS>() && set_gemm_smem<G2_WIDE_ARGS>() &&
              set_gemm_smem<G1_NARROW_ARGS>() && set_gemm_smem<G2_NARROW_ARGS>();
         ok = ok && set_gemm_fp8_smem<G1_WIDE_FP8_ARGS>() && set_gemm_fp8_smem<G2_WIDE_FP8_ARGS>() &&
@@ -151,6 +159,8 @@ int init_device(int *dev_out) {
              set_gemm_fp8_smem<G1_NARROW_NV4_ARGS>() && set_gemm_fp8_smem<G2_NARROW_NV4_ARGS>();
         ok = ok && set_gemm_mx8_smem<G1_WIDE_MX8_ARGS>() && set_gemm_mx8_smem<G2_WIDE_MX8_ARGS>() &&
              set_gemm_mx8_smem<G1_NARROW_MX8_ARGS>() && set_gemm_mx8_smem<G2_NARROW_MX8_ARGS>();
+        ok = ok && set_gemm_mx8_smem<G1_WIDE_NV4X_ARGS>() && set_gemm_mx8_smem<G2_WIDE_NV4X_ARGS>() &&
+             set_gemm_mx8_smem<G1_NARROW_NV4X_ARGS>() && set_gemm_mx8_smem<G2_NARROW_NV4X_ARGS>();
         ok = ok && cudaFuncSetAttribute(combine_norm_residual_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         kMaxBlockHidden * 4) == cudaSuccess;
         if (!ok) d.status = BEAM_MOE_ERR_CUDA;
@@ -314,16 +324,23 @@ int enqueue_route(const beam_moe_config *c, int64_t T, const beam_bf16 *x, const
     p.topk = c->topk;
     p.group_topn = c->group_topn;
     // W_r tiles: 32 fp32 (one 128-byte swizzled row) x all 256 expert slots (rows >= E read as 0);
-    // x tiles: 32 bf16 (64-byte swizzled row) x 64 tokens (rows >= T read as 0)
+    // x tiles: 32 bf16 (64-byte swizzled row) x 64 tokens, or 16 for batches of at most 1024 tokens,
+    // so that they still spread over most of the SMs (rows >= T read as 0)
+    const int tok = T <= 1024 ? kRtTokSmall : kRtTok;
     CUtensorMap m_w, m_x;
     if (!encode_fn()) return BEAM_MOE_ERR_CUDA;
     if (!make_map_2d_any(&m_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, w_router, c->hidden, c->n_experts, kRtBK, kRtSlots,
                          CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map_2d_any(&m_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, c->hidden, T, kRtBK, kRtTok,
+        !make_map_2d_any(&m_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, x, c->hidden, T, kRtBK, tok,
                          CU_TENSOR_MAP_SWIZZLE_64B))
         return BEAM_MOE_ERR_CUDA;
-    const int64_t tiles = (T + kRtTok - 1) / kRtTok;
-    router_topk_kernel<<<static_cast<unsigned>(tiles * kRtCluster), kRtThreads, kRtSmemBytes, s>>>(m_w, m_x, p);
+    const int64_t tiles = (T + tok - 1) / tok;
+    if (tok == kRtTok)
+        router_topk_kernel<kRtTok><<<static_cast<unsigned>(tiles * kRtCluster), kRtThreads, rt_smem_bytes(kRtTok), s>>>(
+            m_w, m_x, p);
+    else
+        router_topk_kernel<kRtTokSmall><<<static_cast<unsigned>(tiles * kRtCluster), kRtThreads,
+                                          rt_smem_bytes(kRtTokSmall), s>>>(m_w, m_x, p);
     return launch_status();
 }
 
@@ -533,15 +550,115 @@ int enqueue_experts_mx8(const beam_moe_config *c, int dev, int64_t T, const beam
         return BEAM_MOE_ERR_CUDA;
     const int grid = g_dev[dev].num_sms;
     Mx8Params p1{counts, offsets, E, H, I, once, kDefaultTimeoutCycles, row_src, k, ws + L.xs, 1, ws + L.hq, ws + L.hs,
-                 nullptr};
+                 nullptr, nullptr, nullptr, nullptr};
     Mx8Params p2{counts, offsets, E, I, H, once, kDefaultTimeoutCycles, row_src, k, ws + L.hs, 0, nullptr, nullptr,
-                 reinterpret_cast<float *>(ws + L.o)};
+                 reinterpret_cast<float *>(ws + L.o), nullptr, nullptr, nullptr};
     if (narrow) launch_gemm_mx8<G1_NARROW_MX8_ARGS>(grid, s, m_wg, m_wu, m_sg, m_su, m_b1, p1);
     else launch_gemm_mx8<G1_WIDE_MX8_ARGS>(grid, s, m_wg, m_wu, m_sg, m_su, m_b1, p1);
     if ((rc = launch_status())) return rc;
     if (!record(ev, 4, s)) return BEAM_MOE_ERR_CUDA;
     if (narrow) launch_gemm_mx8<G2_NARROW_MX8_ARGS>(grid, s, m_wd, m_wd, m_sd, m_sd, m_b2, p2);
     else launch_gemm_mx8<G2_WIDE_MX8_ARGS>(grid, s, m_wd, m_wd, m_sd, m_sd, m_b2, p2);
+    if ((rc = launch_status())) return rc;
+    if (!record(ev, 5, s)) return BEAM_MOE_ERR_CUDA;
+    combine_kernel<<<static_cast<unsigned>(T), 256, 0, s>>>(reinterpret_cast<const float4 *>(ws + L.o), dest_row, w, T,
+                                                            k, H / 4, c->routed_scale, reinterpret_cast<uint2 *>(y));
+    if ((rc = launch_status())) return rc;
+    if (!record(ev, 6, s)) return BEAM_MOE_ERR_CUDA;
+    return BEAM_MOE_OK;
+}
+
+// ---- 4-bit path (NVFP4 weights and activations, tcgen05 kind::mxf4nvf4) -------------------------
+bool w4a4_shape_ok(const beam_moe_config *c) { return c->hidden % 256 == 0 && c->inter % 256 == 0; }
+
+struct W4a4Layout {
+    size_t ids = 0, w = 0, hist = 0, counts = 0, offsets = 0, row_src = 0, dest_row = 0, xq = 0, xs = 0, gx = 0, xqp = 0,
+           hq = 0, hs = 0, o = 0, total = 0;
+};
+
+W4a4Layout w4a4_layout(const beam_moe_config *c, int64_t T) {
+    W4a4Layout L;
+    if (T == 0) return L;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off = align256(off + bytes);
+        return at;
+    };
+    const size_t R = static_cast<size_t>(T) * c->topk;
+    const size_t E = c->n_experts, H = c->hidden, I = c->inter;
+    L.ids = take(R * 4);
+    L.w = take(R * 4);
+    L.hist = take(static_cast<size_t>(n_chunks(T)) * E * 4);
+    L.counts = take(E * 4);
+    L.offsets = take((E + 1) * 8);
+    L.row_src = take(R * 4);
+    L.dest_row = take(R * 4);
+    L.xq = take(static_cast<size_t>(T) * (H / 2));
+    L.xs = take(static_cast<size_t>(T) * (H / 16));
+    L.gx = take(static_cast<size_t>(T) * 4);
+    if (!narrow_tiles(c, T)) L.xqp = take(R * (H / 2));
+    L.hq = take(R * (I / 2));
+    L.hs = take(R * (I / 16));
+    L.o = take(R * H * 4);
+    L.total = off;
+    return L;
+}
+
+int enqueue_experts_w4a4(const beam_moe_config *c, int dev, int64_t T, const beam_bf16 *x, const int32_t *ids,
+                         const float *w, const beam_moe_nvfp4_experts *W, beam_bf16 *y, uint8_t *ws,
+                         const W4a4Layout &L, cudaStream_t s, cudaEvent_t const *ev) {
+    int32_t *counts = reinterpret_cast<int32_t *>(ws + L.counts);
+    int64_t *offsets = reinterpret_cast<int64_t *>(ws + L.offsets);
+    int32_t *row_src = reinterpret_cast<int32_t *>(ws + L.row_src);
+    int32_t *dest_row = reinterpret_cast<int32_t *>(ws + L.dest_row);
+    const int k = c->topk, E = c->n_experts, H = c->hidden, I = c->inter;
+    const uint64_t R = static_cast<uint64_t>(T) * k;
+    const bool narrow = narrow_tiles(c, T);
+
+    int rc = enqueue_permute(c, T, ids, counts, offsets, row_src, dest_row, reinterpret_cast<int32_t *>(ws + L.hist), s);
+    if (rc) return rc;
+    if (!record(ev, 2, s)) return BEAM_MOE_ERR_CUDA;
+    quant_nv4_rows_kernel<<<static_cast<unsigned>(T), 128, 0, s>>>(reinterpret_cast<const uint4 *>(x), H,
+                                                                  reinterpret_cast<uint2 *>(ws + L.xq), ws + L.xs,
+                                                                  reinterpret_cast<float *>(ws + L.gx));
+    if ((rc = launch_status())) return rc;
+    if (!narrow) {
+        gather_rows_kernel<<<static_cast<unsigned>(T), 128, 0, s>>>(reinterpret_cast<const uint4 *>(ws + L.xq), T, k,
+                                                                    H / 32, dest_row, reinterpret_cast<uint4 *>(ws + L.xqp));
+        if ((rc = launch_status())) return rc;
+    }
+    if (!record(ev, 3, s)) return BEAM_MOE_ERR_CUDA;
+
+    const double mean_rows = static_cast<double>(R) / E;
+    const int bn = narrow ? kNarrowBN : 128;
+    const int box = narrow ? kNarrowBox : kWideBox;
+    const int once = (mean_rows + 4.0 * std::sqrt(mean_rows) <= bn) ? 1 : 0;
+    CUtensorMap m_wg, m_wu, m_wd, m_sg, m_su, m_sd, m_b1, m_b2;
+    if (!encode_fn()) return BEAM_MOE_ERR_CUDA;
+    const bool b1_ok = narrow ? make_map_2d_any(&m_b1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws + L.xq, H / 2,
+                                                static_cast<uint64_t>(T), kMxBK, 1, CU_TENSOR_MAP_SWIZZLE_128B)
+                              : make_map_2d_any(&m_b1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws + L.xqp, H / 2, R, kMxBK,
+                                                box, CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!b1_ok ||
+        !make_map_2d_any(&m_b2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws + L.hq, I / 2, R, kMxBK, box,
+                         CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map_3d_fp4(&m_wg, W->w_gate, H, I, E) || !make_map_3d_fp4(&m_wu, W->w_up, H, I, E) ||
+        !make_map_3d_fp4(&m_wd, W->w_down, I, H, E) || !make_map_scale(&m_sg, W->w_gate_scale, I, H / 16, E, 16) ||
+        !make_map_scale(&m_su, W->w_up_scale, I, H / 16, E, 16) ||
+        !make_map_scale(&m_sd, W->w_down_scale, H, I / 16, E, 16))
+        return BEAM_MOE_ERR_CUDA;
+    const int grid = g_dev[dev].num_sms;
+    Mx8Params p1{counts, offsets, E, H, I, once, kDefaultTimeoutCycles, row_src, k, ws + L.xs, 1, ws + L.hq, ws + L.hs,
+                 nullptr, W->w_gate_global, W->w_up_global, reinterpret_cast<const float *>(ws + L.gx)};
+    Mx8Params p2{counts, offsets, E, I, H, once, kDefaultTimeoutCycles, row_src, k, ws + L.hs, 0, nullptr, nullptr,
+                 reinterpret_cast<float *>(ws + L.o), W->w_down_global, nullptr, nullptr};
+    if (narrow) launch_gemm_mx8<G1_NARROW_NV4X_ARGS>(grid, s, m_wg, m_wu, m_sg, m_su, m_b1, p1);
+    else launch_gemm_mx8<G1_WIDE_NV4X_ARGS>(grid, s, m_wg, m_wu, m_sg, m_su, m_b1, p1);
+    if ((rc = launch_status())) return rc;
+    if (!record(ev, 4, s)) return BEAM_MOE_ERR_CUDA;
+    if (narrow) launch_gemm_mx8<G2_NARROW_NV4X_ARGS>(grid, s, m_wd, m_wd, m_sd, m_sd, m_b2, p2);
+    else launch_gemm_mx8<G2_WIDE_NV4X_ARGS>(grid, s, m_wd, m_wd, m_sd, m_sd, m_b2, p2);
     if ((rc = launch_status())) return rc;
     if (!record(ev, 5, s)) return BEAM_MOE_ERR_CUDA;
     combine_kernel<<<static_cast<unsigned>(T), 256, 0, s>>>(reinterpret_cast<const float4 *>(ws + L.o), dest_row, w, T,
@@ -569,8 +686,9 @@ extern "C" {
 
 size_t beam_moe_workspace_size(const beam_moe_config *cfg, int64_t T, int which) {
     if (validate(cfg) || check_T(cfg, T)) return 0;
-    if (which < BEAM_MOE_WS_ROUTE || which > BEAM_MOE_WS_MXFP8) return 0;
+    if (which < BEAM_MOE_WS_ROUTE || which > BEAM_MOE_WS_W4A4) return 0;
     if (which == BEAM_MOE_WS_MXFP8) return mx8_shape_ok(cfg) ? mx8_layout(cfg, T).total : 0;
+    if (which == BEAM_MOE_WS_W4A4) return w4a4_shape_ok(cfg) ? w4a4_layout(cfg, T).total : 0;
     return layout(cfg, T, which).total;
 }
 
@@ -792,6 +910,56 @@ int beam_moe_forward_mxfp8(const beam_moe_config *cfg, int64_t T, const beam_bf1
     if ((rc = enqueue_route(cfg, T, x, w_router, sel_bias, ids, w, s))) return rc;
     if (!record(ev, 1, s)) return BEAM_MOE_ERR_CUDA;
     return enqueue_experts_mx8(cfg, dev, T, x, ids, w, w8, y, wsb, L, s, ev);
+}
+
+namespace {
+int w4a4_common_checks(const beam_moe_config *cfg, int64_t T, const beam_moe_nvfp4_experts *w4, const void *x,
+                       const void *y, void *ws, size_t ws_bytes, void *const *events) {
+    int rc = validate(cfg);
+    if (rc) return rc;
+    if (!w4a4_shape_ok(cfg)) return BEAM_MOE_ERR_INVALID_CONFIG;
+    if ((rc = check_T(cfg, T))) return rc;
+    if (!w4 || (events && !events_ok(events))) return BEAM_MOE_ERR_NULL;
+    if (T == 0) return BEAM_MOE_OK;
+    if (!x || !y || !ws) return BEAM_MOE_ERR_NULL;
+    if ((rc = weights_status(nvfp4_weights(w4)))) return rc;
+    if (!aligned16(x) || !aligned16(y) || !aligned16(ws)) return BEAM_MOE_ERR_MISALIGNED;
+    if (ws_bytes < w4a4_layout(cfg, T).total) return BEAM_MOE_ERR_WORKSPACE_TOO_SMALL;
+    return BEAM_MOE_OK;
+}
+}  // namespace
+
+int beam_moe_experts_w4a4(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const int32_t *topk_ids,
+                          const float *topk_w, const beam_moe_nvfp4_experts *w4, beam_bf16 *y, void *ws,
+                          size_t ws_bytes, void *stream) {
+    int rc = w4a4_common_checks(cfg, T, w4, x, y, ws, ws_bytes, nullptr);
+    if (rc || T == 0) return rc;
+    if (!topk_ids || !topk_w) return BEAM_MOE_ERR_NULL;
+    int dev;
+    if ((rc = init_device(&dev))) return rc;
+    return enqueue_experts_w4a4(cfg, dev, T, x, topk_ids, topk_w, w4, y, static_cast<uint8_t *>(ws),
+                                w4a4_layout(cfg, T), static_cast<cudaStream_t>(stream), nullptr);
+}
+
+int beam_moe_forward_w4a4(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const float *w_router,
+                          const float *sel_bias, const beam_moe_nvfp4_experts *w4, beam_bf16 *y, int32_t *topk_ids_out,
+                          float *topk_w_out, void *ws, size_t ws_bytes, void *stream, void *const *events) {
+    int rc = w4a4_common_checks(cfg, T, w4, x, y, ws, ws_bytes, events);
+    if (rc || T == 0) return rc;
+    if (!w_router) return BEAM_MOE_ERR_NULL;
+    if (!aligned16(w_router)) return BEAM_MOE_ERR_MISALIGNED;
+    int dev;
+    if ((rc = init_device(&dev))) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t *wsb = static_cast<uint8_t *>(ws);
+    const W4a4Layout L = w4a4_layout(cfg, T);
+    int32_t *ids = topk_ids_out ? topk_ids_out : reinterpret_cast<int32_t *>(wsb + L.ids);
+    float *w = topk_w_out ? topk_w_out : reinterpret_cast<float *>(wsb + L.w);
+    cudaEvent_t const *ev = reinterpret_cast<cudaEvent_t const *>(events);
+    if (!record(ev, 0, s)) return BEAM_MOE_ERR_CUDA;
+    if ((rc = enqueue_route(cfg, T, x, w_router, sel_bias, ids, w, s))) return rc;
+    if (!record(ev, 1, s)) return BEAM_MOE_ERR_CUDA;
+    return enqueue_experts_w4a4(cfg, dev, T, x, ids, w, w4, y, wsb, L, s, ev);
 }
 
 int beam_moe_device_status(void *stream) {

@@ -32,6 +32,13 @@
 //                  the stage's sf_ready barrier;
 //   warps 4..11    epilogue: two warps per TMEM lane quarter (warp w reads lanes 32 (w % 4)..+31),
 //                  taking alternate 16-column chunks of the item's tokens.
+// 4-bit variant (FP4 = true): tcgen05.mma kind::mxf4nvf4 .block16 with NVFP4 weights (E2M1 code
+// pairs, one E4M3 scale per 16 K elements, an FP32 scale per weight matrix) and NVFP4 activations
+// (x with a power-of-two scale per token, h with scale 1; E4M3 scale per 16, E2M1 elements).  A
+// 128-byte operand row then holds K = 256, one MMA takes K = 64 and reads one 32-bit word of four
+// scales per row, so each MMA of the stage has its own set of atoms (four per operand and stage).
+// The FP32 scales multiply the accumulators in the epilogues (G1: weight matrix x token; G2: weight
+// matrix).
 // Every wait is bounded (status word BEAM_MOE_ERR_DEVICE_TIMEOUT on expiry).
 #pragma once
 
@@ -44,20 +51,24 @@ constexpr int kMxThreads = 384;   // warps 0..3 producer / MMA / scale factors /
 constexpr int kMxEpiWarps = 8;
 constexpr int kMxAtom = 512;      // scale atom: 128 rows x 4 K-blocks
 
-template <bool GATE_UP, int BN, int BOXN, int STAGES, int NSLOT, int SLOT_COLS, bool GATHER>
+template <bool GATE_UP, int BN, int BOXN, int STAGES, int NSLOT, int SLOT_COLS, bool GATHER, bool FP4 = false>
 struct Mx8GemmCfg {
     static constexpr int kNumA = GATE_UP ? 2 : 1;
     static constexpr int kA = kBM * kMxBK;                 // 16 KB
     static constexpr int kB = BN * kMxBK;
     static constexpr int kBox = BOXN * kMxBK;
     static constexpr int kSfbAtoms = (BN + 127) / 128;
-    static constexpr int kRawA = 4 * kBM;                  // raw scale tile [4][128]
-    // stage: [A tiles][B][raw SFA x kNumA][SFA atoms x kNumA][SFB atoms]
+    static constexpr int kSets = FP4 ? 4 : 1;              // atom sets per stage (one per MMA for FP4)
+    static constexpr int kKbStage = FP4 ? 16 : 4;          // scale blocks per row per stage
+    static constexpr int kRawA = kKbStage * kBM;           // raw scale tile [K-blocks][128 rows]
+    static constexpr int kSetAtoms = kNumA + kSfbAtoms;    // atoms of one set: A tile(s), then B
+    // stage: [A tiles][B][raw SFA x kNumA][atom sets]
     static constexpr int kBOff = kNumA * kA;
     static constexpr int kRawOff = kBOff + kB;
     static constexpr int kAtomOff = kRawOff + kNumA * kRawA;
-    static constexpr int kStage = (kAtomOff + (kNumA + kSfbAtoms) * kMxAtom + 1023) / 1024 * 1024;
-    static constexpr int kSfColsPerStage = 4 * (kNumA + kSfbAtoms);
+    static constexpr int kStage = (kAtomOff + kSets * kSetAtoms * kMxAtom + 1023) / 1024 * 1024;
+    static constexpr int kSfColsPerSet = 4 * kSetAtoms;
+    static constexpr int kSfColsPerStage = kSets * kSfColsPerSet;
     static constexpr int kSfCol = NSLOT * SLOT_COLS;       // first TMEM scale column
     static constexpr int kTmemCols = 512;
     static constexpr int kBarOff = STAGES * kStage;
@@ -77,7 +88,7 @@ struct Mx8Params {
     const int32_t *counts;     // [E]
     const int64_t *offsets;    // [E + 1]
     int E;
-    int K;                     // reduction length (G1: H, G2: I), multiple of 128
+    int K;                     // reduction length in elements (G1: H, G2: I); a multiple of 128 (FP4: 256)
     int M;                     // weight rows (G1: I, G2: H)
     int weights_once;
     long long timeout;
@@ -87,10 +98,15 @@ struct Mx8Params {
     // s_rows[sf_token ? row_src[r] / topk : r] with K/32 bytes per row
     const uint8_t *b_scale;
     int sf_token;
-    // G1 outputs: h codes [R][M] and scales [R][M/32]; G2 output: o [R][M] fp32
+    // G1 outputs: h codes [R][M] (FP4: [R][M/2], two codes per byte) and scales [R][M/32] (FP4:
+    // [R][M/16]); G2 output: o [R][M] fp32
     uint8_t *h_q;
     uint8_t *h_s;
     float *o;
+    // FP4: FP32 scale per weight matrix [E] (g_a0: gate or down; g_a1: up) and per token [T]
+    const float *g_a0;
+    const float *g_a1;
+    const float *g_tok;
 };
 
 // Instruction descriptor, kind::mxf8f6f4 with block scaling: A and B E4M3 (format 0), K-major,
@@ -107,6 +123,23 @@ __device__ __forceinline__ void umma_mx8(uint32_t d_tmem, uint64_t adesc, uint64
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %6, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+        : "memory");
+}
+
+// Instruction descriptor, kind::mxf4nvf4: A and B E2M1 (format 1), UE4M3 scales (bit 23 = 0),
+// K = 64 per MMA, one scale word (four blocks of 16) per row.
+__device__ __forceinline__ uint32_t umma_idesc_nv4(int M, int N) {
+    return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_nv4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%4], [%5], p;\n\t}\n" ::"r"(
+            d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
         : "memory");
 }
@@ -153,6 +186,31 @@ __device__ __forceinline__ uint32_t e4m3x2_from_f32(float lo, float hi) {
     uint16_t r;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
     return r;
+}
+
+// Two FP32 values -> two E2M1 codes (nearest, ties to even, saturating at 6): lo in bits 0..3.
+__device__ __forceinline__ uint32_t e2m1x2_from_f32(float lo, float hi) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}" : "=r"(r) : "f"(hi),
+        "f"(lo));
+    return r;
+}
+
+// An E4M3 code -> its value (exact in FP32).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
+    uint32_t h2;
+    const uint16_t c = static_cast<uint16_t>(code & 0xFFu);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(c));
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+}
+
+// The NVFP4 block of 16 (row scale 1) of the value v held by each of 16 lanes (lanes 0..15 or 16..31):
+// returns this lane's E2M1 code and sets the block's E4M3 scale code.
+__device__ __forceinline__ uint32_t nv4_quant16(float v, uint32_t half_mask, uint32_t &scale_code) {
+    const float amax = __uint_as_float(__reduce_max_sync(half_mask, __float_as_uint(fabsf(v))));
+    scale_code = e4m3x2_from_f32(fminf(__fdiv_rn(amax, 6.0f), 448.0f), 0.0f) & 0xFFu;
+    const float s = e4m3_to_f32(scale_code);
+    return s > 0.0f ? (e2m1x2_from_f32(__fdiv_rn(v, s), 0.0f) & 0xFu) : 0u;
 }
 
 // G1 epilogue with MXFP8 h: the 32 lanes of warp q hold weight rows (i) 32q..32q+31 of the tile,
@@ -208,8 +266,67 @@ __device__ __forceinline__ void mx8_epilogue_g1(int q, int half, const int *tile
     }
 }
 
-// G2 epilogue: FP32 o rows in dispatch order.
+// G1 epilogue of the 4-bit path: accumulators times the FP32 scales (weight matrix x token), SwiGLU,
+// then h~ = NVFP4(h) with row scale 1: lanes 0..15 and 16..31 of warp q are two blocks of 16 along i.
+// Codes are packed two per byte (even i in the low nibble) by the even lanes.
 template <int BN, int NSLOT, int SLOT_COLS>
+__device__ __forceinline__ void nv4_epilogue_g1(int q, int half, const int *tile_start, int total, const Mx8Params &p,
+                                                uint32_t tmem_base, uint64_t *acc_full, uint64_t *acc_empty) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t half_mask = lane < 16 ? 0x0000FFFFu : 0xFFFF0000u;
+    uint32_t uses = 0;
+    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+        const Item it = decode_item(item, tile_start, p.E, BN, p.counts, p.offsets);
+        const int u = slots_of<true, SLOT_COLS>(it.n_mma);
+        bool ok = true;
+        for (int i = 0; i < u && ok; ++i) {
+            const uint32_t c = uses + i;
+            ok = mbar_wait(&acc_full[c % NSLOT], (c / NSLOT) & 1u, p.timeout);
+        }
+        if (!ok) break;
+        tc_fence_after();
+        const int s0 = uses % NSLOT, s1 = (uses + 1) % NSLOT;
+        const int m = it.mt * kBM + q * 32 + lane;
+        const bool row_ok = m < p.M;
+        const int blk = m >> 4;  // this lane's block of 16 along i
+        const bool blk_ok = (blk << 4) < p.M;
+        const float gg = __ldg(p.g_a0 + it.e), gu = __ldg(p.g_a1 + it.e);
+        const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+        const uint32_t t0 = tmem_base + lane_off + static_cast<uint32_t>(s0 * SLOT_COLS);
+        const uint32_t t1 = tmem_base + lane_off +
+                            static_cast<uint32_t>(u == 2 ? s1 * SLOT_COLS : s0 * SLOT_COLS + SLOT_COLS / 2);
+        for (int c = 16 * half; c < it.n_valid; c += 32) {
+            uint32_t rg[16], ru[16];
+            tmem_ld16(t0 + c, rg);
+            tmem_ld16(t1 + c, ru);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const bool col_ok = c + j < it.n_valid;
+                const int64_t r = it.row0 + c + j;
+                const float gt = col_ok ? __ldg(p.g_tok + p.row_src[r] / p.topk) : 0.0f;
+                const float hv = row_ok && col_ok ? silu_mul(__uint_as_float(rg[j]) * (gg * gt),
+                                                             __uint_as_float(ru[j]) * (gu * gt))
+                                                  : 0.0f;
+                uint32_t sc;
+                const uint32_t code = nv4_quant16(hv, half_mask, sc);
+                const uint32_t odd = __shfl_down_sync(0xffffffffu, code, 1);
+                if (col_ok && blk_ok) {
+                    if (row_ok && (lane & 1) == 0) p.h_q[r * (p.M >> 1) + (m >> 1)] = static_cast<uint8_t>(code | (odd << 4));
+                    if ((lane & 15) == 0) p.h_s[r * (p.M >> 4) + blk] = static_cast<uint8_t>(sc);
+                }
+            }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0)
+            for (int i = 0; i < u; ++i) mbar_arrive(&acc_empty[(uses + i) % NSLOT]);
+        uses += u;
+    }
+}
+
+// G2 epilogue: FP32 o rows in dispatch order (FP4: times the weight matrix's FP32 scale).
+template <int BN, int NSLOT, int SLOT_COLS, bool FP4>
 __device__ __forceinline__ void mx8_epilogue_g2(int q, int half, const int *tile_start, int total, const Mx8Params &p,
                                                 uint32_t tmem_base, uint64_t *acc_full, uint64_t *acc_empty) {
     const int lane = threadIdx.x & 31;
@@ -219,6 +336,7 @@ __device__ __forceinline__ void mx8_epilogue_g2(int q, int half, const int *tile
         if (!mbar_wait(&acc_full[uses % NSLOT], (uses / NSLOT) & 1u, p.timeout)) break;
         tc_fence_after();
         const int m = it.mt * kBM + q * 32 + lane;
+        const float gd = FP4 ? __ldg(p.g_a0 + it.e) : 1.0f;
         const uint32_t t0 =
             tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>((uses % NSLOT) * SLOT_COLS);
         for (int c = 16 * half; c < it.n_valid; c += 32) {
@@ -228,7 +346,7 @@ __device__ __forceinline__ void mx8_epilogue_g2(int q, int half, const int *tile
             if (m < p.M) {
 #pragma unroll
                 for (int j = 0; j < 16; ++j)
-                    if (c + j < it.n_valid) p.o[(it.row0 + c + j) * p.M + m] = __uint_as_float(r0[j]);
+                    if (c + j < it.n_valid) p.o[(it.row0 + c + j) * p.M + m] = __uint_as_float(r0[j]) * gd;
             }
         }
         tc_fence_before();
@@ -238,7 +356,7 @@ __device__ __forceinline__ void mx8_epilogue_g2(int q, int half, const int *tile
     }
 }
 
-template <bool GATE_UP, int BN, int BOXN, int STAGES, int NSLOT, int SLOT_COLS, bool GATHER>
+template <bool GATE_UP, int BN, int BOXN, int STAGES, int NSLOT, int SLOT_COLS, bool GATHER, bool FP4>
 __global__ void __launch_bounds__(kMxThreads, 1)
     grouped_gemm_mx8_kernel(const __grid_constant__ CUtensorMap tm_a0,  // W_gate (G1) / W_down (G2): E4M3 [E][M][K]
                             const __grid_constant__ CUtensorMap tm_a1,  // W_up (G1); unused for G2
@@ -246,7 +364,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
                             const __grid_constant__ CUtensorMap tm_s1,  // of a1
                             const __grid_constant__ CUtensorMap tm_b,   // B rows E4M3 [rows][K]
                             const Mx8Params p) {
-    using C = Mx8GemmCfg<GATE_UP, BN, BOXN, STAGES, NSLOT, SLOT_COLS, GATHER>;
+    using C = Mx8GemmCfg<GATE_UP, BN, BOXN, STAGES, NSLOT, SLOT_COLS, GATHER, FP4>;
     extern __shared__ uint8_t mx8_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(mx8_smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
@@ -262,7 +380,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = p.E;
     const int n_mt = (p.M + kBM - 1) / kBM;
-    const int n_kb = p.K / kMxBK;
+    const int n_kb = p.K / (FP4 ? 2 * kMxBK : kMxBK);  // stages: one 128-byte row of codes each
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -323,11 +441,11 @@ __global__ void __launch_bounds__(kMxThreads, 1)
                     uint8_t *st = smem + stage * C::kStage;
                     mbar_arrive_expect_tx(&full[stage], bytes);
                     tma_load_3d(st, &tm_a0, &full[stage], kb * kMxBK, it.mt * kBM, it.e, pol_w);
-                    tma_load_3d(st + C::kRawOff, &tm_s0, &full[stage], it.mt * kBM, 4 * kb, it.e, pol_w);
+                    tma_load_3d(st + C::kRawOff, &tm_s0, &full[stage], it.mt * kBM, C::kKbStage * kb, it.e, pol_w);
                     if (GATE_UP) {
                         tma_load_3d(st + C::kA, &tm_a1, &full[stage], kb * kMxBK, it.mt * kBM, it.e, pol_w);
-                        tma_load_3d(st + C::kRawOff + C::kRawA, &tm_s1, &full[stage], it.mt * kBM, 4 * kb, it.e,
-                                    pol_w);
+                        tma_load_3d(st + C::kRawOff + C::kRawA, &tm_s1, &full[stage], it.mt * kBM, C::kKbStage * kb,
+                                    it.e, pol_w);
                     }
                     uint8_t *sb = st + C::kBOff;
                     if (GATHER) {
@@ -356,23 +474,26 @@ __global__ void __launch_bounds__(kMxThreads, 1)
                 if ((issued >> s) & 1u) mbar_wait(&full[s], (issued_phase >> s) & 1u, p.timeout);
     } else if (warp == 2) {
         // ---------------- scale-factor builder ----------------
-        const int kbs = p.K >> 5;  // scale bytes per activation row
+        const int kbs = p.K / (FP4 ? 16 : 32);  // scale bytes per activation row
+        constexpr int kRowIt = (BN + 31) / 32;
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
             const Item it = decode_item(item, tile_start, E, BN, p.counts, p.offsets);
             for (int kb = 0; kb < n_kb && ok; ++kb) {
-                // B: one word (the stage's 4 K-blocks) per row, loaded before the stage's data lands
-                uint32_t wb[(BN + 31) / 32];
+                // B: the stage's scale words of every row (FP8: one word = 4 K-blocks; FP4: four words,
+                // one per MMA), loaded before the stage's data lands
+                uint4 wb[kRowIt];
 #pragma unroll
-                for (int i = 0; i < (BN + 31) / 32; ++i) {
+                for (int i = 0; i < kRowIt; ++i) {
                     const int n = lane + 32 * i;
-                    wb[i] = 0u;
+                    wb[i] = make_uint4(0u, 0u, 0u, 0u);
                     if (n < it.n_valid) {
                         const int64_t r = it.row0 + n;
                         const int64_t srow = p.sf_token ? static_cast<int64_t>(p.row_src[r] / p.topk) : r;
-                        wb[i] = __ldg(reinterpret_cast<const uint32_t *>(p.b_scale + srow * kbs + 4 * kb));
+                        if (FP4) wb[i] = __ldg(reinterpret_cast<const uint4 *>(p.b_scale + srow * kbs + 16 * kb));
+                        else wb[i].x = __ldg(reinterpret_cast<const uint32_t *>(p.b_scale + srow * kbs + 4 * kb));
                     }
                 }
                 ok = __all_sync(0xffffffffu, mbar_wait(&full[stage], phase, p.timeout));
@@ -380,24 +501,34 @@ __global__ void __launch_bounds__(kMxThreads, 1)
                 uint8_t *st = smem + stage * C::kStage;
                 uint8_t *atoms = st + C::kAtomOff;
 #pragma unroll
-                for (int i = 0; i < (BN + 31) / 32; ++i) {
+                for (int i = 0; i < kRowIt; ++i) {
                     const int n = lane + 32 * i;
-                    if (n < BN) *reinterpret_cast<uint32_t *>(atoms + C::kNumA * kMxAtom + sf_atom_off(n)) = wb[i];
+                    if (n < BN) {
+                        const uint32_t w4[4] = {wb[i].x, wb[i].y, wb[i].z, wb[i].w};
+#pragma unroll
+                        for (int set = 0; set < C::kSets; ++set)
+                            *reinterpret_cast<uint32_t *>(atoms + (set * C::kSetAtoms + C::kNumA) * kMxAtom +
+                                                          sf_atom_off(n)) = w4[set];
+                    }
                 }
-                // A: raw [4 K-blocks][128 rows] -> atom; lane l takes rows 4l..4l+3
+                // A: raw [K-blocks][128 rows] -> atoms; lane l takes rows 4l..4l+3, set by set
 #pragma unroll
                 for (int a = 0; a < C::kNumA; ++a) {
                     const uint8_t *raw = st + C::kRawOff + a * C::kRawA;
-                    uint32_t w[4];
 #pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) w[k4] = *reinterpret_cast<const uint32_t *>(raw + k4 * kBM + 4 * lane);
+                    for (int set = 0; set < C::kSets; ++set) {
+                        uint32_t w[4];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const uint32_t sel = static_cast<uint32_t>(i | ((4 + i) << 4));
-                        const uint32_t lo = __byte_perm(w[0], w[1], sel);
-                        const uint32_t hi = __byte_perm(w[2], w[3], sel);
-                        *reinterpret_cast<uint32_t *>(atoms + a * kMxAtom + sf_atom_off(4 * lane + i)) =
-                            __byte_perm(lo, hi, 0x5410);
+                        for (int k4 = 0; k4 < 4; ++k4)
+                            w[k4] = *reinterpret_cast<const uint32_t *>(raw + (4 * set + k4) * kBM + 4 * lane);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const uint32_t sel = static_cast<uint32_t>(i | ((4 + i) << 4));
+                            const uint32_t lo = __byte_perm(w[0], w[1], sel);
+                            const uint32_t hi = __byte_perm(w[2], w[3], sel);
+                            *reinterpret_cast<uint32_t *>(atoms + (set * C::kSetAtoms + a) * kMxAtom +
+                                                          sf_atom_off(4 * lane + i)) = __byte_perm(lo, hi, 0x5410);
+                        }
                     }
                 }
                 fence_proxy_async_smem();
@@ -439,20 +570,31 @@ __global__ void __launch_bounds__(kMxThreads, 1)
                     const uint32_t atoms = sa + C::kAtomOff;
                     const uint32_t sf_col = tmem_base + static_cast<uint32_t>(C::kSfCol + stage * C::kSfColsPerStage);
 #pragma unroll
-                    for (int a = 0; a < C::kNumA + C::kSfbAtoms; ++a)
+                    for (int a = 0; a < C::kSets * C::kSetAtoms; ++a)
                         tmem_cp_sf_atom(sf_col + 4 * a, sf_atom_desc(atoms + a * kMxAtom));
-                    const uint32_t sfb = sf_col + 4 * C::kNumA;
                     const uint64_t da0 = umma_desc_sw128(sa);
                     const uint64_t da1 = umma_desc_sw128(sa + C::kA);
                     const uint64_t db = umma_desc_sw128(sa + C::kBOff);
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4) {
                         const uint32_t accum = (kb > 0 || k4 > 0) ? 1u : 0u;
-                        const uint32_t idesc = umma_idesc_mx8(kBM, it.n_mma, static_cast<uint32_t>(k4));
-                        const uint32_t byte = static_cast<uint32_t>(k4) << 30;
                         // +32 bytes along K inside the swizzle row = +2 in the 16-byte address field
-                        umma_mx8(d0, da0 + 2 * k4, db + 2 * k4, idesc, sf_col | byte, sfb | byte, accum);
-                        if (GATE_UP) umma_mx8(d1, da1 + 2 * k4, db + 2 * k4, idesc, (sf_col + 4) | byte, sfb | byte, accum);
+                        if (FP4) {
+                            // MMA k4 reads its own atom set (a whole scale word per row)
+                            const uint32_t set_col = sf_col + static_cast<uint32_t>(k4 * C::kSfColsPerSet);
+                            const uint32_t idesc = umma_idesc_nv4(kBM, it.n_mma);
+                            umma_nv4(d0, da0 + 2 * k4, db + 2 * k4, idesc, set_col, set_col + 4 * C::kNumA, accum);
+                            if (GATE_UP) umma_nv4(d1, da1 + 2 * k4, db + 2 * k4, idesc, set_col + 4, set_col + 4 * C::kNumA,
+                                                  accum);
+                        } else {
+                            // MMA k4 reads byte k4 of the stage's scale words
+                            const uint32_t idesc = umma_idesc_mx8(kBM, it.n_mma, static_cast<uint32_t>(k4));
+                            const uint32_t byte = static_cast<uint32_t>(k4) << 30;
+                            const uint32_t sfb = sf_col + 4 * C::kNumA;
+                            umma_mx8(d0, da0 + 2 * k4, db + 2 * k4, idesc, sf_col | byte, sfb | byte, accum);
+                            if (GATE_UP)
+                                umma_mx8(d1, da1 + 2 * k4, db + 2 * k4, idesc, (sf_col + 4) | byte, sfb | byte, accum);
+                        }
                     }
                     umma_commit(&empty[stage]);
                     if (++stage == STAGES) {
@@ -469,8 +611,9 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         }
     } else if (warp >= 4) {
         const int q = warp & 3, half = (warp - 4) >> 2;
-        if (GATE_UP) mx8_epilogue_g1<BN, NSLOT, SLOT_COLS>(q, half, tile_start, total, p, tmem_base, acc_full, acc_empty);
-        else mx8_epilogue_g2<BN, NSLOT, SLOT_COLS>(q, half, tile_start, total, p, tmem_base, acc_full, acc_empty);
+        if (GATE_UP && FP4) nv4_epilogue_g1<BN, NSLOT, SLOT_COLS>(q, half, tile_start, total, p, tmem_base, acc_full, acc_empty);
+        else if (GATE_UP) mx8_epilogue_g1<BN, NSLOT, SLOT_COLS>(q, half, tile_start, total, p, tmem_base, acc_full, acc_empty);
+        else mx8_epilogue_g2<BN, NSLOT, SLOT_COLS, FP4>(q, half, tile_start, total, p, tmem_base, acc_full, acc_empty);
     }
     tc_fence_before();
     __syncthreads();
@@ -509,6 +652,64 @@ __global__ void __launch_bounds__(256) quant_mx8_rows_kernel(const uint4 *__rest
     if (live) {
         q[t] = out;
         if ((t & 3) == 0) s[blk] = static_cast<uint8_t>(code);
+    }
+}
+
+}  // namespace beam
+
+namespace beam {
+
+// x [T][H] bf16 -> NVFP4 codes x_q [T][H/2] (two per byte, even k low), E4M3 scale codes x_s [T][H/16]
+// and the token's power-of-two scale g[T] (the smallest g with amax_row <= 6 * 448 * g).  One CTA per
+// token; each thread takes blocks of 16.
+__global__ void __launch_bounds__(128) quant_nv4_rows_kernel(const uint4 *__restrict__ x, int H,
+                                                             uint2 *__restrict__ q, uint8_t *__restrict__ s,
+                                                             float *__restrict__ g_out) {
+    __shared__ uint32_t warp_max[4];
+    const int64_t t = blockIdx.x;
+    const uint4 *row = x + t * (H / 8);
+    const int nb = H / 16;
+    uint32_t amax_bits = 0;
+    for (int b = threadIdx.x; b < nb; b += blockDim.x) {
+        const uint4 v0 = __ldg(row + 2 * b), v1 = __ldg(row + 2 * b + 1);
+        const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            amax_bits = max(amax_bits, max((w[i] << 16) & 0x7FFFFFFFu, w[i] & 0x7FFF0000u));
+    }
+    amax_bits = __reduce_max_sync(0xffffffffu, amax_bits);
+    if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = amax_bits;
+    __syncthreads();
+    amax_bits = max(max(warp_max[0], warp_max[1]), max(warp_max[2], warp_max[3]));
+    // 6 * 448 = 2688 = 1.3125 * 2^11: e = E - 11, plus one when the mantissa exceeds 1.3125
+    float g = 1.0f;
+    if (amax_bits != 0u) {
+        const int E = static_cast<int>(amax_bits >> 23) - 127;
+        const int e = E - 11 + ((amax_bits & 0x7FFFFFu) > 0x280000u ? 1 : 0);
+        g = __uint_as_float(static_cast<uint32_t>(127 + e) << 23);
+    }
+    if (threadIdx.x == 0) g_out[t] = g;
+    for (int b = threadIdx.x; b < nb; b += blockDim.x) {
+        const uint4 v0 = __ldg(row + 2 * b), v1 = __ldg(row + 2 * b + 1);
+        const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+        float f[16];
+        float bmax = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+            bmax = fmaxf(bmax, fmaxf(fabsf(f[2 * i]), fabsf(f[2 * i + 1])));
+        }
+        const uint32_t sc = e4m3x2_from_f32(fminf(__fdiv_rn(bmax, 6.0f * g), 448.0f), 0.0f) & 0xFFu;
+        const float sg = e4m3_to_f32(sc) * g;
+        uint32_t packed[2] = {0u, 0u};
+        if (sg > 0.0f) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                packed[i >> 2] |= e2m1x2_from_f32(__fdiv_rn(f[2 * i], sg), __fdiv_rn(f[2 * i + 1], sg)) << (8 * (i & 3));
+        }
+        q[t * nb + b] = make_uint2(packed[0], packed[1]);
+        s[t * nb + b] = static_cast<uint8_t>(sc);
     }
 }
 

@@ -28,18 +28,21 @@ namespace beam {
 
 namespace cg = cooperative_groups;
 
-constexpr int kRtTok = 64;        // tokens per cluster tile
+constexpr int kRtTok = 64;        // tokens per cluster tile (kRtTokSmall for small batches)
+constexpr int kRtTokSmall = 16;
 constexpr int kRtBK = 32;         // K per pipeline stage (one 128-byte row of fp32 W)
 constexpr int kRtThreads = 128;   // 4 warps
 constexpr int kRtCluster = 8;     // CTAs per cluster (split-K factor)
 constexpr int kRtSlots = 256;     // expert slots per tile (E <= 256)
 constexpr int kRtStages = 3;      // TMA pipeline depth
 constexpr int kRtWBytes = kRtSlots * kRtBK * 4;  // W stage: [256 rows][32 fp32], 128-byte swizzle (32 KB)
-constexpr int kRtXBytes = kRtTok * kRtBK * 2;    // x stage: [64 rows][32 bf16], 64-byte swizzle (4 KB)
-constexpr int kRtStageBytes = kRtWBytes + kRtXBytes;
-constexpr int kRtSmemBytes = 1024 + kRtStages * kRtStageBytes + 128;  // + alignment + barriers: two CTAs per SM
-static_assert(kRtTok * kRtSlots * 4 <= kRtStages * kRtStageBytes, "partial logits must fit in the stages");
-static_assert(kRtStageBytes % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
+// x stage: [TOK rows][32 bf16], 64-byte swizzle (TOK * 64 bytes)
+constexpr int rt_stage_bytes(int tok) { return kRtWBytes + tok * kRtBK * 2; }
+// + alignment + barriers: two CTAs per SM
+constexpr int rt_smem_bytes(int tok) { return 1024 + kRtStages * rt_stage_bytes(tok) + 128; }
+static_assert(kRtTok * kRtSlots * 4 <= kRtStages * rt_stage_bytes(kRtTok), "partial logits must fit in the stages");
+static_assert(rt_stage_bytes(kRtTok) % 1024 == 0 && rt_stage_bytes(kRtTokSmall) % 1024 == 0,
+              "stages keep the 1024-byte swizzle alignment");
 
 struct RouterParams {
     const __nv_bfloat16 *x;  // [T, H]
@@ -76,25 +79,30 @@ __device__ __forceinline__ void top2_insert(float &a1, float &a2, float v) {
     a1 = fmaxf(a1, v);
 }
 
+// TOK tokens per cluster tile: 64 (8 per thread), or 16 (2 per thread) so that small batches still
+// spread over most of the SMs.
+template <int TOK>
 __global__ void __cluster_dims__(kRtCluster, 1, 1) __launch_bounds__(kRtThreads, 2)
     router_topk_kernel(const __grid_constant__ CUtensorMap tm_w,  // W_r [E][H] fp32, box {32, 256}
                        const __grid_constant__ CUtensorMap tm_x,  // x [T][H] bf16, box {32, 64}
                        const RouterParams p) {
     extern __shared__ uint8_t rt_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(rt_smem_raw) + 1023) & ~uintptr_t(1023));
+    constexpr int kRtStageBytes = rt_stage_bytes(TOK);
+    constexpr int kTi = TOK / 8;  // tokens per thread
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + kRtStages * kRtStageBytes);
     uint64_t *empty = full + kRtStages;
-    float *part = reinterpret_cast<float *>(smem);  // [kRtTok][kRtSlots] after the K loop
+    float *part = reinterpret_cast<float *>(smem);  // [TOK][kRtSlots] after the K loop
 
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = static_cast<int>(cluster.block_rank());
-    const int64_t t0 = static_cast<int64_t>(blockIdx.x / kRtCluster) * kRtTok;
+    const int64_t t0 = static_cast<int64_t>(blockIdx.x / kRtCluster) * TOK;
     const int tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
-    // warp tile: tokens 32*(warp&1) + [0,32) x experts 128*(warp>>1) + [0,128).  Lane (a = lane>>3,
-    // b = lane&7) owns tokens tokA + 4i (i < 8) and experts expB + 8j (j < 16).
+    // warp tile: tokens (TOK/2)*(warp&1) + [0,TOK/2) x experts 128*(warp>>1) + [0,128).  Lane
+    // (a = lane>>3, b = lane&7) owns tokens tokA + 4i (i < TOK/8) and experts expB + 8j (j < 16).
     const int a = lane >> 3, b = lane & 7;
-    const int tokA = 32 * (warp & 1) + a;
+    const int tokA = (TOK / 2) * (warp & 1) + a;
     const int expB = 128 * (warp >> 1) + b;
 
     // ---- split-K FP32 projection --------------------------------------------------------------
@@ -124,9 +132,9 @@ __global__ void __cluster_dims__(kRtCluster, 1, 1) __launch_bounds__(kRtThreads,
     if (tid == 0)
         for (; n_issued < kRtStages && n_issued < n_my; ++n_issued) issue(n_issued);
 
-    float acc[8][16];
+    float acc[kTi][16];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < kTi; ++i)
 #pragma unroll
         for (int j = 0; j < 16; ++j) acc[i][j] = 0.0f;
 
@@ -149,9 +157,9 @@ __global__ void __cluster_dims__(kRtCluster, 1, 1) __launch_bounds__(kRtThreads,
             for (int j = 0; j < 16; ++j)
                 wv[j] = *reinterpret_cast<const float2 *>(wsb + (expB + 8 * j) * 128 + woff);
             // x row t, bf16 pair k = 2kp, 2kp+1: 16-byte chunk (kp>>2) ^ ((t>>1)&3) of the 64-byte row
-            uint32_t xp[8];
+            uint32_t xp[kTi];
 #pragma unroll
-            for (int i2 = 0; i2 < 8; ++i2) {
+            for (int i2 = 0; i2 < kTi; ++i2) {
                 const int t = tokA + 4 * i2;
                 xp[i2] = *reinterpret_cast<const uint32_t *>(
                     xsb + t * 64 + ((((kp >> 2) ^ ((t >> 1) & 3)) << 4) | ((kp & 3) << 2)));
@@ -162,7 +170,7 @@ __global__ void __cluster_dims__(kRtCluster, 1, 1) __launch_bounds__(kRtThreads,
                 for (int j = 0; j < 16; ++j) {
                     const float wj = kk == 0 ? wv[j].x : wv[j].y;
 #pragma unroll
-                    for (int i2 = 0; i2 < 8; ++i2) {
+                    for (int i2 = 0; i2 < kTi; ++i2) {
                         // bf16 -> fp32 is a 16-bit shift of the bit pattern (exact)
                         const float xv = __uint_as_float(kk == 0 ? (xp[i2] << 16) : (xp[i2] & 0xffff0000u));
                         acc[i2][j] = fmaf(xv, wj, acc[i2][j]);
@@ -189,16 +197,19 @@ __global__ void __cluster_dims__(kRtCluster, 1, 1) __launch_bounds__(kRtThreads,
 
     // partial logits -> shared memory
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < kTi; ++i)
 #pragma unroll
         for (int j = 0; j < 16; ++j) part[(tokA + 4 * i) * kRtSlots + expB + 8 * j] = acc[i][j];
     cluster.sync();
 
-    // ---- reduction over the cluster + selection: warp w owns tokens 8*rank + w and 8*rank + w + 4
+    // ---- reduction over the cluster + selection: CTA rank takes tokens kTi*rank + [0, kTi), warp w
+    // the tokens w and w + 4 among them
     const int per = p.E / p.G;
 #define EID(j) (lane + 32 * (j))
     for (int u = 0; u < 2; ++u) {
-        const int tt = rank * 8 + warp + 4 * u;
+        const int lt = warp + 4 * u;
+        if (lt >= kTi) continue;
+        const int tt = rank * kTi + lt;
         const int64_t t = t0 + tt;
         if (t >= p.T) continue;
         float sc[8], sel[8];

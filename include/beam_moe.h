@@ -81,7 +81,8 @@ enum {
     BEAM_MOE_WS_EXPERTS = 2,
     BEAM_MOE_WS_FORWARD = 3,
     BEAM_MOE_WS_BLOCK = 4,
-    BEAM_MOE_WS_MXFP8 = 5  /* beam_moe_experts_mxfp8 and beam_moe_forward_mxfp8 */
+    BEAM_MOE_WS_MXFP8 = 5, /* beam_moe_experts_mxfp8 and beam_moe_forward_mxfp8 */
+    BEAM_MOE_WS_W4A4 = 6   /* beam_moe_experts_w4a4 and beam_moe_forward_w4a4 */
 };
 
 /*
@@ -306,6 +307,27 @@ BEAM_MOE_API int beam_moe_forward_mxfp8(const beam_moe_config *cfg, int64_t T, c
                                         const float *w_router, const float *sel_bias, const beam_moe_fp8_experts *w8,
                                         beam_bf16 *y, int32_t *topk_ids_out, float *topk_w_out, void *ws,
                                         size_t ws_bytes, void *stream, void *const *events);
+
+/*
+ * 4-bit path: the NVFP4 expert weights (beam_moe_nvfp4_experts) multiplied on the tensor cores with
+ * block scaling (tcgen05.mma kind::mxf4nvf4, block16: E2M1 x E2M1, one E4M3 scale per 16 K elements
+ * on each side, FP32 accumulation), the per-matrix FP32 scales applied to the accumulators.  The
+ * activations are quantised to NVFP4 as well: x per token with a power-of-two token scale g (the
+ * smallest with max|x_t| <= 6 * 448 * g), h per dispatch row with scale 1; in blocks of 16 along the
+ * reduction axis, an E4M3 scale nearest to amax / (6 g) and E2M1 elements nearest to v / (s g)
+ * (ties to even, saturating at 6).  This is a reading (the pages give no recipe): 4-bit activations
+ * change the result by far more than the weights' rounding; beam_moe_forward_nvfp4 keeps bf16
+ * activations.  Requires hidden and inter to be multiples of 256.  Workspace:
+ * beam_moe_workspace_size(cfg, T, BEAM_MOE_WS_W4A4).  Other arguments, outputs and error codes as
+ * beam_moe_experts_nvfp4 / beam_moe_forward_nvfp4.
+ */
+BEAM_MOE_API int beam_moe_experts_w4a4(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x,
+                                       const int32_t *topk_ids, const float *topk_w, const beam_moe_nvfp4_experts *w4,
+                                       beam_bf16 *y, void *ws, size_t ws_bytes, void *stream);
+BEAM_MOE_API int beam_moe_forward_w4a4(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x,
+                                       const float *w_router, const float *sel_bias, const beam_moe_nvfp4_experts *w4,
+                                       beam_bf16 *y, int32_t *topk_ids_out, float *topk_w_out, void *ws,
+                                       size_t ws_bytes, void *stream, void *const *events);
 
 /*
  * Expert parallelism ("Welcome Beam" page, section "Multi-GPU and multi-node": each expert lives on

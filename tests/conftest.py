@@ -26,7 +26,8 @@ def cuda_available() -> bool:
 # then the whole block and the expert half, then the sublayer, the dense MLP and the low-precision
 # checkpoints.  Tests marked `last` run after all others.
 _ORDER = ["test_gpu_route.py", "test_gpu_permute.py", "test_gpu_forward.py", "test_gpu_experts.py", "test_gpu_ep.py",
-          "test_gpu_block.py", "test_gpu_dense.py", "test_gpu_fp8.py", "test_gpu_mxfp8.py", "test_gpu_nvfp4.py"]
+          "test_gpu_block.py", "test_gpu_dense.py", "test_gpu_fp8.py", "test_gpu_mxfp8.py", "test_gpu_nvfp4.py",
+          "test_gpu_w4a4.py"]
 
 
 def _rank(item) -> tuple:

@@ -75,6 +75,8 @@ class Bank:
         "mxfp8" (the native FP8 path) reads the FP8 checkpoint like "fp8"."""
         if fmt == "mxfp8":
             fmt = "fp8"
+        if fmt == "w4a4":
+            fmt = "nvfp4"
         if fmt == "bf16":
             h = self.host()
             return lambda e: (h[0][e], h[1][e], h[2][e])
@@ -136,7 +138,7 @@ class Bank:
 
 # the oracle's expert half per weight format
 _RUN = {"bf16": oracle.experts_tokens, "fp8": oracle.experts_tokens, "nvfp4": oracle.experts_tokens_f64,
-        "mxfp8": oracle.experts_tokens_mx8}
+        "mxfp8": oracle.experts_tokens_mx8, "w4a4": oracle.experts_tokens_w4a4}
 
 _BANK: Optional[Bank] = None
 
