@@ -501,7 +501,7 @@ Mx8Layout mx8_layout(const beam_moe_config *c, int64_t T) {
     if (!narrow_tiles(c, T)) L.xqp = take(R * H);  // x codes in dispatch order (wide tiles only)
     L.hq = take(R * I);
     L.hs = take(R * (I / 32));
-    L.o = take(R * H * 4);
+    L.o = take(R * H * 2);  // bf16 expert outputs
     L.total = off;
     return L;
 }
@@ -552,7 +552,7 @@ int enqueue_experts_mx8(const beam_moe_config *c, int dev, int64_t T, const beam
     Mx8Params p1{counts, offsets, E, H, I, once, kDefaultTimeoutCycles, row_src, k, ws + L.xs, 1, ws + L.hq, ws + L.hs,
                  nullptr, nullptr, nullptr, nullptr};
     Mx8Params p2{counts, offsets, E, I, H, once, kDefaultTimeoutCycles, row_src, k, ws + L.hs, 0, nullptr, nullptr,
-                 reinterpret_cast<float *>(ws + L.o), nullptr, nullptr, nullptr};
+                 reinterpret_cast<__nv_bfloat16 *>(ws + L.o), nullptr, nullptr, nullptr};
     if (narrow) launch_gemm_mx8<G1_NARROW_MX8_ARGS>(grid, s, m_wg, m_wu, m_sg, m_su, m_b1, p1);
     else launch_gemm_mx8<G1_WIDE_MX8_ARGS>(grid, s, m_wg, m_wu, m_sg, m_su, m_b1, p1);
     if ((rc = launch_status())) return rc;
@@ -561,8 +561,9 @@ int enqueue_experts_mx8(const beam_moe_config *c, int dev, int64_t T, const beam
     else launch_gemm_mx8<G2_WIDE_MX8_ARGS>(grid, s, m_wd, m_wd, m_sd, m_sd, m_b2, p2);
     if ((rc = launch_status())) return rc;
     if (!record(ev, 5, s)) return BEAM_MOE_ERR_CUDA;
-    combine_kernel<<<static_cast<unsigned>(T), 256, 0, s>>>(reinterpret_cast<const float4 *>(ws + L.o), dest_row, w, T,
-                                                            k, H / 4, c->routed_scale, reinterpret_cast<uint2 *>(y));
+    combine_bf16_kernel<<<static_cast<unsigned>(T), 256, 0, s>>>(reinterpret_cast<const uint4 *>(ws + L.o), dest_row,
+                                                                 w, T, k, H / 8, c->routed_scale,
+                                                                 reinterpret_cast<uint4 *>(y));
     if ((rc = launch_status())) return rc;
     if (!record(ev, 6, s)) return BEAM_MOE_ERR_CUDA;
     return BEAM_MOE_OK;
@@ -600,7 +601,7 @@ W4a4Layout w4a4_layout(const beam_moe_config *c, int64_t T) {
     if (!narrow_tiles(c, T)) L.xqp = take(R * (H / 2));
     L.hq = take(R * (I / 2));
     L.hs = take(R * (I / 16));
-    L.o = take(R * H * 4);
+    L.o = take(R * H * 2);  // bf16 expert outputs
     L.total = off;
     return L;
 }
@@ -652,7 +653,7 @@ int enqueue_experts_w4a4(const beam_moe_config *c, int dev, int64_t T, const bea
     Mx8Params p1{counts, offsets, E, H, I, once, kDefaultTimeoutCycles, row_src, k, ws + L.xs, 1, ws + L.hq, ws + L.hs,
                  nullptr, W->w_gate_global, W->w_up_global, reinterpret_cast<const float *>(ws + L.gx)};
     Mx8Params p2{counts, offsets, E, I, H, once, kDefaultTimeoutCycles, row_src, k, ws + L.hs, 0, nullptr, nullptr,
-                 reinterpret_cast<float *>(ws + L.o), W->w_down_global, nullptr, nullptr};
+                 reinterpret_cast<__nv_bfloat16 *>(ws + L.o), W->w_down_global, nullptr, nullptr};
     if (narrow) launch_gemm_mx8<G1_NARROW_NV4X_ARGS>(grid, s, m_wg, m_wu, m_sg, m_su, m_b1, p1);
     else launch_gemm_mx8<G1_WIDE_NV4X_ARGS>(grid, s, m_wg, m_wu, m_sg, m_su, m_b1, p1);
     if ((rc = launch_status())) return rc;
@@ -661,8 +662,9 @@ int enqueue_experts_w4a4(const beam_moe_config *c, int dev, int64_t T, const bea
     else launch_gemm_mx8<G2_WIDE_NV4X_ARGS>(grid, s, m_wd, m_wd, m_sd, m_sd, m_b2, p2);
     if ((rc = launch_status())) return rc;
     if (!record(ev, 5, s)) return BEAM_MOE_ERR_CUDA;
-    combine_kernel<<<static_cast<unsigned>(T), 256, 0, s>>>(reinterpret_cast<const float4 *>(ws + L.o), dest_row, w, T,
-                                                            k, H / 4, c->routed_scale, reinterpret_cast<uint2 *>(y));
+    combine_bf16_kernel<<<static_cast<unsigned>(T), 256, 0, s>>>(reinterpret_cast<const uint4 *>(ws + L.o), dest_row,
+                                                                 w, T, k, H / 8, c->routed_scale,
+                                                                 reinterpret_cast<uint4 *>(y));
     if ((rc = launch_status())) return rc;
     if (!record(ev, 6, s)) return BEAM_MOE_ERR_CUDA;
     return BEAM_MOE_OK;
@@ -1052,19 +1054,8 @@ __global__ void dense_schedule_kernel(int32_t *counts, int64_t *offsets, int64_t
     offsets[1] = T;
 }
 
-__global__ void f32_to_bf16_kernel(const float4 *__restrict__ in, uint2 *__restrict__ out, int64_t n4) {
-    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
-         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const float4 v = __ldg(in + i);
-        uint2 r;
-        r.x = pack_bf16x2(v.x, v.y);
-        r.y = pack_bf16x2(v.z, v.w);
-        out[i] = r;
-    }
-}
-
 struct DenseLayout {
-    size_t counts = 0, offsets = 0, h = 0, o = 0, total = 0;
+    size_t counts = 0, offsets = 0, h = 0, total = 0;
 };
 
 bool dense_shape_ok(int32_t H, int32_t I) {
@@ -1083,7 +1074,6 @@ DenseLayout dense_layout(int32_t H, int32_t I, int64_t T) {
     L.counts = take(4);
     L.offsets = take(16);
     L.h = take(static_cast<size_t>(T) * I * 2);
-    L.o = take(static_cast<size_t>(T) * H * 4);
     L.total = off;
     return L;
 }
@@ -1115,7 +1105,6 @@ extern "C" int beam_moe_dense_swiglu(int32_t hidden, int32_t inter, int64_t T, c
     int32_t *counts = reinterpret_cast<int32_t *>(wsb + L.counts);
     int64_t *offsets = reinterpret_cast<int64_t *>(wsb + L.offsets);
     void *h = wsb + L.h;
-    void *o = wsb + L.o;
     dense_schedule_kernel<<<1, 1, 0, s>>>(counts, offsets, T);
     if ((rc = launch_status())) return rc;
     // x itself is the token-ordered B operand of the gate/up GEMM (wide tiles, 64-row boxes)
@@ -1128,14 +1117,11 @@ extern "C" int beam_moe_dense_swiglu(int32_t hidden, int32_t inter, int64_t T, c
         return BEAM_MOE_ERR_CUDA;
     const int grid = g_dev[dev].num_sms;
     GemmParams p1{counts, offsets, h, 1, hidden, inter, 0, kDefaultTimeoutCycles, nullptr, 1};
-    GemmParams p2{counts, offsets, o, 1, inter, hidden, 0, kDefaultTimeoutCycles, nullptr, 1};
+    // the down projection's rows, rounded to bf16, are the output: one token-ordered expert needs no combine
+    GemmParams p2{counts, offsets, y, 1, inter, hidden, 0, kDefaultTimeoutCycles, nullptr, 1, nullptr, 1};
     launch_gemm<G1_WIDE_ARGS>(grid, s, m_wg, m_wu, m_x, p1);
     if ((rc = launch_status())) return rc;
     launch_gemm<G2_WIDE_ARGS>(grid, s, m_wd, m_wd, m_h, p2);
-    if ((rc = launch_status())) return rc;
-    const int64_t n4 = T * static_cast<int64_t>(hidden) / 4;
-    f32_to_bf16_kernel<<<static_cast<unsigned>(std::min<int64_t>((n4 + 255) / 256, 16384)), 256, 0, s>>>(
-        reinterpret_cast<const float4 *>(o), reinterpret_cast<uint2 *>(y), n4);
     return launch_status();
 }
 

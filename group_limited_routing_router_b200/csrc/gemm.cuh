@@ -60,7 +60,7 @@ struct GemmCfg {
 struct GemmParams {
     const int32_t *counts;    // [E]
     const int64_t *offsets;   // [E + 1]
-    void *out;                // G1: h [R, I] bf16; G2: o [R, H] fp32
+    void *out;                // G1: h [R, I] bf16; G2: o [R, H] fp32 (bf16 when out_bf16)
     int E;
     int K;                    // reduction length (G1: H, G2: I)
     int M;                    // weight rows (G1: I, G2: H)
@@ -69,6 +69,7 @@ struct GemmParams {
     const int32_t *row_src;   // GATHER: dispatch row -> (token, slot) pair q; token = q / topk
     int topk;
     const int32_t *out_row;   // G2 only, nullable: dispatch row r is stored at output row out_row[r]
+    int out_bf16;             // G2 only: 1 stores the accumulators rounded to bf16 (RNE) instead of fp32
 };
 
 // Work-item decode from the per-CTA prefix table.
@@ -167,7 +168,12 @@ __device__ __forceinline__ void gemm_epilogue(int q, const int *tile_start, int 
                 }
             } else {
                 tmem_ld_wait();
-                if (m < p.M) {
+                if (m < p.M && p.out_bf16) {
+                    __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.out);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        if (c + j < it.n_valid) o[(it.row0 + c + j) * p.M + m] = __float2bfloat16_rn(__uint_as_float(r0[j]));
+                } else if (m < p.M) {
                     float *o = reinterpret_cast<float *>(p.out);
 #pragma unroll
                     for (int j = 0; j < 16; ++j)

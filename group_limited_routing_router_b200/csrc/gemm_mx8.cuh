@@ -8,7 +8,7 @@
 //   G1 (gate/up + SwiGLU): h[r, i] = SiLU(x~[r] . W_gate[e, i]) * (x~[r] . W_up[e, i]) in FP32,
 //        then h~ = MXFP8(h) per row: blocks of 32 consecutive i are the 32 lanes of one epilogue
 //        warp, so the block maximum is a warp reduction; codes h_q [R][I], scales h_s [R][I/32].
-//   G2 (down): o[r, j] = h~[r] . W_down[e, j]  (FP32)
+//   G2 (down): o[r, j] = h~[r] . W_down[e, j]  (FP32, stored bf16)
 //
 // Same work items, swap-AB orientation (weight rows on the MMA's M side, the expert's tokens on N),
 // accumulator slots and persistent grid as gemm.cuh.  Per stage K = 128 (one 128-byte row of E4M3
@@ -99,10 +99,10 @@ struct Mx8Params {
     const uint8_t *b_scale;
     int sf_token;
     // G1 outputs: h codes [R][M] (FP4: [R][M/2], two codes per byte) and scales [R][M/32] (FP4:
-    // [R][M/16]); G2 output: o [R][M] fp32
+    // [R][M/16]); G2 output: o [R][M] bf16
     uint8_t *h_q;
     uint8_t *h_s;
-    float *o;
+    __nv_bfloat16 *o;
     // FP4: FP32 scale per weight matrix [E] (g_a0: gate or down; g_a1: up) and per token [T]
     const float *g_a0;
     const float *g_a1;
@@ -296,6 +296,9 @@ __device__ __forceinline__ void nv4_epilogue_g1(int q, int half, const int *tile
         const uint32_t t1 = tmem_base + lane_off +
                             static_cast<uint32_t>(u == 2 ? s1 * SLOT_COLS : s0 * SLOT_COLS + SLOT_COLS / 2);
         for (int c = 16 * half; c < it.n_valid; c += 32) {
+            // lanes j and j + 16 load the token scale of column c + j; the loop below broadcasts it
+            const int jl = c + (lane & 15);
+            const float gt_l = jl < it.n_valid ? __ldg(p.g_tok + p.row_src[it.row0 + jl] / p.topk) : 0.0f;
             uint32_t rg[16], ru[16];
             tmem_ld16(t0 + c, rg);
             tmem_ld16(t1 + c, ru);
@@ -304,7 +307,7 @@ __device__ __forceinline__ void nv4_epilogue_g1(int q, int half, const int *tile
             for (int j = 0; j < 16; ++j) {
                 const bool col_ok = c + j < it.n_valid;
                 const int64_t r = it.row0 + c + j;
-                const float gt = col_ok ? __ldg(p.g_tok + p.row_src[r] / p.topk) : 0.0f;
+                const float gt = __shfl_sync(0xffffffffu, gt_l, j);
                 const float hv = row_ok && col_ok ? silu_mul(__uint_as_float(rg[j]) * (gg * gt),
                                                              __uint_as_float(ru[j]) * (gu * gt))
                                                   : 0.0f;
@@ -325,7 +328,8 @@ __device__ __forceinline__ void nv4_epilogue_g1(int q, int half, const int *tile
     }
 }
 
-// G2 epilogue: FP32 o rows in dispatch order (FP4: times the weight matrix's FP32 scale).
+// G2 epilogue: o rows in dispatch order, FP32 accumulators (FP4: times the weight matrix's FP32 scale)
+// rounded to bf16.
 template <int BN, int NSLOT, int SLOT_COLS, bool FP4>
 __device__ __forceinline__ void mx8_epilogue_g2(int q, int half, const int *tile_start, int total, const Mx8Params &p,
                                                 uint32_t tmem_base, uint64_t *acc_full, uint64_t *acc_empty) {
@@ -346,7 +350,8 @@ __device__ __forceinline__ void mx8_epilogue_g2(int q, int half, const int *tile
             if (m < p.M) {
 #pragma unroll
                 for (int j = 0; j < 16; ++j)
-                    if (c + j < it.n_valid) p.o[(it.row0 + c + j) * p.M + m] = __uint_as_float(r0[j]) * gd;
+                    if (c + j < it.n_valid)
+                        p.o[(it.row0 + c + j) * p.M + m] = __float2bfloat16_rn(__uint_as_float(r0[j]) * gd);
             }
         }
         tc_fence_before();
@@ -476,26 +481,48 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         // ---------------- scale-factor builder ----------------
         const int kbs = p.K / (FP4 ? 16 : 32);  // scale bytes per activation row
         constexpr int kRowIt = (BN + 31) / 32;
+        // B's scale words are loaded two stages ahead of the stage they belong to (a load cursor that
+        // runs over the same (item, kb) sequence), so their global-memory latency overlaps the
+        // building of the two stages before; each item's scale rows are looked up once.
+        int l_item = blockIdx.x, l_kb = 0;
+        int64_t l_srow[kRowIt];
+        auto l_rows = [&]() {
+            if (l_item >= total) return;
+            const Item li = decode_item(l_item, tile_start, E, BN, p.counts, p.offsets);
+#pragma unroll
+            for (int i = 0; i < kRowIt; ++i) {
+                const int n = lane + 32 * i;
+                const int64_t r = li.row0 + n;
+                l_srow[i] = n < li.n_valid ? (p.sf_token ? static_cast<int64_t>(p.row_src[r] / p.topk) : r) : -1;
+            }
+        };
+        // the stage's scale words of every row (FP8: one word = 4 K-blocks; FP4: four words, one per MMA)
+        auto l_next = [&](uint4 (&wb)[kRowIt]) {
+#pragma unroll
+            for (int i = 0; i < kRowIt; ++i) {
+                wb[i] = make_uint4(0u, 0u, 0u, 0u);
+                if (l_item < total && l_srow[i] >= 0) {
+                    if (FP4) wb[i] = __ldg(reinterpret_cast<const uint4 *>(p.b_scale + l_srow[i] * kbs + 16 * l_kb));
+                    else wb[i].x = __ldg(reinterpret_cast<const uint32_t *>(p.b_scale + l_srow[i] * kbs + 4 * l_kb));
+                }
+            }
+            if (++l_kb == n_kb) {
+                l_kb = 0;
+                l_item += gridDim.x;
+                l_rows();
+            }
+        };
+        l_rows();
+        uint4 wb[kRowIt], wb1[kRowIt];
+        l_next(wb);
+        l_next(wb1);
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
-            const Item it = decode_item(item, tile_start, E, BN, p.counts, p.offsets);
             for (int kb = 0; kb < n_kb && ok; ++kb) {
-                // B: the stage's scale words of every row (FP8: one word = 4 K-blocks; FP4: four words,
-                // one per MMA), loaded before the stage's data lands
-                uint4 wb[kRowIt];
-#pragma unroll
-                for (int i = 0; i < kRowIt; ++i) {
-                    const int n = lane + 32 * i;
-                    wb[i] = make_uint4(0u, 0u, 0u, 0u);
-                    if (n < it.n_valid) {
-                        const int64_t r = it.row0 + n;
-                        const int64_t srow = p.sf_token ? static_cast<int64_t>(p.row_src[r] / p.topk) : r;
-                        if (FP4) wb[i] = __ldg(reinterpret_cast<const uint4 *>(p.b_scale + srow * kbs + 16 * kb));
-                        else wb[i].x = __ldg(reinterpret_cast<const uint32_t *>(p.b_scale + srow * kbs + 4 * kb));
-                    }
-                }
+                uint4 wb2[kRowIt];
+                l_next(wb2);
                 ok = __all_sync(0xffffffffu, mbar_wait(&full[stage], phase, p.timeout));
                 if (!ok) break;
                 uint8_t *st = smem + stage * C::kStage;
@@ -534,6 +561,11 @@ __global__ void __launch_bounds__(kMxThreads, 1)
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sf_ready[stage]);
+#pragma unroll
+                for (int i = 0; i < kRowIt; ++i) {
+                    wb[i] = wb1[i];
+                    wb1[i] = wb2[i];
+                }
                 if (++stage == STAGES) {
                     stage = 0;
                     phase ^= 1u;

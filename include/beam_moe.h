@@ -295,8 +295,9 @@ BEAM_MOE_API int beam_moe_forward_nvfp4(const beam_moe_config *cfg, int64_t T, c
  * token and h per dispatch row, in blocks of 32 along the reduction axis, each block scaled by the
  * smallest power of two that brings its largest magnitude to <= 448, elements rounded to the
  * nearest E4M3 value (ties to even).  This is a reading (the pages give no FP8 recipe): results
- * differ from beam_moe_forward_fp8 (bf16 activations) by the activation rounding.  Requires hidden
- * and inter to be multiples of 128.  Workspace: beam_moe_workspace_size(cfg, T, BEAM_MOE_WS_MXFP8).
+ * differ from beam_moe_forward_fp8 (bf16 activations) by the activation rounding.  The expert
+ * outputs are kept in bf16 between the down projection and the combine (their 2^-9 relative rounding
+ * is far below the activations' own).  Requires hidden and inter to be multiples of 128.  Workspace: beam_moe_workspace_size(cfg, T, BEAM_MOE_WS_MXFP8).
  * Other arguments, outputs and error codes as beam_moe_experts_fp8 / beam_moe_forward_fp8
  * (`events`: NULL or 7 events recorded between the stages).
  */
@@ -317,7 +318,8 @@ BEAM_MOE_API int beam_moe_forward_mxfp8(const beam_moe_config *cfg, int64_t T, c
  * reduction axis, an E4M3 scale nearest to amax / (6 g) and E2M1 elements nearest to v / (s g)
  * (ties to even, saturating at 6).  This is a reading (the pages give no recipe): 4-bit activations
  * change the result by far more than the weights' rounding; beam_moe_forward_nvfp4 keeps bf16
- * activations.  Requires hidden and inter to be multiples of 256.  Workspace:
+ * activations.  Expert outputs in bf16 between the down projection and the combine, as for the
+ * MXFP8 path.  Requires hidden and inter to be multiples of 256.  Workspace:
  * beam_moe_workspace_size(cfg, T, BEAM_MOE_WS_W4A4).  Other arguments, outputs and error codes as
  * beam_moe_experts_nvfp4 / beam_moe_forward_nvfp4.
  */

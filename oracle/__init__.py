@@ -81,6 +81,13 @@ def lib():
         L.oracle_quant_nvfp4_rows.restype = ctypes.c_int
         L.oracle_expert_mlp_w4a4.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, _u16p, _dp, _dp, _dp, _dp]
         L.oracle_expert_mlp_w4a4.restype = ctypes.c_int
+        L.oracle_expert_mlp_w4a4_env.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, _u16p, _dp, _dp, _dp,
+                                                 ctypes.c_double, _dp, _dp]
+        L.oracle_expert_mlp_w4a4_env.restype = ctypes.c_int
+        L.oracle_quant_nvfp4_rows_alt.argtypes = [ctypes.c_int64, ctypes.c_int, _dp, ctypes.c_int,
+                                                  ctypes.POINTER(ctypes.c_uint8), ctypes.POINTER(ctypes.c_uint8), _dp,
+                                                  _dp, ctypes.c_double, _dp]
+        L.oracle_quant_nvfp4_rows_alt.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -395,32 +402,54 @@ def quant_nvfp4_rows(v: np.ndarray, per_row_scale: bool = True):
     return q, sc, g, deq
 
 
-def expert_mlp_w4a4(x_rows_bits: np.ndarray, wg: np.ndarray, wu: np.ndarray, wd: np.ndarray) -> np.ndarray:
+def quant_nvfp4_rows_alt(v: np.ndarray, per_row_scale: bool, eps: float) -> np.ndarray:
+    """For each element of quant_nvfp4_rows(v), the largest change of its dequantised value that a
+    quantiser deciding on values within eps (relative to the block) could legitimately make."""
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    rows, K = v.shape
+    g = np.empty(rows, dtype=np.float64)
+    deq = np.empty((rows, K), dtype=np.float64)
+    alt = np.empty((rows, K), dtype=np.float64)
+    if lib().oracle_quant_nvfp4_rows_alt(rows, K, _ptr(v, _dp), int(per_row_scale), None, None, _ptr(g, _dp),
+                                         _ptr(deq, _dp), float(eps), _ptr(alt, _dp)) != 0:
+        raise ValueError("NVFP4 activations: K not a multiple of 16")
+    return alt
+
+
+def expert_mlp_w4a4(x_rows_bits: np.ndarray, wg: np.ndarray, wu: np.ndarray, wd: np.ndarray, eps=None):
     """The 4-bit path's SwiGLU expert: NVFP4 x (per-row power-of-two scale), h quantised to NVFP4 (row
-    scale 1) before the down projection; FP64 weights (dequantised NVFP4).  Returns [n,H] fp64."""
+    scale 1) before the down projection; FP64 weights (dequantised NVFP4).  Returns [n,H] fp64; with
+    eps, also the envelope |W_d| alt(h) of quantisation decisions on h taken within eps of a boundary."""
     x_rows_bits = np.ascontiguousarray(x_rows_bits, dtype=np.uint16)
     n, H = x_rows_bits.shape
     I = wg.shape[0]
     assert wg.shape == (I, H) and wu.shape == (I, H) and wd.shape == (H, I)
     out = np.empty((n, H), dtype=np.float64)
-    if n == 0:
-        return out
-    if lib().oracle_expert_mlp_w4a4(n, H, I, _ptr(x_rows_bits, _u16p),
-                                    *(_ptr(np.ascontiguousarray(w, dtype=np.float64), _dp) for w in (wg, wu, wd)),
-                                    _ptr(out, _dp)) != 0:
+    env = np.zeros((n, H), dtype=np.float64) if eps is not None else None
+    if n > 0 and lib().oracle_expert_mlp_w4a4_env(
+            n, H, I, _ptr(x_rows_bits, _u16p),
+            *(_ptr(np.ascontiguousarray(w, dtype=np.float64), _dp) for w in (wg, wu, wd)),
+            float(eps or 0.0), _ptr(out, _dp), _ptr(env, _dp)) != 0:
         raise ValueError("4-bit expert: hidden and inter must be multiples of 16")
-    return out
+    return out if eps is None else (out, env)
 
 
 def experts_tokens_w4a4(x_bits: np.ndarray, ids: np.ndarray, weight: np.ndarray, fetch,
-                        n_experts: int, routed_scale: float) -> np.ndarray:
-    """experts_tokens of the 4-bit path (expert_mlp_w4a4 per expert; fetch gives FP64 weights)."""
+                        n_experts: int, routed_scale: float, eps=None):
+    """experts_tokens of the 4-bit path (expert_mlp_w4a4 per expert; fetch gives FP64 weights).  With
+    eps, returns (y, envelope of y): routed_scale * sum_j weight_j * envelope_j."""
     n, H = x_bits.shape
     k = ids.shape[1]
     out = np.zeros((n, k, H), dtype=np.float64)
+    env = np.zeros((n, k, H), dtype=np.float64) if eps is not None else None
     for e in range(n_experts):
         rows, slots = np.nonzero(ids == e)
         if rows.size == 0:
             continue
-        out[rows, slots, :] = expert_mlp_w4a4(x_bits[rows], *fetch(e))
-    return combine(out, weight, routed_scale)
+        r = expert_mlp_w4a4(x_bits[rows], *fetch(e), eps=eps)
+        if eps is None:
+            out[rows, slots, :] = r
+        else:
+            out[rows, slots, :], env[rows, slots, :] = r
+    y = combine(out, weight, routed_scale)
+    return y if eps is None else (y, combine(env, np.abs(weight), abs(routed_scale)))

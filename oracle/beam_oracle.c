@@ -661,8 +661,47 @@ static uint8_t e2m1_code_of(double v)  /* v already on the E2M1 grid */
     return (uint8_t)(s | ((e + 1) << 1) | mant);
 }
 
+/*
+ * alt (nullable): for each element, the largest change of its dequantised value that a decision taken
+ * on a value off by at most eps (relative) could make: the block's E4M3 scale rounded the other way
+ * (amax / (6 g) within eps of a rounding boundary) or the element's E2M1 code rounded the other way
+ * (v / (s g) within 6 eps of a boundary; the decision variable's error is relative to the block's
+ * largest element, 6 s g).  0 where no such decision is that close.  It bounds what a quantiser
+ * working on values within eps of these (FP32 ones, say) may legitimately give.
+ */
+static void nvfp4_block_alt(const double *blk, double g, double a, double s, double eps, double *alt)
+{
+    for (int i = 0; i < 16; ++i) {
+        const double m = s > 0.0 ? fabs(blk[i]) / (s * g) : 0.0;
+        const double q = s > 0.0 ? e2m1_round(m) : 0.0;
+        double d = 0.0;
+        if (s > 0.0) {
+            const double lo = e2m1_round(fmax(0.0, m - 6.0 * eps)), hi = e2m1_round(m + 6.0 * eps);
+            d = fmax(fabs(lo - q), fabs(hi - q)) * s * g;
+        }
+        /* the other scale: both E4M3 roundings of a within eps */
+        const double cand[2] = {e4m3_value(e4m3_round_code(fmin(a * (1.0 - eps), 448.0))),
+                                e4m3_value(e4m3_round_code(fmin(a * (1.0 + eps), 448.0)))};
+        for (int c = 0; c < 2; ++c) {
+            if (cand[c] == s) continue;
+            const double q2 = cand[c] > 0.0 ? e2m1_round(fabs(blk[i]) / (cand[c] * g)) : 0.0;
+            d = fmax(d, fabs(q2 * cand[c] - q * s) * g);
+        }
+        alt[i] = d;
+    }
+}
+
+int oracle_quant_nvfp4_rows_alt(int64_t rows, int K, const double *v, int per_row_scale, uint8_t *codes,
+                                uint8_t *scale, double *g_out, double *deq, double eps, double *alt);
+
 int oracle_quant_nvfp4_rows(int64_t rows, int K, const double *v, int per_row_scale, uint8_t *codes,
                             uint8_t *scale, double *g_out, double *deq)
+{
+    return oracle_quant_nvfp4_rows_alt(rows, K, v, per_row_scale, codes, scale, g_out, deq, 0.0, NULL);
+}
+
+int oracle_quant_nvfp4_rows_alt(int64_t rows, int K, const double *v, int per_row_scale, uint8_t *codes,
+                                uint8_t *scale, double *g_out, double *deq, double eps, double *alt)
 {
     if (K % 16) return -1;
     #pragma omp parallel for schedule(static)
@@ -698,6 +737,7 @@ int oracle_quant_nvfp4_rows(int64_t rows, int K, const double *v, int per_row_sc
                 if (codes) codes[r * K + kb * 16 + i] = e2m1_code_of(q);
                 deq[r * K + kb * 16 + i] = q * s * g;
             }
+            if (alt) nvfp4_block_alt(row + kb * 16, g, a, s, eps, alt + r * K + kb * 16);
         }
     }
     return 0;
@@ -710,8 +750,21 @@ int oracle_quant_nvfp4_rows(int64_t rows, int K, const double *v, int per_row_sc
  * quantised), out = Wd h~, FP64 on the dequantised values; weights FP64 (NVFP4 dequantised).
  * x_rows [n,H] bf16 bits; wg, wu [I,H]; wd [H,I]; out [n,H].
  */
+int oracle_expert_mlp_w4a4_env(int64_t n, int H, int I, const uint16_t *x_rows, const double *wg, const double *wu,
+                               const double *wd, double eps, double *out, double *env);
+
 int oracle_expert_mlp_w4a4(int64_t n, int H, int I, const uint16_t *x_rows, const double *wg, const double *wu,
                            const double *wd, double *out)
+{
+    return oracle_expert_mlp_w4a4_env(n, H, I, x_rows, wg, wu, wd, 0.0, out, NULL);
+}
+
+/*
+ * The same with the envelope env [n,H] (nullable): env[r][o] = sum_i |Wd[o,i]| alt_i, alt the largest
+ * legitimate change of h~_i (see oracle_quant_nvfp4_rows_alt) for decisions on values within eps.
+ */
+int oracle_expert_mlp_w4a4_env(int64_t n, int H, int I, const uint16_t *x_rows, const double *wg, const double *wu,
+                               const double *wd, double eps, double *out, double *env)
 {
     if (H % 16 || I % 16) return -1;
     const int64_t nb = (n + RB - 1) / RB;
@@ -741,19 +794,38 @@ int oracle_expert_mlp_w4a4(int64_t n, int H, int I, const uint16_t *x_rows, cons
                 hd[(b * RB + r) * I + i] = silu4 * u[r];
             }
         }
-    oracle_quant_nvfp4_rows(n, I, hd, 0, NULL, NULL, gh, h4);
+    double *halt = env ? (double *)malloc(sizeof(double) * (size_t)(n * I)) : NULL;
+    double *ab = env ? (double *)malloc(sizeof(double) * (size_t)(nb * I * RB)) : NULL;
+    oracle_quant_nvfp4_rows_alt(n, I, hd, 0, NULL, NULL, gh, h4, eps, halt);
+    if (env)
+        for (int64_t b = 0; b < nb; ++b)
+            for (int i = 0; i < I; ++i)
+                for (int r = 0; r < RB; ++r)
+                    ab[(b * I + i) * RB + r] = b * RB + r < n ? halt[(b * RB + r) * I + i] : 0.0;
     for (int64_t b = 0; b < nb; ++b)
         for (int i = 0; i < I; ++i)
             for (int r = 0; r < RB; ++r)
                 hb[(b * I + i) * RB + r] = b * RB + r < n ? h4[(b * RB + r) * I + i] : 0.0;
 
-    #pragma omp parallel for collapse(2) schedule(static)
-    for (int64_t b = 0; b < nb; ++b)
-        for (int o = 0; o < H; ++o) {
-            double acc[RB];
-            dot_rows(I, hb + b * I * RB, wd + (int64_t)o * I, acc);
-            for (int r = 0; r < RB && b * RB + r < n; ++r) out[(b * RB + r) * H + o] = acc[r];
-        }
+    #pragma omp parallel
+    {
+        double *wabs = env ? (double *)malloc(sizeof(double) * (size_t)I) : NULL;
+        #pragma omp for collapse(2) schedule(static)
+        for (int64_t b = 0; b < nb; ++b)
+            for (int o = 0; o < H; ++o) {
+                double acc[RB];
+                dot_rows(I, hb + b * I * RB, wd + (int64_t)o * I, acc);
+                for (int r = 0; r < RB && b * RB + r < n; ++r) out[(b * RB + r) * H + o] = acc[r];
+                if (env) {
+                    for (int i = 0; i < I; ++i) wabs[i] = fabs(wd[(int64_t)o * I + i]);
+                    dot_rows(I, ab + b * I * RB, wabs, acc);
+                    for (int r = 0; r < RB && b * RB + r < n; ++r) env[(b * RB + r) * H + o] = acc[r];
+                }
+            }
+        free(wabs);
+    }
+    free(halt);
+    free(ab);
     free(xd);
     free(x4);
     free(gx);

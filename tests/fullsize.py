@@ -26,6 +26,7 @@ import oracle
 from tests import parity
 
 SAMPLE = {"decode": None, "prefill": 512, "skew": 4096, "long": 4096}
+W4A4_EPS = 3e-5  # tolerance of the 4-bit path's near-boundary envelope (tests/test_gpu_w4a4.py)
 SAMPLE_LOWP = {"decode": None, "prefill": 256}
 FULL = ("decode", "prefill", "skew", "long")
 
@@ -111,8 +112,9 @@ class Bank:
         return y_of
 
     def oracle_y(self, fmt: str, name: str) -> np.ndarray:
-        """The oracle's outputs on the token sample of `name`, on the oracle's own routing.  The first
-        request of a format computes every workload of that format in one pass over the experts."""
+        """The oracle's outputs on the token sample of `name`, on the oracle's own routing (for "w4a4",
+        the pair (outputs, envelope)).  The first request of a format computes every workload of
+        that format in one pass over the experts."""
         key = (fmt, name)
         if key not in self._y:
             names = FULL if fmt == "bf16" else tuple(SAMPLE_LOWP)
@@ -130,7 +132,13 @@ class Bank:
             x = np.ascontiguousarray(np.concatenate(xs))
             run = _RUN[fmt]
             L = self.wl.layer
-            y = run(x, np.concatenate(ids), np.concatenate(ws), self.fetch(fmt), L["n_experts"], L["routed_scale"])
+            args = (x, np.concatenate(ids), np.concatenate(ws), self.fetch(fmt), L["n_experts"], L["routed_scale"])
+            if fmt == "w4a4":  # with the envelope of h's near-boundary quantisation decisions
+                y, env = run(*args, eps=W4A4_EPS)
+                for n, a, b in spans:
+                    self._y[(fmt, n)] = (y[a:b], env[a:b])
+                return self._y[key]
+            y = run(*args)
             for n, a, b in spans:
                 self._y[(fmt, n)] = y[a:b]
         return self._y[key]

@@ -5,8 +5,10 @@ expert (oracle.expert_mlp_w4a4: x quantised per token with a power-of-two scale,
 
 Protocol as for bf16 (tests/parity.py): routing bit-exact outside near-ties, outputs under compare_y.
 x's codes are decided identically on both sides (exact power-of-two scales, single roundings of
-bf16 values); h is quantised from FP32 values on the GPU and FP64 ones in the oracle, so an E2M1
-code can differ where the two straddle a rounding midpoint, which the output bound absorbs.
+bf16 values).  h is quantised from FP32 values on the GPU and from FP64 ones in the oracle: where an
+E2M1 code or a block's E4M3 scale is decided within EPS (relative to the block) of a rounding
+boundary, either result is correct, and the oracle's envelope of those alternatives (|W_down| times
+the change of h~, through the combine) is added to the bound as slack; its size is printed.
 """
 import numpy as np
 import pytest
@@ -18,6 +20,10 @@ import oracle
 from tests import fullsize, parity
 
 pytestmark = pytest.mark.gpu
+
+# relative error of the GPU's FP32 h (tensor-core FP32 accumulation over up to 5120 products, SwiGLU
+# in FP32) that the near-boundary envelope allows for
+EPS = 3e-5
 
 SMALL = ["mid_b", "mid_big_expert", "beam_small_T"]  # hidden, inter multiples of 256
 
@@ -31,9 +37,9 @@ class W4Case(parity.Case):
         return tuple(oracle.dequant_nvfp4(self.w4["q_" + n][e].cpu().numpy(), self.w4["s_" + n][e].cpu().numpy(),
                                           float(self.w4["g_" + n][e].cpu())) for n in ("gate", "up", "down"))
 
-    def oracle_y(self, ids, w, tokens):
+    def oracle_y(self, ids, w, tokens, eps=None):
         return oracle.experts_tokens_w4a4(np.ascontiguousarray(self.x_bits[tokens]), ids[tokens], w[tokens],
-                                          self.fetch64, self.layer["n_experts"], self.layer["routed_scale"])
+                                          self.fetch64, self.layer["n_experts"], self.layer["routed_scale"], eps)
 
 
 def _case(name, bank):
@@ -52,7 +58,8 @@ def test_w4a4_experts_small(name, bank):
     y = bm.experts_w4a4(case.layer, case.x, ids, w, case.w4)
     torch.cuda.synchronize()
     assert bm.device_status() == bm.OK
-    st = parity.compare_y(y.float().cpu().numpy(), case.oracle_y(r["ids"], r["weight"], np.arange(case.T)), name)
+    yo, env = case.oracle_y(r["ids"], r["weight"], np.arange(case.T), EPS)
+    st = parity.compare_y(y.float().cpu().numpy(), yo, name, slack=env)
     print(f"{name}: {st}")
 
 
@@ -67,8 +74,9 @@ def test_w4a4_forward_full_size(name, bank):
     r = case.oracle_route()
     st = parity.compare_routing(r, case.layer, ids, w, case.bias_np)
     tok = fullsize.sample(name, "w4a4")
-    yo = parity.oracle_y_checked(r, st, ids, tok, bank.oracle_y("w4a4", name), bank.y_of("w4a4", name))
-    print(f"{name}: {len(tok)} tokens: {parity.compare_y(y[tok], yo, name)}")
+    assert st["set_equal"][tok].all()  # (no near-tie tokens at decode/prefill: the envelope is per oracle set)
+    yo, env = bank.oracle_y("w4a4", name)
+    print(f"{name}: {len(tok)} tokens: {parity.compare_y(y[tok], yo, name, slack=env)}")
 
 
 def test_w4a4_deterministic_and_rejects_shapes(bank):

@@ -67,7 +67,7 @@ MUTANTS = {
     "e2m1_round_truncate": ("const double rounded = nearbyint(m / quantum) * quantum;",
                             "const double rounded = floor(m / quantum) * quantum;"),
     "nvfp4_act_scale_without_6": ("double a = amax / (6.0 * g);", "double a = amax / g;"),
-    "w4a4_h_row_scale": ("oracle_quant_nvfp4_rows(n, I, hd, 0,", "oracle_quant_nvfp4_rows(n, I, hd, 1,"),
+    "w4a4_h_row_scale": ("oracle_quant_nvfp4_rows_alt(n, I, hd, 0,", "oracle_quant_nvfp4_rows_alt(n, I, hd, 1,"),
     "w4a4_silu_missing": ("hd[(b * RB + r) * I + i] = silu4 * u[r];", "hd[(b * RB + r) * I + i] = g[r] * u[r];"),
     "expert_f64_silu_missing": ("const double act = g[r] / (1.0 + exp(-g[r]));", "const double act = g[r];"),
 }

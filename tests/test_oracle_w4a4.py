@@ -90,3 +90,20 @@ def test_expert_w4a4_matches_torch_float64_composition():
         hq, _ = _ref_quant(h, False)
         ref = hq @ wd.T
         np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+
+
+def test_alternative_quantisation_envelope():
+    """alt: 0 without tolerance; one E2M1 step at an element exactly on a rounding midpoint; the other
+    scale's dequantisation for a block whose amax/6 sits on an E4M3 midpoint; 0 far from boundaries."""
+    v = np.zeros((3, 16))
+    v[0, 0], v[0, 1], v[0, 2] = 6.0, 2.5, 1.1                  # scale 1: 2.5 is the midpoint of 2 and 3
+    v[1, 0], v[1, 1] = 6.0 * 1.0625, 1.0                        # amax / 6 = 1.0625: E4M3 midpoint of 1 and 1.125
+    v[2, 0], v[2, 1] = 6.0, 1.1                                 # nothing near a boundary
+    assert np.all(oracle.quant_nvfp4_rows_alt(v, False, 0.0) == 0.0)
+    alt = oracle.quant_nvfp4_rows_alt(v, False, 1e-6)
+    assert alt[0, 1] == 1.0 and alt[0, 2] == 0.0 and alt[0, 0] == 0.0
+    _, _, _, deq = oracle.quant_nvfp4_rows(v[1:2], False)
+    s_other = 1.125 if deq[0, 0] == 6.0 else 1.0                 # the scale not taken
+    q_other = _nearest_e2m1(np.minimum(np.abs(v[1]) / s_other, 6.0)) * s_other
+    np.testing.assert_allclose(alt[1], np.abs(q_other - deq[0]), rtol=0, atol=0)
+    assert np.all(alt[2] == 0.0)
