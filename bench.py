@@ -41,21 +41,28 @@ METRIC_MXFP8 = ("MoE-layer tokens/s (Beam shape, MXFP8 expert weights and activa
 METRIC_NVFP4 = "MoE-layer tokens/s (Beam shape, NVFP4 expert weights, T=4096) and % of tensor/HBM roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
-# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu capture of the
-# full-size launch, keyed by (kernel, workload).  An entry counts only while the sources it was
-# captured from hash the same; otherwise the JSON line reports null.
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant kernel, keyed by
+# (kernel, workload).  Taken with ncu on a 32-expert case with the same rows per expert as the workload
+# (decode: T=32, prefill: T=512, long: T=8192; one launch each) and scaled by 256/32 = 8 to the full
+# layer: each expert's weights and rows are its own traffic, so reads grow in proportion.  Writes of the
+# small case partly stay in the 126 MB L2, so the scaled figure understates full-size writes by up to
+# the kernel's output size.  An entry counts only while the sources it was captured from hash the same;
+# otherwise the JSON line reports null.
 _CSRC = os.path.join(ROOT, "group_limited_routing_router_b200", "csrc")
+_BF16_SRC = ("gemm.cuh", "common.cuh")
 NCU_TRAFFIC = {
-    ("gate_up_swiglu", "prefill"): {"bytes": 14067322368 + 151537152, "files": ("gemm.cuh", "common.cuh"),
-                                    "hash": "22b37ecce7f0f5cc"},
-    ("down", "prefill"): {"bytes": 7047173120 + 620304384, "files": ("gemm.cuh", "common.cuh"),
-                          "hash": "22b37ecce7f0f5cc"},
-    ("gate_up_swiglu_fp8", "prefill"): {"bytes": 8139558144 + 150100224,
-                                        "files": ("gemm_fp8.cuh", "gemm.cuh", "common.cuh"),
-                                        "hash": "f225f76d4d9105b4"},
-    ("down_fp8", "prefill"): {"bytes": 3970746368 + 618352896, "files": ("gemm_fp8.cuh", "gemm.cuh", "common.cuh"),
-                              "hash": "f225f76d4d9105b4"},
+    ("gate_up_swiglu", "decode"): {"bytes": 8 * (1678295040 + 1369856), "files": _BF16_SRC, "hash": "fbd3f5b6bb402249"},
+    ("gate_up_swiglu", "prefill"): {"bytes": 8 * (1724978688 + 2582016), "files": _BF16_SRC, "hash": "fbd3f5b6bb402249"},
+    ("gate_up_swiglu", "long"): {"bytes": 8 * (3484946688 + 326665216), "files": _BF16_SRC, "hash": "fbd3f5b6bb402249"},
+    ("down", "decode"): {"bytes": 8 * (840219392 + 3311616), "files": _BF16_SRC, "hash": "fbd3f5b6bb402249"},
+    ("down", "prefill"): {"bytes": 8 * (869167616 + 32409088), "files": _BF16_SRC, "hash": "fbd3f5b6bb402249"},
+    ("down", "long"): {"bytes": 8 * (1221652480 + 1301204736), "files": _BF16_SRC, "hash": "fbd3f5b6bb402249"},
 }
+
+
+def traffic_of(kernel, fmt, workload):
+    tr = NCU_TRAFFIC.get((kernel + ("" if fmt == "bf16" else "_" + fmt), workload))
+    return tr["bytes"] if tr and files_hash(tr["files"]) == tr["hash"] else None
 
 
 def files_hash(names) -> str:
@@ -584,8 +591,9 @@ def run_ours(args):
     clocks.cleanup()
 
     roofline = head["roofline"]
-    tr = NCU_TRAFFIC.get((roofline["kernel"] + ("" if fmt == "bf16" else "_" + fmt), wl.name))
-    roofline["traffic"] = tr["bytes"] if tr and files_hash(tr["files"]) == tr["hash"] else None
+    roofline["traffic"] = traffic_of(roofline["kernel"], fmt, wl.name)
+    for n in others:
+        others[n]["roofline"]["traffic"] = traffic_of(others[n]["roofline"]["kernel"], fmt, n)
     src_hash = kernel_source_hash()
 
     cpu = None

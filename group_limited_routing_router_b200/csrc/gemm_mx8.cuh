@@ -205,12 +205,15 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
 }
 
 // The NVFP4 block of 16 (row scale 1) of the value v held by each of 16 lanes (lanes 0..15 or 16..31):
-// returns this lane's E2M1 code and sets the block's E4M3 scale code.
+// returns this lane's E2M1 code and sets the block's E4M3 scale code.  The block scale is the E4M3
+// value nearest to amax / 6 and the element the E2M1 value nearest to v / s; both quotients are formed
+// with a multiply by a rounded reciprocal (within two FP32 ulp of the quotient), which moves a decision
+// only for values within that distance of a rounding boundary.
 __device__ __forceinline__ uint32_t nv4_quant16(float v, uint32_t half_mask, uint32_t &scale_code) {
     const float amax = __uint_as_float(__reduce_max_sync(half_mask, __float_as_uint(fabsf(v))));
-    scale_code = e4m3x2_from_f32(fminf(__fdiv_rn(amax, 6.0f), 448.0f), 0.0f) & 0xFFu;
+    scale_code = e4m3x2_from_f32(fminf(amax * (1.0f / 6.0f), 448.0f), 0.0f) & 0xFFu;
     const float s = e4m3_to_f32(scale_code);
-    return s > 0.0f ? (e2m1x2_from_f32(__fdiv_rn(v, s), 0.0f) & 0xFu) : 0u;
+    return s > 0.0f ? (e2m1x2_from_f32(v * __frcp_rn(s), 0.0f) & 0xFu) : 0u;
 }
 
 // G1 epilogue with MXFP8 h: the 32 lanes of warp q hold weight rows (i) 32q..32q+31 of the tile,
@@ -218,6 +221,7 @@ __device__ __forceinline__ uint32_t nv4_quant16(float v, uint32_t half_mask, uin
 template <int BN, int NSLOT, int SLOT_COLS>
 __device__ __forceinline__ void mx8_epilogue_g1(int q, int half, const int *tile_start, int total, const Mx8Params &p,
                                                 uint32_t tmem_base, uint64_t *acc_full, uint64_t *acc_empty) {
+    constexpr int kCh = (BN + 31) / 32;  // 16-column chunks of this warp (the quarter's two warps alternate)
     const int lane = threadIdx.x & 31;
     uint32_t uses = 0;
     for (int item = blockIdx.x; item < total; item += gridDim.x) {
@@ -239,23 +243,20 @@ __device__ __forceinline__ void mx8_epilogue_g1(int q, int half, const int *tile
         const uint32_t t0 = tmem_base + lane_off + static_cast<uint32_t>(s0 * SLOT_COLS);
         const uint32_t t1 = tmem_base + lane_off +
                             static_cast<uint32_t>(u == 2 ? s1 * SLOT_COLS : s0 * SLOT_COLS + SLOT_COLS / 2);
-        for (int c = 16 * half; c < it.n_valid; c += 32) {
-            uint32_t rg[16], ru[16];
-            tmem_ld16(t0 + c, rg);
-            tmem_ld16(t1 + c, ru);
-            tmem_ld_wait();
+        // SwiGLU of this warp's columns into registers; the accumulator slots go back to the MMA before
+        // the quantisation, so the next item's products overlap it
+        float hv[kCh][16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const float hv = row_ok ? silu_mul(__uint_as_float(rg[j]), __uint_as_float(ru[j])) : 0.0f;
-                // the block maximum: |h| >= 0, so its bit pattern orders like the value
-                const float amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(hv))));
-                float inv;
-                const uint32_t code = mx_scale_code(amax, inv);
-                if (c + j < it.n_valid && blk_ok) {
-                    const int64_t r = it.row0 + c + j;
-                    if (row_ok) p.h_q[r * p.M + m] = static_cast<uint8_t>(e4m3x2_from_f32(hv * inv, 0.0f) & 0xFFu);
-                    if (lane == 0) p.h_s[r * (p.M >> 5) + blk] = static_cast<uint8_t>(code);
-                }
+        for (int cc = 0; cc < kCh; ++cc) {
+            const int c = 16 * half + 32 * cc;
+            if (c < it.n_valid) {
+                uint32_t rg[16], ru[16];
+                tmem_ld16(t0 + c, rg);
+                tmem_ld16(t1 + c, ru);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 16; ++j)
+                    hv[cc][j] = row_ok ? silu_mul(__uint_as_float(rg[j]), __uint_as_float(ru[j])) : 0.0f;
             }
         }
         tc_fence_before();
@@ -263,6 +264,26 @@ __device__ __forceinline__ void mx8_epilogue_g1(int q, int half, const int *tile
         if (lane == 0)
             for (int i = 0; i < u; ++i) mbar_arrive(&acc_empty[(uses + i) % NSLOT]);
         uses += u;
+#pragma unroll
+        for (int cc = 0; cc < kCh; ++cc) {
+            const int c = 16 * half + 32 * cc;
+            if (c < it.n_valid) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    // the block maximum: |h| >= 0, so its bit pattern orders like the value
+                    const float amax =
+                        __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(hv[cc][j]))));
+                    float inv;
+                    const uint32_t code = mx_scale_code(amax, inv);
+                    if (c + j < it.n_valid && blk_ok) {
+                        const int64_t r = it.row0 + c + j;
+                        if (row_ok)
+                            p.h_q[r * p.M + m] = static_cast<uint8_t>(e4m3x2_from_f32(hv[cc][j] * inv, 0.0f) & 0xFFu);
+                        if (lane == 0) p.h_s[r * (p.M >> 5) + blk] = static_cast<uint8_t>(code);
+                    }
+                }
+            }
+        }
     }
 }
 
@@ -272,12 +293,22 @@ __device__ __forceinline__ void mx8_epilogue_g1(int q, int half, const int *tile
 template <int BN, int NSLOT, int SLOT_COLS>
 __device__ __forceinline__ void nv4_epilogue_g1(int q, int half, const int *tile_start, int total, const Mx8Params &p,
                                                 uint32_t tmem_base, uint64_t *acc_full, uint64_t *acc_empty) {
+    constexpr int kCh = (BN + 31) / 32;  // 16-column chunks of this warp (the quarter's two warps alternate)
     const int lane = threadIdx.x & 31;
     const uint32_t half_mask = lane < 16 ? 0x0000FFFFu : 0xFFFF0000u;
     uint32_t uses = 0;
     for (int item = blockIdx.x; item < total; item += gridDim.x) {
         const Item it = decode_item(item, tile_start, p.E, BN, p.counts, p.offsets);
         const int u = slots_of<true, SLOT_COLS>(it.n_mma);
+        // token scales of this warp's columns (lanes j and j + 16 hold column c + j), loaded before the
+        // accumulators are ready
+        float gtl[kCh];
+#pragma unroll
+        for (int cc = 0; cc < kCh; ++cc) {
+            const int jl = 16 * half + 32 * cc + (lane & 15);
+            gtl[cc] = jl < it.n_valid ? __ldg(p.g_tok + p.row_src[it.row0 + jl] / p.topk) : 0.0f;
+        }
+        const float gg = __ldg(p.g_a0 + it.e), gu = __ldg(p.g_a1 + it.e);
         bool ok = true;
         for (int i = 0; i < u && ok; ++i) {
             const uint32_t c = uses + i;
@@ -290,33 +321,27 @@ __device__ __forceinline__ void nv4_epilogue_g1(int q, int half, const int *tile
         const bool row_ok = m < p.M;
         const int blk = m >> 4;  // this lane's block of 16 along i
         const bool blk_ok = (blk << 4) < p.M;
-        const float gg = __ldg(p.g_a0 + it.e), gu = __ldg(p.g_a1 + it.e);
         const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
         const uint32_t t0 = tmem_base + lane_off + static_cast<uint32_t>(s0 * SLOT_COLS);
         const uint32_t t1 = tmem_base + lane_off +
                             static_cast<uint32_t>(u == 2 ? s1 * SLOT_COLS : s0 * SLOT_COLS + SLOT_COLS / 2);
-        for (int c = 16 * half; c < it.n_valid; c += 32) {
-            // lanes j and j + 16 load the token scale of column c + j; the loop below broadcasts it
-            const int jl = c + (lane & 15);
-            const float gt_l = jl < it.n_valid ? __ldg(p.g_tok + p.row_src[it.row0 + jl] / p.topk) : 0.0f;
-            uint32_t rg[16], ru[16];
-            tmem_ld16(t0 + c, rg);
-            tmem_ld16(t1 + c, ru);
-            tmem_ld_wait();
+        // SwiGLU of this warp's columns into registers; the accumulator slots go back to the MMA before
+        // the quantisation, so the next item's products overlap it
+        float hv[kCh][16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const bool col_ok = c + j < it.n_valid;
-                const int64_t r = it.row0 + c + j;
-                const float gt = __shfl_sync(0xffffffffu, gt_l, j);
-                const float hv = row_ok && col_ok ? silu_mul(__uint_as_float(rg[j]) * (gg * gt),
-                                                             __uint_as_float(ru[j]) * (gu * gt))
-                                                  : 0.0f;
-                uint32_t sc;
-                const uint32_t code = nv4_quant16(hv, half_mask, sc);
-                const uint32_t odd = __shfl_down_sync(0xffffffffu, code, 1);
-                if (col_ok && blk_ok) {
-                    if (row_ok && (lane & 1) == 0) p.h_q[r * (p.M >> 1) + (m >> 1)] = static_cast<uint8_t>(code | (odd << 4));
-                    if ((lane & 15) == 0) p.h_s[r * (p.M >> 4) + blk] = static_cast<uint8_t>(sc);
+        for (int cc = 0; cc < kCh; ++cc) {
+            const int c = 16 * half + 32 * cc;
+            if (c < it.n_valid) {
+                uint32_t rg[16], ru[16];
+                tmem_ld16(t0 + c, rg);
+                tmem_ld16(t1 + c, ru);
+                tmem_ld_wait();
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const float gt = __shfl_sync(0xffffffffu, gtl[cc], j);
+                    hv[cc][j] = row_ok && c + j < it.n_valid
+                                    ? silu_mul(__uint_as_float(rg[j]) * (gg * gt), __uint_as_float(ru[j]) * (gu * gt))
+                                    : 0.0f;
                 }
             }
         }
@@ -325,6 +350,24 @@ __device__ __forceinline__ void nv4_epilogue_g1(int q, int half, const int *tile
         if (lane == 0)
             for (int i = 0; i < u; ++i) mbar_arrive(&acc_empty[(uses + i) % NSLOT]);
         uses += u;
+#pragma unroll
+        for (int cc = 0; cc < kCh; ++cc) {
+            const int c = 16 * half + 32 * cc;
+            if (c < it.n_valid) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    uint32_t sc;
+                    const uint32_t code = nv4_quant16(hv[cc][j], half_mask, sc);
+                    const uint32_t odd = __shfl_down_sync(0xffffffffu, code, 1);
+                    if (c + j < it.n_valid && blk_ok) {
+                        const int64_t r = it.row0 + c + j;
+                        if (row_ok && (lane & 1) == 0)
+                            p.h_q[r * (p.M >> 1) + (m >> 1)] = static_cast<uint8_t>(code | (odd << 4));
+                        if ((lane & 15) == 0) p.h_s[r * (p.M >> 4) + blk] = static_cast<uint8_t>(sc);
+                    }
+                }
+            }
+        }
     }
 }
 
