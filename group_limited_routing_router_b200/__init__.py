@@ -34,7 +34,7 @@ ERR_DEVICE_TIMEOUT = 7
 ERR_BAD_INDEX = 8
 ERR_INVALID_ARG = 9
 
-WS_ROUTE, WS_PERMUTE, WS_EXPERTS, WS_FORWARD, WS_BLOCK, WS_MXFP8, WS_W4A4 = 0, 1, 2, 3, 4, 5, 6
+WS_ROUTE, WS_PERMUTE, WS_EXPERTS, WS_FORWARD, WS_BLOCK, WS_MXFP8, WS_W4A4, WS_ROUTE_SCREENED = 0, 1, 2, 3, 4, 5, 6, 7
 
 
 class BeamMoeConfig(ctypes.Structure):
@@ -99,6 +99,8 @@ def lib() -> ctypes.CDLL:
         L.beam_moe_workspace_size.argtypes = [_cfgp, ctypes.c_int64, ctypes.c_int]
         L.beam_moe_workspace_size.restype = ctypes.c_size_t
         L.beam_moe_route.argtypes = [_cfgp, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp, _vp]
+        L.beam_moe_route_screened.argtypes = [_cfgp, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t,
+                                              _vp]
         L.beam_moe_permute.argtypes = [_cfgp, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
         L.beam_moe_experts.argtypes = [_cfgp, ctypes.c_int64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                        ctypes.c_size_t, _vp]
@@ -227,6 +229,24 @@ def route(cfg, x: torch.Tensor, w_router: torch.Tensor, bias: Optional[torch.Ten
     _dev(w, "w", torch.float32, (T, c.topk))
     _check(lib().beam_moe_route(ctypes.byref(c), T, _ptr(x), _ptr(w_router), _ptr(bias), _ptr(ids), _ptr(w),
                                 _stream(stream)), "beam_moe_route")
+    return ids, w
+
+
+def route_screened(cfg, x: torch.Tensor, w_router: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                   ids: Optional[torch.Tensor] = None, w: Optional[torch.Tensor] = None, ws=None, stream=None):
+    """route() with the projection screened on the tensor cores (same outputs): (topk_ids, topk_w)."""
+    c = _cfg(cfg)
+    T = x.shape[0]
+    _dev(x, "x", torch.bfloat16, (T, c.hidden))
+    _dev(w_router, "w_router", torch.float32, (c.n_experts, c.hidden))
+    _dev(bias, "bias", torch.float32, (c.n_experts,))
+    ids = torch.empty(T, c.topk, dtype=torch.int32, device=x.device) if ids is None else ids
+    w = torch.empty(T, c.topk, dtype=torch.float32, device=x.device) if w is None else w
+    _dev(ids, "ids", torch.int32, (T, c.topk))
+    _dev(w, "w", torch.float32, (T, c.topk))
+    ws, nbytes = _workspace(c, T, WS_ROUTE_SCREENED, ws, x.device)
+    _check(lib().beam_moe_route_screened(ctypes.byref(c), T, _ptr(x), _ptr(w_router), _ptr(bias), _ptr(ids),
+                                         _ptr(w), _ptr(ws), nbytes, _stream(stream)), "beam_moe_route_screened")
     return ids, w
 
 

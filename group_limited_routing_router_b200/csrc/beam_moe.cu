@@ -23,6 +23,7 @@
 #include "gemm_mx8.cuh"
 #include "norm.cuh"
 #include "router.cuh"
+#include "router_tc.cuh"
 
 namespace beam {
 namespace {
@@ -129,6 +130,12 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
 std::once_flag g_encode_once;
 EncodeTiledFn g_encode = nullptr;
 
+template <int BN>
+bool set_router_tc_smem() {
+    return cudaFuncSetAttribute(router_logits_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                RsCfg<BN>::kSmem) == cudaSuccess;
+}
+
 int init_device(int *dev_out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return BEAM_MOE_ERR_CUDA;
@@ -150,7 +157,9 @@ int init_device(int *dev_out) {
         bool ok = cudaFuncSetAttribute(router_topk_kernel<kRtTok>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        rt_smem_bytes(kRtTok)) == cudaSuccess &&
                   cudaFuncSetAttribute(router_topk_kernel<kRtTokSmall>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       rt_smem_bytes(kRtTokSmall)) == cudaSuccess;
+                                       rt_smem_bytes(kRtTokSmall)) == cudaSuccess &&
+                  cudaFuncSetAttribute(router_topk_kernel<kRtTokTiny>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       rt_smem_bytes(kRtTokTiny)) == cudaSuccess;
         ok = ok && set_gemm_smem<G1_WIDE_ARGS>() && set_gemm_smem<G2_WIDE_ARGS>() &&
              set_gemm_smem<G1_NARROW_ARGS>() && set_gemm_smem<G2_NARROW_ARGS>();
         ok = ok && set_gemm_fp8_smem<G1_WIDE_FP8_ARGS>() && set_gemm_fp8_smem<G2_WIDE_FP8_ARGS>() &&
@@ -163,6 +172,9 @@ int init_device(int *dev_out) {
              set_gemm_mx8_smem<G1_NARROW_NV4X_ARGS>() && set_gemm_mx8_smem<G2_NARROW_NV4X_ARGS>();
         ok = ok && cudaFuncSetAttribute(combine_norm_residual_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         kMaxBlockHidden * 4) == cudaSuccess;
+        ok = ok && set_router_tc_smem<32>() && set_router_tc_smem<64>() && set_router_tc_smem<128>();
+        ok = ok && cudaFuncSetAttribute(router_exact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        kRsPathSmem) == cudaSuccess;
         if (!ok) d.status = BEAM_MOE_ERR_CUDA;
     });
     *dev_out = dev;
@@ -205,8 +217,51 @@ int check_T(const beam_moe_config *c, int64_t T) {
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
+// Screened router (router_tc.cuh) scratch: the three bf16 planes of W_r, the split partial projections,
+// the exact-path token list and its projections.  Pure host arithmetic: the split count aims at two
+// items per SM of a 148-SM B200 whatever device runs it, so the workspace size is device independent.
+struct RoutePlan {
+    bool ok = false;  // false: the configuration takes the direct router
+    int bn = 0, S = 0, kps = 0, n_nt = 0, n_mt = 0;
+    size_t planes = 0, part = 0, list = 0, list_n = 0, exact = 0, total = 0;
+};
+
+RoutePlan route_plan(const beam_moe_config *c, int64_t T) {
+    RoutePlan P;
+    // below ~2k tokens the direct router is faster: the screen's exact recomputation streams 8 rows of
+    // W_r per token either way, and the direct router's tiles already fill the GPU
+    if (T < kRsMinTokens || c->n_experts > kRtSlots || c->topk > 8 || c->n_groups > 32 || c->hidden % kBK) return P;
+    P.ok = true;
+    P.bn = T >= 2048 ? 128 : (T >= 512 ? 64 : 32);
+    P.n_nt = static_cast<int>((T + P.bn - 1) / P.bn);
+    P.n_mt = (c->n_experts + kBM - 1) / kBM;
+    const int nk = c->hidden / kBK;
+    P.S = 1;
+    for (int d = 1; d <= std::min(kRsMaxSplit, nk); ++d) {
+        if (nk % d) continue;
+        P.S = d;
+        if (static_cast<int64_t>(P.n_nt) * P.n_mt * d >= 2 * 148) break;
+    }
+    P.kps = nk / P.S;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = off;
+        off = align256(off + bytes);
+        return at;
+    };
+    const size_t E = c->n_experts, H = c->hidden;
+    P.planes = take(3 * E * H * 2);
+    P.part = take(static_cast<size_t>(P.S) * T * E * 4);
+    P.list = take(static_cast<size_t>(T) * 4);
+    P.list_n = take(4);
+    P.exact = take(static_cast<size_t>(T) * E * 4);
+    P.total = off;
+    return P;
+}
+
 struct Layout {
-    size_t u = 0, ids = 0, w = 0, hist = 0, counts = 0, offsets = 0, row_src = 0, dest_row = 0, xp = 0, h = 0, o = 0;
+    size_t u = 0, ids = 0, w = 0, rt = 0, hist = 0, counts = 0, offsets = 0, row_src = 0, dest_row = 0, xp = 0, h = 0,
+           o = 0;
     size_t total = 0;
 };
 
@@ -227,6 +282,7 @@ Layout layout(const beam_moe_config *c, int64_t T, int which) {
     if (which == BEAM_MOE_WS_FORWARD || which == BEAM_MOE_WS_BLOCK) {
         L.ids = take(R * 4);
         L.w = take(R * 4);
+        L.rt = take(route_plan(c, T).total);
     }
     L.hist = take(static_cast<size_t>(n_chunks(T)) * E * 4);
     if (which == BEAM_MOE_WS_PERMUTE) {
@@ -326,7 +382,7 @@ int enqueue_route(const beam_moe_config *c, int64_t T, const beam_bf16 *x, const
     // W_r tiles: 32 fp32 (one 128-byte swizzled row) x all 256 expert slots (rows >= E read as 0);
     // x tiles: 32 bf16 (64-byte swizzled row) x 64 tokens, or 16 for batches of at most 1024 tokens,
     // so that they still spread over most of the SMs (rows >= T read as 0)
-    const int tok = T <= 1024 ? kRtTokSmall : kRtTok;
+    const int tok = T <= 512 ? kRtTokTiny : (T <= 1024 ? kRtTokSmall : kRtTok);
     CUtensorMap m_w, m_x;
     if (!encode_fn()) return BEAM_MOE_ERR_CUDA;
     if (!make_map_2d_any(&m_w, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, w_router, c->hidden, c->n_experts, kRtBK, kRtSlots,
@@ -338,9 +394,53 @@ int enqueue_route(const beam_moe_config *c, int64_t T, const beam_bf16 *x, const
     if (tok == kRtTok)
         router_topk_kernel<kRtTok><<<static_cast<unsigned>(tiles * kRtCluster), kRtThreads, rt_smem_bytes(kRtTok), s>>>(
             m_w, m_x, p);
-    else
+    else if (tok == kRtTokSmall)
         router_topk_kernel<kRtTokSmall><<<static_cast<unsigned>(tiles * kRtCluster), kRtThreads,
                                           rt_smem_bytes(kRtTokSmall), s>>>(m_w, m_x, p);
+    else
+        router_topk_kernel<kRtTokTiny><<<static_cast<unsigned>(tiles * kRtCluster), kRtThreads,
+                                         rt_smem_bytes(kRtTokTiny), s>>>(m_w, m_x, p);
+    return launch_status();
+}
+
+// The routing of enqueue_route (bit for bit) through the screened router when the configuration fits
+// it and the caller's workspace holds its scratch (route_plan); the direct router otherwise.
+int enqueue_route_ws(const beam_moe_config *c, int dev, int64_t T, const beam_bf16 *x, const float *w_router,
+                     const float *bias, int32_t *ids, float *w, uint8_t *scratch, cudaStream_t s) {
+    const RoutePlan P = route_plan(c, T);
+    if (!P.ok || !scratch) return enqueue_route(c, T, x, w_router, bias, ids, w, s);
+    const int E = c->n_experts, H = c->hidden;
+    void *planes = scratch + P.planes;
+    float *part = reinterpret_cast<float *>(scratch + P.part);
+    int32_t *list = reinterpret_cast<int32_t *>(scratch + P.list);
+    int32_t *list_n = reinterpret_cast<int32_t *>(scratch + P.list_n);
+    float *exact = reinterpret_cast<float *>(scratch + P.exact);
+    const int sms = g_dev[dev].num_sms;
+    if (cudaMemsetAsync(list_n, 0, sizeof(int32_t), s) != cudaSuccess) return BEAM_MOE_ERR_CUDA;
+    const int64_t n4 = static_cast<int64_t>(E) * H / 4;
+    router_split_kernel<<<static_cast<unsigned>(std::min<int64_t>((n4 + 255) / 256, 4 * sms)), 256, 0, s>>>(
+        reinterpret_cast<const float4 *>(w_router), n4, reinterpret_cast<uint2 *>(planes));
+    int rc;
+    if ((rc = launch_status())) return rc;
+    CUtensorMap m_w, m_x;
+    if (!encode_fn() || !make_map_3d(&m_w, planes, H, E, 3) || !make_map_2d(&m_x, x, H, T, P.bn))
+        return BEAM_MOE_ERR_CUDA;
+    const RouterTcParams q{T, H, E, P.S, P.kps, P.n_nt, P.n_mt, part, kDefaultTimeoutCycles};
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(static_cast<int64_t>(P.n_nt) * P.n_mt * P.S, sms));
+    if (P.bn == 128) router_logits_kernel<128><<<grid, kRsThreads, RsCfg<128>::kSmem, s>>>(m_w, m_x, q);
+    else if (P.bn == 64) router_logits_kernel<64><<<grid, kRsThreads, RsCfg<64>::kSmem, s>>>(m_w, m_x, q);
+    else router_logits_kernel<32><<<grid, kRsThreads, RsCfg<32>::kSmem, s>>>(m_w, m_x, q);
+    if ((rc = launch_status())) return rc;
+    const RouterSelParams r{reinterpret_cast<const __nv_bfloat16 *>(x), w_router, bias, ids, w, T, H, E,
+                            c->n_groups, c->topk_groups, c->topk, c->group_topn, P.S, part, list, list_n, exact};
+    router_screen_kernel<<<static_cast<unsigned>((T + 7) / 8), 256, 0, s>>>(r);
+    if ((rc = launch_status())) return rc;
+    // the listed tokens' CTAs first (they start early and overlap the refinement), then one warp per token
+    const int n_chunk = (E + 31) / 32;
+    const int n_exact = n_chunk * static_cast<int>(std::min<int64_t>((T + 7) / 8, 64));
+    router_exact_kernel<<<static_cast<unsigned>(n_exact + (T + 7) / 8), 256, kRsPathSmem, s>>>(r, exact, n_exact);
+    if ((rc = launch_status())) return rc;
+    router_list_select_kernel<<<static_cast<unsigned>(std::min<int64_t>((T + 7) / 8, 2 * sms)), 256, 0, s>>>(r);
     return launch_status();
 }
 
@@ -474,7 +574,7 @@ int enqueue_experts(const beam_moe_config *c, int dev, int64_t T, const beam_bf1
 bool mx8_shape_ok(const beam_moe_config *c) { return c->hidden % 128 == 0 && c->inter % 128 == 0; }
 
 struct Mx8Layout {
-    size_t ids = 0, w = 0, hist = 0, counts = 0, offsets = 0, row_src = 0, dest_row = 0, xq = 0, xs = 0, xqp = 0,
+    size_t ids = 0, w = 0, rt = 0, hist = 0, counts = 0, offsets = 0, row_src = 0, dest_row = 0, xq = 0, xs = 0, xqp = 0,
            hq = 0, hs = 0, o = 0, total = 0;
 };
 
@@ -491,6 +591,7 @@ Mx8Layout mx8_layout(const beam_moe_config *c, int64_t T) {
     const size_t E = c->n_experts, H = c->hidden, I = c->inter;
     L.ids = take(R * 4);
     L.w = take(R * 4);
+    L.rt = take(route_plan(c, T).total);
     L.hist = take(static_cast<size_t>(n_chunks(T)) * E * 4);
     L.counts = take(E * 4);
     L.offsets = take((E + 1) * 8);
@@ -573,7 +674,7 @@ int enqueue_experts_mx8(const beam_moe_config *c, int dev, int64_t T, const beam
 bool w4a4_shape_ok(const beam_moe_config *c) { return c->hidden % 256 == 0 && c->inter % 256 == 0; }
 
 struct W4a4Layout {
-    size_t ids = 0, w = 0, hist = 0, counts = 0, offsets = 0, row_src = 0, dest_row = 0, xq = 0, xs = 0, gx = 0, xqp = 0,
+    size_t ids = 0, w = 0, rt = 0, hist = 0, counts = 0, offsets = 0, row_src = 0, dest_row = 0, xq = 0, xs = 0, gx = 0, xqp = 0,
            hq = 0, hs = 0, o = 0, total = 0;
 };
 
@@ -590,6 +691,7 @@ W4a4Layout w4a4_layout(const beam_moe_config *c, int64_t T) {
     const size_t E = c->n_experts, H = c->hidden, I = c->inter;
     L.ids = take(R * 4);
     L.w = take(R * 4);
+    L.rt = take(route_plan(c, T).total);
     L.hist = take(static_cast<size_t>(n_chunks(T)) * E * 4);
     L.counts = take(E * 4);
     L.offsets = take((E + 1) * 8);
@@ -688,9 +790,10 @@ extern "C" {
 
 size_t beam_moe_workspace_size(const beam_moe_config *cfg, int64_t T, int which) {
     if (validate(cfg) || check_T(cfg, T)) return 0;
-    if (which < BEAM_MOE_WS_ROUTE || which > BEAM_MOE_WS_W4A4) return 0;
+    if (which < BEAM_MOE_WS_ROUTE || which > BEAM_MOE_WS_ROUTE_SCREENED) return 0;
     if (which == BEAM_MOE_WS_MXFP8) return mx8_shape_ok(cfg) ? mx8_layout(cfg, T).total : 0;
     if (which == BEAM_MOE_WS_W4A4) return w4a4_shape_ok(cfg) ? w4a4_layout(cfg, T).total : 0;
+    if (which == BEAM_MOE_WS_ROUTE_SCREENED) return route_plan(cfg, T).total;
     return layout(cfg, T, which).total;
 }
 
@@ -705,6 +808,27 @@ int beam_moe_route(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, co
     int dev;
     if ((rc = init_device(&dev))) return rc;
     return enqueue_route(cfg, T, x, w_router, sel_bias, topk_ids, topk_w, static_cast<cudaStream_t>(stream));
+}
+
+int beam_moe_route_screened(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const float *w_router,
+                            const float *sel_bias, int32_t *topk_ids, float *topk_w, void *ws, size_t ws_bytes,
+                            void *stream) {
+    int rc = validate(cfg);
+    if (rc) return rc;
+    if ((rc = check_T(cfg, T))) return rc;
+    if (T == 0) return BEAM_MOE_OK;
+    if (!x || !w_router || !topk_ids || !topk_w) return BEAM_MOE_ERR_NULL;
+    if (!aligned16(x) || !aligned16(w_router)) return BEAM_MOE_ERR_MISALIGNED;
+    const RoutePlan P = route_plan(cfg, T);
+    if (P.ok) {
+        if (!ws) return BEAM_MOE_ERR_NULL;
+        if (!aligned16(ws)) return BEAM_MOE_ERR_MISALIGNED;
+        if (ws_bytes < P.total) return BEAM_MOE_ERR_WORKSPACE_TOO_SMALL;
+    }
+    int dev;
+    if ((rc = init_device(&dev))) return rc;
+    return enqueue_route_ws(cfg, dev, T, x, w_router, sel_bias, topk_ids, topk_w,
+                            P.ok ? static_cast<uint8_t *>(ws) : nullptr, static_cast<cudaStream_t>(stream));
 }
 
 int beam_moe_permute(const beam_moe_config *cfg, int64_t T, const int32_t *topk_ids, int32_t *counts,
@@ -795,7 +919,7 @@ int forward_impl(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, cons
     int32_t *ids = topk_ids_out ? topk_ids_out : reinterpret_cast<int32_t *>(wsb + L.ids);
     float *w = topk_w_out ? topk_w_out : reinterpret_cast<float *>(wsb + L.w);
     if (!record(ev, 0, s)) return BEAM_MOE_ERR_CUDA;
-    if ((rc = enqueue_route(cfg, T, x, w_router, sel_bias, ids, w, s))) return rc;
+    if ((rc = enqueue_route_ws(cfg, dev, T, x, w_router, sel_bias, ids, w, wsb + L.rt, s))) return rc;
     if (!record(ev, 1, s)) return BEAM_MOE_ERR_CUDA;
     return enqueue_experts(cfg, dev, T, x, ids, w, W, y, wsb, L, s, ev);
 }
@@ -909,7 +1033,7 @@ int beam_moe_forward_mxfp8(const beam_moe_config *cfg, int64_t T, const beam_bf1
     float *w = topk_w_out ? topk_w_out : reinterpret_cast<float *>(wsb + L.w);
     cudaEvent_t const *ev = reinterpret_cast<cudaEvent_t const *>(events);
     if (!record(ev, 0, s)) return BEAM_MOE_ERR_CUDA;
-    if ((rc = enqueue_route(cfg, T, x, w_router, sel_bias, ids, w, s))) return rc;
+    if ((rc = enqueue_route_ws(cfg, dev, T, x, w_router, sel_bias, ids, w, wsb + L.rt, s))) return rc;
     if (!record(ev, 1, s)) return BEAM_MOE_ERR_CUDA;
     return enqueue_experts_mx8(cfg, dev, T, x, ids, w, w8, y, wsb, L, s, ev);
 }
@@ -959,7 +1083,7 @@ int beam_moe_forward_w4a4(const beam_moe_config *cfg, int64_t T, const beam_bf16
     float *w = topk_w_out ? topk_w_out : reinterpret_cast<float *>(wsb + L.w);
     cudaEvent_t const *ev = reinterpret_cast<cudaEvent_t const *>(events);
     if (!record(ev, 0, s)) return BEAM_MOE_ERR_CUDA;
-    if ((rc = enqueue_route(cfg, T, x, w_router, sel_bias, ids, w, s))) return rc;
+    if ((rc = enqueue_route_ws(cfg, dev, T, x, w_router, sel_bias, ids, w, wsb + L.rt, s))) return rc;
     if (!record(ev, 1, s)) return BEAM_MOE_ERR_CUDA;
     return enqueue_experts_w4a4(cfg, dev, T, x, ids, w, w4, y, wsb, L, s, ev);
 }
@@ -1035,7 +1159,7 @@ extern "C" int beam_moe_block_forward(const beam_moe_config *cfg, const beam_moe
         reinterpret_cast<const uint4 *>(stream_in), sub->pre_norm_weight, sub->eps, cfg->hidden,
         reinterpret_cast<uint4 *>(u));
     if ((rc = launch_status())) return rc;
-    if ((rc = enqueue_route(cfg, T, u, w_router, sel_bias, ids, w, s))) return rc;
+    if ((rc = enqueue_route_ws(cfg, dev, T, u, w_router, sel_bias, ids, w, wsb + L.rt, s))) return rc;
     const double k = sub->step;
     const BlockTail tail{stream_in, sub->post_norm_weight, sub->eps, static_cast<float>(std::sqrt((k - 1.0) / k)),
                          static_cast<float>(1.0 / std::sqrt(k))};

@@ -30,6 +30,7 @@ namespace cg = cooperative_groups;
 
 constexpr int kRtTok = 64;        // tokens per cluster tile (kRtTokSmall for small batches)
 constexpr int kRtTokSmall = 16;
+constexpr int kRtTokTiny = 8;
 constexpr int kRtBK = 32;         // K per pipeline stage (one 128-byte row of fp32 W)
 constexpr int kRtThreads = 128;   // 4 warps
 constexpr int kRtCluster = 8;     // CTAs per cluster (split-K factor)
@@ -37,12 +38,13 @@ constexpr int kRtSlots = 256;     // expert slots per tile (E <= 256)
 constexpr int kRtStages = 3;      // TMA pipeline depth
 constexpr int kRtWBytes = kRtSlots * kRtBK * 4;  // W stage: [256 rows][32 fp32], 128-byte swizzle (32 KB)
 // x stage: [TOK rows][32 bf16], 64-byte swizzle (TOK * 64 bytes)
-constexpr int rt_stage_bytes(int tok) { return kRtWBytes + tok * kRtBK * 2; }
+constexpr int rt_stage_bytes(int tok) { return (kRtWBytes + tok * kRtBK * 2 + 1023) / 1024 * 1024; }
 // + alignment + barriers: two CTAs per SM
 constexpr int rt_smem_bytes(int tok) { return 1024 + kRtStages * rt_stage_bytes(tok) + 128; }
 static_assert(kRtTok * kRtSlots * 4 <= kRtStages * rt_stage_bytes(kRtTok), "partial logits must fit in the stages");
-static_assert(rt_stage_bytes(kRtTok) % 1024 == 0 && rt_stage_bytes(kRtTokSmall) % 1024 == 0,
+static_assert(rt_stage_bytes(kRtTok) % 1024 == 0 && rt_stage_bytes(kRtTokTiny) % 1024 == 0,
               "stages keep the 1024-byte swizzle alignment");
+static_assert(kRtTokTiny * kRtSlots * 4 <= kRtStages * rt_stage_bytes(kRtTokTiny), "partial logits fit");
 
 struct RouterParams {
     const __nv_bfloat16 *x;  // [T, H]
@@ -73,14 +75,174 @@ __device__ __forceinline__ ArgMax warp_argmax(float v, int i) {
     return {v, i};
 }
 
+// An order-preserving 32-bit key of a value that is not NaN (-inf lowest; -0.0 and +0.0 share a key),
+// and its inverse: warp max / min reductions (redux.sync) on keys rank values as float comparisons do.
+__device__ __forceinline__ uint32_t order_key(float v) {
+    const uint32_t b = __float_as_uint(v == 0.0f ? 0.0f : v);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_value(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// warp_argmax with two redux.sync reductions: the largest key, then the lowest index holding it.
+__device__ __forceinline__ ArgMax warp_argmax_redux(float v, int i) {
+    const uint32_t k = order_key(v);
+    const uint32_t kmax = __reduce_max_sync(0xffffffffu, k);
+    const uint32_t imin = __reduce_min_sync(0xffffffffu, k == kmax ? static_cast<uint32_t>(i) : 0xffffffffu);
+    return {key_value(kmax), static_cast<int>(imin)};
+}
+
 // Insert v into the descending pair (a1 >= a2).
 __device__ __forceinline__ void top2_insert(float &a1, float &a2, float v) {
     a2 = fmaxf(a2, fminf(a1, v));
     a1 = fmaxf(a1, v);
 }
 
-// TOK tokens per cluster tile: 64 (8 per thread), or 16 (2 per thread) so that small batches still
-// spread over most of the SMs.
+// Group-limited selection for one token, done by one warp.  Lane l holds the scores sc[j] and selection
+// values sel[j] (score + bias; -inf for masked or NaN) of experts l + 32 j.  On return lanes r < topk
+// hold the r-th pick (descending selection value, lower index first on ties): my_id and its score
+// my_s; den is the sum of the picked scores in pick order (every lane).  With margins != nullptr,
+// margins[0] = the last kept group's score - the best dropped group's score and margins[1] = the last
+// picked expert's selection value - the best one left in the kept groups (+inf where nothing is left;
+// NaN where only -inf values compete); every lane gets them.
+__device__ __forceinline__ void select_group_limited(const float (&sc)[8], const float (&sel)[8], int lane, int E,
+                                                     int G, int topk_groups, int topk, int group_topn, int &my_id,
+                                                     float &my_s, float &den, float *margins) {
+    const int per = E / G;
+#define EID(j) (lane + 32 * (j))
+    int grp[8];  // group of expert EID(j), -1 past E
+#pragma unroll
+    for (int j = 0; j < 8; ++j) grp[j] = EID(j) < E ? EID(j) / per : -1;
+    // ---- group scores (sum of the group's top group_topn selection values, in pick order) and the kept
+    // groups (topk_groups best, lower group index first on ties)
+    uint32_t kept = 0;
+    float last_gs = INFINITY, next_gs = -INFINITY;
+    if (group_topn == 2 && G <= 8) {
+        // all groups at once: lane-local top-2 per group, then a butterfly merge of the pairs (the
+        // top-2 of a union is the top-2 of the parts' top-2s; ties do not change the sum); every lane
+        // ends with every group's score and ranks the groups itself
+        float t1[8], t2[8];
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+            t1[g] = -INFINITY;
+            t2[g] = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (grp[j] == g) top2_insert(t1[g], t2[g], sel[j]);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+            for (int g = 0; g < 8; ++g) {
+                const float o1 = __shfl_xor_sync(0xffffffffu, t1[g], off);
+                const float o2 = __shfl_xor_sync(0xffffffffu, t2[g], off);
+                top2_insert(t1[g], t2[g], o1);
+                top2_insert(t1[g], t2[g], o2);
+            }
+        float gs[8];
+#pragma unroll
+        for (int g = 0; g < 8; ++g) gs[g] = t1[g] + t2[g];
+        for (int r = 0; r <= topk_groups && r < G; ++r) {
+            float bv = -INFINITY;
+            int bg = -1;
+#pragma unroll
+            for (int g = 0; g < 8; ++g)
+                if (g < G && !((kept >> g) & 1u) && (bg < 0 || gs[g] > bv)) {
+                    bv = gs[g];
+                    bg = g;
+                }
+            if (r == topk_groups) {
+                next_gs = bv;  // the best dropped group
+            } else {
+                kept |= 1u << bg;
+                last_gs = bv;
+            }
+        }
+    } else {
+        float my_gs = -INFINITY;  // lane g < G holds group g's score
+        uint32_t taken = 0;
+        for (int g = 0; g < G; ++g) {
+            float total = 0.0f;
+            for (int r = 0; r < group_topn; ++r) {
+                float bv = -INFINITY;
+                int bi = 0x7fffffff;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const bool cand = grp[j] == g && !((taken >> j) & 1u);
+                    if (cand && (sel[j] > bv || (sel[j] == bv && EID(j) < bi))) {
+                        bv = sel[j];
+                        bi = EID(j);
+                    }
+                }
+                const ArgMax m = warp_argmax_redux(bv, bi);
+                total = total + m.v;
+                if ((m.i & 31) == lane) taken |= 1u << (m.i >> 5);
+            }
+            if (lane == g) my_gs = total;
+        }
+        for (int r = 0; r <= topk_groups && r < G; ++r) {
+            const bool cand = lane < G && !((kept >> lane) & 1u);
+            const ArgMax m = warp_argmax_redux(cand ? my_gs : -INFINITY, cand ? lane : 0x7fffffff);
+            if (r == topk_groups) {
+                next_gs = m.v;
+            } else {
+                kept |= 1u << m.i;
+                last_gs = m.v;
+            }
+        }
+    }
+    if (margins) margins[0] = topk_groups < G ? last_gs - next_gs : INFINITY;
+    // ---- topk experts inside the kept groups, in pick order (descending selection value)
+    uint32_t taken = 0;
+    float last_sel = -INFINITY;
+    den = 0.0f;
+    my_s = 0.0f;
+    my_id = 0;
+    for (int r = 0; r < topk; ++r) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const bool cand = grp[j] >= 0 && !((taken >> j) & 1u) && ((kept >> grp[j]) & 1u);
+            if (cand && (sel[j] > bv || (sel[j] == bv && EID(j) < bi))) {
+                bv = sel[j];
+                bi = EID(j);
+            }
+        }
+        const ArgMax m = warp_argmax_redux(bv, bi);
+        float s_owner = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (j == (m.i >> 5)) s_owner = sc[j];
+        if ((m.i & 31) == lane) taken |= 1u << (m.i >> 5);
+        const float s = __shfl_sync(0xffffffffu, s_owner, m.i & 31);
+        den = den + s;
+        if (lane == r) {
+            my_id = m.i;
+            my_s = s;
+        }
+        last_sel = m.v;
+    }
+    if (margins) {
+        float bv = -INFINITY;
+        int bi = 0x7fffffff;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const bool cand = grp[j] >= 0 && !((taken >> j) & 1u) && ((kept >> grp[j]) & 1u);
+            if (cand && (sel[j] > bv || (sel[j] == bv && EID(j) < bi))) {
+                bv = sel[j];
+                bi = EID(j);
+            }
+        }
+        const ArgMax m = warp_argmax_redux(bv, bi);
+        margins[1] = m.i == 0x7fffffff ? INFINITY : last_sel - m.v;
+    }
+#undef EID
+}
+
+// TOK tokens per cluster tile: 64 (8 per thread), or 16 or 8 (2 or 1 per thread) so that small batches
+// still spread over most of the SMs.
 template <int TOK>
 __global__ void __cluster_dims__(kRtCluster, 1, 1) __launch_bounds__(kRtThreads, 2)
     router_topk_kernel(const __grid_constant__ CUtensorMap tm_w,  // W_r [E][H] fp32, box {32, 256}
@@ -88,7 +250,7 @@ __global__ void __cluster_dims__(kRtCluster, 1, 1) __launch_bounds__(kRtThreads,
                        const RouterParams p) {
     extern __shared__ uint8_t rt_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(rt_smem_raw) + 1023) & ~uintptr_t(1023));
-    constexpr int kRtStageBytes = rt_stage_bytes(TOK);
+    constexpr int kRtStageBytes = rt_stage_bytes(TOK);  // stage stride (1024-byte aligned)
     constexpr int kTi = TOK / 8;  // tokens per thread
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + kRtStages * kRtStageBytes);
     uint64_t *empty = full + kRtStages;
@@ -124,7 +286,7 @@ __global__ void __cluster_dims__(kRtCluster, 1, 1) __launch_bounds__(kRtThreads,
     auto issue = [&](int i) {  // load step s_begin + i into stage i % kRtStages
         uint8_t *st = smem + (i % kRtStages) * kRtStageBytes;
         const int k0 = (s_begin + i) * kRtBK;
-        mbar_arrive_expect_tx(&full[i % kRtStages], kRtStageBytes);
+        mbar_arrive_expect_tx(&full[i % kRtStages], kRtWBytes + TOK * kRtBK * 2);  // the bytes the two copies land
         tma_load_2d(st, &tm_w, &full[i % kRtStages], k0, 0, policy_evict_last());
         tma_load_2d(st + kRtWBytes, &tm_x, &full[i % kRtStages], k0, static_cast<int>(t0), policy_evict_first());
     };
@@ -204,7 +366,6 @@ __global__ void __cluster_dims__(kRtCluster, 1, 1) __launch_bounds__(kRtThreads,
 
     // ---- reduction over the cluster + selection: CTA rank takes tokens kTi*rank + [0, kTi), warp w
     // the tokens w and w + 4 among them
-    const int per = p.E / p.G;
 #define EID(j) (lane + 32 * (j))
     for (int u = 0; u < 2; ++u) {
         const int lt = warp + 4 * u;
@@ -226,94 +387,14 @@ __global__ void __cluster_dims__(kRtCluster, 1, 1) __launch_bounds__(kRtThreads,
             }
             const float s = 1.0f / (1.0f + expf(-logit));
             sc[j] = s;
-            const float v = p.bias ? s + p.bias[e] : s;
+            const float v = (p.bias && e < p.E) ? s + p.bias[e] : s;
             // a NaN (from NaN in x, W_r or the bias) ranks below every number, so the ids stay in [0, E)
             sel[j] = (e < p.E && v == v) ? v : -INFINITY;
         }
 
-        // group scores: sum of the group's top group_topn selection values, in pick order
-        float my_gs = -INFINITY;  // lane g < G holds group g's score
-        if (p.group_topn == 2 && p.G <= 8) {
-            // all groups at once: lane-local top-2 per group, then a butterfly merge of the pairs
-            // (the top-2 of a union is the top-2 of the parts' top-2s; ties do not change the sum)
-            float t1[8], t2[8];
-#pragma unroll
-            for (int g = 0; g < 8; ++g) {
-                t1[g] = -INFINITY;
-                t2[g] = -INFINITY;
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    if (EID(j) < p.E && EID(j) / per == g) top2_insert(t1[g], t2[g], sel[j]);
-            }
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1)
-#pragma unroll
-                for (int g = 0; g < 8; ++g) {
-                    const float o1 = __shfl_xor_sync(0xffffffffu, t1[g], off);
-                    const float o2 = __shfl_xor_sync(0xffffffffu, t2[g], off);
-                    top2_insert(t1[g], t2[g], o1);
-                    top2_insert(t1[g], t2[g], o2);
-                }
-#pragma unroll
-            for (int g = 0; g < 8; ++g)
-                if (lane == g && g < p.G) my_gs = t1[g] + t2[g];
-        } else {
-            uint32_t taken = 0;
-            for (int g = 0; g < p.G; ++g) {
-                float total = 0.0f;
-                for (int r = 0; r < p.group_topn; ++r) {
-                    float bv = -INFINITY;
-                    int bi = 0x7fffffff;
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const bool cand = EID(j) < p.E && !((taken >> j) & 1u) && (EID(j) / per) == g;
-                        if (cand && (sel[j] > bv || (sel[j] == bv && EID(j) < bi))) {
-                            bv = sel[j];
-                            bi = EID(j);
-                        }
-                    }
-                    const ArgMax m = warp_argmax(bv, bi);
-                    total = total + m.v;
-                    if ((m.i & 31) == lane) taken |= 1u << (m.i >> 5);
-                }
-                if (lane == g) my_gs = total;
-            }
-        }
-        // keep the topk_groups best groups (lower group index on ties)
-        uint32_t kept = 0;
-        for (int r = 0; r < p.topk_groups; ++r) {
-            const bool cand = lane < p.G && !((kept >> lane) & 1u);
-            const ArgMax m = warp_argmax(cand ? my_gs : -INFINITY, cand ? lane : 0x7fffffff);
-            kept |= 1u << m.i;
-        }
-        // topk experts inside the kept groups, in pick order (descending selection value)
-        uint32_t taken = 0;
-        float den = 0.0f, my_s = 0.0f;
-        int my_id = 0;
-        for (int r = 0; r < p.topk; ++r) {
-            float bv = -INFINITY;
-            int bi = 0x7fffffff;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const bool cand = EID(j) < p.E && !((taken >> j) & 1u) && ((kept >> (EID(j) / per)) & 1u);
-                if (cand && (sel[j] > bv || (sel[j] == bv && EID(j) < bi))) {
-                    bv = sel[j];
-                    bi = EID(j);
-                }
-            }
-            const ArgMax m = warp_argmax(bv, bi);
-            float s_owner = 0.0f;
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-                if (j == (m.i >> 5)) s_owner = sc[j];
-            if ((m.i & 31) == lane) taken |= 1u << (m.i >> 5);
-            const float s = __shfl_sync(0xffffffffu, s_owner, m.i & 31);
-            den = den + s;
-            if (lane == r) {
-                my_id = m.i;
-                my_s = s;
-            }
-        }
+        float den, my_s;
+        int my_id;
+        select_group_limited(sc, sel, lane, p.E, p.G, p.topk_groups, p.topk, p.group_topn, my_id, my_s, den, nullptr);
         if (lane < p.topk) {
             p.ids[t * p.topk + lane] = my_id;
             p.wts[t * p.topk + lane] = my_s / den;

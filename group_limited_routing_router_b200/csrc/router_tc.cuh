@@ -1,0 +1,594 @@
+// Screened router: the same routing as router_topk_kernel (bit for bit), with the 256-way projection
+// screened on the tensor cores.
+//
+// Beam launch post ("Welcome Beam" page, section "Mixture of Experts": sigmoid scores, 8 groups of 32,
+// the 4 groups with the best top-2 sums, the top 8 experts inside them, normalised weights; section
+// "Residual Stream": the router computes in FP32).  The FP32 router spends its time on the projection
+// x . W_r for all 256 experts, while only the 8 chosen experts' values enter the weights and only a
+// narrow band of values decides the choice.  So:
+//
+//   1. router_split_kernel: W_r (fp32) = W_hi + W_mid + W_lo exactly, three bf16 planes (each keeps
+//      the next 8 significant bits of the residual);
+//   2. router_logits_kernel: l~[t, e] = sum over the three planes of x_t . W_p,e on tcgen05 (bf16
+//      products are exact, accumulation in FP32 in the tensor core), K split S ways, partial sums
+//      written per split;
+//   3. router_screen_kernel (one warp per token): the selection on sigmoid(l~) with its two decision
+//      margins (last kept group vs best dropped group; last picked expert vs best one left).  Where
+//      both margins are at least kRsMargin, the chosen set is the one exact FP32 values give (the
+//      screened values are within 2e-5 of them, so a set decided by more than 4 times that cannot
+//      change).  Other tokens go to a list;
+//   4. router_exact_kernel, one launch: for each screened token (a warp each), the exact FP32
+//      projections of the chosen experts in the direct router's order (8 K ranges, each a sequential
+//      fused multiply-add chain over ascending k, summed in rank order), ordered and normalised as
+//      router_topk_kernel does; for the listed tokens (eight per CTA), every expert's exact projection
+//      in the same order;
+//   5. router_list_select_kernel: the selection on the listed tokens' projections, as in
+//      router_topk_kernel.
+// Every output therefore equals router_topk_kernel's.
+#pragma once
+
+#include "router.cuh"
+
+namespace beam {
+
+constexpr int kRsStages = 3;
+constexpr int kRsThreads = 192;      // warp 0 TMA, warp 1 MMA, warps 2..5 epilogue (TMEM lane quarters)
+constexpr float kRsMargin = 2e-4f;   // decision margin below which a token takes the exact path
+constexpr int kRsMaxSplit = 16;
+constexpr int kRsMinTokens = 2048;  // smaller batches take the direct router
+
+struct RouterTcParams {
+    int64_t T;
+    int H, E;
+    int S;          // K splits
+    int kps;        // 64-wide k-steps per split
+    int n_nt;       // token tiles
+    int n_mt;       // expert tiles of 128
+    float *part;    // [S][T][E] partial projections
+    long long timeout;
+};
+
+template <int BN>
+struct RsCfg {
+    static constexpr int kA = kBM * kBK * 2;    // one plane's expert tile: 128 rows x 64 bf16 (16 KB)
+    static constexpr int kB = BN * kBK * 2;     // token tile: BN rows x 64 bf16
+    static constexpr int kStage = 3 * kA + kB;
+    static constexpr int kBarOff = kRsStages * kStage;
+    static constexpr int kSmem = 1024 + kBarOff + 256;
+    static constexpr int kTmemCols = 2 * BN < 32 ? 32 : 2 * BN;  // two accumulator slots of BN columns
+    static_assert(kStage % 1024 == 0, "stages keep the 1024-byte swizzle alignment");
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
+    static_assert(kSmem <= 232448, "shared memory per CTA");
+};
+
+// W_r [E][H] fp32 -> planes [3][E][H] bf16 with hi + mid + lo == W_r (each residual is exact in FP32).
+__global__ void __launch_bounds__(256) router_split_kernel(const float4 *__restrict__ w, int64_t n4,
+                                                           uint2 *__restrict__ planes) {
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n4;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const float4 v = __ldg(w + i);
+        const float a[4] = {v.x, v.y, v.z, v.w};
+        uint32_t hi[2], mid[2], lo[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            float p0[2], p1[2], p2[2];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const float x0 = a[2 * h + q];
+                p0[q] = __bfloat162float(__float2bfloat16_rn(x0));
+                const float r1 = x0 - p0[q];
+                p1[q] = __bfloat162float(__float2bfloat16_rn(r1));
+                p2[q] = __bfloat162float(__float2bfloat16_rn(r1 - p1[q]));
+            }
+            hi[h] = pack_bf16x2(p0[0], p0[1]);
+            mid[h] = pack_bf16x2(p1[0], p1[1]);
+            lo[h] = pack_bf16x2(p2[0], p2[1]);
+        }
+        planes[i] = make_uint2(hi[0], hi[1]);
+        planes[n4 + i] = make_uint2(mid[0], mid[1]);
+        planes[2 * n4 + i] = make_uint2(lo[0], lo[1]);
+    }
+}
+
+// Screened projection: item = (token tile nt, expert tile mt, K split s); part[s][t][e] = sum over the
+// split's K range and the three planes, FP32 accumulation in TMEM.  Persistent CTAs, two accumulator
+// slots so an item's epilogue overlaps the next item's products.
+template <int BN>
+__global__ void __launch_bounds__(kRsThreads, 1)
+    router_logits_kernel(const __grid_constant__ CUtensorMap tm_w,  // planes [3][E][H] bf16, box {64, 128, 1}
+                         const __grid_constant__ CUtensorMap tm_x,  // x [T][H] bf16, box {64, BN}
+                         const RouterTcParams p) {
+    using C = RsCfg<BN>;
+    extern __shared__ uint8_t rs_smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(rs_smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
+    uint64_t *empty = full + kRsStages;
+    uint64_t *acc_full = empty + kRsStages;
+    uint64_t *acc_empty = acc_full + 2;
+    uint64_t *drain = acc_empty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int total = p.n_nt * p.n_mt * p.S;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kRsStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&acc_full[a], 1);
+            mbar_init(&acc_empty[a], 4);
+        }
+        mbar_init(drain, 1);
+        fence_mbar_init();
+        prefetch_tensormap(&tm_w);
+        prefetch_tensormap(&tm_x);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer ----------------
+            const uint64_t pol = policy_evict_last();  // planes and x are re-read by other items
+            int stage = 0;
+            uint32_t phase = 0, issued = 0, issued_phase = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+                const int s = item % p.S, mt = (item / p.S) % p.n_mt, nt = item / (p.S * p.n_mt);
+                for (int kb = 0; kb < p.kps; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, p.timeout)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *st = smem + stage * C::kStage;
+                    const int k0 = (s * p.kps + kb) * kBK;
+                    mbar_arrive_expect_tx(&full[stage], C::kStage);
+#pragma unroll
+                    for (int pl = 0; pl < 3; ++pl) tma_load_3d(st + pl * C::kA, &tm_w, &full[stage], k0, mt * kBM, pl, pol);
+                    tma_load_2d(st + 3 * C::kA, &tm_x, &full[stage], k0, nt * BN, pol);
+                    issued |= 1u << stage;
+                    issued_phase = (issued_phase & ~(1u << stage)) | (phase << stage);
+                    if (++stage == kRsStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            for (int s = 0; s < kRsStages; ++s)
+                if ((issued >> s) & 1u) mbar_wait(&full[s], (issued_phase >> s) & 1u, p.timeout);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer ----------------
+            const uint32_t idesc = umma_idesc_bf16(kBM, BN);
+            int stage = 0;
+            uint32_t phase = 0, uses = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+                const int slot = uses & 1;
+                if (!mbar_wait(&acc_empty[slot], ((uses >> 1) & 1u) ^ 1u, p.timeout)) break;
+                tc_fence_after();
+                const uint32_t d = tmem_base + static_cast<uint32_t>(slot * BN);
+                for (int kb = 0; kb < p.kps; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, p.timeout)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(smem + stage * C::kStage);
+                    const uint64_t db = umma_desc_sw128(sa + 3 * C::kA);
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk)
+#pragma unroll
+                        for (int pl = 0; pl < 3; ++pl) {
+                            const uint32_t accum = (kb > 0 || kk > 0 || pl > 0) ? 1u : 0u;
+                            umma_bf16(d, umma_desc_sw128(sa + pl * C::kA) + 2 * kk, db + 2 * kk, idesc, accum);
+                        }
+                    umma_commit(&empty[stage]);
+                    if (++stage == kRsStages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit(&acc_full[slot]);
+                ++uses;
+            }
+            umma_commit(drain);
+            mbar_wait(drain, 0, p.timeout);
+        }
+    } else {
+        // ---------------- epilogue: warp w reads TMEM lanes 32 (w % 4) .. + 31 ----------------
+        const int q = warp & 3;
+        uint32_t uses = 0;
+        for (int item = blockIdx.x; item < total; item += gridDim.x) {
+            const int s = item % p.S, mt = (item / p.S) % p.n_mt, nt = item / (p.S * p.n_mt);
+            const int slot = uses & 1;
+            if (!mbar_wait(&acc_full[slot], (uses >> 1) & 1u, p.timeout)) break;
+            tc_fence_after();
+            const int e = mt * kBM + q * 32 + lane;
+            const uint32_t t0 = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(slot * BN);
+            float *out = p.part + static_cast<int64_t>(s) * p.T * p.E;
+#pragma unroll 1
+            for (int c = 0; c < BN; c += 16) {
+                uint32_t r[16];
+                tmem_ld16(t0 + c, r);
+                tmem_ld_wait();
+                if (e < p.E) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int64_t t = static_cast<int64_t>(nt) * BN + c + j;
+                        if (t < p.T) out[t * p.E + e] = __uint_as_float(r[j]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[slot]);
+            ++uses;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+}
+
+// The direct router's K range of cluster rank r: 32-wide steps [r n / 8, (r + 1) n / 8), n = H / 32.
+__device__ __forceinline__ void rank_range(int H, int r, int &k0, int &k1) {
+    const int n = H / kRtBK;
+    k0 = (r * n / kRtCluster) * kRtBK;
+    k1 = ((r + 1) * n / kRtCluster) * kRtBK;
+}
+
+// ---- exact projections in router_topk_kernel's order -------------------------------------------------
+// The direct router forms logit_e = ((p_0 + p_1) + ...) + p_7 with p_r = fma(x_k, w_k, ...) over the
+// ascending k of rank r's range, from 0.  The kernels below keep exactly those chains; their operands
+// are staged through shared memory 32 k per rank at a time, with coalesced 16-byte cp.async copies
+// (double buffered), so each thread's chain reads its segment without uncoalesced global loads.
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+constexpr int kRsSegWords = 36;  // a 32-float segment padded to 36 words: 8 consecutive segments hit distinct banks
+constexpr int kRsXWords = 20;    // a 32-bf16 segment (16 words) padded to 20
+
+// 4 fused multiply-adds in k order: w (4 fp32) against x (4 bf16 in two words, low half first)
+__device__ __forceinline__ float fma4(float4 w, uint2 x, float acc) {
+    acc = fmaf(__uint_as_float(x.x << 16), w.x, acc);  // bf16 -> fp32: the bits move up 16 places (exact)
+    acc = fmaf(__uint_as_float(x.x & 0xffff0000u), w.y, acc);
+    acc = fmaf(__uint_as_float(x.y << 16), w.z, acc);
+    return fmaf(__uint_as_float(x.y & 0xffff0000u), w.w, acc);
+}
+
+__device__ __forceinline__ float4 lds_f4(const uint32_t *base, int word) {
+    return *reinterpret_cast<const float4 *>(base + word);
+}
+__device__ __forceinline__ uint2 lds_u2(const uint32_t *base, int word) {
+    return *reinterpret_cast<const uint2 *>(base + word);
+}
+
+struct RouterSelParams {
+    const __nv_bfloat16 *x;  // [T, H]
+    const float *w;          // [E, H]
+    const float *bias;       // [E] or nullptr
+    int32_t *ids;            // [T, k]
+    float *wts;              // [T, k]
+    int64_t T;
+    int H, E, G, topk_groups, topk, group_topn;
+    int S;                   // splits in part
+    const float *part;       // [S][T][E]
+    int32_t *list;           // [T] tokens for the exact path
+    int32_t *list_n;         // their count
+    const float *exact;      // [T][E] exact projections of the listed tokens (by list position)
+};
+
+// sigmoid score and selection value of expert e from its projection (as router_topk_kernel)
+__device__ __forceinline__ void score_of(float logit, int e, const RouterSelParams &p, float &sc, float &sel) {
+    const float s = 1.0f / (1.0f + expf(-logit));
+    sc = s;
+    const float v = (p.bias && e < p.E) ? s + p.bias[e] : s;
+    sel = (e < p.E && v == v) ? v : -INFINITY;
+}
+
+// One warp per token: the selection on the screened projections.  A token decided by both margins
+// keeps its picks in ids[t] (for router_refine_kernel); any other is listed for the exact path and
+// marked ids[t][0] = -1.
+__global__ void __launch_bounds__(256) router_screen_kernel(const RouterSelParams p) {
+    const int lane = threadIdx.x & 31;
+    const int64_t t = blockIdx.x * 8LL + (threadIdx.x >> 5);
+    if (t >= p.T) return;
+    float sc[8], sel[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int e = lane + 32 * j;
+        float l = 0.0f;
+        if (e < p.E) {
+            float v[kRsMaxSplit];
+#pragma unroll
+            for (int s = 0; s < kRsMaxSplit; ++s)  // issue every split's load before summing them in order
+                v[s] = s < p.S ? __ldg(p.part + (static_cast<int64_t>(s) * p.T + t) * p.E + e) : 0.0f;
+#pragma unroll
+            for (int s = 0; s < kRsMaxSplit; ++s)
+                if (s < p.S) l += v[s];
+        }
+        score_of(l, e, p, sc[j], sel[j]);
+    }
+    float den, my_s, margins[2];
+    int my_id;
+    select_group_limited(sc, sel, lane, p.E, p.G, p.topk_groups, p.topk, p.group_topn, my_id, my_s, den, margins);
+    const bool certain = margins[0] >= kRsMargin && margins[1] >= kRsMargin;  // NaN margins are not
+    if (!certain && lane == 0) p.list[atomicAdd(p.list_n, 1)] = static_cast<int32_t>(t);
+    if (lane < p.topk) p.ids[t * p.topk + lane] = certain ? my_id : -1;
+}
+
+// ---- exact path: one launch, two kinds of CTAs ------------------------------------------------------
+// The first kRsExactCtas-many CTAs (blockIdx.x < n_exact) project the listed tokens onto every expert,
+// eight tokens at a time (exact_batch); the rest refine the screened tokens, one warp per token
+// (refine_token).  Both stage their operands with an NS-deep cp.async ring.
+
+constexpr int kRsRefineStages = 3;
+constexpr int kRsRefineW = 64 * 32;                          // 64 segments of 32 fp32, 16-byte chunks XOR-swizzled
+constexpr int kRsRefineStage = kRsRefineW + 8 * kRsXWords;   // + x's eight rank segments (padded)
+constexpr int kRsRefineWarpWords = kRsRefineStages * kRsRefineStage;
+constexpr int kRsExactStages = 4;
+constexpr int kRsExactW = 256 * kRsSegWords, kRsExactX = 8 * 8 * kRsXWords, kRsExactBuf = kRsExactW + kRsExactX;
+constexpr int kRsExactWords = kRsExactStages * kRsExactBuf + 8 * 256;
+constexpr int kRsPathSmem = (8 * kRsRefineWarpWords > kRsExactWords ? 8 * kRsRefineWarpWords : kRsExactWords) * 4;
+static_assert(kRsPathSmem <= 232448, "shared memory per CTA");
+
+// One warp: the picks' exact projections of screened token t in the direct router's order (lane l runs
+// the chains of pick l / 4, ranks r0 = 2 (l % 4) and r0 + 1), then the order and the weights exactly as
+// the direct router.  Per 32-k step the warp stages the picks' eight rank segments of W_r (segment
+// (chain, lane), 16-byte chunk c stored at c ^ (lane % 8)) and x's eight rank segments.
+__device__ __forceinline__ void refine_token(const RouterSelParams &p, int64_t t, uint32_t *wbuf, int lane) {
+    const int my_id = lane < p.topk ? p.ids[t * p.topk + lane] : 0;
+    if (__shfl_sync(0xffffffffu, my_id, 0) < 0) return;  // listed for the exact path
+    int e_of[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) e_of[j] = __shfl_sync(0xffffffffu, my_id, j < p.topk ? j : 0);
+    const int pick = lane >> 2, r0 = 2 * (lane & 3);
+    const int e_pick = __shfl_sync(0xffffffffu, my_id, pick < p.topk ? pick : 0);
+    // rank ranges this lane touches: its W copies (ranks 2 (lane / 8) and + 1), its x copy (rank
+    // lane / 4) and its chains (r0, r0 + 1)
+    const int n_steps = (p.H / kRtBK + kRtCluster - 1) / kRtCluster;
+    int wk0[2], wlen[2], xk0, xlen, len0, len1;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+        int a, b;
+        rank_range(p.H, 2 * (lane >> 3) + c, a, b);
+        wk0[c] = a;
+        wlen[c] = b - a;
+    }
+    {
+        int a, b;
+        rank_range(p.H, lane >> 2, a, b);
+        xk0 = a;
+        xlen = b - a;
+        rank_range(p.H, r0, a, b);
+        len0 = b - a;
+        rank_range(p.H, r0 + 1, a, b);
+        len1 = b - a;
+    }
+    const __nv_bfloat16 *xr = p.x + t * p.H;
+    auto issue = [&](int st) {  // stage st into ring slot st % NS; always one commit group
+        if (st < n_steps) {
+            uint32_t *buf = wbuf + (st % kRsRefineStages) * kRsRefineStage;
+            // W: chunk i of this lane = pick i % 8, rank 2 (lane / 8) + i / 8, 16-byte part lane % 8
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const int j = i & 7, c = i >> 3, r = 2 * (lane >> 3) + c, part = lane & 7;
+                if (j < p.topk && 32 * st < wlen[c]) {
+                    const int seg = c * 32 + 4 * j + (r >> 1);
+                    cp_async16(smem_u32(buf + seg * 32 + 4 * (part ^ (seg & 7))),
+                               p.w + static_cast<int64_t>(e_of[j]) * p.H + wk0[c] + 32 * st + 4 * part);
+                }
+            }
+            // x: rank lane / 4, 16-byte part lane % 4
+            if (32 * st < xlen)
+                cp_async16(smem_u32(buf + kRsRefineW + (lane >> 2) * kRsXWords + 4 * (lane & 3)),
+                           xr + xk0 + 32 * st + 8 * (lane & 3));
+        }
+        cp_async_commit();
+    };
+    float part0 = 0.0f, part1 = 0.0f;
+#pragma unroll
+    for (int st = 0; st < kRsRefineStages - 1; ++st) issue(st);
+    for (int st = 0; st < n_steps; ++st) {
+        issue(st + kRsRefineStages - 1);
+        cp_async_wait<kRsRefineStages - 1>();
+        __syncwarp();
+        if (pick < p.topk) {
+            const uint32_t *cur = wbuf + (st % kRsRefineStages) * kRsRefineStage;
+            const uint32_t *w0 = cur + lane * 32, *w1 = cur + (32 + lane) * 32;
+            const uint32_t *x0 = cur + kRsRefineW + r0 * kRsXWords, *x1 = x0 + kRsXWords;
+            const bool on0 = 32 * st < len0, on1 = 32 * st < len1;
+#pragma unroll
+            for (int kk = 0; kk < 32; kk += 4) {
+                const int ch = 4 * ((kk >> 2) ^ (lane & 7));
+                if (on0) part0 = fma4(lds_f4(w0, ch), lds_u2(x0, kk / 2), part0);
+                if (on1) part1 = fma4(lds_f4(w1, ch), lds_u2(x1, kk / 2), part1);
+            }
+        }
+        __syncwarp();
+    }
+    cp_async_wait<0>();
+    // sum in rank order (every lane of the pick's group of four forms the same value)
+    float logit = 0.0f;
+#pragma unroll
+    for (int r = 0; r < kRtCluster; ++r) {
+        const float a = __shfl_sync(0xffffffffu, part0, (lane & ~3) | (r >> 1));
+        const float b = __shfl_sync(0xffffffffu, part1, (lane & ~3) | (r >> 1));
+        logit += (r & 1) ? b : a;
+    }
+    float s_p, sel_p;
+    score_of(logit, e_pick, p, s_p, sel_p);
+    // order the picks by (selection value desc, expert asc) and normalise in that order
+    float sv[8], ss[8];
+    int ev[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        sv[j] = __shfl_sync(0xffffffffu, sel_p, 4 * j);
+        ss[j] = __shfl_sync(0xffffffffu, s_p, 4 * j);
+        ev[j] = __shfl_sync(0xffffffffu, e_pick, 4 * j);
+    }
+    float s_slot = 0.0f, den = 0.0f;
+    int e_slot = 0;
+    for (int r = 0; r < p.topk; ++r) {  // slot r holds the pick with exactly r picks ahead of it
+        float s_r = 0.0f;
+        int e_r = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if (j >= p.topk) continue;
+            int ahead = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (i < p.topk && (sv[i] > sv[j] || (sv[i] == sv[j] && ev[i] < ev[j]))) ++ahead;
+            if (ahead == r) {
+                s_r = ss[j];
+                e_r = ev[j];
+            }
+        }
+        den = den + s_r;
+        if (lane == r) {
+            s_slot = s_r;
+            e_slot = e_r;
+        }
+    }
+    if (lane < p.topk) {
+        p.ids[t * p.topk + lane] = e_slot;
+        p.wts[t * p.topk + lane] = s_slot / den;
+    }
+}
+
+// One CTA: the exact projections of listed tokens 8 bt .. 8 bt + 7 onto experts e0 .. e0 + 31.  Thread
+// (e, r) runs rank r's chain of expert e for the eight tokens; per 32-k step the CTA stages the 256 W_r
+// segments ([e][r][36 words]) and the tokens' x segments ([token][r][20 words]).
+__device__ __forceinline__ void exact_batch(const RouterSelParams &p, float *exact, int n, int bt, int e0,
+                                            uint32_t *smem) {
+    float *partial = reinterpret_cast<float *>(smem + kRsExactStages * kRsExactBuf);  // [token][e][r]
+    const int tid = threadIdx.x, el = tid >> 3, r = tid & 7;
+    // rank ranges this thread touches: its W copies (rank (tid / 8) % 8), its x copy (rank (tid / 4) % 8)
+    // and its chain (rank tid % 8)
+    const int n_steps = (p.H / kRtBK + kRtCluster - 1) / kRtCluster;
+    int wk0, wlen, xk0, xlen, clen;
+    {
+        int a, b;
+        rank_range(p.H, (tid >> 3) & 7, a, b);
+        wk0 = a;
+        wlen = b - a;
+        rank_range(p.H, (tid >> 2) & 7, a, b);
+        xk0 = a;
+        xlen = b - a;
+        rank_range(p.H, r, a, b);
+        clen = b - a;
+    }
+    const int nt = min(8, n - 8 * bt);
+    auto issue = [&](int st) {
+        if (st < n_steps) {
+            uint32_t *buf = smem + (st % kRsExactStages) * kRsExactBuf;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {  // W: chunk q = tid + 256 i -> segment q / 8 = (e, r), part q % 8
+                const int q = tid + 256 * i, seg = q >> 3, part = q & 7, e = seg >> 3;
+                if (e0 + e < p.E && 32 * st < wlen)
+                    cp_async16(smem_u32(buf + seg * kRsSegWords + 4 * part),
+                               p.w + static_cast<int64_t>(e0 + e) * p.H + wk0 + 32 * st + 4 * part);
+            }
+            // x: token tid / 32, rank (tid / 4) % 8, part tid % 4
+            const int tk = tid >> 5, rr = (tid >> 2) & 7, part = tid & 3;
+            if (tk < nt && 32 * st < xlen)
+                cp_async16(smem_u32(buf + kRsExactW + (tk * 8 + rr) * kRsXWords + 4 * part),
+                           p.x + static_cast<int64_t>(p.list[8 * bt + tk]) * p.H + xk0 + 32 * st + 8 * part);
+        }
+        cp_async_commit();
+    };
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int st = 0; st < kRsExactStages - 1; ++st) issue(st);
+    for (int st = 0; st < n_steps; ++st) {
+        issue(st + kRsExactStages - 1);
+        cp_async_wait<kRsExactStages - 1>();
+        __syncthreads();
+        if (32 * st < clen) {
+            const uint32_t *cur = smem + (st % kRsExactStages) * kRsExactBuf;
+            const uint32_t *wseg = cur + tid * kRsSegWords;
+#pragma unroll
+            for (int kk = 0; kk < 32; kk += 4) {
+                const float4 w4 = lds_f4(wseg, kk);
+#pragma unroll
+                for (int tk = 0; tk < 8; ++tk)
+                    acc[tk] = fma4(w4, lds_u2(cur + kRsExactW + (tk * 8 + r) * kRsXWords, kk / 2), acc[tk]);
+            }
+        }
+        __syncthreads();
+    }
+    cp_async_wait<0>();
+#pragma unroll
+    for (int tk = 0; tk < 8; ++tk) partial[(tk * 32 + el) * 8 + r] = acc[tk];
+    __syncthreads();
+    {  // thread (token tid / 32, expert tid % 32): the ranks in order
+        const int tk = tid >> 5, e = tid & 31;
+        if (tk < nt && e0 + e < p.E) {
+            float l = 0.0f;
+#pragma unroll
+            for (int q = 0; q < kRtCluster; ++q) l += partial[(tk * 32 + e) * 8 + q];
+            exact[static_cast<int64_t>(8 * bt + tk) * p.E + e0 + e] = l;
+        }
+    }
+    __syncthreads();
+}
+
+// blockIdx.x < n_exact: exact_batch over (expert chunk blockIdx.x % n_chunk, batches blockIdx.x / n_chunk
+// + k n_exact / n_chunk); the rest: refine_token, one warp per token.
+__global__ void __launch_bounds__(256, 1) router_exact_kernel(const RouterSelParams p, float *exact, int n_exact) {
+    extern __shared__ __align__(16) uint32_t rs_path_smem[];
+    if (static_cast<int>(blockIdx.x) < n_exact) {
+        const int n = *p.list_n;
+        const int n_chunk = (p.E + 31) / 32, slots = n_exact / n_chunk;
+        const int chunk = blockIdx.x % n_chunk;
+        for (int bt = blockIdx.x / n_chunk; bt < (n + 7) / 8; bt += slots) exact_batch(p, exact, n, bt, 32 * chunk, rs_path_smem);
+        return;
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t = (blockIdx.x - n_exact) * 8LL + warp;
+    if (t < p.T) refine_token(p, t, rs_path_smem + warp * kRsRefineWarpWords, lane);
+}
+
+// The selection of router_topk_kernel on the listed tokens' exact projections: one warp per entry.
+__global__ void __launch_bounds__(256) router_list_select_kernel(const RouterSelParams p) {
+    const int lane = threadIdx.x & 31;
+    const int n = *p.list_n;
+    for (int i = blockIdx.x * 8 + (threadIdx.x >> 5); i < n; i += gridDim.x * 8) {
+        const int64_t t = p.list[i];
+        float sc[8], sel[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int e = lane + 32 * j;
+            score_of(e < p.E ? p.exact[static_cast<int64_t>(i) * p.E + e] : 0.0f, e, p, sc[j], sel[j]);
+        }
+        float den, my_s;
+        int my_id;
+        select_group_limited(sc, sel, lane, p.E, p.G, p.topk_groups, p.topk, p.group_topn, my_id, my_s, den, nullptr);
+        if (lane < p.topk) {
+            p.ids[t * p.topk + lane] = my_id;
+            p.wts[t * p.topk + lane] = my_s / den;
+        }
+    }
+}
+
+}  // namespace beam

@@ -82,7 +82,8 @@ enum {
     BEAM_MOE_WS_FORWARD = 3,
     BEAM_MOE_WS_BLOCK = 4,
     BEAM_MOE_WS_MXFP8 = 5, /* beam_moe_experts_mxfp8 and beam_moe_forward_mxfp8 */
-    BEAM_MOE_WS_W4A4 = 6   /* beam_moe_experts_w4a4 and beam_moe_forward_w4a4 */
+    BEAM_MOE_WS_W4A4 = 6,  /* beam_moe_experts_w4a4 and beam_moe_forward_w4a4 */
+    BEAM_MOE_WS_ROUTE_SCREENED = 7 /* beam_moe_route_screened */
 };
 
 /*
@@ -118,6 +119,26 @@ BEAM_MOE_API size_t beam_moe_workspace_size(const beam_moe_config *cfg, int64_t 
  */
 BEAM_MOE_API int beam_moe_route(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x, const float *w_router,
                    const float *sel_bias, int32_t *topk_ids, float *topk_w, void *stream);
+
+/*
+ * beam_moe_route with the projection screened on the tensor cores; the same outputs, bit for bit.
+ * W_r is split exactly into three bf16 planes and x . W_r is formed for every expert with tcgen05
+ * (exact products, FP32 accumulation); the selection on those values reports its two decision
+ * margins (last kept group vs best dropped group, last picked expert vs best one left).  A token
+ * whose margins are both at least 2e-4 keeps that set, and its picks' projections are recomputed in
+ * beam_moe_route's FP32 order (8 K ranges of sequential fused multiply-adds, summed in range order),
+ * then ordered and normalised as there; any other token (a near-tie, NaN or infinite input) is
+ * routed from its recomputed projections of every expert.  The screened values are within ~4e-5
+ * of the FP32 ones (measured on Beam-shaped inputs), a fifth of the smallest margin that keeps a set.
+ * The forward entry points route this way when the configuration fits (E <= 256, k <= 8, G <= 32);
+ * otherwise, and for beam_moe_route, the direct FP32 router runs.
+ *   Arguments as beam_moe_route, plus a workspace of beam_moe_workspace_size(cfg, T,
+ *   BEAM_MOE_WS_ROUTE_SCREENED) bytes (16-byte aligned).  A configuration outside those bounds runs
+ *   the direct router and needs no workspace.
+ */
+BEAM_MOE_API int beam_moe_route_screened(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x,
+                                         const float *w_router, const float *sel_bias, int32_t *topk_ids,
+                                         float *topk_w, void *ws, size_t ws_bytes, void *stream);
 
 /*
  * Token -> expert dispatch: stable grouping of the T*k (token, slot) pairs by expert (the pages

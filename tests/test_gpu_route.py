@@ -85,3 +85,57 @@ def test_route_hand_cases():
         import math
         s = [1.0 / (1.0 + math.exp(-c["logits"][e])) for e in c["expected_ids"]]
         np.testing.assert_allclose(w.cpu().numpy()[0], [v / sum(s) for v in s], rtol=0, atol=1e-6)
+
+
+# ---- screened router (tensor-core projection, exact FP32 recomputation of the picks): it must return
+# beam_moe_route's outputs bit for bit, near-ties and degenerate rows included
+
+
+def _same_routing(case, x=None):
+    x = case.x if x is None else x
+    a_ids, a_w = bm.route(case.layer, x, case.w_router, case.bias)
+    b_ids, b_w = bm.route_screened(case.layer, x, case.w_router, case.bias)
+    torch.cuda.synchronize()
+    assert bm.device_status() == bm.OK
+    assert torch.equal(a_ids, b_ids)
+    assert torch.equal(a_w.view(torch.int32), b_w.view(torch.int32))
+    return b_ids, b_w
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_screened_route_equals_direct_small(name, beam_weights):
+    wl = bs.get(name)
+    _same_routing(parity.Case(wl, weights=beam_weights if wl.expert_device == "cuda" else None))
+
+
+@pytest.mark.parametrize("name", ["decode", "prefill", "skew", "long"])
+def test_screened_route_equals_direct_full_size(name, bank):
+    case = bank.case(name)
+    ids, w = _same_routing(case)
+    # and against the oracle, as the direct router is
+    parity.compare_routing(case.oracle_route(), case.layer, ids.cpu().numpy(), w.cpu().numpy(), case.bias_np)
+
+
+def test_screened_route_ties_ragged_and_nan():
+    """Ragged token tiles; all-zero rows (every projection 0: all experts tie, the exact path decides);
+    duplicated rows; a NaN row (its ids stay valid, as in the direct router)."""
+    wl = bs.get("mid_b")
+    for T in (1, 31, 33, 63, 65, 129, 300):
+        case = parity.Case(wl, T=T)
+        x = case.x.clone()
+        x[::7] = 0
+        if T > 2:
+            x[1] = x[2]
+        if T > 5:
+            x[5, 3] = float("nan")
+        ids, _ = _same_routing(case, x)
+        assert int(ids.min()) >= 0 and int(ids.max()) < wl.n_experts
+
+
+def test_forward_routes_like_the_direct_router(bank):
+    case = bank.case("prefill")
+    _, ids, w = bm.forward(case.layer, case.x, case.w_router, case.bias, case.wg, case.wu, case.wd,
+                           return_routing=True)
+    a_ids, a_w = bm.route(case.layer, case.x, case.w_router, case.bias)
+    torch.cuda.synchronize()
+    assert torch.equal(ids, a_ids) and torch.equal(w.view(torch.int32), a_w.view(torch.int32))
