@@ -204,16 +204,27 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
     return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
 }
 
+// The E2M1 code (sign in bit 3) of the value nearest to v / s, ties to even, saturating at 6, for an
+// E4M3 scale s > 0, without dividing: the rounding boundaries between the E2M1 magnitudes (0.25,
+// 0.75, 1.25, 1.75, 2.5, 3.5, 5) times s are exact in FP32 (at most 3 + 4 significant bits), so
+// comparing |v| with them decides the rounding of the exact quotient.  A value on a boundary goes
+// to the even code: above the boundaries with an odd index only when equal.
+__device__ __forceinline__ uint32_t e2m1_code_of_quotient(float v, float s) {
+    const float m = fabsf(v);
+    uint32_t k = (m > 0.25f * s) + (m >= 0.75f * s) + (m > 1.25f * s) + (m >= 1.75f * s) + (m > 2.5f * s) +
+                 (m >= 3.5f * s) + (m > 5.0f * s);
+    return k | (v < 0.0f ? 8u : 0u);
+}
+
 // The NVFP4 block of 16 (row scale 1) of the value v held by each of 16 lanes (lanes 0..15 or 16..31):
 // returns this lane's E2M1 code and sets the block's E4M3 scale code.  The block scale is the E4M3
-// value nearest to amax / 6 and the element the E2M1 value nearest to v / s; both quotients are formed
-// with a multiply by a rounded reciprocal (within two FP32 ulp of the quotient), which moves a decision
-// only for values within that distance of a rounding boundary.
+// value nearest to amax / 6, formed as amax times a rounded 1/6 (within two FP32 ulp of the quotient,
+// which moves the decision only for values that close to an E4M3 rounding boundary).
 __device__ __forceinline__ uint32_t nv4_quant16(float v, uint32_t half_mask, uint32_t &scale_code) {
     const float amax = __uint_as_float(__reduce_max_sync(half_mask, __float_as_uint(fabsf(v))));
     scale_code = e4m3x2_from_f32(fminf(amax * (1.0f / 6.0f), 448.0f), 0.0f) & 0xFFu;
     const float s = e4m3_to_f32(scale_code);
-    return s > 0.0f ? (e2m1x2_from_f32(v * __frcp_rn(s), 0.0f) & 0xFu) : 0u;
+    return s > 0.0f ? e2m1_code_of_quotient(v, s) : 0u;
 }
 
 // G1 epilogue with MXFP8 h: the 32 lanes of warp q hold weight rows (i) 32q..32q+31 of the tile,
