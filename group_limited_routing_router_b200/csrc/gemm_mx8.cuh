@@ -73,7 +73,9 @@ struct Mx8GemmCfg {
     static constexpr int kTmemCols = 512;
     static constexpr int kBarOff = STAGES * kStage;
     static constexpr int kTokOff = kBarOff + 512 + 4 * (kPmMaxE + 1);
-    static constexpr int kSmem = 1024 + kTokOff + 4 * BN + 64;
+    static constexpr int kEpiOff = (kTokOff + 4 * BN + 15) / 16 * 16;  // gate/up epilogue: per-warp staging of h~
+    static constexpr int kEpiWarp = GATE_UP ? 16 * 32 + 16 * 2 : 0;     // 16 columns x (32 code bytes + 2 scale bytes)
+    static constexpr int kSmem = 1024 + kEpiOff + kMxEpiWarps * kEpiWarp + 64;
     static_assert(kA % 1024 == 0 && kB % 1024 == 0 && (GATHER || kBox % 1024 == 0), "swizzled tiles");
     static_assert(BN % BOXN == 0 && BN % 16 == 0 && BN <= 256, "token tile");
     static_assert(!GATHER || BOXN == 1, "gathered B rows: one-row boxes, four per instruction");
@@ -81,7 +83,7 @@ struct Mx8GemmCfg {
     static_assert(GATE_UP ? (BN <= SLOT_COLS && (NSLOT >= 2 || BN <= SLOT_COLS / 2)) : BN <= SLOT_COLS,
                   "an item must fit in its TMEM slots");
     static_assert((3 * STAGES + 2 * NSLOT + 1) * 8 + 4 <= 512, "barriers");
-    static_assert(kSmem <= 232448, "shared memory per CTA");
+    static_assert(kSmem + 256 <= 232448, "shared memory per CTA (dynamic + the kernel's static bytes)");
 };
 
 struct Mx8Params {
@@ -231,7 +233,8 @@ __device__ __forceinline__ uint32_t nv4_quant16(float v, uint32_t half_mask, uin
 // one block of 32 along i per token column.
 template <int BN, int NSLOT, int SLOT_COLS>
 __device__ __forceinline__ void mx8_epilogue_g1(int q, int half, const int *tile_start, int total, const Mx8Params &p,
-                                                uint32_t tmem_base, uint64_t *acc_full, uint64_t *acc_empty) {
+                                                uint32_t tmem_base, uint64_t *acc_full, uint64_t *acc_empty,
+                                                uint8_t *stg) {
     constexpr int kCh = (BN + 31) / 32;  // 16-column chunks of this warp (the quarter's two warps alternate)
     const int lane = threadIdx.x & 31;
     uint32_t uses = 0;
@@ -275,6 +278,8 @@ __device__ __forceinline__ void mx8_epilogue_g1(int q, int half, const int *tile
         if (lane == 0)
             for (int i = 0; i < u; ++i) mbar_arrive(&acc_empty[(uses + i) % NSLOT]);
         uses += u;
+        // the warp's 32 rows of a token column are 32 code bytes and one scale byte: staged in shared
+        // memory per 16 columns, then lane j writes column j's pieces (two 16-byte and one 1-byte store)
 #pragma unroll
         for (int cc = 0; cc < kCh; ++cc) {
             const int c = 16 * half + 32 * cc;
@@ -286,13 +291,21 @@ __device__ __forceinline__ void mx8_epilogue_g1(int q, int half, const int *tile
                         __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(fabsf(hv[cc][j]))));
                     float inv;
                     const uint32_t code = mx_scale_code(amax, inv);
-                    if (c + j < it.n_valid && blk_ok) {
-                        const int64_t r = it.row0 + c + j;
-                        if (row_ok)
-                            p.h_q[r * p.M + m] = static_cast<uint8_t>(e4m3x2_from_f32(hv[cc][j] * inv, 0.0f) & 0xFFu);
-                        if (lane == 0) p.h_s[r * (p.M >> 5) + blk] = static_cast<uint8_t>(code);
-                    }
+                    stg[32 * j + lane] = static_cast<uint8_t>(e4m3x2_from_f32(hv[cc][j] * inv, 0.0f) & 0xFFu);
+                    if (lane == 0) stg[512 + j] = static_cast<uint8_t>(code);
                 }
+                __syncwarp();
+                if (lane < 16 && c + lane < it.n_valid && blk_ok) {
+                    const int64_t r = it.row0 + c + lane;
+                    const int m0 = it.mt * kBM + q * 32;  // this warp's first row (a multiple of 32)
+                    if (m0 + 32 <= p.M) {
+                        uint4 *dst = reinterpret_cast<uint4 *>(p.h_q + r * p.M + m0);
+                        dst[0] = *reinterpret_cast<const uint4 *>(stg + 32 * lane);
+                        dst[1] = *reinterpret_cast<const uint4 *>(stg + 32 * lane + 16);
+                    }
+                    p.h_s[r * (p.M >> 5) + blk] = stg[512 + lane];
+                }
+                __syncwarp();
             }
         }
     }
@@ -303,7 +316,8 @@ __device__ __forceinline__ void mx8_epilogue_g1(int q, int half, const int *tile
 // Codes are packed two per byte (even i in the low nibble) by the even lanes.
 template <int BN, int NSLOT, int SLOT_COLS>
 __device__ __forceinline__ void nv4_epilogue_g1(int q, int half, const int *tile_start, int total, const Mx8Params &p,
-                                                uint32_t tmem_base, uint64_t *acc_full, uint64_t *acc_empty) {
+                                                uint32_t tmem_base, uint64_t *acc_full, uint64_t *acc_empty,
+                                                uint8_t *stg) {
     constexpr int kCh = (BN + 31) / 32;  // 16-column chunks of this warp (the quarter's two warps alternate)
     const int lane = threadIdx.x & 31;
     const uint32_t half_mask = lane < 16 ? 0x0000FFFFu : 0xFFFF0000u;
@@ -361,6 +375,8 @@ __device__ __forceinline__ void nv4_epilogue_g1(int q, int half, const int *tile
         if (lane == 0)
             for (int i = 0; i < u; ++i) mbar_arrive(&acc_empty[(uses + i) % NSLOT]);
         uses += u;
+        // the warp's 32 rows of a token column are 16 code bytes and 2 scale bytes: staged in shared
+        // memory per 16 columns, then lane j writes column j's pieces (one 16-byte and one 2-byte store)
 #pragma unroll
         for (int cc = 0; cc < kCh; ++cc) {
             const int c = 16 * half + 32 * cc;
@@ -370,13 +386,19 @@ __device__ __forceinline__ void nv4_epilogue_g1(int q, int half, const int *tile
                     uint32_t sc;
                     const uint32_t code = nv4_quant16(hv[cc][j], half_mask, sc);
                     const uint32_t odd = __shfl_down_sync(0xffffffffu, code, 1);
-                    if (c + j < it.n_valid && blk_ok) {
-                        const int64_t r = it.row0 + c + j;
-                        if (row_ok && (lane & 1) == 0)
-                            p.h_q[r * (p.M >> 1) + (m >> 1)] = static_cast<uint8_t>(code | (odd << 4));
-                        if ((lane & 15) == 0) p.h_s[r * (p.M >> 4) + blk] = static_cast<uint8_t>(sc);
-                    }
+                    if ((lane & 1) == 0) stg[16 * j + (lane >> 1)] = static_cast<uint8_t>(code | (odd << 4));
+                    if ((lane & 15) == 0) stg[256 + 2 * j + (lane >> 4)] = static_cast<uint8_t>(sc);
                 }
+                __syncwarp();
+                if (lane < 16 && c + lane < it.n_valid && row_ok && blk_ok) {
+                    const int64_t r = it.row0 + c + lane;
+                    const int m0 = it.mt * kBM + q * 32;  // this warp's first row (a multiple of 32)
+                    *reinterpret_cast<uint4 *>(p.h_q + r * (p.M >> 1) + (m0 >> 1)) =
+                        *reinterpret_cast<const uint4 *>(stg + 16 * lane);
+                    *reinterpret_cast<uint16_t *>(p.h_s + r * (p.M >> 4) + (m0 >> 4)) =
+                        *reinterpret_cast<const uint16_t *>(stg + 256 + 2 * lane);
+                }
+                __syncwarp();
             }
         }
     }
@@ -697,8 +719,11 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         }
     } else if (warp >= 4) {
         const int q = warp & 3, half = (warp - 4) >> 2;
-        if (GATE_UP && FP4) nv4_epilogue_g1<BN, NSLOT, SLOT_COLS>(q, half, tile_start, total, p, tmem_base, acc_full, acc_empty);
-        else if (GATE_UP) mx8_epilogue_g1<BN, NSLOT, SLOT_COLS>(q, half, tile_start, total, p, tmem_base, acc_full, acc_empty);
+        uint8_t *stg = smem + C::kEpiOff + (warp - 4) * C::kEpiWarp;
+        if (GATE_UP && FP4)
+            nv4_epilogue_g1<BN, NSLOT, SLOT_COLS>(q, half, tile_start, total, p, tmem_base, acc_full, acc_empty, stg);
+        else if (GATE_UP)
+            mx8_epilogue_g1<BN, NSLOT, SLOT_COLS>(q, half, tile_start, total, p, tmem_base, acc_full, acc_empty, stg);
         else mx8_epilogue_g2<BN, NSLOT, SLOT_COLS, FP4>(q, half, tile_start, total, p, tmem_base, acc_full, acc_empty);
     }
     tc_fence_before();
