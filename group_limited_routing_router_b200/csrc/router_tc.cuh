@@ -385,24 +385,31 @@ __device__ __forceinline__ void refine_token(const RouterSelParams &p, int64_t t
         rank_range(p.H, r0 + 1, a, b);
         len1 = b - a;
     }
-    const __nv_bfloat16 *xr = p.x + t * p.H;
+    // this lane's copy addresses, fixed over the steps: W chunk i = pick i % 8, rank 2 (lane / 8) + i / 8,
+    // 16-byte part lane % 8 (source row start and shared-memory offset); x: rank lane / 4, part lane % 4
+    const int part = lane & 7;
+    const float *wsrc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) wsrc[j] = p.w + static_cast<int64_t>(e_of[j]) * p.H + 4 * part;
+    uint32_t wdst[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int j = i & 7, c = i >> 3, seg = c * 32 + 4 * j + (lane >> 3);
+        wdst[i] = static_cast<uint32_t>((seg * 32 + 4 * (part ^ (seg & 7))) * 4);
+    }
+    const __nv_bfloat16 *xsrc = p.x + t * p.H + xk0 + 8 * (lane & 3);
+    const uint32_t xdst = static_cast<uint32_t>((kRsRefineW + (lane >> 2) * kRsXWords + 4 * (lane & 3)) * 4);
+    const uint32_t ring = smem_u32(wbuf);
     auto issue = [&](int st) {  // stage st into ring slot st % NS; always one commit group
         if (st < n_steps) {
-            uint32_t *buf = wbuf + (st % kRsRefineStages) * kRsRefineStage;
-            // W: chunk i of this lane = pick i % 8, rank 2 (lane / 8) + i / 8, 16-byte part lane % 8
+            const uint32_t buf = ring + static_cast<uint32_t>((st % kRsRefineStages) * kRsRefineStage * 4);
+            const int k = 32 * st;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const int j = i & 7, c = i >> 3, r = 2 * (lane >> 3) + c, part = lane & 7;
-                if (j < p.topk && 32 * st < wlen[c]) {
-                    const int seg = c * 32 + 4 * j + (r >> 1);
-                    cp_async16(smem_u32(buf + seg * 32 + 4 * (part ^ (seg & 7))),
-                               p.w + static_cast<int64_t>(e_of[j]) * p.H + wk0[c] + 32 * st + 4 * part);
-                }
+                const int j = i & 7, c = i >> 3;
+                if (j < p.topk && k < wlen[c]) cp_async16(buf + wdst[i], wsrc[j] + wk0[c] + k);
             }
-            // x: rank lane / 4, 16-byte part lane % 4
-            if (32 * st < xlen)
-                cp_async16(smem_u32(buf + kRsRefineW + (lane >> 2) * kRsXWords + 4 * (lane & 3)),
-                           xr + xk0 + 32 * st + 8 * (lane & 3));
+            if (k < xlen) cp_async16(buf + xdst, xsrc + k);
         }
         cp_async_commit();
     };
@@ -499,21 +506,28 @@ __device__ __forceinline__ void exact_batch(const RouterSelParams &p, float *exa
         clen = b - a;
     }
     const int nt = min(8, n - 8 * bt);
+    // this thread's copy addresses, fixed over the steps: W chunk q = tid + 256 i -> segment q / 8 (expert
+    // q / 64, rank (tid / 8) % 8), part tid % 8; x: token tid / 32, rank (tid / 4) % 8, part tid % 4
+    const int wpart = tid & 7, xtok = tid >> 5;
+    const uint32_t ring = smem_u32(smem);
+    const int64_t xrow = xtok < nt ? static_cast<int64_t>(p.list[8 * bt + xtok]) : 0;
+    const __nv_bfloat16 *xsrc = p.x + xrow * p.H + xk0 + 8 * (tid & 3);
+    const uint32_t xdst =
+        static_cast<uint32_t>((kRsExactW + (xtok * 8 + ((tid >> 2) & 7)) * kRsXWords + 4 * (tid & 3)) * 4);
     auto issue = [&](int st) {
         if (st < n_steps) {
-            uint32_t *buf = smem + (st % kRsExactStages) * kRsExactBuf;
+            const uint32_t buf = ring + static_cast<uint32_t>((st % kRsExactStages) * kRsExactBuf * 4);
+            const int k = 32 * st;
+            if (k < wlen) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {  // W: chunk q = tid + 256 i -> segment q / 8 = (e, r), part q % 8
-                const int q = tid + 256 * i, seg = q >> 3, part = q & 7, e = seg >> 3;
-                if (e0 + e < p.E && 32 * st < wlen)
-                    cp_async16(smem_u32(buf + seg * kRsSegWords + 4 * part),
-                               p.w + static_cast<int64_t>(e0 + e) * p.H + wk0 + 32 * st + 4 * part);
+                for (int i = 0; i < 8; ++i) {  // W: chunk q = tid + 256 i -> segment q / 8 = (e, r), part q % 8
+                    const int seg = (tid >> 3) + 32 * i, e = seg >> 3;
+                    if (e0 + e < p.E)
+                        cp_async16(buf + static_cast<uint32_t>((seg * kRsSegWords + 4 * wpart) * 4),
+                                   p.w + static_cast<int64_t>(e0 + e) * p.H + wk0 + k + 4 * wpart);
+                }
             }
-            // x: token tid / 32, rank (tid / 4) % 8, part tid % 4
-            const int tk = tid >> 5, rr = (tid >> 2) & 7, part = tid & 3;
-            if (tk < nt && 32 * st < xlen)
-                cp_async16(smem_u32(buf + kRsExactW + (tk * 8 + rr) * kRsXWords + 4 * part),
-                           p.x + static_cast<int64_t>(p.list[8 * bt + tk]) * p.H + xk0 + 32 * st + 8 * part);
+            if (xtok < nt && k < xlen) cp_async16(buf + xdst, xsrc + k);
         }
         cp_async_commit();
     };
