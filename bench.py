@@ -437,12 +437,18 @@ def roofline_of(wl, fmt, stage_ms, n_act, ms_step, pk, pk_kind):
     """Layer roofline and the dominant kernel's roofline (HBM GB/s or tensor TFLOP/s, whichever
     bounds it at this workload) from the measured stage times."""
     alg = algorithmic(wl, n_act, fmt)
-    t_tensor = alg["layer_flops"] / (pk["bf16_tflops"] * 1e12)
+    # the expert products run on the tensor cores at their own dtype's rate (nominal ratio to bf16:
+    # 2x for FP8, 4x for FP4 operands; the weight-only low-precision paths multiply in bf16); the router
+    # projection is counted at the bf16 rate
+    ratio = {"mxfp8": 2.0, "w4a4": 4.0}.get(fmt, 1.0)
+    router_flops = alg["stage_flops"]["router"]
+    t_tensor = (router_flops + (alg["layer_flops"] - router_flops) / ratio) / (pk["bf16_tflops"] * 1e12)
     t_hbm = alg["layer_bytes"] / (pk["hbm_gbs"] * 1e9)
     t_roof = max(t_tensor, t_hbm)
     layer = {"bound": "hbm" if t_hbm >= t_tensor else "tensor", "roofline_ms": t_roof * 1e3,
              "roofline_tokens_s": wl.T / t_roof, "frac": t_roof / (ms_step / 1e3),
-             "tensor_ms": t_tensor * 1e3, "hbm_ms": t_hbm * 1e3, "active_experts": n_act,
+             "tensor_ms": t_tensor * 1e3, "tensor_peak_ratio_to_bf16": ratio, "hbm_ms": t_hbm * 1e3,
+             "active_experts": n_act,
              "achieved_tflops": alg["layer_flops"] / (ms_step / 1e3) / 1e12,
              "achieved_gbs": alg["layer_bytes"] / (ms_step / 1e3) / 1e9}
     dom = max(stage_ms, key=stage_ms.get)
