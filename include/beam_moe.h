@@ -130,11 +130,12 @@ BEAM_MOE_API int beam_moe_route(const beam_moe_config *cfg, int64_t T, const bea
  * then ordered and normalised as there; any other token (a near-tie, NaN or infinite input) is
  * routed from its recomputed projections of every expert.  The screened values are within ~4e-5
  * of the FP32 ones (measured on Beam-shaped inputs), a fifth of the smallest margin that keeps a set.
- * The forward entry points route this way when the configuration fits (E <= 256, k <= 8, G <= 32);
- * otherwise, and for beam_moe_route, the direct FP32 router runs.
+ * The forward entry points route this way when the configuration fits (E <= 256, k <= 8, G <= 32)
+ * and T >= 2048 (below that the direct router is the faster one); otherwise, and for
+ * beam_moe_route, the direct FP32 router runs.
  *   Arguments as beam_moe_route, plus a workspace of beam_moe_workspace_size(cfg, T,
- *   BEAM_MOE_WS_ROUTE_SCREENED) bytes (16-byte aligned).  A configuration outside those bounds runs
- *   the direct router and needs no workspace.
+ *   BEAM_MOE_WS_ROUTE_SCREENED) bytes (16-byte aligned).  That size is 0 where the direct router runs
+ *   (T < 2048 or a configuration outside those bounds); ws may then be NULL.
  */
 BEAM_MOE_API int beam_moe_route_screened(const beam_moe_config *cfg, int64_t T, const beam_bf16 *x,
                                          const float *w_router, const float *sel_bias, int32_t *topk_ids,

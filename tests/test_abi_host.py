@@ -54,6 +54,20 @@ def test_workspace_sizes(L):
     assert bm.workspace_size(_cfg(hidden=100), 4, bm.WS_FORWARD) == 0
 
 
+def test_screened_route_workspace(L):
+    """The screened router's scratch: none below 2048 tokens (the direct router runs); from 2048 the
+    three bf16 planes of W_r, the split partial projections, the exact-path list and its projections,
+    and the forward workspace holds it."""
+    c = _cfg()
+    E, H = 256, 5120
+    assert bm.workspace_size(c, 2047, bm.WS_ROUTE_SCREENED) == 0
+    for T in (2048, 4096, 65536):
+        n = bm.workspace_size(c, T, bm.WS_ROUTE_SCREENED)
+        assert n >= 3 * E * H * 2 + T * E * 4 * 2 + T * 4  # planes + >= one split + exact projections + list
+        assert bm.workspace_size(c, T, bm.WS_FORWARD) > n
+    assert bm.workspace_size(_cfg(topk=9, topk_groups=8), 4096, bm.WS_ROUTE_SCREENED) == 0  # k > 8: direct
+
+
 @pytest.mark.parametrize("bad", [dict(hidden=96), dict(inter=0), dict(n_experts=257), dict(n_groups=3),
                                  dict(topk_groups=9), dict(topk=17), dict(topk=0), dict(group_topn=0),
                                  dict(group_topn=9), dict(n_groups=64, n_experts=256),
