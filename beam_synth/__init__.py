@@ -1,4 +1,4 @@
-"""Seeded synthetic inputs for the Beam MoE block (shared by the tests, the bench and the oracle driver).
+"""Seeded synthetic inputs for the Beam MoE block (shared by the tests, the bench and the oracle's callers).
 
 This module draws random numbers and nothing else: it holds none of the routing or expert arithmetic.
 Both the CUDA path and the CPU oracle read the tensors it returns; neither is imported here.

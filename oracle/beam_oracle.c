@@ -380,7 +380,7 @@ int oracle_scaled_residual(int64_t T, int H, const double *stream, const double 
 /*
  * FP8 expert weights ("Checkpoint formats: BF16, FP8, and NVFP4": "Welcome Beam" page, TL;DR; the
  * pages give no recipe).  Reading: the OCP MXFP8 layout, E4M3 elements with one power-of-two
- * (UE8M0) scale per 32 consecutive K elements of a weight row; this build stores the scales
+ * (UE8M0) scale per 32 consecutive K elements of a weight row; the scales are stored
  * K-block-major, scale[kb][row].
  *   E4M3: sign s, exponent e (4 bits, bias 7), mantissa m (3 bits); e = 15 with m = 7 is NaN;
  *         e = 0 is subnormal, m * 2^-9; otherwise (1 + m/8) * 2^(e-7).

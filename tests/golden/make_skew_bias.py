@@ -2,8 +2,8 @@
 
 The skewed workload asks for expert popularity that follows Zipf(1.1) over a seeded random
 permutation of the experts, with some experts that receive no token.  The pages never mention a
-router bias; this build reads the DeepSeek-V3 scheme the pages name as adding a per-expert bias
-to the sigmoid scores for selection only, and uses that bias to shape the load.
+router bias; the reading taken here is the DeepSeek-V3 scheme the pages name, a per-expert bias added
+to the sigmoid scores for selection only, and that bias shapes the load.
 
 Recipe (uses only the CPU oracle and the seeded input generator):
   1. draw a separate calibration batch x_cal (seed offset 77, T_cal tokens) and the workload's W_r;
