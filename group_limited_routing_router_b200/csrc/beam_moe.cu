@@ -32,15 +32,21 @@ constexpr int kMaxDevices = 64;
 constexpr int kMaxBlockHidden = 32768;  // the block's FP32 output row stays in shared memory
 constexpr int64_t kMaxTokens = int64_t(1) << 24;
 
-// ---- GEMM variants: <gate/up?, BN, B box rows, smem stages, TMEM slots, slot columns, gather?> -----
+// ---- GEMM variants: <gate/up?, BN, B box rows, smem stages, TMEM slots, slot columns, gather?,
+// weight-row pairs?> -----
 // "wide": experts see up to ~190 tokens per tile (prefill): the dispatch also gathers x into
 // dispatch order (x_perm) and both GEMMs read their token rows with tiled 64-row TMA boxes.
 // "narrow": a few tokens per expert (decode): the gate/up GEMM gathers its rows straight from x
 // with TMA gather4 (four rows per instruction; cheap when an expert has a handful of tokens).
-#define G1_WIDE_ARGS true, 192, 64, 4, 2, 256, false
-#define G2_WIDE_ARGS false, 192, 64, 5, 2, 256, false
-#define G1_NARROW_ARGS true, 32, 1, 6, 4, 64, true
-#define G2_NARROW_ARGS false, 32, 32, 10, 4, 32, false
+#define G1_WIDE_ARGS true, 192, 64, 4, 2, 256, false, false
+#define G2_WIDE_ARGS false, 192, 64, 5, 2, 256, false, false
+// "pair": the down projection with two 128-row weight tiles per token tile.  Half the token-row bytes
+// per weight byte, but an item then fills both TMEM slots whenever it has more than 128 tokens, so
+// its epilogue is not overlapped with the next item's products: used where every expert fits one
+// token tile (the weights are read once) and for the dense MLP (K = 20480 makes the epilogue small).
+#define G2_PAIR_ARGS false, 192, 64, 4, 2, 256, false, true
+#define G1_NARROW_ARGS true, 32, 1, 6, 4, 64, true, false
+#define G2_NARROW_ARGS false, 32, 32, 10, 4, 32, false, false
 // FP8 variants: <gate/up?, BN, B box rows, weight stages (K = 128), B stages (K = 64), TMEM slots,
 // slot columns, gather?, bf16 A ring stages in TMEM>.  The A ring takes the TMEM columns the
 // accumulators leave; the prefill gate/up variant gives its accumulators 2 slots of 192 columns
@@ -69,11 +75,11 @@ constexpr int64_t kMaxTokens = int64_t(1) << 24;
 #define G2_NARROW_NV4X_ARGS false, 32, 32, 8, 4, 32, false, true
 constexpr int kWideBN = 192, kWideBox = 64, kNarrowBN = 32, kNarrowBox = 32;
 
-template <bool G, int BN, int BOXN, int ST, int NS, int SC, bool GA>
+template <bool G, int BN, int BOXN, int ST, int NS, int SC, bool GA, bool PR>
 bool set_gemm_smem() {
-    return cudaFuncSetAttribute(grouped_gemm_kernel<G, BN, BOXN, ST, NS, SC, GA>,
+    return cudaFuncSetAttribute(grouped_gemm_kernel<G, BN, BOXN, ST, NS, SC, GA, PR>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                GemmCfg<G, BN, BOXN, ST, NS, SC, GA>::kSmem) == cudaSuccess;
+                                GemmCfg<G, BN, BOXN, ST, NS, SC, GA, PR>::kSmem) == cudaSuccess;
 }
 template <bool G, int BN, int BOXN, int W8, int BS, int NS, int SC, bool GA, int AS, bool F4>
 bool set_gemm_fp8_smem() {
@@ -96,11 +102,11 @@ void launch_gemm_mx8(int grid, cudaStream_t s, const CUtensorMap &a0, const CUte
 }
 
 // a1 is ignored by the down projection.
-template <bool G, int BN, int BOXN, int ST, int NS, int SC, bool GA>
+template <bool G, int BN, int BOXN, int ST, int NS, int SC, bool GA, bool PR>
 void launch_gemm(int grid, cudaStream_t s, const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b,
                  const GemmParams &p) {
-    grouped_gemm_kernel<G, BN, BOXN, ST, NS, SC, GA>
-        <<<grid, kGemmThreads, GemmCfg<G, BN, BOXN, ST, NS, SC, GA>::kSmem, s>>>(a0, a1, b, p);
+    grouped_gemm_kernel<G, BN, BOXN, ST, NS, SC, GA, PR>
+        <<<grid, kGemmThreads, GemmCfg<G, BN, BOXN, ST, NS, SC, GA, PR>::kSmem, s>>>(a0, a1, b, p);
 }
 // a1 and s1 are ignored by the down projection.
 template <bool G, int BN, int BOXN, int W8, int BS, int NS, int SC, bool GA, int AS, bool F4>
@@ -160,7 +166,7 @@ int init_device(int *dev_out) {
                                        rt_smem_bytes(kRtTokSmall)) == cudaSuccess &&
                   cudaFuncSetAttribute(router_topk_kernel<kRtTokTiny>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        rt_smem_bytes(kRtTokTiny)) == cudaSuccess;
-        ok = ok && set_gemm_smem<G1_WIDE_ARGS>() && set_gemm_smem<G2_WIDE_ARGS>() &&
+        ok = ok && set_gemm_smem<G1_WIDE_ARGS>() && set_gemm_smem<G2_WIDE_ARGS>() && set_gemm_smem<G2_PAIR_ARGS>() &&
              set_gemm_smem<G1_NARROW_ARGS>() && set_gemm_smem<G2_NARROW_ARGS>();
         ok = ok && set_gemm_fp8_smem<G1_WIDE_FP8_ARGS>() && set_gemm_fp8_smem<G2_WIDE_FP8_ARGS>() &&
              set_gemm_fp8_smem<G1_NARROW_FP8_ARGS>() && set_gemm_fp8_smem<G2_NARROW_FP8_ARGS>();
@@ -553,6 +559,7 @@ int enqueue_experts(const beam_moe_config *c, int dev, int64_t T, const beam_bf1
         else launch_gemm_fp8<G2_WIDE_FP8_ARGS>(grid, s, m_wd, m_wd, m_sd, m_sd, m_h, p2, a2);
     } else {
         if (narrow) launch_gemm<G2_NARROW_ARGS>(grid, s, m_wd, m_wd, m_h, p2);
+        else if (once) launch_gemm<G2_PAIR_ARGS>(grid, s, m_wd, m_wd, m_h, p2);
         else launch_gemm<G2_WIDE_ARGS>(grid, s, m_wd, m_wd, m_h, p2);
     }
     if ((rc = launch_status())) return rc;
@@ -1245,7 +1252,7 @@ extern "C" int beam_moe_dense_swiglu(int32_t hidden, int32_t inter, int64_t T, c
     GemmParams p2{counts, offsets, y, 1, inter, hidden, 0, kDefaultTimeoutCycles, nullptr, 1, nullptr, 1};
     launch_gemm<G1_WIDE_ARGS>(grid, s, m_wg, m_wu, m_x, p1);
     if ((rc = launch_status())) return rc;
-    launch_gemm<G2_WIDE_ARGS>(grid, s, m_wd, m_wd, m_h, p2);
+    launch_gemm<G2_PAIR_ARGS>(grid, s, m_wd, m_wd, m_h, p2);
     return launch_status();
 }
 
@@ -1436,6 +1443,7 @@ int beam_moe_expert_rows(int32_t hidden, int32_t inter, int32_t n_experts, int64
     else launch_gemm<G1_WIDE_ARGS>(grid, s, m_wg, m_wu, m_b1, p1);
     if ((rc = launch_status())) return rc;
     if (narrow) launch_gemm<G2_NARROW_ARGS>(grid, s, m_wd, m_wd, m_h, p2);
+    else if (once) launch_gemm<G2_PAIR_ARGS>(grid, s, m_wd, m_wd, m_h, p2);
     else launch_gemm<G2_WIDE_ARGS>(grid, s, m_wd, m_wd, m_h, p2);
     return launch_status();
 }

@@ -11,12 +11,16 @@
 // ~8 tokens in a decode batch and 128 +- 11 in a 4096-token prefill, so one token tile covers all of
 // an expert's tokens and every weight byte crosses HBM once per call.
 //
-// Work item = (expert e, weight-row tile mt of 128, token tile nt of BN).  Items are numbered
+// Work item = (expert e, weight-row tile mt, token tile nt of BN); a weight-row tile is 128 rows, or
+// with PAIR (down projection) two adjacent 128-row tiles that share the item's token tile, so that
+// each token-row byte staged from L2 feeds twice the weight bytes (as W_gate and W_up share it in G1).  Items are numbered
 // expert-major, then mt, then nt, from the per-expert counts (read on the device; no host sync);
 // a persistent grid of one CTA per SM takes items round-robin.
 //
-// Warp roles (256 threads): warp 0 lane 0 = TMA producer; warp 1 = TMEM owner, lane 0 issues
-// tcgen05.mma; warps 4..7 = epilogue (warp 4+q reads TMEM lanes 32q..32q+31).  Shared memory is a
+// Warp roles (320 threads): warp 0 lane 0 = TMA producer; warp 1 = TMEM owner, lane 0 issues
+// tcgen05.mma; warps 2..9 = epilogue, two per TMEM lane quadrant (warp w reads lanes 32(w%4)..+31 and
+// takes every other 16-token chunk of the item, so that an item's slots drain in half the time:
+// while they drain the next item's MMAs wait whenever it needs both slots).  Shared memory is a
 // STAGES-deep ring of {A tile(s) 128x64 bf16, B tile of up to BN x 64 bf16}, 128-byte swizzled by
 // TMA; the B tile is loaded in boxes of BOXN rows, only as many as the item's tokens need.
 //
@@ -33,16 +37,19 @@ namespace beam {
 
 constexpr int kBM = 128;  // weight rows per tile (UMMA M)
 constexpr int kBK = 64;   // K per stage: one 128-byte swizzle row of bf16
-constexpr int kGemmThreads = 256;
+constexpr int kGemmThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2..9 epilogue
+constexpr int kGemmEpiWarps = 8;
 
 constexpr int pow2_cols(int c) { return c <= 32 ? 32 : c <= 64 ? 64 : c <= 128 ? 128 : c <= 256 ? 256 : 512; }
 
-template <bool GATE_UP, int BN, int BOXN, int STAGES, int NSLOT, int SLOT_COLS, bool GATHER = false>
+template <bool GATE_UP, int BN, int BOXN, int STAGES, int NSLOT, int SLOT_COLS, bool GATHER = false,
+          bool PAIR = false>
 struct GemmCfg {
     static constexpr int kA = kBM * kBK * 2;                 // one A tile, bytes
     static constexpr int kB = BN * kBK * 2;                  // B tile, bytes (room for BN rows)
     static constexpr int kBox = BOXN * kBK * 2;              // one B box, bytes
-    static constexpr int kNumA = GATE_UP ? 2 : 1;
+    static constexpr int kNumA = (GATE_UP || PAIR) ? 2 : 1;   // A tiles per stage
+    static constexpr int kRows = PAIR ? 2 * kBM : kBM;        // weight rows per item
     static constexpr int kStage = kNumA * kA + kB;
     static constexpr int kTmemCols = pow2_cols(NSLOT * SLOT_COLS);
     static constexpr int kBarOff = STAGES * kStage;
@@ -52,8 +59,9 @@ struct GemmCfg {
     static_assert(BN % BOXN == 0 && BN % 16 == 0 && BN <= 256, "token tile");
     static_assert(!GATHER || BOXN == 1, "gathered B rows come one row per box, four per instruction");
     static_assert(NSLOT * SLOT_COLS <= 512, "TMEM has 512 columns");
-    static_assert(GATE_UP ? (BN <= SLOT_COLS && (NSLOT >= 2 || BN <= SLOT_COLS / 2)) : BN <= SLOT_COLS,
+    static_assert((GATE_UP || PAIR) ? (BN <= SLOT_COLS && (NSLOT >= 2 || BN <= SLOT_COLS / 2)) : BN <= SLOT_COLS,
                   "an item must fit in its TMEM slots");
+    static_assert(!(GATE_UP && PAIR), "PAIR is a down-projection layout");
     static_assert(kSmem <= 232448, "shared memory per CTA");
 };
 
@@ -121,23 +129,48 @@ __device__ __forceinline__ void item_prefix(const int32_t *counts, int E, int n_
 }
 
 // TMEM slots an item occupies.
-template <bool GATE_UP, int SLOT_COLS>
+// TWO: the item has two accumulators (G1: gate and up; PAIR: its two weight-row halves).
+template <bool TWO, int SLOT_COLS>
 __device__ __forceinline__ int slots_of(int n_mma) {
-    return (GATE_UP && n_mma > SLOT_COLS / 2) ? 2 : 1;
+    return (TWO && n_mma > SLOT_COLS / 2) ? 2 : 1;
 }
 
-// Epilogue (warps 4..7; q = warp - 4 reads TMEM lanes 32q..32q+31): per item, wait for its
-// accumulator slot(s), then write G1: h = bf16(SiLU(gate) * up) or G2: o = fp32 accumulator for the
-// item's rows, and release the slot(s).
-template <bool GATE_UP, int BN, int NSLOT, int SLOT_COLS>
-__device__ __forceinline__ void gemm_epilogue(int q, const int *tile_start, int total, const GemmParams &p,
-                                              uint32_t tmem_base, uint64_t *acc_full, uint64_t *acc_empty) {
+// G2: the accumulators of weight row m for the item's tokens c..c+15 go to o (fp32, or bf16 when
+// out_bf16), row out_row[r] when that map is given.
+__device__ __forceinline__ void store_down_row(const GemmParams &p, const Item &it, int c, int m, const uint32_t (&r)[16]) {
+    if (m >= p.M) return;
+    if (p.out_bf16) {
+        __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.out);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (c + j < it.n_valid) o[(it.row0 + c + j) * p.M + m] = __float2bfloat16_rn(__uint_as_float(r[j]));
+    } else {
+        float *o = reinterpret_cast<float *>(p.out);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (c + j < it.n_valid) {
+                const int64_t row = it.row0 + c + j;
+                const int64_t dst = p.out_row ? static_cast<int64_t>(__ldg(p.out_row + row)) : row;
+                o[dst * p.M + m] = __uint_as_float(r[j]);
+            }
+    }
+}
+
+// Epilogue (q reads TMEM lanes 32q..32q+31; nsub warps share a lane quadrant, warp sub taking the
+// 16-column chunks sub, sub + nsub, ...): per item, wait for its accumulator slot(s), then write G1:
+// h = bf16(SiLU(gate) * up) or G2: o = the accumulators (both halves of the weight-row pair with
+// PAIR), and release the slot(s) (acc_empty counts 4 * nsub arrivals).
+template <bool GATE_UP, int BN, int NSLOT, int SLOT_COLS, bool PAIR>
+__device__ __forceinline__ void gemm_epilogue(int q, int sub, int nsub, const int *tile_start, int total,
+                                              const GemmParams &p, uint32_t tmem_base, uint64_t *acc_full,
+                                              uint64_t *acc_empty) {
+    constexpr int kRows = PAIR ? 2 * kBM : kBM;
     const int lane = threadIdx.x & 31;
     const int E = p.E;
     uint32_t uses = 0;
     for (int item = blockIdx.x; item < total; item += gridDim.x) {
         const Item it = decode_item(item, tile_start, E, BN, p.counts, p.offsets);
-        const int u = slots_of<GATE_UP, SLOT_COLS>(it.n_mma);
+        const int u = slots_of<GATE_UP || PAIR, SLOT_COLS>(it.n_mma);
         bool ok = true;
         for (int i = 0; i < u && ok; ++i) {
             const uint32_t c = uses + i;
@@ -146,12 +179,12 @@ __device__ __forceinline__ void gemm_epilogue(int q, const int *tile_start, int 
         if (!ok) break;
         tc_fence_after();
         const int s0 = uses % NSLOT, s1 = (uses + 1) % NSLOT;
-        const int m = it.mt * kBM + q * 32 + lane;  // weight row of this thread
+        const int m = it.mt * kRows + q * 32 + lane;  // weight row of this thread (PAIR: and m + 128)
         const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
         const uint32_t t0 = tmem_base + lane_off + static_cast<uint32_t>(s0 * SLOT_COLS);
         const uint32_t t1 = tmem_base + lane_off +
                             static_cast<uint32_t>(u == 2 ? s1 * SLOT_COLS : s0 * SLOT_COLS + SLOT_COLS / 2);
-        for (int c = 0; c < it.n_valid; c += 16) {
+        for (int c = 16 * sub; c < it.n_valid; c += 16 * nsub) {
             uint32_t r0[16];
             tmem_ld16(t0 + c, r0);
             if (GATE_UP) {
@@ -166,23 +199,15 @@ __device__ __forceinline__ void gemm_epilogue(int q, const int *tile_start, int 
                             h[(it.row0 + c + j) * p.M + m] =
                                 __float2bfloat16_rn(silu_mul(__uint_as_float(r0[j]), __uint_as_float(r1[j])));
                 }
+            } else if (PAIR) {
+                uint32_t r1[16];
+                tmem_ld16(t1 + c, r1);
+                tmem_ld_wait();
+                store_down_row(p, it, c, m, r0);
+                store_down_row(p, it, c, m + kBM, r1);
             } else {
                 tmem_ld_wait();
-                if (m < p.M && p.out_bf16) {
-                    __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(p.out);
-#pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        if (c + j < it.n_valid) o[(it.row0 + c + j) * p.M + m] = __float2bfloat16_rn(__uint_as_float(r0[j]));
-                } else if (m < p.M) {
-                    float *o = reinterpret_cast<float *>(p.out);
-#pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        if (c + j < it.n_valid) {
-                            const int64_t r = it.row0 + c + j;
-                            const int64_t dst = p.out_row ? static_cast<int64_t>(__ldg(p.out_row + r)) : r;
-                            o[dst * p.M + m] = __uint_as_float(r0[j]);
-                        }
-                }
+                store_down_row(p, it, c, m, r0);
             }
         }
         tc_fence_before();
@@ -193,14 +218,15 @@ __device__ __forceinline__ void gemm_epilogue(int q, const int *tile_start, int 
     }
 }
 
-template <bool GATE_UP, int BN, int BOXN, int STAGES, int NSLOT, int SLOT_COLS, bool GATHER = false>
+template <bool GATE_UP, int BN, int BOXN, int STAGES, int NSLOT, int SLOT_COLS, bool GATHER = false,
+          bool PAIR = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tm_a0,  // W_gate (G1) / W_down (G2): [E][M][K]
                         const __grid_constant__ CUtensorMap tm_a1,  // W_up (G1); unused for G2
                         const __grid_constant__ CUtensorMap tm_b,   // B rows [rows][K]: box BOXN rows, or
                                                                     // GATHER: x [T][K] with a one-row box
                         const GemmParams p) {
-    using C = GemmCfg<GATE_UP, BN, BOXN, STAGES, NSLOT, SLOT_COLS, GATHER>;
+    using C = GemmCfg<GATE_UP, BN, BOXN, STAGES, NSLOT, SLOT_COLS, GATHER, PAIR>;
     extern __shared__ uint8_t gemm_smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(gemm_smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::kBarOff);
@@ -214,7 +240,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = p.E;
-    const int n_mt = (p.M + kBM - 1) / kBM;
+    const int n_mt = (p.M + C::kRows - 1) / C::kRows;
     const int n_kb = p.K / kBK;
 
     if (threadIdx.x == 0) {
@@ -224,7 +250,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         for (int a = 0; a < NSLOT; ++a) {
             mbar_init(&acc_full[a], 1);
-            mbar_init(&acc_empty[a], 4);
+            mbar_init(&acc_empty[a], kGemmEpiWarps);
         }
         mbar_init(drain, 1);
         fence_mbar_init();
@@ -271,8 +297,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                     }
                     uint8_t *sa = smem + stage * C::kStage;
                     mbar_arrive_expect_tx(&full[stage], bytes);
-                    tma_load_3d(sa, &tm_a0, &full[stage], kb * kBK, it.mt * kBM, it.e, pol_w);
+                    tma_load_3d(sa, &tm_a0, &full[stage], kb * kBK, it.mt * C::kRows, it.e, pol_w);
                     if (GATE_UP) tma_load_3d(sa + C::kA, &tm_a1, &full[stage], kb * kBK, it.mt * kBM, it.e, pol_w);
+                    // PAIR: the second half may start past M (zero-filled by the TMA unit; never stored)
+                    if (PAIR) tma_load_3d(sa + C::kA, &tm_a0, &full[stage], kb * kBK, it.mt * C::kRows + kBM, it.e, pol_w);
                     uint8_t *sb = sa + C::kNumA * C::kA;
                     if (GATHER) {
                         for (int g = 0; g < nbox; ++g)  // rows 4g..4g+3 land 128 B apart, as a tiled box would
@@ -309,7 +337,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
                 const Item it = decode_item(item, tile_start, E, BN, p.counts, p.offsets);
                 const uint32_t idesc = umma_idesc_bf16(kBM, it.n_mma);
-                const int u = slots_of<GATE_UP, SLOT_COLS>(it.n_mma);
+                const int u = slots_of<GATE_UP || PAIR, SLOT_COLS>(it.n_mma);
                 const int s0 = uses % NSLOT, s1 = (uses + 1) % NSLOT;
                 for (int i = 0; i < u && ok; ++i) {
                     const uint32_t c = uses + i;
@@ -334,7 +362,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                         const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
                         // +32 bytes along K inside the swizzle row = +2 in the 16-byte address field
                         umma_bf16(d0, da0 + 2 * kk, db + 2 * kk, idesc, accum);
-                        if (GATE_UP) umma_bf16(d1, da1 + 2 * kk, db + 2 * kk, idesc, accum);
+                        if (GATE_UP || PAIR) umma_bf16(d1, da1 + 2 * kk, db + 2 * kk, idesc, accum);
                     }
                     umma_commit(&empty[stage]);  // frees the smem stage once these MMAs completed
                     if (++stage == STAGES) {
@@ -350,8 +378,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             umma_commit(drain);
             mbar_wait(drain, 0, p.timeout);
         }
-    } else if (warp >= 4) {
-        gemm_epilogue<GATE_UP, BN, NSLOT, SLOT_COLS>(warp - 4, tile_start, total, p, tmem_base, acc_full, acc_empty);
+    } else {
+        // warps 2..9: two per TMEM lane quadrant (a warp reads the quadrant warp % 4)
+        gemm_epilogue<GATE_UP, BN, NSLOT, SLOT_COLS, PAIR>(warp & 3, (warp - 2) / 4, 2, tile_start, total, p,
+                                                           tmem_base, acc_full, acc_empty);
     }
     tc_fence_before();
     __syncthreads();
