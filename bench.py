@@ -51,12 +51,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 _CSRC = os.path.join(ROOT, "group_limited_routing_router_b200", "csrc")
 _BF16_SRC = ("gemm.cuh", "common.cuh")
 NCU_TRAFFIC = {
-    ("gate_up_swiglu", "decode"): {"bytes": 8 * (1678295040 + 1369856), "files": _BF16_SRC, "hash": "fbd3f5b6bb402249"},
-    ("gate_up_swiglu", "prefill"): {"bytes": 8 * (1724978688 + 2582016), "files": _BF16_SRC, "hash": "fbd3f5b6bb402249"},
-    ("gate_up_swiglu", "long"): {"bytes": 8 * (3484946688 + 326665216), "files": _BF16_SRC, "hash": "fbd3f5b6bb402249"},
-    ("down", "decode"): {"bytes": 8 * (840219392 + 3311616), "files": _BF16_SRC, "hash": "fbd3f5b6bb402249"},
-    ("down", "prefill"): {"bytes": 8 * (869167616 + 32409088), "files": _BF16_SRC, "hash": "fbd3f5b6bb402249"},
-    ("down", "long"): {"bytes": 8 * (1221652480 + 1301204736), "files": _BF16_SRC, "hash": "fbd3f5b6bb402249"},
+    ("gate_up_swiglu", "decode"): {"bytes": 8 * (1678102016 + 1311744), "files": _BF16_SRC, "hash": "0fc4678ac2a79b74"},
+    ("gate_up_swiglu", "prefill"): {"bytes": 8 * (1725097216 + 2001408), "files": _BF16_SRC, "hash": "0fc4678ac2a79b74"},
+    ("gate_up_swiglu", "long"): {"bytes": 8 * (3182454272 + 326637312), "files": _BF16_SRC, "hash": "0fc4678ac2a79b74"},
+    ("down", "decode"): {"bytes": 8 * (840225024 + 3345408), "files": _BF16_SRC, "hash": "0fc4678ac2a79b74"},
+    ("down", "prefill"): {"bytes": 8 * (866353664 + 30267904), "files": _BF16_SRC, "hash": "0fc4678ac2a79b74"},
+    ("down", "long"): {"bytes": 8 * (1181398016 + 1304011264), "files": _BF16_SRC, "hash": "0fc4678ac2a79b74"},
 }
 
 
