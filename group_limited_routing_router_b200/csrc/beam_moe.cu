@@ -7,6 +7,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -19,6 +20,7 @@
 #include "combine.cuh"
 #include "permute.cuh"
 #include "gemm.cuh"
+#include "gemm_2sm.cuh"
 #include "gemm_fp8.cuh"
 #include "gemm_mx8.cuh"
 #include "norm.cuh"
@@ -35,16 +37,22 @@ constexpr int64_t kMaxTokens = int64_t(1) << 24;
 // ---- GEMM variants: <gate/up?, BN, B box rows, smem stages, TMEM slots, slot columns, gather?,
 // weight-row pairs?> -----
 // "wide": experts see up to ~190 tokens per tile (prefill): the dispatch also gathers x into
-// dispatch order (x_perm) and both GEMMs read their token rows with tiled 64-row TMA boxes.
+// dispatch order (x_perm) and both GEMMs read their token rows with tiled TMA boxes (64 rows on
+// single CTAs, 32 rows on CTA pairs).
 // "narrow": a few tokens per expert (decode): the gate/up GEMM gathers its rows straight from x
 // with TMA gather4 (four rows per instruction; cheap when an expert has a handful of tokens).
 #define G1_WIDE_ARGS true, 192, 64, 4, 2, 256, false, false
-#define G2_WIDE_ARGS false, 192, 64, 5, 2, 256, false, false
-// "pair": the down projection with two 128-row weight tiles per token tile.  Half the token-row bytes
-// per weight byte, but an item then fills both TMEM slots whenever it has more than 128 tokens, so
-// its epilogue is not overlapped with the next item's products: used where every expert fits one
-// token tile (the weights are read once) and for the dense MLP (K = 20480 makes the epilogue small).
+// "pair": the down projection with two 128-row weight tiles per token tile (half the token-row bytes
+// per weight byte).  The dense MLP runs G1_WIDE and this on single CTAs: its K = 20480 makes items
+// long, and 440 of them would leave a 10% wave tail on 74 CTA pairs.
 #define G2_PAIR_ARGS false, 192, 64, 4, 2, 256, false, true
+// CTA-pair variants (cta_group::2) for the MoE bf16 wide case (prefill, skew, long; the expert-rows
+// entry point): <gate/up?, BN, B box rows, smem stages, TMEM slots, slot columns>; each CTA stages half
+// of the token tile in 32-row boxes.  Against the single-CTA kernels (same process, alternating calls):
+// prefill 4.19 vs 4.22 ms per layer, skew 12.99 vs 13.67, long 49.4 vs 54.3.
+#define G1_2SM_ARGS true, 192, 32, 5, 2, 256
+#define G2_2SM_ARGS false, 192, 32, 8, 2, 256
+constexpr int k2smBox = 32;
 #define G1_NARROW_ARGS true, 32, 1, 6, 4, 64, true, false
 #define G2_NARROW_ARGS false, 32, 32, 10, 4, 32, false, false
 // FP8 variants: <gate/up?, BN, B box rows, weight stages (K = 128), B stages (K = 64), TMEM slots,
@@ -108,6 +116,31 @@ void launch_gemm(int grid, cudaStream_t s, const CUtensorMap &a0, const CUtensor
     grouped_gemm_kernel<G, BN, BOXN, ST, NS, SC, GA, PR>
         <<<grid, kGemmThreads, GemmCfg<G, BN, BOXN, ST, NS, SC, GA, PR>::kSmem, s>>>(a0, a1, b, p);
 }
+template <bool G, int BN, int BOXN, int ST, int NS, int SC>
+bool set_gemm2_smem() {
+    return cudaFuncSetAttribute(grouped_gemm_2sm_kernel<G, BN, BOXN, ST, NS, SC>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Gemm2Cfg<G, BN, BOXN, ST, NS, SC>::kSmem) == cudaSuccess;
+}
+// CTA pairs of the pair GEMM that fit on the device at once (at most one CTA per SM); 0 on failure.
+template <bool G, int BN, int BOXN, int ST, int NS, int SC>
+int gemm2_pairs(int sms) {
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(static_cast<unsigned>(2 * (sms / 2)), 1, 1);
+    lc.blockDim = dim3(kGemmThreads, 1, 1);
+    lc.dynamicSmemBytes = Gemm2Cfg<G, BN, BOXN, ST, NS, SC>::kSmem;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_2sm_kernel<G, BN, BOXN, ST, NS, SC>, &lc) != cudaSuccess)
+        return 0;
+    return std::min(n, sms / 2);
+}
+// a1 is ignored by the down projection; `pairs` clusters of 2 CTAs.
+template <bool G, int BN, int BOXN, int ST, int NS, int SC>
+void launch_gemm2(int pairs, cudaStream_t s, const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &b,
+                  const GemmParams &p) {
+    grouped_gemm_2sm_kernel<G, BN, BOXN, ST, NS, SC>
+        <<<2 * pairs, kGemmThreads, Gemm2Cfg<G, BN, BOXN, ST, NS, SC>::kSmem, s>>>(a0, a1, b, p);
+}
 // a1 and s1 are ignored by the down projection.
 template <bool G, int BN, int BOXN, int W8, int BS, int NS, int SC, bool GA, int AS, bool F4>
 void launch_gemm_fp8(int grid, cudaStream_t s, const CUtensorMap &a0, const CUtensorMap &a1, const CUtensorMap &s0,
@@ -127,6 +160,7 @@ struct DeviceInfo {
     int status = BEAM_MOE_OK;
     int num_sms = 0;
     int clock_khz = 0;
+    int pairs_g1 = 0, pairs_g2 = 0;  // co-resident CTA pairs of the pair GEMMs (persistent grids)
 };
 DeviceInfo g_dev[kMaxDevices];
 
@@ -166,7 +200,7 @@ int init_device(int *dev_out) {
                                        rt_smem_bytes(kRtTokSmall)) == cudaSuccess &&
                   cudaFuncSetAttribute(router_topk_kernel<kRtTokTiny>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        rt_smem_bytes(kRtTokTiny)) == cudaSuccess;
-        ok = ok && set_gemm_smem<G1_WIDE_ARGS>() && set_gemm_smem<G2_WIDE_ARGS>() && set_gemm_smem<G2_PAIR_ARGS>() &&
+        ok = ok && set_gemm_smem<G1_WIDE_ARGS>() && set_gemm_smem<G2_PAIR_ARGS>() &&
              set_gemm_smem<G1_NARROW_ARGS>() && set_gemm_smem<G2_NARROW_ARGS>();
         ok = ok && set_gemm_fp8_smem<G1_WIDE_FP8_ARGS>() && set_gemm_fp8_smem<G2_WIDE_FP8_ARGS>() &&
              set_gemm_fp8_smem<G1_NARROW_FP8_ARGS>() && set_gemm_fp8_smem<G2_NARROW_FP8_ARGS>();
@@ -181,6 +215,12 @@ int init_device(int *dev_out) {
         ok = ok && set_router_tc_smem<32>() && set_router_tc_smem<64>() && set_router_tc_smem<128>();
         ok = ok && cudaFuncSetAttribute(router_exact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         kRsPathSmem) == cudaSuccess;
+        ok = ok && set_gemm2_smem<G1_2SM_ARGS>() && set_gemm2_smem<G2_2SM_ARGS>();
+        if (ok) {
+            d.pairs_g1 = gemm2_pairs<G1_2SM_ARGS>(d.num_sms);
+            d.pairs_g2 = gemm2_pairs<G2_2SM_ARGS>(d.num_sms);
+            ok = d.pairs_g1 > 0 && d.pairs_g2 > 0;
+        }
         if (!ok) d.status = BEAM_MOE_ERR_CUDA;
     });
     *dev_out = dev;
@@ -511,7 +551,9 @@ int enqueue_experts(const beam_moe_config *c, int dev, int64_t T, const beam_bf1
 
     const double mean_rows = static_cast<double>(R) / E;
     const int bn = narrow ? kNarrowBN : kWideBN;
-    const int box = narrow ? kNarrowBox : kWideBox;
+    // bf16 weights with wide tiles run on CTA pairs, which stage their token rows in 32-row boxes
+    const bool pair2 = !narrow && !W.fp8 && !W.fp4;
+    const int box = narrow ? kNarrowBox : (pair2 ? k2smBox : kWideBox);
     // Weights are read once per call when (almost) every expert fits one token tile: mark them
     // evict-first so they do not push the reused activations out of L2.
     const int once = (mean_rows + 4.0 * std::sqrt(mean_rows) <= bn) ? 1 : 0;
@@ -547,7 +589,7 @@ int enqueue_experts(const beam_moe_config *c, int dev, int64_t T, const beam_bf1
         else launch_gemm_fp8<G1_WIDE_FP8_ARGS>(grid, s, m_wg, m_wu, m_sg, m_su, m_b1, p1, a1);
     } else {
         if (narrow) launch_gemm<G1_NARROW_ARGS>(grid, s, m_wg, m_wu, m_b1, p1);
-        else launch_gemm<G1_WIDE_ARGS>(grid, s, m_wg, m_wu, m_b1, p1);
+        else launch_gemm2<G1_2SM_ARGS>(g_dev[dev].pairs_g1, s, m_wg, m_wu, m_b1, p1);
     }
     if ((rc = launch_status())) return rc;
     if (!record(ev, 4, s)) return BEAM_MOE_ERR_CUDA;
@@ -559,8 +601,7 @@ int enqueue_experts(const beam_moe_config *c, int dev, int64_t T, const beam_bf1
         else launch_gemm_fp8<G2_WIDE_FP8_ARGS>(grid, s, m_wd, m_wd, m_sd, m_sd, m_h, p2, a2);
     } else {
         if (narrow) launch_gemm<G2_NARROW_ARGS>(grid, s, m_wd, m_wd, m_h, p2);
-        else if (once) launch_gemm<G2_PAIR_ARGS>(grid, s, m_wd, m_wd, m_h, p2);
-        else launch_gemm<G2_WIDE_ARGS>(grid, s, m_wd, m_wd, m_h, p2);
+        else launch_gemm2<G2_2SM_ARGS>(g_dev[dev].pairs_g2, s, m_wd, m_wd, m_h, p2);
     }
     if ((rc = launch_status())) return rc;
     if (!record(ev, 5, s)) return BEAM_MOE_ERR_CUDA;
@@ -1422,7 +1463,7 @@ int beam_moe_expert_rows(int32_t hidden, int32_t inter, int32_t n_experts, int64
                                                                     reinterpret_cast<uint4 *>(wsb + L.xp));
         if ((rc = launch_status())) return rc;
     }
-    const int box = narrow ? kNarrowBox : kWideBox;
+    const int box = narrow ? kNarrowBox : k2smBox;
     const int bn = narrow ? kNarrowBN : kWideBN;
     const double mean_rows = static_cast<double>(R) / n_experts;
     const int once = (mean_rows + 4.0 * std::sqrt(mean_rows) <= bn) ? 1 : 0;
@@ -1440,11 +1481,10 @@ int beam_moe_expert_rows(int32_t hidden, int32_t inter, int32_t n_experts, int64
     // the down projection stores dispatch row r at the caller's row row_src[r] (k = 1)
     GemmParams p2{counts, offsets, o_rows, n_experts, inter, hidden, once, kDefaultTimeoutCycles, nullptr, 1, row_src};
     if (narrow) launch_gemm<G1_NARROW_ARGS>(grid, s, m_wg, m_wu, m_b1, p1);
-    else launch_gemm<G1_WIDE_ARGS>(grid, s, m_wg, m_wu, m_b1, p1);
+    else launch_gemm2<G1_2SM_ARGS>(g_dev[dev].pairs_g1, s, m_wg, m_wu, m_b1, p1);
     if ((rc = launch_status())) return rc;
     if (narrow) launch_gemm<G2_NARROW_ARGS>(grid, s, m_wd, m_wd, m_h, p2);
-    else if (once) launch_gemm<G2_PAIR_ARGS>(grid, s, m_wd, m_wd, m_h, p2);
-    else launch_gemm<G2_WIDE_ARGS>(grid, s, m_wd, m_wd, m_h, p2);
+    else launch_gemm2<G2_2SM_ARGS>(g_dev[dev].pairs_g2, s, m_wd, m_wd, m_h, p2);
     return launch_status();
 }
 

@@ -156,15 +156,58 @@ __device__ __forceinline__ void store_down_row(const GemmParams &p, const Item &
     }
 }
 
-// Epilogue (q reads TMEM lanes 32q..32q+31; nsub warps share a lane quadrant, warp sub taking the
-// 16-column chunks sub, sub + nsub, ...): per item, wait for its accumulator slot(s), then write G1:
-// h = bf16(SiLU(gate) * up) or G2: o = the accumulators (both halves of the weight-row pair with
-// PAIR), and release the slot(s) (acc_empty counts 4 * nsub arrivals).
-template <bool GATE_UP, int BN, int NSLOT, int SLOT_COLS, bool PAIR>
-__device__ __forceinline__ void gemm_epilogue(int q, int sub, int nsub, const int *tile_start, int total,
-                                              const GemmParams &p, uint32_t tmem_base, uint64_t *acc_full,
-                                              uint64_t *acc_empty) {
+// G1 with two epilogue warps per lane quadrant (warp `sub` takes the 16-column chunks 16 sub + 32 i):
+// SiLU(gate) * up of the thread's weight row, rounded to bf16 and kept in registers as pairs (token
+// columns 2j, 2j + 1 of chunk i in hv[i][j]), so that the TMEM slots can be released before any h
+// store is issued: an item with more than SLOT_COLS / 2 tokens holds both slots, the next item's
+// products wait for them, and stores issued while the weight stream saturates the memory system
+// would hold that release back.
+template <int BN>
+__device__ __forceinline__ void swiglu_to_regs(uint32_t t0, uint32_t t1, int sub, int n_valid,
+                                               uint32_t (&hv)[(BN + 31) / 32][8]) {
+#pragma unroll
+    for (int i = 0; i < (BN + 31) / 32; ++i) {
+        const int c = 16 * sub + 32 * i;
+        if (c < n_valid) {  // warp-uniform
+            uint32_t r0[16], r1[16];
+            tmem_ld16(t0 + c, r0);
+            tmem_ld16(t1 + c, r1);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const __nv_bfloat162 v =
+                    __floats2bfloat162_rn(silu_mul(__uint_as_float(r0[2 * j]), __uint_as_float(r1[2 * j])),
+                                          silu_mul(__uint_as_float(r0[2 * j + 1]), __uint_as_float(r1[2 * j + 1])));
+                hv[i][j] = *reinterpret_cast<const uint32_t *>(&v);
+            }
+        }
+    }
+}
+// The h values of swiglu_to_regs: weight row m (< M) of the item's tokens.
+template <int BN>
+__device__ __forceinline__ void store_h_regs(const GemmParams &p, const Item &it, int sub, int m,
+                                             const uint32_t (&hv)[(BN + 31) / 32][8]) {
+    const int64_t ld = p.M;
+    uint16_t *h = reinterpret_cast<uint16_t *>(p.out) + (it.row0 + 16 * sub) * ld + m;
+#pragma unroll
+    for (int i = 0; i < (BN + 31) / 32; ++i) {
+        const int left = it.n_valid - (16 * sub + 32 * i);  // valid columns from this chunk on
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            if (j < left) h[(32 * i + j) * ld] = static_cast<uint16_t>(hv[i][j >> 1] >> (16 * (j & 1)));
+    }
+}
+
+// Epilogue (q reads TMEM lanes 32q..32q+31; NSUB warps share a lane quadrant, warp sub taking the
+// 16-column chunks sub, sub + NSUB, ...): per item, wait for its accumulator slot(s), then write G1:
+// h = bf16(SiLU(gate) * up) (with NSUB = 2 through registers, stored after the release) or G2: o =
+// the accumulators (both halves of the weight-row pair with PAIR), and release the slot(s) (acc_empty
+// counts 4 * NSUB arrivals).
+template <bool GATE_UP, int BN, int NSLOT, int SLOT_COLS, bool PAIR, int NSUB>
+__device__ __forceinline__ void gemm_epilogue(int q, int sub, const int *tile_start, int total, const GemmParams &p,
+                                              uint32_t tmem_base, uint64_t *acc_full, uint64_t *acc_empty) {
     constexpr int kRows = PAIR ? 2 * kBM : kBM;
+    constexpr bool kDefer = GATE_UP && NSUB == 2;
     const int lane = threadIdx.x & 31;
     const int E = p.E;
     uint32_t uses = 0;
@@ -184,7 +227,9 @@ __device__ __forceinline__ void gemm_epilogue(int q, int sub, int nsub, const in
         const uint32_t t0 = tmem_base + lane_off + static_cast<uint32_t>(s0 * SLOT_COLS);
         const uint32_t t1 = tmem_base + lane_off +
                             static_cast<uint32_t>(u == 2 ? s1 * SLOT_COLS : s0 * SLOT_COLS + SLOT_COLS / 2);
-        for (int c = 16 * sub; c < it.n_valid; c += 16 * nsub) {
+        uint32_t hv[kDefer ? (BN + 31) / 32 : 1][8];
+        if constexpr (kDefer) swiglu_to_regs<BN>(t0, t1, sub, it.n_valid, hv);
+        for (int c = 16 * sub; c < (kDefer ? 0 : it.n_valid); c += 16 * NSUB) {
             uint32_t r0[16];
             tmem_ld16(t0 + c, r0);
             if (GATE_UP) {
@@ -215,6 +260,8 @@ __device__ __forceinline__ void gemm_epilogue(int q, int sub, int nsub, const in
         if (lane == 0)
             for (int i = 0; i < u; ++i) mbar_arrive(&acc_empty[(uses + i) % NSLOT]);
         uses += u;
+        if constexpr (kDefer)
+            if (m < p.M) store_h_regs<BN>(p, it, sub, m, hv);
     }
 }
 
@@ -380,8 +427,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
     } else {
         // warps 2..9: two per TMEM lane quadrant (a warp reads the quadrant warp % 4)
-        gemm_epilogue<GATE_UP, BN, NSLOT, SLOT_COLS, PAIR>(warp & 3, (warp - 2) / 4, 2, tile_start, total, p,
-                                                           tmem_base, acc_full, acc_empty);
+        gemm_epilogue<GATE_UP, BN, NSLOT, SLOT_COLS, PAIR, 2>(warp & 3, (warp - 2) / 4, tile_start, total, p,
+                                                              tmem_base, acc_full, acc_empty);
     }
     tc_fence_before();
     __syncthreads();

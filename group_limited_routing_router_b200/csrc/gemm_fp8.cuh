@@ -399,8 +399,8 @@ __global__ void __launch_bounds__(fp8_gemm_threads(GATE_UP), 1)
             gemm_epilogue_scaled<GATE_UP, BN, NSLOT, SLOT_COLS>(warp - 4, tile_start, total, p, acc, tmem_base,
                                                                 acc_full, acc_empty);
         else
-            gemm_epilogue<GATE_UP, BN, NSLOT, SLOT_COLS, false>(warp - 4, 0, 1, tile_start, total, p, tmem_base,
-                                                                acc_full, acc_empty);
+            gemm_epilogue<GATE_UP, BN, NSLOT, SLOT_COLS, false, 1>(warp - 4, 0, tile_start, total, p, tmem_base,
+                                                                   acc_full, acc_empty);
     } else if (warp >= 8) {
         // ---------------- converters: codes (smem) -> bf16 A ring (TMEM) ----------------
         // Converter warp wc = w - 8 owns TMEM lane quadrant wc % 4 (weight rows r = 32 (wc % 4) + lane)
