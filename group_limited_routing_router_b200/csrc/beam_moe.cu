@@ -52,6 +52,10 @@ constexpr int64_t kMaxTokens = int64_t(1) << 24;
 // prefill 4.19 vs 4.22 ms per layer, skew 12.99 vs 13.67, long 49.4 vs 54.3.
 #define G1_2SM_ARGS true, 192, 32, 5, 2, 256
 #define G2_2SM_ARGS false, 192, 32, 8, 2, 256
+// 256-token tiles where experts span several token tiles (skew, long: tensor-bound): a third more
+// products per staged byte; the down projection still keeps one TMEM slot per item.
+#define G1_2SM_BIG_ARGS true, 256, 32, 4, 2, 256
+#define G2_2SM_BIG_ARGS false, 256, 32, 7, 2, 256
 constexpr int k2smBox = 32;
 #define G1_NARROW_ARGS true, 32, 1, 6, 4, 64, true, false
 #define G2_NARROW_ARGS false, 32, 32, 10, 4, 32, false, false
@@ -160,7 +164,7 @@ struct DeviceInfo {
     int status = BEAM_MOE_OK;
     int num_sms = 0;
     int clock_khz = 0;
-    int pairs_g1 = 0, pairs_g2 = 0;  // co-resident CTA pairs of the pair GEMMs (persistent grids)
+    int pairs_g1 = 0, pairs_g2 = 0, pairs_g1b = 0, pairs_g2b = 0;  // co-resident CTA pairs (persistent grids)
 };
 DeviceInfo g_dev[kMaxDevices];
 
@@ -215,11 +219,14 @@ int init_device(int *dev_out) {
         ok = ok && set_router_tc_smem<32>() && set_router_tc_smem<64>() && set_router_tc_smem<128>();
         ok = ok && cudaFuncSetAttribute(router_exact_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         kRsPathSmem) == cudaSuccess;
-        ok = ok && set_gemm2_smem<G1_2SM_ARGS>() && set_gemm2_smem<G2_2SM_ARGS>();
+        ok = ok && set_gemm2_smem<G1_2SM_ARGS>() && set_gemm2_smem<G2_2SM_ARGS>() &&
+             set_gemm2_smem<G1_2SM_BIG_ARGS>() && set_gemm2_smem<G2_2SM_BIG_ARGS>();
         if (ok) {
             d.pairs_g1 = gemm2_pairs<G1_2SM_ARGS>(d.num_sms);
             d.pairs_g2 = gemm2_pairs<G2_2SM_ARGS>(d.num_sms);
-            ok = d.pairs_g1 > 0 && d.pairs_g2 > 0;
+            d.pairs_g1b = gemm2_pairs<G1_2SM_BIG_ARGS>(d.num_sms);
+            d.pairs_g2b = gemm2_pairs<G2_2SM_BIG_ARGS>(d.num_sms);
+            ok = d.pairs_g1 > 0 && d.pairs_g2 > 0 && d.pairs_g1b > 0 && d.pairs_g2b > 0;
         }
         if (!ok) d.status = BEAM_MOE_ERR_CUDA;
     });
@@ -589,7 +596,8 @@ int enqueue_experts(const beam_moe_config *c, int dev, int64_t T, const beam_bf1
         else launch_gemm_fp8<G1_WIDE_FP8_ARGS>(grid, s, m_wg, m_wu, m_sg, m_su, m_b1, p1, a1);
     } else {
         if (narrow) launch_gemm<G1_NARROW_ARGS>(grid, s, m_wg, m_wu, m_b1, p1);
-        else launch_gemm2<G1_2SM_ARGS>(g_dev[dev].pairs_g1, s, m_wg, m_wu, m_b1, p1);
+        else if (once) launch_gemm2<G1_2SM_ARGS>(g_dev[dev].pairs_g1, s, m_wg, m_wu, m_b1, p1);
+        else launch_gemm2<G1_2SM_BIG_ARGS>(g_dev[dev].pairs_g1b, s, m_wg, m_wu, m_b1, p1);
     }
     if ((rc = launch_status())) return rc;
     if (!record(ev, 4, s)) return BEAM_MOE_ERR_CUDA;
@@ -601,7 +609,8 @@ int enqueue_experts(const beam_moe_config *c, int dev, int64_t T, const beam_bf1
         else launch_gemm_fp8<G2_WIDE_FP8_ARGS>(grid, s, m_wd, m_wd, m_sd, m_sd, m_h, p2, a2);
     } else {
         if (narrow) launch_gemm<G2_NARROW_ARGS>(grid, s, m_wd, m_wd, m_h, p2);
-        else launch_gemm2<G2_2SM_ARGS>(g_dev[dev].pairs_g2, s, m_wd, m_wd, m_h, p2);
+        else if (once) launch_gemm2<G2_2SM_ARGS>(g_dev[dev].pairs_g2, s, m_wd, m_wd, m_h, p2);
+        else launch_gemm2<G2_2SM_BIG_ARGS>(g_dev[dev].pairs_g2b, s, m_wd, m_wd, m_h, p2);
     }
     if ((rc = launch_status())) return rc;
     if (!record(ev, 5, s)) return BEAM_MOE_ERR_CUDA;
@@ -1481,10 +1490,12 @@ int beam_moe_expert_rows(int32_t hidden, int32_t inter, int32_t n_experts, int64
     // the down projection stores dispatch row r at the caller's row row_src[r] (k = 1)
     GemmParams p2{counts, offsets, o_rows, n_experts, inter, hidden, once, kDefaultTimeoutCycles, nullptr, 1, row_src};
     if (narrow) launch_gemm<G1_NARROW_ARGS>(grid, s, m_wg, m_wu, m_b1, p1);
-    else launch_gemm2<G1_2SM_ARGS>(g_dev[dev].pairs_g1, s, m_wg, m_wu, m_b1, p1);
+    else if (once) launch_gemm2<G1_2SM_ARGS>(g_dev[dev].pairs_g1, s, m_wg, m_wu, m_b1, p1);
+    else launch_gemm2<G1_2SM_BIG_ARGS>(g_dev[dev].pairs_g1b, s, m_wg, m_wu, m_b1, p1);
     if ((rc = launch_status())) return rc;
     if (narrow) launch_gemm<G2_NARROW_ARGS>(grid, s, m_wd, m_wd, m_h, p2);
-    else launch_gemm2<G2_2SM_ARGS>(g_dev[dev].pairs_g2, s, m_wd, m_wd, m_h, p2);
+    else if (once) launch_gemm2<G2_2SM_ARGS>(g_dev[dev].pairs_g2, s, m_wd, m_wd, m_h, p2);
+    else launch_gemm2<G2_2SM_BIG_ARGS>(g_dev[dev].pairs_g2b, s, m_wd, m_wd, m_h, p2);
     return launch_status();
 }
 
