@@ -284,7 +284,7 @@ size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 struct RoutePlan {
     bool ok = false;  // false: the configuration takes the direct router
     int bn = 0, S = 0, kps = 0, n_nt = 0, n_mt = 0;
-    size_t planes = 0, part = 0, list = 0, list_n = 0, exact = 0, total = 0;
+    size_t planes = 0, part = 0, list = 0, counters = 0, exact = 0, bucket = 0, xlogit = 0, listed = 0, total = 0;
 };
 
 RoutePlan route_plan(const beam_moe_config *c, int64_t T) {
@@ -314,8 +314,11 @@ RoutePlan route_plan(const beam_moe_config *c, int64_t T) {
     P.planes = take(3 * E * H * 2);
     P.part = take(static_cast<size_t>(P.S) * T * E * 4);
     P.list = take(static_cast<size_t>(T) * 4);
-    P.list_n = take(4);
+    P.counters = take((1 + E) * 4);  // the list's length, then the picks per expert (zeroed per call)
     P.exact = take(static_cast<size_t>(T) * E * 4);
+    P.bucket = take(static_cast<size_t>(T) * E * 4);
+    P.xlogit = take(static_cast<size_t>(T) * c->topk * 4);
+    P.listed = take(static_cast<size_t>(T));
     P.total = off;
     return P;
 }
@@ -474,10 +477,12 @@ int enqueue_route_ws(const beam_moe_config *c, int dev, int64_t T, const beam_bf
     void *planes = scratch + P.planes;
     float *part = reinterpret_cast<float *>(scratch + P.part);
     int32_t *list = reinterpret_cast<int32_t *>(scratch + P.list);
-    int32_t *list_n = reinterpret_cast<int32_t *>(scratch + P.list_n);
+    int32_t *list_n = reinterpret_cast<int32_t *>(scratch + P.counters);
+    int32_t *bcnt = list_n + 1;
     float *exact = reinterpret_cast<float *>(scratch + P.exact);
     const int sms = g_dev[dev].num_sms;
-    if (cudaMemsetAsync(list_n, 0, sizeof(int32_t), s) != cudaSuccess) return BEAM_MOE_ERR_CUDA;
+    if (cudaMemsetAsync(list_n, 0, (1 + static_cast<size_t>(E)) * sizeof(int32_t), s) != cudaSuccess)
+        return BEAM_MOE_ERR_CUDA;
     const int64_t n4 = static_cast<int64_t>(E) * H / 4;
     router_split_kernel<<<static_cast<unsigned>(std::min<int64_t>((n4 + 255) / 256, 4 * sms)), 256, 0, s>>>(
         reinterpret_cast<const float4 *>(w_router), n4, reinterpret_cast<uint2 *>(planes));
@@ -493,15 +498,18 @@ int enqueue_route_ws(const beam_moe_config *c, int dev, int64_t T, const beam_bf
     else router_logits_kernel<32><<<grid, kRsThreads, RsCfg<32>::kSmem, s>>>(m_w, m_x, q);
     if ((rc = launch_status())) return rc;
     const RouterSelParams r{reinterpret_cast<const __nv_bfloat16 *>(x), w_router, bias, ids, w, T, H, E,
-                            c->n_groups, c->topk_groups, c->topk, c->group_topn, P.S, part, list, list_n, exact};
+                            c->n_groups, c->topk_groups, c->topk, c->group_topn, P.S, part, list, list_n, exact,
+                            bcnt, reinterpret_cast<int32_t *>(scratch + P.bucket),
+                            reinterpret_cast<float *>(scratch + P.xlogit), scratch + P.listed};
     router_screen_kernel<<<static_cast<unsigned>((T + 7) / 8), 256, 0, s>>>(r);
     if ((rc = launch_status())) return rc;
-    // the listed tokens' CTAs first (they start early and overlap the refinement), then one warp per token
+    // the listed tokens' CTAs first (they start early and overlap the picks), then one persistent CTA per
+    // SM for the screened picks
     const int n_chunk = (E + 31) / 32;
     const int n_exact = n_chunk * static_cast<int>(std::min<int64_t>((T + 7) / 8, 64));
-    router_exact_kernel<<<static_cast<unsigned>(n_exact + (T + 7) / 8), 256, kRsPathSmem, s>>>(r, exact, n_exact);
+    router_exact_kernel<<<static_cast<unsigned>(n_exact + sms), 256, kRsPathSmem, s>>>(r, exact, n_exact);
     if ((rc = launch_status())) return rc;
-    router_list_select_kernel<<<static_cast<unsigned>(std::min<int64_t>((T + 7) / 8, 2 * sms)), 256, 0, s>>>(r);
+    router_finish_kernel<<<static_cast<unsigned>((T + 7) / 8), 256, 0, s>>>(r);  // list_n <= T
     return launch_status();
 }
 

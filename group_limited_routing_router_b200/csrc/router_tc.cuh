@@ -17,13 +17,14 @@
 //      both margins are at least kRsMargin, the chosen set is the one exact FP32 values give (the
 //      screened values are within 2e-5 of them, so a set decided by more than 4 times that cannot
 //      change).  Other tokens go to a list;
-//   4. router_exact_kernel, one launch: for each screened token (a warp each), the exact FP32
-//      projections of the chosen experts in the direct router's order (8 K ranges, each a sequential
-//      fused multiply-add chain over ascending k, summed in rank order), ordered and normalised as
-//      router_topk_kernel does; for the listed tokens (eight per CTA), every expert's exact projection
-//      in the same order;
-//   5. router_list_select_kernel: the selection on the listed tokens' projections, as in
-//      router_topk_kernel.
+//   4. router_exact_kernel, one launch: the exact FP32 projections in the direct router's order (8 K
+//      ranges, each a sequential fused multiply-add chain over ascending k, summed in rank order), for
+//      the screened tokens' picks (the screen appends each pick to its expert's bucket; a CTA takes
+//      an expert's picks 64 at a time, so the expert's row of W_r is staged once per 64 picks and
+//      only the tokens' bf16 rows stream per pick) and, for the listed tokens (eight per CTA), onto
+//      every expert;
+//   5. router_finish_kernel: the screened tokens' picks ordered and normalised from their exact
+//      projections, and the selection on the listed tokens' projections, as router_topk_kernel does.
 // Every output therefore equals router_topk_kernel's.
 #pragma once
 
@@ -296,6 +297,10 @@ struct RouterSelParams {
     int32_t *list;           // [T] tokens for the exact path
     int32_t *list_n;         // their count
     const float *exact;      // [T][E] exact projections of the listed tokens (by list position)
+    int32_t *bcnt;           // [E] picks in each expert's bucket (zeroed before the screen)
+    int32_t *bucket;         // [E][T] the screened picks t * topk + slot, per expert, in any order
+    float *xlogit;           // [T][topk] exact projection of each screened pick
+    uint8_t *listed;         // [T] 1: the token takes the exact path (written by the screen for every token)
 };
 
 // sigmoid score and selection value of expert e from its projection (as router_topk_kernel)
@@ -307,8 +312,9 @@ __device__ __forceinline__ void score_of(float logit, int e, const RouterSelPara
 }
 
 // One warp per token: the selection on the screened projections.  A token decided by both margins
-// keeps its picks in ids[t] (for router_refine_kernel); any other is listed for the exact path and
-// marked ids[t][0] = -1.
+// keeps its picks in ids[t] and appends each to its expert's bucket (for exact_picks and
+// router_finish_kernel); any other is listed for the exact path, flagged in listed[t], and its ids are
+// marked -1.
 __global__ void __launch_bounds__(256) router_screen_kernel(const RouterSelParams p) {
     const int lane = threadIdx.x & 31;
     const int64_t t = blockIdx.x * 8LL + (threadIdx.x >> 5);
@@ -334,152 +340,139 @@ __global__ void __launch_bounds__(256) router_screen_kernel(const RouterSelParam
     select_group_limited(sc, sel, lane, p.E, p.G, p.topk_groups, p.topk, p.group_topn, my_id, my_s, den, margins);
     const bool certain = margins[0] >= kRsMargin && margins[1] >= kRsMargin;  // NaN margins are not
     if (!certain && lane == 0) p.list[atomicAdd(p.list_n, 1)] = static_cast<int32_t>(t);
-    if (lane < p.topk) p.ids[t * p.topk + lane] = certain ? my_id : -1;
+    if (lane == 0) p.listed[t] = certain ? 0 : 1;
+    if (lane < p.topk) {
+        p.ids[t * p.topk + lane] = certain ? my_id : -1;
+        if (certain) {
+            const int pos = atomicAdd(p.bcnt + my_id, 1);  // < T: a token picks an expert at most once
+            p.bucket[static_cast<int64_t>(my_id) * p.T + pos] = static_cast<int32_t>(t * p.topk + lane);
+        }
+    }
 }
 
 // ---- exact path: one launch, two kinds of CTAs ------------------------------------------------------
-// The first kRsExactCtas-many CTAs (blockIdx.x < n_exact) project the listed tokens onto every expert,
-// eight tokens at a time (exact_batch); the rest refine the screened tokens, one warp per token
-// (refine_token).  Both stage their operands with an NS-deep cp.async ring.
+// The first n_exact CTAs project the listed tokens onto every expert, eight tokens at a time
+// (exact_batch); the rest (one per SM, persistent) take the screened picks expert by expert, 64 at a
+// time (exact_picks).  Both stage their operands with a cp.async ring.
 
-constexpr int kRsRefineStages = 3;
-constexpr int kRsRefineW = 64 * 32;                          // 64 segments of 32 fp32, 16-byte chunks XOR-swizzled
-constexpr int kRsRefineStage = kRsRefineW + 8 * kRsXWords;   // + x's eight rank segments (padded)
-constexpr int kRsRefineWarpWords = kRsRefineStages * kRsRefineStage;
 constexpr int kRsExactStages = 4;
 constexpr int kRsExactW = 256 * kRsSegWords, kRsExactX = 8 * 8 * kRsXWords, kRsExactBuf = kRsExactW + kRsExactX;
 constexpr int kRsExactWords = kRsExactStages * kRsExactBuf + 8 * 256;
-constexpr int kRsPathSmem = (8 * kRsRefineWarpWords > kRsExactWords ? 8 * kRsRefineWarpWords : kRsExactWords) * 4;
-static_assert(kRsPathSmem <= 232448, "shared memory per CTA");
 
-// One warp: the picks' exact projections of screened token t in the direct router's order (lane l runs
-// the chains of pick l / 4, ranks r0 = 2 (l % 4) and r0 + 1), then the order and the weights exactly as
-// the direct router.  Per 32-k step the warp stages the picks' eight rank segments of W_r (segment
-// (chain, lane), 16-byte chunk c stored at c ^ (lane % 8)) and x's eight rank segments.
-__device__ __forceinline__ void refine_token(const RouterSelParams &p, int64_t t, uint32_t *wbuf, int lane) {
-    const int my_id = lane < p.topk ? p.ids[t * p.topk + lane] : 0;
-    if (__shfl_sync(0xffffffffu, my_id, 0) < 0) return;  // listed for the exact path
-    int e_of[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) e_of[j] = __shfl_sync(0xffffffffu, my_id, j < p.topk ? j : 0);
-    const int pick = lane >> 2, r0 = 2 * (lane & 3);
-    const int e_pick = __shfl_sync(0xffffffffu, my_id, pick < p.topk ? pick : 0);
-    // rank ranges this lane touches: its W copies (ranks 2 (lane / 8) and + 1), its x copy (rank
-    // lane / 4) and its chains (r0, r0 + 1)
+constexpr int kRxPicks = 64;                      // picks per item
+constexpr int kRxStages = 4;
+constexpr int kRxX = 8 * kRxPicks * kRsXWords;    // x segments [rank][pick][20 words]: 16-byte reads of 8 lanes hit distinct banks
+constexpr int kRxW = 8 * 32;                      // the expert's W_r segments [rank][32 fp32]
+constexpr int kRxBuf = kRxX + kRxW;
+constexpr int kRxWords = kRxStages * kRxBuf + 8 * kRxPicks + 2 * kRxPicks + kRtSlots + 1;
+
+constexpr int kRsPathSmem = (kRxWords > kRsExactWords ? kRxWords : kRsExactWords) * 4;
+static_assert(kRsPathSmem <= 232448, "shared memory per CTA");
+static_assert(kRxBuf % 4 == 0 && kRxX % 4 == 0, "16-byte aligned staging");
+
+__device__ __forceinline__ uint4 lds_u4(const uint32_t *base, int word) {
+    return *reinterpret_cast<const uint4 *>(base + word);
+}
+
+// Persistent CTA `cta` of `n_ctas`: items (expert e, chunk c) = picks 64 c .. 64 c + 63 of e's bucket.
+// Warp r runs rank r's chains; lane q the picks q and q + 32.  Per 32-k step the CTA stages the
+// expert's eight W_r segments and the picks' eight x segments each; the rank sums go to xlogit in
+// rank order, exactly as the direct router forms them.
+__device__ __forceinline__ void exact_picks(const RouterSelParams &p, uint32_t *smem, int cta, int n_ctas) {
+    float *partial = reinterpret_cast<float *>(smem + kRxStages * kRxBuf);  // [pick][rank]
+    int32_t *rows = reinterpret_cast<int32_t *>(partial + 8 * kRxPicks);    // token of each pick
+    int32_t *ent = rows + kRxPicks;                                         // pick entry t * topk + slot
+    int *tile_start = ent + kRxPicks;                                       // item prefix [E + 1]
+    const int tid = threadIdx.x, r = tid >> 5, q = tid & 31;
+    item_prefix(p.bcnt, p.E, 1, kRxPicks, tile_start);
+    __syncthreads();
+    const int total = tile_start[p.E];
     const int n_steps = (p.H / kRtBK + kRtCluster - 1) / kRtCluster;
-    int wk0[2], wlen[2], xk0, xlen, len0, len1;
+    int ck0, clen;
+    rank_range(p.H, r, ck0, clen);
+    clen -= ck0;
+    // copies: x part tid % 4 of pick tid / 4 for every rank; W: rank tid / 8, part tid % 8 (tid < 64)
+    const int xp = tid >> 2, xpart = tid & 3;
+    int xk0[kRtCluster], xlen[kRtCluster];
 #pragma unroll
-    for (int c = 0; c < 2; ++c) {
-        int a, b;
-        rank_range(p.H, 2 * (lane >> 3) + c, a, b);
-        wk0[c] = a;
-        wlen[c] = b - a;
+    for (int rr = 0; rr < kRtCluster; ++rr) {
+        rank_range(p.H, rr, xk0[rr], xlen[rr]);
+        xlen[rr] -= xk0[rr];
     }
-    {
-        int a, b;
-        rank_range(p.H, lane >> 2, a, b);
-        xk0 = a;
-        xlen = b - a;
-        rank_range(p.H, r0, a, b);
-        len0 = b - a;
-        rank_range(p.H, r0 + 1, a, b);
-        len1 = b - a;
+    int wk0 = 0, wlen = 0;
+    if (tid < 64) {
+        rank_range(p.H, tid >> 3, wk0, wlen);
+        wlen -= wk0;
     }
-    // this lane's copy addresses, fixed over the steps: W chunk i = pick i % 8, rank 2 (lane / 8) + i / 8,
-    // 16-byte part lane % 8 (source row start and shared-memory offset); x: rank lane / 4, part lane % 4
-    const int part = lane & 7;
-    const float *wsrc[8];
+    const uint32_t ring = smem_u32(smem);
+    for (int item = cta; item < total; item += n_ctas) {
+        int lo = 0, hi = p.E - 1;  // largest e with tile_start[e] <= item
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (tile_start[mid] <= item) lo = mid;
+            else hi = mid - 1;
+        }
+        const int e = lo, c = item - tile_start[e];
+        const int n = min(kRxPicks, p.bcnt[e] - c * kRxPicks);
+        if (tid < kRxPicks) {
+            const int32_t en = tid < n ? p.bucket[static_cast<int64_t>(e) * p.T + c * kRxPicks + tid] : -1;
+            ent[tid] = en;
+            rows[tid] = en >= 0 ? en / p.topk : 0;
+        }
+        __syncthreads();
+        const bool xon = xp < n;
+        const __nv_bfloat16 *xsrc = p.x + static_cast<int64_t>(rows[xp]) * p.H + 8 * xpart;
+        const float *wsrc = p.w + static_cast<int64_t>(e) * p.H + wk0 + 4 * (tid & 7);
+        auto issue = [&](int st) {  // stage st into ring slot st % kRxStages; always one commit group
+            if (st < n_steps) {
+                const uint32_t buf = ring + static_cast<uint32_t>((st % kRxStages) * kRxBuf * 4);
+                const int k = 32 * st;
+                if (xon) {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) wsrc[j] = p.w + static_cast<int64_t>(e_of[j]) * p.H + 4 * part;
-    uint32_t wdst[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const int j = i & 7, c = i >> 3, seg = c * 32 + 4 * j + (lane >> 3);
-        wdst[i] = static_cast<uint32_t>((seg * 32 + 4 * (part ^ (seg & 7))) * 4);
-    }
-    const __nv_bfloat16 *xsrc = p.x + t * p.H + xk0 + 8 * (lane & 3);
-    const uint32_t xdst = static_cast<uint32_t>((kRsRefineW + (lane >> 2) * kRsXWords + 4 * (lane & 3)) * 4);
-    const uint32_t ring = smem_u32(wbuf);
-    auto issue = [&](int st) {  // stage st into ring slot st % NS; always one commit group
-        if (st < n_steps) {
-            const uint32_t buf = ring + static_cast<uint32_t>((st % kRsRefineStages) * kRsRefineStage * 4);
-            const int k = 32 * st;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const int j = i & 7, c = i >> 3;
-                if (j < p.topk && k < wlen[c]) cp_async16(buf + wdst[i], wsrc[j] + wk0[c] + k);
+                    for (int rr = 0; rr < kRtCluster; ++rr)
+                        if (k < xlen[rr])
+                            cp_async16(buf + static_cast<uint32_t>(((rr * kRxPicks + xp) * kRsXWords + 4 * xpart) * 4),
+                                       xsrc + xk0[rr] + k);
+                }
+                if (tid < 64 && k < wlen)
+                    cp_async16(buf + static_cast<uint32_t>((kRxX + (tid >> 3) * 32 + 4 * (tid & 7)) * 4), wsrc + k);
             }
-            if (k < xlen) cp_async16(buf + xdst, xsrc + k);
-        }
-        cp_async_commit();
-    };
-    float part0 = 0.0f, part1 = 0.0f;
+            cp_async_commit();
+        };
+        float a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
-    for (int st = 0; st < kRsRefineStages - 1; ++st) issue(st);
-    for (int st = 0; st < n_steps; ++st) {
-        issue(st + kRsRefineStages - 1);
-        cp_async_wait<kRsRefineStages - 1>();
-        __syncwarp();
-        if (pick < p.topk) {
-            const uint32_t *cur = wbuf + (st % kRsRefineStages) * kRsRefineStage;
-            const uint32_t *w0 = cur + lane * 32, *w1 = cur + (32 + lane) * 32;
-            const uint32_t *x0 = cur + kRsRefineW + r0 * kRsXWords, *x1 = x0 + kRsXWords;
-            const bool on0 = 32 * st < len0, on1 = 32 * st < len1;
+        for (int st = 0; st < kRxStages - 1; ++st) issue(st);
+        for (int st = 0; st < n_steps; ++st) {
+            issue(st + kRxStages - 1);
+            cp_async_wait<kRxStages - 1>();
+            __syncthreads();
+            if (32 * st < clen) {
+                const uint32_t *cur = smem + (st % kRxStages) * kRxBuf;
+                const uint32_t *wr = cur + kRxX + r * 32;
+                const uint32_t *x0 = cur + (r * kRxPicks + q) * kRsXWords, *x1 = x0 + 32 * kRsXWords;
 #pragma unroll
-            for (int kk = 0; kk < 32; kk += 4) {
-                const int ch = 4 * ((kk >> 2) ^ (lane & 7));
-                if (on0) part0 = fma4(lds_f4(w0, ch), lds_u2(x0, kk / 2), part0);
-                if (on1) part1 = fma4(lds_f4(w1, ch), lds_u2(x1, kk / 2), part1);
+                for (int kk = 0; kk < 32; kk += 8) {
+                    const float4 wlo = lds_f4(wr, kk), whi = lds_f4(wr, kk + 4);
+                    const uint4 v0 = lds_u4(x0, kk / 2), v1 = lds_u4(x1, kk / 2);
+                    a0 = fma4(wlo, make_uint2(v0.x, v0.y), a0);
+                    a0 = fma4(whi, make_uint2(v0.z, v0.w), a0);
+                    a1 = fma4(wlo, make_uint2(v1.x, v1.y), a1);
+                    a1 = fma4(whi, make_uint2(v1.z, v1.w), a1);
+                }
             }
+            __syncthreads();
         }
-        __syncwarp();
-    }
-    cp_async_wait<0>();
-    // sum in rank order (every lane of the pick's group of four forms the same value)
-    float logit = 0.0f;
+        cp_async_wait<0>();
+        partial[q * 8 + r] = a0;
+        partial[(q + 32) * 8 + r] = a1;
+        __syncthreads();
+        if (tid < n) {  // the ranks in order
+            float l = 0.0f;
 #pragma unroll
-    for (int r = 0; r < kRtCluster; ++r) {
-        const float a = __shfl_sync(0xffffffffu, part0, (lane & ~3) | (r >> 1));
-        const float b = __shfl_sync(0xffffffffu, part1, (lane & ~3) | (r >> 1));
-        logit += (r & 1) ? b : a;
-    }
-    float s_p, sel_p;
-    score_of(logit, e_pick, p, s_p, sel_p);
-    // order the picks by (selection value desc, expert asc) and normalise in that order
-    float sv[8], ss[8];
-    int ev[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        sv[j] = __shfl_sync(0xffffffffu, sel_p, 4 * j);
-        ss[j] = __shfl_sync(0xffffffffu, s_p, 4 * j);
-        ev[j] = __shfl_sync(0xffffffffu, e_pick, 4 * j);
-    }
-    float s_slot = 0.0f, den = 0.0f;
-    int e_slot = 0;
-    for (int r = 0; r < p.topk; ++r) {  // slot r holds the pick with exactly r picks ahead of it
-        float s_r = 0.0f;
-        int e_r = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            if (j >= p.topk) continue;
-            int ahead = 0;
-#pragma unroll
-            for (int i = 0; i < 8; ++i)
-                if (i < p.topk && (sv[i] > sv[j] || (sv[i] == sv[j] && ev[i] < ev[j]))) ++ahead;
-            if (ahead == r) {
-                s_r = ss[j];
-                e_r = ev[j];
-            }
+            for (int rr = 0; rr < kRtCluster; ++rr) l += partial[tid * 8 + rr];
+            p.xlogit[ent[tid]] = l;
         }
-        den = den + s_r;
-        if (lane == r) {
-            s_slot = s_r;
-            e_slot = e_r;
-        }
-    }
-    if (lane < p.topk) {
-        p.ids[t * p.topk + lane] = e_slot;
-        p.wts[t * p.topk + lane] = s_slot / den;
+        __syncthreads();
     }
 }
 
@@ -568,7 +561,7 @@ __device__ __forceinline__ void exact_batch(const RouterSelParams &p, float *exa
 }
 
 // blockIdx.x < n_exact: exact_batch over (expert chunk blockIdx.x % n_chunk, batches blockIdx.x / n_chunk
-// + k n_exact / n_chunk); the rest: refine_token, one warp per token.
+// + k n_exact / n_chunk); the rest: exact_picks, persistent.
 __global__ void __launch_bounds__(256, 1) router_exact_kernel(const RouterSelParams p, float *exact, int n_exact) {
     extern __shared__ __align__(16) uint32_t rs_path_smem[];
     if (static_cast<int>(blockIdx.x) < n_exact) {
@@ -578,31 +571,72 @@ __global__ void __launch_bounds__(256, 1) router_exact_kernel(const RouterSelPar
         for (int bt = blockIdx.x / n_chunk; bt < (n + 7) / 8; bt += slots) exact_batch(p, exact, n, bt, 32 * chunk, rs_path_smem);
         return;
     }
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t t = (blockIdx.x - n_exact) * 8LL + warp;
-    if (t < p.T) refine_token(p, t, rs_path_smem + warp * kRsRefineWarpWords, lane);
+    exact_picks(p, rs_path_smem, static_cast<int>(blockIdx.x) - n_exact, static_cast<int>(gridDim.x) - n_exact);
 }
 
-// The selection of router_topk_kernel on the listed tokens' exact projections: one warp per entry.
-__global__ void __launch_bounds__(256) router_list_select_kernel(const RouterSelParams p) {
-    const int lane = threadIdx.x & 31;
-    const int n = *p.list_n;
-    for (int i = blockIdx.x * 8 + (threadIdx.x >> 5); i < n; i += gridDim.x * 8) {
-        const int64_t t = p.list[i];
-        float sc[8], sel[8];
+// One warp: the selection of router_topk_kernel for listed token list[i] on its exact projections.
+__device__ __noinline__ void list_select(const RouterSelParams &p, int64_t i, int lane) {
+    const int64_t t = p.list[i];
+    float sc[8], sel[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const int e = lane + 32 * j;
-            score_of(e < p.E ? p.exact[static_cast<int64_t>(i) * p.E + e] : 0.0f, e, p, sc[j], sel[j]);
-        }
-        float den, my_s;
-        int my_id;
-        select_group_limited(sc, sel, lane, p.E, p.G, p.topk_groups, p.topk, p.group_topn, my_id, my_s, den, nullptr);
-        if (lane < p.topk) {
-            p.ids[t * p.topk + lane] = my_id;
-            p.wts[t * p.topk + lane] = my_s / den;
+    for (int j = 0; j < 8; ++j) {
+        const int e = lane + 32 * j;
+        score_of(e < p.E ? p.exact[i * p.E + e] : 0.0f, e, p, sc[j], sel[j]);
+    }
+    float den, my_s;
+    int my_id;
+    select_group_limited(sc, sel, lane, p.E, p.G, p.topk_groups, p.topk, p.group_topn, my_id, my_s, den, nullptr);
+    if (lane < p.topk) {
+        p.ids[t * p.topk + lane] = my_id;
+        p.wts[t * p.topk + lane] = my_s / den;
+    }
+}
+
+// The selection of router_topk_kernel from exact projections, one warp per global warp index g:
+//   (a) screened token g (lane j holds pick j): the picks ordered by (selection value desc, expert asc)
+//       from their exact projections and normalised in that order;
+//   (b) listed token list[g]: the full selection on its projections onto every expert.
+// (a) skips the listed tokens by their flag, not by their ids: (b) of another warp may be writing
+// those ids meanwhile.
+__global__ void __launch_bounds__(256) router_finish_kernel(const RouterSelParams p) {
+    const int lane = threadIdx.x & 31;
+    const int64_t g = blockIdx.x * 8LL + (threadIdx.x >> 5);
+    if (g < p.T && !p.listed[g]) {
+        const int64_t t = g;
+        const int my_id = lane < p.topk ? p.ids[t * p.topk + lane] : 0;
+        {
+            float s_p = 0.0f, sel_p = -INFINITY;
+            if (lane < p.topk) score_of(p.xlogit[t * p.topk + lane], my_id, p, s_p, sel_p);
+            // this pick's slot: the picks ahead of it (the order is total: the experts differ)
+            int ahead = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float sv = __shfl_sync(0xffffffffu, sel_p, i);
+                const int ev = __shfl_sync(0xffffffffu, my_id, i);
+                if (i < p.topk && (sv > sel_p || (sv == sel_p && ev < my_id))) ++ahead;
+            }
+            // lane r takes the pick of slot r; the denominator sums the slots in order
+            float s_slot = 0.0f;
+            int e_slot = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int a = __shfl_sync(0xffffffffu, ahead, i);
+                const float sv = __shfl_sync(0xffffffffu, s_p, i);
+                const int ev = __shfl_sync(0xffffffffu, my_id, i);
+                if (i < p.topk && a == lane) {
+                    s_slot = sv;
+                    e_slot = ev;
+                }
+            }
+            float den = 0.0f;
+            for (int r = 0; r < p.topk; ++r) den = den + __shfl_sync(0xffffffffu, s_slot, r);
+            if (lane < p.topk) {
+                p.ids[t * p.topk + lane] = e_slot;
+                p.wts[t * p.topk + lane] = s_slot / den;
+            }
         }
     }
+    if (g < *p.list_n) list_select(p, g, lane);
 }
 
 }  // namespace beam

@@ -57,13 +57,16 @@ def test_workspace_sizes(L):
 def test_screened_route_workspace(L):
     """The screened router's scratch: none below 2048 tokens (the direct router runs); from 2048 the
     three bf16 planes of W_r, the split partial projections, the exact-path list and its projections,
-    and the forward workspace holds it."""
+    the per-expert buckets of the screened picks and their exact projections; the forward workspace
+    holds it."""
     c = _cfg()
     E, H = 256, 5120
     assert bm.workspace_size(c, 2047, bm.WS_ROUTE_SCREENED) == 0
     for T in (2048, 4096, 65536):
         n = bm.workspace_size(c, T, bm.WS_ROUTE_SCREENED)
-        assert n >= 3 * E * H * 2 + T * E * 4 * 2 + T * 4  # planes + >= one split + exact projections + list
+        # planes + >= one split + the listed tokens' projections + the list + the per-expert buckets of
+        # the screened picks + their exact projections
+        assert n >= 3 * E * H * 2 + T * E * 4 * 2 + T * 4 + T * E * 4 + T * 8 * 4
         assert bm.workspace_size(c, T, bm.WS_FORWARD) > n
     assert bm.workspace_size(_cfg(topk=9, topk_groups=8), 4096, bm.WS_ROUTE_SCREENED) == 0  # k > 8: direct
 

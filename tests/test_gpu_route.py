@@ -132,6 +132,25 @@ def test_screened_route_ties_ragged_and_nan():
         assert int(ids.min()) >= 0 and int(ids.max()) < wl.n_experts
 
 
+@pytest.mark.parametrize("name,T", [("tiny", 2048), ("mid_a", 2500), ("mid_b", 4099), ("mid_c", 2083),
+                                    ("mid_skew", 3000)])
+def test_screened_path_equals_direct_mid_configs(name, T):
+    """The screened kernels themselves (they run from 2048 tokens) on the layouts the Beam workloads do
+    not have: 16-64 experts, top-4 / top-6 / top-8, group_topn = 3, unequal K ranks (H = 320 makes
+    ranks of one and two 32-wide steps), a stored selection bias; with all-zero, duplicated and NaN
+    rows and a ragged T."""
+    wl = bs.get(name)
+    case = parity.Case(wl, T=T)
+    x = case.x.clone()
+    x[::97] = 0
+    x[1] = x[2]
+    x[5, 3] = float("nan")
+    ids, _ = _same_routing(case, x)
+    assert int(ids.min()) >= 0 and int(ids.max()) < wl.n_experts
+    ws = bm.workspace_size(case.layer, T, bm.WS_ROUTE_SCREENED)
+    assert ws > 0, "the screened path must be the one under test"
+
+
 def test_forward_routes_like_the_direct_router(bank):
     case = bank.case("prefill")
     _, ids, w = bm.forward(case.layer, case.x, case.w_router, case.bias, case.wg, case.wu, case.wd,
