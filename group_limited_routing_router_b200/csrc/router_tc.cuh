@@ -443,9 +443,11 @@ __device__ __forceinline__ void exact_picks(const RouterSelParams &p, uint32_t *
 #pragma unroll
         for (int st = 0; st < kRxStages - 1; ++st) issue(st);
         for (int st = 0; st < n_steps; ++st) {
-            issue(st + kRxStages - 1);
-            cp_async_wait<kRxStages - 1>();
+            // stage st has landed for every thread, and every thread is done with stage st - 1, whose
+            // slot the refill below takes: one barrier per step
+            cp_async_wait<kRxStages - 2>();
             __syncthreads();
+            issue(st + kRxStages - 1);
             if (32 * st < clen) {
                 const uint32_t *cur = smem + (st % kRxStages) * kRxBuf;
                 const uint32_t *wr = cur + kRxX + r * 32;
@@ -460,7 +462,6 @@ __device__ __forceinline__ void exact_picks(const RouterSelParams &p, uint32_t *
                     a1 = fma4(whi, make_uint2(v1.z, v1.w), a1);
                 }
             }
-            __syncthreads();
         }
         cp_async_wait<0>();
         partial[q * 8 + r] = a0;
