@@ -183,18 +183,24 @@ __device__ __forceinline__ void swiglu_to_regs(uint32_t t0, uint32_t t1, int sub
         }
     }
 }
-// The h values of swiglu_to_regs: weight row m (< M) of the item's tokens.
+__device__ __forceinline__ void st_b16_hint(uint16_t *addr, uint16_t v, uint64_t policy) {
+    asm volatile("st.global.L2::cache_hint.b16 [%0], %1, %2;" ::"l"(addr), "h"(v), "l"(policy) : "memory");
+}
+// The h values of swiglu_to_regs: weight row m (< M) of the item's tokens.  Stored L2-evict-last: the
+// down projection reads h right after this launch, and lines that stay in L2 are neither re-read from
+// DRAM there nor written back in the middle of this launch's weight stream (evict-first).
 template <int BN>
 __device__ __forceinline__ void store_h_regs(const GemmParams &p, const Item &it, int sub, int m,
                                              const uint32_t (&hv)[(BN + 31) / 32][8]) {
     const int64_t ld = p.M;
     uint16_t *h = reinterpret_cast<uint16_t *>(p.out) + (it.row0 + 16 * sub) * ld + m;
+    const uint64_t pol = policy_evict_last();
 #pragma unroll
     for (int i = 0; i < (BN + 31) / 32; ++i) {
         const int left = it.n_valid - (16 * sub + 32 * i);  // valid columns from this chunk on
 #pragma unroll
         for (int j = 0; j < 16; ++j)
-            if (j < left) h[(32 * i + j) * ld] = static_cast<uint16_t>(hv[i][j >> 1] >> (16 * (j & 1)));
+            if (j < left) st_b16_hint(h + (32 * i + j) * ld, static_cast<uint16_t>(hv[i][j >> 1] >> (16 * (j & 1))), pol);
     }
 }
 
