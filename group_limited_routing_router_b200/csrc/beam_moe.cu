@@ -76,6 +76,9 @@ constexpr int k2smBox = 32;
 // Block-scaled FP8 variants (tcgen05 kind::mxf8f6f4): <gate/up?, BN, B box rows, stages (K = 128),
 // TMEM slots, slot columns, gather?>; each stage also holds its scale atoms and TMEM scale columns.
 #define G1_WIDE_MX8_ARGS true, 192, 64, 3, 2, 192, false, false
+// 160-token gate/up tiles with a fourth stage, for batches whose experts mostly fit one such tile
+// (prefill); TMEM: 2 x 160 accumulator columns + 4 x 16 scale columns.
+#define G1_WIDE_MX8_160_ARGS true, 160, 32, 4, 2, 160, false, false
 #define G2_WIDE_MX8_ARGS false, 192, 64, 5, 2, 192, false, false
 #define G1_NARROW_MX8_ARGS true, 32, 1, 5, 4, 64, true, false
 #define G2_NARROW_MX8_ARGS false, 32, 32, 10, 4, 32, false, false
@@ -218,6 +221,7 @@ int init_device(int *dev_out) {
         ok = ok && set_gemm_fp8_smem<G1_WIDE_NV4_ARGS>() && set_gemm_fp8_smem<G2_WIDE_NV4_ARGS>() &&
              set_gemm_fp8_smem<G1_NARROW_NV4_ARGS>() && set_gemm_fp8_smem<G2_NARROW_NV4_ARGS>();
         ok = ok && set_gemm_mx8_smem<G1_WIDE_MX8_ARGS>() && set_gemm_mx8_smem<G2_WIDE_MX8_ARGS>() &&
+             set_gemm_mx8_smem<G1_WIDE_MX8_160_ARGS>() &&
              set_gemm_mx8_smem<G1_NARROW_MX8_ARGS>() && set_gemm_mx8_smem<G2_NARROW_MX8_ARGS>();
         ok = ok && set_gemm_mx8_smem<G1_WIDE_NV4X_ARGS>() && set_gemm_mx8_smem<G2_WIDE_NV4X_ARGS>() &&
              set_gemm_mx8_smem<G1_WIDE_NV4X_160_ARGS>() && set_gemm_mx8_smem<G2_WIDE_NV4X_160_ARGS>() &&
@@ -707,6 +711,7 @@ int enqueue_experts_mx8(const beam_moe_config *c, int dev, int64_t T, const beam
     if (!record(ev, 3, s)) return BEAM_MOE_ERR_CUDA;
 
     const double mean_rows = static_cast<double>(R) / E;
+    const bool big = !narrow && mean_rows + 2.0 * std::sqrt(mean_rows) <= 160;  // G1_WIDE_MX8_160
     const int bn = narrow ? kNarrowBN : kWideBN;
     const int box = narrow ? kNarrowBox : kWideBox;
     const int once = (mean_rows + 4.0 * std::sqrt(mean_rows) <= bn) ? 1 : 0;
@@ -714,8 +719,8 @@ int enqueue_experts_mx8(const beam_moe_config *c, int dev, int64_t T, const beam
     if (!encode_fn()) return BEAM_MOE_ERR_CUDA;
     const bool b1_ok = narrow ? make_map_2d_any(&m_b1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws + L.xq, H,
                                                 static_cast<uint64_t>(T), kMxBK, 1, CU_TENSOR_MAP_SWIZZLE_128B)
-                              : make_map_2d_any(&m_b1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws + L.xqp, H, R, kMxBK, box,
-                                                CU_TENSOR_MAP_SWIZZLE_128B);
+                              : make_map_2d_any(&m_b1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws + L.xqp, H, R, kMxBK,
+                                                big ? 32 : box, CU_TENSOR_MAP_SWIZZLE_128B);
     if (!b1_ok ||
         !make_map_2d_any(&m_b2, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, ws + L.hq, I, R, kMxBK, box, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map_3d_fp8(&m_wg, W->w_gate, H, I, E) || !make_map_3d_fp8(&m_wu, W->w_up, H, I, E) ||
@@ -728,6 +733,7 @@ int enqueue_experts_mx8(const beam_moe_config *c, int dev, int64_t T, const beam
     Mx8Params p2{counts, offsets, E, I, H, once, kDefaultTimeoutCycles, row_src, k, ws + L.hs, 0, nullptr, nullptr,
                  reinterpret_cast<__nv_bfloat16 *>(ws + L.o), nullptr, nullptr, nullptr};
     if (narrow) launch_gemm_mx8<G1_NARROW_MX8_ARGS>(grid, s, m_wg, m_wu, m_sg, m_su, m_b1, p1);
+    else if (big) launch_gemm_mx8<G1_WIDE_MX8_160_ARGS>(grid, s, m_wg, m_wu, m_sg, m_su, m_b1, p1);
     else launch_gemm_mx8<G1_WIDE_MX8_ARGS>(grid, s, m_wg, m_wu, m_sg, m_su, m_b1, p1);
     if ((rc = launch_status())) return rc;
     if (!record(ev, 4, s)) return BEAM_MOE_ERR_CUDA;

@@ -72,8 +72,11 @@ struct Mx8GemmCfg {
     static constexpr int kSfCol = NSLOT * SLOT_COLS;       // first TMEM scale column
     static constexpr int kTmemCols = 512;
     static constexpr int kBarOff = STAGES * kStage;
-    static constexpr int kTokOff = kBarOff + 512 + 4 * (kPmMaxE + 1);
-    static constexpr int kEpiOff = (kTokOff + 4 * BN + 15) / 16 * 16;  // gate/up epilogue: per-warp staging of h~
+    // full / sf_ready / empty per stage, acc_full / acc_empty per slot, drain, then the TMEM address
+    static constexpr int kBarBytes = ((3 * STAGES + 2 * NSLOT + 1) * 8 + 4 + 15) / 16 * 16;
+    static constexpr int kTileOff = kBarOff + kBarBytes;                 // item prefix [E + 1]
+    static constexpr int kTokOff = kTileOff + 4 * (kPmMaxE + 1);         // GATHER: token of each row [BN]
+    static constexpr int kEpiOff = (kTokOff + (GATHER ? 4 * BN : 0) + 15) / 16 * 16;  // gate/up epilogue: per-warp staging of h~
     static constexpr int kEpiWarp = GATE_UP ? 16 * 32 + 16 * 2 : 0;     // 16 columns x (32 code bytes + 2 scale bytes)
     static constexpr int kSmem = 1024 + kEpiOff + kMxEpiWarps * kEpiWarp + 64;
     static_assert(kA % 1024 == 0 && kB % 1024 == 0 && (GATHER || kBox % 1024 == 0), "swizzled tiles");
@@ -82,7 +85,6 @@ struct Mx8GemmCfg {
     static_assert(kSfCol + STAGES * kSfColsPerStage <= 512, "TMEM has 512 columns");
     static_assert(GATE_UP ? (BN <= SLOT_COLS && (NSLOT >= 2 || BN <= SLOT_COLS / 2)) : BN <= SLOT_COLS,
                   "an item must fit in its TMEM slots");
-    static_assert((3 * STAGES + 2 * NSLOT + 1) * 8 + 4 <= 512, "barriers");
     static_assert(kSmem + 256 <= 232448, "shared memory per CTA (dynamic + the kernel's static bytes)");
 };
 
@@ -455,7 +457,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     uint64_t *acc_empty = acc_full + NSLOT;
     uint64_t *drain = acc_empty + NSLOT;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
-    int *tile_start = reinterpret_cast<int *>(smem + C::kBarOff + 512);
+    int *tile_start = reinterpret_cast<int *>(smem + C::kTileOff);
     int *tok = reinterpret_cast<int *>(smem + C::kTokOff);  // GATHER: token of each row of the item
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
