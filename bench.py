@@ -51,22 +51,22 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 _CSRC = os.path.join(ROOT, "group_limited_routing_router_b200", "csrc")
 _BF16_SRC = ("gemm.cuh", "gemm_2sm.cuh", "common.cuh", "beam_moe.cu")  # beam_moe.cu picks the variants
 _MX_SRC = ("gemm_mx8.cuh", "gemm.cuh", "common.cuh", "beam_moe.cu")
-_H1, _H2 = "bc891c94d962858a", "014085b9b5167302"
+_H1, _H2 = "8bce63b08c7d3c3b", "6c2e5bcdaf853dd9"
 NCU_TRAFFIC = {
-    ("gate_up_swiglu", "decode"): {"bytes": 8 * (1678104576 + 1089792), "files": _BF16_SRC, "hash": _H1},
-    ("gate_up_swiglu", "prefill"): {"bytes": 8 * (1747472640 + 3496960), "files": _BF16_SRC, "hash": _H1},
-    ("gate_up_swiglu", "long"): {"bytes": 8 * (6969785856 + 329203456), "files": _BF16_SRC, "hash": _H1},
-    ("down", "decode"): {"bytes": 8 * (840216064 + 3835392), "files": _BF16_SRC, "hash": _H1},
-    ("down", "prefill"): {"bytes": 8 * (863825408 + 33734400), "files": _BF16_SRC, "hash": _H1},
-    ("down", "long"): {"bytes": 8 * (1386240000 + 1307799552), "files": _BF16_SRC, "hash": _H1},
-    ("gate_up_swiglu_w4a4", "decode"): {"bytes": 8 * (472057344 + 350208), "files": _MX_SRC, "hash": _H2},
-    ("gate_up_swiglu_w4a4", "prefill"): {"bytes": 8 * (483264512 + 3360256), "files": _MX_SRC, "hash": _H2},
-    ("down_w4a4", "decode"): {"bytes": 8 * (236354304 + 1206272), "files": _MX_SRC, "hash": _H2},
-    ("down_w4a4", "prefill"): {"bytes": 8 * (241892352 + 24786176), "files": _MX_SRC, "hash": _H2},
-    ("gate_up_swiglu_mxfp8", "decode"): {"bytes": 8 * (865319168 + 1263616), "files": _MX_SRC, "hash": _H2},
-    ("gate_up_swiglu_mxfp8", "prefill"): {"bytes": 8 * (890544896 + 1557760), "files": _MX_SRC, "hash": _H2},
-    ("down_mxfp8", "decode"): {"bytes": 8 * (433264384 + 1469440), "files": _MX_SRC, "hash": _H2},
-    ("down_mxfp8", "prefill"): {"bytes": 8 * (444304896 + 5500672), "files": _MX_SRC, "hash": _H2},
+    ("gate_up_swiglu", "decode"): {"bytes": 8 * (1678105600 + 444672), "files": _BF16_SRC, "hash": _H1},
+    ("gate_up_swiglu", "prefill"): {"bytes": 8 * (1746670592 + 3784448), "files": _BF16_SRC, "hash": _H1},
+    ("gate_up_swiglu", "long"): {"bytes": 8 * (7197129216 + 327750400), "files": _BF16_SRC, "hash": _H1},
+    ("down", "decode"): {"bytes": 8 * (840216064 + 3649280), "files": _BF16_SRC, "hash": _H1},
+    ("down", "prefill"): {"bytes": 8 * (863619584 + 32772608), "files": _BF16_SRC, "hash": _H1},
+    ("down", "long"): {"bytes": 8 * (1415222272 + 1311474432), "files": _BF16_SRC, "hash": _H1},
+    ("gate_up_swiglu_w4a4", "decode"): {"bytes": 8 * (472043776 + 725248), "files": _MX_SRC, "hash": _H2},
+    ("gate_up_swiglu_w4a4", "prefill"): {"bytes": 8 * (483464448 + 3374080), "files": _MX_SRC, "hash": _H2},
+    ("down_w4a4", "decode"): {"bytes": 8 * (236358144 + 952576), "files": _MX_SRC, "hash": _H2},
+    ("down_w4a4", "prefill"): {"bytes": 8 * (241892864 + 25118208), "files": _MX_SRC, "hash": _H2},
+    ("gate_up_swiglu_mxfp8", "decode"): {"bytes": 8 * (865337088 + 755456), "files": _MX_SRC, "hash": _H2},
+    ("gate_up_swiglu_mxfp8", "prefill"): {"bytes": 8 * (887574016 + 1698816), "files": _MX_SRC, "hash": _H2},
+    ("down_mxfp8", "decode"): {"bytes": 8 * (433264128 + 1815296), "files": _MX_SRC, "hash": _H2},
+    ("down_mxfp8", "prefill"): {"bytes": 8 * (444417280 + 5801472), "files": _MX_SRC, "hash": _H2},
 }
 
 
