@@ -360,7 +360,7 @@ def config_dict(wl):
 
 def launches_per_step(wl: bs.Workload, block: bool, fmt: str = "bf16") -> int:
     """Kernels one forward launches: the router (the direct kernel below 2048 tokens; from 2048 the
-    screened router's five: plane split, tensor-core projection, screen, exact path, list selection),
+    screened router's five: plane split, tensor-core projection, screen, exact path, finish),
     3 dispatch kernels, [row gather for wide tiles], [activation quantiser on the block-scaled paths],
     gate/up, down, combine; the sublayer adds the pre-norm (its combine is the fused post-norm kernel)."""
     wide = wl.T * wl.topk / wl.n_experts > 12.0
