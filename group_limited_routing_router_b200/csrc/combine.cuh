@@ -24,14 +24,28 @@ __global__ void __launch_bounds__(256) combine_kernel(const float4 *__restrict__
     __syncthreads();
     for (int c = threadIdx.x; c < H4; c += blockDim.x) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int j = 0; j < k; ++j) {
-            if (rows[j] < 0) continue;  // a bad expert id (reported through the status word)
-            const float4 v = __ldg(o + rows[j] * H4 + c);
+        // up to 8 slots: every row's load is issued before the sums, which stay in slot order
+        float4 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            v[j] = (j < k && rows[j] >= 0) ? __ldg(o + rows[j] * H4 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            if (j >= k || rows[j] < 0) continue;  // a bad expert id (reported through the status word)
             const float wj = wt[j];
-            acc.x = fmaf(wj, v.x, acc.x);
-            acc.y = fmaf(wj, v.y, acc.y);
-            acc.z = fmaf(wj, v.z, acc.z);
-            acc.w = fmaf(wj, v.w, acc.w);
+            acc.x = fmaf(wj, v[j].x, acc.x);
+            acc.y = fmaf(wj, v[j].y, acc.y);
+            acc.z = fmaf(wj, v[j].z, acc.z);
+            acc.w = fmaf(wj, v[j].w, acc.w);
+        }
+        for (int j = 8; j < k; ++j) {  // more than 8 slots
+            if (rows[j] < 0) continue;
+            const float4 u = __ldg(o + rows[j] * H4 + c);
+            const float wj = wt[j];
+            acc.x = fmaf(wj, u.x, acc.x);
+            acc.y = fmaf(wj, u.y, acc.y);
+            acc.z = fmaf(wj, u.z, acc.z);
+            acc.w = fmaf(wj, u.w, acc.w);
         }
         __nv_bfloat162 lo = __floats2bfloat162_rn(scale * acc.x, scale * acc.y);
         __nv_bfloat162 hi = __floats2bfloat162_rn(scale * acc.z, scale * acc.w);

@@ -139,10 +139,21 @@ __global__ void __launch_bounds__(128) gather_rows_kernel(const uint4 *__restric
     if (threadIdx.x < k) rows[threadIdx.x] = dest_row[t * k + threadIdx.x];
     __syncthreads();
     const uint4 *src = x + t * nvec;
-    for (int c = threadIdx.x; c < nvec; c += blockDim.x) {
-        const uint4 v = __ldg(src + c);
-        for (int j = 0; j < k; ++j)
-            if (rows[j] >= 0) xp[rows[j] * nvec + c] = v;
+    constexpr int U = 4;  // loads in flight per thread before its stores
+    for (int c0 = threadIdx.x; c0 < nvec; c0 += U * blockDim.x) {
+        uint4 v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int c = c0 + u * blockDim.x;
+            if (c < nvec) v[u] = __ldg(src + c);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int c = c0 + u * blockDim.x;
+            if (c < nvec)
+                for (int j = 0; j < k; ++j)
+                    if (rows[j] >= 0) xp[rows[j] * nvec + c] = v[u];
+        }
     }
 }
 
