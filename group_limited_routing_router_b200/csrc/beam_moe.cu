@@ -41,10 +41,9 @@ constexpr int64_t kMaxTokens = int64_t(1) << 24;
 // single CTAs, 32 rows on CTA pairs).
 // "narrow": a few tokens per expert (decode): the gate/up GEMM gathers its rows straight from x
 // with TMA gather4 (four rows per instruction; cheap when an expert has a handful of tokens).
-#define G1_WIDE_ARGS true, 192, 64, 4, 2, 256, false, false
 // "pair": the down projection with two 128-row weight tiles per token tile (half the token-row bytes
-// per weight byte).  The dense MLP runs G1_WIDE and this on single CTAs: its K = 20480 makes items
-// long, and 440 of them would leave a 10% wave tail on 74 CTA pairs.
+// per weight byte), for the dense MLP on single CTAs: its K = 20480 makes items long, and 440 of them
+// would leave a 10% wave tail on 74 CTA pairs (its gate/up runs on CTA pairs, G1_2SM_BIG).
 #define G2_PAIR_ARGS false, 192, 64, 4, 2, 256, false, true
 // CTA-pair variants (cta_group::2) for the MoE bf16 wide case (prefill, skew, long; the expert-rows
 // entry point): <gate/up?, BN, B box rows, smem stages, TMEM slots, slot columns>; each CTA stages half
@@ -214,7 +213,7 @@ int init_device(int *dev_out) {
                                        rt_smem_bytes(kRtTokSmall)) == cudaSuccess &&
                   cudaFuncSetAttribute(router_topk_kernel<kRtTokTiny>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        rt_smem_bytes(kRtTokTiny)) == cudaSuccess;
-        ok = ok && set_gemm_smem<G1_WIDE_ARGS>() && set_gemm_smem<G2_PAIR_ARGS>() &&
+        ok = ok && set_gemm_smem<G2_PAIR_ARGS>() &&
              set_gemm_smem<G1_NARROW_ARGS>() && set_gemm_smem<G2_NARROW_ARGS>();
         ok = ok && set_gemm_fp8_smem<G1_WIDE_FP8_ARGS>() && set_gemm_fp8_smem<G2_WIDE_FP8_ARGS>() &&
              set_gemm_fp8_smem<G1_NARROW_FP8_ARGS>() && set_gemm_fp8_smem<G2_NARROW_FP8_ARGS>();
@@ -1313,11 +1312,11 @@ extern "C" int beam_moe_dense_swiglu(int32_t hidden, int32_t inter, int64_t T, c
     void *h = wsb + L.h;
     dense_schedule_kernel<<<1, 1, 0, s>>>(counts, offsets, T);
     if ((rc = launch_status())) return rc;
-    // x itself is the token-ordered B operand of the gate/up GEMM (wide tiles, 64-row boxes)
+    // x itself is the token-ordered B operand of the gate/up GEMM (CTA pairs, 256-token tiles, 32-row boxes)
     CUtensorMap m_wg, m_wu, m_x, m_wd, m_h;
     if (!encode_fn()) return BEAM_MOE_ERR_CUDA;
     if (!make_map_3d(&m_wg, w_gate, hidden, inter, 1) || !make_map_3d(&m_wu, w_up, hidden, inter, 1) ||
-        !make_map_2d(&m_x, x, hidden, static_cast<uint64_t>(T), kWideBox) ||
+        !make_map_2d(&m_x, x, hidden, static_cast<uint64_t>(T), k2smBox) ||
         !make_map_3d(&m_wd, w_down, inter, hidden, 1) ||
         !make_map_2d(&m_h, h, inter, static_cast<uint64_t>(T), kWideBox))
         return BEAM_MOE_ERR_CUDA;
@@ -1325,7 +1324,7 @@ extern "C" int beam_moe_dense_swiglu(int32_t hidden, int32_t inter, int64_t T, c
     GemmParams p1{counts, offsets, h, 1, hidden, inter, 0, kDefaultTimeoutCycles, nullptr, 1};
     // the down projection's rows, rounded to bf16, are the output: one token-ordered expert needs no combine
     GemmParams p2{counts, offsets, y, 1, inter, hidden, 0, kDefaultTimeoutCycles, nullptr, 1, nullptr, 1};
-    launch_gemm<G1_WIDE_ARGS>(grid, s, m_wg, m_wu, m_x, p1);
+    launch_gemm2<G1_2SM_BIG_ARGS>(g_dev[dev].pairs_g1b, s, m_wg, m_wu, m_x, p1);
     if ((rc = launch_status())) return rc;
     launch_gemm<G2_PAIR_ARGS>(grid, s, m_wd, m_wd, m_h, p2);
     return launch_status();
