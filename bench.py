@@ -51,22 +51,22 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 _CSRC = os.path.join(ROOT, "group_limited_routing_router_b200", "csrc")
 _BF16_SRC = ("gemm.cuh", "gemm_2sm.cuh", "common.cuh", "beam_moe.cu")  # beam_moe.cu picks the variants
 _MX_SRC = ("gemm_mx8.cuh", "gemm.cuh", "common.cuh", "beam_moe.cu")
-_H1, _H2 = "8bce63b08c7d3c3b", "6c2e5bcdaf853dd9"
+_H1, _H2 = "c93cc758952df2fd", "c38934599f27bc8c"
 NCU_TRAFFIC = {
-    ("gate_up_swiglu", "decode"): {"bytes": 8 * (1678105600 + 444672), "files": _BF16_SRC, "hash": _H1},
-    ("gate_up_swiglu", "prefill"): {"bytes": 8 * (1746670592 + 3784448), "files": _BF16_SRC, "hash": _H1},
-    ("gate_up_swiglu", "long"): {"bytes": 8 * (7197129216 + 327750400), "files": _BF16_SRC, "hash": _H1},
-    ("down", "decode"): {"bytes": 8 * (840216064 + 3649280), "files": _BF16_SRC, "hash": _H1},
-    ("down", "prefill"): {"bytes": 8 * (863619584 + 32772608), "files": _BF16_SRC, "hash": _H1},
-    ("down", "long"): {"bytes": 8 * (1415222272 + 1311474432), "files": _BF16_SRC, "hash": _H1},
-    ("gate_up_swiglu_w4a4", "decode"): {"bytes": 8 * (472043776 + 725248), "files": _MX_SRC, "hash": _H2},
-    ("gate_up_swiglu_w4a4", "prefill"): {"bytes": 8 * (483464448 + 3374080), "files": _MX_SRC, "hash": _H2},
-    ("down_w4a4", "decode"): {"bytes": 8 * (236358144 + 952576), "files": _MX_SRC, "hash": _H2},
-    ("down_w4a4", "prefill"): {"bytes": 8 * (241892864 + 25118208), "files": _MX_SRC, "hash": _H2},
-    ("gate_up_swiglu_mxfp8", "decode"): {"bytes": 8 * (865337088 + 755456), "files": _MX_SRC, "hash": _H2},
-    ("gate_up_swiglu_mxfp8", "prefill"): {"bytes": 8 * (887574016 + 1698816), "files": _MX_SRC, "hash": _H2},
-    ("down_mxfp8", "decode"): {"bytes": 8 * (433264128 + 1815296), "files": _MX_SRC, "hash": _H2},
-    ("down_mxfp8", "prefill"): {"bytes": 8 * (444417280 + 5801472), "files": _MX_SRC, "hash": _H2},
+    ("gate_up_swiglu", "decode"): {"bytes": 8 * (1678104832 + 400896), "files": _BF16_SRC, "hash": _H1},
+    ("gate_up_swiglu", "prefill"): {"bytes": 8 * (1748065536 + 4208640), "files": _BF16_SRC, "hash": _H1},
+    ("gate_up_swiglu", "long"): {"bytes": 8 * (6605592576 + 331901184), "files": _BF16_SRC, "hash": _H1},
+    ("down", "decode"): {"bytes": 8 * (840216064 + 3623680), "files": _BF16_SRC, "hash": _H1},
+    ("down", "prefill"): {"bytes": 8 * (863484160 + 33014272), "files": _BF16_SRC, "hash": _H1},
+    ("down", "long"): {"bytes": 8 * (1509199360 + 1311041024), "files": _BF16_SRC, "hash": _H1},
+    ("gate_up_swiglu_w4a4", "decode"): {"bytes": 8 * (472080384 + 357120), "files": _MX_SRC, "hash": _H2},
+    ("gate_up_swiglu_w4a4", "prefill"): {"bytes": 8 * (483272192 + 3281408), "files": _MX_SRC, "hash": _H2},
+    ("down_w4a4", "decode"): {"bytes": 8 * (236404224 + 1159168), "files": _MX_SRC, "hash": _H2},
+    ("down_w4a4", "prefill"): {"bytes": 8 * (241893632 + 25558272), "files": _MX_SRC, "hash": _H2},
+    ("gate_up_swiglu_mxfp8", "decode"): {"bytes": 8 * (865321216 + 864768), "files": _MX_SRC, "hash": _H2},
+    ("gate_up_swiglu_mxfp8", "prefill"): {"bytes": 8 * (887475712 + 1669632), "files": _MX_SRC, "hash": _H2},
+    ("down_mxfp8", "decode"): {"bytes": 8 * (433307392 + 1774592), "files": _MX_SRC, "hash": _H2},
+    ("down_mxfp8", "prefill"): {"bytes": 8 * (444443392 + 5229312), "files": _MX_SRC, "hash": _H2},
 }
 
 
