@@ -6,8 +6,8 @@ synchronise the device.  For them the library offers a dispatch entry point whos
 array inside the library (256 KiB per device, enough for 65,536 tokens at 256 experts).  These tests
 call it through the C ABI and require outputs identical to the workspace entry point's, on
 consecutive calls that reuse the shared array with different sizes.  Its tests carry the `last`
-marker, which the collection hook in conftest.py moves behind every other test (the file name sorts
-last as well), so a run that stops at the first failure has run everything else first.
+marker, which the collection hook in conftest.py moves behind every other test whatever the file's
+name, so a run that stops at the first failure has run everything else first.
 """
 import ctypes
 
