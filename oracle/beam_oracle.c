@@ -666,8 +666,10 @@ static uint8_t e2m1_code_of(double v)  /* v already on the E2M1 grid */
  * on a value off by at most eps (relative) could make: the block's E4M3 scale rounded the other way
  * (amax / (6 g) within eps of a rounding boundary) or the element's E2M1 code rounded the other way
  * (v / (s g) within 6 eps of a boundary; the decision variable's error is relative to the block's
- * largest element, 6 s g).  0 where no such decision is that close.  It bounds what a quantiser
- * working on values within eps of these (FP32 ones, say) may legitimately give.
+ * largest element, 6 s g), or both at once: under the other scale c the element's code is again
+ * either rounding within the same absolute window (6 eps max(s, a) / c in units of c g).  0 where no
+ * such decision is that close.  It bounds what a quantiser working on values within eps of these
+ * (FP32 ones, say) may legitimately give.
  */
 static void nvfp4_block_alt(const double *blk, double g, double a, double s, double eps, double *alt)
 {
@@ -684,8 +686,14 @@ static void nvfp4_block_alt(const double *blk, double g, double a, double s, dou
                                 e4m3_value(e4m3_round_code(fmin(a * (1.0 + eps), 448.0)))};
         for (int c = 0; c < 2; ++c) {
             if (cand[c] == s) continue;
-            const double q2 = cand[c] > 0.0 ? e2m1_round(fabs(blk[i]) / (cand[c] * g)) : 0.0;
-            d = fmax(d, fabs(q2 * cand[c] - q * s) * g);
+            double lo2 = 0.0, hi2 = 0.0;
+            if (cand[c] > 0.0) {
+                const double m2 = fabs(blk[i]) / (cand[c] * g), w2 = 6.0 * eps * fmax(s, a) / cand[c];
+                lo2 = e2m1_round(fmax(0.0, m2 - w2));
+                hi2 = e2m1_round(m2 + w2);
+            }
+            /* the change is convex in the new code, so the two ends of the window bound it */
+            d = fmax(d, fmax(fabs(lo2 * cand[c] - q * s), fabs(hi2 * cand[c] - q * s)) * g);
         }
         alt[i] = d;
     }

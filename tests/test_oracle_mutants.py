@@ -70,6 +70,10 @@ MUTANTS = {
     "w4a4_h_row_scale": ("oracle_quant_nvfp4_rows_alt(n, I, hd, 0,", "oracle_quant_nvfp4_rows_alt(n, I, hd, 1,"),
     "w4a4_silu_missing": ("hd[(b * RB + r) * I + i] = silu4 * u[r];", "hd[(b * RB + r) * I + i] = g[r] * u[r];"),
     "expert_f64_silu_missing": ("const double act = g[r] / (1.0 + exp(-g[r]));", "const double act = g[r];"),
+    "alt_code_window_missing": ("lo = e2m1_round(fmax(0.0, m - 6.0 * eps)), hi = e2m1_round(m + 6.0 * eps);",
+                                "lo = e2m1_round(fmax(0.0, m)), hi = e2m1_round(m);"),
+    "alt_other_scale_ignored": ("if (cand[c] == s) continue;", "continue;"),
+    "alt_other_scale_code_fixed": ("w2 = 6.0 * eps * fmax(s, a) / cand[c];", "w2 = 0.0 * eps * fmax(s, a) / cand[c];"),
 }
 
 PINS = [
@@ -98,6 +102,8 @@ PINS = [
     w4a4.test_nvfp4_rows_match_exhaustive_search_and_torch_e4m3,
     w4a4.test_codes_decode_to_the_dequantised_values,
     w4a4.test_expert_w4a4_matches_torch_float64_composition,
+    w4a4.test_alternative_quantisation_envelope,
+    w4a4.test_envelope_bounds_every_perturbed_quantisation,
 ]
 
 

@@ -107,3 +107,54 @@ def test_alternative_quantisation_envelope():
     q_other = _nearest_e2m1(np.minimum(np.abs(v[1]) / s_other, 6.0)) * s_other
     np.testing.assert_allclose(alt[1], np.abs(q_other - deq[0]), rtol=0, atol=0)
     assert np.all(alt[2] == 0.0)
+
+
+def _boundary_rows(seed, rows=48, K=64, eps=1e-3):
+    """Rows whose 16-blocks sit on or near the quantiser's decision boundaries: a third of the blocks
+    have amax / 6 exactly on an E4M3 midpoint (the scale can round either way), a third within eps / 4
+    of one; elements on E2M1 midpoints under the block's scale or under the neighbouring scale, near
+    them, or uniform.  Returns the rows and each block's E4M3 scale (torch's cast)."""
+    rng = np.random.default_rng(seed)
+    codes = torch.arange(0, 0x7F, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    grid = np.unique(codes[(codes >= 0.5) & (codes <= 4.0)])
+    mids = (E2M1[1:] + E2M1[:-1]) / 2
+    v = np.zeros((rows, K))
+    for r in range(rows):
+        for b in range(K // 16):
+            kind = (r * (K // 16) + b) % 3
+            j = rng.integers(0, len(grid) - 1)
+            mid = (grid[j] + grid[j + 1]) / 2
+            a = (mid, mid * (1 + rng.choice([-1, 1]) * eps / 4), rng.uniform(0.5, 4.0))[kind]
+            s = torch.tensor(a).to(torch.float8_e4m3fn).double().item()
+            other = (grid[j + 1] if s == grid[j] else grid[j]) if kind < 2 else s
+            m = np.stack([rng.choice(mids, 16) * s, rng.choice(mids, 16) * other,
+                          rng.choice(mids, 16) * s * (1 + rng.uniform(-2, 2, 16) * eps), rng.uniform(0, 6 * a, 16)])
+            blk = m[rng.integers(0, 4, 16), np.arange(16)] * rng.choice([-1, 1], 16)
+            blk[rng.integers(0, 16)] = 6 * a * rng.choice([-1, 1])
+            v[r, b * 16:(b + 1) * 16] = blk
+    amax = np.abs(v).reshape(rows, K // 16, 16).max(-1)
+    return v, torch.from_numpy(amax / 6).to(torch.float8_e4m3fn).double().numpy()
+
+
+def test_envelope_bounds_every_perturbed_quantisation():
+    """alt as a bound: quantising v + d, with every |d| at most half the tolerance (eps / 2 of the
+    block's largest element 6 s), changes no dequantised element by more than alt(v, eps) — on rows
+    built to sit on the decision boundaries, where the block scale and the codes do flip, alone and
+    together.  The perturbed quantisation is this file's own (exhaustive E2M1 search, torch's E4M3)."""
+    eps = 1e-3
+    v, s_blk = _boundary_rows(5, eps=eps)
+    alt = oracle.quant_nvfp4_rows_alt(v, False, eps)
+    deq0, _ = _ref_quant(v, False)
+    np.testing.assert_array_equal(oracle.quant_nvfp4_rows(v, False)[3], deq0)
+    budget = np.repeat((eps / 2) * 6 * s_blk, 16, axis=1)
+    rng = np.random.default_rng(6)
+    changed = scale_flips = 0
+    for _ in range(150):
+        w = v + rng.uniform(-1, 1, v.shape) * budget
+        deq1, _ = _ref_quant(w, False)
+        diff = np.abs(deq1 - deq0)
+        assert np.all(diff <= alt), f"{int((diff > alt).sum())} elements moved beyond the envelope"
+        changed += int((diff > 0).sum())
+        s1 = torch.from_numpy(np.abs(w).reshape(s_blk.shape + (16,)).max(-1) / 6).to(torch.float8_e4m3fn)
+        scale_flips += int((s1.double().numpy() != s_blk).sum())
+    assert changed > 10_000 and scale_flips > 1_000   # the boundaries were really crossed
