@@ -74,6 +74,7 @@ MUTANTS = {
                                 "lo = e2m1_round(fmax(0.0, m)), hi = e2m1_round(m);"),
     "alt_other_scale_ignored": ("if (cand[c] == s) continue;", "continue;"),
     "alt_other_scale_code_fixed": ("w2 = 6.0 * eps * fmax(s, a) / cand[c];", "w2 = 0.0 * eps * fmax(s, a) / cand[c];"),
+    "env_signed_down_weights": ("wabs[i] = fabs(wd[(int64_t)o * I + i]);", "wabs[i] = wd[(int64_t)o * I + i];"),
 }
 
 PINS = [
@@ -104,6 +105,7 @@ PINS = [
     w4a4.test_expert_w4a4_matches_torch_float64_composition,
     w4a4.test_alternative_quantisation_envelope,
     w4a4.test_envelope_bounds_every_perturbed_quantisation,
+    w4a4.test_expert_envelope_bounds_a_perturbed_h,
 ]
 
 

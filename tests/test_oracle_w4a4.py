@@ -158,3 +158,29 @@ def test_envelope_bounds_every_perturbed_quantisation():
         s1 = torch.from_numpy(np.abs(w).reshape(s_blk.shape + (16,)).max(-1) / 6).to(torch.float8_e4m3fn)
         scale_flips += int((s1.double().numpy() != s_blk).sum())
     assert changed > 10_000 and scale_flips > 1_000   # the boundaries were really crossed
+
+
+def test_expert_envelope_bounds_a_perturbed_h():
+    """The expert's envelope env = |W_d| alt(h): perturb h (computed here by a torch float64
+    composition) by at most half the tolerance per element, quantise it with this file's quantiser,
+    project, and the output moves by no more than env.  eps = 1e-2 so that many decisions flip."""
+    rng = np.random.default_rng(12)
+    n, H, I, eps = 7, 256, 128, 1e-2
+    x = torch.from_numpy(rng.standard_normal((n, H))).to(torch.bfloat16)
+    bits = x.view(torch.int16).numpy().view(np.uint16)
+    wg, wu = (rng.standard_normal((I, H)) / 16 for _ in range(2))
+    wd = rng.standard_normal((H, I)) / 11
+    out, env = oracle.expert_mlp_w4a4(bits, wg, wu, wd, eps=eps)
+    xq, _ = _ref_quant(x.double().numpy(), True)
+    h = torch.nn.functional.silu(torch.from_numpy(xq @ wg.T)).numpy() * (xq @ wu.T)
+    hq, _ = _ref_quant(h, False)
+    np.testing.assert_allclose(out, hq @ wd.T, rtol=1e-12, atol=1e-12 * np.abs(out).max())
+    s_blk = torch.from_numpy(np.abs(h).reshape(n, I // 16, 16).max(-1) / 6).to(torch.float8_e4m3fn)
+    budget = np.repeat((eps / 2) * 6 * s_blk.double().numpy(), 16, axis=1)
+    slack = 1e-12 * (np.abs(hq) @ np.abs(wd).T).max()    # rounding of the two FP64 projections
+    moved = 0
+    for _ in range(40):
+        hq1, _ = _ref_quant(h + rng.uniform(-1, 1, h.shape) * budget, False)
+        moved += int((hq1 != hq).sum())
+        assert np.all(np.abs(hq1 @ wd.T - out) <= env + slack)
+    assert moved > 100
