@@ -53,3 +53,20 @@ def route(x: np.ndarray, w_router: np.ndarray, E: int, G: int, topk_groups: int,
 
 def n_subsets(E: int, G: int, topk_groups: int, topk: int) -> int:
     return math.comb(G, topk_groups) * math.comb(topk_groups * E // G, topk)
+
+
+def margins(sel: np.ndarray, E: int, G: int, topk_groups: int, topk: int, group_topn: int):
+    """The decision margins of one token stated as smallest gaps between what was chosen and what was
+    not: the smallest kept-minus-dropped group score, the smallest chosen-minus-unchosen value among
+    the kept groups' experts, and the smallest gap between consecutive slots (inf where nothing is
+    compared).  Group scores by subset enumeration."""
+    per = E // G
+    gscore = [max(sum(c) for c in itertools.combinations(sel[g * per:(g + 1) * per].tolist(), group_topn))
+              for g in range(G)]
+    ids, _, kept = route_token(sel, sel, E, G, topk_groups, topk, group_topn)
+    dropped = [g for g in range(G) if g not in kept]
+    m_group = min((gscore[a] - gscore[b] for a in kept for b in dropped), default=math.inf)
+    cand = [e for g in kept for e in range(g * per, (g + 1) * per)]
+    m_expert = min((sel[a] - sel[b] for a in ids for b in cand if b not in ids), default=math.inf)
+    m_order = min((sel[ids[j]] - sel[ids[j + 1]] for j in range(topk - 1)), default=math.inf)
+    return m_group, m_expert, m_order

@@ -74,6 +74,11 @@ MUTANTS = {
                                 "lo = e2m1_round(fmax(0.0, m)), hi = e2m1_round(m);"),
     "alt_other_scale_ignored": ("if (cand[c] == s) continue;", "continue;"),
     "alt_other_scale_code_fixed": ("w2 = 6.0 * eps * fmax(s, a) / cand[c];", "w2 = 0.0 * eps * fmax(s, a) / cand[c];"),
+    "group_margin_wrong_ranks": ("gs_sorted[topk_groups - 1] - gs_sorted[topk_groups] : INFINITY;",
+                                 "gs_sorted[0] - gs_sorted[topk_groups] : INFINITY;"),
+    "expert_margin_wrong_ranks": ("sel_sorted[topk - 1] - sel_sorted[topk] : INFINITY;",
+                                  "sel_sorted[topk - 1] - sel_sorted[nk - 1] : INFINITY;"),
+    "order_margin_skips_last_pair": ("for (int j = 0; j + 1 < topk; ++j) {", "for (int j = 0; j + 2 < topk; ++j) {"),
     "env_signed_down_weights": ("wabs[i] = fabs(wd[(int64_t)o * I + i]);", "wabs[i] = wd[(int64_t)o * I + i];"),
 }
 
@@ -81,6 +86,7 @@ PINS = [
     lambda: pins.test_bruteforce_tiny(False),
     lambda: pins.test_bruteforce_tiny(True),
     pins.test_hand_cases,
+    lambda: pins.test_margins_are_the_smallest_chosen_minus_unchosen_gaps(True),
     pins.test_invariants_beam_groups,
     pins.test_all_groups_kept_is_plain_topk,
     pins.test_single_expert_matches_torch_float64,

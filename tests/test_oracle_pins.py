@@ -58,6 +58,26 @@ def test_bruteforce_tiny(with_bias):
     assert n_cmp > 0.9 * 20 * 64
 
 
+
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_margins_are_the_smallest_chosen_minus_unchosen_gaps(with_bias):
+    """The FP64 decision margins (group, expert, slot order) equal the smallest gaps between what was
+    chosen and what was not, found by subset enumeration on the tiny layer; a margin that compares
+    the wrong ranks or the wrong sets would let near-ties through the bit-exact checks."""
+    rng = np.random.default_rng(8)
+    for seed in range(130, 140):
+        wl, x, W = tiny_inputs(seed)
+        L = wl.layer
+        bias = rng.normal(0, 0.05, size=wl.n_experts).astype(np.float32) if with_bias else None
+        xb = oracle.bf16_bits(x)
+        r = oracle.route(xb, W.numpy(), L, bias)
+        score = bruteforce.sigmoid64(oracle.bf16_bits_to_f64(xb) @ W.numpy().astype(np.float64).T)
+        sel = score + (0.0 if bias is None else bias.astype(np.float64)[None, :])
+        want = np.array([bruteforce.margins(sel[t], L["n_experts"], L["n_groups"], L["topk_groups"], L["topk"],
+                                            L["group_topn"]) for t in range(wl.T)])
+        np.testing.assert_allclose(r["margin"], want, rtol=0, atol=1e-12)
+
+
 def test_hand_cases():
     with open(os.path.join(GOLDEN, "hand_routing_cases.json")) as f:
         cases = json.load(f)["cases"]
