@@ -106,3 +106,48 @@ def test_emulated_ranks_match_one_process_oracle():
     ys = ep.forward_emulated(ranks, xs)
     ref = oracle.forward(oracle.bf16_bits(x), W, b, fetch, wl.layer)
     assert np.array_equal(np.concatenate([y.numpy() for y in ys]), ref["y"])
+
+
+def _failing_rank_main(rank, world, port, out_dir):
+    """Rank 1 fails on the host before its first exchange (an exception, as a crashed step would);
+    rank 0 runs its forward pass and must get an error from the exchange, not wait for ever."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    import time
+
+    import torch.distributed as dist
+
+    from tests.ep_oracle_ops import OracleOps
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=10))
+    wl, x, W, b, fetch = _inputs("tiny")
+    part = ep.Partition(wl.n_experts, world)
+    r = ep.Rank(part, rank, OracleOps(wl.layer, W, b, fetch, part.experts_of(rank).start))
+    if rank == 1:
+        os._exit(3)           # leaves without a word to its peer
+    t0 = time.monotonic()
+    try:
+        ep.forward(r, x[_token_slice(wl.T, world, rank)].contiguous().view(torch.int16))
+        outcome = "completed"
+    except Exception as e:  # noqa: BLE001 - the kind of error depends on how gloo notices the loss
+        outcome = f"error: {type(e).__name__}"
+    with open(os.path.join(out_dir, "rank0.txt"), "w") as f:
+        f.write(f"{outcome}\n{time.monotonic() - t0:.1f}\n")
+    os._exit(0)
+
+
+def test_lost_rank_surfaces_as_an_error_on_the_others():
+    """Failure detection on the host: a rank that dies between steps makes the surviving rank's next
+    exchange raise within the process group's timeout (10 s here) instead of hanging."""
+    ctx = mp.get_context("spawn")
+    port = _free_port()
+    with tempfile.TemporaryDirectory() as d:
+        procs = [ctx.Process(target=_failing_rank_main, args=(r, 2, port, d)) for r in range(2)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(timeout=120)
+        assert [p.exitcode for p in procs] == [0, 3]
+        with open(os.path.join(d, "rank0.txt")) as f:
+            outcome, secs = f.read().splitlines()
+    assert outcome.startswith("error"), outcome
+    assert float(secs) < 60.0
