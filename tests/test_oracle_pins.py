@@ -78,6 +78,29 @@ def test_margins_are_the_smallest_chosen_minus_unchosen_gaps(with_bias):
         np.testing.assert_allclose(r["margin"], want, rtol=0, atol=1e-12)
 
 
+
+@pytest.mark.parametrize("E,G,kg,k,gn", [
+    (16, 4, 2, 4, 1), (16, 4, 2, 4, 3), (16, 4, 3, 6, 4), (16, 8, 3, 5, 2), (12, 3, 1, 3, 2),
+    (24, 6, 4, 7, 3), (16, 2, 1, 8, 8), (16, 4, 4, 4, 2)])
+def test_select_matches_bruteforce_across_layouts(E, G, kg, k, gn):
+    """The selection step on scores drawn directly (continuous, so no ties) for layouts other than
+    Beam's: group sizes 2-8, one to all groups kept, group scores over the top 1 to 8 members, k from
+    3 to 8 -- against subset enumeration, with and without a selection bias."""
+    rng = np.random.default_rng(E * 1000 + G * 100 + kg * 10 + k + gn)
+    L = dict(n_experts=E, n_groups=G, topk_groups=kg, topk=k, group_topn=gn)
+    for with_bias in (False, True):
+        score = rng.uniform(0.01, 0.99, (24, E))
+        bias = rng.normal(0, 0.1, E).astype(np.float32) if with_bias else None
+        r = oracle.select(score, L, bias)
+        sel = score + (0.0 if bias is None else bias.astype(np.float64)[None, :])
+        for t in range(score.shape[0]):
+            ids, w, _ = bruteforce.route_token(sel[t], score[t], E, G, kg, k, gn)
+            assert r["ids64"][t].tolist() == ids
+            if np.all(r["margin"][t] >= 1e-6):
+                assert r["ids"][t].tolist() == ids
+                np.testing.assert_allclose(r["weight"][t], w, rtol=0, atol=1e-12)
+
+
 def test_hand_cases():
     with open(os.path.join(GOLDEN, "hand_routing_cases.json")) as f:
         cases = json.load(f)["cases"]
